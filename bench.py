@@ -1,0 +1,443 @@
+#!/usr/bin/env python
+"""Benchmark of the TurboQuant compressed-KV hot path on B200.
+
+One step = the whole hot path over one batch of synthetic input:
+  1. compress every cached key and value of the workload (rotation, Lloyd-Max
+     codes, QJL signs, value group quantization, packing) in one call;
+  2. decode one new query token per sequence against the packed cache
+     (query prep, split-K attention, combine) in one call.
+The default workload is the Qwen2.5-3B-shaped cache (36 layers x 2 KV heads x
+8192 tokens, 16 query heads per layer, K 3-bit / V 2-bit, bf16 inputs).
+
+Prints ONE JSON line on rank 0. `value` is decode-attention throughput in GB/s
+of packed K/V bytes read (summed over ranks, divided by the slowest rank's decode
+time); compression throughput is reported beside it. The L2 cache is flushed
+(256 MiB write) before each timed phase, since the packed cache (59 MB) fits in L2.
+
+`--impl reference` times the fp64 CPU oracle on this machine's host cores on a
+bounded sample of the same workload (the slow baseline arm).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "decode-attention packed-KV GB/s (% of HBM peak); compress vectors/s"
+FLUSH_BYTES = 256 << 20
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="qwen2.5-3b_8k_k3v2", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def source_sha(names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "kv_cache_vector_05_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+DECODE_SOURCES = ("decode.cu", "tq_device.cuh", "tq_internal.h")
+
+
+def recorded_traffic(kernel_file: str, sha: str):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the source."""
+    p = os.path.join(ROOT, "profiles", kernel_file)
+    if not os.path.exists(p):
+        return None
+    kv = {}
+    with open(p) as f:
+        for line in f:
+            if ":" in line:
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+    if kv.get("source_sha256_16") != sha:
+        return None
+    try:
+        return float(kv["dram_bytes_per_launch_scaled"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------------- inputs
+
+def host_inputs(w: W.Workload, rank: int):
+    """bf16/fp32 K, V [units*tokens, d] and Q [batch, hq, d] as numpy fp32 arrays."""
+    if w.name.startswith("qwen"):
+        K = np.empty((w.units * w.tokens, w.d), np.float32)
+        V = np.empty_like(K)
+        for layer in range(w.batch):
+            for h in range(w.hkv):
+                u = layer * w.hkv + h
+                k, v = W.qwen_layer_head_kv(layer, h, w.tokens, w.d)
+                K[u * w.tokens:(u + 1) * w.tokens] = k
+                V[u * w.tokens:(u + 1) * w.tokens] = v
+    else:
+        K = V = None  # drawn on the device
+    Q = W.queries((w.batch, w.hq, w.d), seed=7 + rank, dtype=w.dtype)
+    return K, V, Q
+
+
+# ---------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", gpu_id], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception as e:  # pragma: no cover - no nvidia-smi
+            log("clock sampler unavailable:", e)
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    smax.append(float(parts[1]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[4:8]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------- CPU oracle
+
+def oracle_sample(w: W.Workload, budget_s: float, K=None, V=None, Q=None):
+    """Time the fp64 oracle on whole (sequence, KV head) units of the workload.
+    Returns dict(decode_gbs, compress_vps, units, decode_s, compress_s, cores)."""
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        cores = 1
+    dr = W.method_draws(w.d, w.m)
+    Pi = O.hadamard_rotation(dr["hadamard_signs"])
+    c, t = O.device_codebook(w.d, w.lm_bits)
+    S = dr["qjl_S"]
+    if Q is None:
+        Q = W.queries((w.batch, w.hq, w.d), seed=7, dtype=w.dtype)
+    rec = w.k_record_bytes() + w.v_record_bytes()
+    comp_s = dec_s = 0.0
+    n_units = 0
+    t_start = time.perf_counter()
+    while n_units < w.units and (n_units == 0 or time.perf_counter() - t_start < budget_s):
+        u = n_units
+        b, kvh = divmod(u, w.hkv)
+        if K is not None:
+            k = K[u * w.tokens:(u + 1) * w.tokens].astype(np.float64)
+            v = V[u * w.tokens:(u + 1) * w.tokens].astype(np.float64)
+        else:
+            k32, v32 = W.unit_keys_values(w, u)
+            k, v = k32.astype(np.float64), v32.astype(np.float64)
+        t0 = time.perf_counter()
+        pk = O.compress_keys(k, Pi, c, t, S)
+        pv = O.quantize_values(v, w.v_bits)
+        t1 = time.perf_counter()
+        O.decode_attention(Q[b, kvh * w.group:(kvh + 1) * w.group].astype(np.float64), pk, pv, Pi, c, S,
+                           w.d, w.v_bits)
+        t2 = time.perf_counter()
+        comp_s += t1 - t0
+        dec_s += t2 - t1
+        n_units += 1
+    return {"decode_gbs": n_units * w.tokens * rec / dec_s / 1e9,
+            "compress_vps": 2 * n_units * w.tokens / comp_s,
+            "units": n_units, "decode_s": dec_s, "compress_s": comp_s, "cores": cores}
+
+
+def run_reference(args, w: W.Workload):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    K, V, Q = host_inputs(w, 0)
+    per_step = max(args.cpu_seconds / max(args.steps, 1), 0.05)
+    for _ in range(args.warmup):
+        oracle_sample(w, 0.0, K, V, Q)
+    res = [oracle_sample(w, per_step, K, V, Q) for _ in range(args.steps)]
+    dec_s = sum(r["decode_s"] for r in res)
+    comp_s = sum(r["compress_s"] for r in res)
+    units = sum(r["units"] for r in res)
+    rec = w.k_record_bytes() + w.v_record_bytes()
+    gbs = units * w.tokens * rec / dec_s / 1e9
+    sample = (f"{units} (sequence, KV head) units over {args.steps} steps; each: compress "
+              f"{w.tokens} keys + {w.tokens} values, decode {w.group} query heads (fp64 numpy oracle)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * (dec_s + comp_s) / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "kv_heads": w.hkv, "q_heads": w.hq,
+                   "tokens": w.tokens, "head_dim": w.d, "k_bits": w.k_bits, "v_bits": w.v_bits},
+        "compress": {"value": 2 * units * w.tokens / comp_s, "unit": "vectors/s"},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": res[0]["cores"], "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------- GPU arm
+
+def run_ours(args, w: W.Workload):
+    import torch
+    import torch.distributed as dist
+    import kv_cache_vector_05_b200 as T
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # --- method tables and inputs
+    dr = W.method_draws(w.d, w.m)
+    c, t = T.tq_lloyd_max_codebook(w.d, w.lm_bits)
+    ctx = T.tq_codebook_load(w.d, w.lm_bits, w.v_bits, c, t, dr["qjl_S"], hadamard_signs=dr["hadamard_signs"])
+    n_vec = w.units * w.tokens
+    Kh, Vh, Qh = host_inputs(w, rank)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    if Kh is not None:
+        K = torch.from_numpy(Kh).to(dev).to(tdt)
+        V = torch.from_numpy(Vh).to(dev).to(tdt)
+        del Kh, Vh
+    else:
+        K = W.device_normal((n_vec, w.d), seed=1000 + rank, device=dev).to(tdt)
+        V = W.device_normal((n_vec, w.d), seed=2000 + rank, device=dev).to(tdt)
+    Q = torch.from_numpy(Qh).to(dev).to(tdt)
+    packed = {
+        "k_codes": torch.empty((n_vec, w.lm_bits * w.d // 8), dtype=torch.uint8, device=dev),
+        "k_signs": torch.empty((n_vec, w.m // 8), dtype=torch.uint8, device=dev),
+        "k_norms": torch.empty((n_vec, 2), dtype=torch.int16, device=dev),
+        "v_codes": torch.empty((n_vec, w.v_bits * w.d // 8), dtype=torch.uint8, device=dev),
+        "v_params": torch.empty((n_vec, w.d // 32, 2), dtype=torch.int16, device=dev),
+    }
+    out = torch.empty((w.batch, w.hq, w.d), dtype=torch.float32, device=dev)
+    ws = torch.empty(T.tq_decode_workspace_bytes(ctx, w.batch, w.hq, w.hkv, w.tokens), dtype=torch.uint8,
+                     device=dev)
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    packed_bytes = n_vec * (w.k_record_bytes() + w.v_record_bytes())
+    in_bytes = 2 * n_vec * w.d * (2 if w.dtype == "bf16" else 4)
+
+    def compress():
+        T.tq_compress_kv(ctx, K, V, **packed)
+
+    def decode():
+        T.tq_decode_attention(ctx, Q, packed, w.batch, w.hq, w.hkv, w.tokens, out=out, workspace=ws)
+
+    E = torch.cuda.Event
+
+    def run_steps(n, record):
+        evs = []
+        for _ in range(n):
+            e = [E(enable_timing=True) for _ in range(8)]
+            flush_buf.zero_()
+            e[0].record()
+            if record:
+                T.tq_set_profile_events(ctx, e[1], e[2])
+            compress()
+            e[3].record()
+            flush_buf.zero_()
+            e[4].record()
+            if record:
+                T.tq_set_profile_events(ctx, e[5], e[6])
+            decode()
+            e[7].record()
+            if record:
+                T.tq_set_profile_events(ctx, None, None)
+            evs.append(e)
+        return evs
+
+    run_steps(args.warmup, True)
+    torch.cuda.synchronize()
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    gpu_id = vis.split(",")[local] if vis else str(local)
+    sampler = ClockSampler(gpu_id) if rank == 0 else None
+    time.sleep(1.0)
+    run_steps(max(3, args.warmup // 2), False)
+
+    barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    evs = run_steps(args.steps, True)
+    torch.cuda.synchronize()
+    barrier()
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop() if sampler else None
+
+    comp = [e[0].elapsed_time(e[3]) for e in evs]
+    comp_k = [e[1].elapsed_time(e[2]) for e in evs]
+    dec = [e[4].elapsed_time(e[7]) for e in evs]
+    dec_k = [e[5].elapsed_time(e[6]) for e in evs]
+    dec_total = max_over_ranks(sum(dec) / 1e3)
+    comp_total = max_over_ranks(sum(comp) / 1e3)
+    dec_k_mean = max_over_ranks(statistics.fmean(dec_k) / 1e3)
+    gbs = world * packed_bytes * args.steps / dec_total / 1e9
+    vps = world * 2 * n_vec * args.steps / comp_total
+
+    # --- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        Kp = K.cpu().pin_memory()
+        Vp = V.cpu().pin_memory()
+        Qp = Q.cpu().pin_memory()
+        outp = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+        Kd, Vd, Qd = torch.empty_like(K), torch.empty_like(V), torch.empty_like(Q)
+
+        def e2e_step():
+            Kd.copy_(Kp, non_blocking=True)
+            Vd.copy_(Vp, non_blocking=True)
+            Qd.copy_(Qp, non_blocking=True)
+            T.tq_compress_kv(ctx, Kd, Vd, **packed)
+            T.tq_decode_attention(ctx, Qd, packed, w.batch, w.hq, w.hkv, w.tokens, out=out, workspace=ws)
+            outp.copy_(out, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        s0, s1 = E(enable_timing=True), E(enable_timing=True)
+        s0.record()
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        s1.record()
+        torch.cuda.synchronize()
+        e2e_s = max_over_ranks(s0.elapsed_time(s1) / 1e3)
+        h2d = Kp.numel() * Kp.element_size() + Vp.numel() * Vp.element_size() + Qp.numel() * Qp.element_size()
+        e2e = {"value": world * packed_bytes * args.e2e_steps / e2e_s / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(outp.numel() * 4),
+               "ms_per_step": 1e3 * e2e_s / args.e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        Kh2, Vh2, _ = host_inputs(w, 0) if w.name.startswith("qwen") else (None, None, None)
+        r = oracle_sample(w, args.cpu_seconds, Kh2, Vh2, Qh)
+        cpu = {"value": r["decode_gbs"], "unit": "GB/s", "cores": r["cores"], "kind": "oracle",
+               "sample": (f"{r['units']} of {w.units} (sequence, KV head) units: compress {w.tokens} keys + "
+                          f"{w.tokens} values and decode {w.group} query heads each; fp64 numpy oracle; "
+                          f"compress {r['compress_vps']:.4g} vectors/s")}
+
+    if rank == 0:
+        peak, peak_kind = measured_peaks()
+        alg_bytes = packed_bytes
+        achieved = alg_bytes / dec_k_mean / 1e9
+        sha = source_sha(DECODE_SOURCES)
+        line = {
+            "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * (dec_total + comp_total) / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "kv_heads": w.hkv, "q_heads": w.hq,
+                       "tokens": w.tokens, "head_dim": w.d, "k_bits": w.k_bits, "v_bits": w.v_bits,
+                       "rotation": w.rotation, "packed_bytes": packed_bytes,
+                       "l2": "flushed (256 MiB write) before each timed phase",
+                       "parallelism": f"dp{world} (independent replicas)"},
+            "pct_of_hbm_peak": 100.0 * gbs / peak,
+            "compress": {"value": vps, "unit": "vectors/s (keys + values)",
+                         "gbs": world * (in_bytes + packed_bytes) * args.steps / comp_total / 1e9,
+                         "kernel_ms": statistics.fmean(comp_k)},
+            "decode_ms": {"call": dec_total * 1e3 / args.steps, "main_kernel": dec_k_mean * 1e3},
+            "roofline": {"kernel": "decode_kernel", "bound": "hbm", "achieved": achieved, "peak": peak,
+                         "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
+                         "alg_bytes_per_launch": alg_bytes,
+                         "traffic": recorded_traffic("decode_kernel_traffic.txt", sha),
+                         "source_sha256_16": sha},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": 4 * args.steps,
+            "clocks": clocks,
+            "wall_s": wall,
+        }
+        print(json.dumps(line), flush=True)
+    ctx.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    w = W.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,192 @@
+/*
+ * tq.h - C ABI of the TurboQuant compressed-KV library for NVIDIA B200 (sm_100a).
+ *
+ * The library compresses transformer key/value cache vectors in two stages and
+ * runs decode attention directly on the packed cache:
+ *
+ *   keys   : n = ||k||, u = k/n, y = Pi u (random orthogonal rotation),
+ *            idx = Lloyd-Max cell of each y_j, r = y - c[idx], gamma = ||r||,
+ *            1-bit QJL signs s = [S r >= 0], packed codes + signs + fp16 (n, gamma)
+ *   values : groups of 32 coordinates, min/max uniform codes at 2 or 4 bits,
+ *            fp16 (scale, min) per group
+ *   decode : qr = Pi q, sq = S qr; logit_t = scale * n_t * (<qr, c[idx_t]>
+ *            + sqrt(pi/2)/m * gamma_t * <sq, s_t>); online softmax over the cache;
+ *            output = sum_t p_t * (min + scale * code_t) / sum_t p_t
+ *
+ * Sources (web pages about TurboQuant):
+ *   - "turboquant-pytorch" skill card, section "Что делает": rotation +
+ *     Lloyd-Max + one-bit QJL residual correction; attention scores computed
+ *     straight from the compressed keys (TurboQuantProd).
+ *   - discosf.com TurboQuant news item, section "一句话看懂": the four steps
+ *     (rotation, Lloyd-Max with pre-generated codebooks, QJL sign bits, value
+ *     group quantization with four 2-bit values per byte); decode runs in fused
+ *     kernels on the compressed cache.
+ *   - tproger.ru "TurboQuant неделю спустя", section "Реализации TurboQuant":
+ *     the dense O(d^2) rotation is slow; a Walsh-Hadamard transform is O(d log d).
+ *
+ * Conventions for every call:
+ *   - All device buffers belong to the caller. The library allocates device
+ *     memory only inside tq_codebook_load (its own tables, freed by tq_free).
+ *   - Device pointers must be 16-byte aligned, else TQ_EINVAL.
+ *   - Calls are asynchronous on the given CUDA stream (a cudaStream_t passed as
+ *     void*, NULL = legacy default stream). Only tq_codebook_load synchronizes.
+ *   - Unsupported sizes or bit widths return TQ_EUNSUPPORTED; CUDA launch or
+ *     runtime errors return TQ_ECUDA (tq_last_error() has the CUDA message).
+ *   - No function throws; no function calls exit() or abort().
+ *
+ * Packed formats (little-endian, one record per vector, records contiguous):
+ *   k_codes  [n_vec][lm_bits*d/8] u8  code j in bits [lm_bits*j, lm_bits*j+lm_bits)
+ *                                     of the record, least significant bit first
+ *   k_signs  [n_vec][m/8]         u8  sign bit i = bit i%8 of byte i/8, 1 <=> (S r)_i >= 0
+ *   k_norms  [n_vec][2]           u16 fp16 bit patterns (n, gamma), round-to-nearest-even
+ *   v_codes  [n_vec][v_bits*d/8]  u8  same stream layout as k_codes
+ *   v_params [n_vec][d/32][2]     u16 fp16 (scale, min) per group of 32 coordinates
+ * A zero key is stored as all-zero bytes.
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_EINVAL = 1,        /* bad pointer, alignment, size or argument combination */
+  TQ_EUNSUPPORTED = 2,  /* d, bit width, m or group size outside what is built */
+  TQ_ECUDA = 3,         /* a CUDA runtime call or kernel launch failed */
+  TQ_ENOMEM = 4         /* device or host allocation failed (tq_codebook_load only) */
+} tq_status;
+
+typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
+
+typedef enum {
+  TQ_ROT_HADAMARD = 0,  /* Pi = H_d diag(sigma) / sqrt(d), applied as sign flip + FWHT */
+  TQ_ROT_HAAR = 1       /* Pi = dense Haar orthogonal matrix (d x d) */
+} tq_rot;
+
+/* Method parameters. Every array is HOST memory and is copied by
+ * tq_codebook_load; the caller may free it afterwards.
+ *   d              head dimension: 64, 128 or 256
+ *   k_lm_bits      Lloyd-Max bits per key coordinate: 1, 2 or 3 (a key then costs
+ *                  k_lm_bits + 1 bits per coordinate with its QJL sign)
+ *   qjl_m          rows of the QJL matrix S: a multiple of 32, at most 256
+ *   v_bits         value bits: 2 or 4
+ *   v_group        value group size: 32
+ *   rot            rotation kind
+ *   centroids      2^k_lm_bits ascending fp32 centroids of the Lloyd-Max codebook
+ *   boundaries     2^k_lm_bits - 1 ascending fp32 cell boundaries; coordinate y
+ *                  gets code #{k : y >= boundaries[k]}
+ *   hadamard_signs d entries, each +1 or -1 (TQ_ROT_HADAMARD; ignored otherwise)
+ *   haar           d*d row-major orthogonal matrix Pi in fp64, y = Pi u (TQ_ROT_HAAR)
+ *   qjl_S          m*d row-major fp32 matrix S (i.i.d. N(0,1) draws)            */
+typedef struct {
+  int d;
+  int k_lm_bits;
+  int qjl_m;
+  int v_bits;
+  int v_group;
+  tq_rot rot;
+  const float* centroids;
+  const float* boundaries;
+  const signed char* hadamard_signs;
+  const double* haar;
+  const float* qjl_S;
+} tq_params;
+
+typedef struct tq_ctx tq_ctx;
+
+/* Load a codebook, rotation and QJL matrix onto the current CUDA device.
+ * Pre-generated codebooks are part of the method (discosf news item,
+ * "一句话看懂" step 2); tq_lloyd_max_codebook below produces them.
+ * Validates the parameters (TQ_EINVAL / TQ_EUNSUPPORTED), allocates the
+ * context's device tables (TQ_ENOMEM), uploads them on `stream` and
+ * synchronizes that stream once. On success *out owns the tables until
+ * tq_free. The context is bound to the device that was current here. */
+tq_status tq_codebook_load(const tq_params* params, void* stream, tq_ctx** out);
+
+/* Release a context and its device tables. NULL is a no-op. The caller must
+ * make sure no work using the context is still running. */
+void tq_free(tq_ctx* ctx);
+
+/* Static, human-readable name of a status code. Never NULL. */
+const char* tq_status_string(tq_status status);
+
+/* Message of the last failing call on this thread ("" if none). */
+const char* tq_last_error(void);
+
+/* HOST ONLY (no GPU needed). Lloyd-Max codebook of one coordinate of a uniform
+ * random unit vector in R^d (the law of every rotated coordinate), with 2^bits
+ * levels: centroids at cell means, boundaries at centroid midpoints, iterated
+ * in fp64 to convergence and rounded to fp32. The skill card ("turboquant-
+ * pytorch", "Что делает") builds these codebooks with scipy; this is a
+ * self-contained solver. Writes 2^bits centroids and 2^bits - 1 boundaries.
+ * d in [4, 4096], bits in [1, 4]; else TQ_EINVAL. */
+tq_status tq_lloyd_max_codebook(int d, int bits, float* centroids, float* boundaries);
+
+/* HOST ONLY. Haar-distributed orthogonal matrix from a d x d row-major matrix
+ * of i.i.d. N(0,1) draws: Q of its QR factorisation with R's diagonal made
+ * positive (Householder, fp64). Writes d*d row-major doubles to pi_out.
+ * d in [1, 1024]; TQ_EINVAL on NULL pointers or a rank-deficient input. */
+tq_status tq_haar_from_gaussian(int d, const double* gaussian, double* pi_out);
+
+/* Compress n_vec keys and/or values (prefill / append path).
+ *   k, v      device [n_vec][d] of `dtype` (fp32 or bf16); either may be NULL to
+ *             skip that half (its output pointers are then ignored)
+ *   k_codes, k_signs, k_norms, v_codes, v_params: device outputs, formats above
+ * Each output record is written in full; n_vec = 0 is a no-op returning TQ_OK.
+ * Keys follow TurboQuantProd (skill card, "Что делает"; discosf steps 1-3),
+ * values the group quantizer (discosf step 4). */
+tq_status tq_compress_kv(const tq_ctx* ctx, const void* k, const void* v, tq_dtype dtype,
+                         int64_t n_vec, uint8_t* k_codes, uint8_t* k_signs, uint16_t* k_norms,
+                         uint8_t* v_codes, uint16_t* v_params, void* stream);
+
+/* Bytes of device workspace tq_decode_attention needs for this shape (split-K
+ * partials and prepared queries). Returns 0 for invalid arguments. */
+size_t tq_decode_workspace_bytes(const tq_ctx* ctx, int batch, int hq, int hkv, int64_t max_len);
+
+/* One decode step of attention over a packed cache (skill card, "Что делает":
+ * scores straight from the compressed keys without dequantizing them; discosf
+ * "一句话看懂": fused decode kernels on the compressed cache).
+ *   q         device [batch][hq][d], fp32 or bf16 (q_dtype)
+ *   seq_lens  device int32 [batch] valid cache lengths (<= max_len), or NULL for
+ *             max_len everywhere; a length of 0 yields a zero output row
+ *   max_len   tokens per (sequence, KV head) slot in the packed arrays
+ *   packed    k_codes ... v_params laid out [batch][hkv][max_len][record]
+ *   hq        a multiple of hkv; query head h reads KV head h / (hq / hkv)
+ *   softmax_scale  logit scale; 0 selects 1/sqrt(d)
+ *   scores    NULL, or device fp32 [batch][hq][max_len] receiving the scaled
+ *             logits of valid positions (others untouched)
+ *   out       device fp32 [batch][hq][d]
+ *   workspace device scratch of at least tq_decode_workspace_bytes(...) bytes
+ * Returns TQ_EINVAL if the workspace is too small or any pointer is misaligned. */
+tq_status tq_decode_attention(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int batch, int hq,
+                              int hkv, const int32_t* seq_lens, int64_t max_len,
+                              const uint8_t* k_codes, const uint8_t* k_signs,
+                              const uint16_t* k_norms, const uint8_t* v_codes,
+                              const uint16_t* v_params, float softmax_scale, float* scores,
+                              float* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Instrumentation: when `start` and `stop` (cudaEvent_t passed as void*) are
+ * non-NULL, every later call on this context records `start` on its stream
+ * right before its main kernel (the compression kernel of tq_compress_kv, the
+ * split-K attention kernel of tq_decode_attention) and `stop` right after it,
+ * so a caller can time that kernel alone with cudaEventElapsedTime. NULL for
+ * both disables it. Not thread-safe with concurrent calls on the same context. */
+tq_status tq_set_profile_events(tq_ctx* ctx, void* start, void* stop);
+
+/* Decompress n_vec packed keys and/or values to fp32 [n_vec][d] (debug / parity;
+ * not on the hot path). Keys: x = n Pi^T (c[idx] + sqrt(pi/2)/m * gamma * S^T s).
+ * Values: min + scale * code. Pass NULL for the half to skip. */
+tq_status tq_decompress(const tq_ctx* ctx, const uint8_t* k_codes, const uint8_t* k_signs,
+                        const uint16_t* k_norms, const uint8_t* v_codes, const uint16_t* v_params,
+                        int64_t n_vec, float* k_out, float* v_out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H_ */

@@ -1,0 +1,81 @@
+// Internal declarations shared by the C-ABI layer and the CUDA kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/tq.h"
+
+namespace tq {
+
+constexpr int kMaxLmBits = 3;
+constexpr int kMaxLevels = 1 << kMaxLmBits;
+constexpr int kMaxD = 256;
+constexpr int kMaxM = 256;
+constexpr int kVGroup = 32;
+
+// Small method tables passed by value to every kernel (parameter space, uniform
+// across the warp, no global loads).
+struct Codebook {
+  float c[kMaxLevels];      // centroids, ascending
+  float t[kMaxLevels - 1];  // boundaries, ascending
+  int levels;               // 2^lm_bits
+  uint32_t sign_bits[kMaxD / 32];  // Hadamard sign diagonal: bit j set <=> sigma_j = -1
+};
+
+struct Shape {
+  int d;
+  int lm_bits;
+  int m;
+  int v_bits;
+  int rot;  // tq_rot
+};
+
+}  // namespace tq
+
+struct tq_ctx {
+  tq::Shape shape;
+  tq::Codebook cb;
+  int device;
+  int num_sms;
+  float* S;        // device [m][d] fp32 row-major
+  float* St;       // device [d][m] fp32 (transpose of S)
+  float* Pi;       // device [d][d] fp32 row-major (Haar only)
+  float* PiT;      // device [d][d] fp32 transpose (Haar only)
+  cudaEvent_t prof_start;  // optional events around the main kernel of each call
+  cudaEvent_t prof_stop;
+};
+
+namespace tq {
+
+// Launchers (defined in the .cu files). Return cudaSuccess or the launch error.
+cudaError_t launch_compress(const tq_ctx* ctx, const void* k, const void* v, int dtype,
+                            int64_t n_vec, uint8_t* k_codes, uint8_t* k_signs, uint16_t* k_norms,
+                            uint8_t* v_codes, uint16_t* v_params, cudaStream_t stream);
+
+struct DecodePlan {
+  int n_chunks;      // split-K chunks per (sequence, KV head)
+  int64_t chunk_len; // tokens per chunk (multiple of the tile)
+  size_t ws_q_bytes;     // prepared queries
+  size_t ws_part_bytes;  // partial (m, l, acc) per chunk and query head
+  size_t total_bytes;
+};
+
+DecodePlan plan_decode(const tq_ctx* ctx, int batch, int hq, int hkv, int64_t max_len);
+
+cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const void* q, int q_dtype,
+                          int batch, int hq, int hkv, const int32_t* seq_lens, int64_t max_len,
+                          const uint8_t* k_codes, const uint8_t* k_signs, const uint16_t* k_norms,
+                          const uint8_t* v_codes, const uint16_t* v_params, float scale,
+                          float* scores, float* out, void* workspace, cudaStream_t stream);
+
+cudaError_t launch_decompress(const tq_ctx* ctx, const uint8_t* k_codes, const uint8_t* k_signs,
+                              const uint16_t* k_norms, const uint8_t* v_codes,
+                              const uint16_t* v_params, int64_t n_vec, float* k_out, float* v_out,
+                              cudaStream_t stream);
+
+// Host math (tq_host_math.cpp).
+int lloyd_max_sphere(int d, int bits, double* centroids, double* boundaries);
+int haar_from_gaussian(int d, const double* g, double* q);
+
+}  // namespace tq

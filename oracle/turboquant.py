@@ -130,8 +130,12 @@ def lloyd_max_sphere(d: int, bits: int):
     """Codebook (centroids, boundaries) for the rotated coordinate at dimension d (R4)."""
     key = (d, bits)
     if key not in _SPHERE_CACHE:
-        _SPHERE_CACHE[key] = lloyd_max(lambda x: sphere_coordinate_pdf(x, d), -1.0, 1.0,
-                                       2 ** bits, 1.0 / math.sqrt(d))
+        c, _ = lloyd_max(lambda x: sphere_coordinate_pdf(x, d), -1.0, 1.0, 2 ** bits,
+                         1.0 / math.sqrt(d))
+        # The law is even, so the exact optimum is odd (c_k = -c_{L-1-k}); imposing it
+        # removes round-off asymmetry and puts the middle boundary exactly at 0.
+        c = 0.5 * (c - c[::-1])
+        _SPHERE_CACHE[key] = (c, 0.5 * (c[:-1] + c[1:]))
     c, t = _SPHERE_CACHE[key]
     return c.copy(), t.copy()
 

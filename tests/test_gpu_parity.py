@@ -1,0 +1,239 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs. Packed bytes must match under the exemption rule; scores and
+attention outputs from identical packed inputs within |g - o| <= 1e-4 + 1e-3 |o|."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle as O
+import workloads as W
+from _parity import (assert_close, assert_key_parity, assert_value_parity, compare_keys,
+                     compare_values, make_ctx, oracle_setup, to_np)
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # pragma: no cover - collected on CPU machines too
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import kv_cache_vector_05_b200 as T  # noqa: E402
+
+DEV = "cuda:0"
+
+
+def _compress_both(K, V, d, lm_bits, v_bits, rotation, dtype, m=None):
+    m = m or d
+    ctx = make_ctx(T, d, lm_bits, v_bits, m, rotation)
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    kt = torch.from_numpy(np.ascontiguousarray(K, np.float32)).to(DEV).to(tdt)
+    vt = torch.from_numpy(np.ascontiguousarray(V, np.float32)).to(DEV).to(tdt)
+    g = to_np(T.tq_compress_kv(ctx, kt, vt))
+    torch.cuda.synchronize()
+    Pi, c, t, S = oracle_setup(d, lm_bits, m, rotation)
+    # the oracle sees exactly the values the device read
+    Kx = kt.float().cpu().numpy().astype(np.float64)
+    Vx = vt.float().cpu().numpy().astype(np.float64)
+    ok = O.compress_keys(Kx, Pi, c, t, S, with_diagnostics=True)
+    ov = O.quantize_values(Vx, v_bits, with_diagnostics=True)
+    return ctx, g, ok, ov
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("lm_bits", [1, 2, 3])
+@pytest.mark.parametrize("rotation", ["hadamard", "haar"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_compress_parity_small(d, lm_bits, rotation, dtype):
+    v_bits = 2 if (d + lm_bits) % 2 else 4
+    n = 1531                                            # several CTAs plus a ragged tail
+    rng = np.random.default_rng([d, lm_bits])
+    K = rng.standard_normal((n, d)).astype(np.float32) * rng.lognormal(0, 1, d).astype(np.float32)
+    V = rng.standard_normal((n, d)).astype(np.float32)
+    K[[0, 700, n - 1]] = 0.0                             # zero keys
+    V[5, :32] = 0.75                                     # a constant value group
+    ctx, g, ok, ov = _compress_both(K, V, d, lm_bits, v_bits, rotation, dtype)
+    ks = compare_keys(g, ok, d, lm_bits, d)
+    vs = compare_values(g, ov, d, v_bits)
+    assert_key_parity(ks)
+    assert_value_parity(vs)
+
+
+def test_compress_parity_qwen_outlier_keys():
+    """One (layer, head) of the Qwen2.5-3B-shaped cache: lognormal channel scales with x20 outliers."""
+    K, V = W.qwen_layer_head_kv(layer=17, head=1)
+    ctx, g, ok, ov = _compress_both(K, V, 128, 2, 2, "hadamard", "bf16")
+    assert_key_parity(compare_keys(g, ok, 128, 2, 128))
+    assert_value_parity(compare_values(g, ov, 128, 2))
+
+
+@pytest.mark.parametrize("rotation", ["hadamard", "haar"])
+def test_compress_parity_full_sweep_size_sampled(rotation):
+    """1,048,576 bf16 N(0,1) vectors (16384 tokens x 64 heads), d=128, 3-bit keys:
+    the whole batch is compressed in one call; the oracle checks a sample."""
+    d, lm_bits, v_bits, n = 128, 2, 2, W.SWEEP_VECTORS
+    ctx = make_ctx(T, d, lm_bits, v_bits, rotation=rotation)
+    gen = torch.Generator(device=DEV)
+    gen.manual_seed(0)
+    kt = torch.randn((n, d), generator=gen, device=DEV).to(torch.bfloat16)
+    vt = torch.randn((n, d), generator=gen, device=DEV).to(torch.bfloat16)
+    g = T.tq_compress_kv(ctx, kt, vt)
+    torch.cuda.synchronize()
+    idx = np.unique(np.concatenate([np.random.default_rng(1).integers(0, n, 12000), [0, n - 1]]))
+    it = torch.from_numpy(idx).to(DEV)
+    gs = to_np({k: v[it] for k, v in g.items()})
+    Pi, c, t, S = oracle_setup(d, lm_bits, d, rotation)
+    Kx = kt[it].float().cpu().numpy().astype(np.float64)
+    Vx = vt[it].float().cpu().numpy().astype(np.float64)
+    ks = compare_keys(gs, O.compress_keys(Kx, Pi, c, t, S, with_diagnostics=True), d, lm_bits, d)
+    vs = compare_values(gs, O.quantize_values(Vx, v_bits, with_diagnostics=True), d, v_bits)
+    assert_key_parity(ks)
+    assert_value_parity(vs)
+
+
+def test_compress_edge_cases():
+    ctx = make_ctx(T, 128, 2, 2)
+    empty = torch.empty((0, 128), device=DEV)
+    T.tq_compress_kv(ctx, empty, empty)                      # n = 0 is a no-op
+    one = torch.randn((1, 128), device=DEV)
+    g = to_np(T.tq_compress_kv(ctx, one, None))
+    Pi, c, t, S = oracle_setup(128, 2)
+    ok = O.compress_keys(one.cpu().numpy().astype(np.float64), Pi, c, t, S, with_diagnostics=True)
+    assert_key_parity(compare_keys(g, ok, 128, 2, 128))
+    big = torch.randn((3, 129), device=DEV)
+    misaligned = big.view(-1)[1:1 + 256].view(2, 128)       # 4-byte offset
+    with pytest.raises(T.TQError):
+        T.tq_compress_kv(ctx, misaligned, None)
+
+
+# ------------------------------------------------------------------ decode
+
+def _upload(packed: dict):
+    out = {}
+    for k, v in packed.items():
+        a = np.ascontiguousarray(v)
+        if a.dtype == np.uint16:
+            a = a.view(np.int16)
+        out[k] = torch.from_numpy(a).to(DEV)
+    return out
+
+
+def _oracle_unit(packed, u, max_len, length, q, Pi, c, S, d, v_bits, scale=None):
+    sl = slice(u * max_len, u * max_len + length)
+    pk = {"codes": packed["k_codes"][sl], "signs": packed["k_signs"][sl], "norms": packed["k_norms"][sl]}
+    pv = {"codes": packed["v_codes"][sl], "params": packed["v_params"][sl]}
+    return O.decode_attention(q, pk, pv, Pi, c, S, d, v_bits, scale=scale)
+
+
+def _decode_check(d, lm_bits, v_bits, batch, hkv, G, max_len, lens, rotation="hadamard",
+                  q_dtype="f32", packed=None, units=None, scale=0.0, with_scores=True):
+    m = d
+    hq = hkv * G
+    ctx = make_ctx(T, d, lm_bits, v_bits, m, rotation)
+    n_vec = batch * hkv * max_len
+    if packed is None:
+        packed = W.random_packed_cache(n_vec, d, lm_bits, m, v_bits, seed=d + lm_bits)
+    q = W.queries((batch, hq, d), dtype=q_dtype)
+    qt = torch.from_numpy(q).to(DEV)
+    if q_dtype == "bf16":
+        qt = qt.to(torch.bfloat16)
+    dp = _upload(packed)
+    lens_t = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    scores = torch.full((batch, hq, max_len), float("nan"), device=DEV) if with_scores else None
+    out, _ = T.tq_decode_attention(ctx, qt, dp, batch, hq, hkv, max_len, seq_lens=lens_t,
+                                   softmax_scale=scale, scores=scores)
+    torch.cuda.synchronize()
+    out = out.cpu().numpy()
+    sc = scores.cpu().numpy() if with_scores else None
+    Pi, c, t, S = oracle_setup(d, lm_bits, m, rotation)
+    units = range(batch * hkv) if units is None else units
+    for u in units:
+        b, kvh = divmod(u, hkv)
+        L = lens[b]
+        qs = q[b, kvh * G:(kvh + 1) * G].astype(np.float64)
+        os_, oo = _oracle_unit(packed, u, max_len, L, qs, Pi, c, S, d, v_bits,
+                               scale=(scale if scale > 0 else None))
+        assert_close(out[b, kvh * G:(kvh + 1) * G], oo, what=f"out unit {u}")
+        if with_scores:
+            assert_close(sc[b, kvh * G:(kvh + 1) * G, :L], os_, what=f"scores unit {u}")
+            assert np.isnan(sc[b, kvh * G:(kvh + 1) * G, L:]).all()
+    return out
+
+
+def test_decode_single_head_fp32_oracle_compressed():
+    """4096 fp32 N(0,1) keys/values, 8 queries on one head: 3-bit keys, 4-bit values;
+    the packed cache comes from the oracle's own compression."""
+    K, V, Q = W.single_head_kvq()
+    Pi, c, t, S = oracle_setup(128, 2)
+    pk = O.compress_keys(K.astype(np.float64), Pi, c, t, S)
+    pv = O.quantize_values(V.astype(np.float64), 4)
+    packed = {"k_codes": pk["codes"], "k_signs": pk["signs"], "k_norms": pk["norms"],
+              "v_codes": pv["codes"], "v_params": pv["params"]}
+    ctx = make_ctx(T, 128, 2, 4)
+    qt = torch.from_numpy(Q).to(DEV).view(1, 8, 128)
+    scores = torch.empty((1, 8, 4096), device=DEV)
+    out, _ = T.tq_decode_attention(ctx, qt, _upload(packed), 1, 8, 1, 4096, scores=scores)
+    torch.cuda.synchronize()
+    os_, oo = O.decode_attention(Q.astype(np.float64), pk, pv, Pi, c, S, 128, 4)
+    assert_close(scores.cpu().numpy()[0], os_, what="scores")
+    assert_close(out.cpu().numpy()[0], oo, what="out")
+
+
+@pytest.mark.parametrize("d,lm_bits,v_bits,G", [
+    (128, 2, 2, 4), (128, 2, 2, 8), (128, 3, 4, 6), (128, 1, 4, 1),
+    (64, 2, 4, 8), (64, 3, 2, 5), (256, 2, 2, 4), (256, 3, 4, 2), (256, 1, 2, 8),
+])
+def test_decode_parity_random_cache(d, lm_bits, v_bits, G):
+    _decode_check(d, lm_bits, v_bits, batch=2, hkv=2, G=G, max_len=1100, lens=[1100, 577])
+
+
+def test_decode_parity_haar_bf16_queries_custom_scale():
+    _decode_check(128, 2, 2, batch=1, hkv=3, G=4, max_len=700, lens=[699], rotation="haar",
+                  q_dtype="bf16", scale=0.05)
+
+
+def test_decode_empty_and_tiny_sequences():
+    out = _decode_check(128, 2, 2, batch=3, hkv=1, G=4, max_len=130, lens=[0, 1, 130])
+    assert not out[0].any()
+
+
+@pytest.mark.parametrize("name,units", [
+    ("qwen2.5-3b_8k_k3v2", [0, 71]),
+    ("llama8b_b32_32k_k3v2", [0, 255]),
+    ("long_1m_k4v4", [3]),
+])
+def test_decode_parity_full_size_sampled(name, units):
+    """Full-size caches in the benchmark's launch configuration; the oracle
+    recomputes every output of the sampled (sequence, KV head) units."""
+    w = W.WORKLOADS[name]
+    packed = W.random_packed_cache(w.units * w.tokens, w.d, w.lm_bits, w.m, w.v_bits, seed=11)
+    lens = [w.tokens] * w.batch
+    _decode_check(w.d, w.lm_bits, w.v_bits, w.batch, w.hkv, w.group, w.tokens, lens,
+                  q_dtype=w.dtype, packed=packed, units=units, with_scores=(name != "long_1m_k4v4"))
+
+
+def test_decode_rejects_small_workspace():
+    ctx = make_ctx(T, 128, 2, 2)
+    packed = _upload(W.random_packed_cache(256, 128, 2, 128, 2))
+    q = torch.randn((1, 4, 128), device=DEV)
+    with pytest.raises(T.TQError):
+        T.tq_decode_attention(ctx, q, packed, 1, 4, 1, 256, workspace=torch.empty(256, dtype=torch.uint8, device=DEV))
+
+
+# ------------------------------------------------------------------ decompress
+
+@pytest.mark.parametrize("rotation", ["hadamard", "haar"])
+@pytest.mark.parametrize("d,lm_bits,v_bits", [(128, 2, 2), (64, 3, 4), (256, 1, 4)])
+def test_decompress_parity(rotation, d, lm_bits, v_bits):
+    rng = np.random.default_rng(6)
+    K = rng.standard_normal((777, d))
+    V = rng.standard_normal((777, d))
+    Pi, c, t, S = oracle_setup(d, lm_bits, d, rotation)
+    pk = O.compress_keys(K, Pi, c, t, S)
+    pv = O.quantize_values(V, v_bits)
+    packed = _upload({"k_codes": pk["codes"], "k_signs": pk["signs"], "k_norms": pk["norms"],
+                      "v_codes": pv["codes"], "v_params": pv["params"]})
+    ctx = make_ctx(T, d, lm_bits, v_bits, d, rotation)
+    kx, vx = T.tq_decompress(ctx, packed, 777)
+    torch.cuda.synchronize()
+    assert_close(kx.cpu().numpy(), O.decompress_keys(pk, Pi, c, S, d), rtol=1e-4, atol=1e-5, what="keys")
+    assert_close(vx.cpu().numpy(), O.dequantize_values(pv, v_bits, d), rtol=1e-6, atol=1e-6, what="values")
