@@ -307,6 +307,8 @@ def run_ours(args, w: W.Workload):
         evs = []
         for _ in range(n):
             e = [E(enable_timing=True) for _ in range(8)]
+            for ev in (e[1], e[2], e[5], e[6]):
+                ev.record()  # torch creates the CUDA event lazily; the library re-records it
             flush_buf.zero_()
             e[0].record()
             if record:

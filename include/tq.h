@@ -137,7 +137,8 @@ tq_status tq_haar_from_gaussian(int d, const double* gaussian, double* pi_out);
  *   k, v      device [n_vec][d] of `dtype` (fp32 or bf16); either may be NULL to
  *             skip that half (its output pointers are then ignored)
  *   k_codes, k_signs, k_norms, v_codes, v_params: device outputs, formats above
- * Each output record is written in full; n_vec = 0 is a no-op returning TQ_OK.
+ * Each output record is written in full. n_vec = 0 returns TQ_OK before any
+ * pointer is examined (NULL buffers are fine then).
  * Keys follow TurboQuantProd (skill card, "Что делает"; discosf steps 1-3),
  * values the group quantizer (discosf step 4). */
 tq_status tq_compress_kv(const tq_ctx* ctx, const void* k, const void* v, tq_dtype dtype,

@@ -191,6 +191,7 @@ tq_status tq_compress_kv(const tq_ctx* c, const void* k, const void* v, tq_dtype
                          uint16_t* v_params, void* stream) {
   if (!c) return fail(TQ_EINVAL, "tq_compress_kv: NULL context");
   if (n_vec < 0) return fail(TQ_EINVAL, "tq_compress_kv: negative n_vec");
+  if (n_vec == 0) return TQ_OK;
   if (dtype != TQ_F32 && dtype != TQ_BF16) return fail(TQ_EINVAL, "tq_compress_kv: bad dtype");
   if (!k && !v) return fail(TQ_EINVAL, "tq_compress_kv: both k and v are NULL");
   if (k && (!k_codes || !k_signs || !k_norms))
@@ -251,6 +252,7 @@ tq_status tq_decompress(const tq_ctx* c, const uint8_t* k_codes, const uint8_t* 
                         int64_t n_vec, float* k_out, float* v_out, void* stream) {
   if (!c) return fail(TQ_EINVAL, "tq_decompress: NULL context");
   if (n_vec < 0) return fail(TQ_EINVAL, "tq_decompress: negative n_vec");
+  if (n_vec == 0) return TQ_OK;
   if (!k_out && !v_out) return fail(TQ_EINVAL, "tq_decompress: both outputs NULL");
   if (k_out && (!k_codes || !k_signs || !k_norms)) return fail(TQ_EINVAL, "tq_decompress: NULL key input");
   if (v_out && (!v_codes || !v_params)) return fail(TQ_EINVAL, "tq_decompress: NULL value input");
