@@ -171,6 +171,34 @@ tq_status tq_decode_attention(const tq_ctx* ctx, const void* q, tq_dtype q_dtype
                               const uint16_t* v_params, float softmax_scale, float* scores,
                               float* out, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Decode attention that allocates nothing and takes no workspace. The paper has
+ * no counterpart; this entry point exists for callers that cannot allocate device
+ * memory: a plugin that is handed only input and output pointers by its host
+ * application, a serving loop that must not call cudaMalloc once running (the
+ * allocation can synchronize the device and stall other streams), or a runtime
+ * without a caching allocator.
+ * Same arguments, layouts and results as tq_decode_attention, minus workspace.
+ * The scratch is a fixed device array of tq_decode_static_scratch_capacity()
+ * bytes (8 MiB) inside this library; every GPU that loads the library holds one
+ * until the process exits. A shape whose workspace (tq_decode_workspace_bytes)
+ * exceeds it returns TQ_EUNSUPPORTED with the sizes in tq_last_error().
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call before
+ * any stream capture. All calls on a device share the one array and it keeps
+ * the last call's contents: every byte a call reads is written earlier in the
+ * same call, but calls whose work overlaps on the GPU (different streams, or
+ * host threads without ordering) race on it and must be serialized.
+ * The context must belong to the current device. */
+tq_status tq_decode_attention_static(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int batch,
+                                     int hq, int hkv, const int32_t* seq_lens, int64_t max_len,
+                                     const uint8_t* k_codes, const uint8_t* k_signs,
+                                     const uint16_t* k_norms, const uint8_t* v_codes,
+                                     const uint16_t* v_params, float softmax_scale, float* scores,
+                                     float* out, void* stream);
+
+/* Bytes of the fixed scratch array tq_decode_attention_static uses (no GPU needed). */
+size_t tq_decode_static_scratch_capacity(void);
+
 /* Instrumentation: when `start` and `stop` (cudaEvent_t passed as void*) are
  * non-NULL, every later call on this context records `start` on its stream
  * right before its main kernel (the compression kernel of tq_compress_kv, the

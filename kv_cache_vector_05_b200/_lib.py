@@ -22,7 +22,7 @@ EXPORTED = (
     "tq_codebook_load", "tq_free", "tq_status_string", "tq_last_error",
     "tq_lloyd_max_codebook", "tq_haar_from_gaussian", "tq_compress_kv",
     "tq_decode_workspace_bytes", "tq_decode_attention", "tq_decompress",
-    "tq_set_profile_events",
+    "tq_set_profile_events", "tq_decode_attention_static", "tq_decode_static_scratch_capacity",
 )
 
 
@@ -76,6 +76,11 @@ def _load() -> ctypes.CDLL:
     lib.tq_decode_attention.restype = c_int
     lib.tq_decompress.argtypes = [vp, vp, vp, vp, vp, vp, i64, vp, vp, vp]
     lib.tq_decompress.restype = c_int
+    lib.tq_decode_attention_static.argtypes = [vp, vp, c_int, c_int, c_int, c_int, vp, i64,
+                                               vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp]
+    lib.tq_decode_attention_static.restype = c_int
+    lib.tq_decode_static_scratch_capacity.argtypes = []
+    lib.tq_decode_static_scratch_capacity.restype = sz
     lib.tq_set_profile_events.argtypes = [vp, vp, vp]
     lib.tq_set_profile_events.restype = c_int
     return lib
@@ -256,6 +261,28 @@ def tq_decode_attention(ctx: Context, q, packed: dict, batch: int, hq: int, hkv:
         _ptr(packed["v_codes"]), _ptr(packed["v_params"]), float(softmax_scale),
         _ptr(scores), _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)), "tq_decode_attention")
     return out, scores
+
+
+def tq_decode_attention_static(ctx: Context, q, packed: dict, batch: int, hq: int, hkv: int,
+                               max_len: int, seq_lens=None, softmax_scale: float = 0.0, scores=None,
+                               out=None, stream=None):
+    """tq_decode_attention without a workspace: the library's fixed scratch array is
+    used instead (for callers that cannot allocate device memory; see include/tq.h)."""
+    import torch
+    q_dtype = TQ_F32 if q.dtype == torch.float32 else TQ_BF16
+    assert q.is_contiguous() and q.numel() == batch * hq * ctx.d
+    if out is None:
+        out = torch.empty((batch, hq, ctx.d), dtype=torch.float32, device=q.device)
+    _check(lib.tq_decode_attention_static(
+        ctx.handle, _ptr(q), q_dtype, batch, hq, hkv, _ptr(seq_lens), max_len,
+        _ptr(packed["k_codes"]), _ptr(packed["k_signs"]), _ptr(packed["k_norms"]),
+        _ptr(packed["v_codes"]), _ptr(packed["v_params"]), float(softmax_scale),
+        _ptr(scores), _ptr(out), _stream(stream)), "tq_decode_attention_static")
+    return out, scores
+
+
+def tq_decode_static_scratch_capacity() -> int:
+    return int(lib.tq_decode_static_scratch_capacity())
 
 
 def tq_decompress(ctx: Context, packed: dict, n_vec: int, keys: bool = True, values: bool = True,

@@ -37,6 +37,10 @@ void free_tables(tq_ctx* c) {
 
 }  // namespace
 
+namespace tq {
+void set_last_error(const char* msg) { std::snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+}  // namespace tq
+
 extern "C" {
 
 const char* tq_status_string(tq_status s) {

@@ -74,6 +74,9 @@ cudaError_t launch_decompress(const tq_ctx* ctx, const uint8_t* k_codes, const u
                               const uint16_t* v_params, int64_t n_vec, float* k_out, float* v_out,
                               cudaStream_t stream);
 
+// Records the message tq_last_error() returns on this thread (tq_api.cpp).
+void set_last_error(const char* msg);
+
 // Host math (tq_host_math.cpp).
 int lloyd_max_sphere(int d, int bits, double* centroids, double* boundaries);
 int haar_from_gaussian(int d, const double* g, double* q);
