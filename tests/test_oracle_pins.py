@@ -145,7 +145,9 @@ def test_sphere_lloyd_max_optimality_conditions(d, bits):
     for k in range(len(c)):
         assert abs(c[k] - _sphere_cell_mean(edges[k], edges[k + 1], d)) < 1e-12
     np.testing.assert_array_equal(t, 0.5 * (c[:-1] + c[1:]))
-    np.testing.assert_allclose(c, -c[::-1], rtol=0, atol=1e-14)
+    np.testing.assert_array_equal(c, -c[::-1])          # the law is even: the optimum is odd
+    if bits > 0:
+        assert t[len(t) // 2] == 0.0                       # middle boundary exactly at zero
     assert np.all(np.diff(c) > 0)
 
 
