@@ -171,6 +171,14 @@ tq_status tq_decode_attention(const tq_ctx* ctx, const void* q, tq_dtype q_dtype
                               const uint16_t* v_params, float softmax_scale, float* scores,
                               float* out, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Synchronize `stream`, then read and clear the context's device error word.
+ * Kernels never spin without a bound: a wait for a staged copy that does not
+ * complete in time sets this word, abandons the rest of its work and exits, so
+ * the CUDA context stays usable. Returns TQ_ECUDA (with tq_last_error() saying
+ * which wait) if any call since the last check hit such a timeout, TQ_OK
+ * otherwise. */
+tq_status tq_check_device(const tq_ctx* ctx, void* stream);
+
 /* Decode attention that allocates nothing and takes no workspace. The paper has
  * no counterpart; this entry point exists for callers that cannot allocate device
  * memory: a plugin that is handed only input and output pointers by its host

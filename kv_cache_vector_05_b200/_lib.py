@@ -22,7 +22,7 @@ EXPORTED = (
     "tq_codebook_load", "tq_free", "tq_status_string", "tq_last_error",
     "tq_lloyd_max_codebook", "tq_haar_from_gaussian", "tq_compress_kv",
     "tq_decode_workspace_bytes", "tq_decode_attention", "tq_decompress",
-    "tq_set_profile_events", "tq_decode_attention_static", "tq_decode_static_scratch_capacity",
+    "tq_set_profile_events", "tq_check_device", "tq_decode_attention_static", "tq_decode_static_scratch_capacity",
 )
 
 
@@ -81,6 +81,8 @@ def _load() -> ctypes.CDLL:
     lib.tq_decode_attention_static.restype = c_int
     lib.tq_decode_static_scratch_capacity.argtypes = []
     lib.tq_decode_static_scratch_capacity.restype = sz
+    lib.tq_check_device.argtypes = [vp, vp]
+    lib.tq_check_device.restype = c_int
     lib.tq_set_profile_events.argtypes = [vp, vp, vp]
     lib.tq_set_profile_events.restype = c_int
     return lib
@@ -199,6 +201,11 @@ def tq_codebook_load(d: int, k_lm_bits: int, v_bits: int, centroids, boundaries,
 
 def tq_free(ctx: Context) -> None:
     ctx.close()
+
+
+def tq_check_device(ctx: Context, stream=None) -> None:
+    """Synchronize and raise TQError if a kernel's bounded wait timed out since the last check."""
+    _check(lib.tq_check_device(ctx.handle, _stream(stream)), "tq_check_device")
 
 
 def tq_set_profile_events(ctx: Context, start=None, stop=None) -> None:

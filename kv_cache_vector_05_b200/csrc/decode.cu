@@ -350,9 +350,11 @@ cudaError_t dispatch_lmb(const DecodeArgs& a, int lmb, int vb, dim3 grid, size_t
 DecodePlan plan_decode(const tq_ctx* ctx, int batch, int hq, int hkv, int64_t max_len) {
   DecodePlan p{};
   const int d = ctx->shape.d, m = ctx->shape.m, G = hq / hkv;
+  p.mma = mma_decode_supported(ctx, G);
   const int64_t units = (int64_t)batch * hkv;
   const int64_t tiles = max_len > 0 ? (max_len + kTile - 1) / kTile : 1;
-  const int64_t target = 4LL * (ctx->num_sms > 0 ? ctx->num_sms : 148);
+  // CTAs to aim for: a few waves of the resident CTAs per SM
+  const int64_t target = (p.mma ? 6LL : 4LL) * (ctx->num_sms > 0 ? ctx->num_sms : 148);
   int64_t chunks = units > 0 ? (target + units - 1) / units : 1;
   if (chunks > tiles) chunks = tiles;
   if (chunks < 1) chunks = 1;
@@ -416,11 +418,16 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const void*
   const dim3 grid(plan.n_chunks, batch * hkv);
   const size_t smem = decode_smem_bytes(d, m, G, ctx->shape.v_bits);
   if (ctx->prof_start) cudaEventRecord(ctx->prof_start, stream);
-  switch (d) {
-    case 64: e = dispatch_lmb<64>(a, ctx->shape.lm_bits, ctx->shape.v_bits, grid, smem, stream); break;
-    case 128: e = dispatch_lmb<128>(a, ctx->shape.lm_bits, ctx->shape.v_bits, grid, smem, stream); break;
-    case 256: e = dispatch_lmb<256>(a, ctx->shape.lm_bits, ctx->shape.v_bits, grid, smem, stream); break;
-    default: return cudaErrorInvalidValue;
+  if (plan.mma) {
+    e = launch_decode_mma(ctx, plan, ws_q, d + m, ws_part, d + kPartPad, batch, hq, hkv, seq_lens, max_len,
+                          k_codes, k_signs, k_norms, v_codes, v_params, scale, scores, stream);
+  } else {
+    switch (d) {
+      case 64: e = dispatch_lmb<64>(a, ctx->shape.lm_bits, ctx->shape.v_bits, grid, smem, stream); break;
+      case 128: e = dispatch_lmb<128>(a, ctx->shape.lm_bits, ctx->shape.v_bits, grid, smem, stream); break;
+      case 256: e = dispatch_lmb<256>(a, ctx->shape.lm_bits, ctx->shape.v_bits, grid, smem, stream); break;
+      default: return cudaErrorInvalidValue;
+    }
   }
   if (ctx->prof_stop) cudaEventRecord(ctx->prof_stop, stream);
   if (e != cudaSuccess) return e;

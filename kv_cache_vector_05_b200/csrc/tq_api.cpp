@@ -33,6 +33,7 @@ void free_tables(tq_ctx* c) {
   cudaFree(c->St);
   cudaFree(c->Pi);
   cudaFree(c->PiT);
+  cudaFree(c->d_err);
 }
 
 }  // namespace
@@ -151,6 +152,7 @@ tq_status tq_codebook_load(const tq_params* p, void* stream, tq_ctx** out) {
   if (e == cudaSuccess) e = alloc(&c->St, St.size());
   if (e == cudaSuccess && !Pi.empty()) e = alloc(&c->Pi, Pi.size());
   if (e == cudaSuccess && !Pi.empty()) e = alloc(&c->PiT, PiT.size());
+  if (e == cudaSuccess) e = cudaMalloc((void**)&c->d_err, sizeof(unsigned int));
   if (e != cudaSuccess) {
     free_tables(c);
     delete c;
@@ -165,6 +167,7 @@ tq_status tq_codebook_load(const tq_params* p, void* stream, tq_ctx** out) {
     e = cudaMemcpyAsync(c->Pi, Pi.data(), Pi.size() * sizeof(float), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess && !Pi.empty())
     e = cudaMemcpyAsync(c->PiT, PiT.data(), PiT.size() * sizeof(float), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(c->d_err, 0, sizeof(unsigned int), s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) {
     free_tables(c);
@@ -181,6 +184,18 @@ tq_status tq_set_profile_events(tq_ctx* c, void* start, void* stop) {
     return fail(TQ_EINVAL, "tq_set_profile_events: give both events or neither");
   c->prof_start = static_cast<cudaEvent_t>(start);
   c->prof_stop = static_cast<cudaEvent_t>(stop);
+  return TQ_OK;
+}
+
+tq_status tq_check_device(const tq_ctx* c, void* stream) {
+  if (!c) return fail(TQ_EINVAL, "tq_check_device: NULL context");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned int flag = 0;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemcpy(&flag, c->d_err, sizeof(flag), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && flag) e = cudaMemset(c->d_err, 0, sizeof(flag));
+  if (e != cudaSuccess) return fail_cuda(e, "tq_check_device");
+  if (flag & 1u) return fail(TQ_ECUDA, "tq_check_device: a bounded wait for a bulk copy timed out; results of that call are invalid");
   return TQ_OK;
 }
 

@@ -44,6 +44,7 @@ struct tq_ctx {
   float* PiT;      // device [d][d] fp32 transpose (Haar only)
   cudaEvent_t prof_start;  // optional events around the main kernel of each call
   cudaEvent_t prof_stop;
+  unsigned int* d_err;     // device error word: bit 0 = a bounded wait in a kernel timed out
 };
 
 namespace tq {
@@ -54,6 +55,7 @@ cudaError_t launch_compress(const tq_ctx* ctx, const void* k, const void* v, int
                             uint8_t* v_codes, uint16_t* v_params, cudaStream_t stream);
 
 struct DecodePlan {
+  bool mma;          // tensor-core kernel (decode_mma.cu) instead of the generic one
   int n_chunks;      // split-K chunks per (sequence, KV head)
   int64_t chunk_len; // tokens per chunk (multiple of the tile)
   size_t ws_q_bytes;     // prepared queries
@@ -68,6 +70,14 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const void*
                           const uint8_t* k_codes, const uint8_t* k_signs, const uint16_t* k_norms,
                           const uint8_t* v_codes, const uint16_t* v_params, float scale,
                           float* scores, float* out, void* workspace, cudaStream_t stream);
+
+bool mma_decode_supported(const tq_ctx* ctx, int G);
+
+cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const float* ws_q, int q_stride,
+                              float* ws_part, int part_stride, int batch, int hq, int hkv,
+                              const int32_t* seq_lens, int64_t max_len, const uint8_t* k_codes,
+                              const uint8_t* k_signs, const uint16_t* k_norms, const uint8_t* v_codes,
+                              const uint16_t* v_params, float scale, float* scores, cudaStream_t stream);
 
 cudaError_t launch_decompress(const tq_ctx* ctx, const uint8_t* k_codes, const uint8_t* k_signs,
                               const uint16_t* k_norms, const uint8_t* v_codes,
