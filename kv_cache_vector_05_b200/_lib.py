@@ -12,7 +12,8 @@ import os
 
 import numpy as np
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtq.so")
+# TQ_LIBRARY may name another build of the same library (e.g. a debug build).
+LIB_PATH = os.environ.get("TQ_LIBRARY") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtq.so")
 
 TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED, TQ_ECUDA, TQ_ENOMEM = 0, 1, 2, 3, 4
 TQ_F32, TQ_BF16 = 0, 1

@@ -11,6 +11,7 @@
 #include <cuda_runtime.h>
 
 #include "tq_device.cuh"
+#include "tq_sm100.cuh"
 
 namespace tq {
 namespace {
@@ -28,13 +29,18 @@ struct CompressArgs {
   uint16_t* v_params;
   const float* St;   // [d][m]
   const float* PiT;  // [d][d], Haar only
+  const uint16_t* S_sw128;  // S as f16 in the swizzled K-major operand layout (tensor-core path)
+  unsigned int* err;
   Codebook cb;
   int lm_bits, m, v_bits, rot;
   float inv_sqrt_d;  // 1/sqrt(d) rounded once from fp64
 };
 
+// Norm, rotation, Lloyd-Max codes and residual of key i; writes the packed codes
+// and (n, gamma). Returns false for a zero key (all its bytes already written as 0);
+// otherwise leaves the lane's residual coordinates in r.
 template <int D, typename T>
-__device__ void compress_key(const CompressArgs& a, int64_t i, int lane, float* rbuf) {
+__device__ bool key_front(const CompressArgs& a, int64_t i, int lane, float* rbuf, float (&r)[D / 32]) {
   constexpr int E = D / 32;
   float x[E];
   load_lane<E>(static_cast<const T*>(a.k) + i * D, lane, x);
@@ -51,7 +57,7 @@ __device__ void compress_key(const CompressArgs& a, int64_t i, int lane, float* 
     if (lane < cbytes / 4) codes_out[lane] = 0u;
     if (lane < a.m / 32) signs_out[lane] = 0u;
     if (lane == 0) reinterpret_cast<uint32_t*>(a.k_norms)[i] = 0u;
-    return;
+    return false;
   }
   const float inv_n = 1.0f / n;
 
@@ -80,7 +86,6 @@ __device__ void compress_key(const CompressArgs& a, int64_t i, int lane, float* 
 
   // Lloyd-Max bucketize: code = #{k : y >= t_k}; residual against its centroid.
   uint32_t code_bits = 0;
-  float r[E];
   float rr = 0.f;
 #pragma unroll
   for (int e = 0; e < E; ++e) {
@@ -98,7 +103,21 @@ __device__ void compress_key(const CompressArgs& a, int64_t i, int lane, float* 
     rr = fmaf(r[e], r[e], rr);
   }
   const float gamma = sqrtf(warp_sum(rr));
+  const uint32_t code_word = pack_stream_word(code_bits, E * a.lm_bits, cbytes / 4, lane);
+  if (lane < cbytes / 4) codes_out[lane] = code_word;
+  if (lane == 0) {
+    const uint32_t nb = __half_as_ushort(__float2half_rn(n));
+    const uint32_t gb = __half_as_ushort(__float2half_rn(gamma));
+    reinterpret_cast<uint32_t*>(a.k_norms)[i] = nb | (gb << 16);
+  }
+  return true;
+}
 
+template <int D, typename T>
+__device__ void compress_key(const CompressArgs& a, int64_t i, int lane, float* rbuf) {
+  constexpr int E = D / 32;
+  float r[E];
+  if (!key_front<D, T>(a, i, lane, rbuf, r)) return;
   // QJL: sign bits of S r; lane computes rows i = lane + 32*q so a ballot gives word q.
 #pragma unroll
   for (int e = 0; e < E; ++e) rbuf[lane * E + e] = r[e];
@@ -112,15 +131,7 @@ __device__ void compress_key(const CompressArgs& a, int64_t i, int lane, float* 
     if (lane == q) my_sign_word = word;
   }
   __syncwarp();
-
-  const uint32_t code_word = pack_stream_word(code_bits, E * a.lm_bits, cbytes / 4, lane);
-  if (lane < cbytes / 4) codes_out[lane] = code_word;
-  if (lane < a.m / 32) signs_out[lane] = my_sign_word;
-  if (lane == 0) {
-    const uint32_t nb = __half_as_ushort(__float2half_rn(n));
-    const uint32_t gb = __half_as_ushort(__float2half_rn(gamma));
-    reinterpret_cast<uint32_t*>(a.k_norms)[i] = nb | (gb << 16);
-  }
+  if (lane < a.m / 32) reinterpret_cast<uint32_t*>(a.k_signs + i * (a.m / 8))[lane] = my_sign_word;
 }
 
 template <int D, typename T>
@@ -188,7 +199,198 @@ cudaError_t launch_d(const tq_ctx* ctx, const CompressArgs& a, int dtype, cudaSt
   return e;
 }
 
+// ---------------------------------------------------------------------------------
+// Tensor-core variant (d = m = 128): the QJL projection S r of 128 keys at a time is
+// one 128 x 128 x 128 MMA on the 5th-generation tensor cores. Warps 0-3 rotate and
+// quantize the keys (one key per warp step, as above) and write the residuals,
+// scaled by 16 and split into f16 hi + lo, to two swizzled shared-memory operand
+// tiles; one thread issues 2 x 8 tcgen05.mma (hi and lo against the f16 matrix S,
+// which is exact in f16) into a 128 x 128 fp32 accumulator in tensor memory; after
+// the commit barrier each thread reads its key's 128 projections back and packs the
+// sign bits. Warps 4-7 group-quantize the values of the same tile meanwhile.
+constexpr int kTcRows = 128;
+constexpr int kTcThreads = 256;
+constexpr uint32_t kTcTileBytes = kTcRows * 128 * 2;  // one f16 operand tile, 32 KB
+
+struct TcSmem {
+  static constexpr uint32_t A_HI = 0, A_LO = kTcTileBytes, S = 2 * kTcTileBytes;
+  static constexpr uint32_t RBUF = 3 * kTcTileBytes;         // [4 warps][128] fp32
+  static constexpr uint32_t ZF = RBUF + 4 * 128 * 4;         // [128] nonzero flags
+  static constexpr uint32_t BAR = ZF + 128;                  // mbarrier
+  static constexpr uint32_t TMEM = BAR + 8;                  // TMEM base address
+  static constexpr uint32_t BYTES = TMEM + 8;
+};
+
+__device__ __forceinline__ bool kwarps_sync_or(bool v) {
+  // barrier 1 over the 128 key threads (warps 0-3), OR-reduced predicate
+  uint32_t r;
+  asm volatile(
+      "{ .reg .pred p, q; setp.ne.u32 p, %1, 0; barrier.red.or.pred q, 1, 128, p; selp.u32 %0, 1, 0, q; }"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kTcThreads, 2) compress_tc_kernel(const __grid_constant__ CompressArgs a) {
+  namespace s1 = tq::sm100;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = s1::smem_u32(sm);
+  float* rbuf = reinterpret_cast<float*>(sm + TcSmem::RBUF);
+  uint8_t* zf = sm + TcSmem::ZF;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + TcSmem::BAR);
+  uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + TcSmem::TMEM);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  if (warp == 0) {
+    s1::tmem_alloc(tmem_s, 128);
+    s1::tmem_relinquish();
+  }
+  if (tid == 0) {
+    s1::mbar_init(bar, 1);
+    s1::mbar_init_fence();
+  }
+  {  // S operand tile, prepacked on the host
+    const uint4* src = reinterpret_cast<const uint4*>(a.S_sw128);
+    uint4* dst = reinterpret_cast<uint4*>(sm + TcSmem::S);
+    for (int w = tid; w < (int)(kTcTileBytes / 16); w += kTcThreads) dst[w] = src[w];
+  }
+  s1::fence_async_smem();
+  s1::fence_before_sync();
+  __syncthreads();
+  s1::fence_after_sync();
+  const uint32_t tmem = *tmem_s;
+  constexpr uint32_t idesc = s1::idesc_f16_f32(128, 128);
+
+  uint32_t phase = 0;
+  bool failed = false;
+  const int64_t ntile = (a.n_vec + kTcRows - 1) / kTcRows;
+  for (int64_t tile = blockIdx.x; tile < ntile; tile += gridDim.x) {
+    const int64_t v0 = tile * kTcRows;
+    const int nrows = (int)min((int64_t)kTcRows, a.n_vec - v0);
+    if (warp < 4) {
+      if (a.k) {
+        for (int vv = 0; vv < 32; ++vv) {
+          const int row = warp * 32 + vv;
+          if (row >= nrows) break;
+          float r[4];
+          const bool nz = key_front<128, T>(a, v0 + row, lane, rbuf + warp * 128, r);
+          // residual coordinates 4 lane .. 4 lane + 3, scaled by 16 (signs unchanged)
+          float x[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) x[e] = nz ? 16.f * r[e] : 0.f;
+          const __half2 h01 = __floats2half2_rn(x[0], x[1]), h23 = __floats2half2_rn(x[2], x[3]);
+          const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+          const __half2 l01 = __floats2half2_rn(x[0] - f01.x, x[1] - f01.y);
+          const __half2 l23 = __floats2half2_rn(x[2] - f23.x, x[3] - f23.y);
+          const uint32_t off = s1::sw128_offset(row, 4 * lane, kTcRows);
+          uint2 hv, lv;
+          hv.x = *reinterpret_cast<const uint32_t*>(&h01);
+          hv.y = *reinterpret_cast<const uint32_t*>(&h23);
+          lv.x = *reinterpret_cast<const uint32_t*>(&l01);
+          lv.y = *reinterpret_cast<const uint32_t*>(&l23);
+          *reinterpret_cast<uint2*>(sm + TcSmem::A_HI + off) = hv;
+          *reinterpret_cast<uint2*>(sm + TcSmem::A_LO + off) = lv;
+          if (lane == 0) zf[row] = nz ? 1 : 0;
+        }
+        s1::fence_async_smem();
+        s1::fence_before_sync();
+        kwarps_sync_or(false);
+        s1::fence_after_sync();
+        if (tid == 0) {
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            s1::umma_f16(tmem, s1::sw128_desc(sbase + TcSmem::A_HI, 16 * ks, kTcRows),
+                         s1::sw128_desc(sbase + TcSmem::S, 16 * ks, 128), idesc, ks > 0 ? 1u : 0u);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            s1::umma_f16(tmem, s1::sw128_desc(sbase + TcSmem::A_LO, 16 * ks, kTcRows),
+                         s1::sw128_desc(sbase + TcSmem::S, 16 * ks, 128), idesc, 1u);
+          s1::umma_commit(bar);
+        }
+        const bool ok = s1::mbar_wait(bar, phase);
+        phase ^= 1u;
+        if (kwarps_sync_or(!ok)) {
+          failed = true;
+          break;
+        }
+        s1::fence_after_sync();
+        // thread = key (TMEM lane 32 warp + lane); 4 x 32 projections -> 4 sign words
+        uint32_t words[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t v[32];
+          s1::tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + 32 * q, v);
+          s1::tmem_ld_wait();
+          uint32_t bits = 0;
+#pragma unroll
+          for (int k = 0; k < 32; ++k) bits |= (__uint_as_float(v[k]) >= 0.f ? 1u : 0u) << k;
+          words[q] = bits;
+        }
+        const int row = 32 * warp + lane;
+        if (row < nrows) {
+          const bool nz = zf[row] != 0;
+          uint4 w4 = nz ? make_uint4(words[0], words[1], words[2], words[3]) : make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(a.k_signs + (v0 + row) * 16) = w4;
+        }
+        s1::fence_before_sync();
+        kwarps_sync_or(false);  // TMEM and the operand tiles are free for the next tile
+      }
+    } else if (a.v) {
+      for (int vv = 0; vv < 32; ++vv) {
+        const int row = (warp - 4) * 32 + vv;
+        if (row >= nrows) break;
+        compress_value<128, T>(a, v0 + row, lane);
+      }
+    }
+  }
+  if (failed && tid == 0) {
+    atomicOr(a.err, 1u);
+    s1::mbar_wait(bar, phase ^ 1u);  // bounded: let the abandoned MMA finish before TMEM is freed
+  }
+  s1::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    s1::fence_after_sync();
+    s1::tmem_dealloc(tmem, 128);
+  }
+}
+
+template <typename T>
+cudaError_t launch_tc(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) {
+  static bool configured = false;
+  const size_t smem = TcSmem::BYTES + 1024;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(compress_tc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  int64_t blocks = (a.n_vec + kTcRows - 1) / kTcRows;
+  if (blocks > 2LL * ctx->num_sms) blocks = 2LL * ctx->num_sms;
+  if (ctx->prof_start) cudaEventRecord(ctx->prof_start, s);
+  compress_tc_kernel<T><<<(unsigned)blocks, kTcThreads, smem, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (ctx->prof_stop) cudaEventRecord(ctx->prof_stop, s);
+  return e;
+}
+
 }  // namespace
+
+// S as f16 in the swizzled K-major operand layout of compress_tc_kernel, or false if
+// S is not exactly representable in f16 (the tensor-core path then is not used).
+bool pack_qjl_operand(const float* S, int m, int d, uint16_t* out) {
+  if (m != 128 || d != 128) return false;
+  for (int i = 0; i < m; ++i)
+    for (int j = 0; j < d; ++j) {
+      const float v = S[(size_t)i * d + j];
+      const __half h = __float2half_rn(v);
+      if (__half2float(h) != v) return false;
+      out[tq::sm100::sw128_offset(i, j, 128) / 2] = __half_as_ushort(h);
+    }
+  return true;
+}
 
 cudaError_t launch_compress(const tq_ctx* ctx, const void* k, const void* v, int dtype, int64_t n_vec,
                             uint8_t* k_codes, uint8_t* k_signs, uint16_t* k_norms, uint8_t* v_codes,
@@ -210,6 +412,10 @@ cudaError_t launch_compress(const tq_ctx* ctx, const void* k, const void* v, int
   a.v_bits = ctx->shape.v_bits;
   a.rot = ctx->shape.rot;
   a.inv_sqrt_d = (float)(1.0 / sqrt((double)ctx->shape.d));
+  a.S_sw128 = ctx->S_sw128;
+  a.err = ctx->d_err;
+  if (ctx->S_sw128 && ctx->shape.d == 128 && ctx->shape.m == 128)
+    return dtype == TQ_F32 ? launch_tc<float>(ctx, a, stream) : launch_tc<__nv_bfloat16>(ctx, a, stream);
   switch (ctx->shape.d) {
     case 64: return launch_d<64>(ctx, a, dtype, stream);
     case 128: return launch_d<128>(ctx, a, dtype, stream);

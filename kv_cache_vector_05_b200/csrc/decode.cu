@@ -353,18 +353,44 @@ DecodePlan plan_decode(const tq_ctx* ctx, int batch, int hq, int hkv, int64_t ma
   p.mma = mma_decode_supported(ctx, G);
   const int64_t units = (int64_t)batch * hkv;
   const int64_t tiles = max_len > 0 ? (max_len + kTile - 1) / kTile : 1;
-  // CTAs to aim for: a few waves of the resident CTAs per SM
-  const int64_t target = (p.mma ? 6LL : 4LL) * (ctx->num_sms > 0 ? ctx->num_sms : 148);
-  int64_t chunks = units > 0 ? (target + units - 1) / units : 1;
-  if (chunks > tiles) chunks = tiles;
-  if (chunks < 1) chunks = 1;
+  const int64_t sms = ctx->num_sms > 0 ? ctx->num_sms : 148;
+  int64_t chunks = 1;
+  if (p.mma) {
+    // Split each (sequence, KV head) into chunks so that the grid fills whole waves
+    // of resident CTAs (4 per SM): minimise waves x tiles-per-CTA, plus a small
+    // per-wave cost.
+    const int64_t slots = 4 * sms;
+    double best = 1e300;
+    const int64_t max_chunks = tiles < 4096 ? tiles : 4096;
+    for (int64_t n = 1; n <= max_chunks && units > 0; ++n) {
+      const int64_t waves = (units * n + slots - 1) / slots;
+      const double cost = (double)waves * (double)((tiles + n - 1) / n) + 0.5 * (double)waves;
+      if (cost < best) {
+        best = cost;
+        chunks = n;
+      }
+    }
+  } else {
+    const int64_t target = 4 * sms;  // a few waves of resident CTAs
+    chunks = units > 0 ? (target + units - 1) / units : 1;
+    if (chunks > tiles) chunks = tiles;
+    if (chunks < 1) chunks = 1;
+  }
   const int64_t tiles_per_chunk = (tiles + chunks - 1) / chunks;
   p.chunk_len = tiles_per_chunk * kTile;
   p.n_chunks = (int)((tiles + tiles_per_chunk - 1) / tiles_per_chunk);
-  const int q_stride = d + m;
-  p.ws_q_bytes = align256((size_t)batch * hq * q_stride * sizeof(float));
   p.ws_part_bytes = align256((size_t)units * p.n_chunks * G * (d + kPartPad) * sizeof(float));
-  p.total_bytes = p.ws_q_bytes + p.ws_part_bytes;
+  if (p.mma) {
+    p.ws_q_bytes = 0;
+    p.off_frag = 0;
+    p.off_part = align256((size_t)units * mma_frag_bytes(ctx->shape.lm_bits));
+    p.off_cnt = p.off_part + p.ws_part_bytes;
+    p.total_bytes = p.off_cnt + align256((size_t)units * sizeof(unsigned int));
+  } else {
+    const int q_stride = d + m;
+    p.ws_q_bytes = align256((size_t)batch * hq * q_stride * sizeof(float));
+    p.total_bytes = p.ws_q_bytes + p.ws_part_bytes;
+  }
   return p;
 }
 
@@ -374,6 +400,9 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const void*
                           const uint16_t* v_params, float scale, float* scores, float* out, void* workspace,
                           cudaStream_t stream) {
   const int d = ctx->shape.d, m = ctx->shape.m, G = hq / hkv;
+  if (plan.mma)
+    return launch_decode_mma(ctx, plan, q, q_dtype, batch, hq, hkv, seq_lens, max_len, k_codes, k_signs,
+                             k_norms, v_codes, v_params, scale, scores, out, workspace, stream);
   if ((G + (kThreads / d) - 1) / (kThreads / d) > kMaxQ) return cudaErrorInvalidValue;
   float* ws_q = static_cast<float*>(workspace);
   float* ws_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + plan.ws_q_bytes);
@@ -418,16 +447,11 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const void*
   const dim3 grid(plan.n_chunks, batch * hkv);
   const size_t smem = decode_smem_bytes(d, m, G, ctx->shape.v_bits);
   if (ctx->prof_start) cudaEventRecord(ctx->prof_start, stream);
-  if (plan.mma) {
-    e = launch_decode_mma(ctx, plan, ws_q, d + m, ws_part, d + kPartPad, batch, hq, hkv, seq_lens, max_len,
-                          k_codes, k_signs, k_norms, v_codes, v_params, scale, scores, stream);
-  } else {
-    switch (d) {
-      case 64: e = dispatch_lmb<64>(a, ctx->shape.lm_bits, ctx->shape.v_bits, grid, smem, stream); break;
-      case 128: e = dispatch_lmb<128>(a, ctx->shape.lm_bits, ctx->shape.v_bits, grid, smem, stream); break;
-      case 256: e = dispatch_lmb<256>(a, ctx->shape.lm_bits, ctx->shape.v_bits, grid, smem, stream); break;
-      default: return cudaErrorInvalidValue;
-    }
+  switch (d) {
+    case 64: e = dispatch_lmb<64>(a, ctx->shape.lm_bits, ctx->shape.v_bits, grid, smem, stream); break;
+    case 128: e = dispatch_lmb<128>(a, ctx->shape.lm_bits, ctx->shape.v_bits, grid, smem, stream); break;
+    case 256: e = dispatch_lmb<256>(a, ctx->shape.lm_bits, ctx->shape.v_bits, grid, smem, stream); break;
+    default: return cudaErrorInvalidValue;
   }
   if (ctx->prof_stop) cudaEventRecord(ctx->prof_stop, stream);
   if (e != cudaSuccess) return e;

@@ -45,6 +45,8 @@ struct tq_ctx {
   cudaEvent_t prof_start;  // optional events around the main kernel of each call
   cudaEvent_t prof_stop;
   unsigned int* d_err;     // device error word: bit 0 = a bounded wait in a kernel timed out
+  uint16_t* frag_table;    // tensor-core decode: operand sources (d = m = 128, lm_bits <= 2)
+  uint16_t* S_sw128;       // tensor-core compression: S as an f16 operand tile (d = m = 128, S exact in f16)
 };
 
 namespace tq {
@@ -55,11 +57,12 @@ cudaError_t launch_compress(const tq_ctx* ctx, const void* k, const void* v, int
                             uint8_t* v_codes, uint16_t* v_params, cudaStream_t stream);
 
 struct DecodePlan {
-  bool mma;          // tensor-core kernel (decode_mma.cu) instead of the generic one
+  bool mma;          // tensor-core kernels (decode_mma.cu) instead of the generic ones
   int n_chunks;      // split-K chunks per (sequence, KV head)
   int64_t chunk_len; // tokens per chunk (multiple of the tile)
-  size_t ws_q_bytes;     // prepared queries
+  size_t ws_q_bytes;     // generic path: prepared queries
   size_t ws_part_bytes;  // partial (m, l, acc) per chunk and query head
+  size_t off_frag, off_part, off_cnt;  // tensor-core path: byte offsets in the workspace
   size_t total_bytes;
 };
 
@@ -73,11 +76,16 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const void*
 
 bool mma_decode_supported(const tq_ctx* ctx, int G);
 
-cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const float* ws_q, int q_stride,
-                              float* ws_part, int part_stride, int batch, int hq, int hkv,
-                              const int32_t* seq_lens, int64_t max_len, const uint8_t* k_codes,
+size_t mma_frag_bytes(int lm_bits);
+bool pack_qjl_operand(const float* S, int m, int d, uint16_t* out);
+void build_frag_table(int lmb, uint16_t* table);
+size_t frag_table_entries(int lmb);
+
+cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const void* q, int q_dtype, int batch,
+                              int hq, int hkv, const int32_t* seq_lens, int64_t max_len, const uint8_t* k_codes,
                               const uint8_t* k_signs, const uint16_t* k_norms, const uint8_t* v_codes,
-                              const uint16_t* v_params, float scale, float* scores, cudaStream_t stream);
+                              const uint16_t* v_params, float scale, float* scores, float* out, void* workspace,
+                              cudaStream_t stream);
 
 cudaError_t launch_decompress(const tq_ctx* ctx, const uint8_t* k_codes, const uint8_t* k_signs,
                               const uint16_t* k_norms, const uint8_t* v_codes,

@@ -1,0 +1,138 @@
+// Thin wrappers over the sm_100a instructions used by the tensor-memory kernels:
+// mbarriers, tcgen05 (tensor-memory allocation, MMA issue and commit, loads) and
+// the shared-memory operand descriptors. Written from the PTX ISA; the bit layouts
+// of the two descriptors follow the canonical K-major, 128-byte-swizzled form.
+#pragma once
+
+#include <stdint.h>
+
+namespace tq {
+namespace sm100 {
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_init_fence() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait on an mbarrier phase: at most `polls` polls and `ns` nanoseconds.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t polls = 1u << 24,
+                                          unsigned long long ns = 2000000000ull) {
+  const uint32_t a = smem_u32(bar);
+  unsigned long long start = 0;
+  for (uint32_t it = 0; it < polls; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+        : "=r"(done)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if (it == 0) start = global_ns();
+    else if ((it & 255) == 0 && global_ns() - start > ns) return false;
+  }
+  return false;
+}
+
+// ---- tensor memory -----------------------------------------------------------------
+
+// One full warp: allocate `ncols` (power of two >= 32) columns; the TMEM address is
+// written to *smem_dst.
+__device__ __forceinline__ void tmem_alloc(uint32_t* smem_dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem_dst)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void fence_before_sync() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after_sync() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Make generic-proxy writes to shared memory visible to the tensor core.
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem] x B[smem], kind::f16, one CTA. `accumulate` = 0 overwrites D.
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on `bar` once every MMA issued so far by this thread has completed.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+// Warp-wide load of 32 consecutive 32-bit columns of the warp's 32 TMEM lanes.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
+      "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// ---- operand layouts ----------------------------------------------------------------
+
+// K-major operand with 128-byte swizzle: rows of 64 f16 (128 bytes), groups of 8
+// rows form a 1 KB atom whose 16-byte chunks are permuted by chunk ^ (row % 8).
+// A [rows][K] matrix (K a multiple of 64) is stored as K/64 panels of rows x 64,
+// each panel rows/8 atoms long. Byte offset of element (row, k):
+__host__ __device__ constexpr uint32_t sw128_offset(int row, int k, int rows) {
+  return (uint32_t)((k / 64) * (rows * 128) + (row / 8) * 1024 + (row % 8) * 128 +
+                    ((((k % 64) / 8) ^ (row % 8)) * 16) + (k % 8) * 2);
+}
+
+// Shared-memory descriptor of the K-step starting at element column k0 (a multiple
+// of 16) of such a matrix: start address, leading offset 16 B (unused by the
+// swizzled form), stride 1024 B between 8-row atoms, sm_100 version bit, 128B swizzle.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_base, int k0, int rows) {
+  const uint32_t addr = smem_base + (uint32_t)((k0 / 64) * (rows * 128) + (k0 % 64) * 2);
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;              // leading byte offset (16 B units)
+  d |= (uint64_t)(1024u >> 4) << 32;    // stride byte offset (16 B units)
+  d |= (uint64_t)1u << 46;              // descriptor version for sm_100
+  d |= (uint64_t)2u << 61;              // layout: 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor, kind::f16: f16 x f16 -> f32, both operands K-major.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+  return (1u << 4)                       // D format f32
+         | (0u << 7) | (0u << 10)        // A, B format f16
+         | ((uint32_t)(N >> 3) << 17)    // N / 8
+         | ((uint32_t)(M >> 4) << 24);   // M / 16
+}
+
+}  // namespace sm100
+}  // namespace tq
