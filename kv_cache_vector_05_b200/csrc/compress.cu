@@ -39,9 +39,11 @@ struct CompressArgs {
 // Norm, rotation, Lloyd-Max codes and residual of key i; writes the packed codes
 // and (n, gamma). Returns false for a zero key (all its bytes already written as 0);
 // otherwise leaves the lane's residual coordinates in r.
-template <int D, typename T>
+template <int D, typename T, int LMB = 0>
 __device__ bool key_front(const CompressArgs& a, int64_t i, int lane, float* rbuf, float (&r)[D / 32]) {
   constexpr int E = D / 32;
+  const int lmb = LMB ? LMB : a.lm_bits;       // compile-time when specialised
+  const int levels = LMB ? (1 << LMB) : a.cb.levels;
   float x[E];
   load_lane<E>(static_cast<const T*>(a.k) + i * D, lane, x);
 
@@ -50,7 +52,7 @@ __device__ bool key_front(const CompressArgs& a, int64_t i, int lane, float* rbu
   for (int e = 0; e < E; ++e) ss = fmaf(x[e], x[e], ss);
   const float n = sqrtf(warp_sum(ss));
 
-  const int cbytes = a.lm_bits * D / 8;
+  const int cbytes = lmb * D / 8;
   uint32_t* codes_out = reinterpret_cast<uint32_t*>(a.k_codes + i * cbytes);
   uint32_t* signs_out = reinterpret_cast<uint32_t*>(a.k_signs + i * (a.m / 8));
   if (n == 0.f) {  // a zero key is stored as zero bytes
@@ -92,18 +94,19 @@ __device__ bool key_front(const CompressArgs& a, int64_t i, int lane, float* rbu
     uint32_t idx = 0;
     float cv = a.cb.c[0];
 #pragma unroll
-    for (int k = 0; k < kMaxLevels - 1; ++k) {
-      if (k + 1 < a.cb.levels && y[e] >= a.cb.t[k]) {
+    for (int k = 0; k < (LMB ? (1 << LMB) - 1 : kMaxLevels - 1); ++k) {
+      if ((LMB || k + 1 < levels) && y[e] >= a.cb.t[k]) {
         idx = k + 1;
         cv = a.cb.c[k + 1];
       }
     }
-    code_bits |= idx << (e * a.lm_bits);
+    code_bits |= idx << (e * lmb);
     r[e] = y[e] - cv;
     rr = fmaf(r[e], r[e], rr);
   }
   const float gamma = sqrtf(warp_sum(rr));
-  const uint32_t code_word = pack_stream_word(code_bits, E * a.lm_bits, cbytes / 4, lane);
+  const uint32_t code_word = LMB ? pack_stream_word_t<E * LMB, LMB * D / 32>(code_bits, lane)
+                                 : pack_stream_word(code_bits, E * lmb, cbytes / 4, lane);
   if (lane < cbytes / 4) codes_out[lane] = code_word;
   if (lane == 0) {
     const uint32_t nb = __half_as_ushort(__float2half_rn(n));
@@ -134,10 +137,11 @@ __device__ void compress_key(const CompressArgs& a, int64_t i, int lane, float* 
   if (lane < a.m / 32) reinterpret_cast<uint32_t*>(a.k_signs + i * (a.m / 8))[lane] = my_sign_word;
 }
 
-template <int D, typename T>
+template <int D, typename T, int VB = 0>
 __device__ void compress_value(const CompressArgs& a, int64_t i, int lane) {
   constexpr int E = D / 32;
   constexpr int W = 32 / E;  // lanes per group of 32 coordinates
+  const int vbits = VB ? VB : a.v_bits;
   float x[E];
   load_lane<E>(static_cast<const T*>(a.v) + i * D, lane, x);
   float lo = x[0], hi = x[0];
@@ -151,7 +155,7 @@ __device__ void compress_value(const CompressArgs& a, int64_t i, int lane) {
     lo = fminf(lo, __shfl_xor_sync(kFull, lo, o));
     hi = fmaxf(hi, __shfl_xor_sync(kFull, hi, o));
   }
-  const int levels = (1 << a.v_bits) - 1;
+  const int levels = (1 << vbits) - 1;
   // Code arithmetic in fp64 so decisions match the exact quantizer except within
   // a few fp64 ulps of a half-step.
   const double dlo = lo, span = (double)hi - dlo;
@@ -162,10 +166,11 @@ __device__ void compress_value(const CompressArgs& a, int64_t i, int lane) {
   for (int e = 0; e < E; ++e) {
     double q = floor(((double)x[e] - dlo) * inv + 0.5);
     q = fmin(fmax(q, 0.0), (double)levels);
-    code_bits |= (uint32_t)q << (e * a.v_bits);
+    code_bits |= (uint32_t)q << (e * vbits);
   }
-  const int cbytes = a.v_bits * D / 8;
-  const uint32_t word = pack_stream_word(code_bits, E * a.v_bits, cbytes / 4, lane);
+  const int cbytes = vbits * D / 8;
+  const uint32_t word = VB ? pack_stream_word_t<E * VB, VB * D / 32>(code_bits, lane)
+                           : pack_stream_word(code_bits, E * vbits, cbytes / 4, lane);
   if (lane < cbytes / 4) reinterpret_cast<uint32_t*>(a.v_codes + i * cbytes)[lane] = word;
   if ((lane % W) == 0) {
     const uint32_t sb = __half_as_ushort(__double2half(scale));
@@ -232,7 +237,7 @@ __device__ __forceinline__ bool kwarps_sync_or(bool v) {
   return r != 0;
 }
 
-template <typename T>
+template <typename T, int LMB, int VB>
 __global__ void __launch_bounds__(kTcThreads, 2) compress_tc_kernel(const __grid_constant__ CompressArgs a) {
   namespace s1 = tq::sm100;
   extern __shared__ unsigned char smem_raw[];
@@ -276,7 +281,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) compress_tc_kernel(const __grid
           const int row = warp * 32 + vv;
           if (row >= nrows) break;
           float r[4];
-          const bool nz = key_front<128, T>(a, v0 + row, lane, rbuf + warp * 128, r);
+          const bool nz = key_front<128, T, LMB>(a, v0 + row, lane, rbuf + warp * 128, r);
           // residual coordinates 4 lane .. 4 lane + 3, scaled by 16 (signs unchanged)
           float x[4];
 #pragma unroll
@@ -342,7 +347,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) compress_tc_kernel(const __grid
       for (int vv = 0; vv < 32; ++vv) {
         const int row = (warp - 4) * 32 + vv;
         if (row >= nrows) break;
-        compress_value<128, T>(a, v0 + row, lane);
+        compress_value<128, T, VB>(a, v0 + row, lane);
       }
     }
   }
@@ -358,22 +363,31 @@ __global__ void __launch_bounds__(kTcThreads, 2) compress_tc_kernel(const __grid
   }
 }
 
-template <typename T>
-cudaError_t launch_tc(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) {
+template <typename T, int LMB, int VB>
+cudaError_t launch_tc_t(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) {
   static bool configured = false;
   const size_t smem = TcSmem::BYTES + 1024;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(compress_tc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(compress_tc_kernel<T, LMB, VB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   int64_t blocks = (a.n_vec + kTcRows - 1) / kTcRows;
   if (blocks > 2LL * ctx->num_sms) blocks = 2LL * ctx->num_sms;
   if (ctx->prof_start) cudaEventRecord(ctx->prof_start, s);
-  compress_tc_kernel<T><<<(unsigned)blocks, kTcThreads, smem, s>>>(a);
+  compress_tc_kernel<T, LMB, VB><<<(unsigned)blocks, kTcThreads, smem, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (ctx->prof_stop) cudaEventRecord(ctx->prof_stop, s);
   return e;
+}
+
+template <typename T>
+cudaError_t launch_tc(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) {
+  const int lmb = ctx->shape.lm_bits, vb = ctx->shape.v_bits;
+  if (lmb == 1) return vb == 2 ? launch_tc_t<T, 1, 2>(ctx, a, s) : launch_tc_t<T, 1, 4>(ctx, a, s);
+  if (lmb == 2) return vb == 2 ? launch_tc_t<T, 2, 2>(ctx, a, s) : launch_tc_t<T, 2, 4>(ctx, a, s);
+  return vb == 2 ? launch_tc_t<T, 3, 2>(ctx, a, s) : launch_tc_t<T, 3, 4>(ctx, a, s);
 }
 
 }  // namespace

@@ -107,6 +107,24 @@ __device__ __forceinline__ uint32_t pack_stream_word(uint32_t v, int nbits, int 
   return mine;
 }
 
+// Same with the bit count per lane and the word count known at compile time.
+template <int NBITS, int NWORDS>
+__device__ __forceinline__ uint32_t pack_stream_word_t(uint32_t v, int lane) {
+  static_assert(NBITS <= 32 && NWORDS <= 32, "stream geometry");
+  const int o = lane * NBITS;
+  const uint64_t wide = (uint64_t)v << (o & 31);
+  const uint32_t lo = (uint32_t)wide, hi = (uint32_t)(wide >> 32);
+  const int w0 = o >> 5;
+  uint32_t mine = 0;
+#pragma unroll
+  for (int w = 0; w < NWORDS; ++w) {
+    const uint32_t c = (w == w0 ? lo : 0u) | ((32 % NBITS != 0 && w == w0 + 1) ? hi : 0u);
+    const uint32_t word = __reduce_or_sync(kFull, c);
+    if (lane == w) mine = word;
+  }
+  return mine;
+}
+
 // Code j (bits [b*j, b*j+b)) from a little-endian stream held in registers.
 template <int B, int NW>
 __device__ __forceinline__ uint32_t stream_code(const uint32_t (&w)[NW], int j) {
