@@ -352,7 +352,8 @@ DecodePlan plan_decode(const tq_ctx* ctx, int batch, int hq, int hkv, int64_t ma
   const int d = ctx->shape.d, m = ctx->shape.m, G = hq / hkv;
   p.mma = mma_decode_supported(ctx, G);
   const int64_t units = (int64_t)batch * hkv;
-  const int64_t tiles = max_len > 0 ? (max_len + kTile - 1) / kTile : 1;
+  const int64_t tile = p.mma ? mma_tile_tokens(G) : kTile;
+  const int64_t tiles = max_len > 0 ? (max_len + tile - 1) / tile : 1;
   const int64_t sms = ctx->num_sms > 0 ? ctx->num_sms : 148;
   int64_t chunks = 1;
   if (p.mma) {
@@ -377,13 +378,13 @@ DecodePlan plan_decode(const tq_ctx* ctx, int batch, int hq, int hkv, int64_t ma
     if (chunks < 1) chunks = 1;
   }
   const int64_t tiles_per_chunk = (tiles + chunks - 1) / chunks;
-  p.chunk_len = tiles_per_chunk * kTile;
+  p.chunk_len = tiles_per_chunk * tile;
   p.n_chunks = (int)((tiles + tiles_per_chunk - 1) / tiles_per_chunk);
   p.ws_part_bytes = align256((size_t)units * p.n_chunks * G * (d + kPartPad) * sizeof(float));
   if (p.mma) {
     p.ws_q_bytes = 0;
     p.off_frag = 0;
-    p.off_part = align256((size_t)units * mma_frag_bytes(ctx->shape.lm_bits));
+    p.off_part = align256((size_t)units * mma_frag_bytes(ctx->shape.lm_bits, G));
     p.off_cnt = p.off_part + p.ws_part_bytes;
     p.total_bytes = p.off_cnt + align256((size_t)units * sizeof(unsigned int));
   } else {

@@ -6,9 +6,14 @@
 // fused decode kernels): logit = scale * n * (<qr, c[idx]> + sqrt(pi/2)/m * gamma *
 // <sq, s>), online softmax, sum of p * (min + scale * code). What changes is how
 // the per-token work is spread: with G query heads sharing a KV head, the three
-// contractions (codes x qr, signs x sq, probabilities x value codes) are small
-// dense products over a tile of tokens, so they run on the tensor cores
+// contractions (key bits x query, signs x S q, value codes x probabilities) are
+// small dense products over a tile of tokens, so they run on the tensor cores
 // (mma.sync m16n8k16, f16 operands, fp32 accumulation) instead of G scalar loops.
+//
+// Operand layout: the 16 rows of every MMA are tokens (scores) or value
+// coordinates (values); the 8 columns of an n-block are 4 query heads x (hi, lo),
+// the two f16 halves of a query or probability operand (about 22 bits together).
+// G <= 4 needs one n-block, G <= 8 two.
 //
 // Operand construction (no unpacking loops):
 //  * A 2-bit code with a symmetric codebook is affine in its two bits:
@@ -16,25 +21,26 @@
 //    c0 sum(qr) + sum over stream bits of (beta_plane * qr_j) * bit. Every packed
 //    bit, keys and signs alike, becomes one MMA operand element.
 //  * Masking one bit per 16-bit half of a word yields an f16 that is 0 or a power
-//    of two (2^-15 .. 2 for bit positions 9..14); the query side is pre-divided by
-//    that power, so one LOP3 turns two bits into two exact operand elements.
+//    of two (2^-15 .. 2^-11 for bit positions 9..12); the query side is pre-divided
+//    by that power. Lane (r, c) rotates each key word so that its bits 4c..4c+3
+//    (and 16 higher) sit at positions 9..12, then one AND per operand register
+//    yields two exact elements.
 //  * A value code placed in the low mantissa bits of an f16 is a subnormal equal
 //    to code * 2^(pos - 24), so a byte permute plus a mask yields two exact
 //    operands; the power of two is undone once at the end.
-//  * Query and probability operands are split hi + lo in f16 (about 22 bits), the
-//    two halves occupying rows h and h + 8 of the 16-row tile.
 //
 // Kernels:
 //  * prep_mma_kernel, one CTA per (sequence, KV head): rotates the G queries
 //    (sign flip + Walsh-Hadamard butterflies, or the dense Haar matrix), forms
-//    S qr, and writes the query operand fragments of that KV head once.
+//    S qr, and writes that KV head's query operand fragments once.
 //  * decode_mma_kernel, one CTA per (sequence x KV head, chunk of the cache),
 //    launched with programmatic dependent launch: it starts streaming its cache
-//    tiles (cp.async.bulk into a 4-deep ring, mbarrier completion) while the prep
-//    kernel finishes, then waits for the fragments. Each warp owns 16 tokens of
-//    each 64-token tile. The last CTA of a (sequence, KV head) to finish - decided
-//    by an atomic ticket, nobody waits - merges the chunk partials (log-sum-exp)
-//    and writes the output rows.
+//    tiles (cp.async.bulk into a ring of stages, mbarrier completion) while the
+//    prep kernel finishes, then waits for the fragments. Each warp owns 16 or 32
+//    consecutive tokens of each tile: it scores them, runs the online softmax for
+//    its heads and accumulates their values. The last CTA of a (sequence, KV head)
+//    to finish - decided by an atomic ticket, nobody waits - merges the chunk
+//    partials (log-sum-exp) and writes the output rows.
 // Every wait is bounded; a timeout sets the context's error word and ends the CTA.
 #include <cuda_runtime.h>
 #include <math.h>
@@ -48,8 +54,6 @@ constexpr int kD = 128;
 constexpr int kM = 128;
 constexpr int kWarpsMma = 4;
 constexpr int kThreadsMma = kWarpsMma * 32;
-constexpr int kTileMma = 64;  // tokens per stage: 16 per warp
-constexpr int kStages = 4;
 constexpr int kPartPadMma = 4;
 constexpr int kPrepThreads = 256;
 // Base-2 slack of the lazy online-softmax rescale: probabilities stay below 2^kSlack,
@@ -58,10 +62,18 @@ constexpr float kSlack = 2.f;
 constexpr uint32_t kWaitLimit = 1u << 24;                 // polls of one mbarrier phase
 constexpr unsigned long long kWaitNs = 2000000000ull;    // and at most 2 s of wall time
 
-__host__ __device__ constexpr int frag_chunks(int lmb) { return 8 * (lmb + 1); }
-// Per (sequence, KV head): A fragments [chunks][32 lanes] uint4, then [8 heads][4] floats
-// (sum of qr, sum of sq, LM scale, sign scale).
-__host__ __device__ constexpr int frag_words(int lmb) { return frag_chunks(lmb) * 32 * 4 + 32; }
+// 32-bit words of key bits per token (code stream, then signs) and the MMA k-steps
+// over them (each word feeds two k-steps of 16 bits).
+__host__ __device__ constexpr int key_words(int lmb) { return 4 * lmb + kM / 32; }
+__host__ __device__ constexpr int key_steps(int lmb) { return 2 * key_words(lmb); }
+// n-blocks of 8 operand columns (4 heads x hi/lo) for G query heads.
+__host__ __device__ constexpr int n_blocks(int G) { return G <= 4 ? 1 : 2; }
+// 16-token row blocks per warp and tile (fewer when two n-blocks need the registers).
+__host__ __device__ constexpr int m_blocks(int nb) { return nb == 1 ? 2 : 1; }
+__host__ __device__ constexpr int tile_tokens(int nb) { return 16 * kWarpsMma * m_blocks(nb); }
+// Per (sequence, KV head): query operand words [k-step][n-block][32 lanes][2], then
+// [8 heads][4] floats (sum of qr, sum of sq, LM scale, sign scale).
+__host__ __device__ constexpr int frag_words(int lmb, int nb) { return key_steps(lmb) * nb * 64 + 32; }
 
 struct PrepArgs {
   const void* q;
@@ -72,9 +84,9 @@ struct PrepArgs {
   const float* PiT;  // [d][d] (Haar)
   Codebook cb;
   float beta0, beta1;
+  int nb;            // n-blocks of the query operand
   uint32_t* frag;    // [units][frag_words]
   unsigned int* cnt; // [units] completion tickets, zeroed here
-  const uint16_t* table;  // [frag_chunks * 32 * 4 * 2] operand sources (frag_source)
 };
 
 struct MmaArgs {
@@ -171,19 +183,6 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-
-// Register rho (0..15) of a key word: which shifted copy of the word it masks,
-// which bit position p of each 16-bit half it keeps, and which original bit o.
-//   rho 0..5   : word       , p = 9 + rho   , o = 9 + rho
-//   rho 6..11  : word << 6  , p = 3 + rho   , o = rho - 3
-//   rho 12..14 : word << 12 , p = rho       , o = rho - 12
-//   rho 15     : word >> 6  , p = 9         , o = 15
-__host__ __device__ constexpr int key_variant(int rho) { return rho < 6 ? 0 : rho < 12 ? 1 : rho < 15 ? 2 : 3; }
-__host__ __device__ constexpr int key_pos(int rho) { return rho < 6 ? 9 + rho : rho < 12 ? 3 + rho : rho < 15 ? rho : 9; }
-__host__ __device__ constexpr int key_orig(int rho) { return rho < 6 ? 9 + rho : rho < 12 ? rho - 3 : rho < 15 ? rho - 12 : 15; }
-
-// log2 of the f16 value of a lone bit at position p (0..14) of a half.
-__host__ __device__ constexpr int lone_bit_log2(int p) { return p <= 9 ? p - 24 : (1 << (p - 10)) - 15; }
 
 // ------------------------------------------------------------------ prep kernel
 
@@ -320,77 +319,89 @@ __global__ void __launch_bounds__(kPrepThreads) prep_mma_kernel(const __grid_con
     }
   }
   __syncthreads();
-  uint32_t* frag = a.frag + (size_t)unit * frag_words(LMB);
-  // A fragment word (chunk k, lane l, register q = a0..a3) holds two f16 (row, slot)
-  // values: a0/a2 rows r (hi part), a1/a3 rows r + 8 (lo part). Where each value
-  // comes from is fixed by the layout and precomputed (see frag_source).
-  const uint32_t* tab = reinterpret_cast<const uint32_t*>(a.table);
-  constexpr int kPerT = frag_chunks(LMB) * 32 * 4 / kPrepThreads;  // 6 or 12 words per thread
-  uint32_t ents[kPerT];
-#pragma unroll
-  for (int u = 0; u < kPerT; ++u) ents[u] = __ldg(tab + tid + u * kPrepThreads);
-#pragma unroll
-  for (int u = 0; u < kPerT; ++u) {
-    const int idx = tid + u * kPrepThreads;
-    const int q = idx & 3, l = (idx >> 2) & 31;
-    const int row_head = l >> 2;
-    const bool lo_part = (q & 1) != 0;
-    const uint32_t ent2 = ents[u];
+  const int nb = a.nb;
+  uint32_t* frag = a.frag + (size_t)unit * frag_words(LMB, nb);
+  // Word (k-step, n-block, lane (r, c), register) holds the two f16 B elements of
+  // the m16n8k16 fragment: column r = head 4 n-block + r / 2, part r % 2 (hi / lo);
+  // rows 2c, 2c + 1 (register 0) or 2c + 8, 2c + 9 (register 1). Register e' of
+  // k-step 2 w + h stands for bit 4c + e (e = 2h + e') of key word w and, in its
+  // upper half, bit 4c + e + 16; after the decode lane's rotation that bit is the
+  // lone f16 bit at position 9 + e, worth 2^-15, 2^-14, 2^-13 or 2^-11.
+  const int nwords = key_steps(LMB) * nb * 64;
+  for (int w = tid; w < nwords; w += kPrepThreads) {
+    const int reg = w & 1, ln = (w >> 1) & 31, blk = w >> 6;
+    const int nbi = blk % nb, kstep = blk / nb;
+    const int rr = ln >> 2, cc = ln & 3;
+    const int head = 4 * nbi + (rr >> 1);
+    const bool lo_part = (rr & 1) != 0;
+    const int wi = kstep >> 1, e = 2 * (kstep & 1) + reg;
+    const float inv = e == 0 ? 32768.f : e == 1 ? 16384.f : e == 2 ? 8192.f : 2048.f;
     float v2[2] = {0.f, 0.f};
-    if (row_head < G) {
+    if (head < G) {
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const uint32_t ent = (ent2 >> (16 * e)) & 0xffffu;
-        const int src = ent & 0xff, plane = (ent >> 8) & 1, ex = (int)((ent >> 9) & 31) - 16;
-        const float pw2 = __int_as_float((ex + 127) << 23);
+      for (int half = 0; half < 2; ++half) {
+        const int o = 4 * cc + e + 16 * half;  // bit of the 32-bit key word
         float x;
-        if (src < kD)
-          x = qr_s[row_head * kD + src] * ((plane ? a.beta1 : a.beta0) * inv_s[row_head * 2 + 0] * pw2);
-        else
-          x = sq_s[row_head * kM + (src - kD)] * (inv_s[row_head * 2 + 1] * pw2);
+        if (wi < 4 * LMB) {
+          const int sbit = 32 * wi + o;  // bit of the code stream: code sbit / LMB, plane sbit % LMB
+          const int j = sbit / LMB, plane = sbit % LMB;
+          x = qr_s[head * kD + j] * ((plane ? a.beta1 : a.beta0) * inv_s[head * 2 + 0]);
+        } else {
+          x = sq_s[head * kM + 32 * (wi - 4 * LMB) + o] * inv_s[head * 2 + 1];
+        }
+        x *= inv;
         const float hi = __half2float(__float2half_rn(x));
-        v2[e] = lo_part ? (x - hi) : hi;
+        v2[half] = lo_part ? (x - hi) : hi;
       }
     }
-    frag[idx] = pack_h2(v2[0], v2[1]);
+    frag[w] = pack_h2(v2[0], v2[1]);
   }
-  if (tid < 32) reinterpret_cast<float*>(frag)[frag_chunks(LMB) * 32 * 4 + tid] = head_s[tid];
+  if (tid < 32) reinterpret_cast<float*>(frag)[nwords + tid] = head_s[tid];
   if (tid == 0) a.cnt[unit] = 0u;
 }
 
 // ------------------------------------------------------------------ decode kernel
 
-template <int LMB, int VB>
+template <int LMB, int VB, int NB>
 struct Layout {
+  static constexpr int MB = m_blocks(NB);
+  static constexpr int TILE = tile_tokens(NB);
+  static constexpr int STAGES = MB == 2 ? 3 : 4;
   static constexpr int KCB = LMB * kD / 8;  // key code bytes per token
   static constexpr int SB = kM / 8;         // sign bytes
   static constexpr int VCB = VB * kD / 8;   // value code bytes
   static constexpr int PB = (kD / kVGroup) * 4;
   static constexpr int REC = KCB + SB + 4 + VCB + PB;
-  static constexpr int STAGE = kTileMma * REC;
+  static constexpr int STAGE = TILE * REC;
   static constexpr int OFF_KC = 0;
-  static constexpr int OFF_KS = OFF_KC + kTileMma * KCB;
-  static constexpr int OFF_KN = OFF_KS + kTileMma * SB;
-  static constexpr int OFF_VC = OFF_KN + kTileMma * 4;
-  static constexpr int OFF_VP = OFF_VC + kTileMma * VCB;
-  static constexpr int KCHUNKS = frag_chunks(LMB);
-  static constexpr int FRAG_BYTES = frag_words(LMB) * 4;
+  static constexpr int OFF_KS = OFF_KC + TILE * KCB;
+  static constexpr int OFF_KN = OFF_KS + TILE * SB;
+  static constexpr int OFF_VC = OFF_KN + TILE * 4;
+  static constexpr int OFF_VP = OFF_VC + TILE * VCB;
+  static constexpr int KS = key_steps(LMB);
+  static constexpr int FRAG_BYTES = frag_words(LMB, NB) * 4;
   static constexpr int RED_BYTES = kWarpsMma * 8 * (kPartPadMma + kD) * 4;  // per-warp partials
-  static constexpr int RING = kStages * STAGE > RED_BYTES ? kStages * STAGE : RED_BYTES;
-  static constexpr size_t SMEM = (size_t)RING + FRAG_BYTES + 8 * kStages + 4 * (1 + 2 * kStages) + 16;
+  static constexpr int RING = STAGES * STAGE > RED_BYTES ? STAGES * STAGE : RED_BYTES;
+  static constexpr size_t SMEM = (size_t)RING + FRAG_BYTES + 8 * STAGES + 4 * (1 + 2 * STAGES) + 16;
+  static_assert(STAGE % 16 == 0 && FRAG_BYTES % 16 == 0, "16-byte aligned stages and fragments");
 };
 
-template <int LMB, int VB>
+__device__ __forceinline__ uint32_t word_of(const uint4& w, int i) {
+  return i == 0 ? w.x : i == 1 ? w.y : i == 2 ? w.z : w.w;
+}
+
+template <int LMB, int VB, int NB>
 __global__ void __launch_bounds__(kThreadsMma, 4) decode_mma_kernel(const __grid_constant__ MmaArgs a) {
-  using L = Layout<LMB, VB>;
+  using L = Layout<LMB, VB, NB>;
+  constexpr int MB = L::MB, TILE = L::TILE, NST = L::STAGES;
   extern __shared__ __align__(128) unsigned char smem[];
-  unsigned char* stage_base = smem;                                     // ring, later per-warp partials
-  uint4* afrag = reinterpret_cast<uint4*>(smem + L::RING);             // [KCHUNKS][32], then head consts
-  const float* head_s = reinterpret_cast<const float*>(afrag + L::KCHUNKS * 32);
+  unsigned char* stage_base = smem;                                       // ring, later per-warp partials
+  const uint2* bq = reinterpret_cast<const uint2*>(smem + L::RING);      // [KS][NB][32 lanes]
+  const float* head_s = reinterpret_cast<const float*>(bq + L::KS * NB * 32);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::RING + L::FRAG_BYTES);
-  int* last_s = reinterpret_cast<int*>(bars + kStages);
-  int* arrive_s = last_s + 1;        // [kStages] warps done with the stage's current tile
-  int* issued_s = arrive_s + kStages; // [kStages] bulk-copy batches issued into the stage
+  int* last_s = reinterpret_cast<int*>(bars + NST);
+  int* arrive_s = last_s + 1;         // [NST] warps done with the stage's current tile
+  int* issued_s = arrive_s + NST;     // [NST] bulk-copy batches issued into the stage
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int r = lane >> 2, c = lane & 3;
@@ -404,10 +415,10 @@ __global__ void __launch_bounds__(kThreadsMma, 4) decode_mma_kernel(const __grid
   const int qrow0 = b * a.hq + kvh * G;
   const int64_t vec0 = (int64_t)unit * a.max_len;
   const int span = t1 > t0 ? (int)(t1 - t0) : 0;  // tokens of this chunk (< 2^31)
-  const int ntiles = (span + kTileMma - 1) / kTileMma;
+  const int ntiles = (span + TILE - 1) / TILE;
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(&bars[s], 1);
       arrive_s[s] = 0;
       issued_s[s] = 0;
@@ -416,22 +427,22 @@ __global__ void __launch_bounds__(kThreadsMma, 4) decode_mma_kernel(const __grid
   }
   __syncthreads();
 
-  auto tile_full = [&](int i) -> bool { return (i + 1) * kTileMma <= span; };
+  auto tile_full = [&](int i) -> bool { return (i + 1) * TILE <= span; };
   auto issue = [&](int i) {  // one thread: bulk-copy tile i into its stage
-    unsigned char* st = stage_base + (i % kStages) * L::STAGE;
-    const int64_t v = vec0 + t0 + (int64_t)i * kTileMma;
-    uint64_t* bar = &bars[i % kStages];
-    issued_s[i % kStages] += 1;
+    unsigned char* st = stage_base + (i % NST) * L::STAGE;
+    const int64_t v = vec0 + t0 + (int64_t)i * TILE;
+    uint64_t* bar = &bars[i % NST];
+    issued_s[i % NST] += 1;
     mbar_expect_tx(bar, (uint32_t)L::STAGE);
-    bulk_g2s(st + L::OFF_KC, a.k_codes + v * L::KCB, kTileMma * L::KCB, bar);
-    bulk_g2s(st + L::OFF_KS, a.k_signs + v * L::SB, kTileMma * L::SB, bar);
-    bulk_g2s(st + L::OFF_KN, reinterpret_cast<const uint8_t*>(a.k_norms) + v * 4, kTileMma * 4, bar);
-    bulk_g2s(st + L::OFF_VC, a.v_codes + v * L::VCB, kTileMma * L::VCB, bar);
-    bulk_g2s(st + L::OFF_VP, reinterpret_cast<const uint8_t*>(a.v_params) + v * L::PB, kTileMma * L::PB, bar);
+    bulk_g2s(st + L::OFF_KC, a.k_codes + v * L::KCB, TILE * L::KCB, bar);
+    bulk_g2s(st + L::OFF_KS, a.k_signs + v * L::SB, TILE * L::SB, bar);
+    bulk_g2s(st + L::OFF_KN, reinterpret_cast<const uint8_t*>(a.k_norms) + v * 4, TILE * 4, bar);
+    bulk_g2s(st + L::OFF_VC, a.v_codes + v * L::VCB, TILE * L::VCB, bar);
+    bulk_g2s(st + L::OFF_VP, reinterpret_cast<const uint8_t*>(a.v_params) + v * L::PB, TILE * L::PB, bar);
   };
   // The packed cache does not depend on the prep kernel: start streaming it now.
   if (tid == 0 && a.use_tma) {
-    for (int i = 0; i < kStages && i < ntiles; ++i)
+    for (int i = 0; i < NST && i < ntiles; ++i)
       if (tile_full(i)) issue(i);
   }
 
@@ -439,42 +450,65 @@ __global__ void __launch_bounds__(kThreadsMma, 4) decode_mma_kernel(const __grid
   // head's query fragments and constants.
   asm volatile("griddepcontrol.wait;" ::: "memory");
   {
-    const uint4* src = reinterpret_cast<const uint4*>(a.frag + (size_t)unit * frag_words(LMB));
-    for (int w = tid; w < L::FRAG_BYTES / 16; w += kThreadsMma) afrag[w] = src[w];
+    const uint4* src = reinterpret_cast<const uint4*>(a.frag + (size_t)unit * frag_words(LMB, NB));
+    uint4* dst = reinterpret_cast<uint4*>(smem + L::RING);
+    for (int w = tid; w < L::FRAG_BYTES / 16; w += kThreadsMma) dst[w] = src[w];
   }
   __syncthreads();
 
-  const bool head_ok = r < G;
   constexpr float kLog2e = 1.4426950408889634f;
   constexpr float kLn2 = 0.6931471805599453f;
-  // logit (base-2 units) = n * (k1 + k2 * lm + gamma * (k3 * sg - k4)), with lm, sg the raw
-  // tensor-core dot products and every per-head constant folded in once.
+  // Lane (r, c) scores heads c + 4 nb. logit (base-2 units) = n * (k1 + k2 * lm +
+  // gamma * (k3 * sg - k4)), with lm, sg the raw tensor-core dot products.
   const float sl2 = a.scale * kLog2e;
-  const float k1 = sl2 * a.c0 * head_s[r * 4 + 0];
-  const float k2 = sl2 * head_s[r * 4 + 2];
-  const float k3 = sl2 * (kQjl / (float)kM) * 2.f * head_s[r * 4 + 3];
-  const float k4 = sl2 * (kQjl / (float)kM) * head_s[r * 4 + 1];
-
-  float m_run = -INFINITY, l_run = 0.f;
-  float dmin[4] = {0.f, 0.f, 0.f, 0.f};  // sum_t p * min(t, g): rows (head, hi/lo), cols = groups
-  float dv[16][4];
+  float k1[NB], k2[NB], k3[NB], k4[NB];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) dv[i][0] = dv[i][1] = dv[i][2] = dv[i][3] = 0.f;
+  for (int nb = 0; nb < NB; ++nb) {
+    const float* hc = head_s + 4 * (c + 4 * nb);
+    k1[nb] = sl2 * a.c0 * hc[0];
+    k2[nb] = sl2 * hc[2];
+    k3[nb] = sl2 * (kQjl / (float)kM) * 2.f * hc[3];
+    k4[nb] = sl2 * (kQjl / (float)kM) * hc[1];
+  }
+
+  float m_run[NB], l_run[NB];
+  float dmin[NB][4];       // rows g < 4: sum_t p * min(t, g); columns: heads x (hi, lo)
+  float dv[4][2][NB][4];   // [group][half of the group][n-block]: rows = coordinates
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb) {
+    m_run[nb] = -INFINITY;
+    l_run[nb] = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dmin[nb][e] = 0.f;
+#pragma unroll
+    for (int g = 0; g < 4; ++g)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dv[g][hf][nb][e] = 0.f;
+  }
+
+  const uint32_t rot = (uint32_t)(9 - 4 * c) & 31u;  // bits 4c..4c+3 (+16) -> 9..12 (+16)
+  // Value-side B column of this lane: head 4 nb + hsel, part (hi / lo). Its tokens,
+  // in K order, are (c, c + 8) and (c + 4, c + 12) of a 16-token block, whose
+  // probabilities the lanes srcA and srcB hold after the score step.
+  const int part = r & 1, hsel = r >> 1;
+  const int srcA = 4 * c + hsel, srcB = 4 * (c + 4) + hsel;
 
   bool failed = false;
   for (int i = 0; i < ntiles; ++i) {
-    unsigned char* st = stage_base + (i % kStages) * L::STAGE;
-    const int nt = min(kTileMma, span - i * kTileMma);
+    unsigned char* st = stage_base + (i % NST) * L::STAGE;
+    const int nt = min(TILE, span - i * TILE);
     if (a.use_tma && tile_full(i)) {
       // Warps run ahead of one another; each waits only for the tile it needs. After
       // a timeout a warp keeps the loop's structure (arrivals, barriers) but does no
       // more work, so every warp of the CTA reaches the same barriers.
-      if (!failed && !mbar_wait(&bars[i % kStages], (uint32_t)((i / kStages) & 1))) failed = true;
+      if (!failed && !mbar_wait(&bars[i % NST], (uint32_t)((i / NST) & 1))) failed = true;
     } else {
       // Ragged or unaligned tile: plain 4-byte copies (all record sizes are multiples
       // of 4), after every warp has left the tile that used this stage before.
       __syncthreads();
-      const int64_t v = vec0 + t0 + (int64_t)i * kTileMma;
+      const int64_t v = vec0 + t0 + (int64_t)i * TILE;
       auto copy = [&](int off, const void* src, int bytes_per_tok) {
         const uint32_t* s32 =
             reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(src) + v * bytes_per_tok);
@@ -489,204 +523,223 @@ __global__ void __launch_bounds__(kThreadsMma, 4) decode_mma_kernel(const __grid
       __syncthreads();
     }
 
-    const int tb = 16 * warp;  // this warp's 16 tokens within the tile
-    if (tb < nt && !failed) {
-      const uint32_t* kc = reinterpret_cast<const uint32_t*>(st + L::OFF_KC);
-      const uint32_t* ks = reinterpret_cast<const uint32_t*>(st + L::OFF_KS);
+    const int wbase = 16 * MB * warp;  // this warp's first token within the tile
+    if (wbase < nt && !failed) {
+      const uint4* kc4 = reinterpret_cast<const uint4*>(st + L::OFF_KC);
+      const uint4* ks4 = reinterpret_cast<const uint4*>(st + L::OFF_KS);
       const uint32_t* kn = reinterpret_cast<const uint32_t*>(st + L::OFF_KN);
       const uint32_t* vc = reinterpret_cast<const uint32_t*>(st + L::OFF_VC);
       const uint4* vp = reinterpret_cast<const uint4*>(st + L::OFF_VP);
+      const uint32_t* vpw = reinterpret_cast<const uint32_t*>(st + L::OFF_VP);
 
-      // ---- logits: D[head hi/lo rows][token columns] ---------------------------
-      float dl[2][4], ds[2][4];
+      // ---- scores: D[token rows][head columns] over all key bits ------------------
+      // Rows r and r + 8 of block mb are tokens wbase + 16 mb + r (+ 8).
+      float dl[MB][NB][4], ds[MB][NB][4];
 #pragma unroll
-      for (int nb = 0; nb < 2; ++nb)
+      for (int mb = 0; mb < MB; ++mb)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) dl[nb][e] = ds[nb][e] = 0.f;
-      uint32_t kw[2][LMB + 1];
+        for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-      for (int nb = 0; nb < 2; ++nb) {
-        const int tok = tb + 8 * nb + (r >> 1) + 4 * (r & 1);  // token of B column r
+          for (int e = 0; e < 4; ++e) dl[mb][nb][e] = ds[mb][nb][e] = 0.f;
 #pragma unroll
-        for (int wi = 0; wi < LMB; ++wi) kw[nb][wi] = kc[tok * (L::KCB / 4) + c + 4 * wi];
-        kw[nb][LMB] = ks[tok * (L::SB / 4) + c];
-      }
+      for (int q = 0; q <= LMB; ++q) {  // 16-byte chunk q: code words 4q..4q+3, or the signs
+        uint4 kw[2 * MB];
 #pragma unroll
-      for (int wi = 0; wi <= LMB; ++wi) {
-        uint32_t var[2][4];
-#pragma unroll
-        for (int nb = 0; nb < 2; ++nb) {
-          const uint32_t w = kw[nb][wi];
-          var[nb][0] = w;
-          var[nb][1] = w << 6;
-          var[nb][2] = w << 12;
-          var[nb][3] = w >> 6;
+        for (int t = 0; t < 2 * MB; ++t) {
+          const int tok = wbase + 8 * t + r;
+          kw[t] = q < LMB ? kc4[tok * LMB + q] : ks4[tok];
         }
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint4 af = afrag[(8 * wi + kk) * 32 + lane];
-          const int r0 = 2 * kk, r1 = 2 * kk + 1;
-          const uint32_t m0 = (1u << key_pos(r0)) | (1u << (key_pos(r0) + 16));
-          const uint32_t m1 = (1u << key_pos(r1)) | (1u << (key_pos(r1) + 16));
+        for (int u = 0; u < 4; ++u) {
+          uint32_t v[2 * MB];
 #pragma unroll
-          for (int nb = 0; nb < 2; ++nb) {
-            const uint32_t b0 = var[nb][key_variant(r0)] & m0;
-            const uint32_t b1 = var[nb][key_variant(r1)] & m1;
-            if (wi < LMB)
-              mma16816(dl[nb], af, b0, b1);
-            else
-              mma16816(ds[nb], af, b0, b1);
+          for (int t = 0; t < 2 * MB; ++t) {
+            const uint32_t w = word_of(kw[t], u);
+            v[t] = __funnelshift_l(w, w, rot);
           }
-        }
-      }
-
-      // ---- logits epilogue and online softmax (thread: head r, 4 tokens) ---------
-      // token order of the thread's four values: c, c + 4, c + 8, c + 12. Rows of
-      // absent heads (r >= G) carry zero query operands, so their values stay finite
-      // and are simply never written out.
-      float lg[4];
-      bool tv[4] = {true, true, true, true};
-      const bool ragged = nt - tb < 16;  // warp-uniform
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int nb = e >> 1, col = e & 1;
-        const float2 ng = unpack_h2(kn[tb + c + 4 * e]);  // (n, gamma)
-        const float lm = dl[nb][col] + dl[nb][col + 2];
-        const float sg = ds[nb][col] + ds[nb][col + 2];
-        lg[e] = ng.x * fmaf(ng.y, fmaf(k3, sg, -k4), fmaf(k2, lm, k1));
-      }
-      if (ragged) {
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int kstep = 2 * (4 * q + u) + h2;
+            const uint32_t mlo = 0x02000200u << (2 * h2);      // bit 9 + 2 h2 of each half
+            const uint32_t mhi = 0x02000200u << (2 * h2 + 1);  // bit 10 + 2 h2
+            uint2 bf[NB];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          tv[e] = c + 4 * e < nt - tb;
-          if (!tv[e]) lg[e] = -INFINITY;  // stale bytes past the end of the cache
-        }
-      }
-      if (a.scores && head_ok) {
-        float* srow = a.scores + (size_t)(qrow0 + r) * a.max_len + (t0 + (int64_t)i * kTileMma + tb);
+            for (int nb = 0; nb < NB; ++nb) bf[nb] = bq[(kstep * NB + nb) * 32 + lane];
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if (tv[e]) srow[c + 4 * e] = lg[e] * kLn2;
-      }
-      float cmax = fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3]));
-      cmax = fmaxf(cmax, __shfl_xor_sync(kFull, cmax, 1));
-      cmax = fmaxf(cmax, __shfl_xor_sync(kFull, cmax, 2));
-      // Lazy rescaling: the reference maximum moves only when a logit exceeds it by
-      // more than kSlack (base 2), so p stays below 2^kSlack and the accumulators are
-      // rescaled a handful of times per CTA instead of at most chunks.
-      if (cmax > m_run + kSlack) {
-        if (m_run != -INFINITY) {
-          const float corr = ex2(m_run - cmax);
-          l_run *= corr;
+            for (int mb = 0; mb < MB; ++mb) {
+              uint4 af;
+              af.x = v[2 * mb] & mlo;
+              af.y = v[2 * mb + 1] & mlo;
+              af.z = v[2 * mb] & mhi;
+              af.w = v[2 * mb + 1] & mhi;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dmin[e] *= corr;
-#pragma unroll
-          for (int nbk = 0; nbk < 16; ++nbk)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) dv[nbk][e] *= corr;
-        }
-        m_run = cmax;
-      }
-      float p[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        p[e] = ex2(lg[e] - m_run);
-        l_run += p[e];
-      }
-
-      // ---- values: D[head hi/lo rows][coordinate columns] += P' x codes ----------
-      // p is split once into f16 hi + lo; for each value group g the operand
-      // P'_g = p * scale_g is formed in half2 arithmetic as an exact product split:
-      // hi = p_hi*s (rounded), err = fma(p_hi, s, -hi) (exact), lo = fma(p_lo, s, err).
-      // The group minima enter through one more MMA: sum_t p_t * min(t, g).
-      // Tokens past the end of a ragged tile carry stale bytes: weight 0, params 0.
-      uint4 par[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) par[e] = vp[tb + c + 4 * e];
-      if (ragged) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if (!tv[e]) par[e] = make_uint4(0u, 0u, 0u, 0u);
-      }
-      const __half2 ph01 = __floats2half2_rn(p[0], p[1]);
-      const __half2 ph23 = __floats2half2_rn(p[2], p[3]);
-      const float2 pf01 = __half22float2(ph01), pf23 = __half22float2(ph23);
-      const __half2 pl01 = __floats2half2_rn(p[0] - pf01.x, p[1] - pf01.y);
-      const __half2 pl23 = __floats2half2_rn(p[2] - pf23.x, p[3] - pf23.y);
-      {
-        // group minima: B[token][group] = min (high half of word g); rows r < 4 are the groups
-        const int gsel = r & 3;
-        auto word = [&](const uint4& w) { return gsel == 0 ? w.x : gsel == 1 ? w.y : gsel == 2 ? w.z : w.w; };
-        const uint32_t m01 = r < 4 ? __byte_perm(word(par[0]), word(par[1]), 0x7632) : 0u;
-        const uint32_t m23 = r < 4 ? __byte_perm(word(par[2]), word(par[3]), 0x7632) : 0u;
-        uint4 ap;
-        ap.x = h2_bits(ph01);
-        ap.y = h2_bits(pl01);
-        ap.z = h2_bits(ph23);
-        ap.w = h2_bits(pl23);
-        mma16816(dmin, ap, m01, m23);
-      }
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const uint32_t w0 = g == 0 ? par[0].x : g == 1 ? par[0].y : g == 2 ? par[0].z : par[0].w;
-        const uint32_t w1 = g == 0 ? par[1].x : g == 1 ? par[1].y : g == 2 ? par[1].z : par[1].w;
-        const uint32_t w2 = g == 0 ? par[2].x : g == 1 ? par[2].y : g == 2 ? par[2].z : par[2].w;
-        const uint32_t w3 = g == 0 ? par[3].x : g == 1 ? par[3].y : g == 2 ? par[3].z : par[3].w;
-        const __half2 s01 = bits_h2(__byte_perm(w0, w1, 0x5410));  // (scale of token c, of c + 4)
-        const __half2 s23 = bits_h2(__byte_perm(w2, w3, 0x5410));
-        const __half2 hi01 = __hmul2(ph01, s01), hi23 = __hmul2(ph23, s23);
-        const __half2 er01 = __hfma2(ph01, s01, __hneg2(hi01)), er23 = __hfma2(ph23, s23, __hneg2(hi23));
-        const __half2 lo01 = __hfma2(pl01, s01, er01), lo23 = __hfma2(pl23, s23, er23);
-        uint4 av;
-        av.x = h2_bits(hi01);
-        av.y = h2_bits(lo01);
-        av.z = h2_bits(hi23);
-        av.w = h2_bits(lo23);
-        // codes of coordinate 32g + 4r + sigma for the 4 tokens
-        uint32_t w4[4];
-        constexpr int WPT = L::VCB / 4;  // value code words per token
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int tok = tb + c + 4 * e;
-          w4[e] = VB == 2 ? vc[tok * WPT + 2 * g + (r >> 2)] : vc[tok * WPT + 4 * g + (r >> 1)];
-        }
-        if (VB == 2) {
-          const uint32_t byte = r & 3;
-          const uint32_t sel = byte | ((4 + byte) << 8);
-          const uint32_t x01 = __byte_perm(w4[0], w4[1], sel);
-          const uint32_t x23 = __byte_perm(w4[2], w4[3], sel);
-#pragma unroll
-          for (int sg = 0; sg < 4; ++sg) {
-            const uint32_t m = (3u << (2 * sg)) | (3u << (16 + 2 * sg));
-            mma16816(dv[4 * g + sg], av, x01 & m, x23 & m);
-          }
-        } else {
-          const uint32_t byte0 = 2 * (r & 1);
-#pragma unroll
-          for (int hb = 0; hb < 2; ++hb) {
-            const uint32_t bt = byte0 + hb;
-            const uint32_t sel = bt | ((4 + bt) << 8);
-            const uint32_t x01 = __byte_perm(w4[0], w4[1], sel);
-            const uint32_t x23 = __byte_perm(w4[2], w4[3], sel);
-#pragma unroll
-            for (int nib = 0; nib < 2; ++nib) {
-              const uint32_t m = (15u << (4 * nib)) | (15u << (16 + 4 * nib));
-              mma16816(dv[4 * g + 2 * hb + nib], av, x01 & m, x23 & m);
+              for (int nb = 0; nb < NB; ++nb) {
+                if (q < LMB)
+                  mma16816(dl[mb][nb], af, bf[nb].x, bf[nb].y);
+                else
+                  mma16816(ds[mb][nb], af, bf[nb].x, bf[nb].y);
+              }
             }
           }
         }
       }
+
+#pragma unroll
+      for (int mb = 0; mb < MB; ++mb) {
+        const int tb = wbase + 16 * mb;
+        if (tb >= nt) break;  // warp-uniform
+        const int nv = nt - tb;  // valid tokens from tb on (rows past it hold stale bytes)
+
+        // ---- logits and online softmax: lane (r, c) has tokens tb + r, tb + r + 8 ----
+        const float2 ng0 = unpack_h2(kn[tb + r]), ng1 = unpack_h2(kn[tb + r + 8]);  // (n, gamma)
+        float lg[NB][2];
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+          const float lm0 = dl[mb][nb][0] + dl[mb][nb][1], lm1 = dl[mb][nb][2] + dl[mb][nb][3];
+          const float sg0 = ds[mb][nb][0] + ds[mb][nb][1], sg1 = ds[mb][nb][2] + ds[mb][nb][3];
+          lg[nb][0] = ng0.x * fmaf(ng0.y, fmaf(k3[nb], sg0, -k4[nb]), fmaf(k2[nb], lm0, k1[nb]));
+          lg[nb][1] = ng1.x * fmaf(ng1.y, fmaf(k3[nb], sg1, -k4[nb]), fmaf(k2[nb], lm1, k1[nb]));
+          if (nv < 16) {
+            if (r >= nv) lg[nb][0] = -INFINITY;
+            if (r + 8 >= nv) lg[nb][1] = -INFINITY;
+          }
+        }
+        if (a.scores) {
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) {
+            const int h = c + 4 * nb;
+            if (h < G) {
+              float* srow = a.scores + (size_t)(qrow0 + h) * a.max_len + (t0 + (int64_t)i * TILE + tb);
+              if (r < nv) srow[r] = lg[nb][0] * kLn2;
+              if (r + 8 < nv) srow[r + 8] = lg[nb][1] * kLn2;
+            }
+          }
+        }
+        uint32_t ph[NB], pl[NB];
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+          float cm = fmaxf(lg[nb][0], lg[nb][1]);
+          cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 4));
+          cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 8));
+          cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 16));
+          // Lazy rescaling: the reference maximum moves only when a logit exceeds it by
+          // more than kSlack (base 2), so p stays below 2^kSlack and the accumulators
+          // are rescaled a handful of times per CTA.
+          if (cm > m_run[nb] + kSlack) {
+            if (m_run[nb] != -INFINITY) {
+              const float corr = ex2(m_run[nb] - cm);
+              l_run[nb] *= corr;
+#pragma unroll
+              for (int e = 0; e < 4; ++e) dmin[nb][e] *= corr;
+#pragma unroll
+              for (int g = 0; g < 4; ++g)
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) dv[g][hf][nb][e] *= corr;
+            }
+            m_run[nb] = cm;
+          }
+          const float p0 = ex2(lg[nb][0] - m_run[nb]), p1 = ex2(lg[nb][1] - m_run[nb]);
+          l_run[nb] += p0 + p1;
+          const __half2 hp = __floats2half2_rn(p0, p1);
+          const float2 hpf = __half22float2(hp);
+          ph[nb] = h2_bits(hp);
+          pl[nb] = h2_bits(__floats2half2_rn(p0 - hpf.x, p1 - hpf.y));
+        }
+
+        // ---- values: D[coordinate rows][head columns] += codes x P' -----------------
+        // B element (token t, head h, part) = p(t, h) * scale(t, g) split in f16 hi + lo:
+        // hi = p_hi*s (rounded), err = fma(p_hi, s, -hi) (exact), lo = fma(p_lo, s, err).
+        // The group minima enter through one more MMA: sum_t p_t * min(t, g).
+        uint32_t phA[NB], plA[NB], phB[NB], plB[NB];
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+          phA[nb] = __shfl_sync(kFull, ph[nb], srcA);
+          plA[nb] = __shfl_sync(kFull, pl[nb], srcA);
+          phB[nb] = __shfl_sync(kFull, ph[nb], srcB);
+          plB[nb] = __shfl_sync(kFull, pl[nb], srcB);
+        }
+        const int tA0 = tb + c, tA1 = tA0 + 8, tB0 = tA0 + 4, tB1 = tA0 + 12;
+        uint4 pA0 = vp[tA0], pA1 = vp[tA1], pB0 = vp[tB0], pB1 = vp[tB1];
+        uint32_t mA0 = 0u, mA1 = 0u, mB0 = 0u, mB1 = 0u;
+        if (r < 4) {
+          mA0 = vpw[tA0 * 4 + r];
+          mA1 = vpw[tA1 * 4 + r];
+          mB0 = vpw[tB0 * 4 + r];
+          mB1 = vpw[tB1 * 4 + r];
+        }
+        if (nv < 16) {  // tokens past the end: weight 0 and params 0 (their bytes are stale)
+          const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+          if (c >= nv) { pA0 = z; mA0 = 0u; }
+          if (c + 8 >= nv) { pA1 = z; mA1 = 0u; }
+          if (c + 4 >= nv) { pB0 = z; mB0 = 0u; }
+          if (c + 12 >= nv) { pB1 = z; mB1 = 0u; }
+        }
+        {
+          uint4 am;  // rows g < 4: (min(t, g) of the two tokens of each K pair); rows 4.. zero
+          am.x = __byte_perm(mA0, mA1, 0x7632);
+          am.y = 0u;
+          am.z = __byte_perm(mB0, mB1, 0x7632);
+          am.w = 0u;
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb)
+            mma16816(dmin[nb], am, part ? plA[nb] : phA[nb], part ? plB[nb] : phB[nb]);
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const __half2 sA = bits_h2(__byte_perm(word_of(pA0, g), word_of(pA1, g), 0x5410));
+          const __half2 sB = bits_h2(__byte_perm(word_of(pB0, g), word_of(pB1, g), 0x5410));
+          uint32_t bA[NB], bB[NB];
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) {
+            const __half2 hA = __hmul2(bits_h2(phA[nb]), sA), hB = __hmul2(bits_h2(phB[nb]), sB);
+            const __half2 eA = __hfma2(bits_h2(phA[nb]), sA, __hneg2(hA));
+            const __half2 eB = __hfma2(bits_h2(phB[nb]), sB, __hneg2(hB));
+            bA[nb] = part ? h2_bits(__hfma2(bits_h2(plA[nb]), sA, eA)) : h2_bits(hA);
+            bB[nb] = part ? h2_bits(__hfma2(bits_h2(plB[nb]), sB, eB)) : h2_bits(hB);
+          }
+          // Row r of block (g, hf) is one byte of the group's codes; the codes of the
+          // two tokens of a K pair go to the low byte of each f16 half.
+          const uint32_t sel = (uint32_t)(r & 3) | ((uint32_t)(4 + (r & 3)) << 8);
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            uint32_t xA, xB;
+            uint4 av;
+            if (VB == 2) {
+              // byte 8g + r: rows r -> coordinate 4(8g + r) + 2hf, rows r + 8 -> + 1
+              constexpr int WPT = L::VCB / 4;
+              const int wv = 2 * g + (r >> 2);
+              if (hf == 0) {
+                xA = __byte_perm(vc[tA0 * WPT + wv], vc[tA1 * WPT + wv], sel);
+                xB = __byte_perm(vc[tB0 * WPT + wv], vc[tB1 * WPT + wv], sel);
+              }
+              const uint32_t m0 = 0x00030003u << (4 * hf), m1 = 0x00030003u << (4 * hf + 2);
+              av = make_uint4(xA & m0, xA & m1, xB & m0, xB & m1);
+            } else {
+              // byte 16g + 8hf + r: rows r -> coordinate 2(16g + 8hf + r), rows r + 8 -> + 1
+              constexpr int WPT = L::VCB / 4;
+              const int wv = 4 * g + 2 * hf + (r >> 2);
+              xA = __byte_perm(vc[tA0 * WPT + wv], vc[tA1 * WPT + wv], sel);
+              xB = __byte_perm(vc[tB0 * WPT + wv], vc[tB1 * WPT + wv], sel);
+              av = make_uint4(xA & 0x000F000Fu, xA & 0x00F000F0u, xB & 0x000F000Fu, xB & 0x00F000F0u);
+            }
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) mma16816(dv[g][hf][nb], av, bA[nb], bB[nb]);
+          }
+        }
+      }
     }
-    // The last warp to finish with this stage refills it with tile i + kStages.
+    // The last warp to finish with this stage refills it with tile i + NST.
     __syncwarp();
     if (lane == 0) {
       __threadfence_block();
-      const int prev = atomicAdd(&arrive_s[i % kStages], 1);
+      const int prev = atomicAdd(&arrive_s[i % NST], 1);
       if (prev == kWarpsMma - 1) {
-        arrive_s[i % kStages] = 0;
-        if (a.use_tma && i + kStages < ntiles && tile_full(i + kStages)) {
+        arrive_s[i % NST] = 0;
+        if (a.use_tma && i + NST < ntiles && tile_full(i + NST)) {
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          issue(i + kStages);
+          issue(i + NST);
         }
       }
     }
@@ -699,45 +752,47 @@ __global__ void __launch_bounds__(kThreadsMma, 4) decode_mma_kernel(const __grid
     if (tid == 0) {
       // Phases of one mbarrier complete in order: waiting for the last batch issued
       // into each stage covers every copy still in flight.
-      for (int st = 0; st < kStages; ++st)
-        if (issued_s[st] > 0) mbar_wait(&bars[st], (uint32_t)((issued_s[st] - 1) & 1));
+      for (int s = 0; s < NST; ++s)
+        if (issued_s[s] > 0) mbar_wait(&bars[s], (uint32_t)((issued_s[s] - 1) & 1));
     }
     __syncthreads();
     return;
   }
 
   // ---- per-warp results -> CTA partial ---------------------------------------------
-  l_run += __shfl_xor_sync(kFull, l_run, 1);
-  l_run += __shfl_xor_sync(kFull, l_run, 2);
-  // thread (r, c) holds sum p*min for groups 2c, 2c+1 (c < 2) in dmin[0] + dmin[2], dmin[1] + dmin[3]
-  float lo_acc[4];
-  {
-    const float own0 = dmin[0] + dmin[2], own1 = dmin[1] + dmin[3];
-#pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      const float v = __shfl_sync(kFull, (g & 1) ? own1 : own0, (lane & ~3) | (g >> 1));
-      lo_acc[g] = v;
-    }
-  }
   float* red = reinterpret_cast<float*>(stage_base);  // [warp][head][kPartPadMma + d]
   constexpr int RS = kPartPadMma + kD;
-  float* mine = red + (warp * 8 + r) * RS;
-  if (c == 0) {
-    mine[0] = m_run;
-    mine[1] = l_run;
-  }
 #pragma unroll
-  for (int nbk = 0; nbk < 16; ++nbk) {
-    const int g = nbk >> 2, sg = nbk & 3;
-    // n-block (g, sg): column n is coordinate 32g + 4n + sg; the code sat at mantissa
-    // bit 2 sg (2-bit) or 4 (sg & 1) (4-bit) of the f16 operand.
-    const int shift = VB == 2 ? 2 * sg : 4 * (sg & 1);
-    const float unscale = ldexpf(1.f, 24 - shift);
+  for (int nb = 0; nb < NB; ++nb) {
+    float l = l_run[nb];
+    l += __shfl_xor_sync(kFull, l, 4);
+    l += __shfl_xor_sync(kFull, l, 8);
+    l += __shfl_xor_sync(kFull, l, 16);
+    // lane (g, c), g < 4, holds sum_t p * min(t, g) for head c + 4 nb in dmin[0] + dmin[1]
+    const float own = dmin[nb][0] + dmin[nb][1];
+    float mt[4];
 #pragma unroll
-    for (int col = 0; col < 2; ++col) {
-      const int j = 32 * g + 4 * (2 * c + col) + sg;
-      mine[kPartPadMma + j] = (dv[nbk][col] + dv[nbk][col + 2]) * unscale + lo_acc[g];
+    for (int g = 0; g < 4; ++g) mt[g] = __shfl_sync(kFull, own, 4 * g + c);
+    float* mine = red + (warp * 8 + c + 4 * nb) * RS;
+    if (r == 0) {
+      mine[0] = m_run[nb];
+      mine[1] = l;
     }
+#pragma unroll
+    for (int g = 0; g < 4; ++g)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const float* d = dv[g][hf][nb];
+        if (VB == 2) {
+          const int j = 4 * (8 * g + r) + 2 * hf;  // code at mantissa bits 4hf (row r), 4hf + 2 (row r + 8)
+          mine[kPartPadMma + j] = (d[0] + d[1]) * ldexpf(1.f, 24 - 4 * hf) + mt[g];
+          mine[kPartPadMma + j + 1] = (d[2] + d[3]) * ldexpf(1.f, 22 - 4 * hf) + mt[g];
+        } else {
+          const int j = 2 * (16 * g + 8 * hf + r);  // low nibble (row r), high nibble (row r + 8)
+          mine[kPartPadMma + j] = (d[0] + d[1]) * 16777216.f + mt[g];
+          mine[kPartPadMma + j + 1] = (d[2] + d[3]) * 1048576.f + mt[g];
+        }
+      }
   }
   __syncthreads();
   float* ws_base = a.ws_part + (size_t)unit * a.n_chunks * G * RS;
@@ -756,11 +811,11 @@ __global__ void __launch_bounds__(kThreadsMma, 4) decode_mma_kernel(const __grid
         den = fmaf(wt, pw[1], den);
       }
     }
-    float* part = ws_base + ((size_t)chunk * G + h) * RS;
-    part[kPartPadMma + j] = num;
+    float* part_out = ws_base + ((size_t)chunk * G + h) * RS;
+    part_out[kPartPadMma + j] = num;
     if (j == 0) {
-      part[0] = mx;
-      part[1] = den;
+      part_out[0] = mx;
+      part_out[1] = den;
     }
   }
 
@@ -845,13 +900,13 @@ __global__ void __launch_bounds__(kThreadsMma, 4) decode_mma_kernel(const __grid
   }
 }
 
-template <int LMB, int VB>
+template <int LMB, int VB, int NB>
 cudaError_t launch_mma_t(const MmaArgs& a, dim3 grid, cudaStream_t s) {
-  using L = Layout<LMB, VB>;
+  using L = Layout<LMB, VB, NB>;
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<LMB, VB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)L::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<LMB, VB, NB>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::SMEM);
     if (e != cudaSuccess) return e;
     configured = true;
   }
@@ -865,45 +920,19 @@ cudaError_t launch_mma_t(const MmaArgs& a, dim3 grid, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_mma_kernel<LMB, VB>, a);
+  return cudaLaunchKernelEx(&cfg, decode_mma_kernel<LMB, VB, NB>, a);
+}
+
+template <int LMB, int VB>
+cudaError_t launch_mma_nb(const MmaArgs& a, int nb, dim3 grid, cudaStream_t s) {
+  return nb == 1 ? launch_mma_t<LMB, VB, 1>(a, grid, s) : launch_mma_t<LMB, VB, 2>(a, grid, s);
 }
 
 }  // namespace
 
-// For every operand element of the query fragments (chunk k, lane l, register q,
-// half e) the layout fixes which query coordinate it scales and by which power of
-// two (the inverse of the lone-bit f16 value its key bit becomes). Encoded per
-// element as src (8 bits: 0..127 = qr index, 128..255 = 128 + sq index), code plane
-// (1 bit), exponent + 16 (5 bits).
-void build_frag_table(int lmb, uint16_t* table) {
-  const int n = frag_chunks(lmb) * 32 * 4;
-  for (int idx = 0; idx < n; ++idx) {
-    const int q = idx & 3, l = (idx >> 2) & 31, k = idx >> 7;
-    const int slot0 = 2 * (l & 3) + ((q & 2) ? 8 : 0);
-    for (int e = 0; e < 2; ++e) {
-      const int s = slot0 + e;
-      const int cs = (s & 7) >> 1, half = s & 1;
-      const int rho = 2 * (k & 7) + (s >> 3), wi = k >> 3;
-      const int o = key_orig(rho) + 16 * half;
-      const int ex = -lone_bit_log2(key_pos(rho));
-      int src, plane = 0;
-      if (wi < lmb) {
-        const int sbit = 32 * (cs + 4 * wi) + o;  // bit of the key's code stream
-        src = sbit / lmb;
-        plane = sbit % lmb;
-      } else {
-        src = kD + 32 * cs + o;
-      }
-      table[2 * idx + e] = (uint16_t)(src | (plane << 8) | ((ex + 16) << 9));
-    }
-  }
-}
-
-size_t frag_table_entries(int lmb) { return (size_t)frag_chunks(lmb) * 32 * 4 * 2; }
-
 bool mma_decode_supported(const tq_ctx* ctx, int G) {
   const Shape& sh = ctx->shape;
-  if (sh.d != kD || sh.m != kM || G < 1 || G > 8 || !ctx->frag_table) return false;
+  if (sh.d != kD || sh.m != kM || G < 1 || G > 8) return false;
   if (sh.lm_bits < 1 || sh.lm_bits > 2) return false;
   if (sh.lm_bits == 2) {
     // the codebook must be affine in its two bits (true for a symmetric codebook)
@@ -914,7 +943,9 @@ bool mma_decode_supported(const tq_ctx* ctx, int G) {
   return sh.v_bits == 2 || sh.v_bits == 4;
 }
 
-size_t mma_frag_bytes(int lm_bits) { return (size_t)frag_words(lm_bits) * 4; }
+size_t mma_frag_bytes(int lm_bits, int G) { return (size_t)frag_words(lm_bits, n_blocks(G)) * 4; }
+
+int mma_tile_tokens(int G) { return tile_tokens(n_blocks(G)); }
 
 cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const void* q, int q_dtype, int batch,
                               int hq, int hkv, const int32_t* seq_lens, int64_t max_len, const uint8_t* k_codes,
@@ -925,8 +956,9 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
   uint32_t* frag = reinterpret_cast<uint32_t*>(ws + plan.off_frag);
   float* part = reinterpret_cast<float*>(ws + plan.off_part);
   unsigned int* cnt = reinterpret_cast<unsigned int*>(ws + plan.off_cnt);
-  const int G = hq / hkv, lmb = ctx->shape.lm_bits, vb = ctx->shape.v_bits;
+  const int G = hq / hkv, lmb = ctx->shape.lm_bits, vb = ctx->shape.v_bits, nb = n_blocks(G);
   const float* cc = ctx->cb.c;
+  if (plan.chunk_len % tile_tokens(nb) != 0) return cudaErrorInvalidValue;
 
   PrepArgs pa;
   pa.q = q;
@@ -941,9 +973,9 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
   pa.cb = ctx->cb;
   pa.beta0 = cc[1] - cc[0];
   pa.beta1 = lmb > 1 ? cc[2] - cc[0] : 0.f;
+  pa.nb = nb;
   pa.frag = frag;
   pa.cnt = cnt;
-  pa.table = ctx->frag_table;
   const size_t prep_smem = sizeof(float) * kD * kM;
   static bool prep_configured = false;
   if (!prep_configured) {
@@ -985,9 +1017,9 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
   const dim3 grid(plan.n_chunks, batch * hkv);
   if (ctx->prof_start) cudaEventRecord(ctx->prof_start, stream);
   if (lmb == 1)
-    e = vb == 2 ? launch_mma_t<1, 2>(a, grid, stream) : launch_mma_t<1, 4>(a, grid, stream);
+    e = vb == 2 ? launch_mma_nb<1, 2>(a, nb, grid, stream) : launch_mma_nb<1, 4>(a, nb, grid, stream);
   else
-    e = vb == 2 ? launch_mma_t<2, 2>(a, grid, stream) : launch_mma_t<2, 4>(a, grid, stream);
+    e = vb == 2 ? launch_mma_nb<2, 2>(a, nb, grid, stream) : launch_mma_nb<2, 4>(a, nb, grid, stream);
   if (ctx->prof_stop) cudaEventRecord(ctx->prof_stop, stream);
   return e;
 }

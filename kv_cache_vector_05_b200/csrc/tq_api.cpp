@@ -34,7 +34,6 @@ void free_tables(tq_ctx* c) {
   cudaFree(c->Pi);
   cudaFree(c->PiT);
   cudaFree(c->d_err);
-  cudaFree(c->frag_table);
   cudaFree(c->S_sw128);
 }
 
@@ -161,12 +160,6 @@ tq_status tq_codebook_load(const tq_params* p, void* stream, tq_ctx** out) {
     if (!tq::pack_qjl_operand(p->qjl_S, m, d, s_op.data())) s_op.clear();
     if (e == cudaSuccess && !s_op.empty()) e = cudaMalloc((void**)&c->S_sw128, s_op.size() * sizeof(uint16_t));
   }
-  std::vector<uint16_t> table;
-  if (d == 128 && m == 128 && b <= 2) {
-    table.resize(tq::frag_table_entries(b));
-    tq::build_frag_table(b, table.data());
-    if (e == cudaSuccess) e = cudaMalloc((void**)&c->frag_table, table.size() * sizeof(uint16_t));
-  }
   if (e != cudaSuccess) {
     free_tables(c);
     delete c;
@@ -184,8 +177,6 @@ tq_status tq_codebook_load(const tq_params* p, void* stream, tq_ctx** out) {
   if (e == cudaSuccess) e = cudaMemsetAsync(c->d_err, 0, sizeof(unsigned int), s);
   if (e == cudaSuccess && !s_op.empty())
     e = cudaMemcpyAsync(c->S_sw128, s_op.data(), s_op.size() * sizeof(uint16_t), cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess && !table.empty())
-    e = cudaMemcpyAsync(c->frag_table, table.data(), table.size() * sizeof(uint16_t), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) {
     free_tables(c);

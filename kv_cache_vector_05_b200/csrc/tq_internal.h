@@ -45,7 +45,6 @@ struct tq_ctx {
   cudaEvent_t prof_start;  // optional events around the main kernel of each call
   cudaEvent_t prof_stop;
   unsigned int* d_err;     // device error word: bit 0 = a bounded wait in a kernel timed out
-  uint16_t* frag_table;    // tensor-core decode: operand sources (d = m = 128, lm_bits <= 2)
   uint16_t* S_sw128;       // tensor-core compression: S as an f16 operand tile (d = m = 128, S exact in f16)
 };
 
@@ -76,10 +75,9 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const void*
 
 bool mma_decode_supported(const tq_ctx* ctx, int G);
 
-size_t mma_frag_bytes(int lm_bits);
+size_t mma_frag_bytes(int lm_bits, int G);  // query operand bytes per (sequence, KV head)
+int mma_tile_tokens(int G);                  // tokens per tile of the tensor-core decode
 bool pack_qjl_operand(const float* S, int m, int d, uint16_t* out);
-void build_frag_table(int lmb, uint16_t* table);
-size_t frag_table_entries(int lmb);
 
 cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const void* q, int q_dtype, int batch,
                               int hq, int hkv, const int32_t* seq_lens, int64_t max_len, const uint8_t* k_codes,

@@ -180,6 +180,7 @@ def test_decode_single_head_fp32_oracle_compressed():
 
 @pytest.mark.parametrize("d,lm_bits,v_bits,G", [
     (128, 2, 2, 4), (128, 2, 2, 8), (128, 3, 4, 6), (128, 1, 4, 1),
+    (128, 1, 2, 2), (128, 1, 2, 6), (128, 1, 4, 7), (128, 2, 4, 3), (128, 2, 4, 6), (128, 2, 2, 5),
     (64, 2, 4, 8), (64, 3, 2, 5), (256, 2, 2, 4), (256, 3, 4, 2), (256, 1, 2, 8),
 ])
 def test_decode_parity_random_cache(d, lm_bits, v_bits, G):
