@@ -187,7 +187,7 @@ tq_status tq_check_device(const tq_ctx* ctx, void* stream);
  * without a caching allocator.
  * Same arguments, layouts and results as tq_decode_attention, minus workspace.
  * The scratch is a fixed device array of tq_decode_static_scratch_capacity()
- * bytes (8 MiB) inside this library; every GPU that loads the library holds one
+ * bytes (32 MiB) inside this library; every GPU that loads the library holds one
  * until the process exits. A shape whose workspace (tq_decode_workspace_bytes)
  * exceeds it returns TQ_EUNSUPPORTED with the sizes in tq_last_error().
  * The first call on each device looks up the array's device address

@@ -352,46 +352,49 @@ DecodePlan plan_decode(const tq_ctx* ctx, int batch, int hq, int hkv, int64_t ma
   const int d = ctx->shape.d, m = ctx->shape.m, G = hq / hkv;
   p.mma = mma_decode_supported(ctx, G);
   const int64_t units = (int64_t)batch * hkv;
-  const int64_t tile = p.mma ? mma_tile_tokens(G) : kTile;
-  const int64_t tiles = max_len > 0 ? (max_len + tile - 1) / tile : 1;
   const int64_t sms = ctx->num_sms > 0 ? ctx->num_sms : 148;
-  int64_t chunks = 1;
   if (p.mma) {
-    // Split each (sequence, KV head) into chunks so that the grid fills whole waves
-    // of resident CTAs (4 per SM): minimise waves x tiles-per-CTA, plus a small
-    // per-wave cost.
-    const int64_t slots = 4 * sms;
-    double best = 1e300;
-    const int64_t max_chunks = tiles < 4096 ? tiles : 4096;
-    for (int64_t n = 1; n <= max_chunks && units > 0; ++n) {
-      const int64_t waves = (units * n + slots - 1) / slots;
-      const double cost = (double)waves * (double)((tiles + n - 1) / n) + 0.5 * (double)waves;
-      if (cost < best) {
-        best = cost;
-        chunks = n;
-      }
+    // Every unit (sequence x KV head) is cut into tiles; the units' tiles, laid end
+    // to end, are split evenly over one wave of resident CTAs (one per SM). A CTA's
+    // range may cross unit boundaries; each unit is merged from the partials of the
+    // CTAs that share it.
+    const int64_t tile = mma_tile_tokens(G);
+    const int64_t Tu = max_len > 0 ? (max_len + tile - 1) / tile : 1;
+    const int64_t Tt = units * Tu;
+    const int64_t slots = (int64_t)mma_ctas_per_sm(ctx->shape.lm_bits, ctx->shape.v_bits, G) * sms;
+    const int64_t P = Tt < slots ? Tt : slots;
+    p.n_ctas = (int)P;
+    p.tiles_per_unit = Tu;
+    p.total_tiles = Tt;
+    int64_t s_max = 1;
+    for (int64_t u = 0; u < units; ++u) {
+      const int64_t first = ((u * Tu + 1) * P - 1) / Tt, last = ((u + 1) * Tu * P - 1) / Tt;
+      if (last - first + 1 > s_max) s_max = last - first + 1;
     }
-  } else {
-    const int64_t target = 4 * sms;  // a few waves of resident CTAs
-    chunks = units > 0 ? (target + units - 1) / units : 1;
-    if (chunks > tiles) chunks = tiles;
-    if (chunks < 1) chunks = 1;
-  }
-  const int64_t tiles_per_chunk = (tiles + chunks - 1) / chunks;
-  p.chunk_len = tiles_per_chunk * tile;
-  p.n_chunks = (int)((tiles + tiles_per_chunk - 1) / tiles_per_chunk);
-  p.ws_part_bytes = align256((size_t)units * p.n_chunks * G * (d + kPartPad) * sizeof(float));
-  if (p.mma) {
+    p.s_max = (int)s_max;
+    p.n_chunks = 0;
+    p.chunk_len = 0;
     p.ws_q_bytes = 0;
+    p.ws_part_bytes =
+        align256((size_t)units * s_max * G * (d + kPartPad) * sizeof(float));
     p.off_frag = 0;
     p.off_part = align256((size_t)units * mma_frag_bytes(ctx->shape.lm_bits, G));
-    p.off_cnt = p.off_part + p.ws_part_bytes;
-    p.total_bytes = p.off_cnt + align256((size_t)units * sizeof(unsigned int));
-  } else {
-    const int q_stride = d + m;
-    p.ws_q_bytes = align256((size_t)batch * hq * q_stride * sizeof(float));
-    p.total_bytes = p.ws_q_bytes + p.ws_part_bytes;
+    p.off_cnt = p.off_part + p.ws_part_bytes;  // no counters on this path
+    p.total_bytes = p.off_cnt;
+    return p;
   }
+  const int64_t tiles = max_len > 0 ? (max_len + kTile - 1) / kTile : 1;
+  const int64_t target = 4 * sms;  // a few waves of resident CTAs
+  int64_t chunks = units > 0 ? (target + units - 1) / units : 1;
+  if (chunks > tiles) chunks = tiles;
+  if (chunks < 1) chunks = 1;
+  const int64_t tiles_per_chunk = (tiles + chunks - 1) / chunks;
+  p.chunk_len = tiles_per_chunk * kTile;
+  p.n_chunks = (int)((tiles + tiles_per_chunk - 1) / tiles_per_chunk);
+  p.ws_part_bytes = align256((size_t)units * p.n_chunks * G * (d + kPartPad) * sizeof(float));
+  const int q_stride = d + m;
+  p.ws_q_bytes = align256((size_t)batch * hq * q_stride * sizeof(float));
+  p.total_bytes = p.ws_q_bytes + p.ws_part_bytes;
   return p;
 }
 

@@ -52,7 +52,7 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kM = 128;
-constexpr int kWarpsMma = 4;
+constexpr int kWarpsMma = 16;  // warps per decode CTA (one CTA per SM)
 constexpr int kThreadsMma = kWarpsMma * 32;
 constexpr int kPartPadMma = 4;
 constexpr int kPrepThreads = 256;
@@ -72,7 +72,7 @@ __host__ __device__ constexpr int n_blocks(int G) { return G <= 4 ? 1 : 2; }
 __host__ __device__ constexpr int m_blocks(int nb) { return nb == 1 ? 2 : 1; }
 __host__ __device__ constexpr int tile_tokens(int nb) { return 16 * kWarpsMma * m_blocks(nb); }
 // Per (sequence, KV head): query operand words [k-step][n-block][32 lanes][2], then
-// [8 heads][4] floats (sum of qr, sum of sq, LM scale, sign scale).
+// [8 heads][4] logit constants (k1..k4 of the decode kernel).
 __host__ __device__ constexpr int frag_words(int lmb, int nb) { return key_steps(lmb) * nb * 64 + 32; }
 
 struct PrepArgs {
@@ -84,9 +84,10 @@ struct PrepArgs {
   const float* PiT;  // [d][d] (Haar)
   Codebook cb;
   float beta0, beta1;
+  float c0;          // lowest centroid
+  float sl2;         // softmax scale * log2(e)
   int nb;            // n-blocks of the query operand
   uint32_t* frag;    // [units][frag_words]
-  unsigned int* cnt; // [units] completion tickets, zeroed here
 };
 
 struct MmaArgs {
@@ -99,14 +100,12 @@ struct MmaArgs {
   const int32_t* seq_lens;
   int64_t max_len;
   int hq, hkv, G;
-  int n_chunks;
-  int64_t chunk_len;
-  float scale;
+  int64_t tiles_per_unit;  // tiles of each (sequence, KV head), from max_len
+  int64_t total_tiles;     // units x tiles_per_unit; CTA k takes [k T / P, (k + 1) T / P)
+  int s_max;               // partial slots per unit (most CTAs sharing one unit)
   float* scores;
   float* out;
-  float* ws_part;
-  unsigned int* cnt;
-  float c0;
+  float* ws_part;          // [units][s_max][G][kPartPadMma + d]
   int use_tma;             // 1 when every record array offset is 16-byte aligned
   unsigned int* err;       // device error word of the context
 };
@@ -122,6 +121,10 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -309,13 +312,17 @@ __global__ void __launch_bounds__(kPrepThreads) prep_mma_kernel(const __grid_con
     smax = warp_max(smax);
     if (lane == 0) {
       const float bmax = fmaxf(fabsf(a.beta0), LMB > 1 ? fabsf(a.beta1) : 0.f);
-      const float qs = qmax * bmax;
-      head_s[h * 4 + 0] = qsum;
-      head_s[h * 4 + 1] = ssum;
-      head_s[h * 4 + 2] = qs > 0.f ? qs : 1.f;
-      head_s[h * 4 + 3] = smax > 0.f ? smax : 1.f;
-      inv_s[h * 2 + 0] = 1.f / head_s[h * 4 + 2];
-      inv_s[h * 2 + 1] = 1.f / head_s[h * 4 + 3];
+      const float qs = qmax * bmax > 0.f ? qmax * bmax : 1.f;  // LM operand scale
+      const float ss = smax > 0.f ? smax : 1.f;                // sign operand scale
+      // logit (base 2) = n * (k1 + k2 * lm + gamma * (k3 * sg - k4)), lm and sg being the
+      // decode kernel's raw tensor-core sums over the normalised operands.
+      constexpr float kSignW = kQjl / (float)kM;
+      head_s[h * 4 + 0] = a.sl2 * a.c0 * qsum;
+      head_s[h * 4 + 1] = a.sl2 * qs;
+      head_s[h * 4 + 2] = a.sl2 * kSignW * 2.f * ss;
+      head_s[h * 4 + 3] = a.sl2 * kSignW * ssum;
+      inv_s[h * 2 + 0] = 1.f / qs;
+      inv_s[h * 2 + 1] = 1.f / ss;
     }
   }
   __syncthreads();
@@ -357,7 +364,6 @@ __global__ void __launch_bounds__(kPrepThreads) prep_mma_kernel(const __grid_con
     frag[w] = pack_h2(v2[0], v2[1]);
   }
   if (tid < 32) reinterpret_cast<float*>(frag)[nwords + tid] = head_s[tid];
-  if (tid == 0) a.cnt[unit] = 0u;
 }
 
 // ------------------------------------------------------------------ decode kernel
@@ -366,72 +372,105 @@ template <int LMB, int VB, int NB>
 struct Layout {
   static constexpr int MB = m_blocks(NB);
   static constexpr int TILE = tile_tokens(NB);
-  static constexpr int STAGES = MB == 2 ? 3 : 4;
   static constexpr int KCB = LMB * kD / 8;  // key code bytes per token
   static constexpr int SB = kM / 8;         // sign bytes
   static constexpr int VCB = VB * kD / 8;   // value code bytes
   static constexpr int PB = (kD / kVGroup) * 4;
   static constexpr int REC = KCB + SB + 4 + VCB + PB;
   static constexpr int STAGE = TILE * REC;
+  static constexpr int FRAG_BYTES = frag_words(LMB, NB) * 4;
+  // As many stages (2..4) as fit in shared memory next to the two operand buffers and
+  // the reduction area (one CTA per SM).
+  static constexpr int RED_BYTES = (8 * kD + 8 + 2 * kWarpsMma * 8 + 16) * 4;
+  static constexpr int BUDGET = 220 * 1024 - 2 * FRAG_BYTES - RED_BYTES - 512;
+  static constexpr int STAGES = 4 * STAGE <= BUDGET ? 4 : 3 * STAGE <= BUDGET ? 3 : 2;
   static constexpr int OFF_KC = 0;
   static constexpr int OFF_KS = OFF_KC + TILE * KCB;
   static constexpr int OFF_KN = OFF_KS + TILE * SB;
   static constexpr int OFF_VC = OFF_KN + TILE * 4;
   static constexpr int OFF_VP = OFF_VC + TILE * VCB;
   static constexpr int KS = key_steps(LMB);
-  static constexpr int FRAG_BYTES = frag_words(LMB, NB) * 4;
-  static constexpr int RED_BYTES = kWarpsMma * 8 * (kPartPadMma + kD) * 4;  // per-warp partials
-  static constexpr int RING = STAGES * STAGE > RED_BYTES ? STAGES * STAGE : RED_BYTES;
-  static constexpr size_t SMEM = (size_t)RING + FRAG_BYTES + 8 * STAGES + 4 * (1 + 2 * STAGES) + 16;
+  static constexpr int RING = STAGES * STAGE;
+  static constexpr int OFF_FRAG = RING;                        // two query-operand buffers
+  static constexpr int OFF_BAR = OFF_FRAG + 2 * FRAG_BYTES;    // STAGES + 2 mbarriers
+  static constexpr int OFF_CNT = OFF_BAR + 8 * (STAGES + 2);   // arrive / issue counters
+  static constexpr int OFF_RED = OFF_CNT + 4 * (2 * STAGES + 4);  // unit-boundary reduction
+  static constexpr size_t SMEM = (size_t)OFF_RED + RED_BYTES;
   static_assert(STAGE % 16 == 0 && FRAG_BYTES % 16 == 0, "16-byte aligned stages and fragments");
+  static_assert(SMEM <= 227 * 1024, "fits one CTA per SM");
 };
 
 __device__ __forceinline__ uint32_t word_of(const uint4& w, int i) {
   return i == 0 ? w.x : i == 1 ? w.y : i == 2 ? w.z : w.w;
 }
 
+// CTA owning global tile g when CTA k takes tiles [k T / P, (k + 1) T / P).
+__device__ __forceinline__ int64_t tile_owner(int64_t g, int64_t P, int64_t T) { return ((g + 1) * P - 1) / T; }
+
 template <int LMB, int VB, int NB>
-__global__ void __launch_bounds__(kThreadsMma, 4) decode_mma_kernel(const __grid_constant__ MmaArgs a) {
+__global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid_constant__ MmaArgs a) {
   using L = Layout<LMB, VB, NB>;
   constexpr int MB = L::MB, TILE = L::TILE, NST = L::STAGES;
+  constexpr int RS = kPartPadMma + kD;
+  constexpr float kLn2 = 0.6931471805599453f;
   extern __shared__ __align__(128) unsigned char smem[];
-  unsigned char* stage_base = smem;                                       // ring, later per-warp partials
-  const uint2* bq = reinterpret_cast<const uint2*>(smem + L::RING);      // [KS][NB][32 lanes]
-  const float* head_s = reinterpret_cast<const float*>(bq + L::KS * NB * 32);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::RING + L::FRAG_BYTES);
-  int* last_s = reinterpret_cast<int*>(bars + NST);
-  int* arrive_s = last_s + 1;         // [NST] warps done with the stage's current tile
-  int* issued_s = arrive_s + NST;     // [NST] bulk-copy batches issued into the stage
+  unsigned char* stage_base = smem;
+  unsigned char* frag_base = smem + L::OFF_FRAG;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);  // [NST] stages
+  uint64_t* fbars = bars + NST;                                      // [2] query operands
+  int* arrive_s = reinterpret_cast<int*>(smem + L::OFF_CNT);  // [NST] warps done with the stage's tile
+  int* issued_s = arrive_s + NST;   // [NST] bulk-copy batches issued into the stage
+  int* fissued_s = issued_s + NST;  // [2] copies issued into the operand buffer
+  float* racc_s = reinterpret_cast<float*>(smem + L::OFF_RED);  // [8 heads][d] rescaled sums
+  float* rl_s = racc_s + 8 * kD;                                 // [8] rescaled sums of p
+  float* rm_s = rl_s + 8;                                        // [warps][8] warp maxima
+  float* rwl_s = rm_s + kWarpsMma * 8;                           // [warps][8] warp sums of p
+  float* rM_s = rwl_s + kWarpsMma * 8;                           // [8] CTA maxima
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int r = lane >> 2, c = lane & 3;
   const int G = a.G;
-  const int chunk = blockIdx.x, unit = blockIdx.y;
-  const int b = unit / a.hkv, kvh = unit % a.hkv;
-  int64_t len = a.max_len;
-  if (a.seq_lens) len = min((int64_t)max(a.seq_lens[b], 0), a.max_len);
-  const int64_t t0 = (int64_t)chunk * a.chunk_len;
-  const int64_t t1 = min(t0 + a.chunk_len, len);
-  const int qrow0 = b * a.hq + kvh * G;
-  const int64_t vec0 = (int64_t)unit * a.max_len;
-  const int span = t1 > t0 ? (int)(t1 - t0) : 0;  // tokens of this chunk (< 2^31)
-  const int ntiles = (span + TILE - 1) / TILE;
+  // Balanced split of the flattened (unit, tile) space: this CTA's tiles [g0, g1) may
+  // span several units (a unit = one sequence x KV head).
+  const int64_t P = gridDim.x, kcta = blockIdx.x;
+  const int64_t Tu = a.tiles_per_unit, Tt = a.total_tiles;
+  const int64_t g0 = kcta * Tt / P, g1 = (kcta + 1) * Tt / P;
+  const int ntl = (int)(g1 - g0);
+  const int u_first = ntl > 0 ? (int)(g0 / Tu) : 0;  // == u0 below
+  const int n_units = ntl > 0 ? (int)((g1 - 1) / Tu) - u_first + 1 : 0;
 
   if (tid == 0) {
-    for (int s = 0; s < NST; ++s) {
-      mbar_init(&bars[s], 1);
-      arrive_s[s] = 0;
-      issued_s[s] = 0;
-    }
+    for (int s = 0; s < NST + 2; ++s) mbar_init(&bars[s], 1);
+    for (int s = 0; s < 2 * NST + 4; ++s) arrive_s[s] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
 
-  auto tile_full = [&](int i) -> bool { return (i + 1) * TILE <= span; };
-  auto issue = [&](int i) {  // one thread: bulk-copy tile i into its stage
-    unsigned char* st = stage_base + (i % NST) * L::STAGE;
-    const int64_t v = vec0 + t0 + (int64_t)i * TILE;
+  auto unit_len = [&](int u) -> int64_t {
+    int64_t len = a.max_len;
+    if (a.seq_lens) len = min((int64_t)max(a.seq_lens[u / a.hkv], 0), a.max_len);
+    return len;
+  };
+  const int u0 = (int)(g0 / Tu);
+  const int64_t tl0 = g0 - (int64_t)u0 * Tu;  // tile index of g0 within its unit
+  // One thread: start tile i. Every tile completes one phase of its stage's barrier:
+  // a full tile (with 16-byte aligned records) through its bulk copies, any other
+  // tile through a plain arrival (its warps then copy it themselves).
+  auto issue = [&](int i) {
+    int u = u0;
+    int64_t tl = tl0 + i;
+    if (tl >= Tu) {
+      u += (int)(tl / Tu);
+      tl -= (tl / Tu) * Tu;
+    }
+    const int64_t tok0 = tl * TILE;
     uint64_t* bar = &bars[i % NST];
+    if (!a.use_tma || unit_len(u) - tok0 < TILE) {
+      mbar_arrive(bar);
+      return;
+    }
+    unsigned char* st = stage_base + (i % NST) * L::STAGE;
+    const int64_t v = (int64_t)u * a.max_len + tok0;
     issued_s[i % NST] += 1;
     mbar_expect_tx(bar, (uint32_t)L::STAGE);
     bulk_g2s(st + L::OFF_KC, a.k_codes + v * L::KCB, TILE * L::KCB, bar);
@@ -440,75 +479,161 @@ __global__ void __launch_bounds__(kThreadsMma, 4) decode_mma_kernel(const __grid
     bulk_g2s(st + L::OFF_VC, a.v_codes + v * L::VCB, TILE * L::VCB, bar);
     bulk_g2s(st + L::OFF_VP, reinterpret_cast<const uint8_t*>(a.v_params) + v * L::PB, TILE * L::PB, bar);
   };
+  auto issue_frag = [&](int j) {  // one thread: query operands of local unit j into buffer j % 2
+    uint64_t* bar = &fbars[j & 1];
+    fissued_s[j & 1] += 1;
+    mbar_expect_tx(bar, (uint32_t)L::FRAG_BYTES);
+    bulk_g2s(frag_base + (j & 1) * L::FRAG_BYTES, a.frag + (size_t)(u_first + j) * frag_words(LMB, NB),
+             L::FRAG_BYTES, bar);
+  };
   // The packed cache does not depend on the prep kernel: start streaming it now.
-  if (tid == 0 && a.use_tma) {
-    for (int i = 0; i < NST && i < ntiles; ++i)
-      if (tile_full(i)) issue(i);
+  if (tid == 0) {
+    for (int i = 0; i < NST && i < ntl; ++i) issue(i);
   }
-
-  // Wait for the prep kernel (programmatic dependent launch), then fetch this KV
-  // head's query fragments and constants.
+  // Wait for the prep kernel (programmatic dependent launch), then fetch the query
+  // operands of this CTA's first two units.
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  {
-    const uint4* src = reinterpret_cast<const uint4*>(a.frag + (size_t)unit * frag_words(LMB, NB));
-    uint4* dst = reinterpret_cast<uint4*>(smem + L::RING);
-    for (int w = tid; w < L::FRAG_BYTES / 16; w += kThreadsMma) dst[w] = src[w];
+  if (tid == 0) {
+    for (int j = 0; j < 2 && j < n_units; ++j) issue_frag(j);
   }
-  __syncthreads();
+  // The combine kernel may launch now; it waits for this grid to finish.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  constexpr float kLog2e = 1.4426950408889634f;
-  constexpr float kLn2 = 0.6931471805599453f;
-  // Lane (r, c) scores heads c + 4 nb. logit (base-2 units) = n * (k1 + k2 * lm +
-  // gamma * (k3 * sg - k4)), with lm, sg the raw tensor-core dot products.
-  const float sl2 = a.scale * kLog2e;
-  float k1[NB], k2[NB], k3[NB], k4[NB];
-#pragma unroll
-  for (int nb = 0; nb < NB; ++nb) {
-    const float* hc = head_s + 4 * (c + 4 * nb);
-    k1[nb] = sl2 * a.c0 * hc[0];
-    k2[nb] = sl2 * hc[2];
-    k3[nb] = sl2 * (kQjl / (float)kM) * 2.f * hc[3];
-    k4[nb] = sl2 * (kQjl / (float)kM) * hc[1];
-  }
-
-  float m_run[NB], l_run[NB];
-  float dmin[NB][4];       // rows g < 4: sum_t p * min(t, g); columns: heads x (hi, lo)
-  float dv[4][2][NB][4];   // [group][half of the group][n-block]: rows = coordinates
-#pragma unroll
-  for (int nb = 0; nb < NB; ++nb) {
-    m_run[nb] = -INFINITY;
-    l_run[nb] = 0.f;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) dmin[nb][e] = 0.f;
-#pragma unroll
-    for (int g = 0; g < 4; ++g)
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dv[g][hf][nb][e] = 0.f;
-  }
-
-  const uint32_t rot = (uint32_t)(9 - 4 * c) & 31u;  // bits 4c..4c+3 (+16) -> 9..12 (+16)
+  // Key bits 4c..4c+3 of each half of a word go to f16 positions 9..12.
+  const uint32_t rot = (uint32_t)(9 - 4 * c) & 31u;
   // Value-side B column of this lane: head 4 nb + hsel, part (hi / lo). Its tokens,
   // in K order, are (c, c + 8) and (c + 4, c + 12) of a 16-token block, whose
   // probabilities the lanes srcA and srcB hold after the score step.
   const int part = r & 1, hsel = r >> 1;
   const int srcA = 4 * c + hsel, srcB = 4 * (c + 4) + hsel;
 
+  float m_run[NB], l_run[NB];
+  float dmin[NB][4];       // rows g < 4: sum_t p * min(t, g); columns: heads x (hi, lo)
+  float dv[4][2][NB][4];   // [group][half of the group][n-block]: rows = coordinates
+  int cur = -1;            // local index of the unit being accumulated
+  int qrow0 = 0;
   bool failed = false;
-  for (int i = 0; i < ntiles; ++i) {
+
+  // End of local unit j (every warp calls this at the same tile): the 16 warps' partials
+  // are merged in shared memory (rescaled to the CTA maximum, summed with shared
+  // atomics) and written as this CTA's partial (m, l, acc) of the unit; combine_mma_kernel
+  // merges the partials of the CTAs that shared the unit. Then buffer j % 2 is refilled
+  // with the operands of unit j + 2.
+  auto finish_unit = [&](int j) {
+    const int u = u_first + j;
+    const int seg = (int)(kcta - tile_owner((int64_t)u * Tu, P, Tt));
+    __syncthreads();  // every warp has left the previous boundary's reduction
+    float lsum[NB];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+      float l = l_run[nb];
+      l += __shfl_xor_sync(kFull, l, 4);
+      l += __shfl_xor_sync(kFull, l, 8);
+      l += __shfl_xor_sync(kFull, l, 16);
+      lsum[nb] = l;
+      if (r == 0) {
+        rm_s[warp * 8 + c + 4 * nb] = failed ? -INFINITY : m_run[nb];
+        rwl_s[warp * 8 + c + 4 * nb] = failed ? 0.f : l;
+      }
+    }
+    for (int x = tid; x < 8 * kD + 8; x += kThreadsMma) racc_s[x] = 0.f;
+    __syncthreads();
+    if (tid < 8) {
+      float M = -INFINITY;
+      for (int w = 0; w < kWarpsMma; ++w) M = fmaxf(M, rm_s[w * 8 + tid]);
+      rM_s[tid] = M;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+      // lane (g, c), g < 4, holds sum_t p * min(t, g) for head c + 4 nb in dmin[0] + dmin[1]
+      const float own = dmin[nb][0] + dmin[nb][1];
+      float mt[4];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) mt[g] = __shfl_sync(kFull, own, 4 * g + c);
+      const int h = c + 4 * nb;
+      const float M = rM_s[h];
+      const float wsc = (failed || m_run[nb] == -INFINITY) ? 0.f : ex2(m_run[nb] - M);
+      if (h < G && wsc != 0.f) {
+        if (r == 0) atomicAdd(&rl_s[h], wsc * lsum[nb]);
+        float* acc = racc_s + h * kD;
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const float* d = dv[g][hf][nb];
+            if (VB == 2) {
+              const int j0 = 4 * (8 * g + r) + 2 * hf;  // code at mantissa bits 4hf (row r), 4hf + 2 (row r + 8)
+              atomicAdd(&acc[j0], wsc * ((d[0] + d[1]) * ldexpf(1.f, 24 - 4 * hf) + mt[g]));
+              atomicAdd(&acc[j0 + 1], wsc * ((d[2] + d[3]) * ldexpf(1.f, 22 - 4 * hf) + mt[g]));
+            } else {
+              const int j0 = 2 * (16 * g + 8 * hf + r);  // low nibble (row r), high nibble (row r + 8)
+              atomicAdd(&acc[j0], wsc * ((d[0] + d[1]) * 16777216.f + mt[g]));
+              atomicAdd(&acc[j0 + 1], wsc * ((d[2] + d[3]) * 1048576.f + mt[g]));
+            }
+          }
+      }
+    }
+    __syncthreads();
+    float* part = a.ws_part + ((size_t)u * a.s_max + seg) * G * RS;
+    for (int x = tid; x < G * kD; x += kThreadsMma) {
+      const int h = x / kD, jj = x - h * kD;
+      part[h * RS + kPartPadMma + jj] = racc_s[x];
+      if (jj == 0) {
+        part[h * RS + 0] = rM_s[h];
+        part[h * RS + 1] = rl_s[h];
+      }
+    }
+    if (tid == 0 && j + 2 < n_units) {
+      // every warp is past unit j: its operand buffer may be refilled
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      issue_frag(j + 2);
+    }
+  };
+
+  int u = u0;
+  int64_t tl = tl0 - 1, ulen = 0;
+  for (int i = 0; i < ntl; ++i) {
+    if (++tl == Tu && i > 0) {
+      tl = 0;
+      ++u;
+    }
+    const int j = u - u_first;
+    if (j != cur) {
+      ulen = unit_len(u);
+      if (cur >= 0) finish_unit(cur);
+      cur = j;
+      // Wait for the unit's query operands; after a timeout the warp keeps the loop's
+      // structure (arrivals, barriers) but does no more work.
+      if (!failed && !mbar_wait(&fbars[j & 1], (uint32_t)((j >> 1) & 1))) failed = true;
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+        m_run[nb] = -INFINITY;
+        l_run[nb] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dmin[nb][e] = 0.f;
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dv[g][hf][nb][e] = 0.f;
+      }
+      const int b = u / a.hkv, kvh = u - b * a.hkv;
+      qrow0 = b * a.hq + kvh * G;
+    }
+    const uint2* bq = reinterpret_cast<const uint2*>(frag_base + (j & 1) * L::FRAG_BYTES);
+    const int64_t tok0 = tl * TILE;
+    const int nt = (int)max((int64_t)0, min((int64_t)TILE, ulen - tok0));
+
     unsigned char* st = stage_base + (i % NST) * L::STAGE;
-    const int nt = min(TILE, span - i * TILE);
-    if (a.use_tma && tile_full(i)) {
-      // Warps run ahead of one another; each waits only for the tile it needs. After
-      // a timeout a warp keeps the loop's structure (arrivals, barriers) but does no
-      // more work, so every warp of the CTA reaches the same barriers.
-      if (!failed && !mbar_wait(&bars[i % NST], (uint32_t)((i / NST) & 1))) failed = true;
-    } else {
+    // Warps run ahead of one another; each waits only for the tile it needs.
+    if (!failed && !mbar_wait(&bars[i % NST], (uint32_t)((i / NST) & 1))) failed = true;
+    if ((nt < TILE || !a.use_tma) && nt > 0) {
       // Ragged or unaligned tile: plain 4-byte copies (all record sizes are multiples
       // of 4), after every warp has left the tile that used this stage before.
       __syncthreads();
-      const int64_t v = vec0 + t0 + (int64_t)i * TILE;
+      const int64_t v = (int64_t)u * a.max_len + tok0;
       auto copy = [&](int off, const void* src, int bytes_per_tok) {
         const uint32_t* s32 =
             reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(src) + v * bytes_per_tok);
@@ -597,8 +722,10 @@ __global__ void __launch_bounds__(kThreadsMma, 4) decode_mma_kernel(const __grid
         for (int nb = 0; nb < NB; ++nb) {
           const float lm0 = dl[mb][nb][0] + dl[mb][nb][1], lm1 = dl[mb][nb][2] + dl[mb][nb][3];
           const float sg0 = ds[mb][nb][0] + ds[mb][nb][1], sg1 = ds[mb][nb][2] + ds[mb][nb][3];
-          lg[nb][0] = ng0.x * fmaf(ng0.y, fmaf(k3[nb], sg0, -k4[nb]), fmaf(k2[nb], lm0, k1[nb]));
-          lg[nb][1] = ng1.x * fmaf(ng1.y, fmaf(k3[nb], sg1, -k4[nb]), fmaf(k2[nb], lm1, k1[nb]));
+          // logit constants of head c + 4 nb (after the operand words of the buffer)
+          const float4 kk = reinterpret_cast<const float4*>(bq + L::KS * NB * 32)[c + 4 * nb];
+          lg[nb][0] = ng0.x * fmaf(ng0.y, fmaf(kk.z, sg0, -kk.w), fmaf(kk.y, lm0, kk.x));
+          lg[nb][1] = ng1.x * fmaf(ng1.y, fmaf(kk.z, sg1, -kk.w), fmaf(kk.y, lm1, kk.x));
           if (nv < 16) {
             if (r >= nv) lg[nb][0] = -INFINITY;
             if (r + 8 >= nv) lg[nb][1] = -INFINITY;
@@ -609,7 +736,7 @@ __global__ void __launch_bounds__(kThreadsMma, 4) decode_mma_kernel(const __grid
           for (int nb = 0; nb < NB; ++nb) {
             const int h = c + 4 * nb;
             if (h < G) {
-              float* srow = a.scores + (size_t)(qrow0 + h) * a.max_len + (t0 + (int64_t)i * TILE + tb);
+              float* srow = a.scores + (size_t)(qrow0 + h) * a.max_len + (tok0 + tb);
               if (r < nv) srow[r] = lg[nb][0] * kLn2;
               if (r + 8 < nv) srow[r + 8] = lg[nb][1] * kLn2;
             }
@@ -737,179 +864,121 @@ __global__ void __launch_bounds__(kThreadsMma, 4) decode_mma_kernel(const __grid
       const int prev = atomicAdd(&arrive_s[i % NST], 1);
       if (prev == kWarpsMma - 1) {
         arrive_s[i % NST] = 0;
-        if (a.use_tma && i + NST < ntiles && tile_full(i + NST)) {
+        if (i + NST < ntl) {
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           issue(i + NST);
         }
       }
     }
   }
+  if (cur >= 0) finish_unit(cur);
 
   if (__syncthreads_or(failed)) {
-    // A bulk copy did not complete in time: flag it, then wait (bounded again) for
-    // every copy this CTA may still have in flight before its shared memory goes away.
+    // A copy did not complete in time: flag it, then wait (bounded again) for every
+    // copy this CTA may still have in flight before its shared memory goes away.
     if (failed && lane == 0) atomicOr(a.err, 1u);
     if (tid == 0) {
       // Phases of one mbarrier complete in order: waiting for the last batch issued
-      // into each stage covers every copy still in flight.
+      // into each stage (and operand buffer) covers every copy still in flight.
       for (int s = 0; s < NST; ++s)
         if (issued_s[s] > 0) mbar_wait(&bars[s], (uint32_t)((issued_s[s] - 1) & 1));
+      for (int s = 0; s < 2; ++s)
+        if (fissued_s[s] > 0) mbar_wait(&fbars[s], (uint32_t)((fissued_s[s] - 1) & 1));
     }
     __syncthreads();
-    return;
   }
+}
 
-  // ---- per-warp results -> CTA partial ---------------------------------------------
-  float* red = reinterpret_cast<float*>(stage_base);  // [warp][head][kPartPadMma + d]
+// ------------------------------------------------------------------ combine kernel
+
+struct CombineArgs {
+  const float* ws_part;
+  float* out;
+  int hq, hkv, G, s_max;
+  int64_t tiles_per_unit, total_tiles, n_ctas;
+};
+
+// One CTA per (unit, query head), one thread per coordinate: log-sum-exp merge of the
+// partials of the CTAs that shared the unit, launched as a programmatic dependent of
+// the decode grid.
+__global__ void __launch_bounds__(kD) combine_mma_kernel(const __grid_constant__ CombineArgs a) {
   constexpr int RS = kPartPadMma + kD;
-#pragma unroll
-  for (int nb = 0; nb < NB; ++nb) {
-    float l = l_run[nb];
-    l += __shfl_xor_sync(kFull, l, 4);
-    l += __shfl_xor_sync(kFull, l, 8);
-    l += __shfl_xor_sync(kFull, l, 16);
-    // lane (g, c), g < 4, holds sum_t p * min(t, g) for head c + 4 nb in dmin[0] + dmin[1]
-    const float own = dmin[nb][0] + dmin[nb][1];
-    float mt[4];
-#pragma unroll
-    for (int g = 0; g < 4; ++g) mt[g] = __shfl_sync(kFull, own, 4 * g + c);
-    float* mine = red + (warp * 8 + c + 4 * nb) * RS;
-    if (r == 0) {
-      mine[0] = m_run[nb];
-      mine[1] = l;
-    }
-#pragma unroll
-    for (int g = 0; g < 4; ++g)
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const float* d = dv[g][hf][nb];
-        if (VB == 2) {
-          const int j = 4 * (8 * g + r) + 2 * hf;  // code at mantissa bits 4hf (row r), 4hf + 2 (row r + 8)
-          mine[kPartPadMma + j] = (d[0] + d[1]) * ldexpf(1.f, 24 - 4 * hf) + mt[g];
-          mine[kPartPadMma + j + 1] = (d[2] + d[3]) * ldexpf(1.f, 22 - 4 * hf) + mt[g];
-        } else {
-          const int j = 2 * (16 * g + 8 * hf + r);  // low nibble (row r), high nibble (row r + 8)
-          mine[kPartPadMma + j] = (d[0] + d[1]) * 16777216.f + mt[g];
-          mine[kPartPadMma + j + 1] = (d[2] + d[3]) * 1048576.f + mt[g];
-        }
-      }
-  }
-  __syncthreads();
-  float* ws_base = a.ws_part + (size_t)unit * a.n_chunks * G * RS;
-  for (int idx = tid; idx < G * kD; idx += kThreadsMma) {
-    const int h = idx / kD, j = idx % kD;
-    float mx = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kWarpsMma; ++w) mx = fmaxf(mx, red[(w * 8 + h) * RS]);
-    float num = 0.f, den = 0.f;
-    if (mx != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < kWarpsMma; ++w) {
-        const float* pw = red + (w * 8 + h) * RS;
-        const float wt = pw[0] == -INFINITY ? 0.f : exp2f(pw[0] - mx);
-        num = fmaf(wt, pw[kPartPadMma + j], num);
-        den = fmaf(wt, pw[1], den);
-      }
-    }
-    float* part_out = ws_base + ((size_t)chunk * G + h) * RS;
-    part_out[kPartPadMma + j] = num;
-    if (j == 0) {
-      part_out[0] = mx;
-      part_out[1] = den;
-    }
-  }
+  __shared__ float w_s[kD];
+  __shared__ float red_s[2][kD / 32];
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int u = blockIdx.x / a.G, h = blockIdx.x - u * a.G;
+  const int64_t Tu = a.tiles_per_unit;
+  const int64_t first = tile_owner((int64_t)u * Tu, a.n_ctas, a.total_tiles);
+  const int n_part = (int)(tile_owner((int64_t)(u + 1) * Tu - 1, a.n_ctas, a.total_tiles) - first + 1);
+  const size_t pstride = (size_t)a.G * RS;  // partial p of head h at base + p * pstride
+  const float* base = a.ws_part + (size_t)u * a.s_max * pstride + (size_t)h * RS;
 
-  // ---- the last CTA of this (sequence, KV head) merges the chunk partials -----------
-  __threadfence();
+  float M = -INFINITY;
+  for (int p = tid; p < n_part; p += kD) M = fmaxf(M, base[p * pstride]);
+  M = warp_max(M);
+  if (lane == 0) red_s[0][warp] = M;
   __syncthreads();
-  if (tid == 0) {
-    const unsigned int prev = atomicAdd(&a.cnt[unit], 1u);
-    *last_s = (prev == (unsigned int)(a.n_chunks - 1)) ? 1 : 0;
-  }
-  __syncthreads();
-  if (*last_s) {
-    __threadfence();
-    // Chunk weights per head first (m, l of every chunk), then one independent
-    // weighted sum per output; the ring is free again and holds the weights.
-    const size_t cs = (size_t)G * RS;
-    const int nwt = a.n_chunks * 8;
-    float* wts = red;        // [n_chunks][8] chunk weights
-    float* hsum = red + nwt; // [8] running max per head, then [8] 1 / sum
-    const bool fits = (size_t)(nwt + 16) * 4 <= (size_t)L::RING;
-    __syncthreads();
-    if (fits) {
-      if (tid < 8) {
-        float mx = -INFINITY;
-        if (tid < G)
-          for (int ch = 0; ch < a.n_chunks; ++ch) mx = fmaxf(mx, __ldcg(ws_base + ch * cs + (size_t)tid * RS));
-        hsum[tid] = mx;
-      }
-      __syncthreads();
-      for (int idx = tid; idx < nwt; idx += kThreadsMma) {
-        const int ch = idx >> 3, h = idx & 7;
-        float wt = 0.f;
-        if (h < G) {
-          const float mc = __ldcg(ws_base + ch * cs + (size_t)h * RS);
-          wt = (mc == -INFINITY || hsum[h] == -INFINITY) ? 0.f : exp2f(mc - hsum[h]);
-        }
-        wts[idx] = wt;
-      }
-      __syncthreads();
-      if (tid < 8) {
-        float den = 0.f;
-        if (tid < G)
-          for (int ch = 0; ch < a.n_chunks; ++ch)
-            den = fmaf(wts[ch * 8 + tid], __ldcg(ws_base + ch * cs + (size_t)tid * RS + 1), den);
-        hsum[8 + tid] = den > 0.f ? 1.f / den : 0.f;
-      }
-      __syncthreads();
-      for (int idx = tid; idx < G * kD; idx += kThreadsMma) {
-        const int h = idx / kD, j = idx % kD;
-        const float* base = ws_base + (size_t)h * RS + kPartPadMma + j;
-        float num0 = 0.f, num1 = 0.f, num2 = 0.f, num3 = 0.f;
-        int ch = 0;
-        for (; ch + 4 <= a.n_chunks; ch += 4) {
-          num0 = fmaf(wts[(ch + 0) * 8 + h], __ldcg(base + (ch + 0) * cs), num0);
-          num1 = fmaf(wts[(ch + 1) * 8 + h], __ldcg(base + (ch + 1) * cs), num1);
-          num2 = fmaf(wts[(ch + 2) * 8 + h], __ldcg(base + (ch + 2) * cs), num2);
-          num3 = fmaf(wts[(ch + 3) * 8 + h], __ldcg(base + (ch + 3) * cs), num3);
-        }
-        for (; ch < a.n_chunks; ++ch) num0 = fmaf(wts[ch * 8 + h], __ldcg(base + ch * cs), num0);
-        a.out[(size_t)(qrow0 + h) * kD + j] = ((num0 + num1) + (num2 + num3)) * hsum[8 + h];
-      }
-    } else {
-      for (int idx = tid; idx < G * kD; idx += kThreadsMma) {
-        const int h = idx / kD, j = idx % kD;
-        const float* base = ws_base + (size_t)h * RS;
-        float mx = -INFINITY;
-        for (int ch = 0; ch < a.n_chunks; ++ch) mx = fmaxf(mx, __ldcg(base + ch * cs));
-        float num = 0.f, den = 0.f;
-        if (mx != -INFINITY) {
-          for (int ch = 0; ch < a.n_chunks; ++ch) {
-            const float* pp = base + ch * cs;
-            const float mc = __ldcg(pp);
-            const float wt = mc == -INFINITY ? 0.f : exp2f(mc - mx);
-            den = fmaf(wt, __ldcg(pp + 1), den);
-            num = fmaf(wt, __ldcg(pp + kPartPadMma + j), num);
-          }
-        }
-        a.out[(size_t)(qrow0 + h) * kD + j] = den > 0.f ? num / den : 0.f;
-      }
+  M = fmaxf(fmaxf(red_s[0][0], red_s[0][1]), fmaxf(red_s[0][2], red_s[0][3]));
+  float den = 0.f, num0 = 0.f, num1 = 0.f;
+  for (int p0 = 0; p0 < n_part; p0 += kD) {
+    const int p = p0 + tid;
+    float w = 0.f;
+    if (p < n_part) {
+      const float mp = base[p * pstride];
+      w = mp == -INFINITY ? 0.f : exp2f(mp - M);
+      den = fmaf(w, base[p * pstride + 1], den);
     }
-    if (tid == 0) a.cnt[unit] = 0u;
+    __syncthreads();  // the previous chunk's weights are consumed
+    w_s[tid] = w;
+    __syncthreads();
+    const int np = min(kD, n_part - p0);
+    const float* acc = base + (size_t)p0 * pstride + kPartPadMma + tid;
+    int q = 0;
+    for (; q + 2 <= np; q += 2) {
+      num0 = fmaf(w_s[q], acc[q * pstride], num0);
+      num1 = fmaf(w_s[q + 1], acc[(q + 1) * pstride], num1);
+    }
+    if (q < np) num0 = fmaf(w_s[q], acc[q * pstride], num0);
   }
+  den = warp_sum(den);
+  if (lane == 0) red_s[1][warp] = den;
+  __syncthreads();
+  den = (red_s[1][0] + red_s[1][1]) + (red_s[1][2] + red_s[1][3]);
+  const int b = u / a.hkv, kvh = u - b * a.hkv;
+  a.out[(size_t)(b * a.hq + kvh * a.G + h) * kD + tid] = den > 0.f ? (num0 + num1) / den : 0.f;
+}
+
+template <int LMB, int VB, int NB>
+cudaError_t configure_mma_t() {
+  using L = Layout<LMB, VB, NB>;
+  static cudaError_t status = cudaFuncSetAttribute(decode_mma_kernel<LMB, VB, NB>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::SMEM);
+  return status;
+}
+
+template <int LMB, int VB, int NB>
+int ctas_per_sm_t() {
+  using L = Layout<LMB, VB, NB>;
+  static int n = [] {
+    int blocks = 0;
+    if (configure_mma_t<LMB, VB, NB>() != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, decode_mma_kernel<LMB, VB, NB>, kThreadsMma,
+                                                      L::SMEM) != cudaSuccess ||
+        blocks < 1) {
+      cudaGetLastError();
+      blocks = 1;
+    }
+    return blocks;
+  }();
+  return n;
 }
 
 template <int LMB, int VB, int NB>
 cudaError_t launch_mma_t(const MmaArgs& a, dim3 grid, cudaStream_t s) {
   using L = Layout<LMB, VB, NB>;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<LMB, VB, NB>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::SMEM);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  cudaError_t e = configure_mma_t<LMB, VB, NB>();
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(kThreadsMma);
@@ -943,6 +1012,16 @@ bool mma_decode_supported(const tq_ctx* ctx, int G) {
   return sh.v_bits == 2 || sh.v_bits == 4;
 }
 
+int mma_ctas_per_sm(int lm_bits, int v_bits, int G) {
+  const int nb = n_blocks(G);
+  if (lm_bits == 1) {
+    if (v_bits == 2) return nb == 1 ? ctas_per_sm_t<1, 2, 1>() : ctas_per_sm_t<1, 2, 2>();
+    return nb == 1 ? ctas_per_sm_t<1, 4, 1>() : ctas_per_sm_t<1, 4, 2>();
+  }
+  if (v_bits == 2) return nb == 1 ? ctas_per_sm_t<2, 2, 1>() : ctas_per_sm_t<2, 2, 2>();
+  return nb == 1 ? ctas_per_sm_t<2, 4, 1>() : ctas_per_sm_t<2, 4, 2>();
+}
+
 size_t mma_frag_bytes(int lm_bits, int G) { return (size_t)frag_words(lm_bits, n_blocks(G)) * 4; }
 
 int mma_tile_tokens(int G) { return tile_tokens(n_blocks(G)); }
@@ -955,10 +1034,9 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
   char* ws = static_cast<char*>(workspace);
   uint32_t* frag = reinterpret_cast<uint32_t*>(ws + plan.off_frag);
   float* part = reinterpret_cast<float*>(ws + plan.off_part);
-  unsigned int* cnt = reinterpret_cast<unsigned int*>(ws + plan.off_cnt);
   const int G = hq / hkv, lmb = ctx->shape.lm_bits, vb = ctx->shape.v_bits, nb = n_blocks(G);
   const float* cc = ctx->cb.c;
-  if (plan.chunk_len % tile_tokens(nb) != 0) return cudaErrorInvalidValue;
+  if (plan.n_ctas < 1 || plan.tiles_per_unit < 1) return cudaErrorInvalidValue;
 
   PrepArgs pa;
   pa.q = q;
@@ -973,9 +1051,10 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
   pa.cb = ctx->cb;
   pa.beta0 = cc[1] - cc[0];
   pa.beta1 = lmb > 1 ? cc[2] - cc[0] : 0.f;
+  pa.c0 = cc[0];
+  pa.sl2 = scale * 1.4426950408889634f;
   pa.nb = nb;
   pa.frag = frag;
-  pa.cnt = cnt;
   const size_t prep_smem = sizeof(float) * kD * kM;
   static bool prep_configured = false;
   if (!prep_configured) {
@@ -1004,24 +1083,44 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
   a.hq = hq;
   a.hkv = hkv;
   a.G = G;
-  a.n_chunks = plan.n_chunks;
-  a.chunk_len = plan.chunk_len;
-  a.scale = scale;
+  a.tiles_per_unit = plan.tiles_per_unit;
+  a.total_tiles = plan.total_tiles;
+  a.s_max = plan.s_max;
   a.scores = scores;
   a.out = out;
   a.ws_part = part;
-  a.cnt = cnt;
-  a.c0 = cc[0];
   a.use_tma = (max_len % 4 == 0) ? 1 : 0;
   a.err = ctx->d_err;
-  const dim3 grid(plan.n_chunks, batch * hkv);
+  const dim3 grid((unsigned)plan.n_ctas);
   if (ctx->prof_start) cudaEventRecord(ctx->prof_start, stream);
   if (lmb == 1)
     e = vb == 2 ? launch_mma_nb<1, 2>(a, nb, grid, stream) : launch_mma_nb<1, 4>(a, nb, grid, stream);
   else
     e = vb == 2 ? launch_mma_nb<2, 2>(a, nb, grid, stream) : launch_mma_nb<2, 4>(a, nb, grid, stream);
   if (ctx->prof_stop) cudaEventRecord(ctx->prof_stop, stream);
-  return e;
+  if (e != cudaSuccess) return e;
+
+  CombineArgs ca;
+  ca.ws_part = part;
+  ca.out = out;
+  ca.hq = hq;
+  ca.hkv = hkv;
+  ca.G = G;
+  ca.s_max = plan.s_max;
+  ca.tiles_per_unit = plan.tiles_per_unit;
+  ca.total_tiles = plan.total_tiles;
+  ca.n_ctas = plan.n_ctas;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((int64_t)batch * hkv * G));
+  cfg.blockDim = dim3(kD);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, combine_mma_kernel, ca);
 }
 
 }  // namespace tq

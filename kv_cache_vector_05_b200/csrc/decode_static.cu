@@ -18,10 +18,10 @@
 namespace {
 
 // Fixed scratch, one copy per device that loads the library, held until the
-// process exits. 8 MiB covers, e.g., 72 (sequence, KV head) pairs x 8192 tokens
-// x 16 query heads at d = 128 (about 3.3 MB) or 256 pairs x 32768 tokens x 32
-// query heads (about 2.7 MB).
-constexpr size_t kStaticScratchBytes = size_t(8) << 20;
+// process exits. 32 MiB covers, e.g., 72 (sequence, KV head) pairs x 8192 tokens
+// x 16 query heads at d = 128 (about 13 MB) or 256 pairs x 32768 tokens x 32
+// query heads (about 10 MB).
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;
 static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
 
 constexpr int kMaxDevices = 64;

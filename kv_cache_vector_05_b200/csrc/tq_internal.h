@@ -62,6 +62,10 @@ struct DecodePlan {
   size_t ws_q_bytes;     // generic path: prepared queries
   size_t ws_part_bytes;  // partial (m, l, acc) per chunk and query head
   size_t off_frag, off_part, off_cnt;  // tensor-core path: byte offsets in the workspace
+  // tensor-core path: the units' tiles are split evenly over n_ctas resident CTAs
+  int n_ctas;
+  int64_t tiles_per_unit, total_tiles;
+  int s_max;         // most CTAs that share one unit (partial slots per unit)
   size_t total_bytes;
 };
 
@@ -77,6 +81,7 @@ bool mma_decode_supported(const tq_ctx* ctx, int G);
 
 size_t mma_frag_bytes(int lm_bits, int G);  // query operand bytes per (sequence, KV head)
 int mma_tile_tokens(int G);                  // tokens per tile of the tensor-core decode
+int mma_ctas_per_sm(int lm_bits, int v_bits, int G);  // resident CTAs per SM of the tensor-core decode
 bool pack_qjl_operand(const float* S, int m, int d, uint16_t* out);
 
 cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const void* q, int q_dtype, int batch,

@@ -187,6 +187,18 @@ def test_decode_parity_random_cache(d, lm_bits, v_bits, G):
     _decode_check(d, lm_bits, v_bits, batch=2, hkv=2, G=G, max_len=1100, lens=[1100, 577])
 
 
+@pytest.mark.parametrize("G", [4, 8])
+def test_decode_ragged_sequences_many_tiles_per_cta(G):
+    """Ragged sequence lengths with several tiles per CTA: the work split hands a CTA a
+    range that runs from the ragged end of one (sequence, KV head) into the next one
+    and wraps around its whole ring of stages, so plain-copied and bulk-copied tiles
+    alternate in the same stage."""
+    batch, hkv, max_len = 6, 8, 10240
+    lens = [max_len - 37, max_len, max_len - 511, max_len - 1, 7000, max_len - 300]
+    _decode_check(128, 2, 2, batch=batch, hkv=hkv, G=G, max_len=max_len, lens=lens,
+                  units=list(range(0, batch * hkv, 3)) + [batch * hkv - 1])
+
+
 def test_decode_parity_haar_bf16_queries_custom_scale():
     _decode_check(128, 2, 2, batch=1, hkv=3, G=4, max_len=700, lens=[699], rotation="haar",
                   q_dtype="bf16", scale=0.05)

@@ -69,7 +69,7 @@ def test_static_scratch_matches_workspace_path_twice(d, lm_bits, v_bits, G):
 def test_static_scratch_rejects_oversized_shape():
     ctx = make_ctx(T, 128, 2, 2)
     cap = T.tq_decode_static_scratch_capacity()
-    batch, hq, hkv, max_len = 512, 64, 8, 1 << 15            # workspace far above 8 MiB
+    batch, hq, hkv, max_len = 512, 64, 8, 1 << 15            # workspace far above 32 MiB
     assert T.tq_decode_workspace_bytes(ctx, batch, hq, hkv, max_len) > cap
     q = torch.zeros((batch, hq, 128), device=DEV)
     dummy = torch.zeros(16, dtype=torch.uint8, device=DEV)
