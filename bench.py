@@ -60,6 +60,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--decode-only", action="store_true",
+                    help="decode a random packed cache of the workload's size (no bf16 inputs, no "
+                         "compression, no e2e): a small process for profiler captures")
     return ap.parse_args()
 
 
@@ -276,9 +279,14 @@ def run_ours(args, w: W.Workload):
     c, t = T.tq_lloyd_max_codebook(w.d, w.lm_bits)
     ctx = T.tq_codebook_load(w.d, w.lm_bits, w.v_bits, c, t, dr["qjl_S"], hadamard_signs=dr["hadamard_signs"])
     n_vec = w.units * w.tokens
-    Kh, Vh, Qh = host_inputs(w, rank)
+    if args.decode_only:
+        args.no_e2e = args.no_cpu_baseline = True
+    Kh, Vh, Qh = host_inputs(w, rank) if not args.decode_only else (None, None, W.queries(
+        (w.batch, w.hq, w.d), seed=7 + rank, dtype=w.dtype))
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
-    if Kh is not None:
+    if args.decode_only:
+        K = V = None
+    elif Kh is not None:
         K = torch.from_numpy(Kh).to(dev).to(tdt)
         V = torch.from_numpy(Vh).to(dev).to(tdt)
         del Kh, Vh
@@ -286,7 +294,14 @@ def run_ours(args, w: W.Workload):
         K = W.device_normal((n_vec, w.d), seed=1000 + rank, device=dev).to(tdt)
         V = W.device_normal((n_vec, w.d), seed=2000 + rank, device=dev).to(tdt)
     Q = torch.from_numpy(Qh).to(dev).to(tdt)
-    packed = {
+    if args.decode_only:
+        pk = W.random_packed_cache(n_vec, w.d, w.lm_bits, w.m, w.v_bits, seed=11 + rank)
+        packed = {k: torch.from_numpy(np.ascontiguousarray(v).view(np.int16) if v.dtype == np.uint16
+                                      else np.ascontiguousarray(v)).to(dev) for k, v in pk.items()}
+        del pk
+    else:
+        packed = None
+    packed = packed or {
         "k_codes": torch.empty((n_vec, w.lm_bits * w.d // 8), dtype=torch.uint8, device=dev),
         "k_signs": torch.empty((n_vec, w.m // 8), dtype=torch.uint8, device=dev),
         "k_norms": torch.empty((n_vec, 2), dtype=torch.int16, device=dev),
@@ -309,7 +324,8 @@ def run_ours(args, w: W.Workload):
     in_bytes = 2 * n_vec * w.d * (2 if w.dtype == "bf16" else 4)
 
     def compress():
-        T.tq_compress_kv(ctx, K, V, **packed)
+        if not args.decode_only:
+            T.tq_compress_kv(ctx, K, V, **packed)
 
     def decode():
         T.tq_decode_attention(ctx, Q, packed, w.batch, w.hq, w.hkv, w.tokens, out=out, workspace=ws)
@@ -372,7 +388,7 @@ def run_ours(args, w: W.Workload):
     comp_total = max_over_ranks(sum(comp) / 1e3)
     dec_k_mean = max_over_ranks(statistics.fmean(dec_k) / 1e3)
     gbs = world * packed_bytes * args.steps / dec_total / 1e9
-    vps = world * 2 * n_vec * args.steps / comp_total
+    vps = world * 2 * n_vec * args.steps / comp_total if not args.decode_only else None
 
     # --- end to end through the public API with host buffers
     e2e = None
@@ -408,7 +424,7 @@ def run_ours(args, w: W.Workload):
                "ms_per_step": 1e3 * e2e_s / args.e2e_steps}
 
     # our kernels per step: compress (1) + decode (query prep + attention + combine)
-    launches_per_step = 1 + 3
+    launches_per_step = (0 if args.decode_only else 1) + 3
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -435,9 +451,10 @@ def run_ours(args, w: W.Workload):
                        "l2": "flushed before each timed phase: 256 MiB write, then 256 MiB read",
                        "parallelism": f"dp{world} (independent replicas)"},
             "pct_of_hbm_peak": 100.0 * gbs / peak,
-            "compress": {"value": vps, "unit": "vectors/s (keys + values)",
-                         "gbs": world * (in_bytes + packed_bytes) * args.steps / comp_total / 1e9,
-                         "kernel_ms": statistics.fmean(comp_k)},
+            "compress": None if args.decode_only else {
+                "value": vps, "unit": "vectors/s (keys + values)",
+                "gbs": world * (in_bytes + packed_bytes) * args.steps / comp_total / 1e9,
+                "kernel_ms": statistics.fmean(comp_k)},
             "decode_ms": {"call": dec_total * 1e3 / args.steps, "main_kernel": dec_k_mean * 1e3,
                           "main_kernel_timing": "separate loop of `steps` steps with events around the kernel"},
             "roofline": {"kernel": "decode_mma_kernel", "bound": "hbm", "achieved": achieved, "peak": peak,

@@ -390,6 +390,337 @@ cudaError_t launch_tc(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) 
   return vb == 2 ? launch_tc_t<T, 3, 2>(ctx, a, s) : launch_tc_t<T, 3, 4>(ctx, a, s);
 }
 
+
+// ---------------------------------------------------------------------------------
+// Fast path (d = m = 128, randomized Hadamard rotation, S exact in f16): four lanes
+// per vector, lane q of a vector holding coordinates [32q, 32q + 32). Norm, sign flip,
+// the first five Walsh-Hadamard stages, bucketize, residual and code packing are
+// lane-local; the last two butterfly stages and the two norms take two shuffles
+// each. A value's group of 32 coordinates is one lane, so min / max and its codes
+// need no shuffles at all. 512 threads handle 128 vectors at a time: the 128
+// residuals (x16, f16 hi + lo) go to two swizzled shared-memory tiles, one thread
+// issues the 128 x 128 x 128 QJL projection on the tensor cores (as in
+// compress_tc_kernel), the values are quantized while it runs, and one thread per key
+// reads its 128 projections back from tensor memory and packs the sign bits.
+constexpr int kQ4Rows = 128;
+constexpr int kQ4Threads = 4 * kQ4Rows;
+
+struct Q4Smem {
+  static constexpr uint32_t A_HI = 0, A_LO = kTcTileBytes, S = 2 * kTcTileBytes;
+  static constexpr uint32_t ZF = 3 * kTcTileBytes;  // [128] nonzero-key flags
+  static constexpr uint32_t BAR = ZF + 128;         // mbarrier
+  static constexpr uint32_t TMEM = BAR + 8;         // TMEM base address
+  static constexpr uint32_t BYTES = TMEM + 8;
+};
+
+// 32 consecutive elements (64 or 128 bytes, 16-byte aligned) as fp32.
+template <typename T>
+__device__ __forceinline__ void load32(const T* __restrict__ p, float (&x)[32]) {
+  if constexpr (sizeof(T) == 2) {
+    const uint4* p4 = reinterpret_cast<const uint4*>(p);
+    uint4 u[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) u[k] = __ldg(p4 + k);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t w[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        x[8 * k + 2 * h] = __uint_as_float(w[h] << 16);
+        x[8 * k + 2 * h + 1] = __uint_as_float(w[h] & 0xffff0000u);
+      }
+    }
+  } else {
+    const float4* p4 = reinterpret_cast<const float4*>(p);
+    float4 f[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) f[k] = __ldg(p4 + k);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      x[4 * k] = f[k].x;
+      x[4 * k + 1] = f[k].y;
+      x[4 * k + 2] = f[k].z;
+      x[4 * k + 3] = f[k].w;
+    }
+  }
+}
+
+// Unnormalised Sylvester Walsh-Hadamard transform of 32 values held by one thread.
+__device__ __forceinline__ void fwht32(float (&x)[32]) {
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      if ((e & h) == 0) {
+        const float u = x[e], w = x[e + h];
+        x[e] = u + w;
+        x[e + h] = u - w;
+      }
+    }
+  }
+}
+
+// OR `v` (NB bits) into a little-endian stream of 32-bit words at bit `o` (o and
+// NB compile-time after unrolling).
+template <int NB, int NW>
+__device__ __forceinline__ void put_bits(uint32_t (&w)[NW], int o, uint32_t v) {
+  const int wi = o >> 5, sh = o & 31;
+  w[wi] += v << sh;  // the bits are still zero: add == or
+  if (sh + NB > 32) w[wi + 1] += v >> (32 - sh);
+}
+
+template <typename T, int LMB, int VB>
+__global__ void __launch_bounds__(kQ4Threads, 1) compress_q4_kernel(const __grid_constant__ CompressArgs a) {
+  namespace s1 = tq::sm100;
+  constexpr int KW = LMB;  // code words per lane (32 codes x LMB bits)
+  constexpr int VW = VB;   // value code words per lane
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = s1::smem_u32(sm);
+  uint8_t* zf = sm + Q4Smem::ZF;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Q4Smem::BAR);
+  uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + Q4Smem::TMEM);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int R = tid >> 2, q = tid & 3;  // vector row within the pass, quarter of the vector
+
+  if (warp == 0) {
+    s1::tmem_alloc(tmem_s, 128);
+    s1::tmem_relinquish();
+  }
+  if (tid == 0) {
+    s1::mbar_init(bar, 1);
+    s1::mbar_init_fence();
+  }
+  if (a.k) {  // S operand tile, prepacked on the host
+    const uint4* src = reinterpret_cast<const uint4*>(a.S_sw128);
+    uint4* dst = reinterpret_cast<uint4*>(sm + Q4Smem::S);
+    for (int w = tid; w < (int)(kTcTileBytes / 16); w += kQ4Threads) dst[w] = src[w];
+  }
+  s1::fence_async_smem();
+  s1::fence_before_sync();
+  __syncthreads();
+  s1::fence_after_sync();
+  const uint32_t tmem = *tmem_s;
+  constexpr uint32_t idesc = s1::idesc_f16_f32(128, 128);
+
+  const uint32_t sbits = a.cb.sign_bits[q];   // Hadamard signs of this lane's coordinates
+  const float up1 = (q & 1) ? -1.f : 1.f;     // butterfly across lanes q ^ 1 (stride 32)
+  const float up2 = (q & 2) ? -1.f : 1.f;     // and across lanes q ^ 2 (stride 64)
+  float cb_t[(1 << LMB) - 1], cb_c[1 << LMB];
+#pragma unroll
+  for (int k = 0; k < (1 << LMB) - 1; ++k) cb_t[k] = a.cb.t[k];
+#pragma unroll
+  for (int k = 0; k < (1 << LMB); ++k) cb_c[k] = a.cb.c[k];
+
+  uint32_t phase = 0;
+  bool failed = false;
+  const int64_t ntile = (a.n_vec + kQ4Rows - 1) / kQ4Rows;
+  for (int64_t tile = blockIdx.x; tile < ntile; tile += gridDim.x) {
+    const int64_t i = tile * kQ4Rows + R;
+    const bool valid = i < a.n_vec;
+
+    // ---------------------------------------------------------------- keys
+    if (a.k) {
+      float x[32];
+      if (valid) {
+        load32<T>(static_cast<const T*>(a.k) + i * 128 + 32 * q, x);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[e] = 0.f;
+      }
+      float ss = 0.f;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) ss = fmaf(x[e], x[e], ss);
+      ss += __shfl_xor_sync(kFull, ss, 1);
+      ss += __shfl_xor_sync(kFull, ss, 2);
+      const float n = sqrtf(ss);
+      const bool nz = n > 0.f;
+      // y = H diag(sigma) (k / n) / sqrt(d): sign flip, butterflies, one scale at the end
+#pragma unroll
+      for (int e = 0; e < 32; ++e) x[e] = flip_sign(x[e], (sbits >> e) & 1u);
+      fwht32(x);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) x[e] = fmaf(up1, x[e], __shfl_xor_sync(kFull, x[e], 1));
+#pragma unroll
+      for (int e = 0; e < 32; ++e) x[e] = fmaf(up2, x[e], __shfl_xor_sync(kFull, x[e], 2));
+      const float sc = nz ? (1.0f / n) * a.inv_sqrt_d : 0.f;
+      // Lloyd-Max bucketize: code = #{k : y >= t_k}; residual against its centroid.
+      uint32_t cw[KW];
+#pragma unroll
+      for (int w = 0; w < KW; ++w) cw[w] = 0u;
+      float rr = 0.f;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float y = x[e] * sc;
+        uint32_t idx = 0;
+        float cv = cb_c[0];
+#pragma unroll
+        for (int k = 0; k < (1 << LMB) - 1; ++k) {
+          if (y >= cb_t[k]) {
+            idx = k + 1;
+            cv = cb_c[k + 1];
+          }
+        }
+        put_bits<LMB, KW>(cw, LMB * e, idx);
+        x[e] = y - cv;
+        rr = fmaf(x[e], x[e], rr);
+      }
+      rr += __shfl_xor_sync(kFull, rr, 1);
+      rr += __shfl_xor_sync(kFull, rr, 2);
+      const float gamma = sqrtf(rr);
+      if (valid) {
+        uint32_t* co = reinterpret_cast<uint32_t*>(a.k_codes + i * (LMB * 16) + q * (LMB * 4));
+#pragma unroll
+        for (int w = 0; w < KW; ++w) co[w] = nz ? cw[w] : 0u;
+        if (q == 0) {
+          const uint32_t nb = __half_as_ushort(__float2half_rn(n));
+          const uint32_t gb = __half_as_ushort(__float2half_rn(gamma));
+          reinterpret_cast<uint32_t*>(a.k_norms)[i] = nz ? (nb | (gb << 16)) : 0u;
+        }
+      }
+      // Residual x16 (signs unchanged) as f16 hi + lo into the operand tiles (the
+      // previous pass's projection is complete: every thread waited for it).
+      const bool use = valid && nz;
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8) {  // 8 coordinates = one 16-byte chunk of each tile
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const float f0 = use ? 16.f * x[8 * c8 + 2 * p] : 0.f, f1 = use ? 16.f * x[8 * c8 + 2 * p + 1] : 0.f;
+          const __half2 h = __floats2half2_rn(f0, f1);
+          const float2 hf = __half22float2(h);
+          const __half2 l = __floats2half2_rn(f0 - hf.x, f1 - hf.y);
+          hw[p] = *reinterpret_cast<const uint32_t*>(&h);
+          lw[p] = *reinterpret_cast<const uint32_t*>(&l);
+        }
+        const uint32_t off = s1::sw128_offset(R, 32 * q + 8 * c8, kQ4Rows);
+        *reinterpret_cast<uint4*>(sm + Q4Smem::A_HI + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(sm + Q4Smem::A_LO + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      }
+      if (q == 0) zf[R] = use ? 1 : 0;
+      s1::fence_async_smem();
+      s1::fence_before_sync();
+      __syncthreads();
+      s1::fence_after_sync();
+      if (tid == 0) {
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          s1::umma_f16(tmem, s1::sw128_desc(sbase + Q4Smem::A_HI, 16 * ks, kQ4Rows),
+                       s1::sw128_desc(sbase + Q4Smem::S, 16 * ks, 128), idesc, ks > 0 ? 1u : 0u);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          s1::umma_f16(tmem, s1::sw128_desc(sbase + Q4Smem::A_LO, 16 * ks, kQ4Rows),
+                       s1::sw128_desc(sbase + Q4Smem::S, 16 * ks, 128), idesc, 1u);
+        s1::umma_commit(bar);
+      }
+    }
+
+    // ---------------------------------------------------------------- values
+    if (a.v && valid) {
+      float x[32];
+      load32<T>(static_cast<const T*>(a.v) + i * 128 + 32 * q, x);
+      float lo = x[0], hi = x[0];
+#pragma unroll
+      for (int e = 1; e < 32; ++e) {
+        lo = fminf(lo, x[e]);
+        hi = fmaxf(hi, x[e]);
+      }
+      constexpr int levels = (1 << VB) - 1;
+      // scale in fp64 as the reference quantizer; codes in fp32, redone in fp64 when
+      // (v - min) / scale lies within 1e-5 of a half step.
+      const double dlo = lo, span = (double)hi - dlo;
+      const float inv = span > 0.0 ? (float)(levels / span) : 0.f;
+      uint32_t vw[VW];
+#pragma unroll
+      for (int w = 0; w < VW; ++w) vw[w] = 0u;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float t = (x[e] - lo) * inv;
+        float qv = floorf(t + 0.5f);
+        if (fabsf(t - floorf(t) - 0.5f) < 1e-5f) qv = (float)floor(((double)x[e] - dlo) * (levels / span) + 0.5);
+        qv = fminf(fmaxf(qv, 0.f), (float)levels);
+        put_bits<VB, VW>(vw, VB * e, (uint32_t)qv);
+      }
+      uint32_t* vo = reinterpret_cast<uint32_t*>(a.v_codes + i * (VB * 16) + q * (VB * 4));
+#pragma unroll
+      for (int w = 0; w < VW; ++w) vo[w] = vw[w];
+      const uint32_t sb = __half_as_ushort(__double2half(span / levels));
+      const uint32_t mb = __half_as_ushort(__float2half_rn(lo));
+      reinterpret_cast<uint32_t*>(a.v_params)[i * 4 + q] = sb | (mb << 16);
+    }
+
+    // ---------------------------------------------------------------- QJL signs
+    if (a.k) {
+      const bool ok = s1::mbar_wait(bar, phase);
+      if (__syncthreads_or(!ok)) {
+        failed = true;
+        break;
+      }
+      phase ^= 1u;
+      s1::fence_after_sync();
+      if (warp < 4) {
+        // thread = key (TMEM lane 32 warp + lane); 4 x 32 projections -> 4 sign words
+        uint32_t words[4];
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint32_t v[32];
+          s1::tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + 32 * c4, v);
+          s1::tmem_ld_wait();
+          uint32_t bits = 0;
+#pragma unroll
+          for (int k = 31; k >= 0; --k) bits = __funnelshift_l(v[k] ^ 0x80000000u, bits, 1);
+          words[c4] = bits;
+        }
+        const int row = 32 * warp + lane;
+        const int64_t ik = tile * kQ4Rows + row;
+        if (ik < a.n_vec) {
+          const bool nzk = zf[row] != 0;
+          const uint4 w4 = nzk ? make_uint4(words[0], words[1], words[2], words[3]) : make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(a.k_signs + ik * 16) = w4;
+        }
+      }
+      s1::fence_before_sync();
+    }
+  }
+  if (failed && tid == 0) {
+    atomicOr(a.err, 1u);
+    s1::mbar_wait(bar, phase);  // bounded: let an abandoned MMA finish before TMEM is freed
+  }
+  s1::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    s1::fence_after_sync();
+    s1::tmem_dealloc(tmem, 128);
+  }
+}
+
+template <typename T, int LMB, int VB>
+cudaError_t launch_q4_t(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) {
+  static bool configured = false;
+  const size_t smem = Q4Smem::BYTES + 1024;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(compress_q4_kernel<T, LMB, VB>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  int64_t blocks = (a.n_vec + kQ4Rows - 1) / kQ4Rows;
+  if (blocks > ctx->num_sms) blocks = ctx->num_sms;
+  if (ctx->prof_start) cudaEventRecord(ctx->prof_start, s);
+  compress_q4_kernel<T, LMB, VB><<<(unsigned)blocks, kQ4Threads, smem, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (ctx->prof_stop) cudaEventRecord(ctx->prof_stop, s);
+  return e;
+}
+
+template <typename T>
+cudaError_t launch_q4(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) {
+  const int lmb = ctx->shape.lm_bits, vb = ctx->shape.v_bits;
+  if (lmb == 1) return vb == 2 ? launch_q4_t<T, 1, 2>(ctx, a, s) : launch_q4_t<T, 1, 4>(ctx, a, s);
+  if (lmb == 2) return vb == 2 ? launch_q4_t<T, 2, 2>(ctx, a, s) : launch_q4_t<T, 2, 4>(ctx, a, s);
+  return vb == 2 ? launch_q4_t<T, 3, 2>(ctx, a, s) : launch_q4_t<T, 3, 4>(ctx, a, s);
+}
+
 }  // namespace
 
 // S as f16 in the swizzled K-major operand layout of compress_tc_kernel, or false if
@@ -428,8 +759,11 @@ cudaError_t launch_compress(const tq_ctx* ctx, const void* k, const void* v, int
   a.inv_sqrt_d = (float)(1.0 / sqrt((double)ctx->shape.d));
   a.S_sw128 = ctx->S_sw128;
   a.err = ctx->d_err;
-  if (ctx->S_sw128 && ctx->shape.d == 128 && ctx->shape.m == 128)
+  if (ctx->S_sw128 && ctx->shape.d == 128 && ctx->shape.m == 128) {
+    if (ctx->shape.rot == TQ_ROT_HADAMARD)
+      return dtype == TQ_F32 ? launch_q4<float>(ctx, a, stream) : launch_q4<__nv_bfloat16>(ctx, a, stream);
     return dtype == TQ_F32 ? launch_tc<float>(ctx, a, stream) : launch_tc<__nv_bfloat16>(ctx, a, stream);
+  }
   switch (ctx->shape.d) {
     case 64: return launch_d<64>(ctx, a, dtype, stream);
     case 128: return launch_d<128>(ctx, a, dtype, stream);

@@ -118,7 +118,7 @@ __device__ __forceinline__ uint32_t pack_stream_word_t(uint32_t v, int lane) {
   uint32_t mine = 0;
 #pragma unroll
   for (int w = 0; w < NWORDS; ++w) {
-    const uint32_t c = (w == w0 ? lo : 0u) | ((32 % NBITS != 0 && w == w0 + 1) ? hi : 0u);
+    const uint32_t c = (w == w0 ? lo : 0u) | ((32 % (NBITS > 0 ? NBITS : 32) != 0 && w == w0 + 1) ? hi : 0u);
     const uint32_t word = __reduce_or_sync(kFull, c);
     if (lane == w) mine = word;
   }

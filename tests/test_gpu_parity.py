@@ -99,6 +99,11 @@ def test_compress_edge_cases():
     Pi, c, t, S = oracle_setup(128, 2)
     ok = O.compress_keys(one.cpu().numpy().astype(np.float64), Pi, c, t, S, with_diagnostics=True)
     assert_key_parity(compare_keys(g, ok, 128, 2, 128))
+    vals = torch.randn((300, 128), device=DEV).to(torch.bfloat16)   # values only, 3 passes
+    gv = to_np(T.tq_compress_kv(ctx, None, vals))
+    assert "k_codes" not in gv
+    ov = O.quantize_values(vals.float().cpu().numpy().astype(np.float64), 2, with_diagnostics=True)
+    assert_value_parity(compare_values(gv, ov, 128, 2))
     big = torch.randn((3, 129), device=DEV)
     misaligned = big.view(-1)[1:1 + 256].view(2, 128)       # 4-byte offset
     with pytest.raises(T.TQError):
