@@ -30,6 +30,7 @@ struct CompressArgs {
   const float* St;   // [d][m]
   const float* PiT;  // [d][d], Haar only
   const uint16_t* S_sw128;  // S as f16 in the swizzled K-major operand layout (tensor-core path)
+  const uint16_t* H_sw128;  // H diag(sigma) as bf16 in the same layout (tensor-core rotation)
   unsigned int* err;
   Codebook cb;
   int lm_bits, m, v_bits, rot;
@@ -748,6 +749,372 @@ cudaError_t launch_q4(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) 
   return vb == 2 ? launch_q4_t<T, 3, 2>(ctx, a, s) : launch_q4_t<T, 3, 4>(ctx, a, s);
 }
 
+
+// ---------------------------------------------------------------------------------
+// bf16 keys, randomized Hadamard rotation, d = m = 128: the rotation runs on the
+// tensor cores too. The keys are bf16 and H diag(sigma) is +-1, both exact in bf16, so
+// Y = K (H diag(sigma))^T is one bf16 x bf16 -> fp32 MMA per 128 keys with exact
+// products (fp32 sums, like the butterflies). As Pi = H diag(sigma) / sqrt(d) is
+// orthogonal, ||k|| = ||Y|| / sqrt(d) and y = Pi k / ||k|| = Y / ||Y||: the norm comes
+// out of Y as well. Eight key warps read Y back from tensor memory (a warp reaches
+// the 32 lanes of its sub-partition, so two warps share each row, one per half of
+// the columns), bucketize, pack the codes and stage the residual for the QJL MMA;
+// eight value warps quantize the 128 values meanwhile.
+constexpr int kRotThreads = 512;
+constexpr int kRotKeyThreads = 256;
+
+struct RotSmem {
+  static constexpr uint32_t KT = 0;                          // keys, bf16 operand tile
+  static constexpr uint32_t HB = kTcTileBytes;               // H diag(sigma), bf16 operand tile
+  static constexpr uint32_t A_HI = 2 * kTcTileBytes, A_LO = 3 * kTcTileBytes;  // residual x16, f16
+  static constexpr uint32_t S = 4 * kTcTileBytes;            // QJL matrix, f16 operand tile
+  static constexpr uint32_t KR = 5 * kTcTileBytes;           // next pass's keys, raw rows (bulk copy)
+  static constexpr uint32_t XS = 6 * kTcTileBytes;           // [2][128] fp32 half-row sums
+  static constexpr uint32_t ZF = XS + 2 * 128 * 4;           // [128] nonzero-key flags
+  static constexpr uint32_t BAR = ZF + 128;                  // three mbarriers
+  static constexpr uint32_t TMEM = BAR + 24;                 // TMEM base address
+  static constexpr uint32_t BYTES = TMEM + 8;
+};
+
+__device__ __forceinline__ void key_warps_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kRotKeyThreads) : "memory");
+}
+
+// Instruction descriptor, kind::f16 with bf16 operands, f32 accumulate, both K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+  return sm100::idesc_f16_f32(M, N) | (1u << 7) | (1u << 10);
+}
+
+template <int LMB, int VB>
+__global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __grid_constant__ CompressArgs a) {
+  namespace s1 = tq::sm100;
+  constexpr int KW = 2 * LMB;  // code words per key thread (64 codes x LMB bits)
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = s1::smem_u32(sm);
+  float* xs = reinterpret_cast<float*>(sm + RotSmem::XS);
+  uint8_t* zf = sm + RotSmem::ZF;
+  uint64_t* bar1 = reinterpret_cast<uint64_t*>(sm + RotSmem::BAR);  // rotation MMA done
+  uint64_t* bar2 = bar1 + 1;                                         // projection MMA done
+  uint64_t* bar3 = bar1 + 2;                                         // raw key rows landed
+  uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + RotSmem::TMEM);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool key_warp = warp < 8;
+  const int sp = warp & 3, ch = (warp >> 2) & 1;  // key warps: sub-partition, column half
+  const int R = 32 * sp + lane;                    // key warps: row = key within the pass
+
+  if (warp == 0) {
+    s1::tmem_alloc(tmem_s, 256);
+    s1::tmem_relinquish();
+  }
+  if (tid == 0) {
+    s1::mbar_init(bar1, 1);
+    s1::mbar_init(bar2, 1);
+    s1::mbar_init(bar3, 1);
+    s1::mbar_init_fence();
+  }
+  {  // H diag(sigma) and S operand tiles, prepacked on the host
+    const uint4* hsrc = reinterpret_cast<const uint4*>(a.H_sw128);
+    const uint4* ssrc = reinterpret_cast<const uint4*>(a.S_sw128);
+    uint4* hdst = reinterpret_cast<uint4*>(sm + RotSmem::HB);
+    uint4* sdst = reinterpret_cast<uint4*>(sm + RotSmem::S);
+    for (int w = tid; w < (int)(kTcTileBytes / 16); w += kRotThreads) {
+      hdst[w] = hsrc[w];
+      sdst[w] = ssrc[w];
+    }
+  }
+  s1::fence_async_smem();
+  s1::fence_before_sync();
+  __syncthreads();
+  s1::fence_after_sync();
+  const uint32_t tmem = *tmem_s;
+  const uint32_t tmem_y = tmem, tmem_p = tmem + 128;  // columns 0..127: Y, 128..255: S r
+  const uint32_t lane_base = (uint32_t)(32 * sp) << 16;
+  float cb_t[(1 << LMB) - 1], cb_c[1 << LMB];
+#pragma unroll
+  for (int k = 0; k < (1 << LMB) - 1; ++k) cb_t[k] = a.cb.t[k];
+#pragma unroll
+  for (int k = 0; k < (1 << LMB); ++k) cb_c[k] = a.cb.c[k];
+
+  uint32_t phase = 0;
+  bool failed = false;
+  const int64_t ntile = (a.n_vec + kQ4Rows - 1) / kQ4Rows;
+  // One thread: bring the raw rows of pass `tile` (contiguous in memory) into KR.
+  auto fetch_keys = [&](int64_t tile) {
+    const int64_t v0 = tile * kQ4Rows;
+    const uint32_t bytes = (uint32_t)(min((int64_t)kQ4Rows, a.n_vec - v0) * 256);
+    s1::mbar_expect_tx(bar3, bytes);
+    s1::bulk_g2s(sm + RotSmem::KR, static_cast<const __nv_bfloat16*>(a.k) + v0 * 128, bytes, bar3);
+  };
+  if (a.k && tid == 0 && blockIdx.x < ntile) fetch_keys(blockIdx.x);
+  for (int64_t tile = blockIdx.x; tile < ntile; tile += gridDim.x, phase ^= 1u) {
+    const int64_t v0 = tile * kQ4Rows;
+    // ---- stage the 128 keys: raw rows -> swizzled operand tile, once they landed and
+    // the previous pass's rotation MMA has finished reading the tile.
+    if (a.k && tile != blockIdx.x && !failed && !s1::mbar_wait(bar1, phase ^ 1u)) failed = true;
+    if (a.k && !failed && !s1::mbar_wait(bar3, phase)) failed = true;
+    if (__syncthreads_or(failed)) break;
+    if (a.k) {
+      const int nrows = (int)min((int64_t)kQ4Rows, a.n_vec - v0);
+      uint4 kv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int id = tid + kRotThreads * u, row = id >> 4;
+        kv[u] = row < nrows ? reinterpret_cast<const uint4*>(sm + RotSmem::KR)[id] : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int id = tid + kRotThreads * u, row = id >> 4, c16 = id & 15;
+        *reinterpret_cast<uint4*>(sm + RotSmem::KT + s1::sw128_offset(row, 8 * c16, kQ4Rows)) = kv[u];
+      }
+      s1::fence_async_smem();
+      s1::fence_before_sync();
+      __syncthreads();
+      s1::fence_after_sync();
+      if (tid == 0) {
+        constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          s1::umma_f16(tmem_y, s1::sw128_desc(sbase + RotSmem::KT, 16 * ks, kQ4Rows),
+                       s1::sw128_desc(sbase + RotSmem::HB, 16 * ks, 128), idesc, ks > 0 ? 1u : 0u);
+        s1::umma_commit(bar1);
+        // KR has been read by every thread (the barrier above): fetch the next pass.
+        if (tile + gridDim.x < ntile) {
+          s1::fence_async_smem();
+          fetch_keys(tile + gridDim.x);
+        }
+      }
+    }
+
+    if (key_warp && a.k) {
+      // ---------------------------------------------------------------- keys
+      const int64_t i = v0 + R;
+      const bool valid = i < a.n_vec;
+      if (!failed && !s1::mbar_wait(bar1, phase)) failed = true;
+      s1::fence_after_sync();
+      float y[64];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t v[32];
+        s1::tmem_ld32(tmem_y + lane_base + 64 * ch + 32 * h, v);
+        s1::tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) y[32 * h + k] = __uint_as_float(v[k]);
+      }
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int e = 0; e < 64; ++e) s4[e & 3] = fmaf(y[e], y[e], s4[e & 3]);
+      xs[ch * 128 + R] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+      key_warps_sync();
+      const float tot = xs[R] + xs[128 + R];  // ||Y||^2 = d ||k||^2
+      key_warps_sync();                      // both halves read before xs is reused
+      const bool nz = tot > 0.f;
+      const float sc = nz ? 1.0f / sqrtf(tot) : 0.f;
+      uint32_t cw[KW], cw2[KW];  // even / odd codes: two independent insert chains per word
+#pragma unroll
+      for (int w = 0; w < KW; ++w) cw[w] = cw2[w] = 0u;
+      float r4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int e = 0; e < 64; ++e) {
+        const float yy = y[e] * sc;
+        uint32_t idx = 0;
+        float cv = cb_c[0];
+#pragma unroll
+        for (int k = 0; k < (1 << LMB) - 1; ++k) {
+          if (yy >= cb_t[k]) {
+            idx = k + 1;
+            cv = cb_c[k + 1];
+          }
+        }
+        if (e & 1)
+          put_bits<LMB, KW>(cw2, LMB * e, idx);
+        else
+          put_bits<LMB, KW>(cw, LMB * e, idx);
+        y[e] = yy - cv;
+        r4[e & 3] = fmaf(y[e], y[e], r4[e & 3]);
+      }
+#pragma unroll
+      for (int w = 0; w < KW; ++w) cw[w] |= cw2[w];
+      xs[ch * 128 + R] = (r4[0] + r4[1]) + (r4[2] + r4[3]);
+      key_warps_sync();
+      const float gamma = sqrtf(xs[R] + xs[128 + R]);
+      if (valid) {
+        uint32_t* co = reinterpret_cast<uint32_t*>(a.k_codes + i * (LMB * 16) + ch * (LMB * 8));
+#pragma unroll
+        for (int w = 0; w < KW; ++w) co[w] = nz ? cw[w] : 0u;
+        if (ch == 0) {
+          const float n = sqrtf(tot * (1.0f / 128.f));
+          const uint32_t nb = __half_as_ushort(__float2half_rn(n));
+          const uint32_t gb = __half_as_ushort(__float2half_rn(gamma));
+          reinterpret_cast<uint32_t*>(a.k_norms)[i] = nz ? (nb | (gb << 16)) : 0u;
+        }
+      }
+      // residual x16 as f16 hi + lo (the previous projection finished: it was waited for)
+      const bool use = valid && nz;
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const float f0 = use ? 16.f * y[8 * c8 + 2 * p] : 0.f, f1 = use ? 16.f * y[8 * c8 + 2 * p + 1] : 0.f;
+          const __half2 hh = __floats2half2_rn(f0, f1);
+          const float2 hf = __half22float2(hh);
+          const __half2 ll = __floats2half2_rn(f0 - hf.x, f1 - hf.y);
+          hw[p] = *reinterpret_cast<const uint32_t*>(&hh);
+          lw[p] = *reinterpret_cast<const uint32_t*>(&ll);
+        }
+        const uint32_t off = s1::sw128_offset(R, 64 * ch + 8 * c8, kQ4Rows);
+        *reinterpret_cast<uint4*>(sm + RotSmem::A_HI + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(sm + RotSmem::A_LO + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      }
+      if (ch == 0) zf[R] = use ? 1 : 0;
+      s1::fence_async_smem();
+      s1::fence_before_sync();
+      key_warps_sync();
+      s1::fence_after_sync();
+      if (tid == 0) {
+        constexpr uint32_t idesc = s1::idesc_f16_f32(128, 128);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          s1::umma_f16(tmem_p, s1::sw128_desc(sbase + RotSmem::A_HI, 16 * ks, kQ4Rows),
+                       s1::sw128_desc(sbase + RotSmem::S, 16 * ks, 128), idesc, ks > 0 ? 1u : 0u);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          s1::umma_f16(tmem_p, s1::sw128_desc(sbase + RotSmem::A_LO, 16 * ks, kQ4Rows),
+                       s1::sw128_desc(sbase + RotSmem::S, 16 * ks, 128), idesc, 1u);
+        s1::umma_commit(bar2);
+      }
+      // ---- QJL signs of this thread's 64 projections
+      if (!failed && !s1::mbar_wait(bar2, phase)) failed = true;
+      s1::fence_after_sync();
+      uint32_t words[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t v[32];
+        s1::tmem_ld32(tmem_p + lane_base + 64 * ch + 32 * h, v);
+        s1::tmem_ld_wait();
+        uint32_t b4[4] = {0u, 0u, 0u, 0u};  // four independent 8-bit chains
+#pragma unroll
+        for (int k = 7; k >= 0; --k)
+#pragma unroll
+          for (int g = 0; g < 4; ++g) b4[g] = __funnelshift_l(v[8 * g + k] ^ 0x80000000u, b4[g], 1);
+        words[h] = b4[0] | (b4[1] << 8) | (b4[2] << 16) | (b4[3] << 24);
+      }
+      if (valid) {
+        const uint2 w2 = zf[R] ? make_uint2(words[0], words[1]) : make_uint2(0u, 0u);
+        *reinterpret_cast<uint2*>(a.k_signs + i * 16 + 8 * ch) = w2;
+      }
+      s1::fence_before_sync();
+    } else if (!key_warp && a.v) {
+      // ---------------------------------------------------------------- values
+      const int vt = tid - kRotKeyThreads, q = vt & 3;
+      uint4 raw[2][4];  // both rounds' loads in flight before either is worked on
+#pragma unroll
+      for (int round = 0; round < 2; ++round) {
+        const int64_t i = v0 + (vt >> 2) + 64 * round;
+        if (i < a.n_vec) {
+          const uint4* p4 = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.v) + i * 128 + 32 * q);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) raw[round][k] = __ldg(p4 + k);
+        }
+      }
+#pragma unroll
+      for (int round = 0; round < 2; ++round) {
+        const int64_t i = v0 + (vt >> 2) + 64 * round;
+        if (i >= a.n_vec) break;
+        float x[32];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t w[4] = {raw[round][k].x, raw[round][k].y, raw[round][k].z, raw[round][k].w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            x[8 * k + 2 * h] = __uint_as_float(w[h] << 16);
+            x[8 * k + 2 * h + 1] = __uint_as_float(w[h] & 0xffff0000u);
+          }
+        }
+        // min / max as four independent chains
+        float lo4[4] = {x[0], x[1], x[2], x[3]}, hi4[4] = {x[0], x[1], x[2], x[3]};
+#pragma unroll
+        for (int e = 4; e < 32; ++e) {
+          lo4[e & 3] = fminf(lo4[e & 3], x[e]);
+          hi4[e & 3] = fmaxf(hi4[e & 3], x[e]);
+        }
+        const float lo = fminf(fminf(lo4[0], lo4[1]), fminf(lo4[2], lo4[3]));
+        const float hi = fmaxf(fmaxf(hi4[0], hi4[1]), fmaxf(hi4[2], hi4[3]));
+        constexpr int levels = (1 << VB) - 1;
+        // scale in fp64 as the reference quantizer; codes rounded to nearest by adding
+        // 1.5 * 2^23, redone in fp64 with floor(t + 1/2) within 1e-5 of a half step.
+        const double dlo = lo, span = (double)hi - dlo;
+        const float inv = span > 0.0 ? (float)(levels / span) : 0.f;
+        uint32_t vw[VB], vw2[VB];  // even / odd codes: two independent insert chains per word
+#pragma unroll
+        for (int w = 0; w < VB; ++w) vw[w] = vw2[w] = 0u;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float t = (x[e] - lo) * inv;
+          const float tr = t + 12582912.0f;
+          uint32_t qv = __float_as_uint(tr) & 0xffu;
+          if (fabsf(t - (tr - 12582912.0f)) > 0.5f - 1e-5f)
+            qv = (uint32_t)floor(((double)x[e] - dlo) * (levels / span) + 0.5);
+          qv = min(qv, (uint32_t)levels);
+          if (e & 1)
+            put_bits<VB, VB>(vw2, VB * e, qv);
+          else
+            put_bits<VB, VB>(vw, VB * e, qv);
+        }
+#pragma unroll
+        for (int w = 0; w < VB; ++w) vw[w] |= vw2[w];
+        uint32_t* vo = reinterpret_cast<uint32_t*>(a.v_codes + i * (VB * 16) + q * (VB * 4));
+#pragma unroll
+        for (int w = 0; w < VB; ++w) vo[w] = vw[w];
+        const uint32_t sb = __half_as_ushort(__double2half(span / levels));
+        const uint32_t mb = __half_as_ushort(__float2half_rn(lo));
+        reinterpret_cast<uint32_t*>(a.v_params)[i * 4 + q] = sb | (mb << 16);
+      }
+    }
+  }
+  if (__syncthreads_or(failed) && tid == 0) {
+    atomicOr(a.err, 1u);
+    // bounded: let abandoned MMAs (the last ones issued completed phase ^ 1) finish
+    // before TMEM is freed
+    s1::mbar_wait(bar1, phase ^ 1u);
+    s1::mbar_wait(bar2, phase ^ 1u);
+    s1::mbar_wait(bar3, phase);  // a key fetch issued for the pass that never ran
+  }
+  s1::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    s1::fence_after_sync();
+    s1::tmem_dealloc(tmem, 256);
+  }
+}
+
+template <int LMB, int VB>
+cudaError_t launch_rot_t(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) {
+  static bool configured = false;
+  const size_t smem = RotSmem::BYTES + 1024;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(compress_rot_kernel<LMB, VB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  int64_t blocks = (a.n_vec + kQ4Rows - 1) / kQ4Rows;
+  if (blocks > ctx->num_sms) blocks = ctx->num_sms;
+  if (ctx->prof_start) cudaEventRecord(ctx->prof_start, s);
+  compress_rot_kernel<LMB, VB><<<(unsigned)blocks, kRotThreads, smem, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (ctx->prof_stop) cudaEventRecord(ctx->prof_stop, s);
+  return e;
+}
+
+cudaError_t launch_rot(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) {
+  const int lmb = ctx->shape.lm_bits, vb = ctx->shape.v_bits;
+  if (lmb == 1) return vb == 2 ? launch_rot_t<1, 2>(ctx, a, s) : launch_rot_t<1, 4>(ctx, a, s);
+  if (lmb == 2) return vb == 2 ? launch_rot_t<2, 2>(ctx, a, s) : launch_rot_t<2, 4>(ctx, a, s);
+  return vb == 2 ? launch_rot_t<3, 2>(ctx, a, s) : launch_rot_t<3, 4>(ctx, a, s);
+}
+
 }  // namespace
 
 // S as f16 in the swizzled K-major operand layout of compress_tc_kernel, or false if
@@ -762,6 +1129,18 @@ bool pack_qjl_operand(const float* S, int m, int d, uint16_t* out) {
       out[tq::sm100::sw128_offset(i, j, 128) / 2] = __half_as_ushort(h);
     }
   return true;
+}
+
+// H diag(sigma) (Sylvester H[n][j] = (-1)^popcount(n & j), sigma_j = -1 where sign bit j is
+// set) as bf16 +-1 in the swizzled K-major operand layout of compress_rot_kernel:
+// element (n, j) multiplies key coordinate j into rotated coordinate n.
+void pack_hadamard_operand(const uint32_t* sign_bits, uint16_t* out) {
+  for (int n = 0; n < 128; ++n)
+    for (int j = 0; j < 128; ++j) {
+      bool neg = (__builtin_popcount((unsigned)(n & j)) & 1) != 0;
+      if ((sign_bits[j / 32] >> (j % 32)) & 1u) neg = !neg;
+      out[tq::sm100::sw128_offset(n, j, 128) / 2] = neg ? 0xBF80u : 0x3F80u;  // bf16 -1, +1
+    }
 }
 
 cudaError_t launch_compress(const tq_ctx* ctx, const void* k, const void* v, int dtype, int64_t n_vec,
@@ -785,8 +1164,10 @@ cudaError_t launch_compress(const tq_ctx* ctx, const void* k, const void* v, int
   a.rot = ctx->shape.rot;
   a.inv_sqrt_d = (float)(1.0 / sqrt((double)ctx->shape.d));
   a.S_sw128 = ctx->S_sw128;
+  a.H_sw128 = ctx->H_sw128;
   a.err = ctx->d_err;
   if (ctx->S_sw128 && ctx->shape.d == 128 && ctx->shape.m == 128) {
+    if (ctx->shape.rot == TQ_ROT_HADAMARD && dtype == TQ_BF16 && ctx->H_sw128) return launch_rot(ctx, a, stream);
     if (ctx->shape.rot == TQ_ROT_HADAMARD)
       return dtype == TQ_F32 ? launch_q4<float>(ctx, a, stream) : launch_q4<__nv_bfloat16>(ctx, a, stream);
     return dtype == TQ_F32 ? launch_tc<float>(ctx, a, stream) : launch_tc<__nv_bfloat16>(ctx, a, stream);

@@ -35,6 +35,7 @@ void free_tables(tq_ctx* c) {
   cudaFree(c->PiT);
   cudaFree(c->d_err);
   cudaFree(c->S_sw128);
+  cudaFree(c->H_sw128);
 }
 
 }  // namespace
@@ -160,6 +161,12 @@ tq_status tq_codebook_load(const tq_params* p, void* stream, tq_ctx** out) {
     if (!tq::pack_qjl_operand(p->qjl_S, m, d, s_op.data())) s_op.clear();
     if (e == cudaSuccess && !s_op.empty()) e = cudaMalloc((void**)&c->S_sw128, s_op.size() * sizeof(uint16_t));
   }
+  std::vector<uint16_t> h_op;
+  if (d == 128 && m == 128 && !s_op.empty() && p->rot == TQ_ROT_HADAMARD) {
+    h_op.assign((size_t)d * d, 0);
+    tq::pack_hadamard_operand(c->cb.sign_bits, h_op.data());
+    if (e == cudaSuccess) e = cudaMalloc((void**)&c->H_sw128, h_op.size() * sizeof(uint16_t));
+  }
   if (e != cudaSuccess) {
     free_tables(c);
     delete c;
@@ -177,6 +184,8 @@ tq_status tq_codebook_load(const tq_params* p, void* stream, tq_ctx** out) {
   if (e == cudaSuccess) e = cudaMemsetAsync(c->d_err, 0, sizeof(unsigned int), s);
   if (e == cudaSuccess && !s_op.empty())
     e = cudaMemcpyAsync(c->S_sw128, s_op.data(), s_op.size() * sizeof(uint16_t), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && !h_op.empty())
+    e = cudaMemcpyAsync(c->H_sw128, h_op.data(), h_op.size() * sizeof(uint16_t), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) {
     free_tables(c);
