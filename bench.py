@@ -84,10 +84,12 @@ def source_sha(names):
 
 
 DECODE_SOURCES = ("decode_mma.cu", "decode.cu", "tq_device.cuh", "tq_internal.h")
+COMPRESS_SOURCES = ("compress.cu", "tq_device.cuh", "tq_sm100.cuh", "tq_internal.h")
 
 
-def recorded_traffic(kernel_file: str, sha: str):
-    """DRAM bytes per launch from a committed ncu summary, if it matches the source."""
+def recorded_traffic(kernel_file: str, sha: str, units: int):
+    """DRAM bytes of one launch over `units` units, from a committed ncu summary that
+    gives DRAM bytes per unit for the same source (None if absent or stale)."""
     p = os.path.join(ROOT, "profiles", kernel_file)
     if not os.path.exists(p):
         return None
@@ -100,7 +102,7 @@ def recorded_traffic(kernel_file: str, sha: str):
     if kv.get("source_sha256_16") != sha:
         return None
     try:
-        return float(kv["dram_bytes_per_launch_scaled"])
+        return float(kv["dram_bytes_per_unit"]) * units
     except (KeyError, ValueError):
         return None
 
@@ -437,9 +439,28 @@ def run_ours(args, w: W.Workload):
 
     if rank == 0:
         peak, peak_kind = measured_peaks()
-        alg_bytes = packed_bytes
-        achieved = alg_bytes / dec_k_mean / 1e9
-        sha = source_sha(DECODE_SOURCES)
+        dsha = source_sha(DECODE_SOURCES)
+        units_dec = w.units * w.tokens  # (token, KV head) pairs
+        roof_dec = {"kernel": "decode_mma_kernel", "bound": "hbm", "achieved": packed_bytes / dec_k_mean / 1e9,
+                    "peak": peak, "unit": "GB/s", "frac": packed_bytes / dec_k_mean / 1e9 / peak,
+                    "peak_kind": peak_kind, "alg_bytes_per_launch": packed_bytes,
+                    "alg_bytes_per_unit": w.k_record_bytes() + w.v_record_bytes(), "unit_of_work": "token x KV head",
+                    "traffic": recorded_traffic("decode_kernel_traffic.txt", dsha, units_dec),
+                    "source_sha256_16": dsha}
+        roof = roof_dec
+        if not args.decode_only:
+            # The compression kernel takes most of a step, so it is the step's dominant kernel.
+            csha = source_sha(COMPRESS_SOURCES)
+            comp_bytes = in_bytes + packed_bytes
+            comp_k_mean = statistics.fmean(comp_k) / 1e3
+            ckern = "compress_rot_kernel" if (w.dtype == "bf16" and w.d == 128 and w.rotation == "hadamard") \
+                else "compress_q4_kernel"
+            roof = {"kernel": ckern, "bound": "hbm", "achieved": comp_bytes / comp_k_mean / 1e9, "peak": peak,
+                    "unit": "GB/s", "frac": comp_bytes / comp_k_mean / 1e9 / peak, "peak_kind": peak_kind,
+                    "alg_bytes_per_launch": comp_bytes, "alg_bytes_per_unit": comp_bytes // n_vec,
+                    "unit_of_work": "key + value vector pair",
+                    "traffic": recorded_traffic("compress_kernel_traffic.txt", csha, n_vec),
+                    "source_sha256_16": csha}
         line = {
             "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * (dec_total + comp_total) / args.steps,
@@ -457,11 +478,8 @@ def run_ours(args, w: W.Workload):
                 "kernel_ms": statistics.fmean(comp_k)},
             "decode_ms": {"call": dec_total * 1e3 / args.steps, "main_kernel": dec_k_mean * 1e3,
                           "main_kernel_timing": "separate loop of `steps` steps with events around the kernel"},
-            "roofline": {"kernel": "decode_mma_kernel", "bound": "hbm", "achieved": achieved, "peak": peak,
-                         "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
-                         "alg_bytes_per_launch": alg_bytes,
-                         "traffic": recorded_traffic("decode_kernel_traffic.txt", sha),
-                         "source_sha256_16": sha},
+            "roofline": roof,
+            "roofline_decode": roof_dec,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
