@@ -769,12 +769,14 @@ struct RotSmem {
   static constexpr uint32_t A_HI = 2 * kTcTileBytes, A_LO = 3 * kTcTileBytes;  // residual x16, f16
   static constexpr uint32_t S = 4 * kTcTileBytes;            // QJL matrix, f16 operand tile
   static constexpr uint32_t KR = 5 * kTcTileBytes;           // next pass's keys, raw rows (bulk copy)
-  static constexpr uint32_t XS = 6 * kTcTileBytes;           // [2][128] fp32 half-row sums
+  static constexpr uint32_t VR = 6 * kTcTileBytes;           // next pass's values, raw rows (bulk copy)
+  static constexpr uint32_t XS = 7 * kTcTileBytes;           // [2][128] fp32 half-row sums
   static constexpr uint32_t ZF = XS + 2 * 128 * 4;           // [128] nonzero-key flags
-  static constexpr uint32_t BAR = ZF + 128;                  // three mbarriers
-  static constexpr uint32_t TMEM = BAR + 24;                 // TMEM base address
+  static constexpr uint32_t BAR = ZF + 128;                  // four mbarriers
+  static constexpr uint32_t TMEM = BAR + 32;                 // TMEM base address
   static constexpr uint32_t BYTES = TMEM + 8;
 };
+static_assert(RotSmem::BYTES + 1024 <= 227 * 1024, "compress_rot_kernel shared memory");
 
 __device__ __forceinline__ void key_warps_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kRotKeyThreads) : "memory");
@@ -797,6 +799,7 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
   uint64_t* bar1 = reinterpret_cast<uint64_t*>(sm + RotSmem::BAR);  // rotation MMA done
   uint64_t* bar2 = bar1 + 1;                                         // projection MMA done
   uint64_t* bar3 = bar1 + 2;                                         // raw key rows landed
+  uint64_t* bar4 = bar1 + 3;                                         // raw value rows landed
   uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + RotSmem::TMEM);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool key_warp = warp < 8;
@@ -811,6 +814,7 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
     s1::mbar_init(bar1, 1);
     s1::mbar_init(bar2, 1);
     s1::mbar_init(bar3, 1);
+    s1::mbar_init(bar4, 1);
     s1::mbar_init_fence();
   }
   {  // H diag(sigma) and S operand tiles, prepacked on the host
@@ -846,7 +850,15 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
     s1::mbar_expect_tx(bar3, bytes);
     s1::bulk_g2s(sm + RotSmem::KR, static_cast<const __nv_bfloat16*>(a.k) + v0 * 128, bytes, bar3);
   };
+  // One thread: bring the raw value rows of pass `tile` into VR.
+  auto fetch_vals = [&](int64_t tile) {
+    const int64_t v0 = tile * kQ4Rows;
+    const uint32_t bytes = (uint32_t)(min((int64_t)kQ4Rows, a.n_vec - v0) * 256);
+    s1::mbar_expect_tx(bar4, bytes);
+    s1::bulk_g2s(sm + RotSmem::VR, static_cast<const __nv_bfloat16*>(a.v) + v0 * 128, bytes, bar4);
+  };
   if (a.k && tid == 0 && blockIdx.x < ntile) fetch_keys(blockIdx.x);
+  if (a.v && tid == 0 && blockIdx.x < ntile) fetch_vals(blockIdx.x);
   for (int64_t tile = blockIdx.x; tile < ntile; tile += gridDim.x, phase ^= 1u) {
     const int64_t v0 = tile * kQ4Rows;
     // ---- stage the 128 keys: raw rows -> swizzled operand tile, once they landed and
@@ -1008,24 +1020,19 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
     } else if (!key_warp && a.v) {
       // ---------------------------------------------------------------- values
       const int vt = tid - kRotKeyThreads, q = vt & 3;
-      uint4 raw[2][4];  // both rounds' loads in flight before either is worked on
+      // the pass's value rows were bulk-copied into VR one pass ahead
+      if (!failed && !s1::mbar_wait(bar4, phase)) failed = true;
 #pragma unroll
       for (int round = 0; round < 2; ++round) {
-        const int64_t i = v0 + (vt >> 2) + 64 * round;
-        if (i < a.n_vec) {
-          const uint4* p4 = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.v) + i * 128 + 32 * q);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) raw[round][k] = __ldg(p4 + k);
-        }
-      }
-#pragma unroll
-      for (int round = 0; round < 2; ++round) {
-        const int64_t i = v0 + (vt >> 2) + 64 * round;
-        if (i >= a.n_vec) break;
+        const int row = (vt >> 2) + 64 * round;
+        const int64_t i = v0 + row;
+        if (i >= a.n_vec || failed) break;
         float x[32];
+        const uint4* p4 = reinterpret_cast<const uint4*>(sm + RotSmem::VR + row * 256 + 64 * q);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const uint32_t w[4] = {raw[round][k].x, raw[round][k].y, raw[round][k].z, raw[round][k].w};
+          const uint4 rv = p4[k];
+          const uint32_t w[4] = {rv.x, rv.y, rv.z, rv.w};
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
             x[8 * k + 2 * h] = __uint_as_float(w[h] << 16);
@@ -1071,6 +1078,12 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
         const uint32_t mb = __half_as_ushort(__float2half_rn(lo));
         reinterpret_cast<uint32_t*>(a.v_params)[i * 4 + q] = sb | (mb << 16);
       }
+      // every value thread has read VR: fetch the next pass's values
+      asm volatile("bar.sync 2, %0;" ::"n"(kRotThreads - kRotKeyThreads) : "memory");
+      if (tid == kRotKeyThreads && tile + gridDim.x < ntile) {
+        s1::fence_async_smem();
+        fetch_vals(tile + gridDim.x);
+      }
     }
   }
   if (__syncthreads_or(failed) && tid == 0) {
@@ -1079,7 +1092,8 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
     // before TMEM is freed
     s1::mbar_wait(bar1, phase ^ 1u);
     s1::mbar_wait(bar2, phase ^ 1u);
-    s1::mbar_wait(bar3, phase);  // a key fetch issued for the pass that never ran
+    s1::mbar_wait(bar3, phase);  // key / value fetches issued for the pass that never ran
+    s1::mbar_wait(bar4, phase);
   }
   s1::fence_before_sync();
   __syncthreads();
