@@ -10,6 +10,8 @@
 // every global load and store of a record is a contiguous warp-wide access.
 #include <cuda_runtime.h>
 
+#include <cstring>
+
 #include "tq_device.cuh"
 #include "tq_sm100.cuh"
 
@@ -763,20 +765,25 @@ cudaError_t launch_q4(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) 
 constexpr int kRotThreads = 512;
 constexpr int kRotKeyThreads = 256;
 
+// Shared memory of compress_rot_kernel. The Haar rotation needs three bf16 tiles of Pi
+// (its 24-bit split), so that variant loads keys and values straight from global
+// memory instead of staging raw rows.
+template <bool HAAR>
 struct RotSmem {
+  static constexpr uint32_t NT = HAAR ? 3 : 1;               // bf16 terms of the rotation
   static constexpr uint32_t KT = 0;                          // keys, bf16 operand tile
-  static constexpr uint32_t HB = kTcTileBytes;               // H diag(sigma), bf16 operand tile
-  static constexpr uint32_t A_HI = 2 * kTcTileBytes, A_LO = 3 * kTcTileBytes;  // residual x16, f16
-  static constexpr uint32_t S = 4 * kTcTileBytes;            // QJL matrix, f16 operand tile
-  static constexpr uint32_t KR = 5 * kTcTileBytes;           // next pass's keys, raw rows (bulk copy)
-  static constexpr uint32_t VR = 6 * kTcTileBytes;           // next pass's values, raw rows (bulk copy)
-  static constexpr uint32_t XS = 7 * kTcTileBytes;           // [2][128] fp32 half-row sums
+  static constexpr uint32_t HB = kTcTileBytes;               // rotation, NT bf16 operand tiles
+  static constexpr uint32_t A_HI = (1 + NT) * kTcTileBytes, A_LO = (2 + NT) * kTcTileBytes;  // residual x16
+  static constexpr uint32_t S = (3 + NT) * kTcTileBytes;     // QJL matrix, f16 operand tile
+  static constexpr uint32_t KR = (4 + NT) * kTcTileBytes;    // Hadamard: next pass's raw key rows
+  static constexpr uint32_t VR = (5 + NT) * kTcTileBytes;    // Hadamard: next pass's raw value rows
+  static constexpr uint32_t XS = (HAAR ? 4 + NT : 6 + NT) * kTcTileBytes;  // [2][128] half-row sums
   static constexpr uint32_t ZF = XS + 2 * 128 * 4;           // [128] nonzero-key flags
   static constexpr uint32_t BAR = ZF + 128;                  // four mbarriers
   static constexpr uint32_t TMEM = BAR + 32;                 // TMEM base address
   static constexpr uint32_t BYTES = TMEM + 8;
+  static_assert(BYTES + 1024 <= 227 * 1024, "compress_rot_kernel shared memory");
 };
-static_assert(RotSmem::BYTES + 1024 <= 227 * 1024, "compress_rot_kernel shared memory");
 
 __device__ __forceinline__ void key_warps_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kRotKeyThreads) : "memory");
@@ -787,20 +794,21 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return sm100::idesc_f16_f32(M, N) | (1u << 7) | (1u << 10);
 }
 
-template <int LMB, int VB>
+template <int LMB, int VB, bool HAAR>
 __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __grid_constant__ CompressArgs a) {
+  using RS = RotSmem<HAAR>;
   namespace s1 = tq::sm100;
   constexpr int KW = 2 * LMB;  // code words per key thread (64 codes x LMB bits)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = s1::smem_u32(sm);
-  float* xs = reinterpret_cast<float*>(sm + RotSmem::XS);
-  uint8_t* zf = sm + RotSmem::ZF;
-  uint64_t* bar1 = reinterpret_cast<uint64_t*>(sm + RotSmem::BAR);  // rotation MMA done
+  float* xs = reinterpret_cast<float*>(sm + RS::XS);
+  uint8_t* zf = sm + RS::ZF;
+  uint64_t* bar1 = reinterpret_cast<uint64_t*>(sm + RS::BAR);  // rotation MMA done
   uint64_t* bar2 = bar1 + 1;                                         // projection MMA done
   uint64_t* bar3 = bar1 + 2;                                         // raw key rows landed
   uint64_t* bar4 = bar1 + 3;                                         // raw value rows landed
-  uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + RotSmem::TMEM);
+  uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + RS::TMEM);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool key_warp = warp < 8;
   const int sp = warp & 3, ch = (warp >> 2) & 1;  // key warps: sub-partition, column half
@@ -820,12 +828,10 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
   {  // H diag(sigma) and S operand tiles, prepacked on the host
     const uint4* hsrc = reinterpret_cast<const uint4*>(a.H_sw128);
     const uint4* ssrc = reinterpret_cast<const uint4*>(a.S_sw128);
-    uint4* hdst = reinterpret_cast<uint4*>(sm + RotSmem::HB);
-    uint4* sdst = reinterpret_cast<uint4*>(sm + RotSmem::S);
-    for (int w = tid; w < (int)(kTcTileBytes / 16); w += kRotThreads) {
-      hdst[w] = hsrc[w];
-      sdst[w] = ssrc[w];
-    }
+    uint4* hdst = reinterpret_cast<uint4*>(sm + RS::HB);
+    uint4* sdst = reinterpret_cast<uint4*>(sm + RS::S);
+    for (int w = tid; w < (int)(kTcTileBytes / 16); w += kRotThreads) sdst[w] = ssrc[w];
+    for (int w = tid; w < (int)(RS::NT * kTcTileBytes / 16); w += kRotThreads) hdst[w] = hsrc[w];
   }
   s1::fence_async_smem();
   s1::fence_before_sync();
@@ -848,23 +854,23 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
     const int64_t v0 = tile * kQ4Rows;
     const uint32_t bytes = (uint32_t)(min((int64_t)kQ4Rows, a.n_vec - v0) * 256);
     s1::mbar_expect_tx(bar3, bytes);
-    s1::bulk_g2s(sm + RotSmem::KR, static_cast<const __nv_bfloat16*>(a.k) + v0 * 128, bytes, bar3);
+    s1::bulk_g2s(sm + RS::KR, static_cast<const __nv_bfloat16*>(a.k) + v0 * 128, bytes, bar3);
   };
   // One thread: bring the raw value rows of pass `tile` into VR.
   auto fetch_vals = [&](int64_t tile) {
     const int64_t v0 = tile * kQ4Rows;
     const uint32_t bytes = (uint32_t)(min((int64_t)kQ4Rows, a.n_vec - v0) * 256);
     s1::mbar_expect_tx(bar4, bytes);
-    s1::bulk_g2s(sm + RotSmem::VR, static_cast<const __nv_bfloat16*>(a.v) + v0 * 128, bytes, bar4);
+    s1::bulk_g2s(sm + RS::VR, static_cast<const __nv_bfloat16*>(a.v) + v0 * 128, bytes, bar4);
   };
-  if (a.k && tid == 0 && blockIdx.x < ntile) fetch_keys(blockIdx.x);
-  if (a.v && tid == 0 && blockIdx.x < ntile) fetch_vals(blockIdx.x);
+  if (!HAAR && a.k && tid == 0 && blockIdx.x < ntile) fetch_keys(blockIdx.x);
+  if (!HAAR && a.v && tid == 0 && blockIdx.x < ntile) fetch_vals(blockIdx.x);
   for (int64_t tile = blockIdx.x; tile < ntile; tile += gridDim.x, phase ^= 1u) {
     const int64_t v0 = tile * kQ4Rows;
     // ---- stage the 128 keys: raw rows -> swizzled operand tile, once they landed and
     // the previous pass's rotation MMA has finished reading the tile.
     if (a.k && tile != blockIdx.x && !failed && !s1::mbar_wait(bar1, phase ^ 1u)) failed = true;
-    if (a.k && !failed && !s1::mbar_wait(bar3, phase)) failed = true;
+    if (!HAAR && a.k && !failed && !s1::mbar_wait(bar3, phase)) failed = true;
     if (__syncthreads_or(failed)) break;
     if (a.k) {
       const int nrows = (int)min((int64_t)kQ4Rows, a.n_vec - v0);
@@ -872,12 +878,16 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int id = tid + kRotThreads * u, row = id >> 4;
-        kv[u] = row < nrows ? reinterpret_cast<const uint4*>(sm + RotSmem::KR)[id] : make_uint4(0u, 0u, 0u, 0u);
+        if constexpr (HAAR)
+          kv[u] = row < nrows ? __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.k) + v0 * 128) + id)
+                              : make_uint4(0u, 0u, 0u, 0u);
+        else
+          kv[u] = row < nrows ? reinterpret_cast<const uint4*>(sm + RS::KR)[id] : make_uint4(0u, 0u, 0u, 0u);
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int id = tid + kRotThreads * u, row = id >> 4, c16 = id & 15;
-        *reinterpret_cast<uint4*>(sm + RotSmem::KT + s1::sw128_offset(row, 8 * c16, kQ4Rows)) = kv[u];
+        *reinterpret_cast<uint4*>(sm + RS::KT + s1::sw128_offset(row, 8 * c16, kQ4Rows)) = kv[u];
       }
       s1::fence_async_smem();
       s1::fence_before_sync();
@@ -886,12 +896,15 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
       if (tid == 0) {
         constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          s1::umma_f16(tmem_y, s1::sw128_desc(sbase + RotSmem::KT, 16 * ks, kQ4Rows),
-                       s1::sw128_desc(sbase + RotSmem::HB, 16 * ks, 128), idesc, ks > 0 ? 1u : 0u);
+        for (int t = 0; t < (int)RS::NT; ++t)
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            s1::umma_f16(tmem_y, s1::sw128_desc(sbase + RS::KT, 16 * ks, kQ4Rows),
+                         s1::sw128_desc(sbase + RS::HB + t * kTcTileBytes, 16 * ks, 128), idesc,
+                         (t > 0 || ks > 0) ? 1u : 0u);
         s1::umma_commit(bar1);
         // KR has been read by every thread (the barrier above): fetch the next pass.
-        if (tile + gridDim.x < ntile) {
+        if (!HAAR && tile + gridDim.x < ntile) {
           s1::fence_async_smem();
           fetch_keys(tile + gridDim.x);
         }
@@ -918,7 +931,7 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
       for (int e = 0; e < 64; ++e) s4[e & 3] = fmaf(y[e], y[e], s4[e & 3]);
       xs[ch * 128 + R] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
       key_warps_sync();
-      const float tot = xs[R] + xs[128 + R];  // ||Y||^2 = d ||k||^2
+      const float tot = xs[R] + xs[128 + R];  // ||Y||^2 = d ||k||^2 (Hadamard), ||k||^2 (Haar)
       key_warps_sync();                      // both halves read before xs is reused
       const bool nz = tot > 0.f;
       const float sc = nz ? 1.0f / sqrtf(tot) : 0.f;
@@ -955,7 +968,7 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
 #pragma unroll
         for (int w = 0; w < KW; ++w) co[w] = nz ? cw[w] : 0u;
         if (ch == 0) {
-          const float n = sqrtf(tot * (1.0f / 128.f));
+          const float n = HAAR ? sqrtf(tot) : sqrtf(tot * (1.0f / 128.f));
           const uint32_t nb = __half_as_ushort(__float2half_rn(n));
           const uint32_t gb = __half_as_ushort(__float2half_rn(gamma));
           reinterpret_cast<uint32_t*>(a.k_norms)[i] = nz ? (nb | (gb << 16)) : 0u;
@@ -976,8 +989,8 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
           lw[p] = *reinterpret_cast<const uint32_t*>(&ll);
         }
         const uint32_t off = s1::sw128_offset(R, 64 * ch + 8 * c8, kQ4Rows);
-        *reinterpret_cast<uint4*>(sm + RotSmem::A_HI + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        *reinterpret_cast<uint4*>(sm + RotSmem::A_LO + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        *reinterpret_cast<uint4*>(sm + RS::A_HI + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(sm + RS::A_LO + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
       }
       if (ch == 0) zf[R] = use ? 1 : 0;
       s1::fence_async_smem();
@@ -988,12 +1001,12 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
         constexpr uint32_t idesc = s1::idesc_f16_f32(128, 128);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          s1::umma_f16(tmem_p, s1::sw128_desc(sbase + RotSmem::A_HI, 16 * ks, kQ4Rows),
-                       s1::sw128_desc(sbase + RotSmem::S, 16 * ks, 128), idesc, ks > 0 ? 1u : 0u);
+          s1::umma_f16(tmem_p, s1::sw128_desc(sbase + RS::A_HI, 16 * ks, kQ4Rows),
+                       s1::sw128_desc(sbase + RS::S, 16 * ks, 128), idesc, ks > 0 ? 1u : 0u);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          s1::umma_f16(tmem_p, s1::sw128_desc(sbase + RotSmem::A_LO, 16 * ks, kQ4Rows),
-                       s1::sw128_desc(sbase + RotSmem::S, 16 * ks, 128), idesc, 1u);
+          s1::umma_f16(tmem_p, s1::sw128_desc(sbase + RS::A_LO, 16 * ks, kQ4Rows),
+                       s1::sw128_desc(sbase + RS::S, 16 * ks, 128), idesc, 1u);
         s1::umma_commit(bar2);
       }
       // ---- QJL signs of this thread's 64 projections
@@ -1020,18 +1033,32 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
     } else if (!key_warp && a.v) {
       // ---------------------------------------------------------------- values
       const int vt = tid - kRotKeyThreads, q = vt & 3;
-      // the pass's value rows were bulk-copied into VR one pass ahead
-      if (!failed && !s1::mbar_wait(bar4, phase)) failed = true;
+      // Hadamard: the pass's value rows were bulk-copied into VR one pass ahead.
+      // Haar: both rounds' rows are loaded before either is worked on.
+      uint4 raw[HAAR ? 2 : 1][4];
+      if constexpr (HAAR) {
+#pragma unroll
+        for (int round = 0; round < 2; ++round) {
+          const int64_t i = v0 + (vt >> 2) + 64 * round;
+          if (i < a.n_vec) {
+            const uint4* g4 = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.v) + i * 128 + 32 * q);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) raw[round][k] = __ldg(g4 + k);
+          }
+        }
+      } else {
+        if (!failed && !s1::mbar_wait(bar4, phase)) failed = true;
+      }
 #pragma unroll
       for (int round = 0; round < 2; ++round) {
         const int row = (vt >> 2) + 64 * round;
         const int64_t i = v0 + row;
         if (i >= a.n_vec || failed) break;
         float x[32];
-        const uint4* p4 = reinterpret_cast<const uint4*>(sm + RotSmem::VR + row * 256 + 64 * q);
+        const uint4* p4 = reinterpret_cast<const uint4*>(sm + RS::VR + row * 256 + 64 * q);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const uint4 rv = p4[k];
+          const uint4 rv = HAAR ? raw[HAAR ? round : 0][k] : p4[k];
           const uint32_t w[4] = {rv.x, rv.y, rv.z, rv.w};
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
@@ -1078,11 +1105,13 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
         const uint32_t mb = __half_as_ushort(__float2half_rn(lo));
         reinterpret_cast<uint32_t*>(a.v_params)[i * 4 + q] = sb | (mb << 16);
       }
-      // every value thread has read VR: fetch the next pass's values
-      asm volatile("bar.sync 2, %0;" ::"n"(kRotThreads - kRotKeyThreads) : "memory");
-      if (tid == kRotKeyThreads && tile + gridDim.x < ntile) {
-        s1::fence_async_smem();
-        fetch_vals(tile + gridDim.x);
+      if constexpr (!HAAR) {
+        // every value thread has read VR: fetch the next pass's values
+        asm volatile("bar.sync 2, %0;" ::"n"(kRotThreads - kRotKeyThreads) : "memory");
+        if (tid == kRotKeyThreads && tile + gridDim.x < ntile) {
+          s1::fence_async_smem();
+          fetch_vals(tile + gridDim.x);
+        }
       }
     }
   }
@@ -1092,8 +1121,10 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
     // before TMEM is freed
     s1::mbar_wait(bar1, phase ^ 1u);
     s1::mbar_wait(bar2, phase ^ 1u);
-    s1::mbar_wait(bar3, phase);  // key / value fetches issued for the pass that never ran
-    s1::mbar_wait(bar4, phase);
+    if (!HAAR) {
+      s1::mbar_wait(bar3, phase);  // key / value fetches issued for the pass that never ran
+      s1::mbar_wait(bar4, phase);
+    }
   }
   s1::fence_before_sync();
   __syncthreads();
@@ -1103,30 +1134,31 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
   }
 }
 
-template <int LMB, int VB>
+template <int LMB, int VB, bool HAAR>
 cudaError_t launch_rot_t(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) {
   static bool configured = false;
-  const size_t smem = RotSmem::BYTES + 1024;
+  const size_t smem = RotSmem<HAAR>::BYTES + 1024;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(compress_rot_kernel<LMB, VB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(compress_rot_kernel<LMB, VB, HAAR>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   int64_t blocks = (a.n_vec + kQ4Rows - 1) / kQ4Rows;
   if (blocks > ctx->num_sms) blocks = ctx->num_sms;
   if (ctx->prof_start) cudaEventRecord(ctx->prof_start, s);
-  compress_rot_kernel<LMB, VB><<<(unsigned)blocks, kRotThreads, smem, s>>>(a);
+  compress_rot_kernel<LMB, VB, HAAR><<<(unsigned)blocks, kRotThreads, smem, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (ctx->prof_stop) cudaEventRecord(ctx->prof_stop, s);
   return e;
 }
 
+template <bool HAAR>
 cudaError_t launch_rot(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) {
   const int lmb = ctx->shape.lm_bits, vb = ctx->shape.v_bits;
-  if (lmb == 1) return vb == 2 ? launch_rot_t<1, 2>(ctx, a, s) : launch_rot_t<1, 4>(ctx, a, s);
-  if (lmb == 2) return vb == 2 ? launch_rot_t<2, 2>(ctx, a, s) : launch_rot_t<2, 4>(ctx, a, s);
-  return vb == 2 ? launch_rot_t<3, 2>(ctx, a, s) : launch_rot_t<3, 4>(ctx, a, s);
+  if (lmb == 1) return vb == 2 ? launch_rot_t<1, 2, HAAR>(ctx, a, s) : launch_rot_t<1, 4, HAAR>(ctx, a, s);
+  if (lmb == 2) return vb == 2 ? launch_rot_t<2, 2, HAAR>(ctx, a, s) : launch_rot_t<2, 4, HAAR>(ctx, a, s);
+  return vb == 2 ? launch_rot_t<3, 2, HAAR>(ctx, a, s) : launch_rot_t<3, 4, HAAR>(ctx, a, s);
 }
 
 }  // namespace
@@ -1157,6 +1189,37 @@ void pack_hadamard_operand(const uint32_t* sign_bits, uint16_t* out) {
     }
 }
 
+namespace {
+uint16_t bf16_rn(float x) {  // round to nearest even (finite inputs)
+  uint32_t u;
+  std::memcpy(&u, &x, 4);
+  u += 0x7fffu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+float bf16_value(uint16_t h) {
+  const uint32_t u = (uint32_t)h << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+}  // namespace
+
+// Pi (fp64, row-major, d = 128) as three bf16 terms Pi ~ P1 + P2 + P3 (each the rounded
+// remainder of the previous ones, about 24 bits together), three tiles in the swizzled
+// K-major operand layout of compress_rot_kernel: element (n, j) multiplies key
+// coordinate j into rotated coordinate n.
+void pack_haar_operand(const double* pi, uint16_t* out) {
+  for (int n = 0; n < 128; ++n)
+    for (int j = 0; j < 128; ++j) {
+      double rem = pi[(size_t)n * 128 + j];
+      for (int t = 0; t < 3; ++t) {
+        const uint16_t h = bf16_rn((float)rem);
+        out[(size_t)t * 128 * 128 + tq::sm100::sw128_offset(n, j, 128) / 2] = h;
+        rem -= (double)bf16_value(h);
+      }
+    }
+}
+
 cudaError_t launch_compress(const tq_ctx* ctx, const void* k, const void* v, int dtype, int64_t n_vec,
                             uint8_t* k_codes, uint8_t* k_signs, uint16_t* k_norms, uint8_t* v_codes,
                             uint16_t* v_params, cudaStream_t stream) {
@@ -1181,7 +1244,12 @@ cudaError_t launch_compress(const tq_ctx* ctx, const void* k, const void* v, int
   a.H_sw128 = ctx->H_sw128;
   a.err = ctx->d_err;
   if (ctx->S_sw128 && ctx->shape.d == 128 && ctx->shape.m == 128) {
-    if (ctx->shape.rot == TQ_ROT_HADAMARD && dtype == TQ_BF16 && ctx->H_sw128) return launch_rot(ctx, a, stream);
+    if (ctx->shape.rot == TQ_ROT_HADAMARD && dtype == TQ_BF16 && ctx->H_sw128)
+      return launch_rot<false>(ctx, a, stream);
+    if (ctx->shape.rot == TQ_ROT_HAAR && dtype == TQ_BF16 && ctx->Pi_sw128) {
+      a.H_sw128 = ctx->Pi_sw128;
+      return launch_rot<true>(ctx, a, stream);
+    }
     if (ctx->shape.rot == TQ_ROT_HADAMARD)
       return dtype == TQ_F32 ? launch_q4<float>(ctx, a, stream) : launch_q4<__nv_bfloat16>(ctx, a, stream);
     return dtype == TQ_F32 ? launch_tc<float>(ctx, a, stream) : launch_tc<__nv_bfloat16>(ctx, a, stream);

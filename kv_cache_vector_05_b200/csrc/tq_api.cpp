@@ -36,6 +36,7 @@ void free_tables(tq_ctx* c) {
   cudaFree(c->d_err);
   cudaFree(c->S_sw128);
   cudaFree(c->H_sw128);
+  cudaFree(c->Pi_sw128);
 }
 
 }  // namespace
@@ -167,6 +168,12 @@ tq_status tq_codebook_load(const tq_params* p, void* stream, tq_ctx** out) {
     tq::pack_hadamard_operand(c->cb.sign_bits, h_op.data());
     if (e == cudaSuccess) e = cudaMalloc((void**)&c->H_sw128, h_op.size() * sizeof(uint16_t));
   }
+  std::vector<uint16_t> pi_op;
+  if (d == 128 && m == 128 && !s_op.empty() && p->rot == TQ_ROT_HAAR) {
+    pi_op.assign((size_t)3 * d * d, 0);
+    tq::pack_haar_operand(p->haar, pi_op.data());
+    if (e == cudaSuccess) e = cudaMalloc((void**)&c->Pi_sw128, pi_op.size() * sizeof(uint16_t));
+  }
   if (e != cudaSuccess) {
     free_tables(c);
     delete c;
@@ -186,6 +193,8 @@ tq_status tq_codebook_load(const tq_params* p, void* stream, tq_ctx** out) {
     e = cudaMemcpyAsync(c->S_sw128, s_op.data(), s_op.size() * sizeof(uint16_t), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess && !h_op.empty())
     e = cudaMemcpyAsync(c->H_sw128, h_op.data(), h_op.size() * sizeof(uint16_t), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && !pi_op.empty())
+    e = cudaMemcpyAsync(c->Pi_sw128, pi_op.data(), pi_op.size() * sizeof(uint16_t), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) {
     free_tables(c);

@@ -47,6 +47,7 @@ struct tq_ctx {
   unsigned int* d_err;     // device error word: bit 0 = a bounded wait in a kernel timed out
   uint16_t* S_sw128;       // tensor-core compression: S as an f16 operand tile (d = m = 128, S exact in f16)
   uint16_t* H_sw128;       // tensor-core compression: H diag(sigma) as a bf16 operand tile (d = 128, Hadamard)
+  uint16_t* Pi_sw128;      // tensor-core compression: Haar Pi as three bf16 operand tiles (d = 128)
 };
 
 namespace tq {
@@ -85,6 +86,7 @@ int mma_tile_tokens(int G);                  // tokens per tile of the tensor-co
 int mma_ctas_per_sm(int lm_bits, int v_bits, int G);  // resident CTAs per SM of the tensor-core decode
 bool pack_qjl_operand(const float* S, int m, int d, uint16_t* out);
 void pack_hadamard_operand(const uint32_t* sign_bits, uint16_t* out);  // d = 128
+void pack_haar_operand(const double* pi, uint16_t* out);                // d = 128, 3 tiles
 
 cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const void* q, int q_dtype, int batch,
                               int hq, int hkv, const int32_t* seq_lens, int64_t max_len, const uint8_t* k_codes,
