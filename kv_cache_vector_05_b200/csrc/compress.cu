@@ -917,80 +917,88 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
       const bool valid = i < a.n_vec;
       if (!failed && !s1::mbar_wait(bar1, phase)) failed = true;
       s1::fence_after_sync();
-      float y[64];
+      // Two 32-column chunks per thread: a first pass for the norm, a second one (a loop
+      // that is not unrolled, to keep the code small) for codes, residual and operands.
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t v[32];
         s1::tmem_ld32(tmem_y + lane_base + 64 * ch + 32 * h, v);
         s1::tmem_ld_wait();
 #pragma unroll
-        for (int k = 0; k < 32; ++k) y[32 * h + k] = __uint_as_float(v[k]);
+        for (int e = 0; e < 32; ++e) {
+          const float yv = __uint_as_float(v[e]);
+          s4[e & 3] = fmaf(yv, yv, s4[e & 3]);
+        }
       }
-      float s4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int e = 0; e < 64; ++e) s4[e & 3] = fmaf(y[e], y[e], s4[e & 3]);
       xs[ch * 128 + R] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
       key_warps_sync();
       const float tot = xs[R] + xs[128 + R];  // ||Y||^2 = d ||k||^2 (Hadamard), ||k||^2 (Haar)
       key_warps_sync();                      // both halves read before xs is reused
       const bool nz = tot > 0.f;
       const float sc = nz ? 1.0f / sqrtf(tot) : 0.f;
-      uint32_t cw[KW], cw2[KW];  // even / odd codes: two independent insert chains per word
-#pragma unroll
-      for (int w = 0; w < KW; ++w) cw[w] = cw2[w] = 0u;
+      const bool use = valid && nz;
+      constexpr int CW = LMB;  // code words of a 32-column chunk
       float r4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        uint32_t v[32];
+        s1::tmem_ld32(tmem_y + lane_base + 64 * ch + 32 * h, v);
+        s1::tmem_ld_wait();
+        uint32_t cw[CW], cw2[CW];  // even / odd codes: two independent insert chains per word
 #pragma unroll
-      for (int e = 0; e < 64; ++e) {
-        const float yy = y[e] * sc;
-        uint32_t idx = 0;
-        float cv = cb_c[0];
+        for (int w = 0; w < CW; ++w) cw[w] = cw2[w] = 0u;
+        float r[32];
 #pragma unroll
-        for (int k = 0; k < (1 << LMB) - 1; ++k) {
-          if (yy >= cb_t[k]) {
-            idx = k + 1;
-            cv = cb_c[k + 1];
+        for (int e = 0; e < 32; ++e) {
+          const float yy = __uint_as_float(v[e]) * sc;
+          uint32_t idx = 0;
+          float cv = cb_c[0];
+#pragma unroll
+          for (int k = 0; k < (1 << LMB) - 1; ++k) {
+            if (yy >= cb_t[k]) {
+              idx = k + 1;
+              cv = cb_c[k + 1];
+            }
           }
+          if (e & 1)
+            put_bits<LMB, CW>(cw2, LMB * e, idx);
+          else
+            put_bits<LMB, CW>(cw, LMB * e, idx);
+          r[e] = yy - cv;
+          r4[e & 3] = fmaf(r[e], r[e], r4[e & 3]);
         }
-        if (e & 1)
-          put_bits<LMB, KW>(cw2, LMB * e, idx);
-        else
-          put_bits<LMB, KW>(cw, LMB * e, idx);
-        y[e] = yy - cv;
-        r4[e & 3] = fmaf(y[e], y[e], r4[e & 3]);
-      }
+        if (valid) {
+          uint32_t* co = reinterpret_cast<uint32_t*>(a.k_codes + i * (LMB * 16) + ch * (LMB * 8) + h * (LMB * 4));
 #pragma unroll
-      for (int w = 0; w < KW; ++w) cw[w] |= cw2[w];
+          for (int w = 0; w < CW; ++w) co[w] = nz ? (cw[w] | cw2[w]) : 0u;
+        }
+        // residual x16 as f16 hi + lo (the previous projection finished: it was waited for)
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) {
+          uint32_t hw[4], lw[4];
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            const float f0 = use ? 16.f * r[8 * c8 + 2 * p] : 0.f, f1 = use ? 16.f * r[8 * c8 + 2 * p + 1] : 0.f;
+            const __half2 hh = __floats2half2_rn(f0, f1);
+            const float2 hf = __half22float2(hh);
+            const __half2 ll = __floats2half2_rn(f0 - hf.x, f1 - hf.y);
+            hw[p] = *reinterpret_cast<const uint32_t*>(&hh);
+            lw[p] = *reinterpret_cast<const uint32_t*>(&ll);
+          }
+          const uint32_t off = s1::sw128_offset(R, 64 * ch + 32 * h + 8 * c8, kQ4Rows);
+          *reinterpret_cast<uint4*>(sm + RS::A_HI + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(sm + RS::A_LO + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        }
+      }
       xs[ch * 128 + R] = (r4[0] + r4[1]) + (r4[2] + r4[3]);
       key_warps_sync();
       const float gamma = sqrtf(xs[R] + xs[128 + R]);
-      if (valid) {
-        uint32_t* co = reinterpret_cast<uint32_t*>(a.k_codes + i * (LMB * 16) + ch * (LMB * 8));
-#pragma unroll
-        for (int w = 0; w < KW; ++w) co[w] = nz ? cw[w] : 0u;
-        if (ch == 0) {
-          const float n = HAAR ? sqrtf(tot) : sqrtf(tot * (1.0f / 128.f));
-          const uint32_t nb = __half_as_ushort(__float2half_rn(n));
-          const uint32_t gb = __half_as_ushort(__float2half_rn(gamma));
-          reinterpret_cast<uint32_t*>(a.k_norms)[i] = nz ? (nb | (gb << 16)) : 0u;
-        }
-      }
-      // residual x16 as f16 hi + lo (the previous projection finished: it was waited for)
-      const bool use = valid && nz;
-#pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        uint32_t hw[4], lw[4];
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          const float f0 = use ? 16.f * y[8 * c8 + 2 * p] : 0.f, f1 = use ? 16.f * y[8 * c8 + 2 * p + 1] : 0.f;
-          const __half2 hh = __floats2half2_rn(f0, f1);
-          const float2 hf = __half22float2(hh);
-          const __half2 ll = __floats2half2_rn(f0 - hf.x, f1 - hf.y);
-          hw[p] = *reinterpret_cast<const uint32_t*>(&hh);
-          lw[p] = *reinterpret_cast<const uint32_t*>(&ll);
-        }
-        const uint32_t off = s1::sw128_offset(R, 64 * ch + 8 * c8, kQ4Rows);
-        *reinterpret_cast<uint4*>(sm + RS::A_HI + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        *reinterpret_cast<uint4*>(sm + RS::A_LO + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      if (valid && ch == 0) {
+        const float n = HAAR ? sqrtf(tot) : sqrtf(tot * (1.0f / 128.f));
+        const uint32_t nb = __half_as_ushort(__float2half_rn(n));
+        const uint32_t gb = __half_as_ushort(__float2half_rn(gamma));
+        reinterpret_cast<uint32_t*>(a.k_norms)[i] = nz ? (nb | (gb << 16)) : 0u;
       }
       if (ch == 0) zf[R] = use ? 1 : 0;
       s1::fence_async_smem();
@@ -1049,7 +1057,7 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
       } else {
         if (!failed && !s1::mbar_wait(bar4, phase)) failed = true;
       }
-#pragma unroll
+#pragma unroll(HAAR ? 2 : 1)
       for (int round = 0; round < 2; ++round) {
         const int row = (vt >> 2) + 64 * round;
         const int64_t i = v0 + row;
