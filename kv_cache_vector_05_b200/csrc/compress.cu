@@ -920,7 +920,7 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
       // Two 32-column chunks per thread: a first pass for the norm, a second one (a loop
       // that is not unrolled, to keep the code small) for codes, residual and operands.
       float s4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
+#pragma unroll 1
       for (int h = 0; h < 2; ++h) {
         uint32_t v[32];
         s1::tmem_ld32(tmem_y + lane_base + 64 * ch + 32 * h, v);
@@ -1020,8 +1020,8 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
       // ---- QJL signs of this thread's 64 projections
       if (!failed && !s1::mbar_wait(bar2, phase)) failed = true;
       s1::fence_after_sync();
-      uint32_t words[2];
-#pragma unroll
+      const bool nzk = zf[R] != 0;
+#pragma unroll 1
       for (int h = 0; h < 2; ++h) {
         uint32_t v[32];
         s1::tmem_ld32(tmem_p + lane_base + 64 * ch + 32 * h, v);
@@ -1031,11 +1031,8 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
         for (int k = 7; k >= 0; --k)
 #pragma unroll
           for (int g = 0; g < 4; ++g) b4[g] = __funnelshift_l(v[8 * g + k] ^ 0x80000000u, b4[g], 1);
-        words[h] = b4[0] | (b4[1] << 8) | (b4[2] << 16) | (b4[3] << 24);
-      }
-      if (valid) {
-        const uint2 w2 = zf[R] ? make_uint2(words[0], words[1]) : make_uint2(0u, 0u);
-        *reinterpret_cast<uint2*>(a.k_signs + i * 16 + 8 * ch) = w2;
+        const uint32_t word = b4[0] | (b4[1] << 8) | (b4[2] << 16) | (b4[3] << 24);
+        if (valid) reinterpret_cast<uint32_t*>(a.k_signs + i * 16 + 8 * ch)[h] = nzk ? word : 0u;
       }
       s1::fence_before_sync();
     } else if (!key_warp && a.v) {
