@@ -107,6 +107,25 @@ def recorded_traffic(kernel_file: str, sha: str, units: int):
         return None
 
 
+# ---------------------------------------------------------------------- ranks
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Slowest rank's value (all-reduce MAX over the default process group)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, slowest_seconds: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time
+    (weak scaling: every rank processes the same units)."""
+    return world * units_per_rank / slowest_seconds
+
+
 # ---------------------------------------------------------------------- inputs
 
 def host_inputs(w: W.Workload, rank: int):
@@ -269,12 +288,8 @@ def run_ours(args, w: W.Workload):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def slowest(x: float) -> float:
+        return max_over_ranks(x, world, dev)
 
     # --- method tables and inputs
     dr = W.method_draws(w.d, w.m)
@@ -386,11 +401,11 @@ def run_ours(args, w: W.Workload):
     comp_k = [e[1].elapsed_time(e[2]) for e in kevs]
     dec = [e[4].elapsed_time(e[7]) for e in evs]
     dec_k = [e[5].elapsed_time(e[6]) for e in kevs]
-    dec_total = max_over_ranks(sum(dec) / 1e3)
-    comp_total = max_over_ranks(sum(comp) / 1e3)
-    dec_k_mean = max_over_ranks(statistics.fmean(dec_k) / 1e3)
-    gbs = world * packed_bytes * args.steps / dec_total / 1e9
-    vps = world * 2 * n_vec * args.steps / comp_total if not args.decode_only else None
+    dec_total = slowest(sum(dec) / 1e3)
+    comp_total = slowest(sum(comp) / 1e3)
+    dec_k_mean = slowest(statistics.fmean(dec_k) / 1e3)
+    gbs = job_throughput(packed_bytes * args.steps, world, dec_total) / 1e9
+    vps = job_throughput(2 * n_vec * args.steps, world, comp_total) if not args.decode_only else None
 
     # --- end to end through the public API with host buffers
     e2e = None
@@ -419,9 +434,9 @@ def run_ours(args, w: W.Workload):
             e2e_step()
         s1.record()
         torch.cuda.synchronize()
-        e2e_s = max_over_ranks(s0.elapsed_time(s1) / 1e3)
+        e2e_s = slowest(s0.elapsed_time(s1) / 1e3)
         h2d = Kp.numel() * Kp.element_size() + Vp.numel() * Vp.element_size() + Qp.numel() * Qp.element_size()
-        e2e = {"value": world * packed_bytes * args.e2e_steps / e2e_s / 1e9, "unit": "GB/s",
+        e2e = {"value": job_throughput(packed_bytes * args.e2e_steps, world, e2e_s) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(outp.numel() * 4),
                "ms_per_step": 1e3 * e2e_s / args.e2e_steps}
 
