@@ -8,6 +8,7 @@
 //
 // One warp owns one vector; lane l holds coordinates [l*E, l*E+E), E = d/32, so
 // every global load and store of a record is a contiguous warp-wide access.
+#include <cuda.h>  // CUtensorMap and its enums (types only: the encoder is fetched at run time)
 #include <cuda_runtime.h>
 
 #include <cstring>
@@ -37,6 +38,8 @@ struct CompressArgs {
   Codebook cb;
   int lm_bits, m, v_bits, rot;
   float inv_sqrt_d;  // 1/sqrt(d) rounded once from fp64
+  CUtensorMap kmap;  // compress_pipe_kernel: bf16 keys [n_vec][128], 64 x 128 boxes, 128-byte swizzle
+  CUtensorMap vmap;  // compress_pipe_kernel: bf16 values [n_vec][128], 64 x 64 boxes, 128-byte swizzle
 };
 
 // Norm, rotation, Lloyd-Max codes and residual of key i; writes the packed codes
@@ -1166,6 +1169,531 @@ cudaError_t launch_rot(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s)
   return vb == 2 ? launch_rot_t<3, 2, HAAR>(ctx, a, s) : launch_rot_t<3, 4, HAAR>(ctx, a, s);
 }
 
+// ---------------------------------------------------------------------------------
+// bf16 keys, randomized Hadamard rotation, d = m = 128, and a codebook symmetric about
+// zero (c[L-1-k] = -c[k], t[L-2-k] = -t[k]; the sphere Lloyd-Max codebook is). The
+// arithmetic is that of compress_rot_kernel; the organisation lets consecutive passes
+// of 128 vectors overlap:
+//  * the key rows arrive by TMA straight into one of two swizzled operand tiles, two
+//    passes ahead;
+//  * the rotation MMA of pass i+1 (into the other half of a double-buffered Y in tensor
+//    memory) runs while the key warps work on pass i, and the projection MMA of pass i
+//    (into a double-buffered S r) while they read out the signs of pass i-1 and start on
+//    pass i+1;
+//  * the value warps run a loop of their own over the same passes, with the value rows
+//    in two half buffers (TMA, 128-byte swizzle, so that the four threads of a row and
+//    the eight rows of a warp read distinct banks): one half is refilled while the other
+//    is quantized.
+// Both threads of a key row compute ||Y||^2 over all 128 columns (no exchange); the
+// residual's squared norm is exchanged through shared memory at the one key-warp
+// barrier of a pass. With the symmetric codebook a coordinate is bucketized on its
+// magnitude and the code's bits follow from its sign; everything is scaled by 16 (an
+// exact power of two) so that the residual comes out as the x16 operand directly.
+constexpr int kPipeThreads = 512;
+
+struct PipeSmem {
+  static constexpr uint32_t KT = 0;                         // [2] key operand tiles (TMA, 128B swizzle)
+  static constexpr uint32_t HB = 2 * kTcTileBytes;          // H diag(sigma), bf16 operand tile
+  static constexpr uint32_t S = 3 * kTcTileBytes;           // QJL matrix, f16 operand tile
+  static constexpr uint32_t A_HI = 4 * kTcTileBytes, A_LO = 5 * kTcTileBytes;  // residual x16
+  static constexpr uint32_t VR = 6 * kTcTileBytes;          // value rows: two halves of 64 (2 swizzled panels)
+  static constexpr uint32_t XR = 7 * kTcTileBytes;          // [2 passes][2 halves][128] sums of r^2
+  static constexpr uint32_t ZF = XR + 2 * 2 * 128 * 4;      // [2 passes][128] nonzero-key flags
+  static constexpr uint32_t BAR = ZF + 2 * 128;             // eight mbarriers
+  static constexpr uint32_t TMEM = BAR + 64;                // TMEM base address
+  static constexpr uint32_t BYTES = TMEM + 8;
+  // The block's dynamic shared memory starts 1024-byte aligned (checked at run time):
+  // the tiles need that alignment and there is no room for padding.
+  static_assert(BYTES <= 227 * 1024, "compress_pipe_kernel shared memory");
+};
+
+// Adds the NB-bit field v at bit offset o of the words w (fields start zero, so add
+// acts as or, and compiles to one integer multiply-add).
+template <int NB, int NW>
+__device__ __forceinline__ void add_field(uint32_t (&w)[NW], int o, uint32_t v) {
+  const int wi = o >> 5, sh = o & 31;
+  w[wi] += v << sh;
+  if (sh + NB > 32) w[wi + 1] += v >> (32 - sh);
+}
+
+// Bucketize y (x16 domain) with a symmetric codebook: magnitude thresholds tm and
+// levels cm (the upper half of t and c, x16). Returns the centroid and sets the code.
+template <int LMB>
+__device__ __forceinline__ float bucket_sym(float y, const float* tm, const float* cm, uint32_t& code) {
+  constexpr int L = 1 << LMB, HL = L / 2;
+  const float a = fabsf(y);
+  uint32_t im = HL;
+  float mag = cm[0];
+#pragma unroll
+  for (int j = 0; j < HL - 1; ++j) {
+    if (a >= tm[j]) {
+      im = HL + j + 1;
+      mag = cm[j + 1];
+    }
+  }
+  const uint32_t yb = __float_as_uint(y);
+  const uint32_t neg = (uint32_t)((int32_t)yb >> 31);  // all ones for a negative y
+  code = im ^ (neg & (uint32_t)(L - 1));               // lower half: L - 1 - im
+  return __uint_as_float(__float_as_uint(mag) | (yb & 0x80000000u));
+}
+
+template <int LMB, int VB>
+__global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __grid_constant__ CompressArgs a) {
+  using PS = PipeSmem;
+  namespace s1 = tq::sm100;
+  constexpr int L = 1 << LMB, HL = L / 2;
+  extern __shared__ __align__(1024) unsigned char smem_pipe[];
+  unsigned char* sm = smem_pipe;
+  if (s1::smem_u32(sm) & 1023u) {  // the layout needs it; report instead of misaddressing
+    if (threadIdx.x == 0) atomicOr(a.err, 2u);
+    return;
+  }
+  const uint32_t sbase = s1::smem_u32(sm);
+  float* xr = reinterpret_cast<float*>(sm + PS::XR);
+  uint8_t* zf = sm + PS::ZF;
+  uint64_t* kfull = reinterpret_cast<uint64_t*>(sm + PS::BAR);  // [2] key tile landed
+  uint64_t* rotd = kfull + 2;                                        // [2] rotation into Y[b] done
+  uint64_t* projd = kfull + 4;                                       // projection done
+  uint64_t* vfull = kfull + 5;                                       // [2] value half landed
+  uint64_t* fin = kfull + 7;                                         // failure path: MMAs drained
+  uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + PS::TMEM);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t ntile = (a.n_vec + 127) / 128, g = gridDim.x;
+
+  if (warp == 0) {
+    s1::tmem_alloc(tmem_s, 512);
+    s1::tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int k = 0; k < 8; ++k) s1::mbar_init(kfull + k, 1);
+    s1::mbar_init_fence();
+  }
+  {  // H diag(sigma) and S operand tiles, prepacked on the host
+    const uint4* hsrc = reinterpret_cast<const uint4*>(a.H_sw128);
+    const uint4* ssrc = reinterpret_cast<const uint4*>(a.S_sw128);
+    uint4* hdst = reinterpret_cast<uint4*>(sm + PS::HB);
+    uint4* sdst = reinterpret_cast<uint4*>(sm + PS::S);
+    for (int w = tid; w < (int)(kTcTileBytes / 16); w += kPipeThreads) {
+      sdst[w] = ssrc[w];
+      hdst[w] = hsrc[w];
+    }
+  }
+  s1::fence_async_smem();
+  s1::fence_before_sync();
+  __syncthreads();
+  s1::fence_after_sync();
+  const uint32_t tmem = *tmem_s;  // columns 0..255: Y[2]; 256..511: S r [2]
+  bool failed = false;
+
+  if (warp < 8) {
+    // ================================================================ keys
+    if (a.k) {
+      const int sp = warp & 3, ch = warp >> 2;  // TMEM sub-partition, column half
+      const int R = 32 * sp + lane;             // key (row) within the pass
+      const uint32_t lane_base = (uint32_t)(32 * sp) << 16;
+      float tm[HL > 1 ? HL - 1 : 1], cm[HL];
+#pragma unroll
+      for (int j = 0; j < HL - 1; ++j) tm[j] = 16.f * a.cb.t[HL + j];
+#pragma unroll
+      for (int j = 0; j < HL; ++j) cm[j] = 16.f * a.cb.c[HL + j];
+      // TMA bookkeeping (thread 0), bit b for key buffer b: next parity, load outstanding
+      uint32_t kpar = 0u, kpend = 0u;
+      auto load_keys = [&](int b, int64_t tile) {
+        s1::mbar_expect_tx(kfull + b, 2u * 128u * 128u);
+        s1::tma_load_2d(sm + PS::KT + b * kTcTileBytes, &a.kmap, 0, (int)(tile * 128), kfull + b);
+        s1::tma_load_2d(sm + PS::KT + b * kTcTileBytes + kTcTileBytes / 2, &a.kmap, 64, (int)(tile * 128),
+                        kfull + b);
+        kpend |= 1u << b;
+      };
+      auto wait_keys = [&](int b) -> bool {
+        if (!s1::mbar_wait(kfull + b, (kpar >> b) & 1u)) return false;
+        kpar ^= 1u << b;
+        kpend &= ~(1u << b);
+        return true;
+      };
+      auto issue_rotation = [&](int b) {
+        constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          s1::umma_f16(tmem + 128 * b, s1::sw128_desc(sbase + PS::KT + b * kTcTileBytes, 16 * ks, 128),
+                       s1::sw128_desc(sbase + PS::HB, 16 * ks, 128), idesc, ks > 0 ? 1u : 0u);
+        s1::umma_commit(rotd + b);
+      };
+      // Sign readout of a pass whose projection has completed: bit j set <=> (S r)_j >= 0.
+      auto read_signs = [&](int b, int64_t pv0) {
+        const int64_t pi = pv0 + R;
+        const bool nzk = zf[b * 128 + R] != 0;
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          uint32_t v[32];
+          s1::tmem_ld32(tmem + 256 + 128 * b + lane_base + 64 * ch + 32 * h, v);
+          s1::tmem_ld_wait();
+          uint32_t b4[4] = {0u, 0u, 0u, 0u};  // sign bits, four independent 8-bit chains
+#pragma unroll
+          for (int k = 7; k >= 0; --k)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) b4[q] = __funnelshift_l(v[8 * q + k], b4[q], 1);
+          const uint32_t word = ~(b4[0] | (b4[1] << 8) | (b4[2] << 16) | (b4[3] << 24));
+          if (pi < a.n_vec) reinterpret_cast<uint32_t*>(a.k_signs + pi * 16 + 8 * ch)[h] = nzk ? word : 0u;
+        }
+      };
+
+      if (tid == 0 && (int64_t)blockIdx.x < ntile) {
+        load_keys(0, blockIdx.x);
+        if (blockIdx.x + g < ntile) load_keys(1, blockIdx.x + g);
+        if (wait_keys(0)) {
+          s1::fence_after_sync();
+          issue_rotation(0);
+        } else {
+          failed = true;
+        }
+      }
+      __syncwarp();  // warp 0 converged again before its tensor-memory loads
+      int it = 0;
+      int64_t prev_v0 = 0;
+      for (int64_t tile = blockIdx.x; tile < ntile; tile += g, ++it) {
+        const int b = it & 1;
+        const int64_t v0 = tile * 128, i = v0 + R;
+        const bool valid = i < a.n_vec;
+        if (!failed && !s1::mbar_wait(rotd + b, (uint32_t)(it >> 1) & 1u)) failed = true;
+        s1::fence_after_sync();
+        if (tid == 0 && !failed) {
+          // KT[b] has been read by the rotation just waited for: refill it two passes ahead;
+          // then start the next pass's rotation into Y[b ^ 1] (read last pass, before the
+          // barrier that ended it).
+          if (tile + 2 * g < ntile) load_keys(b, tile + 2 * g);
+          if (tile + g < ntile) {
+            if (wait_keys(b ^ 1)) issue_rotation(b ^ 1);
+            else failed = true;
+          }
+        }
+        __syncwarp();
+        // ||Y||^2 over the row's 128 columns, as two 64-column halves of four chains each
+        float hs[2];
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
+          float2 s01 = make_float2(0.f, 0.f), s23 = make_float2(0.f, 0.f);
+#pragma unroll 1
+          for (int h = 0; h < 2; ++h) {
+            uint32_t v[32];
+            s1::tmem_ld32(tmem + 128 * b + lane_base + 64 * c2 + 32 * h, v);
+            s1::tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              const float2 y01 = make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+              const float2 y23 = make_float2(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+              s01 = s1::fma2(y01, y01, s01);
+              s23 = s1::fma2(y23, y23, s23);
+            }
+          }
+          hs[c2] = (s01.x + s01.y) + (s23.x + s23.y);
+        }
+        const float tot = hs[0] + hs[1];  // ||Y||^2 = d ||k||^2
+        const bool nz = tot > 0.f;
+        const float sc16 = nz ? 16.f * (1.0f / sqrtf(tot)) : 0.f;
+        const float2 sc2 = make_float2(sc16, sc16);
+        // the previous projection has finished: A tiles free, its S r readable
+        if (it > 0 && !failed && !s1::mbar_wait(projd, (uint32_t)(it - 1) & 1u)) failed = true;
+        s1::fence_after_sync();
+        float2 ra = make_float2(0.f, 0.f), rb = make_float2(0.f, 0.f);  // r^2 chains (0,1), (2,3)
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          uint32_t v[32];
+          s1::tmem_ld32(tmem + 128 * b + lane_base + 64 * ch + 32 * h, v);
+          s1::tmem_ld_wait();
+          uint32_t cw[LMB], cw2[LMB];  // even / odd codes: two independent chains per word
+#pragma unroll
+          for (int w = 0; w < LMB; ++w) cw[w] = cw2[w] = 0u;
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            uint32_t hw[4], lw[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+              const int e = 8 * c8 + 2 * p;
+              const float2 yy = s1::mul2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), sc2);
+              uint32_t q0, q1;
+              const float c0 = bucket_sym<LMB>(yy.x, tm, cm, q0);
+              const float c1 = bucket_sym<LMB>(yy.y, tm, cm, q1);
+              add_field<LMB, LMB>(cw, LMB * e, q0);
+              add_field<LMB, LMB>(cw2, LMB * (e + 1), q1);
+              const float2 r = s1::sub2(yy, make_float2(c0, c1));  // residual x16
+              if (p & 1) rb = s1::fma2(r, r, rb);
+              else ra = s1::fma2(r, r, ra);
+              const __half2 hh = __floats2half2_rn(r.x, r.y);
+              const float2 lo = s1::sub2(r, __half22float2(hh));
+              const __half2 ll = __floats2half2_rn(lo.x, lo.y);
+              hw[p] = *reinterpret_cast<const uint32_t*>(&hh);
+              lw[p] = *reinterpret_cast<const uint32_t*>(&ll);
+            }
+            const uint32_t off = s1::sw128_offset(R, 64 * ch + 32 * h + 8 * c8, 128);
+            *reinterpret_cast<uint4*>(sm + PS::A_HI + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            *reinterpret_cast<uint4*>(sm + PS::A_LO + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+          }
+          if (valid) {
+            uint32_t* co = reinterpret_cast<uint32_t*>(a.k_codes + i * (LMB * 16) + ch * (LMB * 8) + h * (LMB * 4));
+#pragma unroll
+            for (int w = 0; w < LMB; ++w) co[w] = nz ? (cw[w] | cw2[w]) : 0u;
+          }
+        }
+        xr[b * 256 + ch * 128 + R] = (ra.x + ra.y) + (rb.x + rb.y);
+        s1::fence_async_smem();
+        s1::fence_before_sync();
+        failed = s1::bar_sync_or<1, 256>(failed);
+        s1::fence_after_sync();
+        if (failed) break;
+        if (ch == 0) {
+          const float gamma = sqrtf(xr[b * 256 + R] + xr[b * 256 + 128 + R]) * (1.f / 16.f);
+          if (valid) {
+            const uint32_t nb = __half_as_ushort(__float2half_rn(sqrtf(tot * (1.0f / 128.f))));
+            const uint32_t gb = __half_as_ushort(__float2half_rn(gamma));
+            reinterpret_cast<uint32_t*>(a.k_norms)[i] = nz ? (nb | (gb << 16)) : 0u;
+          }
+          zf[b * 128 + R] = (valid && nz) ? 1 : 0;
+        }
+        if (tid == 0) {
+          constexpr uint32_t idesc = s1::idesc_f16_f32(128, 128);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            s1::umma_f16(tmem + 256 + 128 * b, s1::sw128_desc(sbase + PS::A_HI, 16 * ks, 128),
+                         s1::sw128_desc(sbase + PS::S, 16 * ks, 128), idesc, ks > 0 ? 1u : 0u);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            s1::umma_f16(tmem + 256 + 128 * b, s1::sw128_desc(sbase + PS::A_LO, 16 * ks, 128),
+                         s1::sw128_desc(sbase + PS::S, 16 * ks, 128), idesc, 1u);
+          s1::umma_commit(projd);
+        }
+        __syncwarp();
+        if (it > 0) read_signs(b ^ 1, prev_v0);
+        s1::fence_before_sync();
+        prev_v0 = v0;
+      }
+      // the last pass's signs (its nonzero flags were written after the last barrier)
+      failed = s1::bar_sync_or<1, 256>(failed);
+      if (!failed && it > 0) {
+        if (!s1::mbar_wait(projd, (uint32_t)(it - 1) & 1u)) {
+          failed = true;
+        } else {
+          s1::fence_after_sync();
+          read_signs((it - 1) & 1, prev_v0);
+        }
+      }
+      if (failed && tid == 0) {
+        // bounded: drain this thread's MMAs and its outstanding key loads before the
+        // shared and tensor memory they use is released
+        s1::umma_commit(fin);
+        s1::mbar_wait(fin, 0u);
+        for (int b = 0; b < 2; ++b)
+          if ((kpend >> b) & 1u) s1::mbar_wait(kfull + b, (kpar >> b) & 1u);
+      }
+    }
+  } else if (a.v) {
+    // ================================================================ values
+    const int vt = tid - 256, q = vt & 3, vrow = vt >> 2;  // 4 threads per value, 64 per half
+    const bool leader = vt == 0;
+    uint32_t vpar = 0u, vpend = 0u;  // bit h for value half h: next parity, copy outstanding
+    // half h of a pass: rows 64h..64h+63 as two 64-column panels of 64 rows x 128 bytes
+    auto fetch_half = [&](int64_t tile, int h) {
+      const int64_t r0 = tile * 128 + 64 * h;
+      if (r0 >= a.n_vec) return;
+      unsigned char* dst = sm + PS::VR + h * (kTcTileBytes / 2);
+      s1::mbar_expect_tx(vfull + h, 64u * 128u * 2u);
+      s1::tma_load_2d(dst, &a.vmap, 0, (int)r0, vfull + h);
+      s1::tma_load_2d(dst + kTcTileBytes / 4, &a.vmap, 64, (int)r0, vfull + h);
+      vpend |= 1u << h;
+    };
+    // byte offset, within a half, of this thread's 16-byte chunk k (coordinates 32q + 8k ..)
+    const int vsw = vrow & 7;
+    auto chunk_off = [&](int k) -> uint32_t {
+      return (uint32_t)((q >> 1) * (kTcTileBytes / 4) + vrow * 128 + (((4 * (q & 1) + k) ^ vsw) << 4));
+    };
+    if (leader && (int64_t)blockIdx.x < ntile) {
+      fetch_half(blockIdx.x, 0);
+      fetch_half(blockIdx.x, 1);
+    }
+    constexpr int levels = (1 << VB) - 1;
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
+    // sum over a word's fields of the magic constant's bits shifted into place (mod 2^32)
+    uint32_t magic_sum = 0u;
+#pragma unroll
+    for (int f = 0; f < 32 / VB; ++f) magic_sum += __float_as_uint(kMagic) << (VB * f);
+    for (int64_t tile = blockIdx.x; tile < ntile && !failed; tile += g) {
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        const int64_t r0 = tile * 128 + 64 * h;
+        if (r0 >= a.n_vec) break;  // the same for every value thread
+        if (!failed) {
+          if (s1::mbar_wait(vfull + h, (vpar >> h) & 1u)) {
+            vpar ^= 1u << h;
+            vpend &= ~(1u << h);
+          } else {
+            failed = true;
+          }
+        }
+        const int64_t i = r0 + vrow;
+        if (!failed && i < a.n_vec) {
+          const unsigned char* half = sm + PS::VR + h * (kTcTileBytes / 2);
+          uint32_t w[16];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint4 u = *reinterpret_cast<const uint4*>(half + chunk_off(k));
+            w[4 * k] = u.x;
+            w[4 * k + 1] = u.y;
+            w[4 * k + 2] = u.z;
+            w[4 * k + 3] = u.w;
+          }
+          // min / max on the packed bf16 pairs (exact: bf16 -> fp32 is monotone)
+          __nv_bfloat162 mn = *reinterpret_cast<const __nv_bfloat162*>(&w[0]), mx = mn;
+#pragma unroll
+          for (int k = 1; k < 16; ++k) {
+            const __nv_bfloat162 x2 = *reinterpret_cast<const __nv_bfloat162*>(&w[k]);
+            mn = __hmin2(mn, x2);
+            mx = __hmax2(mx, x2);
+          }
+          const float lo = fminf(__low2float(mn), __high2float(mn));
+          const float hi = fmaxf(__low2float(mx), __high2float(mx));
+          // scale in fp64 as the reference quantizer; codes rounded to nearest by adding
+          // 1.5 * 2^23, redone in fp64 with floor(t + 1/2) within 1e-5 of a half step.
+          const double dlo = lo, span = (double)hi - dlo;
+          const float inv = span > 0.0 ? (float)(levels / span) : 0.f;
+          const float2 lo2 = make_float2(lo, lo), inv2 = make_float2(inv, inv), mg2 = make_float2(kMagic, kMagic);
+          uint32_t vw[VB], vw2[VB];
+#pragma unroll
+          for (int k = 0; k < VB; ++k) vw[k] = vw2[k] = 0u;
+          bool near = false;
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const float2 x = make_float2(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xffff0000u));
+            const float2 t = s1::mul2(s1::sub2(x, lo2), inv2);
+            const float2 tr = s1::add2(t, mg2);
+            const float2 e = s1::sub2(t, s1::sub2(tr, mg2));
+            near |= fabsf(e.x) > 0.5f - 1e-5f;
+            near |= fabsf(e.y) > 0.5f - 1e-5f;
+            // tr's bits are those of the magic constant plus the code
+            add_field<VB, VB>(vw, VB * 2 * k, __float_as_uint(tr.x));
+            add_field<VB, VB>(vw2, VB * (2 * k + 1), __float_as_uint(tr.y));
+          }
+#pragma unroll
+          for (int k = 0; k < VB; ++k) vw[k] = vw[k] + vw2[k] - magic_sum;
+          uint32_t* vo = reinterpret_cast<uint32_t*>(a.v_codes + i * (VB * 16) + q * (VB * 4));
+#pragma unroll
+          for (int k = 0; k < VB; ++k) vo[k] = vw[k];
+          if (near) {
+            // Some coordinate lies within 1e-5 of a half step (with bf16 inputs a ratio of
+            // small integers often lands exactly on one): find which, and redo only those
+            // in fp64 as floor(t + 1/2), patching the words just stored.
+            uint32_t mask = 0u;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const uint32_t wk = *reinterpret_cast<const uint32_t*>(half + chunk_off(k >> 2) + 4 * (k & 3));
+              const float2 x = make_float2(__uint_as_float(wk << 16), __uint_as_float(wk & 0xffff0000u));
+              const float2 t = s1::mul2(s1::sub2(x, lo2), inv2);
+              const float2 e = s1::sub2(t, s1::sub2(s1::add2(t, mg2), mg2));
+              if (fabsf(e.x) > 0.5f - 1e-5f) mask |= 1u << (2 * k);
+              if (fabsf(e.y) > 0.5f - 1e-5f) mask |= 2u << (2 * k);
+            }
+            while (mask) {
+              const int e = __ffs(mask) - 1;
+              mask &= mask - 1u;
+              const float xe = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                  half + chunk_off(e >> 3) + 2 * (e & 7)));
+              const uint32_t qf = __float_as_uint((xe - lo) * inv + kMagic) & 0xffu;  // the fast code
+              const uint32_t qv =
+                  min((uint32_t)floor(((double)xe - dlo) * (levels / span) + 0.5), (uint32_t)levels);
+              vo[(VB * e) >> 5] ^= (qf ^ qv) << ((VB * e) & 31);
+            }
+          }
+          const uint32_t sb = __half_as_ushort(__double2half(span / levels));
+          const uint32_t mb = __half_as_ushort(__float2half_rn(lo));
+          reinterpret_cast<uint32_t*>(a.v_params)[i * 4 + q] = sb | (mb << 16);
+        }
+        // every value thread is done with this half: refill it for the next pass
+        failed = s1::bar_sync_or<2, 256>(failed);
+        if (failed) break;
+        if (leader && tile + g < ntile) {
+          s1::fence_async_smem();
+          fetch_half(tile + g, h);
+        }
+      }
+    }
+    if (failed && leader)
+      for (int h = 0; h < 2; ++h)
+        if ((vpend >> h) & 1u) s1::mbar_wait(vfull + h, (vpar >> h) & 1u);  // bounded
+  }
+  if (__syncthreads_or(failed) && tid == 0) atomicOr(a.err, 1u);
+  s1::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    s1::fence_after_sync();
+    s1::tmem_dealloc(tmem, 512);
+  }
+}
+
+// cuTensorMapEncodeTiled, fetched once from the driver through the runtime.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn tensor_map_encoder() {
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// A tensor map of compress_pipe_kernel: [n_vec][128] bf16 rows, boxes of 64 columns x
+// box_rows rows (one 128-byte-swizzled panel each). False if it cannot be made.
+bool encode_rows_map(CUtensorMap* map, const void* k, int64_t n_vec, uint32_t box_rows) {
+  const EncodeTiledFn enc = tensor_map_encoder();
+  if (!enc || n_vec <= 0 || n_vec >= ((int64_t)1 << 31)) return false;
+  const cuuint64_t dims[2] = {128, (cuuint64_t)n_vec};
+  const cuuint64_t strides[1] = {128 * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(k), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// c[L-1-k] == -c[k] and t[L-2-k] == -t[k] exactly.
+bool codebook_symmetric(const Codebook& cb, int lm_bits) {
+  const int L = 1 << lm_bits;
+  for (int k = 0; k < L; ++k)
+    if (cb.c[L - 1 - k] != -cb.c[k]) return false;
+  for (int k = 0; k < L - 1; ++k)
+    if (cb.t[L - 2 - k] != -cb.t[k]) return false;
+  return true;
+}
+
+template <int LMB, int VB>
+cudaError_t launch_pipe_t(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) {
+  static bool configured = false;
+  const size_t smem = PipeSmem::BYTES;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(compress_pipe_kernel<LMB, VB>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  int64_t blocks = (a.n_vec + 127) / 128;
+  if (blocks > ctx->num_sms) blocks = ctx->num_sms;
+  if (ctx->prof_start) cudaEventRecord(ctx->prof_start, s);
+  compress_pipe_kernel<LMB, VB><<<(unsigned)blocks, kPipeThreads, smem, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (ctx->prof_stop) cudaEventRecord(ctx->prof_stop, s);
+  return e;
+}
+
+cudaError_t launch_pipe(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) {
+  const int lmb = ctx->shape.lm_bits, vb = ctx->shape.v_bits;
+  if (lmb == 1) return vb == 2 ? launch_pipe_t<1, 2>(ctx, a, s) : launch_pipe_t<1, 4>(ctx, a, s);
+  if (lmb == 2) return vb == 2 ? launch_pipe_t<2, 2>(ctx, a, s) : launch_pipe_t<2, 4>(ctx, a, s);
+  return vb == 2 ? launch_pipe_t<3, 2>(ctx, a, s) : launch_pipe_t<3, 4>(ctx, a, s);
+}
+
 }  // namespace
 
 // S as f16 in the swizzled K-major operand layout of compress_tc_kernel, or false if
@@ -1249,8 +1777,12 @@ cudaError_t launch_compress(const tq_ctx* ctx, const void* k, const void* v, int
   a.H_sw128 = ctx->H_sw128;
   a.err = ctx->d_err;
   if (ctx->S_sw128 && ctx->shape.d == 128 && ctx->shape.m == 128) {
-    if (ctx->shape.rot == TQ_ROT_HADAMARD && dtype == TQ_BF16 && ctx->H_sw128)
+    if (ctx->shape.rot == TQ_ROT_HADAMARD && dtype == TQ_BF16 && ctx->H_sw128) {
+      if (codebook_symmetric(ctx->cb, ctx->shape.lm_bits) && (!k || encode_rows_map(&a.kmap, k, n_vec, 128)) &&
+          (!v || encode_rows_map(&a.vmap, v, n_vec, 64)))
+        return launch_pipe(ctx, a, stream);
       return launch_rot<false>(ctx, a, stream);
+    }
     if (ctx->shape.rot == TQ_ROT_HAAR && dtype == TQ_BF16 && ctx->Pi_sw128) {
       a.H_sw128 = ctx->Pi_sw128;
       return launch_rot<true>(ctx, a, stream);

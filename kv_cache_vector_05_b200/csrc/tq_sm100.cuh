@@ -60,6 +60,63 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// 2-D tiled TMA load of the box at element coordinates (x, y) of the tensor described by
+// `map` (a kernel parameter) into shared memory, completing its bytes on `bar`. The
+// caller keeps x * element size a multiple of 16 bytes; rows past the tensor's end are
+// filled with zeros and still counted in the transaction bytes.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Named barrier `id` over `count` threads that also ORs a predicate across them.
+template <int ID, int COUNT>
+__device__ __forceinline__ bool bar_sync_or(bool p) {
+  uint32_t r;
+  asm volatile(
+      "{ .reg .pred q, o; setp.ne.u32 q, %1, 0; bar.red.or.pred o, %2, %3, q; selp.u32 %0, 1, 0, o; }"
+      : "=r"(r)
+      : "r"((uint32_t)p), "n"(ID), "n"(COUNT)
+      : "memory");
+  return r != 0;
+}
+
+// ---- paired fp32 arithmetic (one instruction for two lanes of a float2) ------------
+
+__device__ __forceinline__ unsigned long long f2_bits(float2 v) {
+  return (unsigned long long)__float_as_uint(v.x) | ((unsigned long long)__float_as_uint(v.y) << 32);
+}
+__device__ __forceinline__ float2 f2_from(unsigned long long b) {
+  return make_float2(__uint_as_float((uint32_t)b), __uint_as_float((uint32_t)(b >> 32)));
+}
+// a * b, each lane rounded to nearest
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return f2_from(d);
+}
+// a - b, each lane rounded to nearest
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  unsigned long long d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return f2_from(d);
+}
+// a + b, each lane rounded to nearest
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return f2_from(d);
+}
+// a * b + c, each lane fused and rounded once
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+  return f2_from(d);
+}
+
 // ---- tensor memory -----------------------------------------------------------------
 
 // One full warp: allocate `ncols` (power of two >= 32) columns; the TMEM address is
