@@ -174,10 +174,9 @@ tq_status tq_decode_attention(const tq_ctx* ctx, const void* q, tq_dtype q_dtype
 /* Synchronize `stream`, then read and clear the context's device error word.
  * Kernels never spin without a bound: a wait for a staged copy that does not
  * complete in time sets this word, abandons the rest of its work and exits, so
- * the CUDA context stays usable. A compression kernel whose shared memory is not
- * 1024-byte aligned (its tiles need it) also sets the word and does nothing.
- * Returns TQ_ECUDA (with tq_last_error() saying which) if any call since the
- * last check hit either, TQ_OK otherwise. */
+ * the CUDA context stays usable. Returns TQ_ECUDA (with tq_last_error() saying
+ * which wait) if any call since the last check hit such a timeout, TQ_OK
+ * otherwise. */
 tq_status tq_check_device(const tq_ctx* ctx, void* stream);
 
 /* Decode attention that allocates nothing and takes no workspace. The paper has

@@ -1173,39 +1173,40 @@ cudaError_t launch_rot(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s)
 // bf16 keys, randomized Hadamard rotation, d = m = 128, and a codebook symmetric about
 // zero (c[L-1-k] = -c[k], t[L-2-k] = -t[k]; the sphere Lloyd-Max codebook is). The
 // arithmetic is that of compress_rot_kernel; the organisation lets consecutive passes
-// of 128 vectors overlap:
+// of 128 vectors overlap and keeps the tensor cores' shared-memory reads low:
 //  * the key rows arrive by TMA straight into one of two swizzled operand tiles, two
 //    passes ahead;
 //  * the rotation MMA of pass i+1 (into the other half of a double-buffered Y in tensor
-//    memory) runs while the key warps work on pass i, and the projection MMA of pass i
-//    (into a double-buffered S r) while they read out the signs of pass i-1 and start on
-//    pass i+1;
+//    memory) runs while the key warps work on pass i;
+//  * the residual's f16 hi / lo operand goes to tensor memory (tcgen05.st), so the
+//    projection MMA reads only S from shared memory; it runs while the key warps start
+//    on the next pass, which reads its signs out before overwriting the operand;
 //  * the value warps run a loop of their own over the same passes, with the value rows
-//    in two half buffers (TMA, 128-byte swizzle, so that the four threads of a row and
-//    the eight rows of a warp read distinct banks): one half is refilled while the other
-//    is quantized.
+//    in four half buffers (two passes of two halves; TMA, 128-byte swizzle, so that the
+//    four threads of a row and the eight rows of a warp read distinct banks), each
+//    refilled two passes ahead.
 // Both threads of a key row compute ||Y||^2 over all 128 columns (no exchange); the
 // residual's squared norm is exchanged through shared memory at the one key-warp
 // barrier of a pass. With the symmetric codebook a coordinate is bucketized on its
 // magnitude and the code's bits follow from its sign; everything is scaled by 16 (an
 // exact power of two) so that the residual comes out as the x16 operand directly.
 constexpr int kPipeThreads = 512;
+constexpr int kProjIssuer = 128;  // first thread of key warp 4 (thread 0 issues the rotation)
 
 struct PipeSmem {
   static constexpr uint32_t KT = 0;                         // [2] key operand tiles (TMA, 128B swizzle)
   static constexpr uint32_t HB = 2 * kTcTileBytes;          // H diag(sigma), bf16 operand tile
   static constexpr uint32_t S = 3 * kTcTileBytes;           // QJL matrix, f16 operand tile
-  static constexpr uint32_t A_HI = 4 * kTcTileBytes, A_LO = 5 * kTcTileBytes;  // residual x16
-  static constexpr uint32_t VR = 6 * kTcTileBytes;          // value rows: two halves of 64 (2 swizzled panels)
-  static constexpr uint32_t XR = 7 * kTcTileBytes;          // [2 passes][2 halves][128] sums of r^2
-  static constexpr uint32_t ZF = XR + 2 * 2 * 128 * 4;      // [2 passes][128] nonzero-key flags
-  static constexpr uint32_t BAR = ZF + 2 * 128;             // eight mbarriers
-  static constexpr uint32_t TMEM = BAR + 64;                // TMEM base address
+  static constexpr uint32_t VR = 4 * kTcTileBytes;          // [2 passes][2 halves] value rows (2 panels each)
+  static constexpr uint32_t XR = 6 * kTcTileBytes;          // [2 passes][2 halves][128] sums of r^2
+  static constexpr uint32_t BAR = XR + 2 * 2 * 128 * 4;     // eleven mbarriers
+  static constexpr uint32_t TMEM = BAR + 88;                // TMEM base address
   static constexpr uint32_t BYTES = TMEM + 8;
-  // The block's dynamic shared memory starts 1024-byte aligned (checked at run time):
-  // the tiles need that alignment and there is no room for padding.
-  static_assert(BYTES <= 227 * 1024, "compress_pipe_kernel shared memory");
+  static_assert(BYTES + 1024 <= 227 * 1024, "compress_pipe_kernel shared memory");
 };
+// Tensor memory (512 columns): Y[2] at 0 and 128, S r at 256, the residual operand at
+// 384 (hi: 64 columns of f16 pairs, then lo).
+constexpr uint32_t kTmY = 0, kTmP = 256, kTmA = 384;
 
 // Adds the NB-bit field v at bit offset o of the words w (fields start zero, so add
 // acts as or, and compiles to one integer multiply-add).
@@ -1242,20 +1243,15 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
   using PS = PipeSmem;
   namespace s1 = tq::sm100;
   constexpr int L = 1 << LMB, HL = L / 2;
-  extern __shared__ __align__(1024) unsigned char smem_pipe[];
-  unsigned char* sm = smem_pipe;
-  if (s1::smem_u32(sm) & 1023u) {  // the layout needs it; report instead of misaddressing
-    if (threadIdx.x == 0) atomicOr(a.err, 2u);
-    return;
-  }
+  extern __shared__ unsigned char smem_pipe[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>(((uintptr_t)smem_pipe + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = s1::smem_u32(sm);
   float* xr = reinterpret_cast<float*>(sm + PS::XR);
-  uint8_t* zf = sm + PS::ZF;
   uint64_t* kfull = reinterpret_cast<uint64_t*>(sm + PS::BAR);  // [2] key tile landed
   uint64_t* rotd = kfull + 2;                                        // [2] rotation into Y[b] done
   uint64_t* projd = kfull + 4;                                       // projection done
-  uint64_t* vfull = kfull + 5;                                       // [2] value half landed
-  uint64_t* fin = kfull + 7;                                         // failure path: MMAs drained
+  uint64_t* vfull = kfull + 5;                                       // [4] value half landed
+  uint64_t* fin = kfull + 9;                                         // failure path: MMAs drained (2 issuers)
   uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + PS::TMEM);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t ntile = (a.n_vec + 127) / 128, g = gridDim.x;
@@ -1265,7 +1261,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
     s1::tmem_relinquish();
   }
   if (tid == 0) {
-    for (int k = 0; k < 8; ++k) s1::mbar_init(kfull + k, 1);
+    for (int k = 0; k < 9; ++k) s1::mbar_init(kfull + k, 1);
+    s1::mbar_init(fin, 2);
     s1::mbar_init_fence();
   }
   {  // H diag(sigma) and S operand tiles, prepacked on the host
@@ -1282,7 +1279,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
   s1::fence_before_sync();
   __syncthreads();
   s1::fence_after_sync();
-  const uint32_t tmem = *tmem_s;  // columns 0..255: Y[2]; 256..511: S r [2]
+  const uint32_t tmem = *tmem_s;
   bool failed = false;
 
   if (warp < 8) {
@@ -1315,18 +1312,17 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
         constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          s1::umma_f16(tmem + 128 * b, s1::sw128_desc(sbase + PS::KT + b * kTcTileBytes, 16 * ks, 128),
+          s1::umma_f16(tmem + kTmY + 128 * b, s1::sw128_desc(sbase + PS::KT + b * kTcTileBytes, 16 * ks, 128),
                        s1::sw128_desc(sbase + PS::HB, 16 * ks, 128), idesc, ks > 0 ? 1u : 0u);
         s1::umma_commit(rotd + b);
       };
       // Sign readout of a pass whose projection has completed: bit j set <=> (S r)_j >= 0.
-      auto read_signs = [&](int b, int64_t pv0) {
+      auto read_signs = [&](int64_t pv0, bool nzk) {
         const int64_t pi = pv0 + R;
-        const bool nzk = zf[b * 128 + R] != 0;
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
           uint32_t v[32];
-          s1::tmem_ld32(tmem + 256 + 128 * b + lane_base + 64 * ch + 32 * h, v);
+          s1::tmem_ld32(tmem + kTmP + lane_base + 64 * ch + 32 * h, v);
           s1::tmem_ld_wait();
           uint32_t b4[4] = {0u, 0u, 0u, 0u};  // sign bits, four independent 8-bit chains
 #pragma unroll
@@ -1351,6 +1347,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
       __syncwarp();  // warp 0 converged again before its tensor-memory loads
       int it = 0;
       int64_t prev_v0 = 0;
+      bool prev_nz = false;  // the previous pass's key of this row was stored as nonzero
       for (int64_t tile = blockIdx.x; tile < ntile; tile += g, ++it) {
         const int b = it & 1;
         const int64_t v0 = tile * 128, i = v0 + R;
@@ -1376,7 +1373,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
 #pragma unroll 1
           for (int h = 0; h < 2; ++h) {
             uint32_t v[32];
-            s1::tmem_ld32(tmem + 128 * b + lane_base + 64 * c2 + 32 * h, v);
+            s1::tmem_ld32(tmem + kTmY + 128 * b + lane_base + 64 * c2 + 32 * h, v);
             s1::tmem_ld_wait();
 #pragma unroll
             for (int e = 0; e < 32; e += 4) {
@@ -1392,43 +1389,43 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
         const bool nz = tot > 0.f;
         const float sc16 = nz ? 16.f * (1.0f / sqrtf(tot)) : 0.f;
         const float2 sc2 = make_float2(sc16, sc16);
-        // the previous projection has finished: A tiles free, its S r readable
-        if (it > 0 && !failed && !s1::mbar_wait(projd, (uint32_t)(it - 1) & 1u)) failed = true;
-        s1::fence_after_sync();
+        // the previous projection has finished: its S r is readable and the operand free
+        if (it > 0) {
+          if (!failed && !s1::mbar_wait(projd, (uint32_t)(it - 1) & 1u)) failed = true;
+          s1::fence_after_sync();
+          read_signs(prev_v0, prev_nz);
+        }
         float2 ra = make_float2(0.f, 0.f), rb = make_float2(0.f, 0.f);  // r^2 chains (0,1), (2,3)
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
           uint32_t v[32];
-          s1::tmem_ld32(tmem + 128 * b + lane_base + 64 * ch + 32 * h, v);
+          s1::tmem_ld32(tmem + kTmY + 128 * b + lane_base + 64 * ch + 32 * h, v);
           s1::tmem_ld_wait();
           uint32_t cw[LMB], cw2[LMB];  // even / odd codes: two independent chains per word
 #pragma unroll
           for (int w = 0; w < LMB; ++w) cw[w] = cw2[w] = 0u;
+          uint32_t hw[16], lw[16];  // residual x16 as f16 pairs: hi, lo
 #pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8) {
-            uint32_t hw[4], lw[4];
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-              const int e = 8 * c8 + 2 * p;
-              const float2 yy = s1::mul2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), sc2);
-              uint32_t q0, q1;
-              const float c0 = bucket_sym<LMB>(yy.x, tm, cm, q0);
-              const float c1 = bucket_sym<LMB>(yy.y, tm, cm, q1);
-              add_field<LMB, LMB>(cw, LMB * e, q0);
-              add_field<LMB, LMB>(cw2, LMB * (e + 1), q1);
-              const float2 r = s1::sub2(yy, make_float2(c0, c1));  // residual x16
-              if (p & 1) rb = s1::fma2(r, r, rb);
-              else ra = s1::fma2(r, r, ra);
-              const __half2 hh = __floats2half2_rn(r.x, r.y);
-              const float2 lo = s1::sub2(r, __half22float2(hh));
-              const __half2 ll = __floats2half2_rn(lo.x, lo.y);
-              hw[p] = *reinterpret_cast<const uint32_t*>(&hh);
-              lw[p] = *reinterpret_cast<const uint32_t*>(&ll);
-            }
-            const uint32_t off = s1::sw128_offset(R, 64 * ch + 32 * h + 8 * c8, 128);
-            *reinterpret_cast<uint4*>(sm + PS::A_HI + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-            *reinterpret_cast<uint4*>(sm + PS::A_LO + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+          for (int p = 0; p < 16; ++p) {
+            const int e = 2 * p;
+            const float2 yy = s1::mul2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), sc2);
+            uint32_t q0, q1;
+            const float c0 = bucket_sym<LMB>(yy.x, tm, cm, q0);
+            const float c1 = bucket_sym<LMB>(yy.y, tm, cm, q1);
+            add_field<LMB, LMB>(cw, LMB * e, q0);
+            add_field<LMB, LMB>(cw2, LMB * (e + 1), q1);
+            const float2 r = s1::sub2(yy, make_float2(c0, c1));  // residual x16
+            if (p & 1) rb = s1::fma2(r, r, rb);
+            else ra = s1::fma2(r, r, ra);
+            const __half2 hh = __floats2half2_rn(r.x, r.y);
+            const float2 lo = s1::sub2(r, __half22float2(hh));
+            const __half2 ll = __floats2half2_rn(lo.x, lo.y);
+            hw[p] = *reinterpret_cast<const uint32_t*>(&hh);
+            lw[p] = *reinterpret_cast<const uint32_t*>(&ll);
           }
+          // row R's coordinates 64ch + 32h .. + 31: columns 32ch + 16h .. + 15 of hi and lo
+          s1::tmem_st16(tmem + kTmA + lane_base + 32 * ch + 16 * h, hw);
+          s1::tmem_st16(tmem + kTmA + 64 + lane_base + 32 * ch + 16 * h, lw);
           if (valid) {
             uint32_t* co = reinterpret_cast<uint32_t*>(a.k_codes + i * (LMB * 16) + ch * (LMB * 8) + h * (LMB * 4));
 #pragma unroll
@@ -1436,79 +1433,80 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
           }
         }
         xr[b * 256 + ch * 128 + R] = (ra.x + ra.y) + (rb.x + rb.y);
-        s1::fence_async_smem();
+        s1::tmem_st_wait();
         s1::fence_before_sync();
         failed = s1::bar_sync_or<1, 256>(failed);
         s1::fence_after_sync();
         if (failed) break;
-        if (ch == 0) {
+        if (ch == 0 && valid) {
           const float gamma = sqrtf(xr[b * 256 + R] + xr[b * 256 + 128 + R]) * (1.f / 16.f);
-          if (valid) {
-            const uint32_t nb = __half_as_ushort(__float2half_rn(sqrtf(tot * (1.0f / 128.f))));
-            const uint32_t gb = __half_as_ushort(__float2half_rn(gamma));
-            reinterpret_cast<uint32_t*>(a.k_norms)[i] = nz ? (nb | (gb << 16)) : 0u;
-          }
-          zf[b * 128 + R] = (valid && nz) ? 1 : 0;
+          const uint32_t nb = __half_as_ushort(__float2half_rn(sqrtf(tot * (1.0f / 128.f))));
+          const uint32_t gb = __half_as_ushort(__float2half_rn(gamma));
+          reinterpret_cast<uint32_t*>(a.k_norms)[i] = nz ? (nb | (gb << 16)) : 0u;
         }
-        if (tid == 0) {
+        if (tid == kProjIssuer) {  // a thread of another warp than the rotation's issuer
           constexpr uint32_t idesc = s1::idesc_f16_f32(128, 128);
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
-            s1::umma_f16(tmem + 256 + 128 * b, s1::sw128_desc(sbase + PS::A_HI, 16 * ks, 128),
-                         s1::sw128_desc(sbase + PS::S, 16 * ks, 128), idesc, ks > 0 ? 1u : 0u);
+            s1::umma_f16_ts(tmem + kTmP, tmem + kTmA + 8 * ks, s1::sw128_desc(sbase + PS::S, 16 * ks, 128), idesc,
+                            ks > 0 ? 1u : 0u);
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
-            s1::umma_f16(tmem + 256 + 128 * b, s1::sw128_desc(sbase + PS::A_LO, 16 * ks, 128),
-                         s1::sw128_desc(sbase + PS::S, 16 * ks, 128), idesc, 1u);
+            s1::umma_f16_ts(tmem + kTmP, tmem + kTmA + 64 + 8 * ks, s1::sw128_desc(sbase + PS::S, 16 * ks, 128),
+                            idesc, 1u);
           s1::umma_commit(projd);
         }
         __syncwarp();
-        if (it > 0) read_signs(b ^ 1, prev_v0);
-        s1::fence_before_sync();
         prev_v0 = v0;
+        prev_nz = valid && nz;
       }
-      // the last pass's signs (its nonzero flags were written after the last barrier)
-      failed = s1::bar_sync_or<1, 256>(failed);
+      // the last pass's signs
       if (!failed && it > 0) {
         if (!s1::mbar_wait(projd, (uint32_t)(it - 1) & 1u)) {
           failed = true;
         } else {
           s1::fence_after_sync();
-          read_signs((it - 1) & 1, prev_v0);
+          read_signs(prev_v0, prev_nz);
         }
       }
-      if (failed && tid == 0) {
-        // bounded: drain this thread's MMAs and its outstanding key loads before the
+      failed = s1::bar_sync_or<1, 256>(failed);  // both issuers agree on draining
+      if (failed && (tid == 0 || tid == kProjIssuer)) {
+        // bounded: drain both issuers' MMAs and the outstanding key loads before the
         // shared and tensor memory they use is released
         s1::umma_commit(fin);
         s1::mbar_wait(fin, 0u);
-        for (int b = 0; b < 2; ++b)
-          if ((kpend >> b) & 1u) s1::mbar_wait(kfull + b, (kpar >> b) & 1u);
+        if (tid == 0)
+          for (int b = 0; b < 2; ++b)
+            if ((kpend >> b) & 1u) s1::mbar_wait(kfull + b, (kpar >> b) & 1u);
       }
     }
   } else if (a.v) {
     // ================================================================ values
     const int vt = tid - 256, q = vt & 3, vrow = vt >> 2;  // 4 threads per value, 64 per half
     const bool leader = vt == 0;
-    uint32_t vpar = 0u, vpend = 0u;  // bit h for value half h: next parity, copy outstanding
-    // half h of a pass: rows 64h..64h+63 as two 64-column panels of 64 rows x 128 bytes
-    auto fetch_half = [&](int64_t tile, int h) {
+    uint32_t vpar = 0u, vpend = 0u;  // bit f for value half buffer f: next parity, copy outstanding
+    // half h of a pass into buffer f: rows 64h..64h+63 as two panels of 64 rows x 128 bytes
+    auto fetch_half = [&](int64_t tile, int h, int f) {
       const int64_t r0 = tile * 128 + 64 * h;
       if (r0 >= a.n_vec) return;
-      unsigned char* dst = sm + PS::VR + h * (kTcTileBytes / 2);
-      s1::mbar_expect_tx(vfull + h, 64u * 128u * 2u);
-      s1::tma_load_2d(dst, &a.vmap, 0, (int)r0, vfull + h);
-      s1::tma_load_2d(dst + kTcTileBytes / 4, &a.vmap, 64, (int)r0, vfull + h);
-      vpend |= 1u << h;
+      unsigned char* dst = sm + PS::VR + f * (kTcTileBytes / 2);
+      s1::mbar_expect_tx(vfull + f, 64u * 128u * 2u);
+      s1::tma_load_2d(dst, &a.vmap, 0, (int)r0, vfull + f);
+      s1::tma_load_2d(dst + kTcTileBytes / 4, &a.vmap, 64, (int)r0, vfull + f);
+      vpend |= 1u << f;
     };
-    // byte offset, within a half, of this thread's 16-byte chunk k (coordinates 32q + 8k ..)
+    // byte offset, within a half buffer, of this thread's 16-byte chunk k (coordinates 32q + 8k ..)
     const int vsw = vrow & 7;
     auto chunk_off = [&](int k) -> uint32_t {
       return (uint32_t)((q >> 1) * (kTcTileBytes / 4) + vrow * 128 + (((4 * (q & 1) + k) ^ vsw) << 4));
     };
     if (leader && (int64_t)blockIdx.x < ntile) {
-      fetch_half(blockIdx.x, 0);
-      fetch_half(blockIdx.x, 1);
+      fetch_half(blockIdx.x, 0, 0);
+      fetch_half(blockIdx.x, 1, 1);
+      if (blockIdx.x + g < ntile) {
+        fetch_half(blockIdx.x + g, 0, 2);
+        fetch_half(blockIdx.x + g, 1, 3);
+      }
     }
     constexpr int levels = (1 << VB) - 1;
     constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
@@ -1516,22 +1514,24 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
     uint32_t magic_sum = 0u;
 #pragma unroll
     for (int f = 0; f < 32 / VB; ++f) magic_sum += __float_as_uint(kMagic) << (VB * f);
-    for (int64_t tile = blockIdx.x; tile < ntile && !failed; tile += g) {
+    int it = 0;
+    for (int64_t tile = blockIdx.x; tile < ntile && !failed; tile += g, ++it) {
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
+        const int f = 2 * (it & 1) + h;
         const int64_t r0 = tile * 128 + 64 * h;
         if (r0 >= a.n_vec) break;  // the same for every value thread
         if (!failed) {
-          if (s1::mbar_wait(vfull + h, (vpar >> h) & 1u)) {
-            vpar ^= 1u << h;
-            vpend &= ~(1u << h);
+          if (s1::mbar_wait(vfull + f, (vpar >> f) & 1u)) {
+            vpar ^= 1u << f;
+            vpend &= ~(1u << f);
           } else {
             failed = true;
           }
         }
         const int64_t i = r0 + vrow;
         if (!failed && i < a.n_vec) {
-          const unsigned char* half = sm + PS::VR + h * (kTcTileBytes / 2);
+          const unsigned char* half = sm + PS::VR + f * (kTcTileBytes / 2);
           uint32_t w[16];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
@@ -1541,20 +1541,30 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
             w[4 * k + 2] = u.z;
             w[4 * k + 3] = u.w;
           }
-          // min / max on the packed bf16 pairs (exact: bf16 -> fp32 is monotone)
-          __nv_bfloat162 mn = *reinterpret_cast<const __nv_bfloat162*>(&w[0]), mx = mn;
+          // min / max on the packed bf16 pairs (exact: bf16 -> fp32 is monotone), as trees
+          __nv_bfloat162 mn[8], mx[8];
 #pragma unroll
-          for (int k = 1; k < 16; ++k) {
-            const __nv_bfloat162 x2 = *reinterpret_cast<const __nv_bfloat162*>(&w[k]);
-            mn = __hmin2(mn, x2);
-            mx = __hmax2(mx, x2);
+          for (int k = 0; k < 8; ++k) {
+            const __nv_bfloat162 x0 = *reinterpret_cast<const __nv_bfloat162*>(&w[k]);
+            const __nv_bfloat162 x1 = *reinterpret_cast<const __nv_bfloat162*>(&w[k + 8]);
+            mn[k] = __hmin2(x0, x1);
+            mx[k] = __hmax2(x0, x1);
           }
-          const float lo = fminf(__low2float(mn), __high2float(mn));
-          const float hi = fmaxf(__low2float(mx), __high2float(mx));
-          // scale in fp64 as the reference quantizer; codes rounded to nearest by adding
-          // 1.5 * 2^23, redone in fp64 with floor(t + 1/2) within 1e-5 of a half step.
+#pragma unroll
+          for (int s = 4; s >= 1; s >>= 1)
+#pragma unroll
+            for (int k = 0; k < s; ++k) {
+              mn[k] = __hmin2(mn[k], mn[k + s]);
+              mx[k] = __hmax2(mx[k], mx[k + s]);
+            }
+          const float lo = fminf(__low2float(mn[0]), __high2float(mn[0]));
+          const float hi = fmaxf(__low2float(mx[0]), __high2float(mx[0]));
+          // Codes rounded to nearest by adding 1.5 * 2^23 to t = (v - min) * levels / span.
+          // The fp32 t only has to be right away from the half steps: any coordinate within
+          // 1e-5 of one is redone below in fp64 as the reference quantizer computes it.
           const double dlo = lo, span = (double)hi - dlo;
-          const float inv = span > 0.0 ? (float)(levels / span) : 0.f;
+          const float span32 = hi - lo;
+          const float inv = span32 > 0.f ? __fdiv_rn((float)levels, span32) : 0.f;
           const float2 lo2 = make_float2(lo, lo), inv2 = make_float2(inv, inv), mg2 = make_float2(kMagic, kMagic);
           uint32_t vw[VB], vw2[VB];
 #pragma unroll
@@ -1606,18 +1616,18 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
           const uint32_t mb = __half_as_ushort(__float2half_rn(lo));
           reinterpret_cast<uint32_t*>(a.v_params)[i * 4 + q] = sb | (mb << 16);
         }
-        // every value thread is done with this half: refill it for the next pass
+        // every value thread is done with this half: refill it two passes ahead
         failed = s1::bar_sync_or<2, 256>(failed);
         if (failed) break;
-        if (leader && tile + g < ntile) {
+        if (leader && tile + 2 * g < ntile) {
           s1::fence_async_smem();
-          fetch_half(tile + g, h);
+          fetch_half(tile + 2 * g, h, f);
         }
       }
     }
     if (failed && leader)
-      for (int h = 0; h < 2; ++h)
-        if ((vpend >> h) & 1u) s1::mbar_wait(vfull + h, (vpar >> h) & 1u);  // bounded
+      for (int f = 0; f < 4; ++f)
+        if ((vpend >> f) & 1u) s1::mbar_wait(vfull + f, (vpar >> f) & 1u);  // bounded
   }
   if (__syncthreads_or(failed) && tid == 0) atomicOr(a.err, 1u);
   s1::fence_before_sync();
@@ -1671,7 +1681,7 @@ bool codebook_symmetric(const Codebook& cb, int lm_bits) {
 template <int LMB, int VB>
 cudaError_t launch_pipe_t(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) {
   static bool configured = false;
-  const size_t smem = PipeSmem::BYTES;
+  const size_t smem = PipeSmem::BYTES + 1024;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(compress_pipe_kernel<LMB, VB>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -223,9 +223,6 @@ tq_status tq_check_device(const tq_ctx* c, void* stream) {
   if (e == cudaSuccess && flag) e = cudaMemset(c->d_err, 0, sizeof(flag));
   if (e != cudaSuccess) return fail_cuda(e, "tq_check_device");
   if (flag & 1u) return fail(TQ_ECUDA, "tq_check_device: a bounded wait for a bulk copy timed out; results of that call are invalid");
-  if (flag & 2u)
-    return fail(TQ_ECUDA, "tq_check_device: a compression kernel found its shared memory not 1024-byte aligned and "
-                          "did nothing; results of that call are invalid");
   return TQ_OK;
 }
 

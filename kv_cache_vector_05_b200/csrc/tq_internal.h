@@ -44,8 +44,7 @@ struct tq_ctx {
   float* PiT;      // device [d][d] fp32 transpose (Haar only)
   cudaEvent_t prof_start;  // optional events around the main kernel of each call
   cudaEvent_t prof_stop;
-  unsigned int* d_err;     // device error word: bit 0 = a bounded wait in a kernel timed out,
-                           // bit 1 = shared memory not 1024-byte aligned (compression did nothing)
+  unsigned int* d_err;     // device error word: bit 0 = a bounded wait in a kernel timed out
   uint16_t* S_sw128;       // tensor-core compression: S as an f16 operand tile (d = m = 128, S exact in f16)
   uint16_t* H_sw128;       // tensor-core compression: H diag(sigma) as a bf16 operand tile (d = 128, Hadamard)
   uint16_t* Pi_sw128;      // tensor-core compression: Haar Pi as three bf16 operand tiles (d = 128)
