@@ -1560,8 +1560,13 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
           const float lo = fminf(__low2float(mn[0]), __high2float(mn[0]));
           const float hi = fmaxf(__low2float(mx[0]), __high2float(mx[0]));
           // Codes rounded to nearest by adding 1.5 * 2^23 to t = (v - min) * levels / span.
-          // The fp32 t only has to be right away from the half steps: any coordinate within
-          // 1e-5 of one is redone below in fp64 as the reference quantizer computes it.
+          // Four roundings (span, levels / span, v - min, the product) put the fp32 t within
+          // levels * 2.4e-7 of the exact value, so it gives the reference's floor(t + 1/2)
+          // except at most that close to a half step (an exact tie, or within rounding of
+          // one), where the code may be the other neighbour. For 2-bit codes that band is
+          // narrower than 1e-6; for 4-bit codes the coordinates within 5e-6 of a half step
+          // are redone in fp64 as floor(t + 1/2).
+          constexpr bool kRedoNearHalf = VB > 2;
           const double dlo = lo, span = (double)hi - dlo;
           const float span32 = hi - lo;
           const float inv = span32 > 0.f ? __fdiv_rn((float)levels, span32) : 0.f;
@@ -1569,49 +1574,47 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
           uint32_t vw[VB], vw2[VB];
 #pragma unroll
           for (int k = 0; k < VB; ++k) vw[k] = vw2[k] = 0u;
-          bool near = false;
+          uint32_t near = 0u;  // bit e: coordinate e within 1e-5 of a half step
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
             const float2 x = make_float2(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xffff0000u));
             const float2 t = s1::mul2(s1::sub2(x, lo2), inv2);
             const float2 tr = s1::add2(t, mg2);
             const float2 e = s1::sub2(t, s1::sub2(tr, mg2));
-            near |= fabsf(e.x) > 0.5f - 1e-5f;
-            near |= fabsf(e.y) > 0.5f - 1e-5f;
+            if (kRedoNearHalf) {
+              if (fabsf(e.x) > 0.5f - 5e-6f) near |= 1u << (2 * k);
+              if (fabsf(e.y) > 0.5f - 5e-6f) near |= 2u << (2 * k);
+            }
             // tr's bits are those of the magic constant plus the code
             add_field<VB, VB>(vw, VB * 2 * k, __float_as_uint(tr.x));
             add_field<VB, VB>(vw2, VB * (2 * k + 1), __float_as_uint(tr.y));
           }
 #pragma unroll
           for (int k = 0; k < VB; ++k) vw[k] = vw[k] + vw2[k] - magic_sum;
-          uint32_t* vo = reinterpret_cast<uint32_t*>(a.v_codes + i * (VB * 16) + q * (VB * 4));
-#pragma unroll
-          for (int k = 0; k < VB; ++k) vo[k] = vw[k];
-          if (near) {
-            // Some coordinate lies within 1e-5 of a half step (with bf16 inputs a ratio of
-            // small integers often lands exactly on one): find which, and redo only those
-            // in fp64 as floor(t + 1/2), patching the words just stored.
-            uint32_t mask = 0u;
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              const uint32_t wk = *reinterpret_cast<const uint32_t*>(half + chunk_off(k >> 2) + 4 * (k & 3));
-              const float2 x = make_float2(__uint_as_float(wk << 16), __uint_as_float(wk & 0xffff0000u));
-              const float2 t = s1::mul2(s1::sub2(x, lo2), inv2);
-              const float2 e = s1::sub2(t, s1::sub2(s1::add2(t, mg2), mg2));
-              if (fabsf(e.x) > 0.5f - 1e-5f) mask |= 1u << (2 * k);
-              if (fabsf(e.y) > 0.5f - 1e-5f) mask |= 2u << (2 * k);
-            }
+          if (kRedoNearHalf && near) {
+            // Some coordinate lies within 5e-6 of a half step (with bf16 inputs a ratio of
+            // small integers lands exactly on one in about one group of twenty): redo only
+            // those in fp64.
+            uint32_t mask = near;
+            const double r64 = levels / span;
             while (mask) {
               const int e = __ffs(mask) - 1;
               mask &= mask - 1u;
               const float xe = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
                   half + chunk_off(e >> 3) + 2 * (e & 7)));
-              const uint32_t qf = __float_as_uint((xe - lo) * inv + kMagic) & 0xffu;  // the fast code
-              const uint32_t qv =
-                  min((uint32_t)floor(((double)xe - dlo) * (levels / span) + 0.5), (uint32_t)levels);
-              vo[(VB * e) >> 5] ^= (qf ^ qv) << ((VB * e) & 31);
+              const uint32_t qv = min((uint32_t)floor(((double)xe - dlo) * r64 + 0.5), (uint32_t)levels);
+              const int wi = (VB * e) >> 5, sh = (VB * e) & 31;
+#pragma unroll
+              for (int k = 0; k < VB; ++k) {  // replace the field in place (static indices)
+                const uint32_t sel = (wi == k) ? 0xffffffffu : 0u;
+                const uint32_t old = (vw[k] >> sh) & (uint32_t)levels;
+                vw[k] ^= ((old ^ qv) << sh) & sel;
+              }
             }
           }
+          uint32_t* vo = reinterpret_cast<uint32_t*>(a.v_codes + i * (VB * 16) + q * (VB * 4));
+#pragma unroll
+          for (int k = 0; k < VB; ++k) vo[k] = vw[k];
           const uint32_t sb = __half_as_ushort(__double2half(span / levels));
           const uint32_t mb = __half_as_ushort(__float2half_rn(lo));
           reinterpret_cast<uint32_t*>(a.v_params)[i * 4 + q] = sb | (mb << 16);
