@@ -83,7 +83,7 @@ def source_sha(names):
     return h.hexdigest()[:16]
 
 
-DECODE_SOURCES = ("decode_mma.cu", "decode.cu", "tq_device.cuh", "tq_internal.h")
+DECODE_SOURCES = ("decode_mma.cu", "decode.cu", "tq_device.cuh", "tq_sm100.cuh", "tq_internal.h")
 COMPRESS_SOURCES = ("compress.cu", "tq_device.cuh", "tq_sm100.cuh", "tq_internal.h")
 
 
@@ -468,7 +468,8 @@ def run_ours(args, w: W.Workload):
             csha = source_sha(COMPRESS_SOURCES)
             comp_bytes = in_bytes + packed_bytes
             comp_k_mean = statistics.fmean(comp_k) / 1e3
-            ckern = "compress_rot_kernel" if (w.dtype == "bf16" and w.d == 128 and w.rotation == "hadamard") \
+            # bf16 keys, Hadamard rotation, d = 128 and the (symmetric) Lloyd-Max codebook
+            ckern = "compress_pipe_kernel" if (w.dtype == "bf16" and w.d == 128 and w.rotation == "hadamard") \
                 else "compress_q4_kernel"
             roof = {"kernel": ckern, "bound": "hbm", "achieved": comp_bytes / comp_k_mean / 1e9, "peak": peak,
                     "unit": "GB/s", "frac": comp_bytes / comp_k_mean / 1e9 / peak, "peak_kind": peak_kind,

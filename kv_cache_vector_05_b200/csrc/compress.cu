@@ -1174,10 +1174,11 @@ cudaError_t launch_rot(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s)
 // zero (c[L-1-k] = -c[k], t[L-2-k] = -t[k]; the sphere Lloyd-Max codebook is). The
 // arithmetic is that of compress_rot_kernel; the organisation lets consecutive passes
 // of 128 vectors overlap and keeps the tensor cores' shared-memory reads low:
-//  * the key rows arrive by TMA straight into one of two swizzled operand tiles, two
-//    passes ahead;
-//  * the rotation MMA of pass i+1 (into the other half of a double-buffered Y in tensor
-//    memory) runs while the key warps work on pass i;
+//  * one producer thread (warp 16) issues every key TMA and every MMA, so that no
+//    compute warp waits while the tensor core takes the instructions;
+//  * the key rows arrive by TMA straight into one of two swizzled operand tiles, and the
+//    rotation MMA of pass i+2 (into the half of a double-buffered Y in tensor memory
+//    that pass i has just released) runs while the key warps work on pass i+1;
 //  * the residual's f16 hi / lo operand goes to tensor memory (tcgen05.st), so the
 //    projection MMA reads only S from shared memory; it runs while the key warps start
 //    on the next pass, which reads its signs out before overwriting the operand;
@@ -1190,8 +1191,7 @@ cudaError_t launch_rot(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s)
 // barrier of a pass. With the symmetric codebook a coordinate is bucketized on its
 // magnitude and the code's bits follow from its sign; everything is scaled by 16 (an
 // exact power of two) so that the residual comes out as the x16 operand directly.
-constexpr int kPipeThreads = 512;
-constexpr int kProjIssuer = 128;  // first thread of key warp 4 (thread 0 issues the rotation)
+constexpr int kPipeThreads = 640;  // warps 0-7 keys, 8-15 values, 16 producer (17-19 idle)
 
 struct PipeSmem {
   static constexpr uint32_t KT = 0;                         // [2] key operand tiles (TMA, 128B swizzle)
@@ -1251,7 +1251,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
   uint64_t* rotd = kfull + 2;                                        // [2] rotation into Y[b] done
   uint64_t* projd = kfull + 4;                                       // projection done
   uint64_t* vfull = kfull + 5;                                       // [4] value half landed
-  uint64_t* fin = kfull + 9;                                         // failure path: MMAs drained (2 issuers)
+  uint64_t* aready = kfull + 9;                                      // key warps done with a pass (8 arrivals)
+  uint64_t* fin = kfull + 10;                                        // failure path: MMAs drained
   uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + PS::TMEM);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t ntile = (a.n_vec + 127) / 128, g = gridDim.x;
@@ -1262,7 +1263,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
   }
   if (tid == 0) {
     for (int k = 0; k < 9; ++k) s1::mbar_init(kfull + k, 1);
-    s1::mbar_init(fin, 2);
+    s1::mbar_init(aready, 8);
+    s1::mbar_init(fin, 1);
     s1::mbar_init_fence();
   }
   {  // H diag(sigma) and S operand tiles, prepacked on the host
@@ -1293,29 +1295,6 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
       for (int j = 0; j < HL - 1; ++j) tm[j] = 16.f * a.cb.t[HL + j];
 #pragma unroll
       for (int j = 0; j < HL; ++j) cm[j] = 16.f * a.cb.c[HL + j];
-      // TMA bookkeeping (thread 0), bit b for key buffer b: next parity, load outstanding
-      uint32_t kpar = 0u, kpend = 0u;
-      auto load_keys = [&](int b, int64_t tile) {
-        s1::mbar_expect_tx(kfull + b, 2u * 128u * 128u);
-        s1::tma_load_2d(sm + PS::KT + b * kTcTileBytes, &a.kmap, 0, (int)(tile * 128), kfull + b);
-        s1::tma_load_2d(sm + PS::KT + b * kTcTileBytes + kTcTileBytes / 2, &a.kmap, 64, (int)(tile * 128),
-                        kfull + b);
-        kpend |= 1u << b;
-      };
-      auto wait_keys = [&](int b) -> bool {
-        if (!s1::mbar_wait(kfull + b, (kpar >> b) & 1u)) return false;
-        kpar ^= 1u << b;
-        kpend &= ~(1u << b);
-        return true;
-      };
-      auto issue_rotation = [&](int b) {
-        constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          s1::umma_f16(tmem + kTmY + 128 * b, s1::sw128_desc(sbase + PS::KT + b * kTcTileBytes, 16 * ks, 128),
-                       s1::sw128_desc(sbase + PS::HB, 16 * ks, 128), idesc, ks > 0 ? 1u : 0u);
-        s1::umma_commit(rotd + b);
-      };
       // Sign readout of a pass whose projection has completed: bit j set <=> (S r)_j >= 0.
       auto read_signs = [&](int64_t pv0, bool nzk) {
         const int64_t pi = pv0 + R;
@@ -1333,18 +1312,6 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
           if (pi < a.n_vec) reinterpret_cast<uint32_t*>(a.k_signs + pi * 16 + 8 * ch)[h] = nzk ? word : 0u;
         }
       };
-
-      if (tid == 0 && (int64_t)blockIdx.x < ntile) {
-        load_keys(0, blockIdx.x);
-        if (blockIdx.x + g < ntile) load_keys(1, blockIdx.x + g);
-        if (wait_keys(0)) {
-          s1::fence_after_sync();
-          issue_rotation(0);
-        } else {
-          failed = true;
-        }
-      }
-      __syncwarp();  // warp 0 converged again before its tensor-memory loads
       int it = 0;
       int64_t prev_v0 = 0;
       bool prev_nz = false;  // the previous pass's key of this row was stored as nonzero
@@ -1354,17 +1321,6 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
         const bool valid = i < a.n_vec;
         if (!failed && !s1::mbar_wait(rotd + b, (uint32_t)(it >> 1) & 1u)) failed = true;
         s1::fence_after_sync();
-        if (tid == 0 && !failed) {
-          // KT[b] has been read by the rotation just waited for: refill it two passes ahead;
-          // then start the next pass's rotation into Y[b ^ 1] (read last pass, before the
-          // barrier that ended it).
-          if (tile + 2 * g < ntile) load_keys(b, tile + 2 * g);
-          if (tile + g < ntile) {
-            if (wait_keys(b ^ 1)) issue_rotation(b ^ 1);
-            else failed = true;
-          }
-        }
-        __syncwarp();
         // ||Y||^2 over the row's 128 columns, as two 64-column halves of four chains each
         float hs[2];
 #pragma unroll
@@ -1404,28 +1360,32 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
           uint32_t cw[LMB], cw2[LMB];  // even / odd codes: two independent chains per word
 #pragma unroll
           for (int w = 0; w < LMB; ++w) cw[w] = cw2[w] = 0u;
-          uint32_t hw[16], lw[16];  // residual x16 as f16 pairs: hi, lo
 #pragma unroll
-          for (int p = 0; p < 16; ++p) {
-            const int e = 2 * p;
-            const float2 yy = s1::mul2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), sc2);
-            uint32_t q0, q1;
-            const float c0 = bucket_sym<LMB>(yy.x, tm, cm, q0);
-            const float c1 = bucket_sym<LMB>(yy.y, tm, cm, q1);
-            add_field<LMB, LMB>(cw, LMB * e, q0);
-            add_field<LMB, LMB>(cw2, LMB * (e + 1), q1);
-            const float2 r = s1::sub2(yy, make_float2(c0, c1));  // residual x16
-            if (p & 1) rb = s1::fma2(r, r, rb);
-            else ra = s1::fma2(r, r, ra);
-            const __half2 hh = __floats2half2_rn(r.x, r.y);
-            const float2 lo = s1::sub2(r, __half22float2(hh));
-            const __half2 ll = __floats2half2_rn(lo.x, lo.y);
-            hw[p] = *reinterpret_cast<const uint32_t*>(&hh);
-            lw[p] = *reinterpret_cast<const uint32_t*>(&ll);
+          for (int o8 = 0; o8 < 2; ++o8) {
+            uint32_t hw[8], lw[8];  // residual x16 as f16 pairs: hi, lo
+#pragma unroll
+            for (int pp = 0; pp < 8; ++pp) {
+              const int p = 8 * o8 + pp, e = 2 * p;
+              const float2 yy = s1::mul2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), sc2);
+              uint32_t q0, q1;
+              const float c0 = bucket_sym<LMB>(yy.x, tm, cm, q0);
+              const float c1 = bucket_sym<LMB>(yy.y, tm, cm, q1);
+              add_field<LMB, LMB>(cw, LMB * e, q0);
+              add_field<LMB, LMB>(cw2, LMB * (e + 1), q1);
+              const float2 r = s1::sub2(yy, make_float2(c0, c1));  // residual x16
+              if (p & 1) rb = s1::fma2(r, r, rb);
+              else ra = s1::fma2(r, r, ra);
+              const __half2 hh = __floats2half2_rn(r.x, r.y);
+              const float2 lo = s1::sub2(r, __half22float2(hh));
+              const __half2 ll = __floats2half2_rn(lo.x, lo.y);
+              hw[pp] = *reinterpret_cast<const uint32_t*>(&hh);
+              lw[pp] = *reinterpret_cast<const uint32_t*>(&ll);
+            }
+            // row R's coordinates 64ch + 32h + 16o8 .. + 15: 8 columns of hi and of lo
+            const uint32_t col = 32 * ch + 16 * h + 8 * o8;
+            s1::tmem_st8(tmem + kTmA + lane_base + col, hw);
+            s1::tmem_st8(tmem + kTmA + 64 + lane_base + col, lw);
           }
-          // row R's coordinates 64ch + 32h .. + 31: columns 32ch + 16h .. + 15 of hi and lo
-          s1::tmem_st16(tmem + kTmA + lane_base + 32 * ch + 16 * h, hw);
-          s1::tmem_st16(tmem + kTmA + 64 + lane_base + 32 * ch + 16 * h, lw);
           if (valid) {
             uint32_t* co = reinterpret_cast<uint32_t*>(a.k_codes + i * (LMB * 16) + ch * (LMB * 8) + h * (LMB * 4));
 #pragma unroll
@@ -1433,10 +1393,12 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
           }
         }
         xr[b * 256 + ch * 128 + R] = (ra.x + ra.y) + (rb.x + rb.y);
+        // Y[b] read, S r read, operand written: hand the pass to the producer
         s1::tmem_st_wait();
         s1::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) s1::mbar_arrive(aready);
         failed = s1::bar_sync_or<1, 256>(failed);
-        s1::fence_after_sync();
         if (failed) break;
         if (ch == 0 && valid) {
           const float gamma = sqrtf(xr[b * 256 + R] + xr[b * 256 + 128 + R]) * (1.f / 16.f);
@@ -1444,19 +1406,6 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
           const uint32_t gb = __half_as_ushort(__float2half_rn(gamma));
           reinterpret_cast<uint32_t*>(a.k_norms)[i] = nz ? (nb | (gb << 16)) : 0u;
         }
-        if (tid == kProjIssuer) {  // a thread of another warp than the rotation's issuer
-          constexpr uint32_t idesc = s1::idesc_f16_f32(128, 128);
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks)
-            s1::umma_f16_ts(tmem + kTmP, tmem + kTmA + 8 * ks, s1::sw128_desc(sbase + PS::S, 16 * ks, 128), idesc,
-                            ks > 0 ? 1u : 0u);
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks)
-            s1::umma_f16_ts(tmem + kTmP, tmem + kTmA + 64 + 8 * ks, s1::sw128_desc(sbase + PS::S, 16 * ks, 128),
-                            idesc, 1u);
-          s1::umma_commit(projd);
-        }
-        __syncwarp();
         prev_v0 = v0;
         prev_nz = valid && nz;
       }
@@ -1469,19 +1418,10 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
           read_signs(prev_v0, prev_nz);
         }
       }
-      failed = s1::bar_sync_or<1, 256>(failed);  // both issuers agree on draining
-      if (failed && (tid == 0 || tid == kProjIssuer)) {
-        // bounded: drain both issuers' MMAs and the outstanding key loads before the
-        // shared and tensor memory they use is released
-        s1::umma_commit(fin);
-        s1::mbar_wait(fin, 0u);
-        if (tid == 0)
-          for (int b = 0; b < 2; ++b)
-            if ((kpend >> b) & 1u) s1::mbar_wait(kfull + b, (kpar >> b) & 1u);
-      }
     }
-  } else if (a.v) {
+  } else if (warp < 16) {
     // ================================================================ values
+    if (a.v) {
     const int vt = tid - 256, q = vt & 3, vrow = vt >> 2;  // 4 threads per value, 64 per half
     const bool leader = vt == 0;
     uint32_t vpar = 0u, vpend = 0u;  // bit f for value half buffer f: next parity, copy outstanding
@@ -1631,6 +1571,92 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
     if (failed && leader)
       for (int f = 0; f < 4; ++f)
         if ((vpend >> f) & 1u) s1::mbar_wait(vfull + f, (vpar >> f) & 1u);  // bounded
+    }
+  } else if (warp == 16 && lane == 0 && a.k && (int64_t)blockIdx.x < ntile) {
+    // ================================================================ producer
+    const int64_t n_my = (ntile - blockIdx.x + g - 1) / g;  // passes of this CTA
+    auto tile_of = [&](int64_t j) { return (int64_t)blockIdx.x + j * g; };
+    uint32_t kpar = 0u, kpend = 0u;  // bit b for key buffer b: next parity, load outstanding
+    auto load_keys = [&](int b, int64_t tile) {
+      s1::mbar_expect_tx(kfull + b, 2u * 128u * 128u);
+      s1::tma_load_2d(sm + PS::KT + b * kTcTileBytes, &a.kmap, 0, (int)(tile * 128), kfull + b);
+      s1::tma_load_2d(sm + PS::KT + b * kTcTileBytes + kTcTileBytes / 2, &a.kmap, 64, (int)(tile * 128), kfull + b);
+      kpend |= 1u << b;
+    };
+    auto wait_keys = [&](int b) -> bool {
+      if (!s1::mbar_wait(kfull + b, (kpar >> b) & 1u)) return false;
+      kpar ^= 1u << b;
+      kpend &= ~(1u << b);
+      return true;
+    };
+    auto rotation = [&](int b) {  // Y[b] = KT[b] (H diag sigma)^T
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        s1::umma_f16(tmem + kTmY + 128 * b, s1::sw128_desc(sbase + PS::KT + b * kTcTileBytes, 16 * ks, 128),
+                     s1::sw128_desc(sbase + PS::HB, 16 * ks, 128), idesc, ks > 0 ? 1u : 0u);
+      s1::umma_commit(rotd + b);
+    };
+    auto projection = [&]() {  // S r = (A_hi + A_lo) S^T, A in tensor memory
+      constexpr uint32_t idesc = s1::idesc_f16_f32(128, 128);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        s1::umma_f16_ts(tmem + kTmP, tmem + kTmA + 8 * ks, s1::sw128_desc(sbase + PS::S, 16 * ks, 128), idesc,
+                        ks > 0 ? 1u : 0u);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        s1::umma_f16_ts(tmem + kTmP, tmem + kTmA + 64 + 8 * ks, s1::sw128_desc(sbase + PS::S, 16 * ks, 128), idesc,
+                        1u);
+      s1::umma_commit(projd);
+    };
+    // Prologue: passes 0 and 1 loaded and rotated, pass 2's keys on their way.
+    load_keys(0, tile_of(0));
+    if (n_my > 1) load_keys(1, tile_of(1));
+    if (!wait_keys(0)) failed = true;
+    else rotation(0);
+    if (!failed && n_my > 1) {
+      if (!wait_keys(1)) failed = true;
+      else rotation(1);
+    }
+    if (!failed && n_my > 2) {
+      if (!s1::mbar_wait(rotd, 0u)) failed = true;
+      else load_keys(0, tile_of(2));
+    }
+    for (int64_t j = 0; j < n_my && !failed; ++j) {
+      const int b = (int)(j & 1);
+      // KT[b^1] holds pass j+1, whose rotation was issued: once it has completed, refill
+      // that buffer with pass j+3
+      if (j + 3 < n_my) {
+        if (!s1::mbar_wait(rotd + (b ^ 1), (uint32_t)((j + 1) >> 1) & 1u)) {
+          failed = true;
+          break;
+        }
+        load_keys(b ^ 1, tile_of(j + 3));
+      }
+      // pass j's residual operand is in tensor memory (and its S r slot read out): project
+      if (!s1::mbar_wait(aready, (uint32_t)j & 1u)) {
+        failed = true;
+        break;
+      }
+      s1::fence_after_sync();
+      projection();
+      // Y[b] is free again: rotate pass j+2 once its keys have landed
+      if (j + 2 < n_my) {
+        if (!wait_keys(b)) {
+          failed = true;
+          break;
+        }
+        rotation(b);
+      }
+    }
+    if (failed) {
+      // bounded: drain the issued MMAs and the outstanding key loads before the shared
+      // and tensor memory they use is released
+      s1::umma_commit(fin);
+      s1::mbar_wait(fin, 0u);
+      for (int b = 0; b < 2; ++b)
+        if ((kpend >> b) & 1u) s1::mbar_wait(kfull + b, (kpar >> b) & 1u);
+    }
   }
   if (__syncthreads_or(failed) && tid == 0) atomicOr(a.err, 1u);
   s1::fence_before_sync();
