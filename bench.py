@@ -58,6 +58,7 @@ def parse():
     ap.add_argument("--workload", default="llama8b_b32_32k_k3v2", choices=sorted(W.WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-paged", action="store_true", help="skip the paged-cache timings")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--decode-only", action="store_true",
@@ -407,6 +408,52 @@ def run_ours(args, w: W.Workload):
     gbs = job_throughput(packed_bytes * args.steps, world, dec_total) / 1e9
     vps = job_throughput(2 * n_vec * args.steps, world, comp_total) if not args.decode_only else None
 
+    # --- the same cache through the append / paged calls: the packed arrays scattered over
+    # pages of 512 tokens in a shuffled order (block table); compression through the
+    # matching slot map. Kernel times, L2 flushed before each, like the main loop.
+    paged_line = None
+    if not args.no_paged:
+        P = 512
+        mp = (w.tokens + P - 1) // P
+        n_pages = w.units * mp
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(5 + rank)
+        table = torch.randperm(n_pages, generator=gen, device=dev).view(w.units, mp).to(torch.int32)
+        tok = torch.arange(w.tokens, device=dev)
+        rows = (table[:, tok // P].long() * P + tok % P).reshape(-1)   # record row of token (u, t)
+        paged = {k: torch.empty((n_pages * P,) + tuple(v.shape[1:]), dtype=v.dtype, device=dev)
+                 for k, v in packed.items()}
+        for k in packed:
+            paged[k].index_copy_(0, rows, packed[k])
+        bt = table.view(w.batch, w.hkv, mp).contiguous()
+        pdec, pcomp = [], []
+        for it in range(args.warmup + args.steps):
+            e = [E(enable_timing=True) for _ in range(4)]
+            for ev in e:
+                ev.record()
+            flush_l2()
+            T.tq_set_profile_events(ctx, e[0], e[1])
+            T.tq_decode_attention_paged(ctx, Q, paged, w.batch, w.hq, w.hkv, w.tokens, bt, P, n_pages,
+                                        out=out, workspace=ws)
+            if not args.decode_only:
+                flush_l2()
+                T.tq_set_profile_events(ctx, e[2], e[3])
+                T.tq_compress_kv_slots(ctx, K, V, rows, paged)
+            T.tq_set_profile_events(ctx, None, None)
+            if it >= args.warmup:
+                pdec.append(e)
+        torch.cuda.synchronize()
+        T.tq_check_device(ctx)
+        pd = slowest(statistics.fmean(e[0].elapsed_time(e[1]) for e in pdec) / 1e3)
+        paged_line = {"page_size": P, "pages": n_pages, "block_order": "shuffled",
+                      "decode_main_kernel_ms": pd * 1e3,
+                      "decode_gbs": job_throughput(packed_bytes, world, pd) / 1e9}
+        if not args.decode_only:
+            pc = slowest(statistics.fmean(e[2].elapsed_time(e[3]) for e in pdec) / 1e3)
+            paged_line.update({"compress_slots_kernel_ms": pc * 1e3,
+                               "compress_slots_vectors_per_s": job_throughput(2 * n_vec, world, pc)})
+        del paged, rows, table, bt
+
     # --- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
@@ -494,6 +541,7 @@ def run_ours(args, w: W.Workload):
                 "kernel_ms": statistics.fmean(comp_k)},
             "decode_ms": {"call": dec_total * 1e3 / args.steps, "main_kernel": dec_k_mean * 1e3,
                           "main_kernel_timing": "separate loop of `steps` steps with events around the kernel"},
+            "paged": paged_line,
             "roofline": roof,
             "roofline_decode": roof_dec,
             "cpu_baseline": cpu,

@@ -145,6 +145,19 @@ tq_status tq_compress_kv(const tq_ctx* ctx, const void* k, const void* v, tq_dty
                          int64_t n_vec, uint8_t* k_codes, uint8_t* k_signs, uint16_t* k_norms,
                          uint8_t* v_codes, uint16_t* v_params, void* stream);
 
+/* tq_compress_kv with a slot map: vector i's records go to row slot[i] of the output
+ * arrays instead of row i. This appends new tokens to a growing cache in place (slots
+ * after each sequence's last token) and fills paged layouts (slots inside pages). The
+ * arrays hold n_rows records; rows not named by the map are not touched.
+ *   slot    device int64 [n_vec], 8-byte aligned; distinct entries in [0, n_rows).
+ *           An entry outside that range is not written and sets the context's device
+ *           error word (tq_check_device then returns TQ_EINVAL).
+ * Other arguments, ownership and errors as tq_compress_kv; NULL slot is TQ_EINVAL. */
+tq_status tq_compress_kv_slots(const tq_ctx* ctx, const void* k, const void* v, tq_dtype dtype,
+                               int64_t n_vec, const int64_t* slot, int64_t n_rows, uint8_t* k_codes,
+                               uint8_t* k_signs, uint16_t* k_norms, uint8_t* v_codes,
+                               uint16_t* v_params, void* stream);
+
 /* Bytes of device workspace tq_decode_attention needs for this shape (split-K
  * partials and prepared queries). Returns 0 for invalid arguments. */
 size_t tq_decode_workspace_bytes(const tq_ctx* ctx, int batch, int hq, int hkv, int64_t max_len);
@@ -171,12 +184,35 @@ tq_status tq_decode_attention(const tq_ctx* ctx, const void* q, tq_dtype q_dtype
                               const uint16_t* v_params, float softmax_scale, float* scores,
                               float* out, void* workspace, size_t workspace_bytes, void* stream);
 
+/* tq_decode_attention over a paged cache: the packed arrays hold n_pages pages of
+ * page_size consecutive records, each page belonging to one (sequence, KV head), in
+ * any order (filled e.g. by tq_compress_kv_slots).
+ *   block_table  device int32 [batch][hkv][max_pages], 16-byte aligned: the page that
+ *                holds tokens [j page_size, (j+1) page_size) of (sequence b, KV head h)
+ *                is block_table[(b hkv + h) max_pages + j]; only entries of blocks below
+ *                the sequence's length are read. An entry outside [0, n_pages) sets the
+ *                device error word (tq_check_device returns TQ_EINVAL) and reads page 0.
+ *   page_size    tokens per page, a positive multiple of 512 (a whole number of every
+ *                decode kernel's tiles)
+ *   max_pages    block-table entries per (sequence, KV head), >= ceil(max_len / page_size)
+ * max_len bounds seq_lens and sizes the scores rows; the workspace is the one
+ * tq_decode_workspace_bytes gives for the same shape. Other arguments and errors as
+ * tq_decode_attention. */
+tq_status tq_decode_attention_paged(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int batch,
+                                    int hq, int hkv, const int32_t* seq_lens, int64_t max_len,
+                                    const int32_t* block_table, int64_t page_size,
+                                    int64_t max_pages, int64_t n_pages, const uint8_t* k_codes,
+                                    const uint8_t* k_signs, const uint16_t* k_norms,
+                                    const uint8_t* v_codes, const uint16_t* v_params,
+                                    float softmax_scale, float* scores, float* out,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronize `stream`, then read and clear the context's device error word.
  * Kernels never spin without a bound: a wait for a staged copy that does not
  * complete in time sets this word, abandons the rest of its work and exits, so
  * the CUDA context stays usable. Returns TQ_ECUDA (with tq_last_error() saying
- * which wait) if any call since the last check hit such a timeout, TQ_OK
- * otherwise. */
+ * which wait) if any call since the last check hit such a timeout, TQ_EINVAL if a
+ * slot or page index was out of range, TQ_OK otherwise. */
 tq_status tq_check_device(const tq_ctx* ctx, void* stream);
 
 /* Decode attention that allocates nothing and takes no workspace. The paper has

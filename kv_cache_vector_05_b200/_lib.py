@@ -21,8 +21,8 @@ TQ_ROT_HADAMARD, TQ_ROT_HAAR = 0, 1
 
 EXPORTED = (
     "tq_codebook_load", "tq_free", "tq_status_string", "tq_last_error",
-    "tq_lloyd_max_codebook", "tq_haar_from_gaussian", "tq_compress_kv",
-    "tq_decode_workspace_bytes", "tq_decode_attention", "tq_decompress",
+    "tq_lloyd_max_codebook", "tq_haar_from_gaussian", "tq_compress_kv", "tq_compress_kv_slots",
+    "tq_decode_workspace_bytes", "tq_decode_attention", "tq_decode_attention_paged", "tq_decompress",
     "tq_set_profile_events", "tq_check_device", "tq_decode_attention_static", "tq_decode_static_scratch_capacity",
 )
 
@@ -70,11 +70,16 @@ def _load() -> ctypes.CDLL:
     lib.tq_haar_from_gaussian.restype = c_int
     lib.tq_compress_kv.argtypes = [vp, vp, vp, c_int, i64, vp, vp, vp, vp, vp, vp]
     lib.tq_compress_kv.restype = c_int
+    lib.tq_compress_kv_slots.argtypes = [vp, vp, vp, c_int, i64, vp, i64, vp, vp, vp, vp, vp, vp]
+    lib.tq_compress_kv_slots.restype = c_int
     lib.tq_decode_workspace_bytes.argtypes = [vp, c_int, c_int, c_int, i64]
     lib.tq_decode_workspace_bytes.restype = sz
     lib.tq_decode_attention.argtypes = [vp, vp, c_int, c_int, c_int, c_int, vp, i64,
                                         vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp, sz, vp]
     lib.tq_decode_attention.restype = c_int
+    lib.tq_decode_attention_paged.argtypes = [vp, vp, c_int, c_int, c_int, c_int, vp, i64, vp, i64, i64, i64,
+                                              vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp, sz, vp]
+    lib.tq_decode_attention_paged.restype = c_int
     lib.tq_decompress.argtypes = [vp, vp, vp, vp, vp, vp, i64, vp, vp, vp]
     lib.tq_decompress.restype = c_int
     lib.tq_decode_attention_static.argtypes = [vp, vp, c_int, c_int, c_int, c_int, vp, i64,
@@ -244,6 +249,28 @@ def tq_compress_kv(ctx: Context, k, v, k_codes=None, k_signs=None, k_norms=None,
     return out
 
 
+def tq_compress_kv_slots(ctx: Context, k, v, slot, packed: dict, stream=None) -> dict:
+    """Compress keys and/or values (torch CUDA tensors [n, d]) into the existing packed arrays
+    of `packed` (k_codes ... v_params, each [n_rows, ...]), vector i into row slot[i]
+    (int64 CUDA tensor [n]). Returns `packed`."""
+    import torch
+    src = k if k is not None else v
+    n = src.shape[0]
+    dtype = TQ_F32 if src.dtype == torch.float32 else TQ_BF16
+    for t in (k, v):
+        if t is not None:
+            assert t.is_contiguous() and t.shape == (n, ctx.d) and t.dtype == src.dtype
+    assert slot.is_contiguous() and slot.dtype == torch.int64 and slot.numel() == n
+    ref = packed["k_codes"] if k is not None else packed["v_codes"]
+    n_rows = ref.shape[0]
+    _check(lib.tq_compress_kv_slots(
+        ctx.handle, _ptr(k), _ptr(v), dtype, n, _ptr(slot), n_rows,
+        _ptr(packed.get("k_codes") if k is not None else None), _ptr(packed.get("k_signs") if k is not None else None),
+        _ptr(packed.get("k_norms") if k is not None else None), _ptr(packed.get("v_codes") if v is not None else None),
+        _ptr(packed.get("v_params") if v is not None else None), _stream(stream)), "tq_compress_kv_slots")
+    return packed
+
+
 def tq_decode_workspace_bytes(ctx: Context, batch: int, hq: int, hkv: int, max_len: int) -> int:
     return int(lib.tq_decode_workspace_bytes(ctx.handle, batch, hq, hkv, max_len))
 
@@ -268,6 +295,32 @@ def tq_decode_attention(ctx: Context, q, packed: dict, batch: int, hq: int, hkv:
         _ptr(packed["k_codes"]), _ptr(packed["k_signs"]), _ptr(packed["k_norms"]),
         _ptr(packed["v_codes"]), _ptr(packed["v_params"]), float(softmax_scale),
         _ptr(scores), _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)), "tq_decode_attention")
+    return out, scores
+
+
+def tq_decode_attention_paged(ctx: Context, q, packed: dict, batch: int, hq: int, hkv: int, max_len: int,
+                              block_table, page_size: int, n_pages: int, seq_lens=None,
+                              softmax_scale: float = 0.0, scores=None, out=None, workspace=None, stream=None):
+    """Decode attention over a paged cache: the packed arrays hold n_pages pages of page_size
+    records; block_table (int32 [batch, hkv, max_pages]) names the page of each block of
+    page_size tokens. Returns (out [batch, hq, d] fp32, scores or None)."""
+    import torch
+    dev = q.device
+    q_dtype = TQ_F32 if q.dtype == torch.float32 else TQ_BF16
+    assert q.is_contiguous() and q.numel() == batch * hq * ctx.d
+    assert block_table.is_contiguous() and block_table.dtype == torch.int32 and block_table.dim() == 3
+    if out is None:
+        out = torch.empty((batch, hq, ctx.d), dtype=torch.float32, device=dev)
+    need = tq_decode_workspace_bytes(ctx, batch, hq, hkv, max_len)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.tq_decode_attention_paged(
+        ctx.handle, _ptr(q), q_dtype, batch, hq, hkv, _ptr(seq_lens), max_len, _ptr(block_table),
+        int(page_size), int(block_table.shape[2]), int(n_pages),
+        _ptr(packed["k_codes"]), _ptr(packed["k_signs"]), _ptr(packed["k_norms"]),
+        _ptr(packed["v_codes"]), _ptr(packed["v_params"]), float(softmax_scale),
+        _ptr(scores), _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)), "tq_decode_attention_paged")
     return out, scores
 
 

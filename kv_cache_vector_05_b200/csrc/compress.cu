@@ -38,15 +38,29 @@ struct CompressArgs {
   Codebook cb;
   int lm_bits, m, v_bits, rot;
   float inv_sqrt_d;  // 1/sqrt(d) rounded once from fp64
+  const int64_t* slot;  // output row of each input vector (null: row i), each in [0, n_rows)
+  int64_t n_rows;       // rows the output arrays hold (slot mode)
   CUtensorMap kmap;  // compress_pipe_kernel: bf16 keys [n_vec][128], 64 x 128 boxes, 128-byte swizzle
   CUtensorMap vmap;  // compress_pipe_kernel: bf16 values [n_vec][128], 64 x 64 boxes, 128-byte swizzle
 };
+
+// Output row of input vector i: slot[i] when a slot map is given, else i. A slot outside
+// [0, n_rows) sets bit 2 of the error word and gives -1: that vector is not written.
+__device__ __forceinline__ int64_t out_row(const CompressArgs& a, int64_t i) {
+  if (!a.slot) return i;
+  const int64_t o = __ldg(a.slot + i);
+  if (o < 0 || o >= a.n_rows) {
+    atomicOr(a.err, 4u);
+    return -1;
+  }
+  return o;
+}
 
 // Norm, rotation, Lloyd-Max codes and residual of key i; writes the packed codes
 // and (n, gamma). Returns false for a zero key (all its bytes already written as 0);
 // otherwise leaves the lane's residual coordinates in r.
 template <int D, typename T, int LMB = 0>
-__device__ bool key_front(const CompressArgs& a, int64_t i, int lane, float* rbuf, float (&r)[D / 32]) {
+__device__ bool key_front(const CompressArgs& a, int64_t i, int64_t o, int lane, float* rbuf, float (&r)[D / 32]) {
   constexpr int E = D / 32;
   const int lmb = LMB ? LMB : a.lm_bits;       // compile-time when specialised
   const int levels = LMB ? (1 << LMB) : a.cb.levels;
@@ -59,12 +73,12 @@ __device__ bool key_front(const CompressArgs& a, int64_t i, int lane, float* rbu
   const float n = sqrtf(warp_sum(ss));
 
   const int cbytes = lmb * D / 8;
-  uint32_t* codes_out = reinterpret_cast<uint32_t*>(a.k_codes + i * cbytes);
-  uint32_t* signs_out = reinterpret_cast<uint32_t*>(a.k_signs + i * (a.m / 8));
+  uint32_t* codes_out = reinterpret_cast<uint32_t*>(a.k_codes + o * cbytes);
+  uint32_t* signs_out = reinterpret_cast<uint32_t*>(a.k_signs + o * (a.m / 8));
   if (n == 0.f) {  // a zero key is stored as zero bytes
     if (lane < cbytes / 4) codes_out[lane] = 0u;
     if (lane < a.m / 32) signs_out[lane] = 0u;
-    if (lane == 0) reinterpret_cast<uint32_t*>(a.k_norms)[i] = 0u;
+    if (lane == 0) reinterpret_cast<uint32_t*>(a.k_norms)[o] = 0u;
     return false;
   }
   const float inv_n = 1.0f / n;
@@ -117,7 +131,7 @@ __device__ bool key_front(const CompressArgs& a, int64_t i, int lane, float* rbu
   if (lane == 0) {
     const uint32_t nb = __half_as_ushort(__float2half_rn(n));
     const uint32_t gb = __half_as_ushort(__float2half_rn(gamma));
-    reinterpret_cast<uint32_t*>(a.k_norms)[i] = nb | (gb << 16);
+    reinterpret_cast<uint32_t*>(a.k_norms)[o] = nb | (gb << 16);
   }
   return true;
 }
@@ -126,7 +140,8 @@ template <int D, typename T>
 __device__ void compress_key(const CompressArgs& a, int64_t i, int lane, float* rbuf) {
   constexpr int E = D / 32;
   float r[E];
-  if (!key_front<D, T>(a, i, lane, rbuf, r)) return;
+  const int64_t o = out_row(a, i);  // the same in every lane
+  if (o < 0 || !key_front<D, T>(a, i, o, lane, rbuf, r)) return;
   // QJL: sign bits of S r; lane computes rows i = lane + 32*q so a ballot gives word q.
 #pragma unroll
   for (int e = 0; e < E; ++e) rbuf[lane * E + e] = r[e];
@@ -140,7 +155,7 @@ __device__ void compress_key(const CompressArgs& a, int64_t i, int lane, float* 
     if (lane == q) my_sign_word = word;
   }
   __syncwarp();
-  if (lane < a.m / 32) reinterpret_cast<uint32_t*>(a.k_signs + i * (a.m / 8))[lane] = my_sign_word;
+  if (lane < a.m / 32) reinterpret_cast<uint32_t*>(a.k_signs + o * (a.m / 8))[lane] = my_sign_word;
 }
 
 template <int D, typename T, int VB = 0>
@@ -148,6 +163,8 @@ __device__ void compress_value(const CompressArgs& a, int64_t i, int lane) {
   constexpr int E = D / 32;
   constexpr int W = 32 / E;  // lanes per group of 32 coordinates
   const int vbits = VB ? VB : a.v_bits;
+  const int64_t o = out_row(a, i);  // the same in every lane
+  if (o < 0) return;
   float x[E];
   load_lane<E>(static_cast<const T*>(a.v) + i * D, lane, x);
   float lo = x[0], hi = x[0];
@@ -177,11 +194,11 @@ __device__ void compress_value(const CompressArgs& a, int64_t i, int lane) {
   const int cbytes = vbits * D / 8;
   const uint32_t word = VB ? pack_stream_word_t<E * VB, VB * D / 32>(code_bits, lane)
                            : pack_stream_word(code_bits, E * vbits, cbytes / 4, lane);
-  if (lane < cbytes / 4) reinterpret_cast<uint32_t*>(a.v_codes + i * cbytes)[lane] = word;
+  if (lane < cbytes / 4) reinterpret_cast<uint32_t*>(a.v_codes + o * cbytes)[lane] = word;
   if ((lane % W) == 0) {
     const uint32_t sb = __half_as_ushort(__double2half(scale));
     const uint32_t mb = __half_as_ushort(__float2half_rn(lo));
-    reinterpret_cast<uint32_t*>(a.v_params)[i * (D / kVGroup) + lane / W] = sb | (mb << 16);
+    reinterpret_cast<uint32_t*>(a.v_params)[o * (D / kVGroup) + lane / W] = sb | (mb << 16);
   }
 }
 
@@ -286,8 +303,9 @@ __global__ void __launch_bounds__(kTcThreads, 2) compress_tc_kernel(const __grid
         for (int vv = 0; vv < 32; ++vv) {
           const int row = warp * 32 + vv;
           if (row >= nrows) break;
-          float r[4];
-          const bool nz = key_front<128, T, LMB>(a, v0 + row, lane, rbuf + warp * 128, r);
+          float r[4] = {0.f, 0.f, 0.f, 0.f};
+          const int64_t o = out_row(a, v0 + row);  // the same in every lane
+          const bool nz = o >= 0 && key_front<128, T, LMB>(a, v0 + row, o, lane, rbuf + warp * 128, r);
           // residual coordinates 4 lane .. 4 lane + 3, scaled by 16 (signs unchanged)
           float x[4];
 #pragma unroll
@@ -341,10 +359,11 @@ __global__ void __launch_bounds__(kTcThreads, 2) compress_tc_kernel(const __grid
           words[q] = bits;
         }
         const int row = 32 * warp + lane;
-        if (row < nrows) {
+        const int64_t so = row < nrows ? out_row(a, v0 + row) : -1;
+        if (so >= 0) {
           const bool nz = zf[row] != 0;
           uint4 w4 = nz ? make_uint4(words[0], words[1], words[2], words[3]) : make_uint4(0u, 0u, 0u, 0u);
-          *reinterpret_cast<uint4*>(a.k_signs + (v0 + row) * 16) = w4;
+          *reinterpret_cast<uint4*>(a.k_signs + so * 16) = w4;
         }
         s1::fence_before_sync();
         kwarps_sync_or(false);  // TMEM and the operand tiles are free for the next tile
@@ -524,6 +543,7 @@ __global__ void __launch_bounds__(kQ4Threads, 1) compress_q4_kernel(const __grid
   for (int64_t tile = blockIdx.x; tile < ntile; tile += gridDim.x) {
     const int64_t i = tile * kQ4Rows + R;
     const bool valid = i < a.n_vec;
+    const int64_t o = valid ? out_row(a, i) : -1;  // output row
 
     // The values' loads are issued first, so that they are in flight while the keys
     // are worked on (bf16: 4 x 16 bytes per lane).
@@ -585,14 +605,14 @@ __global__ void __launch_bounds__(kQ4Threads, 1) compress_q4_kernel(const __grid
       rr += __shfl_xor_sync(kFull, rr, 1);
       rr += __shfl_xor_sync(kFull, rr, 2);
       const float gamma = sqrtf(rr);
-      if (valid) {
-        uint32_t* co = reinterpret_cast<uint32_t*>(a.k_codes + i * (LMB * 16) + q * (LMB * 4));
+      if (o >= 0) {
+        uint32_t* co = reinterpret_cast<uint32_t*>(a.k_codes + o * (LMB * 16) + q * (LMB * 4));
 #pragma unroll
         for (int w = 0; w < KW; ++w) co[w] = nz ? cw[w] : 0u;
         if (q == 0) {
           const uint32_t nb = __half_as_ushort(__float2half_rn(n));
           const uint32_t gb = __half_as_ushort(__float2half_rn(gamma));
-          reinterpret_cast<uint32_t*>(a.k_norms)[i] = nz ? (nb | (gb << 16)) : 0u;
+          reinterpret_cast<uint32_t*>(a.k_norms)[o] = nz ? (nb | (gb << 16)) : 0u;
         }
       }
       // Residual x16 (signs unchanged) as f16 hi + lo into the operand tiles (the
@@ -633,7 +653,7 @@ __global__ void __launch_bounds__(kQ4Threads, 1) compress_q4_kernel(const __grid
     }
 
     // ---------------------------------------------------------------- values
-    if (a.v && valid) {
+    if (a.v && o >= 0) {
       float x[32];
       if constexpr (sizeof(T) == 2) {
 #pragma unroll
@@ -674,12 +694,12 @@ __global__ void __launch_bounds__(kQ4Threads, 1) compress_q4_kernel(const __grid
         qv = min(qv, (uint32_t)levels);
         put_bits<VB, VW>(vw, VB * e, qv);
       }
-      uint32_t* vo = reinterpret_cast<uint32_t*>(a.v_codes + i * (VB * 16) + q * (VB * 4));
+      uint32_t* vo = reinterpret_cast<uint32_t*>(a.v_codes + o * (VB * 16) + q * (VB * 4));
 #pragma unroll
       for (int w = 0; w < VW; ++w) vo[w] = vw[w];
       const uint32_t sb = __half_as_ushort(__double2half(span / levels));
       const uint32_t mb = __half_as_ushort(__float2half_rn(lo));
-      reinterpret_cast<uint32_t*>(a.v_params)[i * 4 + q] = sb | (mb << 16);
+      reinterpret_cast<uint32_t*>(a.v_params)[o * 4 + q] = sb | (mb << 16);
     }
 
     // ---------------------------------------------------------------- QJL signs
@@ -706,10 +726,11 @@ __global__ void __launch_bounds__(kQ4Threads, 1) compress_q4_kernel(const __grid
         }
         const int row = 32 * warp + lane;
         const int64_t ik = tile * kQ4Rows + row;
-        if (ik < a.n_vec) {
+        const int64_t so = ik < a.n_vec ? out_row(a, ik) : -1;
+        if (so >= 0) {
           const bool nzk = zf[row] != 0;
           const uint4 w4 = nzk ? make_uint4(words[0], words[1], words[2], words[3]) : make_uint4(0u, 0u, 0u, 0u);
-          *reinterpret_cast<uint4*>(a.k_signs + ik * 16) = w4;
+          *reinterpret_cast<uint4*>(a.k_signs + so * 16) = w4;
         }
       }
       s1::fence_before_sync();
@@ -801,7 +822,6 @@ template <int LMB, int VB, bool HAAR>
 __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __grid_constant__ CompressArgs a) {
   using RS = RotSmem<HAAR>;
   namespace s1 = tq::sm100;
-  constexpr int KW = 2 * LMB;  // code words per key thread (64 codes x LMB bits)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = s1::smem_u32(sm);
@@ -918,6 +938,7 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
       // ---------------------------------------------------------------- keys
       const int64_t i = v0 + R;
       const bool valid = i < a.n_vec;
+      const int64_t o = valid ? out_row(a, i) : -1;  // output row
       if (!failed && !s1::mbar_wait(bar1, phase)) failed = true;
       s1::fence_after_sync();
       // Two 32-column chunks per thread: a first pass for the norm, a second one (a loop
@@ -971,8 +992,8 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
           r[e] = yy - cv;
           r4[e & 3] = fmaf(r[e], r[e], r4[e & 3]);
         }
-        if (valid) {
-          uint32_t* co = reinterpret_cast<uint32_t*>(a.k_codes + i * (LMB * 16) + ch * (LMB * 8) + h * (LMB * 4));
+        if (o >= 0) {
+          uint32_t* co = reinterpret_cast<uint32_t*>(a.k_codes + o * (LMB * 16) + ch * (LMB * 8) + h * (LMB * 4));
 #pragma unroll
           for (int w = 0; w < CW; ++w) co[w] = nz ? (cw[w] | cw2[w]) : 0u;
         }
@@ -997,11 +1018,11 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
       xs[ch * 128 + R] = (r4[0] + r4[1]) + (r4[2] + r4[3]);
       key_warps_sync();
       const float gamma = sqrtf(xs[R] + xs[128 + R]);
-      if (valid && ch == 0) {
+      if (o >= 0 && ch == 0) {
         const float n = HAAR ? sqrtf(tot) : sqrtf(tot * (1.0f / 128.f));
         const uint32_t nb = __half_as_ushort(__float2half_rn(n));
         const uint32_t gb = __half_as_ushort(__float2half_rn(gamma));
-        reinterpret_cast<uint32_t*>(a.k_norms)[i] = nz ? (nb | (gb << 16)) : 0u;
+        reinterpret_cast<uint32_t*>(a.k_norms)[o] = nz ? (nb | (gb << 16)) : 0u;
       }
       if (ch == 0) zf[R] = use ? 1 : 0;
       s1::fence_async_smem();
@@ -1035,7 +1056,7 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
 #pragma unroll
           for (int g = 0; g < 4; ++g) b4[g] = __funnelshift_l(v[8 * g + k] ^ 0x80000000u, b4[g], 1);
         const uint32_t word = b4[0] | (b4[1] << 8) | (b4[2] << 16) | (b4[3] << 24);
-        if (valid) reinterpret_cast<uint32_t*>(a.k_signs + i * 16 + 8 * ch)[h] = nzk ? word : 0u;
+        if (o >= 0) reinterpret_cast<uint32_t*>(a.k_signs + o * 16 + 8 * ch)[h] = nzk ? word : 0u;
       }
       s1::fence_before_sync();
     } else if (!key_warp && a.v) {
@@ -1062,6 +1083,8 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
         const int row = (vt >> 2) + 64 * round;
         const int64_t i = v0 + row;
         if (i >= a.n_vec || failed) break;
+        const int64_t o = out_row(a, i);
+        if (o < 0) continue;
         float x[32];
         const uint4* p4 = reinterpret_cast<const uint4*>(sm + RS::VR + row * 256 + 64 * q);
 #pragma unroll
@@ -1106,12 +1129,12 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
         }
 #pragma unroll
         for (int w = 0; w < VB; ++w) vw[w] |= vw2[w];
-        uint32_t* vo = reinterpret_cast<uint32_t*>(a.v_codes + i * (VB * 16) + q * (VB * 4));
+        uint32_t* vo = reinterpret_cast<uint32_t*>(a.v_codes + o * (VB * 16) + q * (VB * 4));
 #pragma unroll
         for (int w = 0; w < VB; ++w) vo[w] = vw[w];
         const uint32_t sb = __half_as_ushort(__double2half(span / levels));
         const uint32_t mb = __half_as_ushort(__float2half_rn(lo));
-        reinterpret_cast<uint32_t*>(a.v_params)[i * 4 + q] = sb | (mb << 16);
+        reinterpret_cast<uint32_t*>(a.v_params)[o * 4 + q] = sb | (mb << 16);
       }
       if constexpr (!HAAR) {
         // every value thread has read VR: fetch the next pass's values
@@ -1296,8 +1319,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
 #pragma unroll
       for (int j = 0; j < HL; ++j) cm[j] = 16.f * a.cb.c[HL + j];
       // Sign readout of a pass whose projection has completed: bit j set <=> (S r)_j >= 0.
-      auto read_signs = [&](int64_t pv0, bool nzk) {
-        const int64_t pi = pv0 + R;
+      auto read_signs = [&](int64_t po, bool nzk) {  // po: the row's output row, or -1
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
           uint32_t v[32];
@@ -1309,16 +1331,16 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
 #pragma unroll
             for (int q = 0; q < 4; ++q) b4[q] = __funnelshift_l(v[8 * q + k], b4[q], 1);
           const uint32_t word = ~(b4[0] | (b4[1] << 8) | (b4[2] << 16) | (b4[3] << 24));
-          if (pi < a.n_vec) reinterpret_cast<uint32_t*>(a.k_signs + pi * 16 + 8 * ch)[h] = nzk ? word : 0u;
+          if (po >= 0) reinterpret_cast<uint32_t*>(a.k_signs + po * 16 + 8 * ch)[h] = nzk ? word : 0u;
         }
       };
       int it = 0;
-      int64_t prev_v0 = 0;
-      bool prev_nz = false;  // the previous pass's key of this row was stored as nonzero
+      int64_t prev_o = -1;   // the previous pass's output row of this row's key (-1: none)
+      bool prev_nz = false;  // and whether it was stored as nonzero
       for (int64_t tile = blockIdx.x; tile < ntile; tile += g, ++it) {
         const int b = it & 1;
         const int64_t v0 = tile * 128, i = v0 + R;
-        const bool valid = i < a.n_vec;
+        const int64_t o = i < a.n_vec ? out_row(a, i) : -1;  // output row
         if (!failed && !s1::mbar_wait(rotd + b, (uint32_t)(it >> 1) & 1u)) failed = true;
         s1::fence_after_sync();
         // ||Y||^2 over the row's 128 columns, as two 64-column halves of four chains each
@@ -1349,7 +1371,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
         if (it > 0) {
           if (!failed && !s1::mbar_wait(projd, (uint32_t)(it - 1) & 1u)) failed = true;
           s1::fence_after_sync();
-          read_signs(prev_v0, prev_nz);
+          read_signs(prev_o, prev_nz);
         }
         float2 ra = make_float2(0.f, 0.f), rb = make_float2(0.f, 0.f);  // r^2 chains (0,1), (2,3)
 #pragma unroll 1
@@ -1386,8 +1408,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
             s1::tmem_st8(tmem + kTmA + lane_base + col, hw);
             s1::tmem_st8(tmem + kTmA + 64 + lane_base + col, lw);
           }
-          if (valid) {
-            uint32_t* co = reinterpret_cast<uint32_t*>(a.k_codes + i * (LMB * 16) + ch * (LMB * 8) + h * (LMB * 4));
+          if (o >= 0) {
+            uint32_t* co = reinterpret_cast<uint32_t*>(a.k_codes + o * (LMB * 16) + ch * (LMB * 8) + h * (LMB * 4));
 #pragma unroll
             for (int w = 0; w < LMB; ++w) co[w] = nz ? (cw[w] | cw2[w]) : 0u;
           }
@@ -1400,14 +1422,14 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
         if (lane == 0) s1::mbar_arrive(aready);
         failed = s1::bar_sync_or<1, 256>(failed);
         if (failed) break;
-        if (ch == 0 && valid) {
+        if (ch == 0 && o >= 0) {
           const float gamma = sqrtf(xr[b * 256 + R] + xr[b * 256 + 128 + R]) * (1.f / 16.f);
           const uint32_t nb = __half_as_ushort(__float2half_rn(sqrtf(tot * (1.0f / 128.f))));
           const uint32_t gb = __half_as_ushort(__float2half_rn(gamma));
-          reinterpret_cast<uint32_t*>(a.k_norms)[i] = nz ? (nb | (gb << 16)) : 0u;
+          reinterpret_cast<uint32_t*>(a.k_norms)[o] = nz ? (nb | (gb << 16)) : 0u;
         }
-        prev_v0 = v0;
-        prev_nz = valid && nz;
+        prev_o = o;
+        prev_nz = nz;
       }
       // the last pass's signs
       if (!failed && it > 0) {
@@ -1415,7 +1437,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
           failed = true;
         } else {
           s1::fence_after_sync();
-          read_signs(prev_v0, prev_nz);
+          read_signs(prev_o, prev_nz);
         }
       }
     }
@@ -1470,7 +1492,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
           }
         }
         const int64_t i = r0 + vrow;
-        if (!failed && i < a.n_vec) {
+        const int64_t o = i < a.n_vec ? out_row(a, i) : -1;  // output row
+        if (!failed && o >= 0) {
           const unsigned char* half = sm + PS::VR + f * (kTcTileBytes / 2);
           uint32_t w[16];
 #pragma unroll
@@ -1552,12 +1575,12 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
               }
             }
           }
-          uint32_t* vo = reinterpret_cast<uint32_t*>(a.v_codes + i * (VB * 16) + q * (VB * 4));
+          uint32_t* vo = reinterpret_cast<uint32_t*>(a.v_codes + o * (VB * 16) + q * (VB * 4));
 #pragma unroll
           for (int k = 0; k < VB; ++k) vo[k] = vw[k];
           const uint32_t sb = __half_as_ushort(__double2half(span / levels));
           const uint32_t mb = __half_as_ushort(__float2half_rn(lo));
-          reinterpret_cast<uint32_t*>(a.v_params)[i * 4 + q] = sb | (mb << 16);
+          reinterpret_cast<uint32_t*>(a.v_params)[o * 4 + q] = sb | (mb << 16);
         }
         // every value thread is done with this half: refill it two passes ahead
         failed = s1::bar_sync_or<2, 256>(failed);
@@ -1793,12 +1816,14 @@ void pack_haar_operand(const double* pi, uint16_t* out) {
 }
 
 cudaError_t launch_compress(const tq_ctx* ctx, const void* k, const void* v, int dtype, int64_t n_vec,
-                            uint8_t* k_codes, uint8_t* k_signs, uint16_t* k_norms, uint8_t* v_codes,
-                            uint16_t* v_params, cudaStream_t stream) {
+                            const int64_t* slot, int64_t n_rows, uint8_t* k_codes, uint8_t* k_signs,
+                            uint16_t* k_norms, uint8_t* v_codes, uint16_t* v_params, cudaStream_t stream) {
   CompressArgs a;
   a.k = k;
   a.v = v;
   a.n_vec = n_vec;
+  a.slot = slot;
+  a.n_rows = n_rows;
   a.k_codes = k_codes;
   a.k_signs = k_signs;
   a.k_norms = k_norms;

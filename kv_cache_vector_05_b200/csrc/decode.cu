@@ -87,6 +87,8 @@ struct DecodeArgs {
   const uint16_t* v_params;
   const int32_t* seq_lens;
   int64_t max_len;
+  Paging pg;           // contiguous or paged cache addressing
+  unsigned int* err;   // device error word (bit 2: a page index out of range)
   int hq, hkv, G, m;
   int n_chunks;
   int64_t chunk_len;
@@ -125,7 +127,6 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
   const int64_t t0 = (int64_t)chunk * a.chunk_len;
   const int64_t t1 = min(t0 + a.chunk_len, len);
   const int qrow0 = b * a.hq + kvh * G;
-  const int64_t vec0 = (int64_t)unit * a.max_len;
 
   for (int idx = tid; idx < G * D; idx += kThreads) {
     const int h = idx / D, j = idx % D;
@@ -157,16 +158,17 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
   const float qjl = kQjl / (float)M;
   for (int64_t tt = t0; tt < t1; tt += kTile) {
     const int nt = (int)min((int64_t)kTile, t1 - tt);
+    const int64_t row0 = record_row(a.pg, a.max_len, unit, tt, a.err);  // the tile's first record
     // Stage this tile's value codes and (scale, min) pairs.
-    const uint32_t* vsrc = reinterpret_cast<const uint32_t*>(a.v_codes + (vec0 + tt) * (VW * 4));
+    const uint32_t* vsrc = reinterpret_cast<const uint32_t*>(a.v_codes + row0 * (VW * 4));
     for (int w = tid; w < nt * VW; w += kThreads) vcode_s[w] = vsrc[w];
-    const uint32_t* psrc = reinterpret_cast<const uint32_t*>(a.v_params) + (vec0 + tt) * NG;
+    const uint32_t* psrc = reinterpret_cast<const uint32_t*>(a.v_params) + row0 * NG;
     for (int w = tid; w < nt * NG; w += kThreads) vpar_s[w] = psrc[w];
 
     // Logits: thread (token tl, slice sl) scores heads sl, sl + kSlices, ...
     const int tl = tid % kTile, sl = tid / kTile;
     if (tl < nt) {
-      const int64_t vec = vec0 + tt + tl;
+      const int64_t vec = row0 + tl;
       const uint32_t* ksrc = reinterpret_cast<const uint32_t*>(a.k_codes + vec * (KW * 4));
       uint32_t sw[kMaxM / 32];
       const uint32_t* ssrc = reinterpret_cast<const uint32_t*>(a.k_signs + vec * (M / 8));
@@ -399,13 +401,14 @@ DecodePlan plan_decode(const tq_ctx* ctx, int batch, int hq, int hkv, int64_t ma
 }
 
 cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const void* q, int q_dtype, int batch,
-                          int hq, int hkv, const int32_t* seq_lens, int64_t max_len, const uint8_t* k_codes,
+                          int hq, int hkv, const int32_t* seq_lens, int64_t max_len, const Paging& pg,
+                          const uint8_t* k_codes,
                           const uint8_t* k_signs, const uint16_t* k_norms, const uint8_t* v_codes,
                           const uint16_t* v_params, float scale, float* scores, float* out, void* workspace,
                           cudaStream_t stream) {
   const int d = ctx->shape.d, m = ctx->shape.m, G = hq / hkv;
   if (plan.mma)
-    return launch_decode_mma(ctx, plan, q, q_dtype, batch, hq, hkv, seq_lens, max_len, k_codes, k_signs,
+    return launch_decode_mma(ctx, plan, q, q_dtype, batch, hq, hkv, seq_lens, max_len, pg, k_codes, k_signs,
                              k_norms, v_codes, v_params, scale, scores, out, workspace, stream);
   if ((G + (kThreads / d) - 1) / (kThreads / d) > kMaxQ) return cudaErrorInvalidValue;
   float* ws_q = static_cast<float*>(workspace);
@@ -437,6 +440,8 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const void*
   a.v_params = v_params;
   a.seq_lens = seq_lens;
   a.max_len = max_len;
+  a.pg = pg;
+  a.err = ctx->d_err;
   a.hq = hq;
   a.hkv = hkv;
   a.G = G;

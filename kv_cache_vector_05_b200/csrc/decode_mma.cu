@@ -99,6 +99,7 @@ struct MmaArgs {
   const uint16_t* v_params;
   const int32_t* seq_lens;
   int64_t max_len;
+  Paging pg;               // contiguous or paged cache addressing
   int hq, hkv, G;
   int64_t tiles_per_unit;  // tiles of each (sequence, KV head), from max_len
   int64_t total_tiles;     // units x tiles_per_unit; CTA k takes [k T / P, (k + 1) T / P)
@@ -470,7 +471,7 @@ __global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid
       return;
     }
     unsigned char* st = stage_base + (i % NST) * L::STAGE;
-    const int64_t v = (int64_t)u * a.max_len + tok0;
+    const int64_t v = record_row(a.pg, a.max_len, u, tok0, a.err);
     issued_s[i % NST] += 1;
     mbar_expect_tx(bar, (uint32_t)L::STAGE);
     bulk_g2s(st + L::OFF_KC, a.k_codes + v * L::KCB, TILE * L::KCB, bar);
@@ -633,7 +634,7 @@ __global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid
       // Ragged or unaligned tile: plain 4-byte copies (all record sizes are multiples
       // of 4), after every warp has left the tile that used this stage before.
       __syncthreads();
-      const int64_t v = (int64_t)u * a.max_len + tok0;
+      const int64_t v = record_row(a.pg, a.max_len, u, tok0, a.err);
       auto copy = [&](int off, const void* src, int bytes_per_tok) {
         const uint32_t* s32 =
             reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(src) + v * bytes_per_tok);
@@ -1027,7 +1028,8 @@ size_t mma_frag_bytes(int lm_bits, int G) { return (size_t)frag_words(lm_bits, n
 int mma_tile_tokens(int G) { return tile_tokens(n_blocks(G)); }
 
 cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const void* q, int q_dtype, int batch,
-                              int hq, int hkv, const int32_t* seq_lens, int64_t max_len, const uint8_t* k_codes,
+                              int hq, int hkv, const int32_t* seq_lens, int64_t max_len, const Paging& pg,
+                              const uint8_t* k_codes,
                               const uint8_t* k_signs, const uint16_t* k_norms, const uint8_t* v_codes,
                               const uint16_t* v_params, float scale, float* scores, float* out, void* workspace,
                               cudaStream_t stream) {
@@ -1080,6 +1082,7 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
   a.v_params = v_params;
   a.seq_lens = seq_lens;
   a.max_len = max_len;
+  a.pg = pg;
   a.hq = hq;
   a.hkv = hkv;
   a.G = G;

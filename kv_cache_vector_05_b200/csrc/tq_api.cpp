@@ -1,6 +1,7 @@
 // C ABI entry points: argument validation, context management and dispatch to
 // the kernel launchers. No exception crosses this boundary.
 #include <cmath>
+#include <string>
 #include <cstdio>
 #include <cstring>
 #include <new>
@@ -16,6 +17,7 @@ tq_status fail(tq_status st, const char* msg) {
   std::snprintf(g_last_error, sizeof(g_last_error), "%s", msg);
   return st;
 }
+tq_status fail(tq_status st, const std::string& msg) { return fail(st, msg.c_str()); }
 
 tq_status fail_cuda(cudaError_t e, const char* where) {
   std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)", where, cudaGetErrorName(e),
@@ -223,6 +225,9 @@ tq_status tq_check_device(const tq_ctx* c, void* stream) {
   if (e == cudaSuccess && flag) e = cudaMemset(c->d_err, 0, sizeof(flag));
   if (e != cudaSuccess) return fail_cuda(e, "tq_check_device");
   if (flag & 1u) return fail(TQ_ECUDA, "tq_check_device: a bounded wait for a bulk copy timed out; results of that call are invalid");
+  if (flag & 4u)
+    return fail(TQ_EINVAL, "tq_check_device: a slot or page index was outside the caller's arrays; those vectors "
+                           "were not written (compression) or read as page 0 (decode)");
   return TQ_OK;
 }
 
@@ -232,27 +237,46 @@ void tq_free(tq_ctx* c) {
   delete c;
 }
 
+namespace {
+// Shared by tq_compress_kv (slot = NULL: vector i to row i) and tq_compress_kv_slots.
+tq_status compress_impl(const char* name, const tq_ctx* c, const void* k, const void* v, tq_dtype dtype,
+                        int64_t n_vec, const int64_t* slot, int64_t n_rows, uint8_t* k_codes, uint8_t* k_signs,
+                        uint16_t* k_norms, uint8_t* v_codes, uint16_t* v_params, void* stream) {
+  const std::string nm(name);
+  if (!c) return fail(TQ_EINVAL, nm + ": NULL context");
+  if (n_vec < 0) return fail(TQ_EINVAL, nm + ": negative n_vec");
+  if (dtype != TQ_F32 && dtype != TQ_BF16) return fail(TQ_EINVAL, nm + ": bad dtype");
+  if (!k && !v) return fail(TQ_EINVAL, nm + ": both k and v are NULL");
+  if (k && (!k_codes || !k_signs || !k_norms)) return fail(TQ_EINVAL, nm + ": NULL key output");
+  if (v && (!v_codes || !v_params)) return fail(TQ_EINVAL, nm + ": NULL value output");
+  if (k && !(aligned16(k) && aligned16(k_codes) && aligned16(k_signs) && aligned16(k_norms)))
+    return fail(TQ_EINVAL, nm + ": key pointers must be 16-byte aligned");
+  if (v && !(aligned16(v) && aligned16(v_codes) && aligned16(v_params)))
+    return fail(TQ_EINVAL, nm + ": value pointers must be 16-byte aligned");
+  if (slot && ((reinterpret_cast<uintptr_t>(slot) & 7u) || n_rows <= 0))
+    return fail(TQ_EINVAL, nm + ": the slot map must be 8-byte aligned and n_rows positive");
+  if (n_vec == 0) return TQ_OK;
+  if (n_vec > (int64_t(1) << 40)) return fail(TQ_EINVAL, nm + ": n_vec too large");
+  cudaError_t e = tq::launch_compress(c, k, v, (int)dtype, n_vec, slot, n_rows, k_codes, k_signs, k_norms,
+                                      v_codes, v_params, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e, name);
+  return TQ_OK;
+}
+}  // namespace
+
 tq_status tq_compress_kv(const tq_ctx* c, const void* k, const void* v, tq_dtype dtype, int64_t n_vec,
                          uint8_t* k_codes, uint8_t* k_signs, uint16_t* k_norms, uint8_t* v_codes,
                          uint16_t* v_params, void* stream) {
-  if (!c) return fail(TQ_EINVAL, "tq_compress_kv: NULL context");
-  if (n_vec < 0) return fail(TQ_EINVAL, "tq_compress_kv: negative n_vec");
-  if (n_vec == 0) return TQ_OK;
-  if (dtype != TQ_F32 && dtype != TQ_BF16) return fail(TQ_EINVAL, "tq_compress_kv: bad dtype");
-  if (!k && !v) return fail(TQ_EINVAL, "tq_compress_kv: both k and v are NULL");
-  if (k && (!k_codes || !k_signs || !k_norms))
-    return fail(TQ_EINVAL, "tq_compress_kv: NULL key output");
-  if (v && (!v_codes || !v_params)) return fail(TQ_EINVAL, "tq_compress_kv: NULL value output");
-  if (k && !(aligned16(k) && aligned16(k_codes) && aligned16(k_signs) && aligned16(k_norms)))
-    return fail(TQ_EINVAL, "tq_compress_kv: key pointers must be 16-byte aligned");
-  if (v && !(aligned16(v) && aligned16(v_codes) && aligned16(v_params)))
-    return fail(TQ_EINVAL, "tq_compress_kv: value pointers must be 16-byte aligned");
-  if (n_vec == 0) return TQ_OK;
-  if (n_vec > (int64_t(1) << 40)) return fail(TQ_EINVAL, "tq_compress_kv: n_vec too large");
-  cudaError_t e = tq::launch_compress(c, k, v, (int)dtype, n_vec, k_codes, k_signs, k_norms, v_codes,
-                                      v_params, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return fail_cuda(e, "tq_compress_kv");
-  return TQ_OK;
+  return compress_impl("tq_compress_kv", c, k, v, dtype, n_vec, nullptr, 0, k_codes, k_signs, k_norms, v_codes,
+                       v_params, stream);
+}
+
+tq_status tq_compress_kv_slots(const tq_ctx* c, const void* k, const void* v, tq_dtype dtype, int64_t n_vec,
+                               const int64_t* slot, int64_t n_rows, uint8_t* k_codes, uint8_t* k_signs,
+                               uint16_t* k_norms, uint8_t* v_codes, uint16_t* v_params, void* stream) {
+  if (!slot) return fail(TQ_EINVAL, "tq_compress_kv_slots: NULL slot map");
+  return compress_impl("tq_compress_kv_slots", c, k, v, dtype, n_vec, slot, n_rows, k_codes, k_signs, k_norms,
+                       v_codes, v_params, stream);
 }
 
 size_t tq_decode_workspace_bytes(const tq_ctx* c, int batch, int hq, int hkv, int64_t max_len) {
@@ -260,37 +284,71 @@ size_t tq_decode_workspace_bytes(const tq_ctx* c, int batch, int hq, int hkv, in
   return tq::plan_decode(c, batch, hq, hkv, max_len).total_bytes;
 }
 
+namespace {
+// Shared by tq_decode_attention (contiguous cache) and tq_decode_attention_paged.
+tq_status decode_impl(const char* name, const tq_ctx* c, const void* q, tq_dtype q_dtype, int batch, int hq,
+                      int hkv, const int32_t* seq_lens, int64_t max_len, const tq::Paging& pg,
+                      const uint8_t* k_codes, const uint8_t* k_signs, const uint16_t* k_norms,
+                      const uint8_t* v_codes, const uint16_t* v_params, float softmax_scale, float* scores,
+                      float* out, void* workspace, size_t workspace_bytes, void* stream) {
+  const std::string nm(name);
+  if (!c) return fail(TQ_EINVAL, nm + ": NULL context");
+  if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return fail(TQ_EINVAL, nm + ": bad dtype");
+  if (batch < 0 || hq <= 0 || hkv <= 0 || hq % hkv || max_len < 0)
+    return fail(TQ_EINVAL, nm + ": bad batch/head/length arguments");
+  if (hq / hkv > 64 || (c->shape.d == 256 && hq / hkv > 32))
+    return fail(TQ_EUNSUPPORTED, nm + ": too many query heads per KV head (max 64; 32 at d=256)");
+  if (!std::isfinite(softmax_scale) || softmax_scale < 0.f)
+    return fail(TQ_EINVAL, nm + ": softmax_scale must be finite and >= 0");
+  if (batch == 0) return TQ_OK;
+  if (!q || !out) return fail(TQ_EINVAL, nm + ": NULL q or out");
+  if (max_len > 0 && (!k_codes || !k_signs || !k_norms || !v_codes || !v_params))
+    return fail(TQ_EINVAL, nm + ": NULL packed cache");
+  const void* ptrs[] = {q, out, k_codes, k_signs, k_norms, v_codes, v_params, workspace, scores, seq_lens};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return fail(TQ_EINVAL, nm + ": pointers must be 16-byte aligned");
+  if (max_len > (int64_t(1) << 31)) return fail(TQ_EINVAL, nm + ": max_len too large");
+  tq::DecodePlan plan = tq::plan_decode(c, batch, hq, hkv, max_len);
+  if (!workspace || workspace_bytes < plan.total_bytes)
+    return fail(TQ_EINVAL, nm + ": workspace missing or too small");
+  float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)c->shape.d);
+  cudaError_t e = tq::launch_decode(c, plan, q, (int)q_dtype, batch, hq, hkv, seq_lens, max_len, pg, k_codes,
+                                    k_signs, k_norms, v_codes, v_params, scale, scores, out, workspace,
+                                    static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e, name);
+  return TQ_OK;
+}
+}  // namespace
+
 tq_status tq_decode_attention(const tq_ctx* c, const void* q, tq_dtype q_dtype, int batch, int hq,
                               int hkv, const int32_t* seq_lens, int64_t max_len,
                               const uint8_t* k_codes, const uint8_t* k_signs,
                               const uint16_t* k_norms, const uint8_t* v_codes,
                               const uint16_t* v_params, float softmax_scale, float* scores,
                               float* out, void* workspace, size_t workspace_bytes, void* stream) {
-  if (!c) return fail(TQ_EINVAL, "tq_decode_attention: NULL context");
-  if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return fail(TQ_EINVAL, "tq_decode_attention: bad dtype");
-  if (batch < 0 || hq <= 0 || hkv <= 0 || hq % hkv || max_len < 0)
-    return fail(TQ_EINVAL, "tq_decode_attention: bad batch/head/length arguments");
-  if (hq / hkv > 64 || (c->shape.d == 256 && hq / hkv > 32))
-    return fail(TQ_EUNSUPPORTED, "tq_decode_attention: too many query heads per KV head (max 64; 32 at d=256)");
-  if (!std::isfinite(softmax_scale) || softmax_scale < 0.f)
-    return fail(TQ_EINVAL, "tq_decode_attention: softmax_scale must be finite and >= 0");
-  if (batch == 0) return TQ_OK;
-  if (!q || !out) return fail(TQ_EINVAL, "tq_decode_attention: NULL q or out");
-  if (max_len > 0 && (!k_codes || !k_signs || !k_norms || !v_codes || !v_params))
-    return fail(TQ_EINVAL, "tq_decode_attention: NULL packed cache");
-  const void* ptrs[] = {q, out, k_codes, k_signs, k_norms, v_codes, v_params, workspace, scores, seq_lens};
-  for (const void* ptr : ptrs)
-    if (ptr && !aligned16(ptr)) return fail(TQ_EINVAL, "tq_decode_attention: pointers must be 16-byte aligned");
-  if (max_len > (int64_t(1) << 31)) return fail(TQ_EINVAL, "tq_decode_attention: max_len too large");
-  tq::DecodePlan plan = tq::plan_decode(c, batch, hq, hkv, max_len);
-  if (!workspace || workspace_bytes < plan.total_bytes)
-    return fail(TQ_EINVAL, "tq_decode_attention: workspace missing or too small");
-  float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)c->shape.d);
-  cudaError_t e = tq::launch_decode(c, plan, q, (int)q_dtype, batch, hq, hkv, seq_lens, max_len, k_codes,
-                                    k_signs, k_norms, v_codes, v_params, scale, scores, out, workspace,
-                                    static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return fail_cuda(e, "tq_decode_attention");
-  return TQ_OK;
+  const tq::Paging contiguous{nullptr, 0, 0, 0};
+  return decode_impl("tq_decode_attention", c, q, q_dtype, batch, hq, hkv, seq_lens, max_len, contiguous,
+                     k_codes, k_signs, k_norms, v_codes, v_params, softmax_scale, scores, out, workspace,
+                     workspace_bytes, stream);
+}
+
+tq_status tq_decode_attention_paged(const tq_ctx* c, const void* q, tq_dtype q_dtype, int batch, int hq,
+                                    int hkv, const int32_t* seq_lens, int64_t max_len,
+                                    const int32_t* block_table, int64_t page_size, int64_t max_pages,
+                                    int64_t n_pages, const uint8_t* k_codes, const uint8_t* k_signs,
+                                    const uint16_t* k_norms, const uint8_t* v_codes, const uint16_t* v_params,
+                                    float softmax_scale, float* scores, float* out, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  if (!block_table || !aligned16(block_table))
+    return fail(TQ_EINVAL, "tq_decode_attention_paged: block_table NULL or not 16-byte aligned");
+  if (page_size <= 0 || page_size % 512)
+    return fail(TQ_EINVAL, "tq_decode_attention_paged: page_size must be a positive multiple of 512");
+  if (max_len < 0 || max_pages < (max_len + page_size - 1) / page_size || n_pages <= 0)
+    return fail(TQ_EINVAL, "tq_decode_attention_paged: max_pages below ceil(max_len / page_size), or no pages");
+  const tq::Paging paged{block_table, page_size, max_pages, n_pages};
+  return decode_impl("tq_decode_attention_paged", c, q, q_dtype, batch, hq, hkv, seq_lens, max_len, paged, k_codes,
+                     k_signs, k_norms, v_codes, v_params, softmax_scale, scores, out, workspace, workspace_bytes,
+                     stream);
 }
 
 tq_status tq_decompress(const tq_ctx* c, const uint8_t* k_codes, const uint8_t* k_signs,

@@ -15,6 +15,20 @@ constexpr unsigned kFull = 0xffffffffu;
 // is an unbiased estimate of <x, r>.
 constexpr float kQjl = 1.2533141373155003f;
 
+// Record row of token t of unit u under the cache addressing p (t the first token of a
+// tile, which never crosses a page). A page index outside [0, n_pages) sets bit 2 of
+// *err and reads page 0 instead.
+__device__ __forceinline__ int64_t record_row(const Paging& p, int64_t max_len, int64_t u, int64_t t,
+                                              unsigned int* err) {
+  if (!p.block_table) return u * max_len + t;
+  int64_t pg = __ldg(p.block_table + u * p.max_pages + t / p.page_size);
+  if (pg < 0 || pg >= p.n_pages) {
+    atomicOr(err, 4u);
+    pg = 0;
+  }
+  return pg * p.page_size + t % p.page_size;
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);

@@ -31,6 +31,15 @@ struct Shape {
   int rot;  // tq_rot
 };
 
+// Cache addressing of the decode kernels. Contiguous (block_table null): token t of unit
+// u = (sequence, KV head) is record row u * max_len + t. Paged: it is row
+// block_table[u * max_pages + t / page_size] * page_size + t % page_size, page_size a
+// multiple of every kernel's tile so that a tile never crosses a page.
+struct Paging {
+  const int32_t* block_table;
+  int64_t page_size, max_pages, n_pages;
+};
+
 }  // namespace tq
 
 struct tq_ctx {
@@ -44,7 +53,8 @@ struct tq_ctx {
   float* PiT;      // device [d][d] fp32 transpose (Haar only)
   cudaEvent_t prof_start;  // optional events around the main kernel of each call
   cudaEvent_t prof_stop;
-  unsigned int* d_err;     // device error word: bit 0 = a bounded wait in a kernel timed out
+  unsigned int* d_err;     // device error word: bit 0 = a bounded wait in a kernel timed out,
+                           // bit 2 = a slot or page index outside the caller's arrays
   uint16_t* S_sw128;       // tensor-core compression: S as an f16 operand tile (d = m = 128, S exact in f16)
   uint16_t* H_sw128;       // tensor-core compression: H diag(sigma) as a bf16 operand tile (d = 128, Hadamard)
   uint16_t* Pi_sw128;      // tensor-core compression: Haar Pi as three bf16 operand tiles (d = 128)
@@ -53,9 +63,11 @@ struct tq_ctx {
 namespace tq {
 
 // Launchers (defined in the .cu files). Return cudaSuccess or the launch error.
+// slot: null (vector i -> row i) or the output row of each vector, checked against n_rows.
 cudaError_t launch_compress(const tq_ctx* ctx, const void* k, const void* v, int dtype,
-                            int64_t n_vec, uint8_t* k_codes, uint8_t* k_signs, uint16_t* k_norms,
-                            uint8_t* v_codes, uint16_t* v_params, cudaStream_t stream);
+                            int64_t n_vec, const int64_t* slot, int64_t n_rows, uint8_t* k_codes,
+                            uint8_t* k_signs, uint16_t* k_norms, uint8_t* v_codes, uint16_t* v_params,
+                            cudaStream_t stream);
 
 struct DecodePlan {
   bool mma;          // tensor-core kernels (decode_mma.cu) instead of the generic ones
@@ -75,9 +87,9 @@ DecodePlan plan_decode(const tq_ctx* ctx, int batch, int hq, int hkv, int64_t ma
 
 cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const void* q, int q_dtype,
                           int batch, int hq, int hkv, const int32_t* seq_lens, int64_t max_len,
-                          const uint8_t* k_codes, const uint8_t* k_signs, const uint16_t* k_norms,
-                          const uint8_t* v_codes, const uint16_t* v_params, float scale,
-                          float* scores, float* out, void* workspace, cudaStream_t stream);
+                          const Paging& pg, const uint8_t* k_codes, const uint8_t* k_signs,
+                          const uint16_t* k_norms, const uint8_t* v_codes, const uint16_t* v_params,
+                          float scale, float* scores, float* out, void* workspace, cudaStream_t stream);
 
 bool mma_decode_supported(const tq_ctx* ctx, int G);
 
@@ -89,7 +101,8 @@ void pack_hadamard_operand(const uint32_t* sign_bits, uint16_t* out);  // d = 12
 void pack_haar_operand(const double* pi, uint16_t* out);                // d = 128, 3 tiles
 
 cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const void* q, int q_dtype, int batch,
-                              int hq, int hkv, const int32_t* seq_lens, int64_t max_len, const uint8_t* k_codes,
+                              int hq, int hkv, const int32_t* seq_lens, int64_t max_len, const Paging& pg,
+                              const uint8_t* k_codes,
                               const uint8_t* k_signs, const uint16_t* k_norms, const uint8_t* v_codes,
                               const uint16_t* v_params, float scale, float* scores, float* out, void* workspace,
                               cudaStream_t stream);
