@@ -245,6 +245,7 @@ tq_status compress_impl(const char* name, const tq_ctx* c, const void* k, const 
   const std::string nm(name);
   if (!c) return fail(TQ_EINVAL, nm + ": NULL context");
   if (n_vec < 0) return fail(TQ_EINVAL, nm + ": negative n_vec");
+  if (n_vec == 0) return TQ_OK;
   if (dtype != TQ_F32 && dtype != TQ_BF16) return fail(TQ_EINVAL, nm + ": bad dtype");
   if (!k && !v) return fail(TQ_EINVAL, nm + ": both k and v are NULL");
   if (k && (!k_codes || !k_signs || !k_norms)) return fail(TQ_EINVAL, nm + ": NULL key output");
@@ -255,7 +256,6 @@ tq_status compress_impl(const char* name, const tq_ctx* c, const void* k, const 
     return fail(TQ_EINVAL, nm + ": value pointers must be 16-byte aligned");
   if (slot && ((reinterpret_cast<uintptr_t>(slot) & 7u) || n_rows <= 0))
     return fail(TQ_EINVAL, nm + ": the slot map must be 8-byte aligned and n_rows positive");
-  if (n_vec == 0) return TQ_OK;
   if (n_vec > (int64_t(1) << 40)) return fail(TQ_EINVAL, nm + ": n_vec too large");
   cudaError_t e = tq::launch_compress(c, k, v, (int)dtype, n_vec, slot, n_rows, k_codes, k_signs, k_norms,
                                       v_codes, v_params, static_cast<cudaStream_t>(stream));
