@@ -73,7 +73,10 @@ typedef enum {
  *   d              head dimension: 64, 128 or 256
  *   k_lm_bits      Lloyd-Max bits per key coordinate: 1, 2 or 3 (a key then costs
  *                  k_lm_bits + 1 bits per coordinate with its QJL sign)
- *   qjl_m          rows of the QJL matrix S: a multiple of 32, at most 256
+ *   qjl_m          rows of the QJL matrix S: a multiple of 32, at most 256; or 0 for
+ *                  keys without the QJL stage (Lloyd-Max codes only, the MSE-optimal
+ *                  first stage): no sign bytes (k_signs may be NULL), gamma is still
+ *                  stored, and scores and decompressed keys use the codes alone
  *   v_bits         value bits: 2 or 4
  *   v_group        value group size: 32
  *   rot            rotation kind
@@ -82,7 +85,7 @@ typedef enum {
  *                  gets code #{k : y >= boundaries[k]}
  *   hadamard_signs d entries, each +1 or -1 (TQ_ROT_HADAMARD; ignored otherwise)
  *   haar           d*d row-major orthogonal matrix Pi in fp64, y = Pi u (TQ_ROT_HAAR)
- *   qjl_S          m*d row-major fp32 matrix S (i.i.d. N(0,1) draws)            */
+ *   qjl_S          m*d row-major fp32 matrix S (i.i.d. N(0,1) draws); NULL if m = 0 */
 typedef struct {
   int d;
   int k_lm_bits;

@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
 #pragma unroll
   for (int q = 0; q < kMaxQ; ++q) acc[q] = 0.f;
 
-  const float qjl = kQjl / (float)M;
+  const float qjl = M > 0 ? kQjl / (float)M : 0.f;  // M = 0: no QJL stage
   for (int64_t tt = t0; tt < t1; tt += kTile) {
     const int nt = (int)min((int64_t)kTile, t1 - tt);
     const int64_t row0 = record_row(a.pg, a.max_len, unit, tt, a.err);  // the tile's first record

@@ -54,7 +54,7 @@ __device__ void decompress_key(const DecompressArgs& a, int64_t i, int lane, flo
         acc += ((bits >> bb) & 1u) ? s : -s;
       }
     }
-    y[e] = cv + (kQjl / (float)a.m) * gamma * acc;
+    y[e] = a.m > 0 ? cv + (kQjl / (float)a.m) * gamma * acc : cv;  // m = 0: no QJL stage
   }
   float x[E];
   if (a.rot == TQ_ROT_HADAMARD) {

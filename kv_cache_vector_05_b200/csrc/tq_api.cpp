@@ -90,15 +90,15 @@ tq_status tq_codebook_load(const tq_params* p, void* stream, tq_ctx** out) {
     return fail(TQ_EUNSUPPORTED, "tq_codebook_load: d must be 64, 128 or 256");
   if (b < 1 || b > tq::kMaxLmBits)
     return fail(TQ_EUNSUPPORTED, "tq_codebook_load: k_lm_bits must be 1, 2 or 3");
-  if (m < 32 || m > tq::kMaxM || m % 32)
-    return fail(TQ_EUNSUPPORTED, "tq_codebook_load: qjl_m must be a multiple of 32 up to 256");
+  if (m < 0 || m > tq::kMaxM || m % 32)
+    return fail(TQ_EUNSUPPORTED, "tq_codebook_load: qjl_m must be 0 (no QJL stage) or a multiple of 32 up to 256");
   if (!(p->v_bits == 2 || p->v_bits == 4))
     return fail(TQ_EUNSUPPORTED, "tq_codebook_load: v_bits must be 2 or 4");
   if (p->v_group != tq::kVGroup)
     return fail(TQ_EUNSUPPORTED, "tq_codebook_load: v_group must be 32");
   if (p->rot != TQ_ROT_HADAMARD && p->rot != TQ_ROT_HAAR)
     return fail(TQ_EINVAL, "tq_codebook_load: unknown rotation");
-  if (!p->centroids || !p->boundaries || !p->qjl_S)
+  if (!p->centroids || !p->boundaries || (m > 0 && !p->qjl_S))
     return fail(TQ_EINVAL, "tq_codebook_load: NULL codebook or QJL matrix");
   if (p->rot == TQ_ROT_HADAMARD && !p->hadamard_signs)
     return fail(TQ_EINVAL, "tq_codebook_load: NULL Hadamard signs");
@@ -153,8 +153,8 @@ tq_status tq_codebook_load(const tq_params* p, void* stream, tq_ctx** out) {
       }
   }
   auto alloc = [&](float** dst, size_t n) -> cudaError_t { return cudaMalloc((void**)dst, n * sizeof(float)); };
-  e = alloc(&c->S, S.size());
-  if (e == cudaSuccess) e = alloc(&c->St, St.size());
+  if (m > 0) e = alloc(&c->S, S.size());  // m = 0: no QJL stage, no S
+  if (e == cudaSuccess && m > 0) e = alloc(&c->St, St.size());
   if (e == cudaSuccess && !Pi.empty()) e = alloc(&c->Pi, Pi.size());
   if (e == cudaSuccess && !Pi.empty()) e = alloc(&c->PiT, PiT.size());
   if (e == cudaSuccess) e = cudaMalloc((void**)&c->d_err, sizeof(unsigned int));
@@ -183,8 +183,8 @@ tq_status tq_codebook_load(const tq_params* p, void* stream, tq_ctx** out) {
     return e == cudaErrorMemoryAllocation ? fail(TQ_ENOMEM, "tq_codebook_load: cudaMalloc failed")
                                           : fail_cuda(e, "tq_codebook_load: cudaMalloc");
   }
-  e = cudaMemcpyAsync(c->S, S.data(), S.size() * sizeof(float), cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess)
+  if (m > 0) e = cudaMemcpyAsync(c->S, S.data(), S.size() * sizeof(float), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && m > 0)
     e = cudaMemcpyAsync(c->St, St.data(), St.size() * sizeof(float), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess && !Pi.empty())
     e = cudaMemcpyAsync(c->Pi, Pi.data(), Pi.size() * sizeof(float), cudaMemcpyHostToDevice, s);
@@ -248,7 +248,7 @@ tq_status compress_impl(const char* name, const tq_ctx* c, const void* k, const 
   if (n_vec == 0) return TQ_OK;
   if (dtype != TQ_F32 && dtype != TQ_BF16) return fail(TQ_EINVAL, nm + ": bad dtype");
   if (!k && !v) return fail(TQ_EINVAL, nm + ": both k and v are NULL");
-  if (k && (!k_codes || !k_signs || !k_norms)) return fail(TQ_EINVAL, nm + ": NULL key output");
+  if (k && (!k_codes || (c->shape.m > 0 && !k_signs) || !k_norms)) return fail(TQ_EINVAL, nm + ": NULL key output");
   if (v && (!v_codes || !v_params)) return fail(TQ_EINVAL, nm + ": NULL value output");
   if (k && !(aligned16(k) && aligned16(k_codes) && aligned16(k_signs) && aligned16(k_norms)))
     return fail(TQ_EINVAL, nm + ": key pointers must be 16-byte aligned");
@@ -302,7 +302,7 @@ tq_status decode_impl(const char* name, const tq_ctx* c, const void* q, tq_dtype
     return fail(TQ_EINVAL, nm + ": softmax_scale must be finite and >= 0");
   if (batch == 0) return TQ_OK;
   if (!q || !out) return fail(TQ_EINVAL, nm + ": NULL q or out");
-  if (max_len > 0 && (!k_codes || !k_signs || !k_norms || !v_codes || !v_params))
+  if (max_len > 0 && (!k_codes || (c->shape.m > 0 && !k_signs) || !k_norms || !v_codes || !v_params))
     return fail(TQ_EINVAL, nm + ": NULL packed cache");
   const void* ptrs[] = {q, out, k_codes, k_signs, k_norms, v_codes, v_params, workspace, scores, seq_lens};
   for (const void* ptr : ptrs)
@@ -358,7 +358,8 @@ tq_status tq_decompress(const tq_ctx* c, const uint8_t* k_codes, const uint8_t* 
   if (n_vec < 0) return fail(TQ_EINVAL, "tq_decompress: negative n_vec");
   if (n_vec == 0) return TQ_OK;
   if (!k_out && !v_out) return fail(TQ_EINVAL, "tq_decompress: both outputs NULL");
-  if (k_out && (!k_codes || !k_signs || !k_norms)) return fail(TQ_EINVAL, "tq_decompress: NULL key input");
+  if (k_out && (!k_codes || (c->shape.m > 0 && !k_signs) || !k_norms))
+    return fail(TQ_EINVAL, "tq_decompress: NULL key input");
   if (v_out && (!v_codes || !v_params)) return fail(TQ_EINVAL, "tq_decompress: NULL value input");
   const void* ptrs[] = {k_codes, k_signs, k_norms, v_codes, v_params, k_out, v_out};
   for (const void* ptr : ptrs)

@@ -324,7 +324,7 @@ def decompress_keys(packed: dict, Pi, centroids, S, d: int):
     s = 2.0 * unpack_signs(packed["signs"], m).astype(np.float64) - 1.0
     norms = np.asarray(packed["norms"], dtype=np.uint16).view(np.float16).astype(np.float64)
     n, gamma = norms[:, 0], norms[:, 1]
-    y_hat = c[idx] + (QJL_CONST / m) * gamma[:, None] * (s @ S)
+    y_hat = c[idx] + (QJL_CONST / m) * gamma[:, None] * (s @ S) if m else c[idx]  # m = 0: codes alone
     return n[:, None] * (y_hat @ np.asarray(Pi, dtype=np.float64))
 
 
@@ -397,7 +397,7 @@ def key_scores(q, packed_k: dict, Pi, centroids, S, d: int, scale: float | None 
     norms = np.asarray(packed_k["norms"], dtype=np.uint16).view(np.float16).astype(np.float64)
     n, gamma = norms[:, 0], norms[:, 1]
     lut = c[idx] @ qr.T                       # [N, G]
-    qjl = (QJL_CONST / m) * gamma[:, None] * (s @ sq.T)
+    qjl = (QJL_CONST / m) * gamma[:, None] * (s @ sq.T) if m else 0.0  # m = 0: no QJL stage
     return (scale * n[:, None] * (lut + qjl)).T
 
 

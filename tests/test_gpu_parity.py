@@ -343,3 +343,50 @@ def test_sweep_mse_and_inner_product_distortion_vs_oracle(d, b, rotation):
     assert ip_g == pytest.approx(ip_o, rel=1e-3)
     # and the reconstruction is informative: well below the MSE of reconstructing zero (1)
     assert mse_g < 0.75
+
+
+# ------------------------------------------------------------------ keys without the QJL stage
+
+@pytest.mark.parametrize("d,lm_bits,v_bits,rotation,dtype", [
+    (128, 2, 2, "hadamard", "bf16"), (128, 1, 4, "haar", "f32"), (64, 3, 4, "hadamard", "bf16")])
+def test_keys_without_qjl_stage(d, lm_bits, v_bits, rotation, dtype):
+    """qjl_m = 0 (Lloyd-Max codes only; no sign bytes): compression, decode attention and
+    decompression through the C ABI against the oracle given an empty S."""
+    dr = W.method_draws(d, d, 1234)
+    c32, t32 = T.tq_lloyd_max_codebook(d, lm_bits)
+    haar = T.tq_haar_from_gaussian(dr["haar_gaussian"]) if rotation == "haar" else None
+    S0 = np.zeros((0, d))
+    ctx = T.tq_codebook_load(d, lm_bits, v_bits, c32, t32, S0, rotation=rotation,
+                             hadamard_signs=dr["hadamard_signs"], haar=haar)
+    assert ctx.m == 0
+    n, G = 3000, 4
+    rng = np.random.default_rng([d, lm_bits])
+    K = rng.standard_normal((n, d)) * rng.lognormal(0, 1, d)
+    V = rng.standard_normal((n, d))
+    K[[0, n - 1]] = 0.0
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    kt = torch.from_numpy(K.astype(np.float32)).to(DEV).to(tdt)
+    vt = torch.from_numpy(V.astype(np.float32)).to(DEV).to(tdt)
+    gp = T.tq_compress_kv(ctx, kt, vt)
+    T.tq_check_device(ctx)
+    g = to_np(gp)
+    assert g["k_signs"].shape == (n, 0)
+    Pi, c, t, _ = oracle_setup(d, lm_bits, d, rotation)
+    ok = O.compress_keys(kt.float().cpu().numpy().astype(np.float64), Pi, c, t, S0, with_diagnostics=True)
+    ov = O.quantize_values(vt.float().cpu().numpy().astype(np.float64), v_bits, with_diagnostics=True)
+    assert_key_parity(compare_keys(g, ok, d, lm_bits, 0))
+    assert_value_parity(compare_values(g, ov, d, v_bits))
+    # decode attention over the compressed cache (one sequence, one KV head)
+    q = W.queries((1, G, d), dtype="f32")
+    scores = torch.full((1, G, n), float("nan"), device=DEV)
+    out, _ = T.tq_decode_attention(ctx, torch.from_numpy(q).to(DEV), gp, 1, G, 1, n, scores=scores)
+    T.tq_check_device(ctx)
+    pk = {"codes": g["k_codes"], "signs": g["k_signs"], "norms": g["k_norms"]}
+    pv = {"codes": g["v_codes"], "params": g["v_params"]}
+    os_, oo = O.decode_attention(q[0].astype(np.float64), pk, pv, Pi, c, S0, d, v_bits)
+    assert_close(scores[0].cpu().numpy(), os_, what="scores")
+    assert_close(out[0].cpu().numpy(), oo, what="out")
+    # decompression
+    kx, _ = T.tq_decompress(ctx, gp, n)
+    torch.cuda.synchronize()
+    assert_close(kx.cpu().numpy(), O.decompress_keys(pk, Pi, c, S0, d), rtol=1e-4, atol=1e-5, what="keys")

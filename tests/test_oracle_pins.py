@@ -427,3 +427,28 @@ def test_compression_distortion_is_near_lloyd_max():
     cl, tl = O.lloyd_max_sphere(d, 2)
     want = d * O.quantizer_mse(lambda x: O.sphere_coordinate_pdf(x, d), -1, 1, cl, tl)
     assert abs(rel - want) / want < 0.02
+
+
+def test_keys_without_qjl_stage():
+    """m = 0 (Lloyd-Max codes only, no QJL signs): the score from the codes equals the score
+    against the reconstruction n Pi^T c[idx], and the reconstruction's relative squared error
+    averages d times the per-coordinate MSE the sphere codebook was solved for (quadrature),
+    d = 64, 2-bit codes, 20000 uniformly random unit directions (well within 4 sigma)."""
+    d, bits, n = 64, 2, 20000
+    rng = np.random.default_rng(42)
+    Pi = O.haar_rotation(rng.standard_normal((d, d)))
+    c, t = O.lloyd_max_sphere(d, bits)
+    S = np.zeros((0, d))
+    K = rng.standard_normal((n, d)) * rng.uniform(0.5, 3.0, size=(n, 1))
+    pk = O.compress_keys(K, Pi, c, t, S)
+    assert pk["signs"].shape == (n, 0)
+    packed = {"codes": pk["codes"], "signs": pk["signs"], "norms": pk["norms"]}
+    q = rng.standard_normal((3, d))
+    xh = O.decompress_keys(packed, Pi, c, S, d)
+    np.testing.assert_allclose(O.key_scores(q, packed, Pi, c, S, d), q @ xh.T / np.sqrt(d), rtol=1e-12, atol=1e-12)
+    # with the exact norm (the stored one is fp16) the error is that of the unit direction
+    nrm = np.linalg.norm(K, axis=1)
+    n16 = pk["norms"][:, 0].view(np.float16).astype(np.float64)
+    err = np.sum((K / nrm[:, None] - xh / n16[:, None]) ** 2, axis=1)
+    want = d * O.quantizer_mse(lambda x: O.sphere_coordinate_pdf(x, d), -1, 1, c, t)
+    assert abs(err.mean() - want) < 4 * err.std() / np.sqrt(n)
