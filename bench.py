@@ -88,9 +88,9 @@ DECODE_SOURCES = ("decode_mma.cu", "decode.cu", "tq_device.cuh", "tq_sm100.cuh",
 COMPRESS_SOURCES = ("compress.cu", "tq_device.cuh", "tq_sm100.cuh", "tq_internal.h")
 
 
-def recorded_traffic(kernel_file: str, sha: str, units: int):
+def recorded_traffic(kernel_file: str, sha: str, units: int, kernel: str):
     """DRAM bytes of one launch over `units` units, from a committed ncu summary that
-    gives DRAM bytes per unit for the same source (None if absent or stale)."""
+    gives DRAM bytes per unit for the same kernel and source (None if absent or stale)."""
     p = os.path.join(ROOT, "profiles", kernel_file)
     if not os.path.exists(p):
         return None
@@ -100,7 +100,7 @@ def recorded_traffic(kernel_file: str, sha: str, units: int):
             if ":" in line:
                 k, v = line.split(":", 1)
                 kv[k.strip()] = v.strip()
-    if kv.get("source_sha256_16") != sha:
+    if kv.get("source_sha256_16") != sha or kv.get("kernel") != kernel:
         return None
     try:
         return float(kv["dram_bytes_per_unit"]) * units
@@ -503,11 +503,14 @@ def run_ours(args, w: W.Workload):
         peak, peak_kind = measured_peaks()
         dsha = source_sha(DECODE_SOURCES)
         units_dec = w.units * w.tokens  # (token, KV head) pairs
-        roof_dec = {"kernel": "decode_mma_kernel", "bound": "hbm", "achieved": packed_bytes / dec_k_mean / 1e9,
+        # the tensor-core decode serves d = m = 128, 1- or 2-bit Lloyd-Max codes, G <= 8
+        dkern = "decode_mma_kernel" if (w.d == 128 and w.m == 128 and w.lm_bits <= 2 and w.group <= 8) \
+            else "decode_kernel"
+        roof_dec = {"kernel": dkern, "bound": "hbm", "achieved": packed_bytes / dec_k_mean / 1e9,
                     "peak": peak, "unit": "GB/s", "frac": packed_bytes / dec_k_mean / 1e9 / peak,
                     "peak_kind": peak_kind, "alg_bytes_per_launch": packed_bytes,
                     "alg_bytes_per_unit": w.k_record_bytes() + w.v_record_bytes(), "unit_of_work": "token x KV head",
-                    "traffic": recorded_traffic("decode_kernel_traffic.txt", dsha, units_dec),
+                    "traffic": recorded_traffic("decode_kernel_traffic.txt", dsha, units_dec, dkern),
                     "source_sha256_16": dsha}
         roof = roof_dec
         if not args.decode_only:
@@ -515,14 +518,16 @@ def run_ours(args, w: W.Workload):
             csha = source_sha(COMPRESS_SOURCES)
             comp_bytes = in_bytes + packed_bytes
             comp_k_mean = statistics.fmean(comp_k) / 1e3
-            # bf16 keys, Hadamard rotation, d = 128 and the (symmetric) Lloyd-Max codebook
-            ckern = "compress_pipe_kernel" if (w.dtype == "bf16" and w.d == 128 and w.rotation == "hadamard") \
-                else "compress_q4_kernel"
+            # d = m = 128 with the Hadamard rotation: bf16 keys (symmetric Lloyd-Max codebook) take
+            # the pipelined tensor-core kernel, fp32 keys the four-lanes-per-vector one
+            tc = w.d == 128 and w.m == 128 and w.rotation == "hadamard"
+            ckern = ("compress_pipe_kernel" if w.dtype == "bf16" else "compress_q4_kernel") if tc \
+                else "compress_kernel"
             roof = {"kernel": ckern, "bound": "hbm", "achieved": comp_bytes / comp_k_mean / 1e9, "peak": peak,
                     "unit": "GB/s", "frac": comp_bytes / comp_k_mean / 1e9 / peak, "peak_kind": peak_kind,
                     "alg_bytes_per_launch": comp_bytes, "alg_bytes_per_unit": comp_bytes // n_vec,
                     "unit_of_work": "key + value vector pair",
-                    "traffic": recorded_traffic("compress_kernel_traffic.txt", csha, n_vec),
+                    "traffic": recorded_traffic("compress_kernel_traffic.txt", csha, n_vec, ckern),
                     "source_sha256_16": csha}
         line = {
             "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,

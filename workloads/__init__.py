@@ -48,20 +48,21 @@ class Workload:
     hkv: int            # KV heads per sequence
     hq: int             # query heads per sequence
     tokens: int         # cached tokens per (sequence, KV head)
-    k_bits: int         # total key bits = Lloyd-Max bits + 1 QJL bit
+    k_bits: int         # total key bits = Lloyd-Max bits + 1 QJL bit (Lloyd-Max bits alone if not qjl)
     v_bits: int
     dtype: str          # "f32" or "bf16"
     qjl_m: int = 0      # 0 => m = d
     v_group: int = 32
     rotation: str = "hadamard"
+    qjl: bool = True    # False: keys without the QJL stage (m = 0)
 
     @property
     def m(self) -> int:
-        return self.qjl_m or self.d
+        return (self.qjl_m or self.d) if self.qjl else 0
 
     @property
     def lm_bits(self) -> int:
-        return self.k_bits - 1
+        return self.k_bits - 1 if self.qjl else self.k_bits
 
     @property
     def units(self) -> int:
@@ -90,6 +91,8 @@ WORKLOADS = {
     "llama8b_b32_32k_k3v2": Workload("llama8b_b32_32k_k3v2", 128, 32, 8, 32, 32768, 3, 2, "bf16"),
     # long context: one sequence of 1,048,576 tokens, 4 KV heads, 24 query heads
     "long_1m_k4v4": Workload("long_1m_k4v4", 128, 1, 4, 24, 1 << 20, 4, 4, "bf16"),
+    # the Llama-shaped batch with 3-bit Lloyd-Max keys and no QJL stage (same 100 B record)
+    "llama8b_b32_32k_mse3v2": Workload("llama8b_b32_32k_mse3v2", 128, 32, 8, 32, 32768, 3, 2, "bf16", qjl=False),
 }
 
 # compression sweep: 16384 tokens x 64 heads of bf16 N(0,1) vectors
