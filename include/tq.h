@@ -77,7 +77,8 @@ typedef enum {
  *                  keys without the QJL stage (Lloyd-Max codes only, the MSE-optimal
  *                  first stage): no sign bytes (k_signs may be NULL), gamma is still
  *                  stored, and scores and decompressed keys use the codes alone
- *   v_bits         value bits: 2 or 4
+ *   v_bits         value bits: 2, 3 or 4 (3-bit codes straddle 32-bit words and run on
+ *                  the CUDA-core value kernels; keys still take the tensor-core ones)
  *   v_group        value group size: 32
  *   rot            rotation kind
  *   centroids      2^k_lm_bits ascending fp32 centroids of the Lloyd-Max codebook

@@ -1840,7 +1840,24 @@ cudaError_t launch_compress(const tq_ctx* ctx, const void* k, const void* v, int
   a.S_sw128 = ctx->S_sw128;
   a.H_sw128 = ctx->H_sw128;
   a.err = ctx->d_err;
-  if (ctx->S_sw128 && ctx->shape.d == 128 && ctx->shape.m == 128) {
+  auto generic = [&](const CompressArgs& g) -> cudaError_t {
+    switch (ctx->shape.d) {
+      case 64: return launch_d<64>(ctx, g, dtype, stream);
+      case 128: return launch_d<128>(ctx, g, dtype, stream);
+      case 256: return launch_d<256>(ctx, g, dtype, stream);
+    }
+    return cudaErrorInvalidValue;
+  };
+  if (ctx->shape.v_bits == 3 && k && v && ctx->S_sw128) {
+    // 3-bit value codes straddle words: the tensor-core kernels take the keys alone and
+    // the warp-per-vector kernel the values
+    CompressArgs vv = a;
+    vv.k = nullptr;
+    const cudaError_t e = launch_compress(ctx, k, nullptr, dtype, n_vec, slot, n_rows, k_codes, k_signs, k_norms,
+                                          nullptr, nullptr, stream);
+    return e != cudaSuccess ? e : generic(vv);
+  }
+  if (ctx->S_sw128 && ctx->shape.d == 128 && ctx->shape.m == 128 && !(ctx->shape.v_bits == 3 && v)) {
     if (ctx->shape.rot == TQ_ROT_HADAMARD && dtype == TQ_BF16 && ctx->H_sw128) {
       if (codebook_symmetric(ctx->cb, ctx->shape.lm_bits) && (!k || encode_rows_map(&a.kmap, k, n_vec, 128)) &&
           (!v || encode_rows_map(&a.vmap, v, n_vec, 64)))
@@ -1855,12 +1872,7 @@ cudaError_t launch_compress(const tq_ctx* ctx, const void* k, const void* v, int
       return dtype == TQ_F32 ? launch_q4<float>(ctx, a, stream) : launch_q4<__nv_bfloat16>(ctx, a, stream);
     return dtype == TQ_F32 ? launch_tc<float>(ctx, a, stream) : launch_tc<__nv_bfloat16>(ctx, a, stream);
   }
-  switch (ctx->shape.d) {
-    case 64: return launch_d<64>(ctx, a, dtype, stream);
-    case 128: return launch_d<128>(ctx, a, dtype, stream);
-    case 256: return launch_d<256>(ctx, a, dtype, stream);
-  }
-  return cudaErrorInvalidValue;
+  return generic(a);
 }
 
 }  // namespace tq

@@ -256,7 +256,9 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
     const int g = vj / kVGroup;
     const int wsel = (vj * VB) >> 5, shift = (vj * VB) & 31;
     for (int t = 0; t < nt; ++t) {
-      const uint32_t code = (vcode_s[t * VW + wsel] >> shift) & ((1u << VB) - 1u);
+      uint32_t code = vcode_s[t * VW + wsel] >> shift;
+      if (VB == 3 && shift > 29) code |= vcode_s[t * VW + wsel + 1] << (32 - shift);  // straddles two words
+      code &= (1u << VB) - 1u;
       const uint32_t par = vpar_s[t * NG + g];
       const float sc = __half2float(__ushort_as_half((unsigned short)(par & 0xffffu)));
       const float lo = __half2float(__ushort_as_half((unsigned short)(par >> 16)));
@@ -334,6 +336,7 @@ cudaError_t launch_main(const DecodeArgs& a, dim3 grid, size_t smem, cudaStream_
 
 template <int D, int LMB>
 cudaError_t dispatch_vb(const DecodeArgs& a, int vb, dim3 grid, size_t smem, cudaStream_t s) {
+  if (vb == 3) return launch_main<D, LMB, 3>(a, grid, smem, s);
   return vb == 2 ? launch_main<D, LMB, 2>(a, grid, smem, s) : launch_main<D, LMB, 4>(a, grid, smem, s);
 }
 

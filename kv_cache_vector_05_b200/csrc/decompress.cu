@@ -90,7 +90,9 @@ __device__ void decompress_value(const DecompressArgs& a, int64_t i, int lane) {
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     const int j = lane * E + e, o = j * a.v_bits;
-    const uint32_t code = (cw[o >> 5] >> (o & 31)) & ((1u << a.v_bits) - 1u);
+    uint32_t code = cw[o >> 5] >> (o & 31);
+    if ((o & 31) + a.v_bits > 32) code |= cw[(o >> 5) + 1] << (32 - (o & 31));  // 3-bit codes straddle words
+    code &= (1u << a.v_bits) - 1u;
     const uint32_t par = reinterpret_cast<const uint32_t*>(a.v_params)[i * (D / kVGroup) + j / kVGroup];
     const float sc = __half2float(__ushort_as_half((unsigned short)(par & 0xffffu)));
     const float lo = __half2float(__ushort_as_half((unsigned short)(par >> 16)));

@@ -92,8 +92,8 @@ tq_status tq_codebook_load(const tq_params* p, void* stream, tq_ctx** out) {
     return fail(TQ_EUNSUPPORTED, "tq_codebook_load: k_lm_bits must be 1, 2 or 3");
   if (m < 0 || m > tq::kMaxM || m % 32)
     return fail(TQ_EUNSUPPORTED, "tq_codebook_load: qjl_m must be 0 (no QJL stage) or a multiple of 32 up to 256");
-  if (!(p->v_bits == 2 || p->v_bits == 4))
-    return fail(TQ_EUNSUPPORTED, "tq_codebook_load: v_bits must be 2 or 4");
+  if (!(p->v_bits == 2 || p->v_bits == 3 || p->v_bits == 4))
+    return fail(TQ_EUNSUPPORTED, "tq_codebook_load: v_bits must be 2, 3 or 4");
   if (p->v_group != tq::kVGroup)
     return fail(TQ_EUNSUPPORTED, "tq_codebook_load: v_group must be 32");
   if (p->rot != TQ_ROT_HADAMARD && p->rot != TQ_ROT_HAAR)

@@ -390,3 +390,36 @@ def test_keys_without_qjl_stage(d, lm_bits, v_bits, rotation, dtype):
     kx, _ = T.tq_decompress(ctx, gp, n)
     torch.cuda.synchronize()
     assert_close(kx.cpu().numpy(), O.decompress_keys(pk, Pi, c, S0, d), rtol=1e-4, atol=1e-5, what="keys")
+
+
+# ------------------------------------------------------------------ 3-bit values (K = V = 3)
+
+@pytest.mark.parametrize("d,lm_bits,rotation,dtype", [
+    (128, 2, "hadamard", "bf16"), (128, 2, "haar", "f32"), (64, 1, "hadamard", "bf16"), (256, 3, "haar", "bf16")])
+def test_three_bit_values(d, lm_bits, rotation, dtype):
+    """v_bits = 3 (codes straddle 32-bit words): compression, decode attention and
+    decompression of values through the C ABI against the oracle; with 2-bit Lloyd-Max keys
+    and their QJL bit this is the symmetric K = V = 3 configuration."""
+    v_bits, n, G = 3, 2500, 4
+    rng = np.random.default_rng([d, 3])
+    K = rng.standard_normal((n, d)) * rng.lognormal(0, 1, d)
+    V = rng.standard_normal((n, d)) * 2.0 + 0.5
+    V[7, :32] = 1.25                                                      # a constant group
+    ctx, g, ok, ov = _compress_both(K, V, d, lm_bits, v_bits, rotation, dtype)
+    assert g["v_codes"].shape == (n, 3 * d // 8)
+    assert_key_parity(compare_keys(g, ok, d, lm_bits, d))
+    assert_value_parity(compare_values(g, ov, d, v_bits))
+    gp = _upload({k: g[k] for k in ("k_codes", "k_signs", "k_norms", "v_codes", "v_params")})
+    q = W.queries((1, G, d), dtype="f32")
+    scores = torch.full((1, G, n), float("nan"), device=DEV)
+    out, _ = T.tq_decode_attention(ctx, torch.from_numpy(q).to(DEV), gp, 1, G, 1, n, scores=scores)
+    T.tq_check_device(ctx)
+    Pi, c, t, S = oracle_setup(d, lm_bits, d, rotation)
+    pk = {"codes": g["k_codes"], "signs": g["k_signs"], "norms": g["k_norms"]}
+    pv = {"codes": g["v_codes"], "params": g["v_params"]}
+    os_, oo = O.decode_attention(q[0].astype(np.float64), pk, pv, Pi, c, S, d, v_bits)
+    assert_close(scores[0].cpu().numpy(), os_, what="scores")
+    assert_close(out[0].cpu().numpy(), oo, what="out")
+    _, vx = T.tq_decompress(ctx, gp, n, keys=False)
+    torch.cuda.synchronize()
+    assert_close(vx.cpu().numpy(), O.dequantize_values(pv, v_bits, d), rtol=1e-6, atol=1e-6, what="values")
