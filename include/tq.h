@@ -71,8 +71,9 @@ typedef enum {
 /* Method parameters. Every array is HOST memory and is copied by
  * tq_codebook_load; the caller may free it afterwards.
  *   d              head dimension: 64, 128 or 256
- *   k_lm_bits      Lloyd-Max bits per key coordinate: 1, 2 or 3 (a key then costs
- *                  k_lm_bits + 1 bits per coordinate with its QJL sign)
+ *   k_lm_bits      Lloyd-Max bits per key coordinate: 1, 2, 3 or 4 (a key then costs
+ *                  k_lm_bits + 1 bits per coordinate with its QJL sign; 4 runs on the
+ *                  CUDA-core kernels)
  *   qjl_m          rows of the QJL matrix S: a multiple of 32, at most 256; or 0 for
  *                  keys without the QJL stage (Lloyd-Max codes only, the MSE-optimal
  *                  first stage): no sign bytes (k_signs may be NULL), gamma is still

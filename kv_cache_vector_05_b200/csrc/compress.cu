@@ -1848,6 +1848,7 @@ cudaError_t launch_compress(const tq_ctx* ctx, const void* k, const void* v, int
     }
     return cudaErrorInvalidValue;
   };
+  if (ctx->shape.lm_bits > 3) return generic(a);  // the tensor-core kernels take 1-3 Lloyd-Max bits
   if (ctx->shape.v_bits == 3 && k && v && ctx->S_sw128) {
     // 3-bit value codes straddle words: the tensor-core kernels take the keys alone and
     // the warp-per-vector kernel the values

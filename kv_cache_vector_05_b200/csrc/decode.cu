@@ -346,6 +346,7 @@ cudaError_t dispatch_lmb(const DecodeArgs& a, int lmb, int vb, dim3 grid, size_t
     case 1: return dispatch_vb<D, 1>(a, vb, grid, smem, s);
     case 2: return dispatch_vb<D, 2>(a, vb, grid, smem, s);
     case 3: return dispatch_vb<D, 3>(a, vb, grid, smem, s);
+    case 4: return dispatch_vb<D, 4>(a, vb, grid, smem, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -89,7 +89,7 @@ tq_status tq_codebook_load(const tq_params* p, void* stream, tq_ctx** out) {
   if (!(d == 64 || d == 128 || d == 256))
     return fail(TQ_EUNSUPPORTED, "tq_codebook_load: d must be 64, 128 or 256");
   if (b < 1 || b > tq::kMaxLmBits)
-    return fail(TQ_EUNSUPPORTED, "tq_codebook_load: k_lm_bits must be 1, 2 or 3");
+    return fail(TQ_EUNSUPPORTED, "tq_codebook_load: k_lm_bits must be 1, 2, 3 or 4");
   if (m < 0 || m > tq::kMaxM || m % 32)
     return fail(TQ_EUNSUPPORTED, "tq_codebook_load: qjl_m must be 0 (no QJL stage) or a multiple of 32 up to 256");
   if (!(p->v_bits == 2 || p->v_bits == 3 || p->v_bits == 4))

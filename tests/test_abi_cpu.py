@@ -74,7 +74,7 @@ def test_validation_without_gpu():
 
 
 @pytest.mark.parametrize("field,value,status", [
-    ("d", 96, _lib.TQ_EUNSUPPORTED), ("k_lm_bits", 4, _lib.TQ_EUNSUPPORTED),
+    ("d", 96, _lib.TQ_EUNSUPPORTED), ("k_lm_bits", 5, _lib.TQ_EUNSUPPORTED),
     ("qjl_m", 48, _lib.TQ_EUNSUPPORTED), ("v_bits", 5, _lib.TQ_EUNSUPPORTED),
     ("v_group", 16, _lib.TQ_EUNSUPPORTED), ("rot", 7, _lib.TQ_EINVAL),
 ])

@@ -423,3 +423,35 @@ def test_three_bit_values(d, lm_bits, rotation, dtype):
     _, vx = T.tq_decompress(ctx, gp, n, keys=False)
     torch.cuda.synchronize()
     assert_close(vx.cpu().numpy(), O.dequantize_values(pv, v_bits, d), rtol=1e-6, atol=1e-6, what="values")
+
+
+# ------------------------------------------------------------------ 4-bit Lloyd-Max codes
+
+@pytest.mark.parametrize("d,rotation,dtype,v_bits", [
+    (128, "hadamard", "bf16", 4), (64, "haar", "f32", 2), (256, "hadamard", "bf16", 3)])
+def test_four_bit_lloyd_max_keys(d, rotation, dtype, v_bits):
+    """k_lm_bits = 4 (16-level sphere codebook; 5-bit keys with the QJL sign): compression,
+    decode attention and decompression through the C ABI against the oracle."""
+    lm_bits, n, G = 4, 2000, 6
+    rng = np.random.default_rng([d, 4])
+    K = rng.standard_normal((n, d)) * rng.lognormal(0, 1, d)
+    V = rng.standard_normal((n, d))
+    K[[3, n - 2]] = 0.0
+    ctx, g, ok, ov = _compress_both(K, V, d, lm_bits, v_bits, rotation, dtype)
+    assert g["k_codes"].shape == (n, 4 * d // 8)
+    assert_key_parity(compare_keys(g, ok, d, lm_bits, d))
+    assert_value_parity(compare_values(g, ov, d, v_bits))
+    gp = _upload({k: g[k] for k in ("k_codes", "k_signs", "k_norms", "v_codes", "v_params")})
+    q = W.queries((1, G, d), dtype="f32")
+    scores = torch.full((1, G, n), float("nan"), device=DEV)
+    out, _ = T.tq_decode_attention(ctx, torch.from_numpy(q).to(DEV), gp, 1, G, 1, n, scores=scores)
+    T.tq_check_device(ctx)
+    Pi, c, t, S = oracle_setup(d, lm_bits, d, rotation)
+    pk = {"codes": g["k_codes"], "signs": g["k_signs"], "norms": g["k_norms"]}
+    pv = {"codes": g["v_codes"], "params": g["v_params"]}
+    os_, oo = O.decode_attention(q[0].astype(np.float64), pk, pv, Pi, c, S, d, v_bits)
+    assert_close(scores[0].cpu().numpy(), os_, what="scores")
+    assert_close(out[0].cpu().numpy(), oo, what="out")
+    kx, _ = T.tq_decompress(ctx, gp, n, values=False)
+    torch.cuda.synchronize()
+    assert_close(kx.cpu().numpy(), O.decompress_keys(pk, Pi, c, S, d), rtol=1e-4, atol=1e-5, what="keys")
