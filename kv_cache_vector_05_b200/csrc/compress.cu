@@ -112,12 +112,20 @@ __device__ bool key_front(const CompressArgs& a, int64_t i, int64_t o, int lane,
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     uint32_t idx = 0;
-    float cv = a.cb.c[0];
+    float cv;
+    if constexpr (LMB == 0) {
+      // any width: binary search for #{k : y >= t_k} over the power-of-two level count
+      for (int s = levels >> 1; s > 0; s >>= 1)
+        if (y[e] >= a.cb.t[idx + s - 1]) idx += s;
+      cv = a.cb.c[idx];
+    } else {
+      cv = a.cb.c[0];
 #pragma unroll
-    for (int k = 0; k < (LMB ? (1 << LMB) - 1 : kMaxLevels - 1); ++k) {
-      if ((LMB || k + 1 < levels) && y[e] >= a.cb.t[k]) {
-        idx = k + 1;
-        cv = a.cb.c[k + 1];
+      for (int k = 0; k < (1 << LMB) - 1; ++k) {
+        if (y[e] >= a.cb.t[k]) {
+          idx = k + 1;
+          cv = a.cb.c[k + 1];
+        }
       }
     }
     code_bits |= idx << (e * lmb);

@@ -118,6 +118,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
   float* sqsum_s = corr_s + G;              // [G]
   uint32_t* vcode_s = reinterpret_cast<uint32_t*>(sqsum_s + G);  // [kTile][VW]
   uint32_t* vpar_s = vcode_s + kTile * VW;                         // [kTile][NG]
+  float* cb_s = reinterpret_cast<float*>(vpar_s + kTile * NG);     // [2^LMB] centroids (LMB >= 4)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int chunk = blockIdx.x, unit = blockIdx.y;
@@ -136,6 +137,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
     const int h = idx / M, i = idx % M;
     sq_s[i * G + h] = a.ws_q[(size_t)(qrow0 + h) * a.q_stride + D + i];
   }
+  if constexpr (LMB >= 4)
+    for (int k = tid; k < (1 << LMB); k += kThreads) cb_s[k] = a.cb.c[k];
   for (int h = tid; h < G; h += kThreads) {
     m_s[h] = -INFINITY;
     l_s[h] = 0.f;
@@ -187,9 +190,14 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj) {
             const uint32_t code = stream_code<LMB>(kw, jj);
-            float cv = a.cb.c[0];
+            float cv;
+            if constexpr (LMB >= 4) {
+              cv = cb_s[code];  // many levels: a table in shared memory
+            } else {
+              cv = a.cb.c[0];
 #pragma unroll
-            for (int k = 1; k < (1 << LMB); ++k) cv = (code == (uint32_t)k) ? a.cb.c[k] : cv;
+              for (int k = 1; k < (1 << LMB); ++k) cv = (code == (uint32_t)k) ? a.cb.c[k] : cv;
+            }
             const float* qrow = qr_s + (g32 * 32 + jj) * G;
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -318,7 +326,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 size_t decode_smem_bytes(int d, int m, int G, int vbits) {
   const int vw = vbits * d / 32, ng = d / kVGroup;
   return sizeof(float) * ((size_t)d * G + (size_t)m * G + (size_t)G * kTile + 4 * (size_t)G) +
-         sizeof(uint32_t) * ((size_t)kTile * vw + (size_t)kTile * ng);
+         sizeof(uint32_t) * ((size_t)kTile * vw + (size_t)kTile * ng) + sizeof(float) * kMaxLevels;
 }
 
 template <int D, int LMB, int VB>
@@ -347,6 +355,13 @@ cudaError_t dispatch_lmb(const DecodeArgs& a, int lmb, int vb, dim3 grid, size_t
     case 2: return dispatch_vb<D, 2>(a, vb, grid, smem, s);
     case 3: return dispatch_vb<D, 3>(a, vb, grid, smem, s);
     case 4: return dispatch_vb<D, 4>(a, vb, grid, smem, s);
+  }
+  if constexpr (D <= 128) {  // more bits than 32 / (D / 32) do not fit a lane's code word at D = 256
+    switch (lmb) {
+      case 5: return dispatch_vb<D, 5>(a, vb, grid, smem, s);
+      case 6: return dispatch_vb<D, 6>(a, vb, grid, smem, s);
+      case 7: return dispatch_vb<D, 7>(a, vb, grid, smem, s);
+    }
   }
   return cudaErrorInvalidValue;
 }

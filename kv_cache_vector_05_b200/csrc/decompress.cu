@@ -43,9 +43,7 @@ __device__ void decompress_key(const DecompressArgs& a, int64_t i, int lane, flo
     uint32_t v = cw[o >> 5] >> (o & 31);
     if ((o & 31) + a.lm_bits > 32) v |= cw[(o >> 5) + 1] << (32 - (o & 31));
     const uint32_t code = v & ((1u << a.lm_bits) - 1u);
-    float cv = a.cb.c[0];
-#pragma unroll
-    for (int k = 1; k < kMaxLevels; ++k) cv = (k < a.cb.levels && code == (uint32_t)k) ? a.cb.c[k] : cv;
+    const float cv = a.cb.c[code];
     float acc = 0.f;
     for (int w = 0; w < swords; ++w) {
       const uint32_t bits = sw[w];

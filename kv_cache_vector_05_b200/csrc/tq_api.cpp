@@ -64,9 +64,9 @@ const char* tq_last_error(void) { return g_last_error; }
 
 tq_status tq_lloyd_max_codebook(int d, int bits, float* centroids, float* boundaries) {
   if (!centroids || !boundaries) return fail(TQ_EINVAL, "tq_lloyd_max_codebook: NULL output");
-  if (d < 4 || d > 4096 || bits < 1 || bits > 4)
-    return fail(TQ_EINVAL, "tq_lloyd_max_codebook: d must be in [4,4096], bits in [1,4]");
-  double c[16], t[15];
+  if (d < 4 || d > 4096 || bits < 1 || bits > 7)
+    return fail(TQ_EINVAL, "tq_lloyd_max_codebook: d must be in [4,4096], bits in [1,7]");
+  double c[128], t[127];  // up to 7 bits
   if (tq::lloyd_max_sphere(d, bits, c, t) != 0)
     return fail(TQ_EINVAL, "tq_lloyd_max_codebook: iteration did not converge");
   for (int k = 0; k < (1 << bits); ++k) centroids[k] = (float)c[k];
@@ -89,7 +89,9 @@ tq_status tq_codebook_load(const tq_params* p, void* stream, tq_ctx** out) {
   if (!(d == 64 || d == 128 || d == 256))
     return fail(TQ_EUNSUPPORTED, "tq_codebook_load: d must be 64, 128 or 256");
   if (b < 1 || b > tq::kMaxLmBits)
-    return fail(TQ_EUNSUPPORTED, "tq_codebook_load: k_lm_bits must be 1, 2, 3 or 4");
+    return fail(TQ_EUNSUPPORTED, "tq_codebook_load: k_lm_bits must be in [1, 7]");
+  if (b * (d / 32) > 32)
+    return fail(TQ_EUNSUPPORTED, "tq_codebook_load: k_lm_bits * d / 32 must be at most 32 (d = 256: 4 bits)");
   if (m < 0 || m > tq::kMaxM || m % 32)
     return fail(TQ_EUNSUPPORTED, "tq_codebook_load: qjl_m must be 0 (no QJL stage) or a multiple of 32 up to 256");
   if (!(p->v_bits == 2 || p->v_bits == 3 || p->v_bits == 4))

@@ -72,6 +72,87 @@ double integrate_mass(const SphereCoordinate& f, const GaussLegendre& gl, double
   return total;
 }
 
+// Initial boundaries from the high-resolution optimal point density, proportional to
+// f^(1/3) (Panter and Dite): the (i/L)-quantiles of that density, tabulated on a grid.
+void point_density_edges(const SphereCoordinate& f, int L, std::vector<double>& e) {
+  const int n = 200000;
+  std::vector<double> cdf(n + 1, 0.0);
+  const double h = 2.0 / n;
+  double prev = std::cbrt(f.pdf(-1.0));
+  for (int i = 1; i <= n; ++i) {
+    const double cur = std::cbrt(f.pdf(-1.0 + i * h));
+    cdf[i] = cdf[i - 1] + 0.5 * h * (prev + cur);
+    prev = cur;
+  }
+  int j = 0;
+  for (int k = 1; k < L; ++k) {
+    const double target = cdf[n] * k / L;
+    while (j < n && cdf[j + 1] < target) ++j;
+    const double span = cdf[j + 1] - cdf[j];
+    e[k - 1] = -1.0 + h * (j + (span > 0.0 ? (target - cdf[j]) / span : 0.0));
+  }
+}
+
+// The Lloyd-Max conditions solved by Newton's method on the L - 1 boundaries: residual
+// R_i = t_i - (c_i + c_{i+1}) / 2, where a cell mean moves with its right edge b as
+// f(b)(b - c)/M0 and with its left edge a as f(a)(c - a)/M0, so the Jacobian is
+// tridiagonal (Thomas algorithm). Steps are halved until the boundaries stay ordered.
+// Returns 0 and the cell means in c on convergence.
+int lloyd_max_newton(const SphereCoordinate& f, const GaussLegendre& gl, int L, std::vector<double>& c) {
+  std::vector<double> e(L - 1), m0(L), edges(L + 1), res(L - 1), right(L - 1), left(L - 1), diag(L - 1),
+      step(L - 1), cp(L - 1), dp(L - 1), cand(L - 1);
+  point_density_edges(f, L, e);
+  auto cells = [&]() {
+    edges[0] = -1.0;
+    edges[L] = 1.0;
+    for (int k = 1; k < L; ++k) edges[k] = e[k - 1];
+    for (int k = 0; k < L; ++k) {
+      m0[k] = integrate_mass(f, gl, edges[k], edges[k + 1], 96);
+      c[k] = f.first_moment(edges[k], edges[k + 1]) / m0[k];
+    }
+  };
+  for (int it = 0; it < 60; ++it) {
+    cells();
+    for (int i = 0; i < L - 1; ++i) {
+      const double fe = f.pdf(e[i]);
+      res[i] = e[i] - 0.5 * (c[i] + c[i + 1]);
+      right[i] = fe * (e[i] - c[i]) / m0[i];         // d c_i / d t_i
+      left[i] = fe * (c[i + 1] - e[i]) / m0[i + 1];  // d c_{i+1} / d t_i
+      diag[i] = 1.0 - 0.5 * (right[i] + left[i]);
+    }
+    // rows i: -left[i-1]/2 x_{i-1} + diag[i] x_i - right[i+1]/2 x_{i+1} = res[i]
+    const int n = L - 1;
+    cp[0] = n > 1 ? -0.5 * right[1] / diag[0] : 0.0;
+    dp[0] = res[0] / diag[0];
+    for (int i = 1; i < n; ++i) {
+      const double lo = -0.5 * left[i - 1];
+      const double den = diag[i] - lo * cp[i - 1];
+      cp[i] = i < n - 1 ? -0.5 * right[i + 1] / den : 0.0;
+      dp[i] = (res[i] - lo * dp[i - 1]) / den;
+    }
+    step[n - 1] = dp[n - 1];
+    for (int i = n - 2; i >= 0; --i) step[i] = dp[i] - cp[i] * step[i + 1];
+    double lam = 1.0;
+    for (int tries = 0; tries < 60; ++tries) {
+      bool ok = true;
+      for (int i = 0; i < n; ++i) {
+        cand[i] = e[i] - lam * step[i];
+        if (cand[i] <= -1.0 || cand[i] >= 1.0 || (i > 0 && cand[i] <= cand[i - 1])) ok = false;
+      }
+      if (ok) break;
+      lam *= 0.5;
+    }
+    double moved = 0.0;
+    for (int i = 0; i < n; ++i) moved = std::fmax(moved, std::fabs(cand[i] - e[i]));
+    e.swap(cand);
+    if (moved < 1e-12) {  // the cell moments' rounding in the far tails floors the steps near 1e-13
+      cells();
+      return 0;
+    }
+  }
+  return 1;
+}
+
 }  // namespace
 
 // Returns 0 on success, 1 if the iteration did not converge.
@@ -80,6 +161,13 @@ int lloyd_max_sphere(int d, int bits, double* centroids, double* boundaries) {
   SphereCoordinate f(d);
   GaussLegendre gl(24);
   std::vector<double> c(L), next(L), edges(L + 1);
+  if (bits >= 5) {  // many levels: Newton's method on the same two conditions
+    if (lloyd_max_newton(f, gl, L, c)) return 1;
+    for (int k = 0; k < L; ++k) next[k] = 0.5 * (c[k] - c[L - 1 - k]);  // odd by symmetry, exactly
+    for (int k = 0; k < L; ++k) centroids[k] = next[k];
+    for (int k = 1; k < L; ++k) boundaries[k - 1] = 0.5 * (next[k - 1] + next[k]);
+    return 0;
+  }
   const double spread = 2.0 / std::sqrt((double)d);
   for (int k = 0; k < L; ++k) c[k] = (L == 1) ? 0.0 : -spread + 2.0 * spread * k / (L - 1);
   for (int it = 0; it < 20000; ++it) {

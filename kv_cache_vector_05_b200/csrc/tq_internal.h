@@ -8,7 +8,7 @@
 
 namespace tq {
 
-constexpr int kMaxLmBits = 4;  // 1-3 on the tensor-core kernels, 4 on the CUDA-core ones
+constexpr int kMaxLmBits = 7;  // 1-3 on the tensor-core kernels, 4-7 on the CUDA-core ones
 constexpr int kMaxLevels = 1 << kMaxLmBits;
 constexpr int kMaxD = 256;
 constexpr int kMaxM = 256;

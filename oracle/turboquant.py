@@ -55,7 +55,7 @@ import numpy as np
 from scipy import integrate
 
 __all__ = [
-    "sphere_coordinate_pdf", "gaussian_pdf", "lloyd_max", "lloyd_max_sphere",
+    "sphere_coordinate_pdf", "gaussian_pdf", "lloyd_max", "lloyd_max_newton", "lloyd_max_sphere",
     "lloyd_max_gaussian", "quantizer_mse", "device_codebook", "hadamard_matrix",
     "hadamard_rotation", "haar_rotation", "bucketize", "pack_codes", "unpack_codes",
     "pack_signs", "unpack_signs", "compress_keys", "decompress_keys",
@@ -123,6 +123,73 @@ def lloyd_max(pdf, lo: float, hi: float, levels: int, scale: float,
     return c, 0.5 * (c[:-1] + c[1:])
 
 
+def _point_density_edges(pdf, lo: float, hi: float, levels: int, grid: int = 200001):
+    """Initial boundaries from the high-resolution optimal point density, proportional to
+    pdf^(1/3) (Panter and Dite): the (i/L)-quantiles of that normalized density."""
+    x = np.linspace(lo, hi, grid)
+    g = np.cbrt(np.array([float(pdf(v)) for v in x]))
+    cdf = np.concatenate([[0.0], np.cumsum(0.5 * (g[1:] + g[:-1]) * np.diff(x))])
+    return np.interp(np.arange(1, levels) / levels * cdf[-1], cdf, x)
+
+
+def _solve_tridiagonal(lower, diag, upper, rhs):
+    """Thomas algorithm for a tridiagonal system (lower[i] multiplies x[i], row i + 1)."""
+    n = diag.size
+    cp, dp = np.empty(n), np.empty(n)
+    cp[0] = upper[0] / diag[0] if n > 1 else 0.0
+    dp[0] = rhs[0] / diag[0]
+    for i in range(1, n):
+        den = diag[i] - lower[i - 1] * cp[i - 1]
+        cp[i] = upper[i] / den if i < n - 1 else 0.0
+        dp[i] = (rhs[i] - lower[i - 1] * dp[i - 1]) / den
+    out = np.empty(n)
+    out[-1] = dp[-1]
+    for i in range(n - 2, -1, -1):
+        out[i] = dp[i] - cp[i] * out[i + 1]
+    return out
+
+
+def lloyd_max_newton(pdf, lo: float, hi: float, levels: int, tol: float = 1e-14, max_iter: int = 60):
+    """The Lloyd-Max conditions (boundaries at centroid midpoints, centroids at cell means)
+    solved by Newton's method on the L - 1 boundaries, from the point-density start.
+
+    Residual R_i = t_i - (c_i + c_{i+1}) / 2 with c_k = int x f / int f over cell k; a
+    centroid moves with its cell's edges as dc/d(right edge b) = f(b)(b - c)/M0 and
+    dc/d(left edge a) = f(a)(c - a)/M0, so the Jacobian is tridiagonal. Steps are halved
+    until the boundaries stay ordered inside (lo, hi). Same fixed point as ``lloyd_max``,
+    reached in a few iterations where plain Lloyd iteration needs very many (many levels).
+    """
+    e = _point_density_edges(pdf, lo, hi, levels)
+
+    def cells(e):
+        edges = np.concatenate([[lo], e, [hi]])
+        m0 = np.array([_quad(lambda x: float(pdf(x)), edges[k], edges[k + 1]) for k in range(levels)])
+        m1 = np.array([_quad(lambda x: x * float(pdf(x)), edges[k], edges[k + 1]) for k in range(levels)])
+        return m0, m1 / m0
+
+    for _ in range(max_iter):
+        m0, c = cells(e)
+        res = e - 0.5 * (c[:-1] + c[1:])
+        fe = np.array([float(pdf(v)) for v in e])
+        right = fe * (e - c[:-1]) / m0[:-1]    # d c_i / d t_i (t_i is cell i's right edge)
+        left = fe * (c[1:] - e) / m0[1:]       # d c_{i+1} / d t_i (cell i+1's left edge)
+        diag = 1.0 - 0.5 * (right + left)
+        step = _solve_tridiagonal(-0.5 * left[:-1], diag, -0.5 * right[1:], res)
+        lam = 1.0
+        while True:
+            cand = e - lam * step
+            if np.all(np.diff(cand) > 0) and cand[0] > lo and cand[-1] < hi:
+                break
+            lam *= 0.5
+        e = cand
+        if np.max(np.abs(lam * step)) < tol:
+            break
+    else:  # pragma: no cover
+        raise RuntimeError("Lloyd-Max Newton iteration did not converge")
+    _, c = cells(e)
+    return c, 0.5 * (c[:-1] + c[1:])
+
+
 _SPHERE_CACHE: dict = {}
 
 
@@ -130,8 +197,11 @@ def lloyd_max_sphere(d: int, bits: int):
     """Codebook (centroids, boundaries) for the rotated coordinate at dimension d (R4)."""
     key = (d, bits)
     if key not in _SPHERE_CACHE:
-        c, _ = lloyd_max(lambda x: sphere_coordinate_pdf(x, d), -1.0, 1.0, 2 ** bits,
-                         1.0 / math.sqrt(d))
+        pdf = lambda x: sphere_coordinate_pdf(x, d)  # noqa: E731
+        if bits <= 4:
+            c, _ = lloyd_max(pdf, -1.0, 1.0, 2 ** bits, 1.0 / math.sqrt(d))
+        else:  # many levels: Newton's method on the same two conditions
+            c, _ = lloyd_max_newton(pdf, -1.0, 1.0, 2 ** bits)
         # The law is even, so the exact optimum is odd (c_k = -c_{L-1-k}); imposing it
         # removes round-off asymmetry and puts the middle boundary exactly at 0.
         c = 0.5 * (c - c[::-1])

@@ -36,9 +36,11 @@ def test_library_exports_every_declared_symbol():
     assert set(declared_functions()) == set(_lib.EXPORTED)
 
 
-@pytest.mark.parametrize("d", [64, 128, 256])
-@pytest.mark.parametrize("bits", [1, 2, 3])
+@pytest.mark.parametrize("d,bits", [(d, b) for d in (64, 128, 256) for b in (1, 2, 3, 4)]
+                         + [(64, 7), (128, 5), (128, 6), (128, 7)])
 def test_native_codebook_equals_oracle_fp32(d, bits):
+    """The library's fp64 solver (Lloyd iteration up to 4 bits, Newton's method beyond)
+    against the oracle's, after rounding both to fp32."""
     c, t = T.tq_lloyd_max_codebook(d, bits)
     oc, ot = O.device_codebook(d, bits)
     np.testing.assert_array_equal(c.astype(np.float64), oc)
@@ -74,7 +76,7 @@ def test_validation_without_gpu():
 
 
 @pytest.mark.parametrize("field,value,status", [
-    ("d", 96, _lib.TQ_EUNSUPPORTED), ("k_lm_bits", 5, _lib.TQ_EUNSUPPORTED),
+    ("d", 96, _lib.TQ_EUNSUPPORTED), ("k_lm_bits", 8, _lib.TQ_EUNSUPPORTED),
     ("qjl_m", 48, _lib.TQ_EUNSUPPORTED), ("v_bits", 5, _lib.TQ_EUNSUPPORTED),
     ("v_group", 16, _lib.TQ_EUNSUPPORTED), ("rot", 7, _lib.TQ_EINVAL),
 ])

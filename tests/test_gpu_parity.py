@@ -425,20 +425,23 @@ def test_three_bit_values(d, lm_bits, rotation, dtype):
     assert_close(vx.cpu().numpy(), O.dequantize_values(pv, v_bits, d), rtol=1e-6, atol=1e-6, what="values")
 
 
-# ------------------------------------------------------------------ 4-bit Lloyd-Max codes
+# ------------------------------------------------------------------ 4- to 7-bit Lloyd-Max codes
 
-@pytest.mark.parametrize("d,rotation,dtype,v_bits", [
-    (128, "hadamard", "bf16", 4), (64, "haar", "f32", 2), (256, "hadamard", "bf16", 3)])
-def test_four_bit_lloyd_max_keys(d, rotation, dtype, v_bits):
-    """k_lm_bits = 4 (16-level sphere codebook; 5-bit keys with the QJL sign): compression,
-    decode attention and decompression through the C ABI against the oracle."""
-    lm_bits, n, G = 4, 2000, 6
-    rng = np.random.default_rng([d, 4])
+@pytest.mark.parametrize("d,lm_bits,rotation,dtype,v_bits", [
+    (128, 4, "hadamard", "bf16", 4), (64, 4, "haar", "f32", 2), (256, 4, "hadamard", "bf16", 3),
+    (128, 7, "hadamard", "bf16", 4),   # 8-bit keys (7-bit Lloyd-Max + the QJL sign), 4-bit values
+    (64, 5, "haar", "bf16", 2), (128, 6, "haar", "f32", 3)])
+def test_wide_lloyd_max_keys(d, lm_bits, rotation, dtype, v_bits):
+    """k_lm_bits = 4..7 (16- to 128-level sphere codebooks, Lloyd iteration or Newton's
+    method): compression, decode attention and decompression through the C ABI against the
+    oracle."""
+    n, G = 2000, 6
+    rng = np.random.default_rng([d, lm_bits])
     K = rng.standard_normal((n, d)) * rng.lognormal(0, 1, d)
     V = rng.standard_normal((n, d))
     K[[3, n - 2]] = 0.0
     ctx, g, ok, ov = _compress_both(K, V, d, lm_bits, v_bits, rotation, dtype)
-    assert g["k_codes"].shape == (n, 4 * d // 8)
+    assert g["k_codes"].shape == (n, lm_bits * d // 8)
     assert_key_parity(compare_keys(g, ok, d, lm_bits, d))
     assert_value_parity(compare_values(g, ov, d, v_bits))
     gp = _upload({k: g[k] for k in ("k_codes", "k_signs", "k_norms", "v_codes", "v_params")})

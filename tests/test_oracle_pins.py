@@ -137,8 +137,7 @@ def _sphere_cell_mean(a, b, d):
     return first / (cdf(b) - cdf(a))
 
 
-@pytest.mark.parametrize("d", [64, 128, 256])
-@pytest.mark.parametrize("bits", [1, 2, 3])
+@pytest.mark.parametrize("d,bits", [(d, b) for d in (64, 128, 256) for b in (1, 2, 3, 4)] + [(128, 5), (64, 7), (128, 7)])
 def test_sphere_lloyd_max_optimality_conditions(d, bits):
     c, t = O.lloyd_max_sphere(d, bits)
     edges = np.concatenate([[-1.0], t, [1.0]])
@@ -452,3 +451,12 @@ def test_keys_without_qjl_stage():
     err = np.sum((K / nrm[:, None] - xh / n16[:, None]) ** 2, axis=1)
     want = d * O.quantizer_mse(lambda x: O.sphere_coordinate_pdf(x, d), -1, 1, c, t)
     assert abs(err.mean() - want) < 4 * err.std() / np.sqrt(n)
+
+
+@pytest.mark.parametrize("d,bits", [(64, 2), (128, 3), (256, 4)])
+def test_newton_and_lloyd_reach_the_same_codebook(d, bits):
+    """Newton's method on the boundaries (used from 5 bits on) and plain Lloyd iteration are
+    two routes to the same fixed point of the Lloyd-Max conditions."""
+    c1, _ = O.lloyd_max_sphere(d, bits)                     # Lloyd iteration
+    c2, _ = O.lloyd_max_newton(lambda x: O.sphere_coordinate_pdf(x, d), -1.0, 1.0, 2 ** bits)
+    np.testing.assert_allclose(c2, c1, rtol=0, atol=1e-12)
