@@ -46,6 +46,12 @@ R10 Values: groups of 32 consecutive coordinates of one vector; asymmetric
 R11 A zero key stores all-zero bytes.
 R12 Attention logits are scaled by 1/sqrt(d) unless the caller gives a scale;
     the softmax is exact (max-subtracted, two passes).
+R13 A sequence whose tokens are split into disjoint ranges (one per GPU) is
+    decoded range by range: each range yields its own normalized output o_r and
+    the log of its softmax denominator, lse_r = log sum_t exp(l_t); the output
+    over all tokens is sum_r exp(lse_r) o_r / sum_r exp(lse_r). This is an
+    identity of the softmax, not an approximation; an empty range has lse = -inf
+    and weighs nothing.
 """
 from __future__ import annotations
 
@@ -60,7 +66,7 @@ __all__ = [
     "hadamard_rotation", "haar_rotation", "bucketize", "pack_codes", "unpack_codes",
     "pack_signs", "unpack_signs", "compress_keys", "decompress_keys",
     "quantize_values", "dequantize_values", "prepare_query", "key_scores",
-    "decode_attention", "qjl_inner_product", "fp16_midpoint_distance",
+    "decode_attention", "log_partition", "merge_attention", "qjl_inner_product", "fp16_midpoint_distance",
     "k_record_bytes", "v_record_bytes", "QJL_CONST",
 ]
 
@@ -488,6 +494,37 @@ def decode_attention(q, packed_k: dict, packed_v: dict, Pi, centroids, S, d: int
     s = scores[:, :N]
     p = np.exp(s - s.max(axis=1, keepdims=True))
     return scores, (p @ vals[:N]) / p.sum(axis=1, keepdims=True)
+
+
+def log_partition(scores, length: int | None = None):
+    """lse_g = log sum_{t < N} exp(l_{g,t}) of logits [G, N'] over the first N tokens,
+    evaluated around the row maximum (R12, R13); -inf for every row when N = 0."""
+    s = np.atleast_2d(np.asarray(scores, dtype=np.float64))
+    N = s.shape[1] if length is None else length
+    if N == 0:
+        return np.full(s.shape[0], -np.inf)
+    mx = s[:, :N].max(axis=1)
+    return mx + np.log(np.exp(s[:, :N] - mx[:, None]).sum(axis=1))
+
+
+def merge_attention(outs, lses):
+    """Attention over the union of R disjoint token ranges from each range's output
+    o_r [R, G, d] and log-partition lse_r [R, G] (R13): weights exp(lse_r - max_r lse_r),
+    o = sum_r w_r o_r / sum_r w_r, lse = max + log sum_r w_r. Ranges with lse = -inf get
+    weight 0; a row whose ranges are all empty gets a zero output and lse = -inf.
+    Returns (out [G, d], lse [G]) in fp64."""
+    o = np.asarray(outs, dtype=np.float64)
+    ls = np.asarray(lses, dtype=np.float64)
+    G, d = o.shape[1], o.shape[2]
+    out, lse = np.zeros((G, d)), np.full(G, -np.inf)
+    for g in range(G):
+        mx = ls[:, g].max()
+        if mx == -np.inf:
+            continue
+        w = np.where(ls[:, g] == -np.inf, 0.0, np.exp(ls[:, g] - mx))
+        out[g] = (w[:, None] * o[:, g, :]).sum(axis=0) / w.sum()
+        lse[g] = mx + math.log(w.sum())
+    return out, lse
 
 
 def qjl_inner_product(x, r, S):

@@ -413,6 +413,93 @@ def test_decode_empty_sequence():
     assert not out.any()
 
 
+# ---------------------------------------------------------------- split sequence (R13)
+
+def _softmax_by_hand(logits_row, values):
+    """Softmax-weighted value sum and log denominator, token by token in Python floats
+    (no max shift: only for logits of modest size)."""
+    ws = [math.exp(x) for x in logits_row]
+    tot = sum(ws)
+    out = [sum(w * float(v[j]) for w, v in zip(ws, values)) / tot for j in range(len(values[0]))]
+    return out, math.log(tot)
+
+
+def test_log_partition_brute_force_and_large_logits():
+    rng = np.random.default_rng(21)
+    s = rng.standard_normal((3, 9))
+    want = [math.log(sum(math.exp(x) for x in row[:7])) for row in s]
+    np.testing.assert_allclose(O.log_partition(s, 7), want, rtol=1e-14, atol=1e-14)
+    # evaluated around the maximum: logits of 1000 stay finite; two equal ones give x + log 2
+    np.testing.assert_allclose(O.log_partition(np.array([[1000.0, 1000.0, -np.inf]])),
+                               [1000.0 + math.log(2.0)], rtol=1e-15)
+    assert np.all(O.log_partition(s, 0) == -np.inf)
+
+
+def test_merge_of_ranges_is_softmax_over_all_tokens():
+    """Tokens split into four ranges (one empty): merging each range's normalized output
+    and log-partition equals the softmax over all tokens, computed by hand."""
+    rng = np.random.default_rng(22)
+    G, N, d = 2, 23, 5
+    logits = rng.standard_normal((G, N)) * 3.0
+    vals = rng.standard_normal((N, d))
+    cuts = [0, 6, 6, 17, 23]
+    outs, lses = [], []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        o = np.zeros((G, d))
+        for g in range(G):
+            if b > a:
+                o[g] = _softmax_by_hand(logits[g, a:b], vals[a:b])[0]
+        outs.append(o)
+        lses.append(O.log_partition(logits[:, a:b]))
+    out, lse = O.merge_attention(np.stack(outs), np.stack(lses))
+    for g in range(G):
+        want_o, want_l = _softmax_by_hand(logits[g], vals)
+        np.testing.assert_allclose(out[g], want_o, rtol=1e-13, atol=1e-14)
+        assert abs(lse[g] - want_l) < 1e-13
+
+
+def test_merge_special_cases():
+    rng = np.random.default_rng(23)
+    o = rng.standard_normal((2, 3, 4))
+    lse = rng.standard_normal((2, 3))
+    out, l1 = O.merge_attention(o[:1], lse[:1])             # one range: itself
+    np.testing.assert_array_equal(out, o[0])
+    np.testing.assert_allclose(l1, lse[0], rtol=0, atol=1e-15)
+    empty = lse.copy()
+    empty[1] = -np.inf                                      # an empty range weighs nothing
+    out, l2 = O.merge_attention(o, empty)
+    np.testing.assert_allclose(out, o[0], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(l2, lse[0], rtol=0, atol=1e-15)
+    out, l3 = O.merge_attention(o, np.full((2, 3), -np.inf))  # all empty
+    assert not out.any() and np.all(l3 == -np.inf)
+    far = np.array([[0.0] * 3, [800.0] * 3])                # exp(-800) is 0 in fp64
+    out, l4 = O.merge_attention(o, far)
+    np.testing.assert_array_equal(out, o[1])
+    np.testing.assert_array_equal(l4, far[1])
+
+
+def test_split_decode_of_a_packed_cache_equals_whole_decode():
+    """Decoding token ranges of one packed cache separately and merging them (R13)
+    reproduces the decode over all valid tokens, and its log-partition."""
+    Pi, S, c, t, K, V = _small_cache(300, seed=5)
+    pk = O.compress_keys(K, Pi, c, t, S)
+    pv = O.quantize_values(V, 2)
+    q = np.random.default_rng(9).standard_normal((4, 32))
+    scores, whole = O.decode_attention(q, pk, pv, Pi, c, S, 32, 2, length=281)
+    outs, lses = [], []
+    cuts = [0, 128, 128, 200, 281]
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        pk_r = {k: v[a:b] for k, v in pk.items()}
+        pv_r = {k: v[a:b] for k, v in pv.items()}
+        sc, o = O.decode_attention(q, pk_r, pv_r, Pi, c, S, 32, 2, length=b - a)
+        np.testing.assert_array_equal(sc, scores[:, a:b])
+        outs.append(o)
+        lses.append(O.log_partition(sc, b - a))
+    out, lse = O.merge_attention(np.stack(outs), np.stack(lses))
+    np.testing.assert_allclose(out, whole, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse, O.log_partition(scores, 281), rtol=1e-14)
+
+
 def test_compression_distortion_is_near_lloyd_max():
     """Relative MSE of the LM stage alone is d*MSE_d of the codebook (rotation makes
     every coordinate follow the sphere law), checked on 4096 random keys at d=128."""
