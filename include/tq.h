@@ -212,6 +212,41 @@ tq_status tq_decode_attention_paged(const tq_ctx* ctx, const void* q, tq_dtype q
                                     float softmax_scale, float* scores, float* out,
                                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* tq_decode_attention that also returns each row's log-partition, for a sequence
+ * whose tokens are split over several GPUs (or several caches): every part decodes
+ * its own token range and the parts are combined by tq_merge_attention. The pages
+ * describe decode over one cache (skill card, "Что делает"); the split is an exact
+ * identity of that softmax over the union of disjoint ranges (output = sum_r
+ * e^{lse_r} out_r / sum_r e^{lse_r}), the log-sum-exp merge the split-K decode
+ * already applies to its chunks.
+ *   out  device fp32 [batch][hq][d]: attention over this cache's valid tokens only
+ *   lse  device fp32 [batch][hq], float-aligned: log sum_t exp(scaled logit_t) over
+ *        the same tokens (natural log); -inf where the length is 0 (out row zero)
+ * Other arguments, layouts and errors as tq_decode_attention; lse must not be NULL. */
+tq_status tq_decode_attention_partial(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int batch,
+                                      int hq, int hkv, const int32_t* seq_lens, int64_t max_len,
+                                      const uint8_t* k_codes, const uint8_t* k_signs,
+                                      const uint16_t* k_norms, const uint8_t* v_codes,
+                                      const uint16_t* v_params, float softmax_scale, float* scores,
+                                      float* out, float* lse, void* workspace, size_t workspace_bytes,
+                                      void* stream);
+
+/* Combine n_parts attention results over disjoint token ranges of the same rows
+ * (e.g. one tq_decode_attention_partial per GPU, gathered into one buffer) into
+ * the attention over all their tokens.
+ *   outs   device fp32: part r's outputs [rows][d] start at outs + r * outs_stride
+ *   lses   device fp32: part r's log-partitions [rows] start at lses + r * lses_stride
+ *          (-inf marks an empty range, which gets weight 0)
+ *   out    device fp32 [rows][d]: sum_r w_r out_r / sum_r w_r with w_r = exp(lse_r - max lse);
+ *          a row whose parts are all empty gets zeros
+ *   lse    NULL, or device fp32 [rows]: the merged log-partition (for merging again)
+ * Strides are in floats and must be at least rows * d and rows; all pointers float-
+ * aligned; out and lse must not overlap the inputs. Returns TQ_EINVAL for bad sizes
+ * or pointers, TQ_ECUDA if the launch fails; rows = 0 is a no-op. */
+tq_status tq_merge_attention(const float* outs, int64_t outs_stride, const float* lses,
+                             int64_t lses_stride, int n_parts, int64_t rows, int d, float* out,
+                             float* lse, void* stream);
+
 /* Synchronize `stream`, then read and clear the context's device error word.
  * Kernels never spin without a bound: a wait for a staged copy that does not
  * complete in time sets this word, abandons the rest of its work and exits, so

@@ -24,6 +24,7 @@ EXPORTED = (
     "tq_lloyd_max_codebook", "tq_haar_from_gaussian", "tq_compress_kv", "tq_compress_kv_slots",
     "tq_decode_workspace_bytes", "tq_decode_attention", "tq_decode_attention_paged", "tq_decompress",
     "tq_set_profile_events", "tq_check_device", "tq_decode_attention_static", "tq_decode_static_scratch_capacity",
+    "tq_decode_attention_partial", "tq_merge_attention",
 )
 
 
@@ -80,6 +81,11 @@ def _load() -> ctypes.CDLL:
     lib.tq_decode_attention_paged.argtypes = [vp, vp, c_int, c_int, c_int, c_int, vp, i64, vp, i64, i64, i64,
                                               vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp, sz, vp]
     lib.tq_decode_attention_paged.restype = c_int
+    lib.tq_decode_attention_partial.argtypes = [vp, vp, c_int, c_int, c_int, c_int, vp, i64,
+                                                vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp, vp, sz, vp]
+    lib.tq_decode_attention_partial.restype = c_int
+    lib.tq_merge_attention.argtypes = [vp, i64, vp, i64, c_int, i64, c_int, vp, vp, vp]
+    lib.tq_merge_attention.restype = c_int
     lib.tq_decompress.argtypes = [vp, vp, vp, vp, vp, vp, i64, vp, vp, vp]
     lib.tq_decompress.restype = c_int
     lib.tq_decode_attention_static.argtypes = [vp, vp, c_int, c_int, c_int, c_int, vp, i64,
@@ -296,6 +302,54 @@ def tq_decode_attention(ctx: Context, q, packed: dict, batch: int, hq: int, hkv:
         _ptr(packed["v_codes"]), _ptr(packed["v_params"]), float(softmax_scale),
         _ptr(scores), _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)), "tq_decode_attention")
     return out, scores
+
+
+def tq_decode_attention_partial(ctx: Context, q, packed: dict, batch: int, hq: int, hkv: int, max_len: int,
+                                seq_lens=None, softmax_scale: float = 0.0, scores=None, out=None, lse=None,
+                                workspace=None, stream=None):
+    """tq_decode_attention over this cache's tokens that also returns each row's
+    log-partition (for merging with other token ranges by tq_merge_attention).
+    Returns (out [batch, hq, d] fp32, lse [batch, hq] fp32, scores or None)."""
+    import torch
+    dev = q.device
+    q_dtype = TQ_F32 if q.dtype == torch.float32 else TQ_BF16
+    assert q.is_contiguous() and q.numel() == batch * hq * ctx.d
+    if out is None:
+        out = torch.empty((batch, hq, ctx.d), dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty((batch, hq), dtype=torch.float32, device=dev)
+    assert out.is_contiguous() and lse.is_contiguous() and lse.dtype == torch.float32
+    need = tq_decode_workspace_bytes(ctx, batch, hq, hkv, max_len)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.tq_decode_attention_partial(
+        ctx.handle, _ptr(q), q_dtype, batch, hq, hkv, _ptr(seq_lens), max_len,
+        _ptr(packed["k_codes"]), _ptr(packed["k_signs"]), _ptr(packed["k_norms"]),
+        _ptr(packed["v_codes"]), _ptr(packed["v_params"]), float(softmax_scale),
+        _ptr(scores), _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes, _stream(stream)),
+        "tq_decode_attention_partial")
+    return out, lse, scores
+
+
+def tq_merge_attention(outs, lses, out=None, lse=None, stream=None):
+    """Merge R attention results over disjoint token ranges: outs [R, rows..., d] and
+    lses [R, rows...] fp32 device tensors whose trailing dimensions are contiguous (the
+    leading stride may be anything, e.g. views into one gathered buffer). Returns
+    (out [rows..., d], lse or None)."""
+    import torch
+    R, d = outs.shape[0], outs.shape[-1]
+    rows = int(np.prod(outs.shape[1:-1])) if outs.dim() > 2 else 1
+    assert outs.dtype == torch.float32 and lses.dtype == torch.float32 and lses.shape[0] == R
+    assert lses[0].numel() == rows
+    assert outs[0].is_contiguous() and lses[0].is_contiguous()
+    if out is None:
+        out = torch.empty(tuple(outs.shape[1:]), dtype=torch.float32, device=outs.device)
+    assert out.is_contiguous() and out.numel() == rows * d
+    _check(lib.tq_merge_attention(_ptr(outs), int(outs.stride(0)) if R > 1 else rows * d, _ptr(lses),
+                                  int(lses.stride(0)) if R > 1 else rows, R, rows, d, _ptr(out), _ptr(lse),
+                                  _stream(stream)), "tq_merge_attention")
+    return out, lse
 
 
 def tq_decode_attention_paged(ctx: Context, q, packed: dict, batch: int, hq: int, hkv: int, max_len: int,

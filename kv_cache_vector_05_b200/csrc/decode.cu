@@ -297,6 +297,7 @@ struct CombineArgs {
   const float* ws_part;
   int part_stride, n_chunks, G, hq, hkv, d;
   float* out;
+  float* lse;  // null, or the log of each row's softmax denominator
 };
 
 __global__ void __launch_bounds__(kThreads) combine_kernel(const __grid_constant__ CombineArgs a) {
@@ -318,6 +319,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const __grid_constant
       }
     }
     a.out[(size_t)row * a.d + j] = den > 0.f ? num / den : 0.f;
+    if (a.lse && j == 0) a.lse[row] = den > 0.f ? mx + logf(den) : -INFINITY;
   }
 }
 
@@ -423,12 +425,12 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const void*
                           int hq, int hkv, const int32_t* seq_lens, int64_t max_len, const Paging& pg,
                           const uint8_t* k_codes,
                           const uint8_t* k_signs, const uint16_t* k_norms, const uint8_t* v_codes,
-                          const uint16_t* v_params, float scale, float* scores, float* out, void* workspace,
-                          cudaStream_t stream) {
+                          const uint16_t* v_params, float scale, float* scores, float* out, float* lse,
+                          void* workspace, cudaStream_t stream) {
   const int d = ctx->shape.d, m = ctx->shape.m, G = hq / hkv;
   if (plan.mma)
     return launch_decode_mma(ctx, plan, q, q_dtype, batch, hq, hkv, seq_lens, max_len, pg, k_codes, k_signs,
-                             k_norms, v_codes, v_params, scale, scores, out, workspace, stream);
+                             k_norms, v_codes, v_params, scale, scores, out, lse, workspace, stream);
   if ((G + (kThreads / d) - 1) / (kThreads / d) > kMaxQ) return cudaErrorInvalidValue;
   float* ws_q = static_cast<float*>(workspace);
   float* ws_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + plan.ws_q_bytes);
@@ -493,6 +495,7 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const void*
   ca.hkv = hkv;
   ca.d = d;
   ca.out = out;
+  ca.lse = lse;
   combine_kernel<<<batch * hq, d, 0, stream>>>(ca);
   return cudaGetLastError();
 }

@@ -895,6 +895,7 @@ __global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid
 struct CombineArgs {
   const float* ws_part;
   float* out;
+  float* lse;  // null, or the log of each row's softmax denominator
   int hq, hkv, G, s_max;
   int64_t tiles_per_unit, total_tiles, n_ctas;
 };
@@ -947,7 +948,10 @@ __global__ void __launch_bounds__(kD) combine_mma_kernel(const __grid_constant__
   __syncthreads();
   den = (red_s[1][0] + red_s[1][1]) + (red_s[1][2] + red_s[1][3]);
   const int b = u / a.hkv, kvh = u - b * a.hkv;
-  a.out[(size_t)(b * a.hq + kvh * a.G + h) * kD + tid] = den > 0.f ? (num0 + num1) / den : 0.f;
+  const int row = b * a.hq + kvh * a.G + h;
+  a.out[(size_t)row * kD + tid] = den > 0.f ? (num0 + num1) / den : 0.f;
+  // The partial maxima and sums are in base 2 (logits times log2(e)): back to natural log.
+  if (a.lse && tid == 0) a.lse[row] = den > 0.f ? (M + log2f(den)) * 0.6931471805599453f : -INFINITY;
 }
 
 template <int LMB, int VB, int NB>
@@ -1031,8 +1035,8 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
                               int hq, int hkv, const int32_t* seq_lens, int64_t max_len, const Paging& pg,
                               const uint8_t* k_codes,
                               const uint8_t* k_signs, const uint16_t* k_norms, const uint8_t* v_codes,
-                              const uint16_t* v_params, float scale, float* scores, float* out, void* workspace,
-                              cudaStream_t stream) {
+                              const uint16_t* v_params, float scale, float* scores, float* out, float* lse,
+                              void* workspace, cudaStream_t stream) {
   char* ws = static_cast<char*>(workspace);
   uint32_t* frag = reinterpret_cast<uint32_t*>(ws + plan.off_frag);
   float* part = reinterpret_cast<float*>(ws + plan.off_part);
@@ -1106,6 +1110,7 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
   CombineArgs ca;
   ca.ws_part = part;
   ca.out = out;
+  ca.lse = lse;
   ca.hq = hq;
   ca.hkv = hkv;
   ca.G = G;

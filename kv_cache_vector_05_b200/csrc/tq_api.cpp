@@ -292,7 +292,7 @@ tq_status decode_impl(const char* name, const tq_ctx* c, const void* q, tq_dtype
                       int hkv, const int32_t* seq_lens, int64_t max_len, const tq::Paging& pg,
                       const uint8_t* k_codes, const uint8_t* k_signs, const uint16_t* k_norms,
                       const uint8_t* v_codes, const uint16_t* v_params, float softmax_scale, float* scores,
-                      float* out, void* workspace, size_t workspace_bytes, void* stream) {
+                      float* out, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
   const std::string nm(name);
   if (!c) return fail(TQ_EINVAL, nm + ": NULL context");
   if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return fail(TQ_EINVAL, nm + ": bad dtype");
@@ -304,6 +304,8 @@ tq_status decode_impl(const char* name, const tq_ctx* c, const void* q, tq_dtype
     return fail(TQ_EINVAL, nm + ": softmax_scale must be finite and >= 0");
   if (batch == 0) return TQ_OK;
   if (!q || !out) return fail(TQ_EINVAL, nm + ": NULL q or out");
+  if (lse && reinterpret_cast<uintptr_t>(lse) % alignof(float))
+    return fail(TQ_EINVAL, nm + ": lse not aligned to a float");
   if (max_len > 0 && (!k_codes || (c->shape.m > 0 && !k_signs) || !k_norms || !v_codes || !v_params))
     return fail(TQ_EINVAL, nm + ": NULL packed cache");
   const void* ptrs[] = {q, out, k_codes, k_signs, k_norms, v_codes, v_params, workspace, scores, seq_lens};
@@ -314,8 +316,14 @@ tq_status decode_impl(const char* name, const tq_ctx* c, const void* q, tq_dtype
   if (!workspace || workspace_bytes < plan.total_bytes)
     return fail(TQ_EINVAL, nm + ": workspace missing or too small");
   float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)c->shape.d);
+  if (max_len == 0) {  // no tokens anywhere: zero outputs, log-partitions -inf (a merge of no parts)
+    cudaError_t e = tq::launch_merge(nullptr, 0, nullptr, 0, 0, (int64_t)batch * hq, c->shape.d, out, lse,
+                                     static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail_cuda(e, name);
+    return TQ_OK;
+  }
   cudaError_t e = tq::launch_decode(c, plan, q, (int)q_dtype, batch, hq, hkv, seq_lens, max_len, pg, k_codes,
-                                    k_signs, k_norms, v_codes, v_params, scale, scores, out, workspace,
+                                    k_signs, k_norms, v_codes, v_params, scale, scores, out, lse, workspace,
                                     static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail_cuda(e, name);
   return TQ_OK;
@@ -330,8 +338,41 @@ tq_status tq_decode_attention(const tq_ctx* c, const void* q, tq_dtype q_dtype, 
                               float* out, void* workspace, size_t workspace_bytes, void* stream) {
   const tq::Paging contiguous{nullptr, 0, 0, 0};
   return decode_impl("tq_decode_attention", c, q, q_dtype, batch, hq, hkv, seq_lens, max_len, contiguous,
-                     k_codes, k_signs, k_norms, v_codes, v_params, softmax_scale, scores, out, workspace,
+                     k_codes, k_signs, k_norms, v_codes, v_params, softmax_scale, scores, out, nullptr, workspace,
                      workspace_bytes, stream);
+}
+
+tq_status tq_decode_attention_partial(const tq_ctx* c, const void* q, tq_dtype q_dtype, int batch, int hq,
+                                      int hkv, const int32_t* seq_lens, int64_t max_len,
+                                      const uint8_t* k_codes, const uint8_t* k_signs,
+                                      const uint16_t* k_norms, const uint8_t* v_codes,
+                                      const uint16_t* v_params, float softmax_scale, float* scores,
+                                      float* out, float* lse, void* workspace, size_t workspace_bytes,
+                                      void* stream) {
+  if (batch > 0 && !lse) return fail(TQ_EINVAL, "tq_decode_attention_partial: NULL lse");
+  const tq::Paging contiguous{nullptr, 0, 0, 0};
+  return decode_impl("tq_decode_attention_partial", c, q, q_dtype, batch, hq, hkv, seq_lens, max_len,
+                     contiguous, k_codes, k_signs, k_norms, v_codes, v_params, softmax_scale, scores, out, lse,
+                     workspace, workspace_bytes, stream);
+}
+
+tq_status tq_merge_attention(const float* outs, int64_t outs_stride, const float* lses, int64_t lses_stride,
+                             int n_parts, int64_t rows, int d, float* out, float* lse, void* stream) {
+  if (n_parts <= 0 || rows < 0 || d <= 0)
+    return fail(TQ_EINVAL, "tq_merge_attention: n_parts and d must be positive, rows >= 0");
+  if (rows > 0x7fffffff) return fail(TQ_EINVAL, "tq_merge_attention: more than 2^31 - 1 rows");
+  if (outs_stride < rows * d || lses_stride < rows)
+    return fail(TQ_EINVAL, "tq_merge_attention: a part's stride is below its size");
+  if (rows == 0) return TQ_OK;
+  if (!outs || !lses || !out) return fail(TQ_EINVAL, "tq_merge_attention: NULL outs, lses or out");
+  const void* ptrs[] = {outs, lses, out, lse};
+  for (const void* ptr : ptrs)
+    if (ptr && reinterpret_cast<uintptr_t>(ptr) % alignof(float))
+      return fail(TQ_EINVAL, "tq_merge_attention: pointers must be aligned to a float");
+  cudaError_t e = tq::launch_merge(outs, outs_stride, lses, lses_stride, n_parts, rows, d, out, lse,
+                                   static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e, "tq_merge_attention");
+  return TQ_OK;
 }
 
 tq_status tq_decode_attention_paged(const tq_ctx* c, const void* q, tq_dtype q_dtype, int batch, int hq,
@@ -349,8 +390,8 @@ tq_status tq_decode_attention_paged(const tq_ctx* c, const void* q, tq_dtype q_d
     return fail(TQ_EINVAL, "tq_decode_attention_paged: max_pages below ceil(max_len / page_size), or no pages");
   const tq::Paging paged{block_table, page_size, max_pages, n_pages};
   return decode_impl("tq_decode_attention_paged", c, q, q_dtype, batch, hq, hkv, seq_lens, max_len, paged, k_codes,
-                     k_signs, k_norms, v_codes, v_params, softmax_scale, scores, out, workspace, workspace_bytes,
-                     stream);
+                     k_signs, k_norms, v_codes, v_params, softmax_scale, scores, out, nullptr, workspace,
+                     workspace_bytes, stream);
 }
 
 tq_status tq_decompress(const tq_ctx* c, const uint8_t* k_codes, const uint8_t* k_signs,

@@ -89,7 +89,8 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const void*
                           int batch, int hq, int hkv, const int32_t* seq_lens, int64_t max_len,
                           const Paging& pg, const uint8_t* k_codes, const uint8_t* k_signs,
                           const uint16_t* k_norms, const uint8_t* v_codes, const uint16_t* v_params,
-                          float scale, float* scores, float* out, void* workspace, cudaStream_t stream);
+                          float scale, float* scores, float* out, float* lse, void* workspace,
+                          cudaStream_t stream);
 
 bool mma_decode_supported(const tq_ctx* ctx, int G);
 
@@ -104,8 +105,12 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
                               int hq, int hkv, const int32_t* seq_lens, int64_t max_len, const Paging& pg,
                               const uint8_t* k_codes,
                               const uint8_t* k_signs, const uint16_t* k_norms, const uint8_t* v_codes,
-                              const uint16_t* v_params, float scale, float* scores, float* out, void* workspace,
-                              cudaStream_t stream);
+                              const uint16_t* v_params, float scale, float* scores, float* out, float* lse,
+                              void* workspace, cudaStream_t stream);
+
+// Log-sum-exp merge of n_parts attention outputs of disjoint token ranges (merge.cu).
+cudaError_t launch_merge(const float* outs, int64_t outs_stride, const float* lses, int64_t lses_stride,
+                         int n_parts, int64_t rows, int d, float* out, float* lse, cudaStream_t stream);
 
 cudaError_t launch_decompress(const tq_ctx* ctx, const uint8_t* k_codes, const uint8_t* k_signs,
                               const uint16_t* k_norms, const uint8_t* v_codes,

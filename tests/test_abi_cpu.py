@@ -75,6 +75,28 @@ def test_validation_without_gpu():
     assert lib.tq_lloyd_max_codebook(128, 2, None, None) == _lib.TQ_EINVAL
 
 
+def test_split_sequence_entry_points_validate_without_gpu():
+    """The partial decode and the merge reject bad sizes and pointers before any launch;
+    a merge of zero rows is a no-op."""
+    lib, E = _lib.lib, _lib.TQ_EINVAL
+    assert lib.tq_decode_attention_partial(None, None, 0, 1, 8, 1, None, 16, None, None, None, None, None,
+                                           0.0, None, None, None, None, 0, None) == E
+    buf = np.zeros(64, np.float32)
+    p = buf.ctypes.data
+    odd = ctypes.c_void_p(p + 2)                              # not float-aligned
+    ok = ctypes.c_void_p(p)
+    assert lib.tq_merge_attention(ok, 8, ok, 2, 0, 2, 4, ok, None, None) == E       # no parts
+    assert lib.tq_merge_attention(ok, 8, ok, 2, 2, 2, 0, ok, None, None) == E       # d = 0
+    assert lib.tq_merge_attention(ok, 8, ok, 2, 2, -1, 4, ok, None, None) == E      # rows < 0
+    assert lib.tq_merge_attention(ok, 7, ok, 2, 2, 2, 4, ok, None, None) == E       # outs stride < rows*d
+    assert lib.tq_merge_attention(ok, 8, ok, 1, 2, 2, 4, ok, None, None) == E       # lses stride < rows
+    assert lib.tq_merge_attention(None, 8, ok, 2, 2, 2, 4, ok, None, None) == E     # NULL outs
+    assert lib.tq_merge_attention(ok, 8, ok, 2, 2, 2, 4, None, None, None) == E     # NULL out
+    assert lib.tq_merge_attention(odd, 8, ok, 2, 2, 2, 4, ok, None, None) == E
+    assert lib.tq_merge_attention(ok, 8, ok, 2, 2, 2, 4, ok, odd, None) == E
+    assert lib.tq_merge_attention(None, 0, None, 0, 3, 0, 4, None, None, None) == _lib.TQ_OK
+
+
 @pytest.mark.parametrize("field,value,status", [
     ("d", 96, _lib.TQ_EUNSUPPORTED), ("k_lm_bits", 8, _lib.TQ_EUNSUPPORTED),
     ("qjl_m", 48, _lib.TQ_EUNSUPPORTED), ("v_bits", 5, _lib.TQ_EUNSUPPORTED),
