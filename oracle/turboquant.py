@@ -46,7 +46,7 @@ R10 Values: groups of 32 consecutive coordinates of one vector; asymmetric
 R11 A zero key stores all-zero bytes.
 R12 Attention logits are scaled by 1/sqrt(d) unless the caller gives a scale;
     the softmax is exact (max-subtracted, two passes).
-R13 A sequence whose tokens are split into disjoint ranges (one per GPU) is
+R15 A sequence whose tokens are split into disjoint ranges (one per GPU) is
     decoded range by range: each range yields its own normalized output o_r and
     the log of its softmax denominator, lse_r = log sum_t exp(l_t); the output
     over all tokens is sum_r exp(lse_r) o_r / sum_r exp(lse_r). This is an
@@ -498,7 +498,7 @@ def decode_attention(q, packed_k: dict, packed_v: dict, Pi, centroids, S, d: int
 
 def log_partition(scores, length: int | None = None):
     """lse_g = log sum_{t < N} exp(l_{g,t}) of logits [G, N'] over the first N tokens,
-    evaluated around the row maximum (R12, R13); -inf for every row when N = 0."""
+    evaluated around the row maximum (R12, R15); -inf for every row when N = 0."""
     s = np.atleast_2d(np.asarray(scores, dtype=np.float64))
     N = s.shape[1] if length is None else length
     if N == 0:
@@ -509,7 +509,7 @@ def log_partition(scores, length: int | None = None):
 
 def merge_attention(outs, lses):
     """Attention over the union of R disjoint token ranges from each range's output
-    o_r [R, G, d] and log-partition lse_r [R, G] (R13): weights exp(lse_r - max_r lse_r),
+    o_r [R, G, d] and log-partition lse_r [R, G] (R15): weights exp(lse_r - max_r lse_r),
     o = sum_r w_r o_r / sum_r w_r, lse = max + log sum_r w_r. Ranges with lse = -inf get
     weight 0; a row whose ranges are all empty gets a zero output and lse = -inf.
     Returns (out [G, d], lse [G]) in fp64."""

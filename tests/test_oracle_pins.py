@@ -413,7 +413,7 @@ def test_decode_empty_sequence():
     assert not out.any()
 
 
-# ---------------------------------------------------------------- split sequence (R13)
+# ---------------------------------------------------------------- split sequence (R15)
 
 def _softmax_by_hand(logits_row, values):
     """Softmax-weighted value sum and log denominator, token by token in Python floats
@@ -437,7 +437,7 @@ def test_log_partition_brute_force_and_large_logits():
 
 def test_merge_of_ranges_is_softmax_over_all_tokens():
     """Tokens split into four ranges (one empty): merging each range's normalized output
-    and log-partition equals the softmax over all tokens, computed by hand."""
+    and log-partition equals the softmax over all tokens, computed by hand (R15)."""
     rng = np.random.default_rng(22)
     G, N, d = 2, 23, 5
     logits = rng.standard_normal((G, N)) * 3.0
@@ -479,8 +479,8 @@ def test_merge_special_cases():
 
 
 def test_split_decode_of_a_packed_cache_equals_whole_decode():
-    """Decoding token ranges of one packed cache separately and merging them (R13)
-    reproduces the decode over all valid tokens, and its log-partition."""
+    """Decoding token ranges of one packed cache separately and merging them
+    reproduces the decode over all valid tokens, and its log-partition (R15)."""
     Pi, S, c, t, K, V = _small_cache(300, seed=5)
     pk = O.compress_keys(K, Pi, c, t, S)
     pv = O.quantize_values(V, 2)
