@@ -61,6 +61,9 @@ def parse():
     ap.add_argument("--no-paged", action="store_true", help="skip the paged-cache timings")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--sweep", action="store_true",
+                    help="compression sweep instead of the step: 1,048,576 bf16 keys at every head "
+                         "dimension (64, 128, 256), key bit width (2, 3, 4) and rotation (Hadamard, Haar)")
     ap.add_argument("--decode-only", action="store_true",
                     help="decode a random packed cache of the workload's size (no bf16 inputs, no "
                          "compression, no e2e): a small process for profiler captures")
@@ -561,9 +564,65 @@ def run_ours(args, w: W.Workload):
         dist.destroy_process_group()
 
 
+def run_sweep(args):
+    """Keys-only compression of W.SWEEP_VECTORS bf16 N(0,1) keys for every (d, b, rotation)
+    (b total key bits: b - 1 Lloyd-Max bits + 1 QJL bit, m = d). Each configuration is
+    timed over `steps` launches with CUDA events, the L2 flushed before each; one JSON line
+    with a row per configuration (median launch time, keys/s, GB/s of algorithmic bytes:
+    2d bytes of bf16 in, the packed record out)."""
+    import torch
+    import kv_cache_vector_05_b200 as T
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peak, peak_kind = measured_peaks()
+    n = W.SWEEP_VECTORS
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_src = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    rows = []
+    for d in W.SWEEP_D:
+        K = W.device_normal((n, d), seed=1, device=dev).to(torch.bfloat16)
+        dr = W.method_draws(d, d)
+        for b in W.SWEEP_BITS:
+            lm = b - 1
+            c, t = T.tq_lloyd_max_codebook(d, lm)
+            for rot in ("hadamard", "haar"):
+                haar = T.tq_haar_from_gaussian(dr["haar_gaussian"]) if rot == "haar" else None
+                ctx = T.tq_codebook_load(d, lm, 2, c, t, dr["qjl_S"], rotation=rot,
+                                         hadamard_signs=dr["hadamard_signs"], haar=haar)
+                out = T.tq_compress_kv(ctx, K, None)
+                for _ in range(max(3, args.warmup)):
+                    T.tq_compress_kv(ctx, K, None, **out)
+                ms = []
+                for _ in range(args.steps):
+                    flush_buf.zero_()
+                    flush_src.sum()
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    T.tq_compress_kv(ctx, K, None, **out)
+                    e1.record()
+                    torch.cuda.synchronize()
+                    ms.append(e0.elapsed_time(e1))
+                T.tq_check_device(ctx)
+                med = statistics.median(ms)
+                rec = lm * d // 8 + d // 8 + 4
+                alg = n * (2 * d + rec)
+                rows.append({"d": d, "b": b, "rotation": rot, "ms": med, "keys_per_s": n / (med * 1e-3),
+                             "gbs": alg / (med * 1e-3) / 1e9, "frac": alg / (med * 1e-3) / 1e9 / peak,
+                             "alg_bytes_per_key": 2 * d + rec})
+                log(f"sweep d={d} b={b} {rot}: {med:.4f} ms, {rows[-1]['gbs']:.0f} GB/s")
+                ctx.close()
+        del K
+    print(json.dumps({"metric": "compress keys/s (sweep)", "unit": "keys/s", "vectors": n, "dtype": "bf16",
+                      "steps": args.steps, "warmup": max(3, args.warmup), "peak_gbs": peak, "peak_kind": peak_kind,
+                      "l2": "flushed before each launch: 256 MiB write, then 256 MiB read", "sweep": rows}))
+
+
 def main():
     args = parse()
     w = W.WORKLOADS[args.workload]
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.impl == "reference":
         run_reference(args, w)
     else:
