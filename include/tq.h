@@ -7,7 +7,7 @@
  *   keys   : n = ||k||, u = k/n, y = Pi u (random orthogonal rotation),
  *            idx = Lloyd-Max cell of each y_j, r = y - c[idx], gamma = ||r||,
  *            1-bit QJL signs s = [S r >= 0], packed codes + signs + fp16 (n, gamma)
- *   values : groups of 32 coordinates, min/max uniform codes at 2 or 4 bits,
+ *   values : groups of 32 coordinates, min/max uniform codes at 2, 3 or 4 bits,
  *            fp16 (scale, min) per group
  *   decode : qr = Pi q, sq = S qr; logit_t = scale * n_t * (<qr, c[idx_t]>
  *            + sqrt(pi/2)/m * gamma_t * <sq, s_t>); online softmax over the cache;
@@ -71,9 +71,10 @@ typedef enum {
 /* Method parameters. Every array is HOST memory and is copied by
  * tq_codebook_load; the caller may free it afterwards.
  *   d              head dimension: 64, 128 or 256
- *   k_lm_bits      Lloyd-Max bits per key coordinate: 1, 2, 3 or 4 (a key then costs
- *                  k_lm_bits + 1 bits per coordinate with its QJL sign; 4 runs on the
- *                  CUDA-core kernels)
+ *   k_lm_bits      Lloyd-Max bits per key coordinate: 1 to 7 (a key then costs
+ *                  k_lm_bits + 1 bits per coordinate with its QJL sign); a lane's
+ *                  codes must fit one 32-bit word, k_lm_bits * d / 32 <= 32 (so at
+ *                  most 4 bits at d = 256); 4 bits and more run on the CUDA-core kernels
  *   qjl_m          rows of the QJL matrix S: a multiple of 32, at most 256; or 0 for
  *                  keys without the QJL stage (Lloyd-Max codes only, the MSE-optimal
  *                  first stage): no sign bytes (k_signs may be NULL), gamma is still
