@@ -256,8 +256,8 @@ tq_status tq_merge_attention(const float* outs, int64_t outs_stride, const float
  * slot or page index was out of range, TQ_OK otherwise. */
 tq_status tq_check_device(const tq_ctx* ctx, void* stream);
 
-/* Decode attention that allocates nothing and takes no workspace. The paper has
- * no counterpart; this entry point exists for callers that cannot allocate device
+/* Decode attention that allocates nothing and takes no workspace. The pages describe
+ * no such call; this entry point exists for callers that cannot allocate device
  * memory: a plugin that is handed only input and output pointers by its host
  * application, a serving loop that must not call cudaMalloc once running (the
  * allocation can synchronize the device and stall other streams), or a runtime
