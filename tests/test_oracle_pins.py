@@ -203,6 +203,23 @@ def test_packing_hand_examples():
         np.testing.assert_array_equal(O.unpack_codes(got, bits, codes.shape[1]), codes)
 
 
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6, 7])
+def test_packing_round_trip_and_bit_positions(bits):
+    """Every width the library takes: bits * d / 8 bytes per record, unpack(pack(x)) = x, and
+    bit k of code j sits at stream bit bits * j + k (R8), checked bit by bit."""
+    rng = np.random.default_rng(bits)
+    for d in (32, 64, 128):
+        codes = rng.integers(0, 1 << bits, size=(5, d))
+        packed = O.pack_codes(codes, bits)
+        assert packed.shape == (5, bits * d // 8)
+        np.testing.assert_array_equal(O.unpack_codes(packed, bits, d), codes)
+        stream = packed[0]
+        for j in range(d):
+            for k in range(bits):
+                pos = bits * j + k
+                assert (stream[pos // 8] >> (pos % 8)) & 1 == (codes[0, j] >> k) & 1
+
+
 def test_sign_packing_bit_order():
     b = np.zeros((1, 16), dtype=np.uint8)
     b[0, 0] = 1
@@ -476,6 +493,27 @@ def test_merge_special_cases():
     out, l4 = O.merge_attention(o, far)
     np.testing.assert_array_equal(out, o[1])
     np.testing.assert_array_equal(l4, far[1])
+
+
+def test_merge_is_order_free_and_composes():
+    """Merging parts in any order, or merging merged groups with their log-partitions,
+    gives the merge of all parts (R15); shifting every logit by c shifts lse by c."""
+    rng = np.random.default_rng(24)
+    o = rng.standard_normal((5, 3, 8))
+    ls = rng.standard_normal((5, 3)) * 3
+    ls[2, 1] = -np.inf
+    out, lse = O.merge_attention(o, ls)
+    perm = [3, 0, 4, 2, 1]
+    out_p, lse_p = O.merge_attention(o[perm], ls[perm])
+    np.testing.assert_allclose(out_p, out, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(lse_p, lse, rtol=1e-13)
+    a_out, a_lse = O.merge_attention(o[:2], ls[:2])
+    b_out, b_lse = O.merge_attention(o[2:], ls[2:])
+    out2, lse2 = O.merge_attention(np.stack([a_out, b_out]), np.stack([a_lse, b_lse]))
+    np.testing.assert_allclose(out2, out, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(lse2, lse, rtol=1e-13)
+    s = rng.standard_normal((4, 50))
+    np.testing.assert_allclose(O.log_partition(s + 7.5), O.log_partition(s) + 7.5, rtol=1e-14)
 
 
 def test_split_decode_of_a_packed_cache_equals_whole_decode():
