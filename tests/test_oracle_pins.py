@@ -359,7 +359,7 @@ def test_value_quant_hand_example():
     np.testing.assert_allclose(O.dequantize_values(out, 2, 32)[0, :5], [0, 1, 2, 3, 1])
 
 
-@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("bits", [2, 3, 4])
 def test_value_quant_roundtrip_bound(bits):
     rng = np.random.default_rng(4)
     v = rng.standard_normal((500, 128))
@@ -370,6 +370,20 @@ def test_value_quant_roundtrip_bound(bits):
     bound = scale / 2 + 2.0 ** -11 * (np.abs(np.repeat(out["min"], 32, axis=1))
                                       + (2 ** bits - 1) * scale) + 1e-12
     assert np.all(np.abs(vh - v) <= bound)
+
+
+def test_value_quant_three_bit_hand_example():
+    """Values 0..7 (then 3.4) in one group: scale 1, min 0, codes equal to the values (3.4
+    rounds to 3); the 3-bit codes straddle bytes in the LSB-first stream (R8, R10)."""
+    v = np.zeros((1, 32))
+    v[0, :8] = np.arange(8)
+    v[0, 8:] = 3.4
+    out = O.quantize_values(v, 3, with_diagnostics=True)
+    assert list(out["code_values"][0, :9]) == [0, 1, 2, 3, 4, 5, 6, 7, 3]
+    scale, lo = np.asarray(out["params"][0, 0]).view(np.float16).astype(np.float64)
+    assert scale == 1.0 and lo == 0.0
+    # codes 0..7 packed LSB-first: 0b 111 110 101 100 011 010 001 000 = 0xFAC688 (little-endian bytes)
+    assert out["codes"][0, :3].tobytes() == bytes([0x88, 0xC6, 0xFA])
 
 
 def test_value_quant_constant_group():
