@@ -158,7 +158,8 @@ class Context:
                  rotation: str = "hadamard", hadamard_signs=None, haar=None, v_group: int = 32,
                  stream=None):
         self.d, self.lm_bits, self.v_bits, self.v_group = d, k_lm_bits, v_bits, v_group
-        S = np.ascontiguousarray(qjl_S, dtype=np.float32)
+        # qjl_S None (or an empty [0, d] array): keys without the QJL stage, m = 0
+        S = np.zeros((0, d), np.float32) if qjl_S is None else np.ascontiguousarray(qjl_S, dtype=np.float32)
         self.m = S.shape[0]
         c = np.ascontiguousarray(centroids, dtype=np.float32)
         t = np.ascontiguousarray(boundaries, dtype=np.float32)
