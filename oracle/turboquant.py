@@ -318,17 +318,30 @@ def _fp16_bits(x) -> np.ndarray:
 
 
 def fp16_midpoint_distance(x) -> np.ndarray:
-    """Relative distance of |x| to the nearest fp16 rounding midpoint (for exemptions)."""
+    """Relative distance of |x| to the nearest fp16 rounding midpoint (for exemptions).
+
+    The fp16 values lo <= |x| < hi bracket |x|; the midpoints that can be nearest are the
+    one of (lo, hi) and, when |x| is itself an fp16 value at the bottom of a binade, the one
+    below lo, half of the smaller gap beneath it. Past the largest finite value 65504 the
+    next grid point is 65536, so the overflow threshold 65520 is the last midpoint.
+    """
     x = np.abs(np.asarray(x, dtype=np.float64))
-    h = x.astype(np.float16)
+    with np.errstate(over="ignore"):
+        h = x.astype(np.float16)
     hb = h.view(np.uint16).astype(np.int64)
     lo = np.where(h.astype(np.float64) > x, hb - 1, hb)
     lo = np.clip(lo, 0, 0x7BFF)
-    lo_v = lo.astype(np.uint16).view(np.float16).astype(np.float64)
-    hi_v = (lo + 1).astype(np.uint16).view(np.float16).astype(np.float64)
-    mid = 0.5 * (lo_v + hi_v)
+
+    def val(bits):
+        v = np.clip(bits, 0, 0x7BFF).astype(np.uint16).view(np.float16).astype(np.float64)
+        return np.where(bits > 0x7BFF, 65536.0, v)
+
+    lo_v = val(lo)
+    mid_up = 0.5 * (lo_v + val(lo + 1))
+    mid_dn = np.where(lo > 0, 0.5 * (lo_v + val(lo - 1)), -np.inf)
+    dist = np.minimum(np.abs(x - mid_up), np.abs(x - mid_dn))
     with np.errstate(divide="ignore", invalid="ignore"):
-        rel = np.abs(x - mid) / np.where(x > 0, x, 1.0)
+        rel = dist / np.where(x > 0, x, 1.0)
     return np.where(x > 0, rel, np.inf)
 
 

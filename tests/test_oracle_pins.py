@@ -248,7 +248,43 @@ def test_record_sizes_and_skill_card_size_figure():
 
 def test_fp16_midpoint_distance():
     assert O.fp16_midpoint_distance(np.array([1.0 + 2.0 ** -11]))[0] == 0.0
-    assert O.fp16_midpoint_distance(np.array([1.0]))[0] == pytest.approx(2.0 ** -11, rel=1e-12)
+    # 1.0 opens a binade: the gap below it (2^-11) is half the gap above, so the nearest
+    # midpoint is 1 - 2^-12; inside a binade both midpoints are half a gap away
+    assert O.fp16_midpoint_distance(np.array([1.0]))[0] == pytest.approx(2.0 ** -12, rel=1e-12)
+    assert O.fp16_midpoint_distance(np.array([1.5]))[0] == pytest.approx(2.0 ** -11 / 1.5, rel=1e-12)
+
+
+def _half_grid_from_fields():
+    """Every finite non-negative IEEE binary16 value in ascending order, built from the
+    format's fields (exponent e, 10-bit fraction f) without any float16 conversion:
+    e = 0 gives the subnormals f * 2^-24, e = 1..30 the normals (1024 + f) * 2^(e - 25)."""
+    vals = [f * 2.0 ** -24 for f in range(1024)]
+    for e in range(1, 31):
+        vals += [(1024 + f) * 2.0 ** (e - 25) for f in range(1024)]
+    return np.array(vals)
+
+
+def test_fp16_midpoint_distance_exhaustive_walk():
+    """Every pair of consecutive fp16 values, subnormal range and all 30 normal exponents:
+    the midpoint of the pair is at distance exactly 0; the pair's lower end, and points a
+    quarter gap either side of the midpoint, are at the distances the gap fixes."""
+    g = _half_grid_from_fields()
+    assert g.size == 31 * 1024 and g[-1] == 65504.0 and np.all(np.diff(g) > 0)
+    lo, hi = g[:-1], g[1:]
+    gap = hi - lo
+    mid = lo + gap / 2                                   # exact in fp64
+    assert np.all(O.fp16_midpoint_distance(mid) == 0.0)
+    pos = lo > 0
+    # a representable value sits half a gap from the midpoints around it; the nearer one
+    # is the lower midpoint at an exponent step (the gap below is half the gap above)
+    gap_below = np.concatenate([[np.inf], gap[:-1]])
+    d_lo = O.fp16_midpoint_distance(lo[pos])
+    np.testing.assert_allclose(d_lo, np.minimum(gap[pos], gap_below[pos]) / 2 / lo[pos], rtol=1e-12)
+    for side in (-1.0, 1.0):
+        x = mid + side * gap / 4
+        np.testing.assert_allclose(O.fp16_midpoint_distance(x), (gap / 4) / x, rtol=1e-12)
+    # the overflow threshold between 65504 and the next grid point 65536
+    assert O.fp16_midpoint_distance(np.array([65520.0]))[0] == 0.0
 
 
 # ---------------------------------------------------------------- QJL
