@@ -130,7 +130,7 @@ const char* tq_last_error(void);
  * in fp64 to convergence and rounded to fp32. The skill card ("turboquant-
  * pytorch", "Что делает") builds these codebooks with scipy; this is a
  * self-contained solver. Writes 2^bits centroids and 2^bits - 1 boundaries.
- * d in [4, 4096], bits in [1, 4]; else TQ_EINVAL. */
+ * d in [4, 4096], bits in [1, 7]; else TQ_EINVAL. */
 tq_status tq_lloyd_max_codebook(int d, int bits, float* centroids, float* boundaries);
 
 /* HOST ONLY. Haar-distributed orthogonal matrix from a d x d row-major matrix
@@ -267,9 +267,11 @@ tq_status tq_check_device(const tq_ctx* ctx, void* stream);
  * bytes (32 MiB) inside this library; every GPU that loads the library holds one
  * until the process exits. A shape whose workspace (tq_decode_workspace_bytes)
  * exceeds it returns TQ_EUNSUPPORTED with the sizes in tq_last_error().
- * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current); make that first call before
- * any stream capture. All calls on a device share the one array and it keeps
+ * Every call looks up the array's device address in the current CUDA context
+ * (cudaGetSymbolAddress, with the context's device current; nothing is cached, so
+ * a context created after a device reset, or one the caller made current itself,
+ * is served its own copy). The first call in a context loads the library's device
+ * code there: make that first call before any stream capture. All calls on a device share the one array and it keeps
  * the last call's contents: every byte a call reads is written earlier in the
  * same call, but calls whose work overlaps on the GPU (different streams, or
  * host threads without ordering) race on it and must be serialized.

@@ -11,7 +11,6 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
-#include <mutex>
 
 #include "tq_internal.h"
 
@@ -23,10 +22,6 @@ namespace {
 // query heads (about 10 MB).
 constexpr size_t kStaticScratchBytes = size_t(32) << 20;
 static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
-
-constexpr int kMaxDevices = 64;
-std::mutex g_setup_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
 
 }  // namespace
 
@@ -55,7 +50,7 @@ tq_status tq_decode_attention_static(const tq_ctx* ctx, const void* q, tq_dtype 
     return TQ_EUNSUPPORTED;
   }
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
     tq::set_last_error("tq_decode_attention_static: no usable current device");
     return TQ_ECUDA;
   }
@@ -63,23 +58,21 @@ tq_status tq_decode_attention_static(const tq_ctx* ctx, const void* q, tq_dtype 
     tq::set_last_error("tq_decode_attention_static: the context belongs to another device");
     return TQ_EINVAL;
   }
+  // The host-side name of a __device__ array is not a device address, so ask the
+  // runtime for it, with the caller's device current. The address belongs to the
+  // module loaded in the current CUDA context; it is looked up on every call (a host
+  // table lookup once the module is loaded) rather than cached, so that a context
+  // created after a device reset, or a context the caller made current itself, gets
+  // its own copy's address. The first call in a context loads the module: make it
+  // before any stream capture.
   void* ptr = nullptr;
-  {
-    // One-time set-up per device, with that device current: the host-side name of
-    // a __device__ array is not a device address, so ask the runtime for it.
-    std::lock_guard<std::mutex> lock(g_setup_mutex);
-    ptr = g_scratch_ptr[dev];
-    if (!ptr) {
-      cudaError_t e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
-      if (e != cudaSuccess || !ptr) {
-        char msg[256];
-        std::snprintf(msg, sizeof(msg), "tq_decode_attention_static: cudaGetSymbolAddress failed: %s",
-                      cudaGetErrorString(e));
-        tq::set_last_error(msg);
-        return TQ_ECUDA;
-      }
-      g_scratch_ptr[dev] = ptr;
-    }
+  const cudaError_t e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
+  if (e != cudaSuccess || !ptr) {
+    char msg[256];
+    std::snprintf(msg, sizeof(msg), "tq_decode_attention_static: cudaGetSymbolAddress failed: %s",
+                  cudaGetErrorString(e));
+    tq::set_last_error(msg);
+    return TQ_ECUDA;
   }
   // Everything the kernels read from the scratch is written earlier in the same
   // call (prepared queries, then every split-K partial), so nothing needs clearing.

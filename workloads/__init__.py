@@ -126,13 +126,14 @@ def method_draws(d: int, m: int, seed: int = 1234) -> dict:
       Walsh-Hadamard rotation (int8, +-1);
     * ``haar_gaussian``: a d x d matrix of i.i.d. N(0,1) (fp64) from which each
       side builds its own Haar-distributed orthogonal matrix;
-    * ``qjl_S``: the m x d QJL projection, i.i.d. N(0,1) draws kept at fp16
-      precision (fp64 array holding fp16-representable values).
+    * ``qjl_S``: the m x d QJL projection, i.i.d. N(0,1) draws in fp32 (an fp64
+      array holding the fp32 values: the library takes S as fp32, so both sides
+      see exactly the same matrix).
     """
     rng = np.random.default_rng([seed, d, m])
     signs = np.where(rng.integers(0, 2, size=d) == 1, 1, -1).astype(np.int8)
     haar_gaussian = rng.standard_normal((d, d))
-    S = fp16_round(rng.standard_normal((m, d)))
+    S = rng.standard_normal((m, d), dtype=np.float32).astype(np.float64)
     return {"hadamard_signs": signs, "haar_gaussian": haar_gaussian, "qjl_S": S}
 
 
