@@ -60,6 +60,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-paged", action="store_true", help="skip the paged-cache timings")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the kernel timings of the other workloads (the `configs` object)")
+    ap.add_argument("--config-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--sweep", action="store_true",
@@ -88,7 +91,7 @@ def source_sha(names):
     return h.hexdigest()[:16]
 
 
-DECODE_SOURCES = ("decode_mma.cu", "decode.cu", "tq_device.cuh", "tq_sm100.cuh", "tq_internal.h")
+DECODE_SOURCES = ("decode_tc.cu", "decode_mma.cu", "decode.cu", "tq_device.cuh", "tq_sm100.cuh", "tq_internal.h")
 COMPRESS_SOURCES = ("compress.cu", "tq_device.cuh", "tq_sm100.cuh", "tq_internal.h")
 
 
@@ -266,7 +269,10 @@ def run_reference(args, w: W.Workload):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * (dec_s + comp_s) / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "batch": w.batch, "kv_heads": w.hkv, "q_heads": w.hq,
-                   "tokens": w.tokens, "head_dim": w.d, "k_bits": w.k_bits, "v_bits": w.v_bits},
+                   "tokens": w.tokens, "head_dim": w.d, "k_bits": w.k_bits, "v_bits": w.v_bits,
+                   "rotation": w.rotation, "packed_bytes": w.packed_bytes(),
+                   "l2": "flushed before each timed phase: 256 MiB write, then 256 MiB read",
+                   "parallelism": f"dp{args.gpus} (independent replicas)"},
         "compress": {"value": 2 * units * w.tokens / comp_s, "unit": "vectors/s"},
         "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": res[0]["cores"], "kind": "oracle",
                          "sample": sample},
@@ -276,6 +282,66 @@ def run_reference(args, w: W.Workload):
 
 
 # ---------------------------------------------------------------------- GPU arm
+
+SIDE_WORKLOADS = ("single_head_d128_n4096", "qwen2.5-3b_8k_k3v2", "long_1m_k4v4")
+
+
+def time_side_workload(T, torch, w: W.Workload, steps: int, warmup: int, dev, flush_l2, peak: float):
+    """Kernel times of one compression call and one decode call of workload `w` (inputs
+    drawn by its recipe; L2 flushed before every timed launch; CUDA events around the main
+    kernel of each call, recorded by the library on the launching stream)."""
+    dr = W.method_draws(w.d, w.m)
+    c, t = T.tq_lloyd_max_codebook(w.d, w.lm_bits)
+    ctx = T.tq_codebook_load(w.d, w.lm_bits, w.v_bits, c, t, dr["qjl_S"], hadamard_signs=dr["hadamard_signs"])
+    n_vec = w.units * w.tokens
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    if w.name.startswith("single_head"):
+        Kh, Vh, Qh = W.single_head_kvq(w.tokens, w.d, w.hq)
+        K, V = torch.from_numpy(Kh).to(dev).to(tdt), torch.from_numpy(Vh).to(dev).to(tdt)
+        Q = torch.from_numpy(Qh).to(dev).to(tdt).view(w.batch, w.hq, w.d)
+    else:
+        if w.name.startswith("qwen"):
+            Kh, Vh, _ = host_inputs(w, 0)
+            K, V = torch.from_numpy(Kh).to(dev).to(tdt), torch.from_numpy(Vh).to(dev).to(tdt)
+            del Kh, Vh
+        else:
+            K = W.device_normal((n_vec, w.d), seed=3000, device=dev).to(tdt)
+            V = W.device_normal((n_vec, w.d), seed=4000, device=dev).to(tdt)
+        Q = torch.from_numpy(W.queries((w.batch, w.hq, w.d), seed=7, dtype=w.dtype)).to(dev).to(tdt)
+    packed = T.tq_compress_kv(ctx, K, V)
+    out = torch.empty((w.batch, w.hq, w.d), dtype=torch.float32, device=dev)
+    ws = torch.empty(T.tq_decode_workspace_bytes(ctx, w.batch, w.hq, w.hkv, w.tokens), dtype=torch.uint8,
+                     device=dev)
+    E = torch.cuda.Event
+    comp, dec = [], []
+    for it in range(warmup + steps):
+        e = [E(enable_timing=True) for _ in range(4)]
+        for ev in e:
+            ev.record()
+        flush_l2()
+        T.tq_set_profile_events(ctx, e[0], e[1])
+        T.tq_compress_kv(ctx, K, V, **packed)
+        flush_l2()
+        T.tq_set_profile_events(ctx, e[2], e[3])
+        T.tq_decode_attention(ctx, Q, packed, w.batch, w.hq, w.hkv, w.tokens, out=out, workspace=ws)
+        T.tq_set_profile_events(ctx, None, None)
+        if it >= warmup:
+            comp.append(e)
+    torch.cuda.synchronize()
+    T.tq_check_device(ctx)
+    ck = statistics.median(e[0].elapsed_time(e[1]) for e in comp) / 1e3
+    dk = statistics.median(e[2].elapsed_time(e[3]) for e in comp) / 1e3
+    packed_bytes = w.packed_bytes()
+    comp_bytes = 2 * n_vec * w.d * (2 if w.dtype == "bf16" else 4) + packed_bytes
+    ctx.close()
+    return {"batch": w.batch, "kv_heads": w.hkv, "q_heads": w.hq, "tokens": w.tokens, "k_bits": w.k_bits,
+            "v_bits": w.v_bits, "dtype": w.dtype, "packed_bytes": packed_bytes, "steps": steps,
+            "compress_kernel_us": ck * 1e6, "compress_vectors_per_s": 2 * n_vec / ck,
+            "compress_gbs": comp_bytes / ck / 1e9, "compress_frac": comp_bytes / ck / 1e9 / peak,
+            "decode_kernel_us": dk * 1e6, "decode_gbs": packed_bytes / dk / 1e9,
+            "decode_frac": packed_bytes / dk / 1e9 / peak,
+            "timing": "median over steps of CUDA events around each call's main kernel, L2 flushed before each"}
+
 
 def run_ours(args, w: W.Workload):
     import torch
@@ -496,6 +562,17 @@ def run_ours(args, w: W.Workload):
     # our kernels per step: compress (1) + decode (query prep + attention + combine)
     launches_per_step = (0 if args.decode_only else 1) + 3
 
+    side = None
+    if rank == 0 and world == 1 and not args.no_configs and not args.decode_only:
+        peak, _ = measured_peaks()
+        side = {}
+        for name in SIDE_WORKLOADS:
+            if name == w.name:
+                continue
+            side[name] = time_side_workload(T, torch, W.WORKLOADS[name], args.config_steps, 3, dev, flush_l2, peak)
+            log(f"config {name}: compress {side[name]['compress_kernel_us']:.1f} us, "
+                f"decode {side[name]['decode_kernel_us']:.1f} us ({side[name]['decode_gbs']:.0f} GB/s)")
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         Kh2, Vh2, _ = host_inputs(w, 0) if w.name.startswith("qwen") else (None, None, None)
@@ -509,9 +586,10 @@ def run_ours(args, w: W.Workload):
         peak, peak_kind = measured_peaks()
         dsha = source_sha(DECODE_SOURCES)
         units_dec = w.units * w.tokens  # (token, KV head) pairs
-        # the tensor-core decode serves d = m = 128, 1- or 2-bit Lloyd-Max codes, G <= 8
-        dkern = "decode_mma_kernel" if (w.d == 128 and w.m == 128 and w.lm_bits <= 2 and w.group <= 8) \
-            else "decode_kernel"
+        # the tcgen05 decode serves d = 128, m in {0, 128}, 1- to 3-bit Lloyd-Max codes (symmetric
+        # codebook), 2- or 4-bit values, G <= 8
+        dkern = "decode_tc_kernel" if (w.d == 128 and w.m in (0, 128) and w.lm_bits <= 3 and w.group <= 8
+                                       and w.v_bits in (2, 4)) else "decode_kernel"
         roof_dec = {"kernel": dkern, "bound": "hbm", "achieved": packed_bytes / dec_k_mean / 1e9,
                     "peak": peak, "unit": "GB/s", "frac": packed_bytes / dec_k_mean / 1e9 / peak,
                     "peak_kind": peak_kind, "alg_bytes_per_launch": packed_bytes,
@@ -555,6 +633,7 @@ def run_ours(args, w: W.Workload):
             "paged": paged_line,
             "roofline": roof,
             "roofline_decode": roof_dec,
+            "configs": side,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,

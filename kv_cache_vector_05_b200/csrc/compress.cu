@@ -11,7 +11,9 @@
 #include <cuda.h>  // CUtensorMap and its enums (types only: the encoder is fetched at run time)
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstring>
+#include <vector>
 
 #include "tq_device.cuh"
 #include "tq_sm100.cuh"
@@ -240,8 +242,9 @@ cudaError_t launch_d(const tq_ctx* ctx, const CompressArgs& a, int dtype, cudaSt
 // one 128 x 128 x 128 MMA on the 5th-generation tensor cores. Warps 0-3 rotate and
 // quantize the keys (one key per warp step, as above) and write the residuals,
 // scaled by 16 and split into f16 hi + lo, to two swizzled shared-memory operand
-// tiles; one thread issues 2 x 8 tcgen05.mma (hi and lo against the f16 matrix S,
-// which is exact in f16) into a 128 x 128 fp32 accumulator in tensor memory; after
+// tiles; one thread issues 3 x 8 tcgen05.mma (residual hi and lo against S hi, residual
+// hi against S lo, S being split in two f16 terms like the residual) into a 128 x 128
+// fp32 accumulator in tensor memory; after
 // the commit barrier each thread reads its key's 128 projections back and packs the
 // sign bits. Warps 4-7 group-quantize the values of the same tile meanwhile.
 constexpr int kTcRows = 128;
@@ -249,8 +252,8 @@ constexpr int kTcThreads = 256;
 constexpr uint32_t kTcTileBytes = kTcRows * 128 * 2;  // one f16 operand tile, 32 KB
 
 struct TcSmem {
-  static constexpr uint32_t A_HI = 0, A_LO = kTcTileBytes, S = 2 * kTcTileBytes;
-  static constexpr uint32_t RBUF = 3 * kTcTileBytes;         // [4 warps][128] fp32
+  static constexpr uint32_t A_HI = 0, A_LO = kTcTileBytes, S = 2 * kTcTileBytes;  // S: hi tile, then lo tile
+  static constexpr uint32_t RBUF = 4 * kTcTileBytes;         // [4 warps][128] fp32
   static constexpr uint32_t ZF = RBUF + 4 * 128 * 4;         // [128] nonzero flags
   static constexpr uint32_t BAR = ZF + 128;                  // mbarrier
   static constexpr uint32_t TMEM = BAR + 8;                  // TMEM base address
@@ -269,7 +272,7 @@ __device__ __forceinline__ bool kwarps_sync_or(bool v) {
 }
 
 template <typename T, int LMB, int VB>
-__global__ void __launch_bounds__(kTcThreads, 2) compress_tc_kernel(const __grid_constant__ CompressArgs a) {
+__global__ void __launch_bounds__(kTcThreads, 1) compress_tc_kernel(const __grid_constant__ CompressArgs a) {
   namespace s1 = tq::sm100;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -288,10 +291,10 @@ __global__ void __launch_bounds__(kTcThreads, 2) compress_tc_kernel(const __grid
     s1::mbar_init(bar, 1);
     s1::mbar_init_fence();
   }
-  {  // S operand tile, prepacked on the host
+  {  // S operand tiles (hi, lo), prepacked on the host
     const uint4* src = reinterpret_cast<const uint4*>(a.S_sw128);
     uint4* dst = reinterpret_cast<uint4*>(sm + TcSmem::S);
-    for (int w = tid; w < (int)(kTcTileBytes / 16); w += kTcThreads) dst[w] = src[w];
+    for (int w = tid; w < (int)(2 * kTcTileBytes / 16); w += kTcThreads) dst[w] = src[w];
   }
   s1::fence_async_smem();
   s1::fence_before_sync();
@@ -345,6 +348,10 @@ __global__ void __launch_bounds__(kTcThreads, 2) compress_tc_kernel(const __grid
           for (int ks = 0; ks < 8; ++ks)
             s1::umma_f16(tmem, s1::sw128_desc(sbase + TcSmem::A_LO, 16 * ks, kTcRows),
                          s1::sw128_desc(sbase + TcSmem::S, 16 * ks, 128), idesc, 1u);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            s1::umma_f16(tmem, s1::sw128_desc(sbase + TcSmem::A_HI, 16 * ks, kTcRows),
+                         s1::sw128_desc(sbase + TcSmem::S + kTcTileBytes, 16 * ks, 128), idesc, 1u);
           s1::umma_commit(bar);
         }
         const bool ok = s1::mbar_wait(bar, phase);
@@ -407,7 +414,7 @@ cudaError_t launch_tc_t(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s
     configured = true;
   }
   int64_t blocks = (a.n_vec + kTcRows - 1) / kTcRows;
-  if (blocks > 2LL * ctx->num_sms) blocks = 2LL * ctx->num_sms;
+  if (blocks > ctx->num_sms) blocks = ctx->num_sms;
   if (ctx->prof_start) cudaEventRecord(ctx->prof_start, s);
   compress_tc_kernel<T, LMB, VB><<<(unsigned)blocks, kTcThreads, smem, s>>>(a);
   cudaError_t e = cudaGetLastError();
@@ -425,7 +432,7 @@ cudaError_t launch_tc(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) 
 
 
 // ---------------------------------------------------------------------------------
-// Fast path (d = m = 128, randomized Hadamard rotation, S exact in f16): four lanes
+// Fast path (d = m = 128, randomized Hadamard rotation): four lanes
 // per vector, lane q of a vector holding coordinates [32q, 32q + 32). Norm, sign flip,
 // the first five Walsh-Hadamard stages, bucketize, residual and code packing are
 // lane-local; the last two butterfly stages and the two norms take two shuffles
@@ -439,8 +446,8 @@ constexpr int kQ4Rows = 128;
 constexpr int kQ4Threads = 4 * kQ4Rows;
 
 struct Q4Smem {
-  static constexpr uint32_t A_HI = 0, A_LO = kTcTileBytes, S = 2 * kTcTileBytes;
-  static constexpr uint32_t ZF = 3 * kTcTileBytes;  // [128] nonzero-key flags
+  static constexpr uint32_t A_HI = 0, A_LO = kTcTileBytes, S = 2 * kTcTileBytes;  // S: hi tile, then lo tile
+  static constexpr uint32_t ZF = 4 * kTcTileBytes;  // [128] nonzero-key flags
   static constexpr uint32_t BAR = ZF + 128;         // mbarrier
   static constexpr uint32_t TMEM = BAR + 8;         // TMEM base address
   static constexpr uint32_t BYTES = TMEM + 8;
@@ -527,7 +534,7 @@ __global__ void __launch_bounds__(kQ4Threads, 1) compress_q4_kernel(const __grid
   if (a.k) {  // S operand tile, prepacked on the host
     const uint4* src = reinterpret_cast<const uint4*>(a.S_sw128);
     uint4* dst = reinterpret_cast<uint4*>(sm + Q4Smem::S);
-    for (int w = tid; w < (int)(kTcTileBytes / 16); w += kQ4Threads) dst[w] = src[w];
+    for (int w = tid; w < (int)(2 * kTcTileBytes / 16); w += kQ4Threads) dst[w] = src[w];
   }
   s1::fence_async_smem();
   s1::fence_before_sync();
@@ -656,6 +663,10 @@ __global__ void __launch_bounds__(kQ4Threads, 1) compress_q4_kernel(const __grid
         for (int ks = 0; ks < 8; ++ks)
           s1::umma_f16(tmem, s1::sw128_desc(sbase + Q4Smem::A_LO, 16 * ks, kQ4Rows),
                        s1::sw128_desc(sbase + Q4Smem::S, 16 * ks, 128), idesc, 1u);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          s1::umma_f16(tmem, s1::sw128_desc(sbase + Q4Smem::A_HI, 16 * ks, kQ4Rows),
+                       s1::sw128_desc(sbase + Q4Smem::S + kTcTileBytes, 16 * ks, 128), idesc, 1u);
         s1::umma_commit(bar);
       }
     }
@@ -805,11 +816,10 @@ struct RotSmem {
   static constexpr uint32_t NT = HAAR ? 3 : 1;               // bf16 terms of the rotation
   static constexpr uint32_t KT = 0;                          // keys, bf16 operand tile
   static constexpr uint32_t HB = kTcTileBytes;               // rotation, NT bf16 operand tiles
-  static constexpr uint32_t A_HI = (1 + NT) * kTcTileBytes, A_LO = (2 + NT) * kTcTileBytes;  // residual x16
-  static constexpr uint32_t S = (3 + NT) * kTcTileBytes;     // QJL matrix, f16 operand tile
-  static constexpr uint32_t KR = (4 + NT) * kTcTileBytes;    // Hadamard: next pass's raw key rows
-  static constexpr uint32_t VR = (5 + NT) * kTcTileBytes;    // Hadamard: next pass's raw value rows
-  static constexpr uint32_t XS = (HAAR ? 4 + NT : 6 + NT) * kTcTileBytes;  // [2][128] half-row sums
+  static constexpr uint32_t S = (1 + NT) * kTcTileBytes;     // QJL matrix, f16 hi and lo operand tiles
+  static constexpr uint32_t KR = (3 + NT) * kTcTileBytes;    // Hadamard: next pass's raw key rows
+  static constexpr uint32_t VR = (4 + NT) * kTcTileBytes;    // Hadamard: next pass's raw value rows
+  static constexpr uint32_t XS = (HAAR ? 3 + NT : 5 + NT) * kTcTileBytes;  // [2][128] half-row sums
   static constexpr uint32_t ZF = XS + 2 * 128 * 4;           // [128] nonzero-key flags
   static constexpr uint32_t BAR = ZF + 128;                  // four mbarriers
   static constexpr uint32_t TMEM = BAR + 32;                 // TMEM base address
@@ -846,7 +856,7 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
   const int R = 32 * sp + lane;                    // key warps: row = key within the pass
 
   if (warp == 0) {
-    s1::tmem_alloc(tmem_s, 256);
+    s1::tmem_alloc(tmem_s, 512);
     s1::tmem_relinquish();
   }
   if (tid == 0) {
@@ -861,7 +871,7 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
     const uint4* ssrc = reinterpret_cast<const uint4*>(a.S_sw128);
     uint4* hdst = reinterpret_cast<uint4*>(sm + RS::HB);
     uint4* sdst = reinterpret_cast<uint4*>(sm + RS::S);
-    for (int w = tid; w < (int)(kTcTileBytes / 16); w += kRotThreads) sdst[w] = ssrc[w];
+    for (int w = tid; w < (int)(2 * kTcTileBytes / 16); w += kRotThreads) sdst[w] = ssrc[w];
     for (int w = tid; w < (int)(RS::NT * kTcTileBytes / 16); w += kRotThreads) hdst[w] = hsrc[w];
   }
   s1::fence_async_smem();
@@ -869,7 +879,9 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
   __syncthreads();
   s1::fence_after_sync();
   const uint32_t tmem = *tmem_s;
-  const uint32_t tmem_y = tmem, tmem_p = tmem + 128;  // columns 0..127: Y, 128..255: S r
+  // columns 0..127: Y, 128..255: S r, 256..383: the residual operand (hi: 64 columns of
+  // f16 pairs, then lo)
+  const uint32_t tmem_y = tmem, tmem_p = tmem + 128, tmem_a = tmem + 256;
   const uint32_t lane_base = (uint32_t)(32 * sp) << 16;
   float cb_t[(1 << LMB) - 1], cb_c[1 << LMB];
 #pragma unroll
@@ -1005,22 +1017,23 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
 #pragma unroll
           for (int w = 0; w < CW; ++w) co[w] = nz ? (cw[w] | cw2[w]) : 0u;
         }
-        // residual x16 as f16 hi + lo (the previous projection finished: it was waited for)
+        // residual x16 as f16 hi + lo into tensor memory, row R, one f16 pair per column
+        // (the previous projection finished: it was waited for)
 #pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
-          uint32_t hw[4], lw[4];
+        for (int c16 = 0; c16 < 2; ++c16) {
+          uint32_t hw[8], lw[8];
 #pragma unroll
-          for (int p = 0; p < 4; ++p) {
-            const float f0 = use ? 16.f * r[8 * c8 + 2 * p] : 0.f, f1 = use ? 16.f * r[8 * c8 + 2 * p + 1] : 0.f;
+          for (int p = 0; p < 8; ++p) {
+            const float f0 = use ? 16.f * r[16 * c16 + 2 * p] : 0.f, f1 = use ? 16.f * r[16 * c16 + 2 * p + 1] : 0.f;
             const __half2 hh = __floats2half2_rn(f0, f1);
             const float2 hf = __half22float2(hh);
             const __half2 ll = __floats2half2_rn(f0 - hf.x, f1 - hf.y);
             hw[p] = *reinterpret_cast<const uint32_t*>(&hh);
             lw[p] = *reinterpret_cast<const uint32_t*>(&ll);
           }
-          const uint32_t off = s1::sw128_offset(R, 64 * ch + 32 * h + 8 * c8, kQ4Rows);
-          *reinterpret_cast<uint4*>(sm + RS::A_HI + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          *reinterpret_cast<uint4*>(sm + RS::A_LO + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+          const uint32_t col = 32 * ch + 16 * h + 8 * c16;  // coordinates 2 col .. 2 col + 15
+          s1::tmem_st8(tmem_a + lane_base + col, hw);
+          s1::tmem_st8(tmem_a + 64 + lane_base + col, lw);
         }
       }
       xs[ch * 128 + R] = (r4[0] + r4[1]) + (r4[2] + r4[3]);
@@ -1033,20 +1046,25 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
         reinterpret_cast<uint32_t*>(a.k_norms)[o] = nz ? (nb | (gb << 16)) : 0u;
       }
       if (ch == 0) zf[R] = use ? 1 : 0;
-      s1::fence_async_smem();
+      s1::tmem_st_wait();
       s1::fence_before_sync();
       key_warps_sync();
       s1::fence_after_sync();
       if (tid == 0) {
+        // S r = (A_hi + A_lo) S_hi^T + A_hi S_lo^T, A from tensor memory (the A_lo S_lo
+        // term, about 2^-22 of the product, is left out)
         constexpr uint32_t idesc = s1::idesc_f16_f32(128, 128);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          s1::umma_f16(tmem_p, s1::sw128_desc(sbase + RS::A_HI, 16 * ks, kQ4Rows),
-                       s1::sw128_desc(sbase + RS::S, 16 * ks, 128), idesc, ks > 0 ? 1u : 0u);
+          s1::umma_f16_ts(tmem_p, tmem_a + 8 * ks, s1::sw128_desc(sbase + RS::S, 16 * ks, 128), idesc,
+                          ks > 0 ? 1u : 0u);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          s1::umma_f16(tmem_p, s1::sw128_desc(sbase + RS::A_LO, 16 * ks, kQ4Rows),
-                       s1::sw128_desc(sbase + RS::S, 16 * ks, 128), idesc, 1u);
+          s1::umma_f16_ts(tmem_p, tmem_a + 64 + 8 * ks, s1::sw128_desc(sbase + RS::S, 16 * ks, 128), idesc, 1u);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          s1::umma_f16_ts(tmem_p, tmem_a + 8 * ks, s1::sw128_desc(sbase + RS::S + kTcTileBytes, 16 * ks, 128),
+                          idesc, 1u);
         s1::umma_commit(bar2);
       }
       // ---- QJL signs of this thread's 64 projections
@@ -1169,7 +1187,7 @@ __global__ void __launch_bounds__(kRotThreads, 1) compress_rot_kernel(const __gr
   __syncthreads();
   if (warp == 0) {
     s1::fence_after_sync();
-    s1::tmem_dealloc(tmem, 256);
+    s1::tmem_dealloc(tmem, 512);
   }
 }
 
@@ -1227,10 +1245,10 @@ constexpr int kPipeThreads = 640;  // warps 0-7 keys, 8-15 values, 16 producer (
 struct PipeSmem {
   static constexpr uint32_t KT = 0;                         // [2] key operand tiles (TMA, 128B swizzle)
   static constexpr uint32_t HB = 2 * kTcTileBytes;          // H diag(sigma), bf16 operand tile
-  static constexpr uint32_t S = 3 * kTcTileBytes;           // QJL matrix, f16 operand tile
-  static constexpr uint32_t VR = 4 * kTcTileBytes;          // [2 passes][2 halves] value rows (2 panels each)
-  static constexpr uint32_t XR = 6 * kTcTileBytes;          // [2 passes][2 halves][128] sums of r^2
-  static constexpr uint32_t BAR = XR + 2 * 2 * 128 * 4;     // eleven mbarriers
+  static constexpr uint32_t S = 3 * kTcTileBytes;           // QJL matrix, f16 hi and lo operand tiles
+  static constexpr uint32_t VR = 5 * kTcTileBytes;          // [2 passes][2 halves] value rows (2 panels each)
+  static constexpr uint32_t XR = 7 * kTcTileBytes;          // [2 passes][128] second-half sums of r^2
+  static constexpr uint32_t BAR = XR + 2 * 128 * 4;         // eleven mbarriers
   static constexpr uint32_t TMEM = BAR + 88;                // TMEM base address
   static constexpr uint32_t BYTES = TMEM + 8;
   static_assert(BYTES + 1024 <= 227 * 1024, "compress_pipe_kernel shared memory");
@@ -1305,6 +1323,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
     uint4* sdst = reinterpret_cast<uint4*>(sm + PS::S);
     for (int w = tid; w < (int)(kTcTileBytes / 16); w += kPipeThreads) {
       sdst[w] = ssrc[w];
+      sdst[w + kTcTileBytes / 16] = ssrc[w + kTcTileBytes / 16];
       hdst[w] = hsrc[w];
     }
   }
@@ -1422,7 +1441,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
             for (int w = 0; w < LMB; ++w) co[w] = nz ? (cw[w] | cw2[w]) : 0u;
           }
         }
-        xr[b * 256 + ch * 128 + R] = (ra.x + ra.y) + (rb.x + rb.y);
+        const float rsum = (ra.x + ra.y) + (rb.x + rb.y);  // this half's sum of r^2
+        if (ch == 1) xr[b * 128 + R] = rsum;
         // Y[b] read, S r read, operand written: hand the pass to the producer
         s1::tmem_st_wait();
         s1::fence_before_sync();
@@ -1431,7 +1451,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
         failed = s1::bar_sync_or<1, 256>(failed);
         if (failed) break;
         if (ch == 0 && o >= 0) {
-          const float gamma = sqrtf(xr[b * 256 + R] + xr[b * 256 + 128 + R]) * (1.f / 16.f);
+          const float gamma = sqrtf(rsum + xr[b * 128 + R]) * (1.f / 16.f);
           const uint32_t nb = __half_as_ushort(__float2half_rn(sqrtf(tot * (1.0f / 128.f))));
           const uint32_t gb = __half_as_ushort(__float2half_rn(gamma));
           reinterpret_cast<uint32_t*>(a.k_norms)[o] = nz ? (nb | (gb << 16)) : 0u;
@@ -1628,7 +1648,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
                      s1::sw128_desc(sbase + PS::HB, 16 * ks, 128), idesc, ks > 0 ? 1u : 0u);
       s1::umma_commit(rotd + b);
     };
-    auto projection = [&]() {  // S r = (A_hi + A_lo) S^T, A in tensor memory
+    auto projection = [&]() {  // S r = (A_hi + A_lo) S_hi^T + A_hi S_lo^T, A in tensor memory
       constexpr uint32_t idesc = s1::idesc_f16_f32(128, 128);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)
@@ -1638,6 +1658,10 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
       for (int ks = 0; ks < 8; ++ks)
         s1::umma_f16_ts(tmem + kTmP, tmem + kTmA + 64 + 8 * ks, s1::sw128_desc(sbase + PS::S, 16 * ks, 128), idesc,
                         1u);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        s1::umma_f16_ts(tmem + kTmP, tmem + kTmA + 8 * ks,
+                        s1::sw128_desc(sbase + PS::S + kTcTileBytes, 16 * ks, 128), idesc, 1u);
       s1::umma_commit(projd);
     };
     // Prologue: passes 0 and 1 loaded and rotated, pass 2's keys on their way.
@@ -1716,11 +1740,11 @@ EncodeTiledFn tensor_map_encoder() {
 
 // A tensor map of compress_pipe_kernel: [n_vec][128] bf16 rows, boxes of 64 columns x
 // box_rows rows (one 128-byte-swizzled panel each). False if it cannot be made.
-bool encode_rows_map(CUtensorMap* map, const void* k, int64_t n_vec, uint32_t box_rows) {
+bool encode_rows_map(CUtensorMap* map, const void* k, int64_t n_vec, uint32_t box_rows, int cols = 128) {
   const EncodeTiledFn enc = tensor_map_encoder();
   if (!enc || n_vec <= 0 || n_vec >= ((int64_t)1 << 31)) return false;
-  const cuuint64_t dims[2] = {128, (cuuint64_t)n_vec};
-  const cuuint64_t strides[1] = {128 * 2};
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)n_vec};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
   const cuuint32_t box[2] = {64, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(k), dims, strides, box, estr,
@@ -1764,18 +1788,425 @@ cudaError_t launch_pipe(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s
   return vb == 2 ? launch_pipe_t<3, 2>(ctx, a, s) : launch_pipe_t<3, 4>(ctx, a, s);
 }
 
+// ---------------------------------------------------------------------------------
+// bf16 keys at d = 64 or 256 on the tensor cores, with either rotation (the keys only; a
+// call with values runs them through the warp-per-vector kernel). The rotation R is held
+// as NT bf16 terms: H diag(sigma) (+-1, exact, NT = 1) or the Haar matrix split in three
+// terms (NT = 3, about 24 bits); Y = K R^T is exact in its products and accumulates in
+// fp32, then the key work is that of compress_rot_kernel, then S r = (A_hi + A_lo) S_hi^T +
+// A_hi S_lo^T with A, the residual x16 in f16 hi + lo, in tensor memory. 128 keys per pass,
+// one pass at a time; two threads per key (TMEM lane = key, each thread half of the
+// columns). The operand tiles (NW x NW, NW = 64 at d = 64, 128 at d = 256) are prepacked
+// on the host in the swizzled K-major layout: at d = 64 all of them stay in shared memory;
+// at d = 256 (12 or 20 tiles of 32 KB per pass) they stream from global memory (L2-resident)
+// through a ring of three slots, each refilled as soon as the MMAs that read it complete.
+constexpr int kDenseThreads = 288;  // warps 0-7 keys (lane quadrant w % 4, column half w / 4), warp 8 producer
+
+template <int D, int NT>
+struct DenseSmem {
+  static constexpr int NW = D == 256 ? 128 : 64;    // chunk width (N and K) of an operand tile
+  static constexpr int NCH = D / NW;                 // N chunks = K chunks
+  static constexpr uint32_t TILE = (uint32_t)NW * NW * 2;
+  static constexpr int NROT = NCH * NCH * NT;        // rotation tiles per pass
+  static constexpr int NOPS = NROT + NCH * NCH * 2;  // + S hi / lo tiles
+  static constexpr bool STREAM = D == 256;
+  static constexpr int SLOTS = STREAM ? 3 : NOPS;
+  static constexpr uint32_t KT = 0;                              // key tile [128][D] bf16, D/64 panels
+  static constexpr uint32_t OPS = (uint32_t)128 * D * 2;         // operand tiles (ring or resident)
+  static constexpr uint32_t XS = OPS + SLOTS * TILE;             // [2][128] half-row sums
+  static constexpr uint32_t ZF = XS + 2 * 128 * 4;               // [128] nonzero-key flags
+  static constexpr uint32_t BAR = ZF + 128;  // kfull, rotd, aready, projd, pdone, ofull[3], oempty[3], fin
+  static constexpr uint32_t TMEM = BAR + 8 * 12;
+  static constexpr uint32_t BYTES = TMEM + 8;
+  static_assert(BYTES + 1024 <= 227 * 1024, "compress_dense_kernel shared memory");
+};
+// Tensor memory: Y (then S r) at columns [0, D), the residual operand's hi at 256 and lo at
+// 256 + D/2 (one f16 pair per column).
+constexpr uint32_t kDnA = 256;
+
+__device__ __forceinline__ void dense_key_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(256) : "memory");
+}
+
+template <int D, int LMB, int NT>
+__global__ void __launch_bounds__(kDenseThreads, 1) compress_dense_kernel(const __grid_constant__ CompressArgs a,
+                                                                         const uint16_t* __restrict__ ops) {
+  using DS = DenseSmem<D, NT>;
+  namespace s1 = tq::sm100;
+  constexpr int NW = DS::NW, NCH = DS::NCH;
+  constexpr int HALF = D / 2;  // columns per thread
+  extern __shared__ unsigned char smem_dense[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>(((uintptr_t)smem_dense + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = s1::smem_u32(sm);
+  float* xs = reinterpret_cast<float*>(sm + DS::XS);
+  uint8_t* zf = sm + DS::ZF;
+  uint64_t* kfull = reinterpret_cast<uint64_t*>(sm + DS::BAR);  // key tile landed
+  uint64_t* rotd = kfull + 1;     // rotation MMAs done
+  uint64_t* aready = kfull + 2;   // key warps wrote the residual operand (8 arrivals)
+  uint64_t* projd = kfull + 3;    // projection MMAs done
+  uint64_t* pdone = kfull + 4;    // key warps read S r (8 arrivals)
+  uint64_t* ofull = kfull + 5;    // [3] operand slot landed
+  uint64_t* oempty = kfull + 8;   // [3] operand slot read by its MMAs
+  uint64_t* fin = kfull + 11;     // every MMA issued has completed
+  uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + DS::TMEM);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t ntile = (a.n_vec + 127) / 128, g = gridDim.x;
+
+  if (warp == 0) {
+    s1::tmem_alloc(tmem_s, 512);
+    s1::tmem_relinquish();
+  }
+  if (tid == 0) {
+    s1::mbar_init(kfull, 1);
+    s1::mbar_init(rotd, 1);
+    s1::mbar_init(aready, 8);
+    s1::mbar_init(projd, 1);
+    s1::mbar_init(pdone, 8);
+    s1::mbar_init(fin, 1);
+    for (int k = 0; k < 3; ++k) {
+      s1::mbar_init(ofull + k, 1);
+      s1::mbar_init(oempty + k, 1);
+    }
+    s1::mbar_init_fence();
+  }
+  if constexpr (!DS::STREAM) {  // every operand tile stays resident
+    const uint4* src = reinterpret_cast<const uint4*>(ops);
+    uint4* dst = reinterpret_cast<uint4*>(sm + DS::OPS);
+    for (int w = tid; w < (int)(DS::NOPS * DS::TILE / 16); w += kDenseThreads) dst[w] = src[w];
+  }
+  s1::fence_async_smem();
+  s1::fence_before_sync();
+  __syncthreads();
+  s1::fence_after_sync();
+  const uint32_t tmem = *tmem_s;
+  bool failed = false;
+
+  if (warp < 8) {
+    // ================================================================ keys
+    const int sp = warp & 3, ch = warp >> 2;
+    const int R = 32 * sp + lane;
+    const uint32_t lane_base = (uint32_t)(32 * sp) << 16;
+    float cb_t[(1 << LMB) - 1], cb_c[1 << LMB];
+#pragma unroll
+    for (int k = 0; k < (1 << LMB) - 1; ++k) cb_t[k] = a.cb.t[k];
+#pragma unroll
+    for (int k = 0; k < (1 << LMB); ++k) cb_c[k] = a.cb.c[k];
+    // ||Y|| = sqrt(d) ||k|| for H diag(sigma) (not normalised), ||k|| for Haar
+    const float ninv = NT == 1 ? rsqrtf((float)D) : 1.f;
+    int it = 0;
+    for (int64_t tile = blockIdx.x; tile < ntile; tile += g, ++it) {
+      const uint32_t ph = (uint32_t)it & 1u;
+      const int64_t i = tile * 128 + R;
+      const bool valid = i < a.n_vec;
+      const int64_t o = valid ? out_row(a, i) : -1;
+      if (!failed && !s1::mbar_wait(rotd, ph)) failed = true;
+      if (s1::bar_sync_or<1, 256>(failed)) {
+        failed = true;
+        break;
+      }
+      s1::fence_after_sync();
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+      for (int h = 0; h < HALF / 32; ++h) {
+        uint32_t v[32];
+        s1::tmem_ld32(tmem + lane_base + HALF * ch + 32 * h, v);
+        s1::tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float yv = __uint_as_float(v[e]);
+          s4[e & 3] = fmaf(yv, yv, s4[e & 3]);
+        }
+      }
+      xs[ch * 128 + R] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+      dense_key_sync();
+      const float tot = xs[R] + xs[128 + R];
+      dense_key_sync();
+      const bool nz = tot > 0.f;
+      const float sc = nz ? 1.0f / sqrtf(tot) : 0.f;
+      const bool use = valid && nz;
+      float r4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+      for (int h = 0; h < HALF / 32; ++h) {
+        uint32_t v[32];
+        s1::tmem_ld32(tmem + lane_base + HALF * ch + 32 * h, v);
+        s1::tmem_ld_wait();
+        uint32_t cw[LMB], cw2[LMB];
+#pragma unroll
+        for (int w = 0; w < LMB; ++w) cw[w] = cw2[w] = 0u;
+        float r[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float yy = __uint_as_float(v[e]) * sc;
+          uint32_t idx = 0;
+          float cv = cb_c[0];
+#pragma unroll
+          for (int k = 0; k < (1 << LMB) - 1; ++k) {
+            if (yy >= cb_t[k]) {
+              idx = k + 1;
+              cv = cb_c[k + 1];
+            }
+          }
+          if (e & 1)
+            put_bits<LMB, LMB>(cw2, LMB * e, idx);
+          else
+            put_bits<LMB, LMB>(cw, LMB * e, idx);
+          r[e] = yy - cv;
+          r4[e & 3] = fmaf(r[e], r[e], r4[e & 3]);
+        }
+        if (o >= 0) {
+          uint32_t* co = reinterpret_cast<uint32_t*>(a.k_codes + o * (LMB * D / 8) + (HALF * ch + 32 * h) * LMB / 8);
+#pragma unroll
+          for (int w = 0; w < LMB; ++w) co[w] = nz ? (cw[w] | cw2[w]) : 0u;
+        }
+#pragma unroll
+        for (int c16 = 0; c16 < 2; ++c16) {
+          uint32_t hw[8], lw[8];
+#pragma unroll
+          for (int p = 0; p < 8; ++p) {
+            const float f0 = use ? 16.f * r[16 * c16 + 2 * p] : 0.f, f1 = use ? 16.f * r[16 * c16 + 2 * p + 1] : 0.f;
+            const __half2 hh = __floats2half2_rn(f0, f1);
+            const float2 hf = __half22float2(hh);
+            const __half2 ll = __floats2half2_rn(f0 - hf.x, f1 - hf.y);
+            hw[p] = *reinterpret_cast<const uint32_t*>(&hh);
+            lw[p] = *reinterpret_cast<const uint32_t*>(&ll);
+          }
+          const uint32_t col = (HALF * ch + 32 * h + 16 * c16) / 2;
+          s1::tmem_st8(tmem + kDnA + lane_base + col, hw);
+          s1::tmem_st8(tmem + kDnA + HALF + lane_base + col, lw);
+        }
+      }
+      xs[ch * 128 + R] = (r4[0] + r4[1]) + (r4[2] + r4[3]);
+      dense_key_sync();
+      const float gamma = sqrtf(xs[R] + xs[128 + R]);
+      if (o >= 0 && ch == 0) {
+        const uint32_t nb = __half_as_ushort(__float2half_rn(sqrtf(tot) * ninv));
+        const uint32_t gb = __half_as_ushort(__float2half_rn(gamma));
+        reinterpret_cast<uint32_t*>(a.k_norms)[o] = nz ? (nb | (gb << 16)) : 0u;
+      }
+      if (ch == 0) zf[R] = use ? 1 : 0;
+      s1::tmem_st_wait();
+      s1::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) s1::mbar_arrive(aready);
+      // ---- QJL signs of this thread's projections
+      if (!failed && !s1::mbar_wait(projd, ph)) failed = true;
+      dense_key_sync();  // zf of both halves written (and read below)
+      s1::fence_after_sync();
+      const bool nzk = zf[R] != 0;
+#pragma unroll 1
+      for (int h = 0; h < HALF / 32; ++h) {
+        uint32_t v[32];
+        s1::tmem_ld32(tmem + lane_base + HALF * ch + 32 * h, v);
+        s1::tmem_ld_wait();
+        uint32_t b4[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int k = 7; k >= 0; --k)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) b4[q] = __funnelshift_l(v[8 * q + k] ^ 0x80000000u, b4[q], 1);
+        const uint32_t word = b4[0] | (b4[1] << 8) | (b4[2] << 16) | (b4[3] << 24);
+        if (o >= 0 && !failed)
+          reinterpret_cast<uint32_t*>(a.k_signs + o * (D / 8) + (HALF * ch + 32 * h) / 8)[0] = nzk ? word : 0u;
+      }
+      s1::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) s1::mbar_arrive(pdone);
+    }
+  } else if (warp == 8 && lane == 0 && (int64_t)blockIdx.x < ntile) {
+    // ================================================================ producer (TMA and MMA)
+    constexpr uint32_t idesc_rot = s1::idesc_f16_f32(128, NW) | (1u << 7) | (1u << 10);  // bf16 x bf16
+    constexpr uint32_t idesc_prj = s1::idesc_f16_f32(128, NW);                           // f16 x f16
+    const int64_t n_my = (ntile - blockIdx.x + g - 1) / g;
+    int kloads = 0;  // key-tile loads issued (phase kloads - 1 is the last one)
+    auto load_keys = [&](int64_t tile) {
+      ++kloads;
+      s1::mbar_expect_tx(kfull, (uint32_t)128 * D * 2);
+#pragma unroll
+      for (int p = 0; p < D / 64; ++p)
+        s1::tma_load_2d(sm + DS::KT + p * 128 * 128, &a.kmap, 64 * p, (int)(tile * 128), kfull);
+    };
+    // streamed operand q (0 .. n_my * NOPS - 1): tile q % NOPS of the pass sequence, slot q % 3
+    int64_t issued = 0, used = 0;
+    auto issue_op = [&]() {
+      const int slot = (int)(issued % 3);
+      s1::mbar_expect_tx(ofull + slot, DS::TILE);
+      s1::bulk_g2s(sm + DS::OPS + slot * DS::TILE, ops + (size_t)(issued % DS::NOPS) * (DS::TILE / 2), DS::TILE,
+                   ofull + slot);
+      ++issued;
+    };
+    const int64_t n_ops = n_my * DS::NOPS;
+    // the operand tile of sequence number q: its shared-memory address (waits for it to land)
+    auto op_addr = [&](int64_t q, bool& ok) -> uint32_t {
+      if constexpr (!DS::STREAM) {
+        return sbase + DS::OPS + (uint32_t)(q % DS::NOPS) * DS::TILE;
+      } else {
+        const int slot = (int)(q % 3);
+        if (!s1::mbar_wait(ofull + slot, (uint32_t)(q / 3) & 1u)) ok = false;
+        return sbase + DS::OPS + slot * DS::TILE;
+      }
+    };
+    // after the MMAs of operand q are issued: release its slot, refill the slot of q - 1
+    auto done_op = [&](int64_t q, bool& ok) {
+      if constexpr (DS::STREAM) {
+        s1::umma_commit(oempty + (int)(q % 3));
+        ++used;
+        if (q >= 1 && issued < n_ops) {
+          // the slot of q - 1 is the slot of q + 2
+          if (!s1::mbar_wait(oempty + (int)((q - 1) % 3), (uint32_t)((q - 1) / 3) & 1u)) ok = false;
+          else issue_op();
+        }
+      }
+    };
+    if constexpr (DS::STREAM) {
+      for (int k = 0; k < 3 && issued < n_ops; ++k) issue_op();
+    }
+    load_keys(blockIdx.x);
+    int64_t q = 0;  // operand sequence number
+    for (int64_t j = 0; j < n_my && !failed; ++j) {
+      const uint32_t ph = (uint32_t)j & 1u;
+      bool ok = s1::mbar_wait(kfull, ph);
+      if (ok && j > 0) ok = s1::mbar_wait(pdone, ph ^ 1u);  // S r of the previous pass read: TMEM free
+      if (!ok) {
+        failed = true;
+        break;
+      }
+      s1::fence_after_sync();
+      // rotation: Y[:, nc] = sum over kc, t of K[:, kc] R_t[nc, kc]^T
+      for (int nc = 0; nc < NCH && ok; ++nc)
+        for (int kc = 0; kc < NCH && ok; ++kc)
+          for (int t = 0; t < NT && ok; ++t, ++q) {
+            const uint32_t b = op_addr(q, ok);
+            if (!ok) break;
+#pragma unroll
+            for (int ks = 0; ks < NW / 16; ++ks)
+              s1::umma_f16(tmem + nc * NW, s1::sw128_desc(sbase + DS::KT, kc * NW + 16 * ks, 128),
+                           s1::sw128_desc(b, 16 * ks, NW), idesc_rot, (kc > 0 || t > 0 || ks > 0) ? 1u : 0u);
+            done_op(q, ok);
+          }
+      if (!ok) {
+        failed = true;
+        break;
+      }
+      s1::umma_commit(rotd);
+      // the key tile is free once the rotation has completed: fetch the next pass's
+      if (j + 1 < n_my) {
+        if (!s1::mbar_wait(rotd, ph)) {
+          failed = true;
+          break;
+        }
+        load_keys(blockIdx.x + (j + 1) * g);
+      }
+      if (!s1::mbar_wait(aready, ph)) {
+        failed = true;
+        break;
+      }
+      s1::fence_after_sync();
+      // projection: S r[:, nc] = sum over kc of (A_hi + A_lo)[:, kc] S_hi[nc, kc]^T + A_hi S_lo^T
+      for (int nc = 0; nc < NCH && ok; ++nc)
+        for (int kc = 0; kc < NCH && ok; ++kc) {
+          const uint32_t bh = op_addr(q, ok);
+          if (!ok) break;
+#pragma unroll
+          for (int ks = 0; ks < NW / 16; ++ks) {
+            const uint32_t ac = (uint32_t)(kc * NW + 16 * ks) / 2;
+            s1::umma_f16_ts(tmem + nc * NW, tmem + kDnA + ac, s1::sw128_desc(bh, 16 * ks, NW), idesc_prj,
+                            (kc > 0 || ks > 0) ? 1u : 0u);
+            s1::umma_f16_ts(tmem + nc * NW, tmem + kDnA + HALF + ac, s1::sw128_desc(bh, 16 * ks, NW), idesc_prj, 1u);
+          }
+          done_op(q, ok);
+          ++q;
+          const uint32_t bl = op_addr(q, ok);
+          if (!ok) break;
+#pragma unroll
+          for (int ks = 0; ks < NW / 16; ++ks) {
+            const uint32_t ac = (uint32_t)(kc * NW + 16 * ks) / 2;
+            s1::umma_f16_ts(tmem + nc * NW, tmem + kDnA + ac, s1::sw128_desc(bl, 16 * ks, NW), idesc_prj, 1u);
+          }
+          done_op(q, ok);
+          ++q;
+        }
+      if (!ok) {
+        failed = true;
+        break;
+      }
+      s1::umma_commit(projd);
+    }
+    if (failed) atomicOr(a.err, 1u);
+    // every MMA issued and every copy issued completes before the CTA's memory goes away
+    s1::umma_commit(fin);
+    s1::mbar_wait(fin, 0u);
+    if (kloads > 0) s1::mbar_wait(kfull, (uint32_t)(kloads - 1) & 1u);
+    if constexpr (DS::STREAM) {
+      // the operand copies issued ahead of use land before the CTA exits
+      for (int64_t qq = used; qq < issued; ++qq) s1::mbar_wait(ofull + (int)(qq % 3), (uint32_t)(qq / 3) & 1u);
+    }
+  }
+  s1::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    s1::fence_after_sync();
+    s1::tmem_dealloc(tmem, 512);
+  }
+}
+
+
+template <int D, int LMB, int NT>
+cudaError_t launch_dense_t(const tq_ctx* ctx, const CompressArgs& a, const uint16_t* ops, cudaStream_t s) {
+  using DS = DenseSmem<D, NT>;
+  static bool configured = false;
+  // at least 120 KB, so that no two CTAs share an SM (each holds all 512 tensor-memory columns)
+  const size_t smem = DS::BYTES + 1024 > 120 * 1024 ? DS::BYTES + 1024 : 120 * 1024;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(compress_dense_kernel<D, LMB, NT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  int64_t blocks = (a.n_vec + 127) / 128;
+  if (blocks > ctx->num_sms) blocks = ctx->num_sms;
+  if (ctx->prof_start) cudaEventRecord(ctx->prof_start, s);
+  compress_dense_kernel<D, LMB, NT><<<(unsigned)blocks, kDenseThreads, smem, s>>>(a, ops);
+  cudaError_t e = cudaGetLastError();
+  if (ctx->prof_stop) cudaEventRecord(ctx->prof_stop, s);
+  return e;
+}
+
+template <int D, int NT>
+cudaError_t launch_dense_l(const tq_ctx* ctx, const CompressArgs& a, const uint16_t* ops, cudaStream_t s) {
+  switch (ctx->shape.lm_bits) {
+    case 1: return launch_dense_t<D, 1, NT>(ctx, a, ops, s);
+    case 2: return launch_dense_t<D, 2, NT>(ctx, a, ops, s);
+    case 3: return launch_dense_t<D, 3, NT>(ctx, a, ops, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+// The dense tensor-core kernel for bf16 keys at d = 64 or 256 (keys only).
+cudaError_t launch_dense(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) {
+  const bool haar = ctx->shape.rot == TQ_ROT_HAAR;
+  if (ctx->shape.d == 64)
+    return haar ? launch_dense_l<64, 3>(ctx, a, ctx->dense_ops, s) : launch_dense_l<64, 1>(ctx, a, ctx->dense_ops, s);
+  return haar ? launch_dense_l<256, 3>(ctx, a, ctx->dense_ops, s) : launch_dense_l<256, 1>(ctx, a, ctx->dense_ops, s);
+}
+
 }  // namespace
 
-// S as f16 in the swizzled K-major operand layout of compress_tc_kernel, or false if
-// S is not exactly representable in f16 (the tensor-core path then is not used).
+// S split in two f16 terms, hi = S rounded to f16 and lo = the remainder S - hi rounded
+// to f16 (about 22 bits of each fp32 value together; an absolute error below 2^-25 where
+// lo falls in the f16 subnormal range), as two tiles (hi, then lo) in the swizzled K-major
+// operand layout of the compression kernels. False if S holds a value that is not finite
+// or lies beyond the f16 range (the tensor-core kernels are then not used).
 bool pack_qjl_operand(const float* S, int m, int d, uint16_t* out) {
   if (m != 128 || d != 128) return false;
+  constexpr size_t kTile = 128 * 128;
   for (int i = 0; i < m; ++i)
     for (int j = 0; j < d; ++j) {
       const float v = S[(size_t)i * d + j];
+      if (!(std::fabs(v) <= 65504.f)) return false;
       const __half h = __float2half_rn(v);
-      if (__half2float(h) != v) return false;
-      out[tq::sm100::sw128_offset(i, j, 128) / 2] = __half_as_ushort(h);
+      const __half l = __float2half_rn(v - __half2float(h));  // v - hi is exact in fp32
+      const size_t off = tq::sm100::sw128_offset(i, j, 128) / 2;
+      out[off] = __half_as_ushort(h);
+      out[kTile + off] = __half_as_ushort(l);
     }
   return true;
 }
@@ -1806,6 +2237,57 @@ float bf16_value(uint16_t h) {
   return f;
 }
 }  // namespace
+
+// Operand tiles of compress_dense_kernel (d = 64 or 256, m = d): the rotation R as NT bf16
+// terms (H diag(sigma) exact, NT = 1; the Haar matrix as three rounded remainders, NT = 3)
+// and S as f16 hi + lo, cut into NW x NW tiles (NW = 64 at d = 64, 128 at d = 256) in the
+// swizzled K-major layout: rotation tiles in (row chunk, column chunk, term) order, then S
+// tiles in (row chunk, column chunk, hi / lo) order. Element (n, k) of a rotation tile
+// multiplies key coordinate k into rotated coordinate n; of an S tile, residual coordinate k
+// into projection n. False if S is not finite or beyond the f16 range.
+bool pack_dense_operands(int d, int rot, const uint32_t* sign_bits, const double* haar, const float* S,
+                         std::vector<uint16_t>& out) {
+  if (d != 64 && d != 256) return false;
+  const int NW = d == 256 ? 128 : 64, NCH = d / NW, NT = rot == TQ_ROT_HAAR ? 3 : 1;
+  const size_t tile = (size_t)NW * NW;
+  out.assign((size_t)NCH * NCH * (NT + 2) * tile, 0);
+  size_t t_idx = 0;
+  for (int nc = 0; nc < NCH; ++nc)
+    for (int kc = 0; kc < NCH; ++kc)
+      for (int t = 0; t < NT; ++t, ++t_idx)
+        for (int n = 0; n < NW; ++n)
+          for (int k = 0; k < NW; ++k) {
+            const int gn = nc * NW + n, gk = kc * NW + k;
+            uint16_t v;
+            if (rot == TQ_ROT_HAAR) {
+              double rem = haar[(size_t)gn * d + gk];
+              uint16_t h = 0;
+              for (int tt = 0; tt <= t; ++tt) {
+                h = bf16_rn((float)rem);
+                rem -= (double)bf16_value(h);
+              }
+              v = h;
+            } else {
+              bool neg = (__builtin_popcount((unsigned)(gn & gk)) & 1) != 0;
+              if ((sign_bits[gk / 32] >> (gk % 32)) & 1u) neg = !neg;
+              v = neg ? 0xBF80u : 0x3F80u;
+            }
+            out[t_idx * tile + tq::sm100::sw128_offset(n, k, NW) / 2] = v;
+          }
+  for (int nc = 0; nc < NCH; ++nc)
+    for (int kc = 0; kc < NCH; ++kc, t_idx += 2)
+      for (int n = 0; n < NW; ++n)
+        for (int k = 0; k < NW; ++k) {
+          const float v = S[(size_t)(nc * NW + n) * d + kc * NW + k];
+          if (!(std::fabs(v) <= 65504.f)) return false;
+          const __half h = __float2half_rn(v);
+          const __half l = __float2half_rn(v - __half2float(h));
+          const size_t off = tq::sm100::sw128_offset(n, k, NW) / 2;
+          out[t_idx * tile + off] = __half_as_ushort(h);
+          out[(t_idx + 1) * tile + off] = __half_as_ushort(l);
+        }
+  return true;
+}
 
 // Pi (fp64, row-major, d = 128) as three bf16 terms Pi ~ P1 + P2 + P3 (each the rounded
 // remainder of the previous ones, about 24 bits together), three tiles in the swizzled
@@ -1857,6 +2339,18 @@ cudaError_t launch_compress(const tq_ctx* ctx, const void* k, const void* v, int
     return cudaErrorInvalidValue;
   };
   if (ctx->shape.lm_bits > 3) return generic(a);  // the tensor-core kernels take 1-3 Lloyd-Max bits
+  if (ctx->dense_ops && (ctx->shape.d == 64 || ctx->shape.d == 256) && ctx->shape.m == ctx->shape.d &&
+      dtype == TQ_BF16 && k) {
+    // keys on the dense tensor-core kernel; values (if any) on the warp-per-vector kernel
+    CompressArgs ka = a;
+    ka.v = nullptr;
+    if (!encode_rows_map(&ka.kmap, k, n_vec, 128, ctx->shape.d)) return generic(a);
+    const cudaError_t e = launch_dense(ctx, ka, stream);
+    if (e != cudaSuccess || !v) return e;
+    CompressArgs va = a;
+    va.k = nullptr;
+    return generic(va);
+  }
   if (ctx->shape.v_bits == 3 && k && v && ctx->S_sw128) {
     // 3-bit value codes straddle words: the tensor-core kernels take the keys alone and
     // the warp-per-vector kernel the values

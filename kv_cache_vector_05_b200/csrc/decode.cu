@@ -373,9 +373,32 @@ cudaError_t dispatch_lmb(const DecodeArgs& a, int lmb, int vb, dim3 grid, size_t
 DecodePlan plan_decode(const tq_ctx* ctx, int batch, int hq, int hkv, int64_t max_len) {
   DecodePlan p{};
   const int d = ctx->shape.d, m = ctx->shape.m, G = hq / hkv;
-  p.mma = mma_decode_supported(ctx, G);
+  p.tc = tc_decode_supported(ctx, G);
+  p.mma = !p.tc && mma_decode_supported(ctx, G);
   const int64_t units = (int64_t)batch * hkv;
   const int64_t sms = ctx->num_sms > 0 ? ctx->num_sms : 148;
+  if (p.tc) {
+    // As below, with 128-token tiles (the MMA's M) and one CTA per SM.
+    const int64_t tile = 128;
+    const int64_t Tu = max_len > 0 ? (max_len + tile - 1) / tile : 1;
+    const int64_t Tt = units * Tu;
+    const int64_t P = Tt < sms ? Tt : sms;
+    p.n_ctas = (int)P;
+    p.tiles_per_unit = Tu;
+    p.total_tiles = Tt;
+    int64_t s_max = 1;
+    for (int64_t u = 0; u < units; ++u) {
+      const int64_t first = ((u * Tu + 1) * P - 1) / Tt, last = ((u + 1) * Tu * P - 1) / Tt;
+      if (last - first + 1 > s_max) s_max = last - first + 1;
+    }
+    p.s_max = (int)s_max;
+    p.ws_part_bytes = align256((size_t)units * s_max * G * (d + kPartPad) * sizeof(float));
+    p.off_frag = 0;
+    p.off_part = align256((size_t)units * tc_operand_bytes(ctx, G));
+    p.off_cnt = p.off_part + p.ws_part_bytes;
+    p.total_bytes = p.off_cnt;
+    return p;
+  }
   if (p.mma) {
     // Every unit (sequence x KV head) is cut into tiles; the units' tiles, laid end
     // to end, are split evenly over one wave of resident CTAs (one per SM). A CTA's
@@ -428,6 +451,9 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const void*
                           const uint16_t* v_params, float scale, float* scores, float* out, float* lse,
                           void* workspace, cudaStream_t stream) {
   const int d = ctx->shape.d, m = ctx->shape.m, G = hq / hkv;
+  if (plan.tc)
+    return launch_decode_tc(ctx, plan, q, q_dtype, batch, hq, hkv, seq_lens, max_len, pg, k_codes, k_signs,
+                            k_norms, v_codes, v_params, scale, scores, out, lse, workspace, stream);
   if (plan.mma)
     return launch_decode_mma(ctx, plan, q, q_dtype, batch, hq, hkv, seq_lens, max_len, pg, k_codes, k_signs,
                              k_norms, v_codes, v_params, scale, scores, out, lse, workspace, stream);

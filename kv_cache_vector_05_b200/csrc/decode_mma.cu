@@ -33,14 +33,19 @@
 //  * prep_mma_kernel, one CTA per (sequence, KV head): rotates the G queries
 //    (sign flip + Walsh-Hadamard butterflies, or the dense Haar matrix), forms
 //    S qr, and writes that KV head's query operand fragments once.
-//  * decode_mma_kernel, one CTA per (sequence x KV head, chunk of the cache),
-//    launched with programmatic dependent launch: it starts streaming its cache
-//    tiles (cp.async.bulk into a ring of stages, mbarrier completion) while the
-//    prep kernel finishes, then waits for the fragments. Each warp owns 16 or 32
-//    consecutive tokens of each tile: it scores them, runs the online softmax for
-//    its heads and accumulates their values. The last CTA of a (sequence, KV head)
-//    to finish - decided by an atomic ticket, nobody waits - merges the chunk
-//    partials (log-sum-exp) and writes the output rows.
+//  * decode_mma_kernel, one 16-warp CTA per SM, launched with programmatic
+//    dependent launch: the tiles of all (sequence, KV head) units, laid end to end,
+//    are split evenly over the CTAs, so a CTA's range may start and end inside a
+//    unit and may span several. It starts streaming its cache tiles (cp.async.bulk
+//    into a ring of stages, mbarrier completion) while the prep kernel finishes,
+//    then waits for the fragments of its first units (two operand buffers, refilled
+//    by bulk copy at each unit boundary). Each warp owns 16 or 32 consecutive tokens
+//    of each tile: it scores them, runs the online softmax for its heads and
+//    accumulates their values. At a unit boundary the 16 warps merge their partials
+//    in a fixed order and the CTA writes one partial (m, l, acc) of the unit.
+//  * combine_mma_kernel, a programmatic dependent of the decode grid: merges the
+//    partials of the CTAs that shared a unit (log-sum-exp) and writes the output
+//    rows (and, for a partial decode, each row's log-partition).
 // Every wait is bounded; a timeout sets the context's error word and ends the CTA.
 #include <cuda_runtime.h>
 #include <math.h>
@@ -382,8 +387,8 @@ struct Layout {
   static constexpr int FRAG_BYTES = frag_words(LMB, NB) * 4;
   // As many stages (2..4) as fit in shared memory next to the two operand buffers and
   // the reduction area (one CTA per SM).
-  static constexpr int RED_BYTES = (8 * kD + 8 + 2 * kWarpsMma * 8 + 16) * 4;
-  static constexpr int BUDGET = 220 * 1024 - 2 * FRAG_BYTES - RED_BYTES - 512;
+  static constexpr int RED_BYTES = (kWarpsMma * kD + 2 * kWarpsMma * 8 + 8) * 4;
+  static constexpr int BUDGET = 227 * 1024 - 2 * FRAG_BYTES - RED_BYTES - 512;
   static constexpr int STAGES = 4 * STAGE <= BUDGET ? 4 : 3 * STAGE <= BUDGET ? 3 : 2;
   static constexpr int OFF_KC = 0;
   static constexpr int OFF_KS = OFF_KC + TILE * KCB;
@@ -422,9 +427,8 @@ __global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid
   int* arrive_s = reinterpret_cast<int*>(smem + L::OFF_CNT);  // [NST] warps done with the stage's tile
   int* issued_s = arrive_s + NST;   // [NST] bulk-copy batches issued into the stage
   int* fissued_s = issued_s + NST;  // [2] copies issued into the operand buffer
-  float* racc_s = reinterpret_cast<float*>(smem + L::OFF_RED);  // [8 heads][d] rescaled sums
-  float* rl_s = racc_s + 8 * kD;                                 // [8] rescaled sums of p
-  float* rm_s = rl_s + 8;                                        // [warps][8] warp maxima
+  float* red_s = reinterpret_cast<float*>(smem + L::OFF_RED);  // [warps][d] one head's rescaled sums
+  float* rm_s = red_s + kWarpsMma * kD;                          // [warps][8] warp maxima
   float* rwl_s = rm_s + kWarpsMma * 8;                           // [warps][8] warp sums of p
   float* rM_s = rwl_s + kWarpsMma * 8;                           // [8] CTA maxima
 
@@ -516,33 +520,42 @@ __global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid
   bool failed = false;
 
   // End of local unit j (every warp calls this at the same tile): the 16 warps' partials
-  // are merged in shared memory (rescaled to the CTA maximum, summed with shared
-  // atomics) and written as this CTA's partial (m, l, acc) of the unit; combine_mma_kernel
-  // merges the partials of the CTAs that shared the unit. Then buffer j % 2 is refilled
-  // with the operands of unit j + 2.
+  // are merged into this CTA's partial (m, l, acc) of the unit, in a fixed order (warp 0
+  // first) so that the result does not depend on how the warps were scheduled; one head
+  // at a time, each warp rescales its sums to the CTA maximum and stores them in
+  // red_s[warp][coordinate], then one thread per coordinate adds the 16 rows in order.
+  // combine_mma_kernel merges the partials of the CTAs that shared the unit. Then buffer
+  // j % 2 is refilled with the operands of unit j + 2.
   auto finish_unit = [&](int j) {
     const int u = u_first + j;
     const int seg = (int)(kcta - tile_owner((int64_t)u * Tu, P, Tt));
+    float* part = a.ws_part + ((size_t)u * a.s_max + seg) * G * RS;
     __syncthreads();  // every warp has left the previous boundary's reduction
-    float lsum[NB];
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
       float l = l_run[nb];
       l += __shfl_xor_sync(kFull, l, 4);
       l += __shfl_xor_sync(kFull, l, 8);
       l += __shfl_xor_sync(kFull, l, 16);
-      lsum[nb] = l;
       if (r == 0) {
         rm_s[warp * 8 + c + 4 * nb] = failed ? -INFINITY : m_run[nb];
         rwl_s[warp * 8 + c + 4 * nb] = failed ? 0.f : l;
       }
     }
-    for (int x = tid; x < 8 * kD + 8; x += kThreadsMma) racc_s[x] = 0.f;
     __syncthreads();
     if (tid < 8) {
       float M = -INFINITY;
       for (int w = 0; w < kWarpsMma; ++w) M = fmaxf(M, rm_s[w * 8 + tid]);
+      float L = 0.f;
+      for (int w = 0; w < kWarpsMma; ++w) {
+        const float mw = rm_s[w * 8 + tid];
+        if (mw != -INFINITY) L = fmaf(ex2(mw - M), rwl_s[w * 8 + tid], L);
+      }
       rM_s[tid] = M;
+      if (tid < G) {
+        part[tid * RS + 0] = M;
+        part[tid * RS + 1] = L;
+      }
     }
     __syncthreads();
 #pragma unroll
@@ -552,37 +565,41 @@ __global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid
       float mt[4];
 #pragma unroll
       for (int g = 0; g < 4; ++g) mt[g] = __shfl_sync(kFull, own, 4 * g + c);
-      const int h = c + 4 * nb;
-      const float M = rM_s[h];
+      const float M = rM_s[c + 4 * nb];
       const float wsc = (failed || m_run[nb] == -INFINITY) ? 0.f : ex2(m_run[nb] - M);
-      if (h < G && wsc != 0.f) {
-        if (r == 0) atomicAdd(&rl_s[h], wsc * lsum[nb]);
-        float* acc = racc_s + h * kD;
+      float* red = red_s + warp * kD;
+      for (int c4 = 0; c4 < 4; ++c4) {
+        const int h = 4 * nb + c4;
+        if (h >= G) break;  // uniform
+        if (c == c4) {  // the 8 lanes holding head h: 16 coordinates each
 #pragma unroll
-        for (int g = 0; g < 4; ++g)
+          for (int g = 0; g < 4; ++g)
 #pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            const float* d = dv[g][hf][nb];
-            if (VB == 2) {
-              const int j0 = 4 * (8 * g + r) + 2 * hf;  // code at mantissa bits 4hf (row r), 4hf + 2 (row r + 8)
-              atomicAdd(&acc[j0], wsc * ((d[0] + d[1]) * ldexpf(1.f, 24 - 4 * hf) + mt[g]));
-              atomicAdd(&acc[j0 + 1], wsc * ((d[2] + d[3]) * ldexpf(1.f, 22 - 4 * hf) + mt[g]));
-            } else {
-              const int j0 = 2 * (16 * g + 8 * hf + r);  // low nibble (row r), high nibble (row r + 8)
-              atomicAdd(&acc[j0], wsc * ((d[0] + d[1]) * 16777216.f + mt[g]));
-              atomicAdd(&acc[j0 + 1], wsc * ((d[2] + d[3]) * 1048576.f + mt[g]));
+            for (int hf = 0; hf < 2; ++hf) {
+              const float* d = dv[g][hf][nb];
+              int j0;
+              float v0, v1;
+              if (VB == 2) {
+                j0 = 4 * (8 * g + r) + 2 * hf;  // code at mantissa bits 4hf (row r), 4hf + 2 (row r + 8)
+                v0 = (d[0] + d[1]) * ldexpf(1.f, 24 - 4 * hf) + mt[g];
+                v1 = (d[2] + d[3]) * ldexpf(1.f, 22 - 4 * hf) + mt[g];
+              } else {
+                j0 = 2 * (16 * g + 8 * hf + r);  // low nibble (row r), high nibble (row r + 8)
+                v0 = (d[0] + d[1]) * 16777216.f + mt[g];
+                v1 = (d[2] + d[3]) * 1048576.f + mt[g];
+              }
+              red[j0] = wsc != 0.f ? wsc * v0 : 0.f;
+              red[j0 + 1] = wsc != 0.f ? wsc * v1 : 0.f;
             }
-          }
-      }
-    }
-    __syncthreads();
-    float* part = a.ws_part + ((size_t)u * a.s_max + seg) * G * RS;
-    for (int x = tid; x < G * kD; x += kThreadsMma) {
-      const int h = x / kD, jj = x - h * kD;
-      part[h * RS + kPartPadMma + jj] = racc_s[x];
-      if (jj == 0) {
-        part[h * RS + 0] = rM_s[h];
-        part[h * RS + 1] = rl_s[h];
+        }
+        __syncthreads();
+        if (tid < kD) {
+          float acc = 0.f;
+#pragma unroll
+          for (int w = 0; w < kWarpsMma; ++w) acc += red_s[w * kD + tid];
+          part[h * RS + kPartPadMma + tid] = acc;
+        }
+        __syncthreads();
       }
     }
     if (tid == 0 && j + 2 < n_units) {
@@ -1107,6 +1124,13 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
   if (ctx->prof_stop) cudaEventRecord(ctx->prof_stop, stream);
   if (e != cudaSuccess) return e;
 
+  return launch_combine_partials(part, out, lse, batch, hq, hkv, G, plan.s_max, plan.tiles_per_unit,
+                                 plan.total_tiles, plan.n_ctas, stream);
+}
+
+cudaError_t launch_combine_partials(const float* part, float* out, float* lse, int batch, int hq, int hkv, int G,
+                                    int s_max, int64_t tiles_per_unit, int64_t total_tiles, int n_ctas,
+                                    cudaStream_t stream) {
   CombineArgs ca;
   ca.ws_part = part;
   ca.out = out;
@@ -1114,10 +1138,10 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
   ca.hq = hq;
   ca.hkv = hkv;
   ca.G = G;
-  ca.s_max = plan.s_max;
-  ca.tiles_per_unit = plan.tiles_per_unit;
-  ca.total_tiles = plan.total_tiles;
-  ca.n_ctas = plan.n_ctas;
+  ca.s_max = s_max;
+  ca.tiles_per_unit = tiles_per_unit;
+  ca.total_tiles = total_tiles;
+  ca.n_ctas = n_ctas;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)((int64_t)batch * hkv * G));
   cfg.blockDim = dim3(kD);

@@ -39,6 +39,7 @@ void free_tables(tq_ctx* c) {
   cudaFree(c->S_sw128);
   cudaFree(c->H_sw128);
   cudaFree(c->Pi_sw128);
+  cudaFree(c->dense_ops);
 }
 
 }  // namespace
@@ -162,7 +163,7 @@ tq_status tq_codebook_load(const tq_params* p, void* stream, tq_ctx** out) {
   if (e == cudaSuccess) e = cudaMalloc((void**)&c->d_err, sizeof(unsigned int));
   std::vector<uint16_t> s_op;
   if (d == 128 && m == 128) {
-    s_op.assign((size_t)m * d, 0);
+    s_op.assign((size_t)2 * m * d, 0);  // hi and lo tiles
     if (!tq::pack_qjl_operand(p->qjl_S, m, d, s_op.data())) s_op.clear();
     if (e == cudaSuccess && !s_op.empty()) e = cudaMalloc((void**)&c->S_sw128, s_op.size() * sizeof(uint16_t));
   }
@@ -171,6 +172,12 @@ tq_status tq_codebook_load(const tq_params* p, void* stream, tq_ctx** out) {
     h_op.assign((size_t)d * d, 0);
     tq::pack_hadamard_operand(c->cb.sign_bits, h_op.data());
     if (e == cudaSuccess) e = cudaMalloc((void**)&c->H_sw128, h_op.size() * sizeof(uint16_t));
+  }
+  std::vector<uint16_t> dense_op;
+  if ((d == 64 || d == 256) && m == d && b <= 3) {
+    if (!tq::pack_dense_operands(d, p->rot, c->cb.sign_bits, p->haar, p->qjl_S, dense_op)) dense_op.clear();
+    if (e == cudaSuccess && !dense_op.empty())
+      e = cudaMalloc((void**)&c->dense_ops, dense_op.size() * sizeof(uint16_t));
   }
   std::vector<uint16_t> pi_op;
   if (d == 128 && m == 128 && !s_op.empty() && p->rot == TQ_ROT_HAAR) {
@@ -199,6 +206,9 @@ tq_status tq_codebook_load(const tq_params* p, void* stream, tq_ctx** out) {
     e = cudaMemcpyAsync(c->H_sw128, h_op.data(), h_op.size() * sizeof(uint16_t), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess && !pi_op.empty())
     e = cudaMemcpyAsync(c->Pi_sw128, pi_op.data(), pi_op.size() * sizeof(uint16_t), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && !dense_op.empty())
+    e = cudaMemcpyAsync(c->dense_ops, dense_op.data(), dense_op.size() * sizeof(uint16_t), cudaMemcpyHostToDevice,
+                        s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) {
     free_tables(c);

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <vector>
+
 #include "../../include/tq.h"
 
 namespace tq {
@@ -55,9 +57,10 @@ struct tq_ctx {
   cudaEvent_t prof_stop;
   unsigned int* d_err;     // device error word: bit 0 = a bounded wait in a kernel timed out,
                            // bit 2 = a slot or page index outside the caller's arrays
-  uint16_t* S_sw128;       // tensor-core compression: S as an f16 operand tile (d = m = 128, S exact in f16)
+  uint16_t* S_sw128;       // tensor-core compression: S as f16 hi and lo operand tiles (d = m = 128)
   uint16_t* H_sw128;       // tensor-core compression: H diag(sigma) as a bf16 operand tile (d = 128, Hadamard)
   uint16_t* Pi_sw128;      // tensor-core compression: Haar Pi as three bf16 operand tiles (d = 128)
+  uint16_t* dense_ops;     // tensor-core compression at d = 64 / 256 (m = d): rotation and S operand tiles
 };
 
 namespace tq {
@@ -70,7 +73,8 @@ cudaError_t launch_compress(const tq_ctx* ctx, const void* k, const void* v, int
                             cudaStream_t stream);
 
 struct DecodePlan {
-  bool mma;          // tensor-core kernels (decode_mma.cu) instead of the generic ones
+  bool tc;           // tcgen05 score kernels (decode_tc.cu)
+  bool mma;          // mma.sync kernels (decode_mma.cu) instead of the generic ones
   int n_chunks;      // split-K chunks per (sequence, KV head)
   int64_t chunk_len; // tokens per chunk (multiple of the tile)
   size_t ws_q_bytes;     // generic path: prepared queries
@@ -93,6 +97,21 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const void*
                           cudaStream_t stream);
 
 bool mma_decode_supported(const tq_ctx* ctx, int G);
+bool tc_decode_supported(const tq_ctx* ctx, int G);
+size_t tc_operand_bytes(const tq_ctx* ctx, int G);  // query operand bytes per (sequence, KV head)
+
+cudaError_t launch_decode_tc(const tq_ctx* ctx, const DecodePlan& plan, const void* q, int q_dtype, int batch,
+                             int hq, int hkv, const int32_t* seq_lens, int64_t max_len, const Paging& pg,
+                             const uint8_t* k_codes, const uint8_t* k_signs, const uint16_t* k_norms,
+                             const uint8_t* v_codes, const uint16_t* v_params, float scale, float* scores,
+                             float* out, float* lse, void* workspace, cudaStream_t stream);
+
+// Log-sum-exp merge of the CTA partials [units][s_max][G][4 + 128] (m, l in base 2, acc) of
+// the tile-split decode kernels into out (and lse), launched as a programmatic dependent of
+// the decode grid (decode_mma.cu).
+cudaError_t launch_combine_partials(const float* part, float* out, float* lse, int batch, int hq, int hkv, int G,
+                                    int s_max, int64_t tiles_per_unit, int64_t total_tiles, int n_ctas,
+                                    cudaStream_t stream);
 
 size_t mma_frag_bytes(int lm_bits, int G);  // query operand bytes per (sequence, KV head)
 int mma_tile_tokens(int G);                  // tokens per tile of the tensor-core decode
@@ -100,6 +119,8 @@ int mma_ctas_per_sm(int lm_bits, int v_bits, int G);  // resident CTAs per SM of
 bool pack_qjl_operand(const float* S, int m, int d, uint16_t* out);
 void pack_hadamard_operand(const uint32_t* sign_bits, uint16_t* out);  // d = 128
 void pack_haar_operand(const double* pi, uint16_t* out);                // d = 128, 3 tiles
+bool pack_dense_operands(int d, int rot, const uint32_t* sign_bits, const double* haar, const float* S,
+                         std::vector<uint16_t>& out);                   // d = 64 / 256
 
 cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const void* q, int q_dtype, int batch,
                               int hq, int hkv, const int32_t* seq_lens, int64_t max_len, const Paging& pg,

@@ -4,8 +4,8 @@ tq_compress_kv_slots writes each vector's records at a caller-chosen row (append
 growing cache, filling pages); tq_decode_attention_paged reads a cache scattered over pages
 through a block table. Compression is per vector, so the slot-mapped records must equal the
 contiguous ones bit for bit. The decode kernels walk the same tiles under either addressing:
-the scores are bit-identical, the outputs equal up to the order in which the warps' partial
-sums are added (shared-memory atomics); the paged decode is also checked against the oracle."""
+scores and outputs must be bit-identical (every partial sum is added in a fixed order), and
+the paged decode is also checked against the oracle."""
 import numpy as np
 import pytest
 
@@ -189,7 +189,7 @@ def test_paged_decode_equals_contiguous_and_oracle(d, lm_bits, v_bits, G, page_s
                                            n_pages, seq_lens=lens_t, scores=sc_p)
     T.tq_check_device(ctx)
     oc, op = out_c.cpu().numpy(), out_p.cpu().numpy()
-    np.testing.assert_allclose(op, oc, rtol=1e-5, atol=1e-7)
+    np.testing.assert_array_equal(op, oc)                                 # bit for bit
     assert np.array_equal(np.isnan(sc_c.cpu().numpy()), np.isnan(sc_p.cpu().numpy()))
     assert np.array_equal(np.nan_to_num(sc_c.cpu().numpy()), np.nan_to_num(sc_p.cpu().numpy()))
     Pi, c, t, S = oracle_setup(d, lm_bits)
@@ -222,4 +222,22 @@ def test_paged_decode_rejects_bad_arguments_and_flags_bad_pages():
     out, _ = T.tq_decode_attention_paged(ctx, q, packed, batch, hkv * G, hkv, max_len, bt, page_size, 2)
     T.tq_check_device(ctx)                                                # the context is still usable
     ref, _ = T.tq_decode_attention(ctx, q, packed, batch, hkv * G, hkv, max_len)
-    np.testing.assert_allclose(out.cpu().numpy(), ref.cpu().numpy(), rtol=1e-5, atol=1e-7)
+    np.testing.assert_array_equal(out.cpu().numpy(), ref.cpu().numpy())
+
+
+@pytest.mark.parametrize("d,lm_bits,v_bits,G", [(128, 2, 2, 4), (128, 2, 4, 8), (128, 3, 4, 6)])
+def test_decode_is_bit_reproducible(d, lm_bits, v_bits, G):
+    """The same call twice gives the same bits (no order-dependent floating-point sums),
+    on a cache long enough that several CTAs share each unit."""
+    batch, hkv, max_len = 2, 2, 40000
+    hq = hkv * G
+    ctx = make_ctx(T, d, lm_bits, v_bits)
+    packed = _upload(W.random_packed_cache(batch * hkv * max_len, d, lm_bits, d, v_bits, seed=17))
+    q = torch.from_numpy(W.queries((batch, hq, d), seed=5)).to(DEV)
+    outs = []
+    for _ in range(3):
+        o, _ = T.tq_decode_attention(ctx, q, packed, batch, hq, hkv, max_len)
+        outs.append(o.cpu().numpy())
+    T.tq_check_device(ctx)
+    np.testing.assert_array_equal(outs[0], outs[1])
+    np.testing.assert_array_equal(outs[0], outs[2])

@@ -115,6 +115,27 @@ def test_compress_parity_several_passes_per_cta(lm_bits):
         assert np.array_equal(gv[name], g[name]), name
 
 
+@pytest.mark.parametrize("d", [64, 256])
+@pytest.mark.parametrize("rotation", ["hadamard", "haar"])
+@pytest.mark.parametrize("lm_bits", [1, 3])
+def test_compress_dense_tensor_core_several_passes(d, rotation, lm_bits):
+    """bf16 keys at d = 64 and 256 take the dense tensor-core kernel (rotation and QJL
+    projection as tcgen05 MMAs; at d = 256 the operand tiles stream through a ring of three
+    shared-memory slots): two to three passes of 128 keys per CTA and a ragged last pass,
+    zero keys, every vector compared; values in the same call (warp-per-vector kernel)."""
+    v_bits = 2
+    n = 148 * 128 * 2 + 333
+    rng = np.random.default_rng([d, lm_bits, 5])
+    K = rng.standard_normal((n, d)).astype(np.float32) * rng.lognormal(0, 1, d).astype(np.float32)
+    V = rng.standard_normal((n, d)).astype(np.float32)
+    K[[0, 128 * 148 + 5, n - 1]] = 0.0
+    ctx, g, ok, ov = _compress_both(K, V, d, lm_bits, v_bits, rotation, "bf16")
+    ks = compare_keys(g, ok, d, lm_bits, d)
+    assert_key_parity(ks)
+    assert ks["sign_bad"] == 0, ks
+    assert_value_parity(compare_values(g, ov, d, v_bits))
+
+
 def test_compress_parity_asymmetric_codebook():
     """A codebook that is not symmetric about zero (one outer centroid and boundary moved)
     takes the general bucketize; bf16 keys, Hadamard, d = 128, several passes per CTA."""
@@ -136,6 +157,54 @@ def test_compress_parity_asymmetric_codebook():
     ok = O.compress_keys(kt.float().cpu().numpy().astype(np.float64), Pi, c32.astype(np.float64),
                          t32.astype(np.float64), dr["qjl_S"], with_diagnostics=True)
     assert_key_parity(compare_keys(g, ok, d, lm_bits, d))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("rotation", ["hadamard", "haar"])
+def test_compress_unrounded_gaussian_S(dtype, rotation):
+    """The QJL matrix is a plain fp32 N(0,1) draw (almost none of its entries lie on the
+    f16 grid): the tensor-core kernels take it as two f16 terms. d = m = 128, several passes
+    per CTA, every vector compared."""
+    d, lm_bits, v_bits = 128, 2, 2
+    S = W.method_draws(d, d, 1234)["qjl_S"]
+    assert np.mean(S.astype(np.float16).astype(np.float64) == S) < 0.01
+    n = 148 * 128 + 5 * 128 + 19
+    rng = np.random.default_rng([11, d])
+    K = rng.standard_normal((n, d)).astype(np.float32) * rng.lognormal(0, 1, d).astype(np.float32)
+    V = rng.standard_normal((n, d)).astype(np.float32)
+    ctx, g, ok, ov = _compress_both(K, V, d, lm_bits, v_bits, rotation, dtype)
+    ks = compare_keys(g, ok, d, lm_bits, d)
+    assert_key_parity(ks)
+    assert ks["sign_bad"] == 0, ks
+    assert_value_parity(compare_values(g, ov, d, v_bits))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_compress_S_beyond_f16_range_takes_the_warp_per_vector_kernel(dtype):
+    """An S entry beyond the f16 range cannot be an f16 operand term: the call falls back to
+    the warp-per-vector kernel (CUDA-core projection), which must agree with the oracle too."""
+    d, lm_bits, v_bits = 128, 2, 2
+    dr = W.method_draws(d, d, 1234)
+    S = dr["qjl_S"].copy()
+    S[5, 7] = 1.0e5                                       # exact in fp32, above 65504
+    c32, t32 = T.tq_lloyd_max_codebook(d, lm_bits)
+    ctx = T.tq_codebook_load(d, lm_bits, v_bits, c32, t32, S, rotation="hadamard",
+                             hadamard_signs=dr["hadamard_signs"])
+    n = 2 * 148 * 8 + 13
+    rng = np.random.default_rng([12, d])
+    K = rng.standard_normal((n, d)).astype(np.float32)
+    V = rng.standard_normal((n, d)).astype(np.float32)
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    kt = torch.from_numpy(K).to(DEV).to(tdt)
+    vt = torch.from_numpy(V).to(DEV).to(tdt)
+    g = to_np(T.tq_compress_kv(ctx, kt, vt))
+    T.tq_check_device(ctx)
+    Pi = O.hadamard_rotation(dr["hadamard_signs"])
+    c, t = O.device_codebook(d, lm_bits)
+    ok = O.compress_keys(kt.float().cpu().numpy().astype(np.float64), Pi, c, t, S, with_diagnostics=True)
+    ov = O.quantize_values(vt.float().cpu().numpy().astype(np.float64), v_bits, with_diagnostics=True)
+    assert_key_parity(compare_keys(g, ok, d, lm_bits, d))
+    assert_value_parity(compare_values(g, ov, d, v_bits))
 
 
 def test_compress_edge_cases():
@@ -275,6 +344,53 @@ def test_decode_parity_full_size_sampled(name, units):
     lens = [w.tokens] * w.batch
     _decode_check(w.d, w.lm_bits, w.v_bits, w.batch, w.hkv, w.group, w.tokens, lens,
                   q_dtype=w.dtype, packed=packed, units=units, with_scores=(name != "long_1m_k4v4"))
+
+
+@pytest.mark.parametrize("d,lm_bits,v_bits,G", [(128, 2, 2, 4), (128, 2, 4, 8), (128, 3, 4, 6)])
+@pytest.mark.parametrize("k_norm_scale", [10.0, 30.0])
+def test_decode_parity_large_key_norms(d, lm_bits, v_bits, G, k_norm_scale):
+    """Key norms 10-30 times those of a unit-variance key (the Qwen-shaped cache's outlier
+    channels give such norms): logits reach tens, the softmax is sharply peaked, and the
+    online softmax rescales often. Some value groups get scales 100x larger, one a zero
+    scale; the tensor-core decode (first two) and the generic decode (3-bit codes)."""
+    batch, hkv, max_len = 2, 2, 3000
+    n_vec = batch * hkv * max_len
+    packed = W.random_packed_cache(n_vec, d, lm_bits, d, v_bits, seed=41, k_norm_scale=k_norm_scale)
+    vp = packed["v_params"].view(np.float16).copy()
+    rng = np.random.default_rng(42)
+    big = rng.random(vp.shape[:2]) < 0.05
+    vp[..., 0][big] = (vp[..., 0][big].astype(np.float64) * 100.0).astype(np.float16)
+    vp[3, 1, 0] = 0.0                                                     # a constant group
+    packed["v_params"] = vp.view(np.uint16)
+    _decode_check(d, lm_bits, v_bits, batch, hkv, G, max_len, lens=[3000, 2049], packed=packed)
+
+
+@pytest.mark.parametrize("layers", [(0, 17, 35)])
+def test_decode_parity_qwen_shaped_library_compressed(layers):
+    """Qwen2.5-3B-shaped keys and values (lognormal channel scales, four x20 outlier
+    channels, K norms about 100x V norms) compressed by the library, then decoded at G = 8
+    (two query-head blocks of the tensor-core decode) for several layers; scores and outputs
+    against the oracle decoding the same packed bytes."""
+    d, lm_bits, v_bits, G, tokens = 128, 2, 2, 8, 8192
+    ctx = make_ctx(T, d, lm_bits, v_bits)
+    Pi, c, t, S = oracle_setup(d, lm_bits)
+    for layer in layers:
+        K, V = W.qwen_layer_head_kv(layer=layer, head=layer % 2, tokens=tokens)
+        kt = torch.from_numpy(K).to(DEV).to(torch.bfloat16)
+        vt = torch.from_numpy(V).to(DEV).to(torch.bfloat16)
+        gp = T.tq_compress_kv(ctx, kt, vt)
+        q = W.queries((1, G, d), seed=100 + layer, dtype="bf16")
+        qt = torch.from_numpy(q).to(DEV).to(torch.bfloat16)
+        scores = torch.full((1, G, tokens), float("nan"), device=DEV)
+        out, _ = T.tq_decode_attention(ctx, qt, gp, 1, G, 1, tokens, scores=scores)
+        T.tq_check_device(ctx)
+        g = to_np(gp)
+        pk = {"codes": g["k_codes"], "signs": g["k_signs"], "norms": g["k_norms"]}
+        pv = {"codes": g["v_codes"], "params": g["v_params"]}
+        os_, oo = O.decode_attention(q[0].astype(np.float64), pk, pv, Pi, c, S, d, v_bits)
+        assert np.max(np.abs(os_)) > 5.0                                  # large logits indeed
+        assert_close(scores[0].cpu().numpy(), os_, what=f"scores layer {layer}")
+        assert_close(out[0].cpu().numpy(), oo, what=f"out layer {layer}")
 
 
 def test_decode_rejects_small_workspace():
