@@ -182,6 +182,11 @@ size_t tq_decode_workspace_bytes(const tq_ctx* ctx, int batch, int hq, int hkv, 
  *             logits of valid positions (others untouched)
  *   out       device fp32 [batch][hq][d]
  *   workspace device scratch of at least tq_decode_workspace_bytes(...) bytes
+ * At d = 128 with 1- to 3-bit Lloyd-Max codes of a codebook symmetric about zero,
+ * 2- or 4-bit values and at most 8 query heads per KV head, the tensor-core decode
+ * runs; it carries p * scale (p < 4) as f16 operands, so value-group scales must stay
+ * below 16376 (values spanning less than 49000 at 2 bits). Other shapes run the
+ * CUDA-core decode.
  * Returns TQ_EINVAL if the workspace is too small or any pointer is misaligned. */
 tq_status tq_decode_attention(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int batch, int hq,
                               int hkv, const int32_t* seq_lens, int64_t max_len,

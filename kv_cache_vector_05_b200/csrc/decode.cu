@@ -392,7 +392,8 @@ DecodePlan plan_decode(const tq_ctx* ctx, int batch, int hq, int hkv, int64_t ma
       if (last - first + 1 > s_max) s_max = last - first + 1;
     }
     p.s_max = (int)s_max;
-    p.ws_part_bytes = align256((size_t)units * s_max * G * (d + kPartPad) * sizeof(float));
+    // one partial per warp group of every CTA that shares a unit
+    p.ws_part_bytes = align256((size_t)units * s_max * tc_groups(ctx, G) * G * (d + kPartPad) * sizeof(float));
     p.off_frag = 0;
     p.off_part = align256((size_t)units * tc_operand_bytes(ctx, G));
     p.off_cnt = p.off_part + p.ws_part_bytes;

@@ -914,6 +914,7 @@ struct CombineArgs {
   float* out;
   float* lse;  // null, or the log of each row's softmax denominator
   int hq, hkv, G, s_max;
+  int ppc;     // partials per CTA and unit (consecutive slots)
   int64_t tiles_per_unit, total_tiles, n_ctas;
 };
 
@@ -929,9 +930,9 @@ __global__ void __launch_bounds__(kD) combine_mma_kernel(const __grid_constant__
   const int u = blockIdx.x / a.G, h = blockIdx.x - u * a.G;
   const int64_t Tu = a.tiles_per_unit;
   const int64_t first = tile_owner((int64_t)u * Tu, a.n_ctas, a.total_tiles);
-  const int n_part = (int)(tile_owner((int64_t)(u + 1) * Tu - 1, a.n_ctas, a.total_tiles) - first + 1);
+  const int n_part = a.ppc * (int)(tile_owner((int64_t)(u + 1) * Tu - 1, a.n_ctas, a.total_tiles) - first + 1);
   const size_t pstride = (size_t)a.G * RS;  // partial p of head h at base + p * pstride
-  const float* base = a.ws_part + (size_t)u * a.s_max * pstride + (size_t)h * RS;
+  const float* base = a.ws_part + (size_t)u * a.s_max * a.ppc * pstride + (size_t)h * RS;
 
   float M = -INFINITY;
   for (int p = tid; p < n_part; p += kD) M = fmaxf(M, base[p * pstride]);
@@ -946,7 +947,7 @@ __global__ void __launch_bounds__(kD) combine_mma_kernel(const __grid_constant__
     if (p < n_part) {
       const float mp = base[p * pstride];
       w = mp == -INFINITY ? 0.f : exp2f(mp - M);
-      den = fmaf(w, base[p * pstride + 1], den);
+      if (w != 0.f) den = fmaf(w, base[p * pstride + 1], den);
     }
     __syncthreads();  // the previous chunk's weights are consumed
     w_s[tid] = w;
@@ -954,11 +955,12 @@ __global__ void __launch_bounds__(kD) combine_mma_kernel(const __grid_constant__
     const int np = min(kD, n_part - p0);
     const float* acc = base + (size_t)p0 * pstride + kPartPadMma + tid;
     int q = 0;
+    // a partial of weight 0 (no valid token) is skipped: its sums need not be written
     for (; q + 2 <= np; q += 2) {
-      num0 = fmaf(w_s[q], acc[q * pstride], num0);
-      num1 = fmaf(w_s[q + 1], acc[(q + 1) * pstride], num1);
+      if (w_s[q] != 0.f) num0 = fmaf(w_s[q], acc[q * pstride], num0);
+      if (w_s[q + 1] != 0.f) num1 = fmaf(w_s[q + 1], acc[(q + 1) * pstride], num1);
     }
-    if (q < np) num0 = fmaf(w_s[q], acc[q * pstride], num0);
+    if (q < np && w_s[q] != 0.f) num0 = fmaf(w_s[q], acc[q * pstride], num0);
   }
   den = warp_sum(den);
   if (lane == 0) red_s[1][warp] = den;
@@ -1124,14 +1126,15 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
   if (ctx->prof_stop) cudaEventRecord(ctx->prof_stop, stream);
   if (e != cudaSuccess) return e;
 
-  return launch_combine_partials(part, out, lse, batch, hq, hkv, G, plan.s_max, plan.tiles_per_unit,
+  return launch_combine_partials(part, out, lse, batch, hq, hkv, G, plan.s_max, 1, plan.tiles_per_unit,
                                  plan.total_tiles, plan.n_ctas, stream);
 }
 
 cudaError_t launch_combine_partials(const float* part, float* out, float* lse, int batch, int hq, int hkv, int G,
-                                    int s_max, int64_t tiles_per_unit, int64_t total_tiles, int n_ctas,
+                                    int s_max, int ppc, int64_t tiles_per_unit, int64_t total_tiles, int n_ctas,
                                     cudaStream_t stream) {
   CombineArgs ca;
+  ca.ppc = ppc;
   ca.ws_part = part;
   ca.out = out;
   ca.lse = lse;

@@ -66,11 +66,12 @@ namespace s1 = tq::sm100;
 constexpr int kD = 128;
 constexpr int kM = 128;
 constexpr int kTileTc = 128;       // tokens per tile = MMA rows
-constexpr int kThreadsTc = 512;
-constexpr int kPairStride = 68;    // words per (group, head, part) row of the value weights: 64 token pairs + 4
 constexpr int kPrepTcThreads = 256;
 constexpr float kSlackTc = 2.f;
 constexpr uint32_t kWaitPolls = 1u << 24;
+// Suspend-time hint of one mbarrier poll in ns (0: the instruction's own short limit). The
+// roles hand each tile to one another, so a waiting warp must see the phase at once.
+constexpr uint32_t kTryWaitNs = 0;
 constexpr unsigned long long kWaitNs = 2000000000ull;
 // |Q| <= 2^30 keeps the top one of four balanced 8-bit digits in [-64, 64]
 constexpr float kQmax = 1073741824.f;
@@ -90,9 +91,14 @@ struct TcLayout {
   static constexpr int KB = 32 * EW;                   // bytes of one B row
   static constexpr int NC = kDigits * HG;              // code columns (4 digits per head)
   static constexpr int N = ((NC + (QJL ? NC : 0)) + 15) / 16 * 16;
-  static constexpr int TA = 8 * EW;                    // tensor-memory columns of one A buffer
-  static constexpr int TM_D = 2 * TA;                  // D[b] at TM_D + b * N
-  static_assert(2 * TA + 2 * N <= 512, "tensor memory");
+  static constexpr int TA = 8 * EW;                    // tensor-memory columns of one A operand
+  static constexpr int TG = TA + N;                    // tensor-memory columns of one group
+  // groups of four warps, one tile each: as many as tensor memory holds, at most 3, so that
+  // with the producer no scheduler holds more than 4 warps (128 registers each)
+  static constexpr int NG = 512 / TG >= 3 ? 3 : 512 / TG;
+  static_assert(NG >= 2, "tensor memory for two groups");
+  static constexpr int NCW = 4 * NG;                   // compute warps
+  static constexpr int THREADS = 32 * (NCW + 1);       // + the producer warp
   static constexpr int KCB = LMB * 16, SB = QJL ? 16 : 0, VCB = VB * 16, PB = 16;
   static constexpr int REC = KCB + SB + 4 + VCB + PB;
   static constexpr int STAGE = kTileTc * REC;
@@ -101,22 +107,24 @@ struct TcLayout {
   static constexpr int BOP = N * KB;                   // digits, K-major, 128-byte swizzle
   static constexpr int BBUF = BOP + HG * 16;           // + logit constants (float4 per head)
   static constexpr int BBUF_AL = (BBUF + 1023) / 1024 * 1024;
-  static constexpr int PPW = 4 * HG * 2 * kPairStride + 16;  // value weights p * scale [group][head][part][pair]
-  static constexpr int PMW = HG * 2 * kPairStride;     // p [head][part][pair] for the minima
-  static constexpr int PHDR = 16;                      // flag, rescale factors [HG]
-  static constexpr int PBUF = (PPW + PMW + PHDR) * 4;
-  static constexpr int SM_B = 0;
-  static constexpr int SM_P = 2 * BBUF_AL;
-  static constexpr int SM_VR = SM_P + 2 * PBUF;        // [4 value warps][HG][d] unit-end sums
-  static constexpr int SM_LR = SM_VR + 4 * HG * kD * 4;   // [HG][128] unit-end sums of p
-  static constexpr int SM_TMX = SM_LR + HG * kTileTc * 4; // [4 softmax warps][HG] tile maxima
-  static constexpr int SM_BAR = SM_TMX + 4 * HG * 4;
-  static constexpr int NBAR_FIXED = 16;
-  static constexpr int SM_MISC = SM_BAR + 8 * (NBAR_FIXED + 2 * 12);  // TMEM address, abort flag
-  static constexpr int SM_RING = (SM_MISC + 16 + 127) / 128 * 128;
+  // Per compute warp: value weights p * scale [group][head][part][16 token pairs] (rows of
+  // kPS words; groups 2-3 16 words further), then p [head][part][16 pairs] for the minima.
+  static constexpr int kPS = 20;
+  static constexpr int WP_PW = 4 * HG * 2 * kPS + 16;
+  static constexpr int WP_MW = HG * 2 * kPS;
+  static constexpr int WP_WORDS = WP_PW + WP_MW;
+  static constexpr int SM_B = 0;                                  // [2] query operands
+  static constexpr int SM_WP = 2 * BBUF_AL;                       // [NCW] value-weight areas
+  static constexpr int SM_RED = SM_WP + NCW * WP_WORDS * 4;       // [NG][4 warps][d] unit-end sums
+  static constexpr int SM_RM = SM_RED + NG * 4 * kD * 4;          // [NG][4][8] warp maxima
+  static constexpr int SM_RL = SM_RM + NG * 4 * 8 * 4;            // [NG][4][8] warp sums of p
+  static constexpr int SM_BAR = SM_RL + NG * 4 * 8 * 4;
+  static constexpr int NBAR = 2 * 12 + NG + 2;
+  static constexpr int SM_MISC = SM_BAR + 8 * NBAR;               // TMEM address, abort flag, grp_unit[NG]
+  static constexpr int SM_RING = (SM_MISC + 8 + 4 * NG + 127) / 128 * 128;
   static constexpr int BUDGET = 227 * 1024 - 1024 - SM_RING;
   static constexpr int NST = BUDGET / STAGE > 8 ? 8 : BUDGET / STAGE;
-  static_assert(NST >= 3 && NST <= 12, "stages");
+  static_assert(NST >= NG + 2 && NST <= 12, "stages");
   static constexpr size_t SMEM = (size_t)SM_RING + (size_t)NST * STAGE + 1024;
   static_assert(SMEM <= 227 * 1024, "shared memory");
   static_assert(STAGE % 16 == 0 && BBUF % 16 == 0, "16-byte bulk copies");
@@ -153,11 +161,18 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, const
   unsigned long long start = 0;
   for (uint32_t it = 0; it < kWaitPolls; ++it) {
     uint32_t done;
-    asm volatile(
-        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
-        : "=r"(done)
-        : "r"(a), "r"(parity), "r"(20000u)
-        : "memory");
+    if constexpr (kTryWaitNs > 0)
+      asm volatile(
+          "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
+          : "=r"(done)
+          : "r"(a), "r"(parity), "r"(kTryWaitNs)
+          : "memory");
+    else
+      asm volatile(
+          "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+          : "=r"(done)
+          : "r"(a), "r"(parity)
+          : "memory");
     if (done) return true;
     if (*abort_flag) return false;
     if (it == 0) start = s1::global_ns();
@@ -195,6 +210,18 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* v) {
       : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
         "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
       : "r"(taddr));
+}
+
+// Warp-wide store of 32 consecutive 32-bit columns of the warp's 32 lanes.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+      "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+      "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
 }
 
 __device__ __forceinline__ void mma16816_tc(float (&d)[4], const uint4& a, uint32_t b0, uint32_t b1) {
@@ -244,11 +271,45 @@ __device__ __forceinline__ uint32_t parity_word(uint32_t x0, uint32_t x1, uint32
   return (X0 & 0x49249249u) | (X1 & 0x92492492u) | (X2 & 0x24924924u);
 }
 
-// Word offset of the value-weight row (group g, head h, part) in a P buffer; groups 2-3 sit
-// 16 words further so that the even and odd threads of a token pair write distinct banks.
+// Word offset of the value-weight row (group g, head h, part) in a warp's area (rows of 20
+// words: 16 token pairs + 4, so that the 8 rows a fragment load touches fall on distinct
+// banks); groups 2-3 sit 16 words further so that the even and odd threads of a token pair
+// write distinct banks.
 __device__ __forceinline__ int prow(int g, int h, int part, int HG) {
-  return ((g * HG + h) * 2 + part) * kPairStride + (g >> 1) * 16;
+  return ((g * HG + h) * 2 + part) * 20 + (g >> 1) * 16;
 }
+
+// Walks a CTA's tiles in order without dividing: the unit, the tile within it, the unit's
+// valid length.
+struct TileWalk {
+  int64_t Tu, max_len;
+  const int32_t* seq_lens;
+  int hkv;
+  int u;
+  int64_t tl, len;
+  __device__ __forceinline__ int64_t unit_len(int uu) const {
+    int64_t l = max_len;
+    if (seq_lens) l = min((int64_t)max(seq_lens[uu / hkv], 0), max_len);
+    return l;
+  }
+  __device__ __forceinline__ void start(int64_t g0) {
+    u = (int)(g0 / Tu);
+    tl = g0 - (int64_t)u * Tu;
+    len = unit_len(u);
+  }
+  __device__ __forceinline__ void next() {
+    if (++tl == Tu) {
+      tl = 0;
+      ++u;
+      len = unit_len(u);
+    }
+  }
+  __device__ __forceinline__ int64_t tok0() const { return tl * kTileTc; }
+  __device__ __forceinline__ int nt() const {
+    return (int)max((int64_t)0, min((int64_t)kTileTc, len - tl * kTileTc));
+  }
+  __device__ __forceinline__ bool last_tile() const { return tl == Tu - 1; }
+};
 
 // CTA owning global tile g when CTA k takes tiles [k T / P, (k + 1) T / P).
 __device__ __forceinline__ int64_t owner_tc(int64_t g, int64_t P, int64_t T) { return ((g + 1) * P - 1) / T; }
@@ -372,22 +433,23 @@ __global__ void __launch_bounds__(kPrepTcThreads) prep_tc_kernel(const __grid_co
   }
   __syncthreads();
   // The B operand: row n (a column of D), byte k = 32 ks + 4 q + i: element i of mask q of
-  // element word ks. Code columns n = 4 h + digit, sign columns NC + 4 h + digit.
+  // element word ks. Code columns n = 4 h + digit, sign columns NC + 4 h + digit. One thread
+  // per (head, element word, mask): the four weights of the word's bytes are quantized once
+  // and their digits stored as one 32-bit word in each of the four digit columns.
   uint8_t* bop = a.bop + (size_t)unit * L::BBUF;
   constexpr int WPR = L::KB / 4;  // 32-bit words per row
-  for (int w = tid; w < L::N * WPR; w += kPrepTcThreads) {
-    const int n = w / WPR, kw = w % WPR;
-    const int ks = kw / 8, q = kw % 8;
-    const bool code_col = n < L::NC, sign_col = QJL && n >= L::NC && n < 2 * L::NC;
-    const int h = code_col ? n / kDigits : (n - L::NC) / kDigits;
-    const int dg = code_col ? n % kDigits : (n - L::NC) % kDigits;
-    const bool live = (code_col && ks < L::KSC) || (sign_col && ks >= L::KSC);
-    uint32_t packed = 0;
-    if (live && h < G) {
+  auto put = [&](int n, int kw, uint32_t word) {
+    *reinterpret_cast<uint32_t*>(bop + s1::sw128_offset(n, 2 * kw, L::N)) = word;
+  };
+  for (int it = tid; it < HG * L::EW * 8; it += kPrepTcThreads) {
+    const int h = it / (L::EW * 8), ks = (it / 8) % L::EW, q = it % 8;
+    const bool code = ks < L::KSC;
+    uint32_t dw[kDigits] = {0u, 0u, 0u, 0u};
+    if (h < G) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         float wgt, e2;
-        if (code_col) {
+        if (code) {
           int j, plane;
           if (ks < L::CW) {
             const int sbit = 32 * ks + 8 * i + q;  // bit of the code stream
@@ -412,38 +474,45 @@ __global__ void __launch_bounds__(kPrepTcThreads) prep_tc_kernel(const __grid_co
         const int Q2 = (Q1 - d1) >> 8;
         const int d2 = ((Q2 + 128) & 255) - 128;
         const int d3 = (Q2 - d2) >> 8;
-        const int dig = dg == 0 ? d0 : dg == 1 ? d1 : dg == 2 ? d2 : d3;
-        packed |= ((uint32_t)dig & 0xffu) << (8 * i);
+        dw[0] |= ((uint32_t)d0 & 0xffu) << (8 * i);
+        dw[1] |= ((uint32_t)d1 & 0xffu) << (8 * i);
+        dw[2] |= ((uint32_t)d2 & 0xffu) << (8 * i);
+        dw[3] |= ((uint32_t)d3 & 0xffu) << (8 * i);
       }
     }
-    *reinterpret_cast<uint32_t*>(bop + s1::sw128_offset(n, 2 * kw, L::N)) = packed;
+    const int kw = 8 * ks + q;
+    const int n_live = (code ? 0 : L::NC) + kDigits * h;  // this word's four columns
+    const int n_dead = (code ? L::NC : 0) + kDigits * h;  // the other kind's columns: zero
+#pragma unroll
+    for (int dgt = 0; dgt < kDigits; ++dgt) {
+      put(n_live + dgt, kw, dw[dgt]);
+      if (QJL) put(n_dead + dgt, kw, 0u);
+    }
   }
+  // padding columns beyond the code and sign columns
+  constexpr int NUSED = QJL ? 2 * L::NC : L::NC;
+  for (int w = tid; w < (L::N - NUSED) * WPR; w += kPrepTcThreads) put(NUSED + w / WPR, w % WPR, 0u);
 }
 
 // ------------------------------------------------------------------ decode kernel
 
 template <int LMB, bool QJL, int VB, int NB>
-__global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_constant__ TcArgs a) {
+__global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
+    decode_tc_kernel(const __grid_constant__ TcArgs a) {
   using L = TcLayout<LMB, QJL, VB, NB>;
-  constexpr int HG = L::HG, NST = L::NST;
+  constexpr int HG = L::HG, NST = L::NST, NG = L::NG;
   constexpr int RS = 4 + kD;  // partial row: m, l, pad, pad, acc[d]
   constexpr float kLn2 = 0.6931471805599453f;
   extern __shared__ unsigned char smem_tc_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(((uintptr_t)smem_tc_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::SM_BAR);
-  uint64_t* full = bars;                 // [NST] stage landed
-  uint64_t* empty = bars + NST;          // [NST] stage consumed (12 warps)
-  uint64_t* afull = bars + 2 * NST;      // [2] key elements written (4 warps)
-  uint64_t* mmad = afull + 2;            // [2] MMA of the tile done (commit)
-  uint64_t* dempty = mmad + 2;           // [2] digit sums read (4 warps)
-  uint64_t* pfull = dempty + 2;          // [2] value weights written (4 warps)
-  uint64_t* pempty = pfull + 2;          // [2] value weights consumed (4 warps)
-  uint64_t* fbfull = pempty + 2;         // [2] query operand landed
-  uint64_t* fbempty = fbfull + 2;        // [2] query operand released (MMA commit + 4 softmax warps)
+  uint64_t* full = bars;            // [NST] stage landed
+  uint64_t* empty = bars + NST;     // [NST] stage consumed by its group (4 warps)
+  uint64_t* mmad = bars + 2 * NST;  // [NG] the group's MMA done (commit)
+  uint64_t* fbfull = mmad + NG;     // [2] query operand landed
   uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + L::SM_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::SM_MISC + 4);
-  int* issued_s = reinterpret_cast<int*>(sm + L::SM_MISC + 8);  // bulk batches into stages (unused slot)
-  (void)issued_s;
+  volatile int* grp_unit = reinterpret_cast<volatile int*>(sm + L::SM_MISC + 8);  // [NG]
   unsigned char* ring = sm + L::SM_RING;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -462,17 +531,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
   if (tid == 32) {
     for (int s = 0; s < NST; ++s) {
       s1::mbar_init(&full[s], 1);
-      s1::mbar_init(&empty[s], 12);
+      s1::mbar_init(&empty[s], 4);
     }
-    for (int b = 0; b < 2; ++b) {
-      s1::mbar_init(&afull[b], 4);
-      s1::mbar_init(&mmad[b], 1);
-      s1::mbar_init(&dempty[b], 4);
-      s1::mbar_init(&pfull[b], 4);
-      s1::mbar_init(&pempty[b], 4);
-      s1::mbar_init(&fbfull[b], 1);
-      s1::mbar_init(&fbempty[b], 5);
+    for (int g = 0; g < NG; ++g) {
+      s1::mbar_init(&mmad[g], 1);
+      grp_unit[g] = -1;
     }
+    s1::mbar_init(&fbfull[0], 1);
+    s1::mbar_init(&fbfull[1], 1);
     *abort_flag = 0;
     s1::mbar_init_fence();
   }
@@ -482,48 +548,37 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
   const uint32_t tmem = *tmem_s;
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  // Per tile i of this CTA: its unit, its first token and its valid token count.
-  auto unit_len = [&](int u) -> int64_t {
-    int64_t len = a.max_len;
-    if (a.seq_lens) len = min((int64_t)max(a.seq_lens[u / a.hkv], 0), a.max_len);
-    return len;
-  };
-  auto tile_info = [&](int i, int& u, int64_t& tok0, int& nt) {
-    const int64_t g = g0 + i;
-    u = (int)(g / Tu);
-    tok0 = (g - (int64_t)u * Tu) * kTileTc;
-    nt = (int)max((int64_t)0, min((int64_t)kTileTc, unit_len(u) - tok0));
-  };
-  auto last_of_unit = [&](int i) -> bool {
-    const int64_t g = g0 + i;
-    return i == ntl - 1 || (g + 1) % Tu == 0;
-  };
+  TileWalk walk;
+  walk.Tu = Tu;
+  walk.max_len = a.max_len;
+  walk.seq_lens = a.seq_lens;
+  walk.hkv = a.hkv;
+  walk.start(g0);
 
   bool failed = false;
-  if (warp == 0) {
-    // ============================================================ producer: packed tiles
+  if (warp == L::NCW) {
+    // ============================================================ producer
     int bulk_issued[12] = {};  // bulk batches issued per stage (for the failure drain)
     int uses[12] = {};         // phases started per stage
+    int b_issued = 0;          // query operands issued (units in order)
     for (int i = 0; i < ntl && !failed; ++i) {
       const int s = i % NST;
       if (i >= NST) {
         bool ok = true;
         if (lane == 0) ok = wait_phase(&empty[s], (uint32_t)((i / NST) - 1) & 1u, abort_flag);
-        ok = __shfl_sync(kFull, ok, 0);
-        if (!ok) {
+        if (!__shfl_sync(kFull, ok, 0)) {
           failed = true;
           break;
         }
       }
-      int u, nt;
-      int64_t tok0;
-      tile_info(i, u, tok0, nt);
+      const int u = walk.u, nt = walk.nt();
+      const int64_t tok0 = walk.tok0();
+      walk.next();
       unsigned char* st = ring + s * L::STAGE;
       uses[s] += 1;
       if (a.use_tma && nt == kTileTc) {
         if (lane == 0) {
-          // the consumers' generic reads of the stage are ordered before the async-proxy writes
-          s1::fence_async_smem();
+          s1::fence_async_smem();  // the consumers' generic reads come before the async writes
           const int64_t v = record_row(a.pg, a.max_len, u, tok0, a.err);
           s1::mbar_expect_tx(&full[s], (uint32_t)L::STAGE);
           s1::bulk_g2s(st + L::OFF_KC, a.k_codes + v * L::KCB, kTileTc * L::KCB, &full[s]);
@@ -552,104 +607,209 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
         __syncwarp();
         if (lane == 0) s1::mbar_arrive(&full[s]);
       }
+      // The query operand of a unit is loaded when its first tile is: into buffer j % 2, once
+      // every group has moved past unit j - 2 (its MMAs done, its constants read).
+      const int j = u - u_first;
+      if (j == b_issued) {
+        bool ok = true;
+        if (lane == 0) {
+          if (b_issued == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
+          if (j >= 2) {
+            const unsigned long long t0 = s1::global_ns();
+            for (uint32_t it = 0;; ++it) {
+              int mn = 0x7fffffff;
+              for (int g = 0; g < NG; ++g) mn = min(mn, grp_unit[g]);
+              if (mn >= j - 1) break;
+              if (*abort_flag || ((it & 63) == 63 && s1::global_ns() - t0 > kWaitNs)) {
+                ok = false;
+                break;
+              }
+              __nanosleep(64);
+            }
+            asm volatile("fence.acq_rel.cta;" ::: "memory");
+          }
+          if (ok) {
+            s1::fence_async_smem();
+            s1::mbar_expect_tx(&fbfull[j & 1], (uint32_t)L::BBUF);
+            s1::bulk_g2s(sm + L::SM_B + (j & 1) * L::BBUF_AL, a.bop + (size_t)(u_first + j) * L::BBUF, L::BBUF,
+                         &fbfull[j & 1]);
+          }
+        }
+        if (!__shfl_sync(kFull, ok, 0)) {
+          failed = true;
+          break;
+        }
+        ++b_issued;
+      }
     }
     if (failed && lane == 0) raise_abort(abort_flag);
     __syncwarp();
-    if (lane == 0 && *abort_flag) {
-      // Consumers may have left before waiting for every stage: let each stage's last batch
-      // land before the shared memory goes away (the phases of one stage complete in order,
-      // and the producer never runs more than one phase ahead of a stage's consumers).
-      for (int s = 0; s < NST; ++s)
-        if (bulk_issued[s] > 0) s1::mbar_wait(&full[s], (uint32_t)(uses[s] - 1) & 1u);
-    }
-  } else if (warp == 1) {
-    // ============================================================ MMA issue
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_u8s8_s32(kTileTc, L::N);
-      int cur = -1;
-      int committed = 0;  // MMA batches committed to mmad (for the drain)
-      for (int i = 0; i < ntl; ++i) {
-        const int b = i & 1;
-        const int j = (int)((g0 + i) / Tu) - u_first;
-        if (j != cur) {
-          cur = j;
-          if (!wait_phase(&fbfull[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag)) {
-            failed = true;
-            break;
-          }
-        }
-        if (!wait_phase(&afull[b], (uint32_t)(i >> 1) & 1u, abort_flag)) {
-          failed = true;
-          break;
-        }
-        if (i >= 2 && !wait_phase(&dempty[b], (uint32_t)((i >> 1) - 1) & 1u, abort_flag)) {
-          failed = true;
-          break;
-        }
-        s1::fence_after_sync();
-        const uint32_t bbase = smem_addr(sm + L::SM_B + (j & 1) * L::BBUF_AL);
+      // copies still in flight land before the shared memory goes away (phases of one
+      // barrier complete in order; at most one phase per stage runs ahead of its consumers)
+      if (*abort_flag)
+        for (int s = 0; s < NST; ++s)
+          if (bulk_issued[s] > 0) s1::mbar_wait(&full[s], (uint32_t)(uses[s] - 1) & 1u);
+      for (int jj = (b_issued > 2 ? b_issued - 2 : 0); jj < b_issued; ++jj)
+        s1::mbar_wait(&fbfull[jj & 1], (uint32_t)(jj >> 1) & 1u);
+    }
+  } else {
+    // ============================================================ compute warps
+    // group gi (warps 4 gi .. 4 gi + 3) takes tiles gi, gi + NG, ...; warp q of the group owns
+    // tokens 32 q .. 32 q + 31 of each tile (tensor-memory lanes 32 q ..)
+    const int gi = warp >> 2, q = warp & 3;
+    const int R = 32 * q + lane;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    const uint32_t tA = tmem + gi * L::TG + lane_base, tD = tA + L::TA;
+    const int bar_id = 1 + gi;
+    const bool leader = q == 0 && lane == 0;
+    const int r = lane >> 2, c = lane & 3;
+    const int part = r & 1, hsel = r >> 1;
+    uint32_t* wp = reinterpret_cast<uint32_t*>(sm + L::SM_WP) + warp * L::WP_WORDS;  // this warp's area
+    uint32_t* wpm = wp + L::WP_PW;
+    float* red = reinterpret_cast<float*>(sm + L::SM_RED) + gi * 4 * kD;  // [4][d]
+    float* rm = reinterpret_cast<float*>(sm + L::SM_RM) + gi * 32;        // [4][8]
+    float* rl = reinterpret_cast<float*>(sm + L::SM_RL) + gi * 32;        // [4][8]
+
+    float Mref[HG], lsum[HG];
+    float dmin[NB][4];
+    float dv[4][2][NB][4];
+    auto reset = [&]() {
 #pragma unroll
-        for (int ks = 0; ks < L::EW; ++ks)
-          umma_i8_ts(tmem + L::TM_D + b * L::N, tmem + b * L::TA + 8 * ks, s1::sw128_desc(bbase, 16 * ks, L::N),
-                     idesc, ks > 0 ? 1u : 0u);
-        s1::umma_commit(&mmad[b]);
-        ++committed;
-        if (last_of_unit(i)) s1::umma_commit(&fbempty[j & 1]);
+      for (int h = 0; h < HG; ++h) {
+        Mref[h] = -INFINITY;
+        lsum[h] = 0.f;
       }
-      if (failed) raise_abort(abort_flag);
-      // the last committed MMAs complete before the tensor memory is freed
-      if (committed > 0) {
-        const int il = committed - 1;
-        s1::mbar_wait(&mmad[il & 1], (uint32_t)(il >> 1) & 1u);
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dmin[nb][e] = 0.f;
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dv[g][hf][nb][e] = 0.f;
       }
-    }
-  } else if (warp == 2) {
-    // ============================================================ query operands
-    if (lane == 0) {
-      asm volatile("griddepcontrol.wait;" ::: "memory");
-      int issued = 0;
-      for (int j = 0; j < n_units; ++j) {
-        if (j >= 2 && !wait_phase(&fbempty[j & 1], (uint32_t)((j >> 1) - 1) & 1u, abort_flag)) {
-          failed = true;
-          break;
+    };
+    auto part_ptr = [&](int j) -> float* {
+      const int u = u_first + j;
+      const int seg = (int)(kcta - owner_tc((int64_t)u * Tu, P, Tt));
+      return a.ws_part + (((size_t)u * a.s_max + seg) * NG + gi) * G * RS;
+    };
+    // a local unit this group has no tile of: an empty partial (m = -inf, l = 0)
+    auto mark_empty = [&](int j) {
+      if (q == 0 && lane < G) {
+        float* pp = part_ptr(j);
+        pp[lane * RS + 0] = -INFINITY;
+        pp[lane * RS + 1] = 0.f;
+      }
+    };
+    // End of local unit j for this group: the four warps' sums, rescaled to the group's
+    // maximum and added in warp order, are the group's partial (m, l, acc) of the unit.
+    auto finish = [&](int j) {
+      float* pp = part_ptr(j);
+#pragma unroll
+      for (int h = 0; h < HG; ++h) {
+        const float l = warp_sum(lsum[h]);
+        if (lane == 0) {
+          rm[q * 8 + h] = failed ? -INFINITY : Mref[h];
+          rl[q * 8 + h] = failed ? 0.f : l;
         }
-        s1::fence_async_smem();  // generic reads of the buffer's constants come first
-        s1::mbar_expect_tx(&fbfull[j & 1], (uint32_t)L::BBUF);
-        s1::bulk_g2s(sm + L::SM_B + (j & 1) * L::BBUF_AL, a.bop + (size_t)(u_first + j) * L::BBUF, L::BBUF,
-                     &fbfull[j & 1]);
-        ++issued;
       }
-      if (failed) raise_abort(abort_flag);
-      // drain: the copies issued land before the shared memory goes away
-      for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j)
-        s1::mbar_wait(&fbfull[j & 1], (uint32_t)(j >> 1) & 1u);
-    }
-  } else if (warp >= 4 && warp < 8) {
-    // ============================================================ key bits -> tensor memory
-    const int kw = warp - 4, R = 32 * kw + lane;
-    const uint32_t lane_base = (uint32_t)(32 * kw) << 16;
-    for (int i = 0; i < ntl; ++i) {
-      const int s = i % NST, b = i & 1;
-      if (!wait_phase(&full[s], (uint32_t)(i / NST) & 1u, abort_flag)) {
-        failed = true;
-        break;
+      named_sync(bar_id, 128);
+      if (q == 0 && lane < G) {
+        const int h = lane;
+        float M = -INFINITY;
+        for (int w = 0; w < 4; ++w) M = fmaxf(M, rm[w * 8 + h]);
+        float Ls = 0.f;
+        for (int w = 0; w < 4; ++w) {
+          const float mw = rm[w * 8 + h];
+          if (mw != -INFINITY) Ls = fmaf(ex2f(mw - M), rl[w * 8 + h], Ls);
+        }
+        pp[h * RS + 0] = M;
+        pp[h * RS + 1] = Ls;
       }
-      if (i >= 2 && !wait_phase(&mmad[b], (uint32_t)((i >> 1) - 1) & 1u, abort_flag)) {
-        failed = true;
-        break;
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+        const float own = dmin[nb][0] + dmin[nb][1];
+        float mt[4];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) mt[g] = __shfl_sync(kFull, own, 4 * g + c);
+        const int hme = c + 4 * nb;
+        float Mg = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) Mg = fmaxf(Mg, rm[w * 8 + hme]);
+        float mme = rm[q * 8 + hme];
+        const float wsc = (failed || mme == -INFINITY) ? 0.f : ex2f(mme - Mg);
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const int h = 4 * nb + c4;
+          if (h >= G) break;  // uniform
+          if (c == c4) {
+            float* rq = red + q * kD;
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+#pragma unroll
+              for (int hf = 0; hf < 2; ++hf) {
+                const float* d = dv[g][hf][nb];
+                int j0;
+                float v0, v1;
+                if (VB == 2) {
+                  j0 = 4 * (8 * g + r) + 2 * hf;
+                  v0 = (d[0] + d[1]) * ldexpf(1.f, 24 - 4 * hf) + mt[g];
+                  v1 = (d[2] + d[3]) * ldexpf(1.f, 22 - 4 * hf) + mt[g];
+                } else {
+                  j0 = 2 * (16 * g + 8 * hf + r);
+                  v0 = (d[0] + d[1]) * 16777216.f + mt[g];
+                  v1 = (d[2] + d[3]) * 1048576.f + mt[g];
+                }
+                rq[j0] = wsc != 0.f ? wsc * v0 : 0.f;
+                rq[j0 + 1] = wsc != 0.f ? wsc * v1 : 0.f;
+              }
+          }
+          named_sync(bar_id, 128);
+          pp[h * RS + 4 + R] = ((red[R] + red[kD + R]) + red[2 * kD + R]) + red[3 * kD + R];
+          named_sync(bar_id, 128);
+        }
       }
-      s1::fence_after_sync();
+    };
+
+    for (int k = 0; k < gi; ++k) walk.next();
+    reset();
+    int cur = -1, qrow0 = 0, kt = 0;  // local unit, its first query row, tiles of this group so far
+    for (int i = gi; i < ntl; i += NG, ++kt) {
+      const int s = i % NST;
+      const int u = walk.u, nt = walk.nt();
+      const int64_t tok0 = walk.tok0();
+      for (int k = 0; k < NG; ++k) walk.next();
+      const int j = u - u_first;
+      if (j != cur) {
+        if (cur >= 0) finish(cur);
+        for (int jj = cur + 1; jj < j; ++jj) mark_empty(jj);
+        cur = j;
+        reset();
+        const int bq = u / a.hkv, kvh = u - bq * a.hkv;
+        qrow0 = bq * a.hq + kvh * G;
+        if (leader) {
+          // every warp of the group is past its previous unit: its query operand may be reloaded
+          asm volatile("fence.acq_rel.cta;" ::: "memory");
+          grp_unit[gi] = j;
+        }
+        if (!failed && !wait_phase(&fbfull[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag)) failed = true;
+      }
+      if (!failed && !wait_phase(&full[s], (uint32_t)(i / NST) & 1u, abort_flag)) failed = true;
       const unsigned char* st = ring + s * L::STAGE;
-      uint32_t w[L::EW];
+      // ---- key bits -> unsigned 8-bit elements in tensor memory (row R of the A operand)
       {
+        uint32_t w[L::EW];
         const uint4* kc = reinterpret_cast<const uint4*>(st + L::OFF_KC + R * L::KCB);
 #pragma unroll
-        for (int c = 0; c < LMB; ++c) {
-          const uint4 v = kc[c];
-          w[4 * c] = v.x;
-          w[4 * c + 1] = v.y;
-          w[4 * c + 2] = v.z;
-          w[4 * c + 3] = v.w;
+        for (int cc = 0; cc < LMB; ++cc) {
+          const uint4 v = kc[cc];
+          w[4 * cc] = v.x;
+          w[4 * cc + 1] = v.y;
+          w[4 * cc + 2] = v.z;
+          w[4 * cc + 3] = v.w;
         }
         if constexpr (QJL) {
           const uint4 v = *reinterpret_cast<const uint4*>(st + L::OFF_KS + R * L::SB);
@@ -658,114 +818,61 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
           w[L::KSC + 2] = v.z;
           w[L::KSC + 3] = v.w;
         }
-      }
-      __syncwarp();
-      if (lane == 0) s1::mbar_arrive(&empty[s]);  // the stage's key bytes are in registers
-      if constexpr (LMB == 3) {
+        if constexpr (LMB == 3) {
 #pragma unroll
-        for (int gq = 0; gq < 4; ++gq) w[L::CW + gq] = parity_word(w[3 * gq], w[3 * gq + 1], w[3 * gq + 2]);
-      }
-      const uint32_t abase = tmem + b * L::TA + lane_base;
+          for (int gq = 0; gq < 4; ++gq) w[L::CW + gq] = parity_word(w[3 * gq], w[3 * gq + 1], w[3 * gq + 2]);
+        }
+        static_assert(L::EW % 4 == 0, "element words in groups of four");
 #pragma unroll
-      for (int e = 0; e < L::EW; ++e) {
-        const uint32_t x = w[e], x4 = x >> 4;
-        uint32_t m[8];
-        m[0] = bitmask_el<0>(x, x4);
-        m[1] = bitmask_el<1>(x, x4);
-        m[2] = bitmask_el<2>(x, x4);
-        m[3] = bitmask_el<3>(x, x4);
-        m[4] = bitmask_el<4>(x, x4);
-        m[5] = bitmask_el<5>(x, x4);
-        m[6] = bitmask_el<6>(x, x4);
-        m[7] = bitmask_el<7>(x, x4);
-        s1::tmem_st8(abase + 8 * e, m);
+        for (int e4 = 0; e4 < L::EW / 4; ++e4) {
+          uint32_t m[32];  // four element words x eight masks: 32 tensor-memory columns
+#pragma unroll
+          for (int ee = 0; ee < 4; ++ee) {
+            const uint32_t x = w[4 * e4 + ee], x4 = x >> 4;
+            m[8 * ee + 0] = bitmask_el<0>(x, x4);
+            m[8 * ee + 1] = bitmask_el<1>(x, x4);
+            m[8 * ee + 2] = bitmask_el<2>(x, x4);
+            m[8 * ee + 3] = bitmask_el<3>(x, x4);
+            m[8 * ee + 4] = bitmask_el<4>(x, x4);
+            m[8 * ee + 5] = bitmask_el<5>(x, x4);
+            m[8 * ee + 6] = bitmask_el<6>(x, x4);
+            m[8 * ee + 7] = bitmask_el<7>(x, x4);
+          }
+          tmem_st32(tA + 32 * e4, m);
+        }
+        s1::tmem_st_wait();
       }
-      s1::tmem_st_wait();
       s1::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) s1::mbar_arrive(&afull[b]);
-    }
-    if (failed && lane == 0) raise_abort(abort_flag);
-  } else if (warp >= 8 && warp < 12) {
-    // ============================================================ scores, online softmax
-    const int sw = warp - 8, R = 32 * sw + lane;
-    const uint32_t lane_base = (uint32_t)(32 * sw) << 16;
-    float* lred = reinterpret_cast<float*>(sm + L::SM_LR);   // [HG][128]
-    float* tmx = reinterpret_cast<float*>(sm + L::SM_TMX);   // [4][HG]
-    float Mref[HG], lsum[HG];
+      named_sync(bar_id, 128);  // all four quarters of the tile's A operand are written
+      if (leader) {
+        s1::fence_after_sync();
+        if (!failed) {
+          constexpr uint32_t idesc = idesc_u8s8_s32(kTileTc, L::N);
+          const uint32_t bbase = smem_addr(sm + L::SM_B + (j & 1) * L::BBUF_AL);
+          const uint32_t d_tm = tmem + gi * L::TG + L::TA;
+          const uint32_t a_tm = tmem + gi * L::TG;
 #pragma unroll
-    for (int h = 0; h < HG; ++h) {
-      Mref[h] = -INFINITY;
-      lsum[h] = 0.f;
-    }
-    int cur = -1, qrow0 = 0;
-    // End of local unit j: the CTA's (m, l) of each query head, l summed over the 128
-    // threads in a fixed order; then the unit's query operand is released.
-    auto finish_sm = [&](int j) {
-      const int u = u_first + j;
-      const int seg = (int)(kcta - owner_tc((int64_t)u * Tu, P, Tt));
-      float* part = a.ws_part + ((size_t)u * a.s_max + seg) * G * RS;
-#pragma unroll
-      for (int h = 0; h < HG; ++h) lred[h * kTileTc + R] = lsum[h];
-      named_sync(kBarSm, 128);
-#pragma unroll
-      for (int h = 0; h < HG; ++h) {
-        if (R == h && h < G) {
-          float l = 0.f;
-          for (int t = 0; t < kTileTc; ++t) l += lred[h * kTileTc + t];
-          part[h * RS + 0] = failed ? -INFINITY : Mref[h];
-          part[h * RS + 1] = failed ? 0.f : l;
+          for (int ks = 0; ks < L::EW; ++ks)
+            umma_i8_ts(d_tm, a_tm + 8 * ks, s1::sw128_desc(bbase, 16 * ks, L::N), idesc, ks > 0 ? 1u : 0u);
+          s1::umma_commit(&mmad[gi]);
         }
       }
-      named_sync(kBarSm, 128);
-      __syncwarp();
-      if (lane == 0) s1::mbar_arrive(&fbempty[j & 1]);
-    };
-    for (int i = 0; i < ntl; ++i) {
-      const int s = i % NST, b = i & 1, pb = i & 1;
-      int u, nt;
-      int64_t tok0;
-      tile_info(i, u, tok0, nt);
-      const int j = u - u_first;
-      if (j != cur) {
-        cur = j;
-#pragma unroll
-        for (int h = 0; h < HG; ++h) {
-          Mref[h] = -INFINITY;
-          lsum[h] = 0.f;
-        }
-        const int bq = u / a.hkv, kvh = u - bq * a.hkv;
-        qrow0 = bq * a.hq + kvh * G;
-        if (!failed && !wait_phase(&fbfull[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag)) failed = true;
-      }
-      if (!failed && !wait_phase(&mmad[b], (uint32_t)(i >> 1) & 1u, abort_flag)) failed = true;
-      if (!failed && !wait_phase(&full[s], (uint32_t)(i / NST) & 1u, abort_flag)) failed = true;
-      if (!failed && i >= 2 && !wait_phase(&pempty[pb], (uint32_t)((i >> 1) - 1) & 1u, abort_flag)) failed = true;
-      // the four softmax warps share named barriers: they leave together or not at all
-      if (named_sync_or(kBarSm, 128, failed)) {
-        failed = true;
-        break;
-      }
+      if (!failed && !wait_phase(&mmad[gi], (uint32_t)kt & 1u, abort_flag)) failed = true;
       s1::fence_after_sync();
       uint32_t dsum[L::N];
 #pragma unroll
-      for (int c = 0; c < L::N; c += 16) tmem_ld16(tmem + L::TM_D + b * L::N + c + lane_base, dsum + c);
+      for (int cc = 0; cc < L::N; cc += 16) tmem_ld16(tD + cc, dsum + cc);
       s1::tmem_ld_wait();
-      s1::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) s1::mbar_arrive(&dempty[b]);
-      const unsigned char* st = ring + s * L::STAGE;
-      const bool valid = R < nt;
+      // ---- logits and online softmax (per warp: its 32 tokens, one per lane)
+      const bool valid = R < nt && !failed;
       const uint32_t ngw = *reinterpret_cast<const uint32_t*>(st + L::OFF_KN + 4 * R);
       const uint4 vpar = *reinterpret_cast<const uint4*>(st + L::OFF_VP + 16 * R);
-      __syncwarp();
-      if (lane == 0) s1::mbar_arrive(&empty[s]);
       const float2 ng = __half22float2(h2of(ngw));  // (n, gamma)
-      const float4* kc = reinterpret_cast<const float4*>(sm + L::SM_B + (j & 1) * L::BBUF_AL + L::BOP);
+      const float4* kc4 = reinterpret_cast<const float4*>(sm + L::SM_B + (j & 1) * L::BBUF_AL + L::BOP);
       float lg[HG];
 #pragma unroll
       for (int h = 0; h < HG; ++h) {
-        const float4 k = kc[h];
+        const float4 k = kc4[h];
         // digit sums recombined: (s0 + 2^8 s1) + 2^16 (s2 + 2^8 s3), each part an exact int
         const int c0 = kDigits * h;
         const float code = (float)((int)dsum[c0] + ((int)dsum[c0 + 1] << 8)) +
@@ -784,186 +891,27 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
         for (int h = 0; h < HG; ++h)
           if (h < G) a.scores[(size_t)(qrow0 + h) * a.max_len + tok0 + R] = lg[h] * kLn2;
       }
-      // Lazy rescale: the reference maxima move only when a logit exceeds them by more than
-      // the slack; all 128 softmax threads take the same decision.
+      // Lazy rescale: the warp's reference maxima move only when a logit exceeds them by more
+      // than the slack.
       bool need = false;
 #pragma unroll
       for (int h = 0; h < HG; ++h) need |= lg[h] > Mref[h] + kSlackTc;
-      need = named_sync_or(kBarSm, 128, need);
-      float corr[HG];
-#pragma unroll
-      for (int h = 0; h < HG; ++h) corr[h] = 1.f;
-      if (need) {
+      if (__any_sync(kFull, need)) {
+        float corr[HG];
 #pragma unroll
         for (int h = 0; h < HG; ++h) {
-          const float m = warp_max(lg[h]);
-          if (lane == 0) tmx[sw * HG + h] = m;
-        }
-        named_sync(kBarSm, 128);
-#pragma unroll
-        for (int h = 0; h < HG; ++h) {
-          const float tm = fmaxf(fmaxf(tmx[h], tmx[HG + h]), fmaxf(tmx[2 * HG + h], tmx[3 * HG + h]));
-          const float Mn = fmaxf(Mref[h], tm);
+          const float Mn = fmaxf(Mref[h], warp_max(lg[h]));
+          corr[h] = 1.f;
           if (Mn > Mref[h]) {
             corr[h] = Mref[h] == -INFINITY ? 0.f : ex2f(Mref[h] - Mn);
             lsum[h] *= corr[h];
             Mref[h] = Mn;
           }
         }
-      }
-      // p of this token per head, split in f16 hi + lo
-      uint32_t own[HG];  // (p_hi, p_lo) of this token
-#pragma unroll
-      for (int h = 0; h < HG; ++h) {
-        const float p = lg[h] == -INFINITY ? 0.f : ex2f(lg[h] - Mref[h]);
-        lsum[h] += p;
-        const __half hi = __float2half_rn(p);
-        const __half lo = __float2half_rn(p - __half2float(hi));
-        own[h] = (uint32_t)__half_as_ushort(hi) | ((uint32_t)__half_as_ushort(lo) << 16);
-      }
-      // value weights of the token pair (t even, t odd): the even thread writes groups 0-1,
-      // the odd thread groups 2-3 (and the minima's p of the first / second half of the heads)
-      const bool odd = (lane & 1) != 0;
-      uint32_t par[HG];
-#pragma unroll
-      for (int h = 0; h < HG; ++h) par[h] = __shfl_xor_sync(kFull, own[h], 1);
-      const uint32_t sc[4] = {valid ? vpar.x : 0u, valid ? vpar.y : 0u, valid ? vpar.z : 0u, valid ? vpar.w : 0u};
-      // send the partner the (scale, min) words of its two groups, receive ours
-      const uint32_t send0 = odd ? sc[0] : sc[2], send1 = odd ? sc[1] : sc[3];
-      const uint32_t got0 = __shfl_xor_sync(kFull, send0, 1), got1 = __shfl_xor_sync(kFull, send1, 1);
-      uint32_t* pw = reinterpret_cast<uint32_t*>(sm + L::SM_P + pb * L::PBUF);
-      const int pair = R >> 1;
-#pragma unroll
-      for (int gg = 0; gg < 2; ++gg) {
-        const int g = odd ? 2 + gg : gg;
-        const uint32_t mine = odd ? sc[2 + gg] : sc[gg];
-        const uint32_t other = gg == 0 ? got0 : got1;
-        // scales (low halves) of the even and the odd token
-        const uint32_t s2w = odd ? __byte_perm(other, mine, 0x5410) : __byte_perm(mine, other, 0x5410);
-        const __half2 s2 = h2of(s2w);
-#pragma unroll
-        for (int h = 0; h < HG; ++h) {
-          const uint32_t ev = odd ? par[h] : own[h], ov = odd ? own[h] : par[h];
-          const __half2 ph = h2of(__byte_perm(ev, ov, 0x5410));  // p_hi of (even, odd)
-          const __half2 pl = h2of(__byte_perm(ev, ov, 0x7632));  // p_lo of (even, odd)
-          const __half2 hi = __hmul2(ph, s2);
-          const __half2 err = __hfma2(ph, s2, __hneg2(hi));
-          const __half2 lo = __hfma2(pl, s2, err);
-          pw[prow(g, h, 0, HG) + pair] = hbits(hi);
-          pw[prow(g, h, 1, HG) + pair] = hbits(lo);
-        }
-      }
-      uint32_t* pmw = pw + L::PPW;
-#pragma unroll
-      for (int hh = 0; hh < HG / 2; ++hh) {
-        const int h = odd ? HG / 2 + hh : hh;
-        const uint32_t ev = odd ? par[h] : own[h], ov = odd ? own[h] : par[h];
-        pmw[(h * 2 + 0) * kPairStride + pair] = __byte_perm(ev, ov, 0x5410);
-        pmw[(h * 2 + 1) * kPairStride + pair] = __byte_perm(ev, ov, 0x7632);
-      }
-      if (R == 0) {
-        float* hdr = reinterpret_cast<float*>(pw + L::PPW + L::PMW);
-        hdr[0] = need ? 1.f : 0.f;
-#pragma unroll
-        for (int h = 0; h < HG; ++h) hdr[1 + h] = corr[h];
-      }
-      __syncwarp();
-      if (lane == 0) s1::mbar_arrive(&pfull[pb]);
-      if (last_of_unit(i)) finish_sm(j);
-    }
-    if (failed) {
-      if (lane == 0) raise_abort(abort_flag);
-    }
-  } else if (warp >= 12) {
-    // ============================================================ values
-    const int vw = warp - 12;
-    const int r = lane >> 2, c = lane & 3;
-    const int part = r & 1, hsel = r >> 1;
-    float* vred = reinterpret_cast<float*>(sm + L::SM_VR);  // [4][HG][d]
-    float dmin[NB][4];
-    float dv[4][2][NB][4];
-    auto reset = [&]() {
-#pragma unroll
-      for (int nb = 0; nb < NB; ++nb) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dmin[nb][e] = 0.f;
-#pragma unroll
-        for (int g = 0; g < 4; ++g)
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) dv[g][hf][nb][e] = 0.f;
-      }
-    };
-    reset();
-    int cur = -1;
-    // End of local unit j: the four value warps' sums, added in warp order, are the CTA's
-    // acc of each head (all warps share the softmax role's reference maxima).
-    auto finish_v = [&](int j) {
-      const int u = u_first + j;
-      const int seg = (int)(kcta - owner_tc((int64_t)u * Tu, P, Tt));
-      float* partp = a.ws_part + ((size_t)u * a.s_max + seg) * G * RS;
-#pragma unroll
-      for (int nb = 0; nb < NB; ++nb) {
-        const float own = dmin[nb][0] + dmin[nb][1];
-        float mt[4];
-#pragma unroll
-        for (int g = 0; g < 4; ++g) mt[g] = __shfl_sync(kFull, own, 4 * g + c);
-        float* red = vred + (vw * HG + c + 4 * nb) * kD;
-#pragma unroll
-        for (int g = 0; g < 4; ++g)
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            const float* d = dv[g][hf][nb];
-            int j0;
-            float v0, v1;
-            if (VB == 2) {
-              j0 = 4 * (8 * g + r) + 2 * hf;
-              v0 = (d[0] + d[1]) * ldexpf(1.f, 24 - 4 * hf) + mt[g];
-              v1 = (d[2] + d[3]) * ldexpf(1.f, 22 - 4 * hf) + mt[g];
-            } else {
-              j0 = 2 * (16 * g + 8 * hf + r);
-              v0 = (d[0] + d[1]) * 16777216.f + mt[g];
-              v1 = (d[2] + d[3]) * 1048576.f + mt[g];
-            }
-            red[j0] = failed ? 0.f : v0;
-            red[j0 + 1] = failed ? 0.f : v1;
-          }
-      }
-      named_sync(kBarV, 128);
-      const int t = tid - 12 * 32;  // 0..127: one coordinate per thread
-#pragma unroll
-      for (int h = 0; h < HG; ++h) {
-        if (h < G) {
-          const float acc = ((vred[(0 * HG + h) * kD + t] + vred[(1 * HG + h) * kD + t]) +
-                             vred[(2 * HG + h) * kD + t]) + vred[(3 * HG + h) * kD + t];
-          partp[h * RS + 4 + t] = acc;
-        }
-      }
-      named_sync(kBarV, 128);
-      reset();
-    };
-    for (int i = 0; i < ntl; ++i) {
-      const int s = i % NST, pb = i & 1;
-      int u, nt;
-      int64_t tok0;
-      tile_info(i, u, tok0, nt);
-      const int j = u - u_first;
-      if (j != cur) cur = j;
-      if (!failed && !wait_phase(&pfull[pb], (uint32_t)(i >> 1) & 1u, abort_flag)) failed = true;
-      if (!failed && !wait_phase(&full[s], (uint32_t)(i / NST) & 1u, abort_flag)) failed = true;
-      // the four value warps share named barriers: they leave together or not at all
-      if (named_sync_or(kBarV, 128, failed)) {
-        failed = true;
-        break;
-      }
-      const uint32_t* pw = reinterpret_cast<const uint32_t*>(sm + L::SM_P + pb * L::PBUF);
-      const uint32_t* pmw = pw + L::PPW;
-      const float* hdr = reinterpret_cast<const float*>(pw + L::PPW + L::PMW);
-      if (hdr[0] != 0.f) {
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) {
-          const float cf = hdr[1 + c + 4 * nb];
+          const float cf = c == 0 ? corr[4 * nb] : c == 1 ? corr[4 * nb + 1] : c == 2 ? corr[4 * nb + 2]
+                                                                                      : corr[4 * nb + 3];
 #pragma unroll
           for (int e = 0; e < 4; ++e) dmin[nb][e] *= cf;
 #pragma unroll
@@ -974,18 +922,66 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
               for (int e = 0; e < 4; ++e) dv[g][hf][nb][e] *= cf;
         }
       }
-      const unsigned char* st = ring + s * L::STAGE;
+      // p per head, split in f16 hi + lo
+      uint32_t own[HG];
+#pragma unroll
+      for (int h = 0; h < HG; ++h) {
+        const float p = lg[h] == -INFINITY ? 0.f : ex2f(lg[h] - Mref[h]);
+        lsum[h] += p;
+        const __half hi = __float2half_rn(p);
+        const __half lo = __float2half_rn(p - __half2float(hi));
+        own[h] = (uint32_t)__half_as_ushort(hi) | ((uint32_t)__half_as_ushort(lo) << 16);
+      }
+      // value weights of the token pair (even, odd lane): the even lane writes groups 0-1,
+      // the odd lane groups 2-3, and the minima's p of the first / second half of the heads
+      {
+        const bool odd = (lane & 1) != 0;
+        uint32_t par[HG];
+#pragma unroll
+        for (int h = 0; h < HG; ++h) par[h] = __shfl_xor_sync(kFull, own[h], 1);
+        const uint32_t sc[4] = {valid ? vpar.x : 0u, valid ? vpar.y : 0u, valid ? vpar.z : 0u,
+                                valid ? vpar.w : 0u};
+        const uint32_t send0 = odd ? sc[0] : sc[2], send1 = odd ? sc[1] : sc[3];
+        const uint32_t got0 = __shfl_xor_sync(kFull, send0, 1), got1 = __shfl_xor_sync(kFull, send1, 1);
+        const int pair = lane >> 1;
+#pragma unroll
+        for (int gg = 0; gg < 2; ++gg) {
+          const int g = odd ? 2 + gg : gg;
+          const uint32_t mine = odd ? sc[2 + gg] : sc[gg];
+          const uint32_t other = gg == 0 ? got0 : got1;
+          const uint32_t s2w = odd ? __byte_perm(other, mine, 0x5410) : __byte_perm(mine, other, 0x5410);
+          const __half2 s2 = h2of(s2w);
+#pragma unroll
+          for (int h = 0; h < HG; ++h) {
+            const uint32_t ev = odd ? par[h] : own[h], ov = odd ? own[h] : par[h];
+            const __half2 ph = h2of(__byte_perm(ev, ov, 0x5410));  // p_hi of (even, odd)
+            const __half2 pl = h2of(__byte_perm(ev, ov, 0x7632));  // p_lo of (even, odd)
+            const __half2 hi = __hmul2(ph, s2);
+            const __half2 err = __hfma2(ph, s2, __hneg2(hi));
+            const __half2 lo = __hfma2(pl, s2, err);
+            wp[prow(g, h, 0, HG) + pair] = hbits(hi);
+            wp[prow(g, h, 1, HG) + pair] = hbits(lo);
+          }
+        }
+#pragma unroll
+        for (int hh = 0; hh < HG / 2; ++hh) {
+          const int h = odd ? HG / 2 + hh : hh;
+          const uint32_t ev = odd ? par[h] : own[h], ov = odd ? own[h] : par[h];
+          wpm[(h * 2 + 0) * 20 + pair] = __byte_perm(ev, ov, 0x5410);
+          wpm[(h * 2 + 1) * 20 + pair] = __byte_perm(ev, ov, 0x7632);
+        }
+      }
+      __syncwarp();
+      // ---- values of the warp's 32 tokens: two blocks of 16 (mma.sync, k = tokens)
       const uint32_t* vc = reinterpret_cast<const uint32_t*>(st + L::OFF_VC);
       const uint32_t* vpw = reinterpret_cast<const uint32_t*>(st + L::OFF_VP);
-#pragma unroll
+#pragma unroll 1
       for (int mb = 0; mb < 2; ++mb) {
-        const int tb = 32 * vw + 16 * mb;  // first token of the block within the tile
-        if (tb >= nt) break;              // warp-uniform
+        const int tb = 32 * q + 16 * mb;  // first token of the block within the tile
+        if (tb >= nt || failed) break;    // warp-uniform
         const int nv = nt - tb;
-        // k = token - tb: lane (r, c) holds tokens tb + 2c, 2c + 1 (a0/a1) and tb + 2c + 8, 2c + 9 (a2/a3)
         const int tA0 = tb + 2 * c, tA1 = tA0 + 1, tB0 = tA0 + 8, tB1 = tA0 + 9;
-        const int pA = (tb >> 1) + c, pB = pA + 4;  // token pairs of b0 and b1
-        // ---- minima: rows g < 4 = group minima of the k tokens; B = p (hi / lo)
+        const int pA = 8 * mb + c, pB = pA + 4;  // token pairs of b0 and b1 in the warp's area
         {
           uint32_t mA0 = 0u, mA1 = 0u, mB0 = 0u, mB1 = 0u;
           if (r < 4) {
@@ -1001,8 +997,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
           am.w = 0u;
 #pragma unroll
           for (int nb = 0; nb < NB; ++nb) {
-            const int row = ((4 * nb + hsel) * 2 + part) * kPairStride;
-            mma16816_tc(dmin[nb], am, pmw[row + pA], pmw[row + pB]);
+            const int row = ((4 * nb + hsel) * 2 + part) * 20;
+            mma16816_tc(dmin[nb], am, wpm[row + pA], wpm[row + pB]);
           }
         }
         const uint32_t sel = (uint32_t)(r & 3) | ((uint32_t)(4 + (r & 3)) << 8);
@@ -1012,8 +1008,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
 #pragma unroll
           for (int nb = 0; nb < NB; ++nb) {
             const int row = prow(g, 4 * nb + hsel, part, HG);
-            bA[nb] = pw[row + pA];
-            bB[nb] = pw[row + pB];
+            bA[nb] = wp[row + pA];
+            bB[nb] = wp[row + pB];
           }
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
@@ -1040,20 +1036,17 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
         }
       }
       __syncwarp();
-      if (lane == 0) {
-        s1::mbar_arrive(&pempty[pb]);
-        s1::mbar_arrive(&empty[s]);
-      }
-      if (last_of_unit(i)) finish_v(j);
+      if (lane == 0) s1::mbar_arrive(&empty[s]);
     }
+    if (cur >= 0) finish(cur);
+    for (int jj = cur + 1; jj < n_units; ++jj) mark_empty(jj);
+    if (leader) grp_unit[gi] = 0x7fffffff;  // done: the producer may reload any buffer
     if (failed && lane == 0) raise_abort(abort_flag);
   }
 
   // ---------------------------------------------------------------- end
   __syncthreads();
-  if (*abort_flag) {
-    if (tid == 0) atomicOr(a.err, 1u);
-  }
+  if (tid == 0 && *abort_flag) atomicOr(a.err, 1u);
   s1::fence_before_sync();
   __syncthreads();
   if (warp == 0) {
@@ -1080,7 +1073,7 @@ cudaError_t launch_tc_t(const tq_ctx* ctx, const PrepTcArgs& pa, int units, cons
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)n_ctas);
-  cfg.blockDim = dim3(kThreadsTc);
+  cfg.blockDim = dim3(L::THREADS);
   cfg.dynamicSmemBytes = L::SMEM;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -1106,6 +1099,12 @@ cudaError_t launch_tc_vb(const tq_ctx* ctx, const PrepTcArgs& pa, int units, con
                          int vb, cudaStream_t s) {
   return vb == 2 ? launch_tc_nb<LMB, QJL, 2>(ctx, pa, units, a, n_ctas, nb, s)
                  : launch_tc_nb<LMB, QJL, 4>(ctx, pa, units, a, n_ctas, nb, s);
+}
+
+template <int LMB, bool QJL>
+int tc_groups_t(int nb, int vb) {
+  if (vb == 2) return nb == 1 ? TcLayout<LMB, QJL, 2, 1>::NG : TcLayout<LMB, QJL, 2, 2>::NG;
+  return nb == 1 ? TcLayout<LMB, QJL, 4, 1>::NG : TcLayout<LMB, QJL, 4, 2>::NG;
 }
 
 template <int LMB, bool QJL>
@@ -1158,6 +1157,16 @@ bool tc_decode_supported(const tq_ctx* ctx, int G) {
   if (!(sh.v_bits == 2 || sh.v_bits == 4)) return false;
   float kappa, beta[4];
   return codebook_bits(ctx->cb, sh.lm_bits, kappa, beta);
+}
+
+int tc_groups(const tq_ctx* ctx, int G) {
+  const int nb = G <= 4 ? 1 : 2, vb = ctx->shape.v_bits;
+  const bool qjl = ctx->shape.m > 0;
+  switch (ctx->shape.lm_bits) {
+    case 1: return qjl ? tc_groups_t<1, true>(nb, vb) : tc_groups_t<1, false>(nb, vb);
+    case 2: return qjl ? tc_groups_t<2, true>(nb, vb) : tc_groups_t<2, false>(nb, vb);
+    default: return qjl ? tc_groups_t<3, true>(nb, vb) : tc_groups_t<3, false>(nb, vb);
+  }
 }
 
 size_t tc_operand_bytes(const tq_ctx* ctx, int G) {
@@ -1231,8 +1240,8 @@ cudaError_t launch_decode_tc(const tq_ctx* ctx, const DecodePlan& plan, const vo
               : launch_tc_vb<3, false>(ctx, pa, units, a, plan.n_ctas, nb, vb, stream);
   }
   if (e != cudaSuccess) return e;
-  return launch_combine_partials(part, out, lse, batch, hq, hkv, G, plan.s_max, plan.tiles_per_unit,
-                                 plan.total_tiles, plan.n_ctas, stream);
+  return launch_combine_partials(part, out, lse, batch, hq, hkv, G, plan.s_max, tc_groups(ctx, G),
+                                 plan.tiles_per_unit, plan.total_tiles, plan.n_ctas, stream);
 }
 
 }  // namespace tq

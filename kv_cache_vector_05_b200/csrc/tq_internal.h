@@ -99,6 +99,7 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const void*
 bool mma_decode_supported(const tq_ctx* ctx, int G);
 bool tc_decode_supported(const tq_ctx* ctx, int G);
 size_t tc_operand_bytes(const tq_ctx* ctx, int G);  // query operand bytes per (sequence, KV head)
+int tc_groups(const tq_ctx* ctx, int G);            // warp groups (partials per CTA and unit)
 
 cudaError_t launch_decode_tc(const tq_ctx* ctx, const DecodePlan& plan, const void* q, int q_dtype, int batch,
                              int hq, int hkv, const int32_t* seq_lens, int64_t max_len, const Paging& pg,
@@ -106,11 +107,12 @@ cudaError_t launch_decode_tc(const tq_ctx* ctx, const DecodePlan& plan, const vo
                              const uint8_t* v_codes, const uint16_t* v_params, float scale, float* scores,
                              float* out, float* lse, void* workspace, cudaStream_t stream);
 
-// Log-sum-exp merge of the CTA partials [units][s_max][G][4 + 128] (m, l in base 2, acc) of
-// the tile-split decode kernels into out (and lse), launched as a programmatic dependent of
-// the decode grid (decode_mma.cu).
+// Log-sum-exp merge of the partials [units][s_max][ppc][G][4 + 128] (m, l in base 2, acc; ppc
+// partials per CTA) of the tile-split decode kernels into out (and lse), launched as a
+// programmatic dependent of the decode grid (decode_mma.cu). A partial with m = -inf carries
+// no token and its sums are not read.
 cudaError_t launch_combine_partials(const float* part, float* out, float* lse, int batch, int hq, int hkv, int G,
-                                    int s_max, int64_t tiles_per_unit, int64_t total_tiles, int n_ctas,
+                                    int s_max, int ppc, int64_t tiles_per_unit, int64_t total_tiles, int n_ctas,
                                     cudaStream_t stream);
 
 size_t mma_frag_bytes(int lm_bits, int G);  // query operand bytes per (sequence, KV head)
