@@ -77,8 +77,6 @@ constexpr unsigned long long kWaitNs = 2000000000ull;
 constexpr float kQmax = 1073741824.f;
 constexpr int kDigits = 4;
 
-// Named barriers: 1 = softmax warps, 2 = value warps (0 is __syncthreads).
-constexpr int kBarSm = 1, kBarV = 2;
 
 template <int LMB, bool QJL, int VB, int NB>
 struct TcLayout {
@@ -93,17 +91,15 @@ struct TcLayout {
   static constexpr int N = ((NC + (QJL ? NC : 0)) + 15) / 16 * 16;
   static constexpr int TA = 8 * EW;                    // tensor-memory columns of one A operand
   static constexpr int TG = TA + N;                    // tensor-memory columns of one group
-  // groups of four warps, one tile each: as many as tensor memory holds, at most 3, so that
-  // with the producer no scheduler holds more than 4 warps (128 registers each)
-  static constexpr int NG = 512 / TG >= 3 ? 3 : 512 / TG;
-  static_assert(NG >= 2, "tensor memory for two groups");
-  static constexpr int NCW = 4 * NG;                   // compute warps
-  static constexpr int THREADS = 32 * (NCW + 1);       // + the producer warp
+  // A stage holds two tiles (256 tokens): each array of the pair arrives with one bulk copy,
+  // [kc 256 x KCB][ks 256 x SB][kn 256 x 4][vc 256 x VCB][vp 256 x PB]; tile k of the pair sits
+  // 128 k records into each region. (Copies of 128 records streamed at under 60% of the HBM
+  // bandwidth; one thread issues every copy, and fewer, larger copies keep up with HBM.)
   static constexpr int KCB = LMB * 16, SB = QJL ? 16 : 0, VCB = VB * 16, PB = 16;
   static constexpr int REC = KCB + SB + 4 + VCB + PB;
-  static constexpr int STAGE = kTileTc * REC;
-  static constexpr int OFF_KC = 0, OFF_KS = kTileTc * KCB, OFF_KN = OFF_KS + kTileTc * SB;
-  static constexpr int OFF_VC = OFF_KN + kTileTc * 4, OFF_VP = OFF_VC + kTileTc * VCB;
+  static constexpr int STAGE = 2 * kTileTc * REC;
+  static constexpr int OFF_KC = 0, OFF_KS = 2 * kTileTc * KCB, OFF_KN = OFF_KS + 2 * kTileTc * SB;
+  static constexpr int OFF_VC = OFF_KN + 2 * kTileTc * 4, OFF_VP = OFF_VC + 2 * kTileTc * VCB;
   static constexpr int BOP = N * KB;                   // digits, K-major, 128-byte swizzle
   static constexpr int BBUF = BOP + HG * 16;           // + logit constants (float4 per head)
   static constexpr int BBUF_AL = (BBUF + 1023) / 1024 * 1024;
@@ -113,6 +109,26 @@ struct TcLayout {
   static constexpr int WP_PW = 4 * HG * 2 * kPS + 16;
   static constexpr int WP_MW = HG * 2 * kPS;
   static constexpr int WP_WORDS = WP_PW + WP_MW;
+  // Shared memory in front of the stage ring for ng groups, and the stages that fit behind it.
+  static constexpr int ring_at(int ng) {
+    return (2 * BBUF_AL + 4 * ng * WP_WORDS * 4 + ng * 4 * kD * 4 + 2 * ng * 4 * 8 * 4 + 8 * (2 * 12 + ng + 2) +
+            8 + 4 * ng + 127) / 128 * 128;
+  }
+  static constexpr int fit_stages(int ng) {
+    return (227 * 1024 - 1024 - ring_at(ng)) / STAGE > 6 ? 6 : (227 * 1024 - 1024 - ring_at(ng)) / STAGE;
+  }
+  // Group g consumes tiles g, g + ng, ...; tile i sits in stage (i / 2) mod NST. With 2 NST a
+  // multiple of ng, the previous use of a group's stage held a tile of the same group, so the
+  // phase a group waits for can never be confused with the one two uses back.
+  static constexpr int stages_for(int ng) { return ng == 3 ? fit_stages(3) / 3 * 3 : fit_stages(ng); }
+  // Groups of four warps, one tile each: as many as tensor memory holds, at most 3 (with the
+  // producer no scheduler then holds more than 4 warps of 128 registers), and 2 if three
+  // would leave the ring fewer than three stages.
+  static constexpr int NG_TM = 512 / TG >= 3 ? 3 : 512 / TG;
+  static_assert(NG_TM >= 2, "tensor memory for two groups");
+  static constexpr int NG = (NG_TM >= 3 && stages_for(3) >= 3) ? 3 : 2;
+  static constexpr int NCW = 4 * NG;                               // compute warps
+  static constexpr int THREADS = 32 * (NCW + 1);                   // + the producer warp
   static constexpr int SM_B = 0;                                  // [2] query operands
   static constexpr int SM_WP = 2 * BBUF_AL;                       // [NCW] value-weight areas
   static constexpr int SM_RED = SM_WP + NCW * WP_WORDS * 4;       // [NG][4 warps][d] unit-end sums
@@ -122,9 +138,9 @@ struct TcLayout {
   static constexpr int NBAR = 2 * 12 + NG + 2;
   static constexpr int SM_MISC = SM_BAR + 8 * NBAR;               // TMEM address, abort flag, grp_unit[NG]
   static constexpr int SM_RING = (SM_MISC + 8 + 4 * NG + 127) / 128 * 128;
-  static constexpr int BUDGET = 227 * 1024 - 1024 - SM_RING;
-  static constexpr int NST = BUDGET / STAGE > 8 ? 8 : BUDGET / STAGE;
-  static_assert(NST >= NG + 2 && NST <= 12, "stages");
+  static_assert(SM_RING == ring_at(NG), "layout");
+  static constexpr int NST = stages_for(NG);
+  static_assert(NST >= 2 && NST <= 12, "stages");
   static constexpr size_t SMEM = (size_t)SM_RING + (size_t)NST * STAGE + 1024;
   static_assert(SMEM <= 227 * 1024, "shared memory");
   static_assert(STAGE % 16 == 0 && BBUF % 16 == 0, "16-byte bulk copies");
@@ -507,7 +523,7 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
   unsigned char* sm = reinterpret_cast<unsigned char*>(((uintptr_t)smem_tc_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::SM_BAR);
   uint64_t* full = bars;            // [NST] stage landed
-  uint64_t* empty = bars + NST;     // [NST] stage consumed by its group (4 warps)
+  uint64_t* empty = bars + NST;     // [NST] both tiles of the stage consumed (2 x 4 warps)
   uint64_t* mmad = bars + 2 * NST;  // [NG] the group's MMA done (commit)
   uint64_t* fbfull = mmad + NG;     // [2] query operand landed
   uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + L::SM_MISC);
@@ -531,7 +547,7 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
   if (tid == 32) {
     for (int s = 0; s < NST; ++s) {
       s1::mbar_init(&full[s], 1);
-      s1::mbar_init(&empty[s], 4);
+      s1::mbar_init(&empty[s], 8);  // two tiles x four warps
     }
     for (int g = 0; g < NG; ++g) {
       s1::mbar_init(&mmad[g], 1);
@@ -561,86 +577,116 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
     int bulk_issued[12] = {};  // bulk batches issued per stage (for the failure drain)
     int uses[12] = {};         // phases started per stage
     int b_issued = 0;          // query operands issued (units in order)
-    for (int i = 0; i < ntl && !failed; ++i) {
-      const int s = i % NST;
-      if (i >= NST) {
+    // The query operand of a unit is loaded when its first tile is: into buffer j % 2, once
+    // every group has moved past unit j - 2 (its MMAs done, its constants read).
+    auto load_operand = [&](int u) -> bool {
+      const int j = u - u_first;
+      if (j != b_issued) return true;
+      bool ok = true;
+      if (lane == 0) {
+        if (b_issued == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
+        if (j >= 2) {
+          const unsigned long long t0 = s1::global_ns();
+          for (uint32_t it = 0;; ++it) {
+            int mn = 0x7fffffff;
+            for (int g = 0; g < NG; ++g) mn = min(mn, grp_unit[g]);
+            if (mn >= j - 1) break;
+            if (*abort_flag || ((it & 63) == 63 && s1::global_ns() - t0 > kWaitNs)) {
+              ok = false;
+              break;
+            }
+            __nanosleep(64);
+          }
+          asm volatile("fence.acq_rel.cta;" ::: "memory");
+        }
+        if (ok) {
+          s1::fence_async_smem();
+          s1::mbar_expect_tx(&fbfull[j & 1], (uint32_t)L::BBUF);
+          s1::bulk_g2s(sm + L::SM_B + (j & 1) * L::BBUF_AL, a.bop + (size_t)(u_first + j) * L::BBUF, L::BBUF,
+                       &fbfull[j & 1]);
+        }
+      }
+      ok = __shfl_sync(kFull, ok, 0);
+      if (ok) ++b_issued;
+      return ok;
+    };
+    const int npairs = (ntl + 1) / 2;
+    for (int pi = 0; pi < npairs && !failed; ++pi) {
+      const int s = pi % NST;
+      if (pi >= NST) {
         bool ok = true;
-        if (lane == 0) ok = wait_phase(&empty[s], (uint32_t)((i / NST) - 1) & 1u, abort_flag);
+        if (lane == 0) ok = wait_phase(&empty[s], (uint32_t)((pi / NST) - 1) & 1u, abort_flag);
         if (!__shfl_sync(kFull, ok, 0)) {
           failed = true;
           break;
         }
       }
-      const int u = walk.u, nt = walk.nt();
-      const int64_t tok0 = walk.tok0();
-      walk.next();
+      // the pair's tiles: k = 0, 1 (the second may be past the CTA's range)
+      int tu[2], tn[2];
+      int64_t tt[2], tv[2];
+      const int ntiles = min(2, ntl - 2 * pi);
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        tu[k] = u_first;
+        tn[k] = 0;
+        tt[k] = 0;
+        tv[k] = 0;
+        if (k >= ntiles) continue;
+        tu[k] = walk.u;
+        tn[k] = walk.nt();
+        tt[k] = walk.tok0();
+        walk.next();
+        tv[k] = tn[k] > 0 ? record_row(a.pg, a.max_len, tu[k], tt[k], a.err) : 0;
+      }
       unsigned char* st = ring + s * L::STAGE;
       uses[s] += 1;
-      if (a.use_tma && nt == kTileTc) {
-        if (lane == 0) {
-          s1::fence_async_smem();  // the consumers' generic reads come before the async writes
-          const int64_t v = record_row(a.pg, a.max_len, u, tok0, a.err);
-          s1::mbar_expect_tx(&full[s], (uint32_t)L::STAGE);
-          s1::bulk_g2s(st + L::OFF_KC, a.k_codes + v * L::KCB, kTileTc * L::KCB, &full[s]);
-          if constexpr (QJL) s1::bulk_g2s(st + L::OFF_KS, a.k_signs + v * L::SB, kTileTc * L::SB, &full[s]);
-          s1::bulk_g2s(st + L::OFF_KN, reinterpret_cast<const uint8_t*>(a.k_norms) + v * 4, kTileTc * 4, &full[s]);
-          s1::bulk_g2s(st + L::OFF_VC, a.v_codes + v * L::VCB, kTileTc * L::VCB, &full[s]);
-          s1::bulk_g2s(st + L::OFF_VP, reinterpret_cast<const uint8_t*>(a.v_params) + v * L::PB, kTileTc * L::PB,
+      const bool bulk0 = a.use_tma && tn[0] == kTileTc;
+      const bool bulk1 = ntiles == 2 && a.use_tma && tn[1] == kTileTc;
+      const bool one_copy = bulk0 && bulk1 && tv[1] == tv[0] + kTileTc;  // contiguous records
+      // ragged or unaligned tiles first: the warp copies their valid records with 4-byte loads
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        if (k >= ntiles || (k == 0 ? bulk0 : bulk1) || tn[k] == 0) continue;
+        const int64_t v = tv[k];
+        const int nt = tn[k];
+        auto copy = [&](int off, const void* src, int bpt) {
+          const uint32_t* s32 = reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(src) + v * bpt);
+          uint32_t* d32 = reinterpret_cast<uint32_t*>(st + off + k * kTileTc * bpt);
+          for (int w = lane; w < nt * bpt / 4; w += 32) d32[w] = s32[w];
+        };
+        copy(L::OFF_KC, a.k_codes, L::KCB);
+        if constexpr (QJL) copy(L::OFF_KS, a.k_signs, L::SB);
+        copy(L::OFF_KN, a.k_norms, 4);
+        copy(L::OFF_VC, a.v_codes, L::VCB);
+        copy(L::OFF_VP, a.v_params, L::PB);
+      }
+      __syncwarp();
+      if (lane == 0) {
+        // then the bulk copies, after the arrival that announces their bytes
+        const uint32_t tile_bytes = (uint32_t)(L::STAGE / 2);
+        s1::fence_async_smem();  // the consumers' generic reads come before the async writes
+        s1::mbar_expect_tx(&full[s], (bulk0 ? tile_bytes : 0u) + (bulk1 ? tile_bytes : 0u));
+        auto issue = [&](int k, int64_t v, int nrec) {
+          const int o = k * kTileTc;
+          s1::bulk_g2s(st + L::OFF_KC + o * L::KCB, a.k_codes + v * L::KCB, nrec * L::KCB, &full[s]);
+          if constexpr (QJL) s1::bulk_g2s(st + L::OFF_KS + o * L::SB, a.k_signs + v * L::SB, nrec * L::SB, &full[s]);
+          s1::bulk_g2s(st + L::OFF_KN + o * 4, reinterpret_cast<const uint8_t*>(a.k_norms) + v * 4, nrec * 4,
                        &full[s]);
-          bulk_issued[s] += 1;
+          s1::bulk_g2s(st + L::OFF_VC + o * L::VCB, a.v_codes + v * L::VCB, nrec * L::VCB, &full[s]);
+          s1::bulk_g2s(st + L::OFF_VP + o * L::PB, reinterpret_cast<const uint8_t*>(a.v_params) + v * L::PB,
+                       nrec * L::PB, &full[s]);
+        };
+        if (one_copy) {
+          issue(0, tv[0], 2 * kTileTc);
+        } else {
+          if (bulk0) issue(0, tv[0], kTileTc);
+          if (bulk1) issue(1, tv[1], kTileTc);
         }
-      } else {
-        // ragged or unaligned tile: the warp copies the valid records with 4-byte loads
-        if (nt > 0) {
-          const int64_t v = record_row(a.pg, a.max_len, u, tok0, a.err);
-          auto copy = [&](int off, const void* src, int bpt) {
-            const uint32_t* s32 = reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(src) + v * bpt);
-            uint32_t* d32 = reinterpret_cast<uint32_t*>(st + off);
-            for (int w = lane; w < nt * bpt / 4; w += 32) d32[w] = s32[w];
-          };
-          copy(L::OFF_KC, a.k_codes, L::KCB);
-          if constexpr (QJL) copy(L::OFF_KS, a.k_signs, L::SB);
-          copy(L::OFF_KN, a.k_norms, 4);
-          copy(L::OFF_VC, a.v_codes, L::VCB);
-          copy(L::OFF_VP, a.v_params, L::PB);
-        }
-        __syncwarp();
-        if (lane == 0) s1::mbar_arrive(&full[s]);
+        if (bulk0 || bulk1) bulk_issued[s] += 1;
       }
-      // The query operand of a unit is loaded when its first tile is: into buffer j % 2, once
-      // every group has moved past unit j - 2 (its MMAs done, its constants read).
-      const int j = u - u_first;
-      if (j == b_issued) {
-        bool ok = true;
-        if (lane == 0) {
-          if (b_issued == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
-          if (j >= 2) {
-            const unsigned long long t0 = s1::global_ns();
-            for (uint32_t it = 0;; ++it) {
-              int mn = 0x7fffffff;
-              for (int g = 0; g < NG; ++g) mn = min(mn, grp_unit[g]);
-              if (mn >= j - 1) break;
-              if (*abort_flag || ((it & 63) == 63 && s1::global_ns() - t0 > kWaitNs)) {
-                ok = false;
-                break;
-              }
-              __nanosleep(64);
-            }
-            asm volatile("fence.acq_rel.cta;" ::: "memory");
-          }
-          if (ok) {
-            s1::fence_async_smem();
-            s1::mbar_expect_tx(&fbfull[j & 1], (uint32_t)L::BBUF);
-            s1::bulk_g2s(sm + L::SM_B + (j & 1) * L::BBUF_AL, a.bop + (size_t)(u_first + j) * L::BBUF, L::BBUF,
-                         &fbfull[j & 1]);
-          }
-        }
-        if (!__shfl_sync(kFull, ok, 0)) {
-          failed = true;
-          break;
-        }
-        ++b_issued;
-      }
+#pragma unroll
+      for (int k = 0; k < 2; ++k)
+        if (k < ntiles && !failed && !load_operand(tu[k])) failed = true;
     }
     if (failed && lane == 0) raise_abort(abort_flag);
     __syncwarp();
@@ -778,7 +824,7 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
     reset();
     int cur = -1, qrow0 = 0, kt = 0;  // local unit, its first query row, tiles of this group so far
     for (int i = gi; i < ntl; i += NG, ++kt) {
-      const int s = i % NST;
+      const int s = (i >> 1) % NST, slot = i & 1;
       const int u = walk.u, nt = walk.nt();
       const int64_t tok0 = walk.tok0();
       for (int k = 0; k < NG; ++k) walk.next();
@@ -786,23 +832,38 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
       if (j != cur) {
         if (cur >= 0) finish(cur);
         for (int jj = cur + 1; jj < j; ++jj) mark_empty(jj);
+        // Every warp of the group is past its previous unit, so that unit's query operand may be
+        // reloaded. The leader steps through the operand phases of the units this group has no
+        // tile of, in order, releasing each before waiting for the next: a buffer's phases are
+        // then never skipped, and no parity wait can match the phase of two loads back.
+        if (leader) {
+          asm volatile("fence.acq_rel.cta;" ::: "memory");
+          for (int jj = cur + 1; jj < j && !failed; ++jj) {
+            grp_unit[gi] = jj;
+            if (!wait_phase(&fbfull[jj & 1], (uint32_t)(jj >> 1) & 1u, abort_flag)) failed = true;
+          }
+          grp_unit[gi] = j;
+          if (failed) raise_abort(abort_flag);
+        }
+        named_sync(bar_id, 128);
         cur = j;
         reset();
         const int bq = u / a.hkv, kvh = u - bq * a.hkv;
         qrow0 = bq * a.hq + kvh * G;
-        if (leader) {
-          // every warp of the group is past its previous unit: its query operand may be reloaded
-          asm volatile("fence.acq_rel.cta;" ::: "memory");
-          grp_unit[gi] = j;
-        }
         if (!failed && !wait_phase(&fbfull[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag)) failed = true;
       }
-      if (!failed && !wait_phase(&full[s], (uint32_t)(i / NST) & 1u, abort_flag)) failed = true;
+      if (!failed && !wait_phase(&full[s], (uint32_t)((i >> 1) / NST) & 1u, abort_flag)) failed = true;
       const unsigned char* st = ring + s * L::STAGE;
+      // this tile's records in the stage's five regions
+      const unsigned char* t_kc = st + L::OFF_KC + slot * kTileTc * L::KCB;
+      const unsigned char* t_ks = st + L::OFF_KS + slot * kTileTc * L::SB;
+      const unsigned char* t_kn = st + L::OFF_KN + slot * kTileTc * 4;
+      const unsigned char* t_vc = st + L::OFF_VC + slot * kTileTc * L::VCB;
+      const unsigned char* t_vp = st + L::OFF_VP + slot * kTileTc * L::PB;
       // ---- key bits -> unsigned 8-bit elements in tensor memory (row R of the A operand)
       {
         uint32_t w[L::EW];
-        const uint4* kc = reinterpret_cast<const uint4*>(st + L::OFF_KC + R * L::KCB);
+        const uint4* kc = reinterpret_cast<const uint4*>(t_kc + R * L::KCB);
 #pragma unroll
         for (int cc = 0; cc < LMB; ++cc) {
           const uint4 v = kc[cc];
@@ -812,7 +873,7 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
           w[4 * cc + 3] = v.w;
         }
         if constexpr (QJL) {
-          const uint4 v = *reinterpret_cast<const uint4*>(st + L::OFF_KS + R * L::SB);
+          const uint4 v = *reinterpret_cast<const uint4*>(t_ks + R * L::SB);
           w[L::KSC] = v.x;
           w[L::KSC + 1] = v.y;
           w[L::KSC + 2] = v.z;
@@ -865,8 +926,8 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
       s1::tmem_ld_wait();
       // ---- logits and online softmax (per warp: its 32 tokens, one per lane)
       const bool valid = R < nt && !failed;
-      const uint32_t ngw = *reinterpret_cast<const uint32_t*>(st + L::OFF_KN + 4 * R);
-      const uint4 vpar = *reinterpret_cast<const uint4*>(st + L::OFF_VP + 16 * R);
+      const uint32_t ngw = *reinterpret_cast<const uint32_t*>(t_kn + 4 * R);
+      const uint4 vpar = *reinterpret_cast<const uint4*>(t_vp + 16 * R);
       const float2 ng = __half22float2(h2of(ngw));  // (n, gamma)
       const float4* kc4 = reinterpret_cast<const float4*>(sm + L::SM_B + (j & 1) * L::BBUF_AL + L::BOP);
       float lg[HG];
@@ -973,8 +1034,8 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
       }
       __syncwarp();
       // ---- values of the warp's 32 tokens: two blocks of 16 (mma.sync, k = tokens)
-      const uint32_t* vc = reinterpret_cast<const uint32_t*>(st + L::OFF_VC);
-      const uint32_t* vpw = reinterpret_cast<const uint32_t*>(st + L::OFF_VP);
+      const uint32_t* vc = reinterpret_cast<const uint32_t*>(t_vc);
+      const uint32_t* vpw = reinterpret_cast<const uint32_t*>(t_vp);
 #pragma unroll 1
       for (int mb = 0; mb < 2; ++mb) {
         const int tb = 32 * q + 16 * mb;  // first token of the block within the tile
