@@ -2,7 +2,7 @@
 // 1- to 3-bit Lloyd-Max codes from a codebook symmetric about zero, with the 128-bit QJL
 // sketch or without it; 2- or 4-bit values; up to 8 query heads per KV head).
 //
-// Same mathematics as decode_kernel and decode_mma_kernel (the skill card "turboquant-
+// Same mathematics as decode_kernel (the skill card "turboquant-
 // pytorch", "Что делает": attention scores straight from the compressed keys; the discosf
 // news item, "一句话看懂": fused decode kernels on the compressed cache): logit = scale * n *
 // (<qr, c[idx]> + sqrt(pi/2)/m * gamma * <sq, s>), online softmax, sum of p * (min + scale *
@@ -28,29 +28,32 @@
 //    96-bit stream XORed with itself shifted by one and by two, bit 3j of X is code j's
 //    parity, and the bits 3j fall on distinct positions of the three 32-bit words (0, 1, 2
 //    mod 3), so one word keeps them all: bit p holds code (32 (p mod 3) + p) / 3.
-// Values. out = sum_t p_t (min + scale * code): the warps of the value role run mma.sync
-// m16n8k16 with rows = value coordinates, k = tokens, columns = 4 query heads x (hi, lo):
-// a 2- or 4-bit code in the low mantissa bits of an f16 is an exact subnormal (the power of
-// two is undone at the end), and p * scale arrives as an f16 hi + lo pair (an exact
-// TwoProduct) computed once per token by the softmax role; the group minima enter through
-// one more MMA with p itself.
-// Online softmax in base 2 with one reference maximum per query head for the whole CTA,
+// Values. out = sum_t p_t (min + scale * code), also on the tensor cores (kind::f16, f32 sums
+// in tensor memory): rows = the 128 value coordinates, K = the tile's tokens, columns = (value
+// group, query head). A 2- or 4-bit code masked into the low mantissa bits of an f16 is an
+// exact subnormal, code * 2^(position - 24), so one AND makes two elements; the power of two
+// depends only on the row and is undone at the end. The A operand sits in shared memory
+// MN-major (each token's 128 elements contiguous, as the expansion writes them), and so does
+// B, p * scale as an f16 high part and low part (an exact TwoProduct), each its own K pass
+// into the same sums. Only the column of the row's own value group is read back. The group
+// minima, sum_t p_t min_t, are fp32 sums per thread.
+// Online softmax in base 2 with one reference maximum per query head for a group of warps,
 // moved only when a logit exceeds it by more than 2 (p < 4, so p * scale stays finite in f16
-// for value scales below 16376); when it moves, the value role rescales its sums.
+// for value scales below 16376); when it moves, the sums so far are rescaled in place.
 //
-// Roles (512 threads, one CTA per SM, the units' tiles laid end to end and split evenly
-// over the CTAs as in decode_mma_kernel):
-//   warp 0      streams the packed tiles into a ring of shared-memory stages (bulk copies;
-//               warp-wide plain copies for a ragged or unaligned tile);
-//   warp 1      one thread issues every MMA;
-//   warp 2      one thread loads each unit's query operand (digits + logit constants);
-//   warps 4-7   one token per thread: expand the key bits into tensor memory;
-//   warps 8-11  one token per thread: read the scores back, logits, online softmax, write
-//               the value weights (p * scale, hi + lo) to shared memory;
-//   warps 12-15 32 tokens each: accumulate the values.
-// Tensor memory holds two A buffers (key elements) and two D buffers (digit sums), so the
-// expansion of tile i + 1 and the softmax of tile i - 1 overlap the MMA of tile i.
-// Every wait is bounded: on a timeout the CTA raises an abort flag that every role polls,
+// Work split (one CTA per SM; the units' tiles laid end to end and split evenly over the
+// CTAs, so a CTA's range may start and end inside a unit and span several):
+//   one producer warp streams the packed records into a ring of two-tile stages (one bulk
+//   copy per array and stage; a ragged or unaligned tile is copied by the warp) and loads
+//   each unit's query operand (digits + logit constants) when the unit's first tile goes;
+//   groups of four warps take the tiles in turn, one token per thread: expand the key bits
+//   into tensor memory and the value codes into the group's value operand, release the
+//   stage, then (one elected thread) the score MMAs; read the digit sums back, logits,
+//   online softmax, value weights; then the value MMAs. Each group has its own tensor-memory
+//   columns (key elements, digit sums, value sums) and value operands, so one group's MMAs
+//   overlap the others' arithmetic. At the end of a unit each group writes one partial
+//   (m, l, acc) per query head; combine_partials merges them in a fixed order.
+// Every wait is bounded: on a timeout the CTA raises an abort flag that every warp polls,
 // sets the context's error word, drains the copies and MMAs it issued and returns.
 #include <cuda_runtime.h>
 #include <math.h>
@@ -69,9 +72,9 @@ constexpr int kTileTc = 128;       // tokens per tile = MMA rows
 constexpr int kPrepTcThreads = 256;
 constexpr float kSlackTc = 2.f;
 constexpr uint32_t kWaitPolls = 1u << 24;
-// Suspend-time hint of one mbarrier poll in ns (0: the instruction's own short limit). The
-// roles hand each tile to one another, so a waiting warp must see the phase at once.
-constexpr uint32_t kTryWaitNs = 0;
+// Suspend-time hint of one mbarrier poll in ns: a waiting warp sleeps until the phase
+// completes (or this long) instead of spinning, and leaves the issue slots to the others.
+constexpr uint32_t kTryWaitNs = 100000;
 constexpr unsigned long long kWaitNs = 2000000000ull;
 // |Q| <= 2^30 keeps the top one of four balanced 8-bit digits in [-64, 64]
 constexpr float kQmax = 1073741824.f;
@@ -89,8 +92,15 @@ struct TcLayout {
   static constexpr int KB = 32 * EW;                   // bytes of one B row
   static constexpr int NC = kDigits * HG;              // code columns (4 digits per head)
   static constexpr int N = ((NC + (QJL ? NC : 0)) + 15) / 16 * 16;
-  static constexpr int TA = 8 * EW;                    // tensor-memory columns of one A operand
-  static constexpr int TG = TA + N;                    // tensor-memory columns of one group
+  static constexpr int NV = 4 * HG;                    // value weights per part: (value group, head)
+  static constexpr int TA = 8 * EW;                    // tensor-memory columns: key elements
+  // Value sums: with VSPLIT the high and low parts of the weights are separate columns
+  // (g, part, h) of one MMA pass, reading the codes once; otherwise (too few tensor-memory
+  // columns for two groups) they are two passes into the same columns (g, h).
+  static constexpr int groups_fit(int cols) { return 512 / cols >= 3 ? 3 : 512 / cols; }
+  static constexpr bool VSPLIT = groups_fit(TA + N + 2 * NV) >= 2 && groups_fit(TA + N + 2 * NV) == groups_fit(TA + N + NV);
+  static constexpr int NVC = VSPLIT ? 2 * NV : NV;     // value-sum columns
+  static constexpr int TG = TA + N + NVC;              // per group: key elements, scores, value sums
   // A stage holds two tiles (256 tokens): each array of the pair arrives with one bulk copy,
   // [kc 256 x KCB][ks 256 x SB][kn 256 x 4][vc 256 x VCB][vp 256 x PB]; tile k of the pair sits
   // 128 k records into each region. (Copies of 128 records streamed at under 60% of the HBM
@@ -103,47 +113,50 @@ struct TcLayout {
   static constexpr int BOP = N * KB;                   // digits, K-major, 128-byte swizzle
   static constexpr int BBUF = BOP + HG * 16;           // + logit constants (float4 per head)
   static constexpr int BBUF_AL = (BBUF + 1023) / 1024 * 1024;
-  // Per compute warp: value weights p * scale [group][head][part][16 token pairs] (rows of
-  // kPS words; groups 2-3 16 words further), then p [head][part][16 pairs] for the minima.
-  static constexpr int kPS = 20;
-  static constexpr int WP_PW = 4 * HG * 2 * kPS + 16;
-  static constexpr int WP_MW = HG * 2 * kPS;
-  static constexpr int WP_WORDS = WP_PW + WP_MW;
-  // Shared memory in front of the stage ring for ng groups, and the stages that fit behind it.
-  static constexpr int ring_at(int ng) {
-    return (2 * BBUF_AL + 4 * ng * WP_WORDS * 4 + ng * 4 * kD * 4 + 2 * ng * 4 * 8 * 4 + 8 * (2 * 12 + ng + 2) +
-            8 + 4 * ng + 127) / 128 * 128;
+  // Value operands of a group, f16, MN-major without swizzle: core matrices of 8 rows (value
+  // coordinates, or weight columns) x 8 tokens, 128 B each, 128 B apart along the tokens and
+  // 2048 B apart along the rows. The codes [128 rows][128 tokens], then the value weights
+  // p * scale: with VSPLIT one operand [(g, part, h)][128 tokens], else the high and the low
+  // parts [(g, h)][128 tokens] one after the other.
+  static constexpr int AV = kD * kTileTc * 2;
+  static constexpr int BVP = NV * kTileTc * 2;
+  static constexpr int GV = AV + 2 * BVP;
+  static constexpr int RED_F = 5 * HG;                 // per warp: minima sums [HG][4], sums of p [HG]
+  static constexpr int NBAR = 2 * 6 + 2 * 3 + 2;       // full, empty [<= 6]; mmad, vdone [<= 3]; fbfull [2]
+  // Shared memory in front of the stage ring for ng groups and nbuf query-operand buffers, and
+  // the stages that fit behind it.
+  static constexpr int front(int ng, int nbuf) {
+    return (nbuf * BBUF_AL + ng * GV + ng * 4 * RED_F * 4 + ng * 4 * 8 * 4 + 8 * NBAR + 8 + 4 * ng + 127) / 128 * 128;
   }
-  static constexpr int fit_stages(int ng) {
-    return (227 * 1024 - 1024 - ring_at(ng)) / STAGE > 6 ? 6 : (227 * 1024 - 1024 - ring_at(ng)) / STAGE;
+  static constexpr int fit(int ng, int nbuf) {
+    return (227 * 1024 - 1024 - front(ng, nbuf)) / STAGE > 6 ? 6 : (227 * 1024 - 1024 - front(ng, nbuf)) / STAGE;
   }
   // Group g consumes tiles g, g + ng, ...; tile i sits in stage (i / 2) mod NST. With 2 NST a
   // multiple of ng, the previous use of a group's stage held a tile of the same group, so the
   // phase a group waits for can never be confused with the one two uses back.
-  static constexpr int stages_for(int ng) { return ng == 3 ? fit_stages(3) / 3 * 3 : fit_stages(ng); }
-  // Groups of four warps, one tile each: as many as tensor memory holds, at most 3 (with the
-  // producer no scheduler then holds more than 4 warps of 128 registers), and 2 if three
-  // would leave the ring fewer than three stages.
+  static constexpr int stages(int ng, int nbuf) { return ng == 3 ? fit(3, nbuf) / 3 * 3 : fit(ng, nbuf); }
+  // Groups of four warps, one tile each: as many as tensor memory holds, at most 3, and 2 if
+  // three would leave fewer than three stages. Two query-operand buffers (the next unit's
+  // loads while the current one runs) when three stages remain beside them, else one.
   static constexpr int NG_TM = 512 / TG >= 3 ? 3 : 512 / TG;
   static_assert(NG_TM >= 2, "tensor memory for two groups");
-  static constexpr int NG = (NG_TM >= 3 && stages_for(3) >= 3) ? 3 : 2;
-  static constexpr int NCW = 4 * NG;                               // compute warps
-  static constexpr int THREADS = 32 * (NCW + 1);                   // + the producer warp
-  static constexpr int SM_B = 0;                                  // [2] query operands
-  static constexpr int SM_WP = 2 * BBUF_AL;                       // [NCW] value-weight areas
-  static constexpr int SM_RED = SM_WP + NCW * WP_WORDS * 4;       // [NG][4 warps][d] unit-end sums
-  static constexpr int SM_RM = SM_RED + NG * 4 * kD * 4;          // [NG][4][8] warp maxima
-  static constexpr int SM_RL = SM_RM + NG * 4 * 8 * 4;            // [NG][4][8] warp sums of p
-  static constexpr int SM_BAR = SM_RL + NG * 4 * 8 * 4;
-  static constexpr int NBAR = 2 * 12 + NG + 2;
-  static constexpr int SM_MISC = SM_BAR + 8 * NBAR;               // TMEM address, abort flag, grp_unit[NG]
+  static constexpr int NG = (NG_TM >= 3 && stages(3, 1) >= 3) ? 3 : 2;
+  static constexpr int NBUF = stages(NG, 2) >= 3 ? 2 : 1;
+  static constexpr int NST = stages(NG, NBUF);
+  static_assert(NST >= 2 && NST <= 6, "stages");
+  static constexpr int NCW = 4 * NG;                   // compute warps
+  static constexpr int THREADS = 32 * (NCW + 1);       // + the producer warp
+  static constexpr int SM_B = 0;                                   // [NBUF] query operands
+  static constexpr int SM_V = NBUF * BBUF_AL;                      // [NG] value operands
+  static constexpr int SM_RED = SM_V + NG * GV;                    // [NG][4 warps][RED_F]
+  static constexpr int SM_RM = SM_RED + NG * 4 * RED_F * 4;        // [NG][4 warps][8] warp maxima
+  static constexpr int SM_BAR = SM_RM + NG * 4 * 8 * 4;
+  static constexpr int SM_MISC = SM_BAR + 8 * NBAR;                // TMEM address, abort flag, grp_unit[NG]
   static constexpr int SM_RING = (SM_MISC + 8 + 4 * NG + 127) / 128 * 128;
-  static_assert(SM_RING == ring_at(NG), "layout");
-  static constexpr int NST = stages_for(NG);
-  static_assert(NST >= 2 && NST <= 12, "stages");
+  static_assert(SM_RING == front(NG, NBUF), "layout");
   static constexpr size_t SMEM = (size_t)SM_RING + (size_t)NST * STAGE + 1024;
   static_assert(SMEM <= 227 * 1024, "shared memory");
-  static_assert(STAGE % 16 == 0 && BBUF % 16 == 0, "16-byte bulk copies");
+  static_assert(STAGE % 16 == 0 && BBUF % 16 == 0 && SM_V % 1024 == 0 && GV % 16 == 0, "alignment");
 };
 
 struct TcArgs {
@@ -240,14 +253,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
       : "memory");
 }
 
-__device__ __forceinline__ void mma16816_tc(float (&d)[4], const uint4& a, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
-}
-
 __device__ __forceinline__ float ex2f(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -287,12 +292,45 @@ __device__ __forceinline__ uint32_t parity_word(uint32_t x0, uint32_t x1, uint32
   return (X0 & 0x49249249u) | (X1 & 0x92492492u) | (X2 & 0x24924924u);
 }
 
-// Word offset of the value-weight row (group g, head h, part) in a warp's area (rows of 20
-// words: 16 token pairs + 4, so that the 8 rows a fragment load touches fall on distinct
-// banks); groups 2-3 sit 16 words further so that the even and odd threads of a token pair
-// write distinct banks.
-__device__ __forceinline__ int prow(int g, int h, int part, int HG) {
-  return ((g * HG + h) * 2 + part) * 20 + (g >> 1) * 16;
+// 16-byte shared-memory store.
+__device__ __forceinline__ void st_shared_v4(void* p, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_addr(p)), "r"(x), "r"(y), "r"(z), "r"(w)
+               : "memory");
+}
+
+// Instruction descriptor, kind::f16: f16 x f16 -> f32, both operands MN-major.
+__host__ __device__ constexpr uint32_t idesc_f16_mn(int M, int N) {
+  return (1u << 4)                       // D format f32
+         | (1u << 15) | (1u << 16)       // A and B MN-major
+         | ((uint32_t)(N >> 3) << 17)    // N / 8
+         | ((uint32_t)(M >> 4) << 24);   // M / 16
+}
+
+// Shared-memory descriptor of an MN-major operand without swizzle: core matrices of 8 rows x
+// 8 tokens (128 B: 16 B per token), 128 B apart along the tokens (leading byte offset) and
+// 2048 B apart along the rows (stride byte offset), sm_100 version bit, layout 0.
+__device__ __forceinline__ uint64_t desc_mn(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)(128u >> 4) << 16) | ((uint64_t)(2048u >> 4) << 32) |
+         ((uint64_t)1u << 46);
+}
+
+// Row m of the value MMA (tensor-memory lane m of the value sums) holds value coordinate
+// value_coord(m), its code times 2^-value_unscale-exponent (a code in bits b .. of an f16 is
+// the subnormal code * 2^(b - 24)). 2-bit codes: word w of a record (coordinates 16 w ..)
+// gives row chunks 2 w (bytes 0 and 2: codes 0, 1 at bits 6, 8 of the word shifted left by
+// 6, codes 2, 3 of the word shifted left by 2) and 2 w + 1 (bytes 1 and 3, shifted right
+// by 2 and 6). 4-bit codes: word w (coordinates 8 w ..) gives row chunk w, every code at bit
+// 6 (low and high nibbles of bytes 0, 2, then of bytes 1, 3). Either way rows 32 g .. 32 g +
+// 31 are value group g.
+template <int VB>
+__device__ __forceinline__ int value_coord(int m) {
+  if constexpr (VB == 2) return 16 * (m >> 4) + 4 * ((m >> 3) & 1) + ((m & 7) >> 1) + 8 * (m & 1);
+  else return 8 * (m >> 3) + ((m & 7) >> 1) + 4 * (m & 1);
+}
+template <int VB>
+__device__ __forceinline__ float value_unscale(int m) {
+  if constexpr (VB == 2) return __int_as_float((127 + 18 - 2 * (((m & 7) >> 1) & 1)) << 23);
+  else return __int_as_float((127 + 18) << 23);
 }
 
 // Walks a CTA's tiles in order without dividing: the unit, the tile within it, the unit's
@@ -516,16 +554,17 @@ template <int LMB, bool QJL, int VB, int NB>
 __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
     decode_tc_kernel(const __grid_constant__ TcArgs a) {
   using L = TcLayout<LMB, QJL, VB, NB>;
-  constexpr int HG = L::HG, NST = L::NST, NG = L::NG;
+  constexpr int HG = L::HG, NST = L::NST, NG = L::NG, NBUF = L::NBUF;
   constexpr int RS = 4 + kD;  // partial row: m, l, pad, pad, acc[d]
   constexpr float kLn2 = 0.6931471805599453f;
   extern __shared__ unsigned char smem_tc_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(((uintptr_t)smem_tc_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::SM_BAR);
-  uint64_t* full = bars;            // [NST] stage landed
-  uint64_t* empty = bars + NST;     // [NST] both tiles of the stage consumed (2 x 4 warps)
-  uint64_t* mmad = bars + 2 * NST;  // [NG] the group's MMA done (commit)
-  uint64_t* fbfull = mmad + NG;     // [2] query operand landed
+  uint64_t* full = bars;           // [NST] stage landed
+  uint64_t* empty = bars + 6;      // [NST] both tiles of the stage read (2 x 4 warps)
+  uint64_t* mmad = bars + 12;      // [NG] the group's score MMAs done (commit)
+  uint64_t* vdone = bars + 15;     // [NG] the group's value MMAs done (commit)
+  uint64_t* fbfull = bars + 18;    // [NBUF] query operand landed
   uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + L::SM_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::SM_MISC + 4);
   volatile int* grp_unit = reinterpret_cast<volatile int*>(sm + L::SM_MISC + 8);  // [NG]
@@ -551,10 +590,10 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
     }
     for (int g = 0; g < NG; ++g) {
       s1::mbar_init(&mmad[g], 1);
+      s1::mbar_init(&vdone[g], 1);
       grp_unit[g] = -1;
     }
-    s1::mbar_init(&fbfull[0], 1);
-    s1::mbar_init(&fbfull[1], 1);
+    for (int b = 0; b < NBUF; ++b) s1::mbar_init(&fbfull[b], 1);
     *abort_flag = 0;
     s1::mbar_init_fence();
   }
@@ -574,23 +613,24 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
   bool failed = false;
   if (warp == L::NCW) {
     // ============================================================ producer
-    int bulk_issued[12] = {};  // bulk batches issued per stage (for the failure drain)
-    int uses[12] = {};         // phases started per stage
-    int b_issued = 0;          // query operands issued (units in order)
-    // The query operand of a unit is loaded when its first tile is: into buffer j % 2, once
-    // every group has moved past unit j - 2 (its MMAs done, its constants read).
+    int bulk_issued[6] = {};  // bulk batches issued per stage (for the failure drain)
+    int uses[6] = {};         // phases started per stage
+    int b_issued = 0;         // query operands issued (units in order)
+    // The query operand of local unit j is loaded when the unit's first tile is, into buffer
+    // j mod NBUF, once every group has moved past the unit that buffer held (its MMAs done,
+    // its constants read).
     auto load_operand = [&](int u) -> bool {
       const int j = u - u_first;
       if (j != b_issued) return true;
       bool ok = true;
       if (lane == 0) {
         if (b_issued == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
-        if (j >= 2) {
+        if (j >= NBUF) {
           const unsigned long long t0 = s1::global_ns();
           for (uint32_t it = 0;; ++it) {
             int mn = 0x7fffffff;
             for (int g = 0; g < NG; ++g) mn = min(mn, grp_unit[g]);
-            if (mn >= j - 1) break;
+            if (mn >= j - NBUF + 1) break;
             if (*abort_flag || ((it & 63) == 63 && s1::global_ns() - t0 > kWaitNs)) {
               ok = false;
               break;
@@ -601,9 +641,9 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
         }
         if (ok) {
           s1::fence_async_smem();
-          s1::mbar_expect_tx(&fbfull[j & 1], (uint32_t)L::BBUF);
-          s1::bulk_g2s(sm + L::SM_B + (j & 1) * L::BBUF_AL, a.bop + (size_t)(u_first + j) * L::BBUF, L::BBUF,
-                       &fbfull[j & 1]);
+          s1::mbar_expect_tx(&fbfull[j % NBUF], (uint32_t)L::BBUF);
+          s1::bulk_g2s(sm + L::SM_B + (j % NBUF) * L::BBUF_AL, a.bop + (size_t)(u_first + j) * L::BBUF, L::BBUF,
+                       &fbfull[j % NBUF]);
         }
       }
       ok = __shfl_sync(kFull, ok, 0);
@@ -696,47 +736,67 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
       if (*abort_flag)
         for (int s = 0; s < NST; ++s)
           if (bulk_issued[s] > 0) s1::mbar_wait(&full[s], (uint32_t)(uses[s] - 1) & 1u);
-      for (int jj = (b_issued > 2 ? b_issued - 2 : 0); jj < b_issued; ++jj)
-        s1::mbar_wait(&fbfull[jj & 1], (uint32_t)(jj >> 1) & 1u);
+      for (int jj = (b_issued > NBUF ? b_issued - NBUF : 0); jj < b_issued; ++jj)
+        s1::mbar_wait(&fbfull[jj % NBUF], (uint32_t)(jj / NBUF) & 1u);
     }
   } else {
     // ============================================================ compute warps
-    // group gi (warps 4 gi .. 4 gi + 3) takes tiles gi, gi + NG, ...; warp q of the group owns
-    // tokens 32 q .. 32 q + 31 of each tile (tensor-memory lanes 32 q ..)
+    // Group gi (warps 4 gi .. 4 gi + 3) takes tiles gi, gi + NG, ...; warp q of the group owns
+    // tokens 32 q .. 32 q + 31 of each tile (tensor-memory lanes 32 q ..), and for the value
+    // sums the 32 value coordinates of value group q (rows 32 q .. of the value MMA).
     const int gi = warp >> 2, q = warp & 3;
     const int R = 32 * q + lane;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    const uint32_t tA = tmem + gi * L::TG + lane_base, tD = tA + L::TA;
+    const uint32_t tgrp = tmem + gi * L::TG;
+    const uint32_t tA = tgrp + lane_base, tD = tgrp + L::TA + lane_base;
+    // this warp's value-sum columns: group q's (part, h), or (h) without VSPLIT
+    const uint32_t tV = tgrp + L::TA + L::N + lane_base + q * (L::NVC / 4);
     const int bar_id = 1 + gi;
     const bool leader = q == 0 && lane == 0;
-    const int r = lane >> 2, c = lane & 3;
-    const int part = r & 1, hsel = r >> 1;
-    uint32_t* wp = reinterpret_cast<uint32_t*>(sm + L::SM_WP) + warp * L::WP_WORDS;  // this warp's area
-    uint32_t* wpm = wp + L::WP_PW;
-    float* red = reinterpret_cast<float*>(sm + L::SM_RED) + gi * 4 * kD;  // [4][d]
-    float* rm = reinterpret_cast<float*>(sm + L::SM_RM) + gi * 32;        // [4][8]
-    float* rl = reinterpret_cast<float*>(sm + L::SM_RL) + gi * 32;        // [4][8]
+    unsigned char* av = sm + L::SM_V + gi * L::GV;   // codes [16 row chunks][128 tokens]
+    unsigned char* bv = av + L::AV;                   // weights [2 NV / 8 row chunks][128 tokens]
+    float* red = reinterpret_cast<float*>(sm + L::SM_RED) + gi * 4 * L::RED_F;  // [4][RED_F]
+    float* rm = reinterpret_cast<float*>(sm + L::SM_RM) + gi * 32;              // [4][8]
+    // this thread's 16-byte slot of a row chunk: chunk c of token R at c * 2048 + the slot
+    const uint32_t slot_off = (uint32_t)((R >> 3) * 128 + (R & 7) * 16);
 
-    float Mref[HG], lsum[HG];
-    float dmin[NB][4];
-    float dv[4][2][NB][4];
+    // Per thread: the group's reference maxima, this token's share of the sums of p and of
+    // p * min, and (as value row R) the unit's value sums of row R, to which the tensor-memory
+    // sums of each tile are added in fp32 (sums kept in tensor memory over many tiles drift
+    // low: each MMA truncates its result).
+    float Mref[HG], lsum[HG], mn[HG][4], acc[HG];
+    bool vpend = false;  // tensor memory holds value sums of a tile not yet added to acc
     auto reset = [&]() {
 #pragma unroll
       for (int h = 0; h < HG; ++h) {
         Mref[h] = -INFINITY;
         lsum[h] = 0.f;
+        acc[h] = 0.f;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) mn[h][g] = 0.f;
       }
-#pragma unroll
-      for (int nb = 0; nb < NB; ++nb) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dmin[nb][e] = 0.f;
-#pragma unroll
-        for (int g = 0; g < 4; ++g)
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) dv[g][hf][nb][e] = 0.f;
+      vpend = false;
+    };
+    // add the last tile's value sums of row R (issue; tmem_ld_wait before use)
+    uint32_t dvv[L::NVC / 4];
+    auto load_vsums = [&]() {
+      if constexpr (L::NVC / 4 == 8) {
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                     : "=r"(dvv[0]), "=r"(dvv[1]), "=r"(dvv[2]), "=r"(dvv[3]), "=r"(dvv[4]), "=r"(dvv[5]),
+                       "=r"(dvv[6]), "=r"(dvv[7])
+                     : "r"(tV));
+      } else if constexpr (L::NVC / 4 == 4) {
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(dvv[0]), "=r"(dvv[1]), "=r"(dvv[2]), "=r"(dvv[3])
+                     : "r"(tV));
+      } else {
+        tmem_ld16(tV, dvv);
       }
+    };
+    auto add_vsums = [&]() {
+#pragma unroll
+      for (int h = 0; h < HG; ++h)
+        acc[h] += L::VSPLIT ? __uint_as_float(dvv[h]) + __uint_as_float(dvv[HG + h]) : __uint_as_float(dvv[h]);
     };
     auto part_ptr = [&](int j) -> float* {
       const int u = u_first + j;
@@ -751,73 +811,47 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
         pp[lane * RS + 1] = 0.f;
       }
     };
-    // End of local unit j for this group: the four warps' sums, rescaled to the group's
-    // maximum and added in warp order, are the group's partial (m, l, acc) of the unit.
+    int kv = 0;  // value-MMA commits of this group so far
+    // End of local unit j: the group's partial (m, l, acc) of the unit. The reference maxima
+    // are the group's; the sums of p and of p * min are added over the group's 128 lanes in a
+    // fixed order; row R of the value sums is value coordinate coord(R).
     auto finish = [&](int j) {
       float* pp = part_ptr(j);
+      if (vpend) {
+        if (!failed && !wait_phase(&vdone[gi], (uint32_t)(kv - 1) & 1u, abort_flag)) failed = true;
+        s1::fence_after_sync();
+        load_vsums();
+        s1::tmem_ld_wait();
+        add_vsums();
+        vpend = false;
+      }
 #pragma unroll
       for (int h = 0; h < HG; ++h) {
         const float l = warp_sum(lsum[h]);
-        if (lane == 0) {
-          rm[q * 8 + h] = failed ? -INFINITY : Mref[h];
-          rl[q * 8 + h] = failed ? 0.f : l;
+        if (lane == 0) red[q * L::RED_F + 4 * HG + h] = l;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const float v = warp_sum(mn[h][g]);
+          if (lane == 0) red[q * L::RED_F + 4 * h + g] = v;
         }
       }
       named_sync(bar_id, 128);
+      const int coord = value_coord<VB>(R);
+      const float unscale = value_unscale<VB>(R);
+      for (int h = 0; h < G; ++h) {
+        const float msum = ((red[4 * h + q] + red[L::RED_F + 4 * h + q]) + red[2 * L::RED_F + 4 * h + q]) +
+                           red[3 * L::RED_F + 4 * h + q];
+        pp[h * RS + 4 + coord] = failed ? 0.f : fmaf(acc[h], unscale, msum);
+      }
       if (q == 0 && lane < G) {
         const int h = lane;
-        float M = -INFINITY;
-        for (int w = 0; w < 4; ++w) M = fmaxf(M, rm[w * 8 + h]);
-        float Ls = 0.f;
-        for (int w = 0; w < 4; ++w) {
-          const float mw = rm[w * 8 + h];
-          if (mw != -INFINITY) Ls = fmaf(ex2f(mw - M), rl[w * 8 + h], Ls);
-        }
-        pp[h * RS + 0] = M;
-        pp[h * RS + 1] = Ls;
+        const float Ls = ((red[4 * HG + h] + red[L::RED_F + 4 * HG + h]) + red[2 * L::RED_F + 4 * HG + h]) +
+                         red[3 * L::RED_F + 4 * HG + h];
+        pp[h * RS + 0] = failed ? -INFINITY : Mref[h];
+        pp[h * RS + 1] = failed ? 0.f : Ls;
       }
-#pragma unroll
-      for (int nb = 0; nb < NB; ++nb) {
-        const float own = dmin[nb][0] + dmin[nb][1];
-        float mt[4];
-#pragma unroll
-        for (int g = 0; g < 4; ++g) mt[g] = __shfl_sync(kFull, own, 4 * g + c);
-        const int hme = c + 4 * nb;
-        float Mg = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) Mg = fmaxf(Mg, rm[w * 8 + hme]);
-        float mme = rm[q * 8 + hme];
-        const float wsc = (failed || mme == -INFINITY) ? 0.f : ex2f(mme - Mg);
-        for (int c4 = 0; c4 < 4; ++c4) {
-          const int h = 4 * nb + c4;
-          if (h >= G) break;  // uniform
-          if (c == c4) {
-            float* rq = red + q * kD;
-#pragma unroll
-            for (int g = 0; g < 4; ++g)
-#pragma unroll
-              for (int hf = 0; hf < 2; ++hf) {
-                const float* d = dv[g][hf][nb];
-                int j0;
-                float v0, v1;
-                if (VB == 2) {
-                  j0 = 4 * (8 * g + r) + 2 * hf;
-                  v0 = (d[0] + d[1]) * ldexpf(1.f, 24 - 4 * hf) + mt[g];
-                  v1 = (d[2] + d[3]) * ldexpf(1.f, 22 - 4 * hf) + mt[g];
-                } else {
-                  j0 = 2 * (16 * g + 8 * hf + r);
-                  v0 = (d[0] + d[1]) * 16777216.f + mt[g];
-                  v1 = (d[2] + d[3]) * 1048576.f + mt[g];
-                }
-                rq[j0] = wsc != 0.f ? wsc * v0 : 0.f;
-                rq[j0 + 1] = wsc != 0.f ? wsc * v1 : 0.f;
-              }
-          }
-          named_sync(bar_id, 128);
-          pp[h * RS + 4 + R] = ((red[R] + red[kD + R]) + red[2 * kD + R]) + red[3 * kD + R];
-          named_sync(bar_id, 128);
-        }
-      }
+      s1::fence_before_sync();
+      named_sync(bar_id, 128);  // red is reused by the next unit
     };
 
     for (int k = 0; k < gi; ++k) walk.next();
@@ -840,7 +874,7 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
           asm volatile("fence.acq_rel.cta;" ::: "memory");
           for (int jj = cur + 1; jj < j && !failed; ++jj) {
             grp_unit[gi] = jj;
-            if (!wait_phase(&fbfull[jj & 1], (uint32_t)(jj >> 1) & 1u, abort_flag)) failed = true;
+            if (!wait_phase(&fbfull[jj % NBUF], (uint32_t)(jj / NBUF) & 1u, abort_flag)) failed = true;
           }
           grp_unit[gi] = j;
           if (failed) raise_abort(abort_flag);
@@ -850,20 +884,26 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
         reset();
         const int bq = u / a.hkv, kvh = u - bq * a.hkv;
         qrow0 = bq * a.hq + kvh * G;
-        if (!failed && !wait_phase(&fbfull[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag)) failed = true;
+        if (!failed && !wait_phase(&fbfull[j % NBUF], (uint32_t)(j / NBUF) & 1u, abort_flag)) failed = true;
       }
       if (!failed && !wait_phase(&full[s], (uint32_t)((i >> 1) / NST) & 1u, abort_flag)) failed = true;
+      // the value operands are free once the group's previous value MMAs are done
+      if (kv > 0 && !failed && !wait_phase(&vdone[gi], (uint32_t)(kv - 1) & 1u, abort_flag)) failed = true;
+      s1::fence_after_sync();
       const unsigned char* st = ring + s * L::STAGE;
-      // this tile's records in the stage's five regions
-      const unsigned char* t_kc = st + L::OFF_KC + slot * kTileTc * L::KCB;
-      const unsigned char* t_ks = st + L::OFF_KS + slot * kTileTc * L::SB;
-      const unsigned char* t_kn = st + L::OFF_KN + slot * kTileTc * 4;
-      const unsigned char* t_vc = st + L::OFF_VC + slot * kTileTc * L::VCB;
-      const unsigned char* t_vp = st + L::OFF_VP + slot * kTileTc * L::PB;
-      // ---- key bits -> unsigned 8-bit elements in tensor memory (row R of the A operand)
+      const bool valid = R < nt && !failed;
+      // ---- phase 1: this token's records out of the stage
+      uint32_t ngw, vp[4];
       {
+        ngw = *reinterpret_cast<const uint32_t*>(st + L::OFF_KN + (slot * kTileTc + R) * 4);
+        const uint4 v4 = *reinterpret_cast<const uint4*>(st + L::OFF_VP + (slot * kTileTc + R) * L::PB);
+        vp[0] = v4.x;
+        vp[1] = v4.y;
+        vp[2] = v4.z;
+        vp[3] = v4.w;
+        // key bits -> unsigned 8-bit elements in tensor memory (row R of the A operand)
         uint32_t w[L::EW];
-        const uint4* kc = reinterpret_cast<const uint4*>(t_kc + R * L::KCB);
+        const uint4* kc = reinterpret_cast<const uint4*>(st + L::OFF_KC + (slot * kTileTc + R) * L::KCB);
 #pragma unroll
         for (int cc = 0; cc < LMB; ++cc) {
           const uint4 v = kc[cc];
@@ -873,7 +913,7 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
           w[4 * cc + 3] = v.w;
         }
         if constexpr (QJL) {
-          const uint4 v = *reinterpret_cast<const uint4*>(t_ks + R * L::SB);
+          const uint4 v = *reinterpret_cast<const uint4*>(st + L::OFF_KS + (slot * kTileTc + R) * L::SB);
           w[L::KSC] = v.x;
           w[L::KSC + 1] = v.y;
           w[L::KSC + 2] = v.z;
@@ -901,20 +941,49 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
           }
           tmem_st32(tA + 32 * e4, m);
         }
+        // value codes -> f16 elements (row chunks of the value MMA's A operand)
+        const uint4* vc = reinterpret_cast<const uint4*>(st + L::OFF_VC + (slot * kTileTc + R) * L::VCB);
+#pragma unroll
+        for (int c4 = 0; c4 < VB; ++c4) {
+          const uint4 v = vc[c4];
+          const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int wi = 0; wi < 4; ++wi) {
+            // Each code lands in bits 6..9 of its f16 (the largest subnormals: the tensor cores
+            // resolve products with small subnormal elements less finely, which showed as a
+            // 1e-4 error in strongly peaked attention with the codes in bits 0..7).
+            const uint32_t y = x[wi], l6 = y << 6, l2 = y << 2, r2 = y >> 2, r6 = y >> 6;
+            if constexpr (VB == 2) {
+              // word 4 c4 + wi: coordinates 16 (4 c4 + wi) + 0..15 -> chunks 2 (4 c4 + wi) + 0, 1;
+              // bytes 0 and 2 from the left shifts, bytes 1 and 3 from the right shifts
+              const int c = 2 * (4 * c4 + wi);
+              st_shared_v4(av + c * 2048 + slot_off, l6 & 0x00C000C0u, l6 & 0x03000300u, l2 & 0x00C000C0u,
+                           l2 & 0x03000300u);
+              st_shared_v4(av + (c + 1) * 2048 + slot_off, r2 & 0x00C000C0u, r2 & 0x03000300u, r6 & 0x00C000C0u,
+                           r6 & 0x03000300u);
+            } else {
+              // word 4 c4 + wi: coordinates 8 (4 c4 + wi) + 0..7 -> chunk 4 c4 + wi
+              const int c = 4 * c4 + wi;
+              st_shared_v4(av + c * 2048 + slot_off, l6 & 0x03C003C0u, l2 & 0x03C003C0u, r2 & 0x03C003C0u,
+                           r6 & 0x03C003C0u);
+            }
+          }
+        }
         s1::tmem_st_wait();
       }
+      __syncwarp();
+      if (lane == 0) s1::mbar_arrive(&empty[s]);  // the stage is no longer read by this warp
       s1::fence_before_sync();
-      named_sync(bar_id, 128);  // all four quarters of the tile's A operand are written
+      named_sync(bar_id, 128);  // all four quarters of the tile's key elements are written
       if (leader) {
         s1::fence_after_sync();
         if (!failed) {
           constexpr uint32_t idesc = idesc_u8s8_s32(kTileTc, L::N);
-          const uint32_t bbase = smem_addr(sm + L::SM_B + (j & 1) * L::BBUF_AL);
-          const uint32_t d_tm = tmem + gi * L::TG + L::TA;
-          const uint32_t a_tm = tmem + gi * L::TG;
+          const uint32_t bbase = smem_addr(sm + L::SM_B + (j % NBUF) * L::BBUF_AL);
+          const uint32_t d_tm = tgrp + L::TA;
 #pragma unroll
           for (int ks = 0; ks < L::EW; ++ks)
-            umma_i8_ts(d_tm, a_tm + 8 * ks, s1::sw128_desc(bbase, 16 * ks, L::N), idesc, ks > 0 ? 1u : 0u);
+            umma_i8_ts(d_tm, tgrp + 8 * ks, s1::sw128_desc(bbase, 16 * ks, L::N), idesc, ks > 0 ? 1u : 0u);
           s1::umma_commit(&mmad[gi]);
         }
       }
@@ -923,13 +992,13 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
       uint32_t dsum[L::N];
 #pragma unroll
       for (int cc = 0; cc < L::N; cc += 16) tmem_ld16(tD + cc, dsum + cc);
+      if (vpend) load_vsums();  // the previous tile's value sums (its MMAs are done)
       s1::tmem_ld_wait();
-      // ---- logits and online softmax (per warp: its 32 tokens, one per lane)
-      const bool valid = R < nt && !failed;
-      const uint32_t ngw = *reinterpret_cast<const uint32_t*>(t_kn + 4 * R);
-      const uint4 vpar = *reinterpret_cast<const uint4*>(t_vp + 16 * R);
+      if (vpend) add_vsums();
+      vpend = false;
+      // ---- logits
       const float2 ng = __half22float2(h2of(ngw));  // (n, gamma)
-      const float4* kc4 = reinterpret_cast<const float4*>(sm + L::SM_B + (j & 1) * L::BBUF_AL + L::BOP);
+      const float4* kc4 = reinterpret_cast<const float4*>(sm + L::SM_B + (j % NBUF) * L::BBUF_AL + L::BOP);
       float lg[HG];
 #pragma unroll
       for (int h = 0; h < HG; ++h) {
@@ -952,152 +1021,122 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
         for (int h = 0; h < HG; ++h)
           if (h < G) a.scores[(size_t)(qrow0 + h) * a.max_len + tok0 + R] = lg[h] * kLn2;
       }
-      // Lazy rescale: the warp's reference maxima move only when a logit exceeds them by more
-      // than the slack.
+      // ---- online softmax with the group's reference maxima, moved only when a logit exceeds
+      // them by more than the slack; the value sums so far are rescaled then
       bool need = false;
 #pragma unroll
       for (int h = 0; h < HG; ++h) need |= lg[h] > Mref[h] + kSlackTc;
-      if (__any_sync(kFull, need)) {
+      if (named_sync_or(bar_id, 128, need)) {
+#pragma unroll
+        for (int h = 0; h < HG; ++h) {
+          const float wm = warp_max(lg[h]);
+          if (lane == 0) rm[q * 8 + h] = wm;
+        }
+        named_sync(bar_id, 128);
         float corr[HG];
 #pragma unroll
         for (int h = 0; h < HG; ++h) {
-          const float Mn = fmaxf(Mref[h], warp_max(lg[h]));
+          const float Mn = fmaxf(fmaxf(fmaxf(Mref[h], rm[h]), fmaxf(rm[8 + h], rm[16 + h])), rm[24 + h]);
           corr[h] = 1.f;
           if (Mn > Mref[h]) {
             corr[h] = Mref[h] == -INFINITY ? 0.f : ex2f(Mref[h] - Mn);
-            lsum[h] *= corr[h];
             Mref[h] = Mn;
           }
-        }
+          lsum[h] *= corr[h];
+          acc[h] *= corr[h];
 #pragma unroll
-        for (int nb = 0; nb < NB; ++nb) {
-          const float cf = c == 0 ? corr[4 * nb] : c == 1 ? corr[4 * nb + 1] : c == 2 ? corr[4 * nb + 2]
-                                                                                      : corr[4 * nb + 3];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) dmin[nb][e] *= cf;
-#pragma unroll
-          for (int g = 0; g < 4; ++g)
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf)
-#pragma unroll
-              for (int e = 0; e < 4; ++e) dv[g][hf][nb][e] *= cf;
+          for (int g = 0; g < 4; ++g) mn[h][g] *= corr[h];
         }
       }
-      // p per head, split in f16 hi + lo
-      uint32_t own[HG];
+      // p per head; the minima sums in fp32; the value weights p * scale as f16 hi + lo
+      float p[HG];
 #pragma unroll
       for (int h = 0; h < HG; ++h) {
-        const float p = lg[h] == -INFINITY ? 0.f : ex2f(lg[h] - Mref[h]);
-        lsum[h] += p;
-        const __half hi = __float2half_rn(p);
-        const __half lo = __float2half_rn(p - __half2float(hi));
-        own[h] = (uint32_t)__half_as_ushort(hi) | ((uint32_t)__half_as_ushort(lo) << 16);
+        p[h] = lg[h] == -INFINITY ? 0.f : ex2f(lg[h] - Mref[h]);
+        lsum[h] += p[h];
       }
-      // value weights of the token pair (even, odd lane): the even lane writes groups 0-1,
-      // the odd lane groups 2-3, and the minima's p of the first / second half of the heads
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const float mg = valid ? __high2float(h2of(vp[g])) : 0.f;
+#pragma unroll
+        for (int h = 0; h < HG; ++h) mn[h][g] = fmaf(p[h], mg, mn[h][g]);
+      }
       {
-        const bool odd = (lane & 1) != 0;
-        uint32_t par[HG];
+        uint32_t ph2[HG / 2], pl2[HG / 2];
 #pragma unroll
-        for (int h = 0; h < HG; ++h) par[h] = __shfl_xor_sync(kFull, own[h], 1);
-        const uint32_t sc[4] = {valid ? vpar.x : 0u, valid ? vpar.y : 0u, valid ? vpar.z : 0u,
-                                valid ? vpar.w : 0u};
-        const uint32_t send0 = odd ? sc[0] : sc[2], send1 = odd ? sc[1] : sc[3];
-        const uint32_t got0 = __shfl_xor_sync(kFull, send0, 1), got1 = __shfl_xor_sync(kFull, send1, 1);
-        const int pair = lane >> 1;
+        for (int hp = 0; hp < HG / 2; ++hp) {
+          const __half2 hi = __floats2half2_rn(p[2 * hp], p[2 * hp + 1]);
+          const float2 hf = __half22float2(hi);
+          const __half2 lo = __floats2half2_rn(p[2 * hp] - hf.x, p[2 * hp + 1] - hf.y);
+          ph2[hp] = hbits(hi);
+          pl2[hp] = hbits(lo);
+        }
+        // weight (g, h), high and low parts, 2 per word
+        uint32_t whi[L::NV / 2], wlo[L::NV / 2];
 #pragma unroll
-        for (int gg = 0; gg < 2; ++gg) {
-          const int g = odd ? 2 + gg : gg;
-          const uint32_t mine = odd ? sc[2 + gg] : sc[gg];
-          const uint32_t other = gg == 0 ? got0 : got1;
-          const uint32_t s2w = odd ? __byte_perm(other, mine, 0x5410) : __byte_perm(mine, other, 0x5410);
-          const __half2 s2 = h2of(s2w);
+        for (int g = 0; g < 4; ++g) {
+          const uint32_t sw = valid ? vp[g] : 0u;
+          const __half2 s2 = h2of(__byte_perm(sw, sw, 0x1010));  // (scale, scale)
 #pragma unroll
-          for (int h = 0; h < HG; ++h) {
-            const uint32_t ev = odd ? par[h] : own[h], ov = odd ? own[h] : par[h];
-            const __half2 ph = h2of(__byte_perm(ev, ov, 0x5410));  // p_hi of (even, odd)
-            const __half2 pl = h2of(__byte_perm(ev, ov, 0x7632));  // p_lo of (even, odd)
+          for (int hp = 0; hp < HG / 2; ++hp) {
+            const __half2 ph = h2of(ph2[hp]), pl = h2of(pl2[hp]);
             const __half2 hi = __hmul2(ph, s2);
             const __half2 err = __hfma2(ph, s2, __hneg2(hi));
             const __half2 lo = __hfma2(pl, s2, err);
-            wp[prow(g, h, 0, HG) + pair] = hbits(hi);
-            wp[prow(g, h, 1, HG) + pair] = hbits(lo);
+            whi[g * (HG / 2) + hp] = hbits(hi);
+            wlo[g * (HG / 2) + hp] = hbits(lo);
           }
         }
+        if constexpr (L::VSPLIT) {
+          // columns (g, part, h), 2 per word; row chunk c = words 4 c .. 4 c + 3
+          uint32_t wv[L::NV];
 #pragma unroll
-        for (int hh = 0; hh < HG / 2; ++hh) {
-          const int h = odd ? HG / 2 + hh : hh;
-          const uint32_t ev = odd ? par[h] : own[h], ov = odd ? own[h] : par[h];
-          wpm[(h * 2 + 0) * 20 + pair] = __byte_perm(ev, ov, 0x5410);
-          wpm[(h * 2 + 1) * 20 + pair] = __byte_perm(ev, ov, 0x7632);
-        }
-      }
-      __syncwarp();
-      // ---- values of the warp's 32 tokens: two blocks of 16 (mma.sync, k = tokens)
-      const uint32_t* vc = reinterpret_cast<const uint32_t*>(t_vc);
-      const uint32_t* vpw = reinterpret_cast<const uint32_t*>(t_vp);
-#pragma unroll 1
-      for (int mb = 0; mb < 2; ++mb) {
-        const int tb = 32 * q + 16 * mb;  // first token of the block within the tile
-        if (tb >= nt || failed) break;    // warp-uniform
-        const int nv = nt - tb;
-        const int tA0 = tb + 2 * c, tA1 = tA0 + 1, tB0 = tA0 + 8, tB1 = tA0 + 9;
-        const int pA = 8 * mb + c, pB = pA + 4;  // token pairs of b0 and b1 in the warp's area
-        {
-          uint32_t mA0 = 0u, mA1 = 0u, mB0 = 0u, mB1 = 0u;
-          if (r < 4) {
-            if (2 * c < nv) mA0 = vpw[tA0 * 4 + r];
-            if (2 * c + 1 < nv) mA1 = vpw[tA1 * 4 + r];
-            if (2 * c + 8 < nv) mB0 = vpw[tB0 * 4 + r];
-            if (2 * c + 9 < nv) mB1 = vpw[tB1 * 4 + r];
-          }
-          uint4 am;
-          am.x = __byte_perm(mA0, mA1, 0x7632);
-          am.y = 0u;
-          am.z = __byte_perm(mB0, mB1, 0x7632);
-          am.w = 0u;
+          for (int g = 0; g < 4; ++g)
 #pragma unroll
-          for (int nb = 0; nb < NB; ++nb) {
-            const int row = ((4 * nb + hsel) * 2 + part) * 20;
-            mma16816_tc(dmin[nb], am, wpm[row + pA], wpm[row + pB]);
-          }
-        }
-        const uint32_t sel = (uint32_t)(r & 3) | ((uint32_t)(4 + (r & 3)) << 8);
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          uint32_t bA[NB], bB[NB];
-#pragma unroll
-          for (int nb = 0; nb < NB; ++nb) {
-            const int row = prow(g, 4 * nb + hsel, part, HG);
-            bA[nb] = wp[row + pA];
-            bB[nb] = wp[row + pB];
-          }
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            uint32_t xA, xB;
-            uint4 av;
-            constexpr int WPT = L::VCB / 4;
-            if (VB == 2) {
-              const int wv = 2 * g + (r >> 2);
-              if (hf == 0) {
-                xA = __byte_perm(vc[tA0 * WPT + wv], vc[tA1 * WPT + wv], sel);
-                xB = __byte_perm(vc[tB0 * WPT + wv], vc[tB1 * WPT + wv], sel);
-              }
-              const uint32_t m0 = 0x00030003u << (4 * hf), m1 = 0x00030003u << (4 * hf + 2);
-              av = make_uint4(xA & m0, xA & m1, xB & m0, xB & m1);
-            } else {
-              const int wv = 4 * g + 2 * hf + (r >> 2);
-              xA = __byte_perm(vc[tA0 * WPT + wv], vc[tA1 * WPT + wv], sel);
-              xB = __byte_perm(vc[tB0 * WPT + wv], vc[tB1 * WPT + wv], sel);
-              av = make_uint4(xA & 0x000F000Fu, xA & 0x00F000F0u, xB & 0x000F000Fu, xB & 0x00F000F0u);
+            for (int hp = 0; hp < HG / 2; ++hp) {
+              wv[g * HG + hp] = whi[g * (HG / 2) + hp];
+              wv[g * HG + HG / 2 + hp] = wlo[g * (HG / 2) + hp];
             }
 #pragma unroll
-            for (int nb = 0; nb < NB; ++nb) mma16816_tc(dv[g][hf][nb], av, bA[nb], bB[nb]);
+          for (int c = 0; c < L::NV / 4; ++c)
+            st_shared_v4(bv + c * 2048 + slot_off, wv[4 * c], wv[4 * c + 1], wv[4 * c + 2], wv[4 * c + 3]);
+        } else {
+          // columns (g, h) of the high parts, then of the low parts
+#pragma unroll
+          for (int c = 0; c < L::NV / 8; ++c) {
+            st_shared_v4(bv + c * 2048 + slot_off, whi[4 * c], whi[4 * c + 1], whi[4 * c + 2], whi[4 * c + 3]);
+            st_shared_v4(bv + L::BVP + c * 2048 + slot_off, wlo[4 * c], wlo[4 * c + 1], wlo[4 * c + 2],
+                         wlo[4 * c + 3]);
           }
         }
       }
-      __syncwarp();
-      if (lane == 0) s1::mbar_arrive(&empty[s]);
+      s1::fence_async_smem();  // the value operands, written by this thread, are read by the MMA
+      s1::fence_before_sync();
+      named_sync(bar_id, 128);
+      if (leader) {
+        s1::fence_after_sync();
+        if (!failed) {
+          const uint32_t abase = smem_addr(av), bbase = smem_addr(bv);
+          const uint32_t d_tm = tgrp + L::TA + L::N;
+          if constexpr (L::VSPLIT) {
+            constexpr uint32_t idesc = idesc_f16_mn(kTileTc, 2 * L::NV);
+#pragma unroll
+            for (int ks = 0; ks < kTileTc / 16; ++ks)
+              s1::umma_f16(d_tm, desc_mn(abase + 256 * ks), desc_mn(bbase + 256 * ks), idesc, ks > 0 ? 1u : 0u);
+          } else {
+            constexpr uint32_t idesc = idesc_f16_mn(kTileTc, L::NV);
+#pragma unroll
+            for (int ks = 0; ks < kTileTc / 16; ++ks) {
+              const uint64_t ad = desc_mn(abase + 256 * ks);
+              s1::umma_f16(d_tm, ad, desc_mn(bbase + 256 * ks), idesc, ks > 0 ? 1u : 0u);
+              s1::umma_f16(d_tm, ad, desc_mn(bbase + L::BVP + 256 * ks), idesc, 1u);
+            }
+          }
+        }
+        s1::umma_commit(&vdone[gi]);
+      }
+      vpend = true;
+      ++kv;
     }
     if (cur >= 0) finish(cur);
     for (int jj = cur + 1; jj < n_units; ++jj) mark_empty(jj);
