@@ -65,6 +65,8 @@ def parse():
     ap.add_argument("--config-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--decode-kernel", default="auto", choices=["auto", "tcgen05", "mma", "cuda_core"],
+                    help="decode kernel family (default: the library's choice for the shape)")
     ap.add_argument("--sweep", action="store_true",
                     help="compression sweep instead of the step: 1,048,576 bf16 keys at every head "
                          "dimension (64, 128, 256), key bit width (2, 3, 4) and rotation (Hadamard, Haar)")
@@ -91,14 +93,22 @@ def source_sha(names):
     return h.hexdigest()[:16]
 
 
-DECODE_SOURCES = ("decode_tc.cu", "decode_mma.cu", "decode.cu", "tq_device.cuh", "tq_sm100.cuh", "tq_internal.h")
-COMPRESS_SOURCES = ("compress.cu", "tq_device.cuh", "tq_sm100.cuh", "tq_internal.h")
+# Source files of each main kernel: a recorded ncu traffic figure applies while their hash is unchanged.
+KERNEL_SOURCES = {
+    "decode_mma_kernel": ("decode_mma.cu", "tq_device.cuh"),
+    "decode_tc_kernel": ("decode_tc.cu", "tq_device.cuh", "tq_sm100.cuh"),
+    "decode_kernel": ("decode.cu", "tq_device.cuh"),
+    "compress_pipe_kernel": ("compress.cu", "tq_device.cuh", "tq_sm100.cuh"),
+    "compress_q4_kernel": ("compress.cu", "tq_device.cuh", "tq_sm100.cuh"),
+    "compress_kernel": ("compress.cu", "tq_device.cuh", "tq_sm100.cuh"),
+}
 
 
-def recorded_traffic(kernel_file: str, sha: str, units: int, kernel: str):
-    """DRAM bytes of one launch over `units` units, from a committed ncu summary that
-    gives DRAM bytes per unit for the same kernel and source (None if absent or stale)."""
-    p = os.path.join(ROOT, "profiles", kernel_file)
+def recorded_traffic(sha: str, units: int, kernel: str):
+    """DRAM bytes of one launch over `units` units, from the committed ncu summary
+    profiles/<kernel>_traffic.txt that gives DRAM bytes per unit for the same kernel and
+    source hash (None if absent or stale)."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}_traffic.txt")
     if not os.path.exists(p):
         return None
     kv = {}
@@ -284,6 +294,10 @@ def run_reference(args, w: W.Workload):
 # ---------------------------------------------------------------------- GPU arm
 
 SIDE_WORKLOADS = ("single_head_d128_n4096", "qwen2.5-3b_8k_k3v2", "long_1m_k4v4")
+KERNEL_IDS = {"auto": 0, "tcgen05": 1, "mma": 2, "cuda_core": 3}
+KERNEL_NAMES = {1: "tcgen05", 2: "mma", 3: "cuda_core"}
+# main attention kernel of each decode family (the one the library brackets with profile events)
+DECODE_KERNEL_OF = {1: "decode_tc_kernel", 2: "decode_mma_kernel", 3: "decode_kernel"}
 
 
 def time_side_workload(T, torch, w: W.Workload, steps: int, warmup: int, dev, flush_l2, peak: float):
@@ -333,8 +347,9 @@ def time_side_workload(T, torch, w: W.Workload, steps: int, warmup: int, dev, fl
     dk = statistics.median(e[2].elapsed_time(e[3]) for e in comp) / 1e3
     packed_bytes = w.packed_bytes()
     comp_bytes = 2 * n_vec * w.d * (2 if w.dtype == "bf16" else 4) + packed_bytes
+    fam = T.tq_decode_kernel_for(ctx, w.hq, w.hkv)
     ctx.close()
-    return {"batch": w.batch, "kv_heads": w.hkv, "q_heads": w.hq, "tokens": w.tokens, "k_bits": w.k_bits,
+    return {"decode_kernel": DECODE_KERNEL_OF.get(fam), "batch": w.batch, "kv_heads": w.hkv, "q_heads": w.hq, "tokens": w.tokens, "k_bits": w.k_bits,
             "v_bits": w.v_bits, "dtype": w.dtype, "packed_bytes": packed_bytes, "steps": steps,
             "compress_kernel_us": ck * 1e6, "compress_vectors_per_s": 2 * n_vec / ck,
             "compress_gbs": comp_bytes / ck / 1e9, "compress_frac": comp_bytes / ck / 1e9 / peak,
@@ -368,6 +383,10 @@ def run_ours(args, w: W.Workload):
     dr = W.method_draws(w.d, w.m)
     c, t = T.tq_lloyd_max_codebook(w.d, w.lm_bits)
     ctx = T.tq_codebook_load(w.d, w.lm_bits, w.v_bits, c, t, dr["qjl_S"], hadamard_signs=dr["hadamard_signs"])
+    T.tq_set_decode_kernel(ctx, KERNEL_IDS[args.decode_kernel])
+    fam = T.tq_decode_kernel_for(ctx, w.hq, w.hkv)
+    if fam < 0:
+        raise SystemExit(f"the {args.decode_kernel} decode kernel does not take workload {w.name}")
     n_vec = w.units * w.tokens
     if args.decode_only:
         args.no_e2e = args.no_cpu_baseline = True
@@ -562,6 +581,37 @@ def run_ours(args, w: W.Workload):
     # our kernels per step: compress (1) + decode (query prep + attention + combine)
     launches_per_step = (0 if args.decode_only else 1) + 3
 
+    # The other tensor-core decode family on the same cache, when it takes the shape: its
+    # main kernel alone, L2 flushed before each launch (reported beside the chosen one).
+    alt = {}
+    if rank == 0 and world == 1 and not args.no_configs:
+        for f2 in (1, 2):
+            if f2 == fam:
+                continue
+            T.tq_set_decode_kernel(ctx, f2)
+            if T.tq_decode_kernel_for(ctx, w.hq, w.hkv) != f2:
+                continue
+            ws2 = torch.empty(T.tq_decode_workspace_bytes(ctx, w.batch, w.hq, w.hkv, w.tokens), dtype=torch.uint8,
+                              device=dev)
+            ts = []
+            for it in range(3 + args.config_steps):
+                e = [E(enable_timing=True) for _ in range(2)]
+                for ev in e:
+                    ev.record()
+                flush_l2()
+                T.tq_set_profile_events(ctx, e[0], e[1])
+                T.tq_decode_attention(ctx, Q, packed, w.batch, w.hq, w.hkv, w.tokens, out=out, workspace=ws2)
+                T.tq_set_profile_events(ctx, None, None)
+                if it >= 3:
+                    ts.append(e)
+            torch.cuda.synchronize()
+            T.tq_check_device(ctx)
+            k_s = statistics.median(e[0].elapsed_time(e[1]) for e in ts) / 1e3
+            alt[KERNEL_NAMES[f2]] = {"kernel": DECODE_KERNEL_OF[f2], "kernel_us": k_s * 1e6,
+                                     "gbs": packed_bytes / k_s / 1e9, "steps": args.config_steps}
+            del ws2
+        T.tq_set_decode_kernel(ctx, KERNEL_IDS[args.decode_kernel])
+
     side = None
     if rank == 0 and world == 1 and not args.no_configs and not args.decode_only:
         peak, _ = measured_peaks()
@@ -584,22 +634,18 @@ def run_ours(args, w: W.Workload):
 
     if rank == 0:
         peak, peak_kind = measured_peaks()
-        dsha = source_sha(DECODE_SOURCES)
         units_dec = w.units * w.tokens  # (token, KV head) pairs
-        # the tcgen05 decode serves d = 128, m in {0, 128}, 1- to 3-bit Lloyd-Max codes (symmetric
-        # codebook), 2- or 4-bit values, G <= 8
-        dkern = "decode_tc_kernel" if (w.d == 128 and w.m in (0, 128) and w.lm_bits <= 3 and w.group <= 8
-                                       and w.v_bits in (2, 4)) else "decode_kernel"
+        dkern = DECODE_KERNEL_OF[fam]
+        dsha = source_sha(KERNEL_SOURCES[dkern])
         roof_dec = {"kernel": dkern, "bound": "hbm", "achieved": packed_bytes / dec_k_mean / 1e9,
                     "peak": peak, "unit": "GB/s", "frac": packed_bytes / dec_k_mean / 1e9 / peak,
                     "peak_kind": peak_kind, "alg_bytes_per_launch": packed_bytes,
                     "alg_bytes_per_unit": w.k_record_bytes() + w.v_record_bytes(), "unit_of_work": "token x KV head",
-                    "traffic": recorded_traffic("decode_kernel_traffic.txt", dsha, units_dec, dkern),
+                    "traffic": recorded_traffic(dsha, units_dec, dkern),
                     "source_sha256_16": dsha}
         roof = roof_dec
         if not args.decode_only:
             # The compression kernel takes most of a step, so it is the step's dominant kernel.
-            csha = source_sha(COMPRESS_SOURCES)
             comp_bytes = in_bytes + packed_bytes
             comp_k_mean = statistics.fmean(comp_k) / 1e3
             # d = m = 128 with the Hadamard rotation: bf16 keys (symmetric Lloyd-Max codebook) take
@@ -607,11 +653,12 @@ def run_ours(args, w: W.Workload):
             tc = w.d == 128 and w.m == 128 and w.rotation == "hadamard"
             ckern = ("compress_pipe_kernel" if w.dtype == "bf16" else "compress_q4_kernel") if tc \
                 else "compress_kernel"
+            csha = source_sha(KERNEL_SOURCES[ckern])
             roof = {"kernel": ckern, "bound": "hbm", "achieved": comp_bytes / comp_k_mean / 1e9, "peak": peak,
                     "unit": "GB/s", "frac": comp_bytes / comp_k_mean / 1e9 / peak, "peak_kind": peak_kind,
                     "alg_bytes_per_launch": comp_bytes, "alg_bytes_per_unit": comp_bytes // n_vec,
                     "unit_of_work": "key + value vector pair",
-                    "traffic": recorded_traffic("compress_kernel_traffic.txt", csha, n_vec, ckern),
+                    "traffic": recorded_traffic(csha, n_vec, ckern),
                     "source_sha256_16": csha}
         line = {
             "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -633,6 +680,8 @@ def run_ours(args, w: W.Workload):
             "paged": paged_line,
             "roofline": roof,
             "roofline_decode": roof_dec,
+            "decode_kernel": KERNEL_NAMES[fam],
+            "decode_alternatives": alt or None,
             "configs": side,
             "cpu_baseline": cpu,
             "e2e": e2e,

@@ -299,6 +299,35 @@ size_t tq_decode_static_scratch_capacity(void);
  * both disables it. Not thread-safe with concurrent calls on the same context. */
 tq_status tq_set_profile_events(tq_ctx* ctx, void* start, void* stop);
 
+/* Which decode attention kernel family a context uses. Every family computes the
+ * same results within the decode tolerance; they differ in speed and coverage.
+ *   TQ_DECODE_AUTO      the fastest family that supports the shape (default)
+ *   TQ_DECODE_TCGEN05   key scores and value sums on the 5th-generation tensor cores
+ *                       (tcgen05, accumulators in tensor memory): d = 128, m = 128 or 0,
+ *                       1- to 3-bit codes of a symmetric codebook, 2- or 4-bit values,
+ *                       at most 8 query heads per KV head
+ *   TQ_DECODE_MMA       warp-level tensor-core MMAs (mma.sync) over the packed bits:
+ *                       d = m = 128, 1- or 2-bit codes of a symmetric codebook, 2- or
+ *                       4-bit values, at most 8 query heads per KV head
+ *   TQ_DECODE_CUDA_CORE the generic kernels: every shape the library accepts */
+typedef enum {
+  TQ_DECODE_AUTO = 0,
+  TQ_DECODE_TCGEN05 = 1,
+  TQ_DECODE_MMA = 2,
+  TQ_DECODE_CUDA_CORE = 3
+} tq_decode_kernel;
+
+/* Select the decode kernel family for later decode calls on this context (all of
+ * tq_decode_attention, _paged, _partial and _static). A family that does not support
+ * a call's shape makes that call return TQ_EUNSUPPORTED; TQ_DECODE_AUTO never does.
+ * The workspace size (tq_decode_workspace_bytes) depends on the family: query it
+ * after selecting. Not thread-safe with concurrent calls on the same context. */
+tq_status tq_set_decode_kernel(tq_ctx* ctx, tq_decode_kernel kernel);
+
+/* The family a decode call with these head counts would run on this context, or -1
+ * if the selected family does not support the shape (no GPU work). */
+int tq_decode_kernel_for(const tq_ctx* ctx, int hq, int hkv);
+
 /* Decompress n_vec packed keys and/or values to fp32 [n_vec][d] (debug / parity;
  * not on the hot path). Keys: x = n Pi^T (c[idx] + sqrt(pi/2)/m * gamma * S^T s).
  * Values: min + scale * code. Pass NULL for the half to skip. */

@@ -10,5 +10,7 @@ from ._lib import (  # noqa: F401
     tq_decode_attention_paged, tq_decode_attention_partial, tq_merge_attention,
     tq_decode_workspace_bytes, tq_decompress, tq_haar_from_gaussian, tq_lloyd_max_codebook,
     tq_status_string, tq_set_profile_events, tq_check_device, tq_decode_attention_static,
-    tq_decode_static_scratch_capacity, EXPORTED, LIB_PATH, TQ_F32, TQ_BF16, TQ_ROT_HADAMARD, TQ_ROT_HAAR,
+    tq_decode_static_scratch_capacity, tq_set_decode_kernel, tq_decode_kernel_for, EXPORTED, LIB_PATH, TQ_F32,
+    TQ_BF16, TQ_ROT_HADAMARD, TQ_ROT_HAAR, TQ_DECODE_AUTO, TQ_DECODE_TCGEN05, TQ_DECODE_MMA, TQ_DECODE_CUDA_CORE,
+    DECODE_KERNEL_NAMES,
 )

@@ -18,13 +18,15 @@ LIB_PATH = os.environ.get("TQ_LIBRARY") or os.path.join(os.path.dirname(os.path.
 TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED, TQ_ECUDA, TQ_ENOMEM = 0, 1, 2, 3, 4
 TQ_F32, TQ_BF16 = 0, 1
 TQ_ROT_HADAMARD, TQ_ROT_HAAR = 0, 1
+TQ_DECODE_AUTO, TQ_DECODE_TCGEN05, TQ_DECODE_MMA, TQ_DECODE_CUDA_CORE = 0, 1, 2, 3
+DECODE_KERNEL_NAMES = {TQ_DECODE_TCGEN05: "tcgen05", TQ_DECODE_MMA: "mma", TQ_DECODE_CUDA_CORE: "cuda_core"}
 
 EXPORTED = (
     "tq_codebook_load", "tq_free", "tq_status_string", "tq_last_error",
     "tq_lloyd_max_codebook", "tq_haar_from_gaussian", "tq_compress_kv", "tq_compress_kv_slots",
     "tq_decode_workspace_bytes", "tq_decode_attention", "tq_decode_attention_paged", "tq_decompress",
     "tq_set_profile_events", "tq_check_device", "tq_decode_attention_static", "tq_decode_static_scratch_capacity",
-    "tq_decode_attention_partial", "tq_merge_attention",
+    "tq_decode_attention_partial", "tq_merge_attention", "tq_set_decode_kernel", "tq_decode_kernel_for",
 )
 
 
@@ -97,6 +99,10 @@ def _load() -> ctypes.CDLL:
     lib.tq_check_device.restype = c_int
     lib.tq_set_profile_events.argtypes = [vp, vp, vp]
     lib.tq_set_profile_events.restype = c_int
+    lib.tq_set_decode_kernel.argtypes = [vp, c_int]
+    lib.tq_set_decode_kernel.restype = c_int
+    lib.tq_decode_kernel_for.argtypes = [vp, c_int, c_int]
+    lib.tq_decode_kernel_for.restype = c_int
     return lib
 
 
@@ -226,6 +232,16 @@ def tq_set_profile_events(ctx: Context, start=None, stop=None) -> None:
     _check(lib.tq_set_profile_events(ctx.handle, None if start is None else ctypes.c_void_p(start.cuda_event),
                                      None if stop is None else ctypes.c_void_p(stop.cuda_event)),
            "tq_set_profile_events")
+
+
+def tq_set_decode_kernel(ctx: Context, kernel: int) -> None:
+    """Select the decode kernel family (TQ_DECODE_AUTO, _TCGEN05, _MMA or _CUDA_CORE) of later calls."""
+    _check(lib.tq_set_decode_kernel(ctx.handle, int(kernel)), "tq_set_decode_kernel")
+
+
+def tq_decode_kernel_for(ctx: Context, hq: int, hkv: int) -> int:
+    """The decode kernel family a call with these head counts runs on `ctx` (-1: unsupported)."""
+    return int(lib.tq_decode_kernel_for(ctx.handle, hq, hkv))
 
 
 def tq_compress_kv(ctx: Context, k, v, k_codes=None, k_signs=None, k_norms=None,

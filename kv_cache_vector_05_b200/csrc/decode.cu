@@ -373,8 +373,19 @@ cudaError_t dispatch_lmb(const DecodeArgs& a, int lmb, int vb, dim3 grid, size_t
 DecodePlan plan_decode(const tq_ctx* ctx, int batch, int hq, int hkv, int64_t max_len) {
   DecodePlan p{};
   const int d = ctx->shape.d, m = ctx->shape.m, G = hq / hkv;
-  p.tc = tc_decode_supported(ctx, G);
-  p.mma = !p.tc && mma_decode_supported(ctx, G);
+  // TQ_DECODE_AUTO: mma.sync where it applies (1- and 2-bit codes with the QJL stage, the
+  // faster of the two tensor-core kernels on those shapes), then tcgen05, then the generic
+  // kernels. A family selected explicitly runs or the call is refused.
+  const bool tc_ok = tc_decode_supported(ctx, G), mma_ok = mma_decode_supported(ctx, G);
+  p.supported = true;
+  switch (ctx->decode_kernel) {
+    case TQ_DECODE_TCGEN05: p.tc = tc_ok; p.supported = tc_ok; break;
+    case TQ_DECODE_MMA: p.mma = mma_ok; p.supported = mma_ok; break;
+    case TQ_DECODE_CUDA_CORE: break;
+    default: p.mma = mma_ok; p.tc = !mma_ok && tc_ok; break;
+  }
+  p.family = p.tc ? TQ_DECODE_TCGEN05 : p.mma ? TQ_DECODE_MMA : TQ_DECODE_CUDA_CORE;
+  if (!p.supported) return p;
   const int64_t units = (int64_t)batch * hkv;
   const int64_t sms = ctx->num_sms > 0 ? ctx->num_sms : 148;
   if (p.tc) {

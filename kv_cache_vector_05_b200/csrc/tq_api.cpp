@@ -228,6 +228,19 @@ tq_status tq_set_profile_events(tq_ctx* c, void* start, void* stop) {
   return TQ_OK;
 }
 
+tq_status tq_set_decode_kernel(tq_ctx* c, tq_decode_kernel k) {
+  if (!c) return fail(TQ_EINVAL, "tq_set_decode_kernel: NULL context");
+  if (k < TQ_DECODE_AUTO || k > TQ_DECODE_CUDA_CORE) return fail(TQ_EINVAL, "tq_set_decode_kernel: unknown kernel");
+  c->decode_kernel = (int)k;
+  return TQ_OK;
+}
+
+int tq_decode_kernel_for(const tq_ctx* c, int hq, int hkv) {
+  if (!c || hq <= 0 || hkv <= 0 || hq % hkv) return -1;
+  const tq::DecodePlan p = tq::plan_decode(c, 1, hq, hkv, 1);
+  return p.supported ? p.family : -1;
+}
+
 tq_status tq_check_device(const tq_ctx* c, void* stream) {
   if (!c) return fail(TQ_EINVAL, "tq_check_device: NULL context");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -323,6 +336,7 @@ tq_status decode_impl(const char* name, const tq_ctx* c, const void* q, tq_dtype
     if (ptr && !aligned16(ptr)) return fail(TQ_EINVAL, nm + ": pointers must be 16-byte aligned");
   if (max_len > (int64_t(1) << 31)) return fail(TQ_EINVAL, nm + ": max_len too large");
   tq::DecodePlan plan = tq::plan_decode(c, batch, hq, hkv, max_len);
+  if (!plan.supported) return fail(TQ_EUNSUPPORTED, nm + ": the selected decode kernel does not support this shape");
   if (!workspace || workspace_bytes < plan.total_bytes)
     return fail(TQ_EINVAL, nm + ": workspace missing or too small");
   float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)c->shape.d);

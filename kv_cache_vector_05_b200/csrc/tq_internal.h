@@ -53,6 +53,7 @@ struct tq_ctx {
   float* St;       // device [d][m] fp32 (transpose of S)
   float* Pi;       // device [d][d] fp32 row-major (Haar only)
   float* PiT;      // device [d][d] fp32 transpose (Haar only)
+  int decode_kernel;       // tq_decode_kernel selected by tq_set_decode_kernel
   cudaEvent_t prof_start;  // optional events around the main kernel of each call
   cudaEvent_t prof_stop;
   unsigned int* d_err;     // device error word: bit 0 = a bounded wait in a kernel timed out,
@@ -73,6 +74,8 @@ cudaError_t launch_compress(const tq_ctx* ctx, const void* k, const void* v, int
                             cudaStream_t stream);
 
 struct DecodePlan {
+  bool supported;    // false: the context's selected kernel family does not take the shape
+  int family;        // tq_decode_kernel that runs (never TQ_DECODE_AUTO)
   bool tc;           // tcgen05 score kernels (decode_tc.cu)
   bool mma;          // mma.sync kernels (decode_mma.cu) instead of the generic ones
   int n_chunks;      // split-K chunks per (sequence, KV head)

@@ -246,11 +246,18 @@ def _oracle_unit(packed, u, max_len, length, q, Pi, c, S, d, v_bits, scale=None)
     return O.decode_attention(q, pk, pv, Pi, c, S, d, v_bits, scale=scale)
 
 
+KERNELS = {"tcgen05": T.TQ_DECODE_TCGEN05, "mma": T.TQ_DECODE_MMA, "cuda_core": T.TQ_DECODE_CUDA_CORE}
+
+
 def _decode_check(d, lm_bits, v_bits, batch, hkv, G, max_len, lens, rotation="hadamard",
-                  q_dtype="f32", packed=None, units=None, scale=0.0, with_scores=True):
+                  q_dtype="f32", packed=None, units=None, scale=0.0, with_scores=True, kernel=None):
     m = d
     hq = hkv * G
     ctx = make_ctx(T, d, lm_bits, v_bits, m, rotation)
+    if kernel is not None:
+        T.tq_set_decode_kernel(ctx, KERNELS[kernel])
+        if T.tq_decode_kernel_for(ctx, hq, hkv) != KERNELS[kernel]:
+            pytest.skip(f"the {kernel} decode does not take this shape")
     n_vec = batch * hkv * max_len
     if packed is None:
         packed = W.random_packed_cache(n_vec, d, lm_bits, m, v_bits, seed=d + lm_bits)
@@ -309,6 +316,42 @@ def test_decode_parity_random_cache(d, lm_bits, v_bits, G):
     _decode_check(d, lm_bits, v_bits, batch=2, hkv=2, G=G, max_len=1100, lens=[1100, 577])
 
 
+@pytest.mark.parametrize("kernel", ["tcgen05", "mma", "cuda_core"])
+@pytest.mark.parametrize("lm_bits,v_bits,G", [(2, 2, 4), (2, 4, 8), (1, 2, 3), (3, 4, 6), (2, 2, 1)])
+def test_decode_each_kernel_family(kernel, lm_bits, v_bits, G):
+    """Every decode kernel family, selected explicitly, on the shapes it takes: the same
+    packed cache decodes to the oracle's scores and outputs whichever kernel runs."""
+    _decode_check(128, lm_bits, v_bits, batch=2, hkv=2, G=G, max_len=1500, lens=[1500, 701], kernel=kernel)
+
+
+def test_decode_kernel_selection():
+    """TQ_DECODE_AUTO takes the mma.sync kernel for 1- and 2-bit codes with the QJL stage,
+    the tcgen05 kernel for 3-bit codes or keys without QJL, and the generic kernels for
+    every other shape; an explicitly selected family that does not take the shape refuses
+    the call."""
+    ctx = make_ctx(T, 128, 2, 2)
+    assert T.tq_decode_kernel_for(ctx, 32, 8) == T.TQ_DECODE_MMA
+    assert T.tq_decode_kernel_for(ctx, 64, 2) == T.TQ_DECODE_CUDA_CORE        # G = 32
+    ctx3 = make_ctx(T, 128, 3, 4)
+    assert T.tq_decode_kernel_for(ctx3, 24, 4) == T.TQ_DECODE_TCGEN05
+    T.tq_set_decode_kernel(ctx3, T.TQ_DECODE_MMA)
+    assert T.tq_decode_kernel_for(ctx3, 24, 4) == -1
+    packed = _upload(W.random_packed_cache(4 * 256, 128, 3, 128, 4))
+    q = torch.randn((1, 24, 128), device=DEV)
+    with pytest.raises(T.TQError):
+        T.tq_decode_attention(ctx3, q, packed, 1, 24, 4, 256)
+    T.tq_set_decode_kernel(ctx3, T.TQ_DECODE_AUTO)
+    out, _ = T.tq_decode_attention(ctx3, q, packed, 1, 24, 4, 256)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out).all()
+    dr = W.method_draws(128, 128, 1234)
+    c2, t2 = T.tq_lloyd_max_codebook(128, 2)
+    ctx0 = T.tq_codebook_load(128, 2, 2, c2, t2, np.zeros((0, 128)), hadamard_signs=dr["hadamard_signs"])
+    assert T.tq_decode_kernel_for(ctx0, 32, 8) == T.TQ_DECODE_TCGEN05
+    ctx64 = make_ctx(T, 64, 2, 2)
+    assert T.tq_decode_kernel_for(ctx64, 32, 8) == T.TQ_DECODE_CUDA_CORE
+
+
 @pytest.mark.parametrize("G", [4, 8])
 def test_decode_ragged_sequences_many_tiles_per_cta(G):
     """Ragged sequence lengths with several tiles per CTA: the work split hands a CTA a
@@ -346,9 +389,10 @@ def test_decode_parity_full_size_sampled(name, units):
                   q_dtype=w.dtype, packed=packed, units=units, with_scores=(name != "long_1m_k4v4"))
 
 
+@pytest.mark.parametrize("kernel", ["tcgen05", "mma", "cuda_core"])
 @pytest.mark.parametrize("d,lm_bits,v_bits,G", [(128, 2, 2, 4), (128, 2, 4, 8), (128, 3, 4, 6)])
 @pytest.mark.parametrize("k_norm_scale", [10.0, 30.0])
-def test_decode_parity_large_key_norms(d, lm_bits, v_bits, G, k_norm_scale):
+def test_decode_parity_large_key_norms(d, lm_bits, v_bits, G, k_norm_scale, kernel):
     """Key norms 10-30 times those of a unit-variance key (the Qwen-shaped cache's outlier
     channels give such norms): logits reach tens, the softmax is sharply peaked, and the
     online softmax rescales often. Some value groups get scales 100x larger, one a zero
@@ -362,7 +406,7 @@ def test_decode_parity_large_key_norms(d, lm_bits, v_bits, G, k_norm_scale):
     vp[..., 0][big] = (vp[..., 0][big].astype(np.float64) * 100.0).astype(np.float16)
     vp[3, 1, 0] = 0.0                                                     # a constant group
     packed["v_params"] = vp.view(np.uint16)
-    _decode_check(d, lm_bits, v_bits, batch, hkv, G, max_len, lens=[3000, 2049], packed=packed)
+    _decode_check(d, lm_bits, v_bits, batch, hkv, G, max_len, lens=[3000, 2049], packed=packed, kernel=kernel)
 
 
 @pytest.mark.parametrize("layers", [(0, 17, 35)])
