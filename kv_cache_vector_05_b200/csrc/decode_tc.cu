@@ -28,15 +28,16 @@
 //    96-bit stream XORed with itself shifted by one and by two, bit 3j of X is code j's
 //    parity, and the bits 3j fall on distinct positions of the three 32-bit words (0, 1, 2
 //    mod 3), so one word keeps them all: bit p holds code (32 (p mod 3) + p) / 3.
-// Values. out = sum_t p_t (min + scale * code), also on the tensor cores (kind::f16, f32 sums
-// in tensor memory): rows = the 128 value coordinates, K = the tile's tokens, columns = (value
-// group, query head). A 2- or 4-bit code masked into the low mantissa bits of an f16 is an
-// exact subnormal, code * 2^(position - 24), so one AND makes two elements; the power of two
-// depends only on the row and is undone at the end. The A operand sits in shared memory
-// MN-major (each token's 128 elements contiguous, as the expansion writes them), and so does
-// B, p * scale as an f16 high part and low part (an exact TwoProduct), each its own K pass
-// into the same sums. Only the column of the row's own value group is read back. The group
-// minima, sum_t p_t min_t, are fp32 sums per thread.
+// Values. out = sum_t p_t (min + scale * code) on warp-level tensor-core MMAs (mma.sync
+// m16n8k16, f16 operands built in registers, fp32 sums in registers): rows = 16 value
+// coordinates, K = 16 tokens, columns = 4 query heads x (high, low part of p * scale). A 2- or
+// 4-bit code masked into the low mantissa bits of an f16 is an exact subnormal, code *
+// 2^(position - 24): a byte permute pairs the same code byte of two tokens and one AND makes
+// two elements; the power of two depends only on the row and is undone at the end. p * scale
+// is an exact TwoProduct in half2 (high part rounded, low part = the rounding error plus
+// p_low * scale). The group minima, sum_t p_t min_t, are fp32 sums per thread. (Value
+// operands staged in shared memory for tcgen05 cost 512 bytes of shared-memory traffic per
+// token; in registers they cost none.)
 // Online softmax in base 2 with one reference maximum per query head for a group of warps,
 // moved only when a logit exceeds it by more than 2 (p < 4, so p * scale stays finite in f16
 // for value scales below 16376); when it moves, the sums so far are rescaled in place.
@@ -46,13 +47,14 @@
 //   one producer warp streams the packed records into a ring of two-tile stages (one bulk
 //   copy per array and stage; a ragged or unaligned tile is copied by the warp) and loads
 //   each unit's query operand (digits + logit constants) when the unit's first tile goes;
-//   groups of four warps take the tiles in turn, one token per thread: expand the key bits
-//   into tensor memory and the value codes into the group's value operand, release the
-//   stage, then (one elected thread) the score MMAs; read the digit sums back, logits,
-//   online softmax, value weights; then the value MMAs. Each group has its own tensor-memory
-//   columns (key elements, digit sums, value sums) and value operands, so one group's MMAs
-//   overlap the others' arithmetic. At the end of a unit each group writes one partial
-//   (m, l, acc) per query head; combine_partials merges them in a fixed order.
+//   groups of four compute warps take the tiles in turn, one token per thread: a group waits
+//   for tile k's digit sums, reads them and forms the logits, writes tile k + 1's key
+//   elements into its tensor-memory A operand, and only then runs tile k's online softmax
+//   and value MMAs, so that tile k + 1's score MMAs overlap them;
+//   one MMA warp per group issues the group's score MMAs as soon as a tile's key elements
+//   are written (a tcgen05.mma holds its issuing warp for tens of nanoseconds; no compute
+//   warp waits on that). At the end of a unit each group writes one partial (m, l, acc) per
+//   query head; combine_partials merges them in a fixed order.
 // Every wait is bounded: on a timeout the CTA raises an abort flag that every warp polls,
 // sets the context's error word, drains the copies and MMAs it issued and returns.
 #include <cuda_runtime.h>
@@ -92,15 +94,13 @@ struct TcLayout {
   static constexpr int KB = 32 * EW;                   // bytes of one B row
   static constexpr int NC = kDigits * HG;              // code columns (4 digits per head)
   static constexpr int N = ((NC + (QJL ? NC : 0)) + 15) / 16 * 16;
-  static constexpr int NV = 4 * HG;                    // value weights per part: (value group, head)
   static constexpr int TA = 8 * EW;                    // tensor-memory columns: key elements
-  // Value sums: with VSPLIT the high and low parts of the weights are separate columns
-  // (g, part, h) of one MMA pass, reading the codes once; otherwise (too few tensor-memory
-  // columns for two groups) they are two passes into the same columns (g, h).
-  static constexpr int groups_fit(int cols) { return 512 / cols >= 3 ? 3 : 512 / cols; }
-  static constexpr bool VSPLIT = groups_fit(TA + N + 2 * NV) >= 2 && groups_fit(TA + N + 2 * NV) == groups_fit(TA + N + NV);
-  static constexpr int NVC = VSPLIT ? 2 * NV : NV;     // value-sum columns
-  static constexpr int TG = TA + N + NVC;              // per group: key elements, scores, value sums
+  static constexpr int TG = TA + N;                    // per group: key elements, digit sums
+  // Groups of four compute warps, one tile each: as many as tensor memory holds, at most 3 (at
+  // most 2 with two head blocks, whose value sums take twice the registers).
+  static constexpr int NG_MAX = NB == 1 ? 3 : 2;
+  static constexpr int NG = 512 / TG >= NG_MAX ? NG_MAX : 512 / TG;
+  static_assert(NG >= 2, "tensor memory for two groups");
   // A stage holds two tiles (256 tokens): each array of the pair arrives with one bulk copy,
   // [kc 256 x KCB][ks 256 x SB][kn 256 x 4][vc 256 x VCB][vp 256 x PB]; tile k of the pair sits
   // 128 k records into each region. (Copies of 128 records streamed at under 60% of the HBM
@@ -113,50 +113,31 @@ struct TcLayout {
   static constexpr int BOP = N * KB;                   // digits, K-major, 128-byte swizzle
   static constexpr int BBUF = BOP + HG * 16;           // + logit constants (float4 per head)
   static constexpr int BBUF_AL = (BBUF + 1023) / 1024 * 1024;
-  // Value operands of a group, f16, MN-major without swizzle: core matrices of 8 rows (value
-  // coordinates, or weight columns) x 8 tokens, 128 B each, 128 B apart along the tokens and
-  // 2048 B apart along the rows. The codes [128 rows][128 tokens], then the value weights
-  // p * scale: with VSPLIT one operand [(g, part, h)][128 tokens], else the high and the low
-  // parts [(g, h)][128 tokens] one after the other.
-  static constexpr int AV = kD * kTileTc * 2;
-  static constexpr int BVP = NV * kTileTc * 2;
-  static constexpr int GV = AV + 2 * BVP;
-  static constexpr int RED_F = 5 * HG;                 // per warp: minima sums [HG][4], sums of p [HG]
-  static constexpr int NBAR = 2 * 6 + 2 * 3 + 2;       // full, empty [<= 6]; mmad, vdone [<= 3]; fbfull [2]
-  // Shared memory in front of the stage ring for ng groups and nbuf query-operand buffers, and
-  // the stages that fit behind it.
-  static constexpr int front(int ng, int nbuf) {
-    return (nbuf * BBUF_AL + ng * GV + ng * 4 * RED_F * 4 + ng * 4 * 8 * 4 + 8 * NBAR + 8 + 4 * ng + 127) / 128 * 128;
-  }
-  static constexpr int fit(int ng, int nbuf) {
-    return (227 * 1024 - 1024 - front(ng, nbuf)) / STAGE > 6 ? 6 : (227 * 1024 - 1024 - front(ng, nbuf)) / STAGE;
-  }
-  // Group g consumes tiles g, g + ng, ...; tile i sits in stage (i / 2) mod NST. With 2 NST a
-  // multiple of ng, the previous use of a group's stage held a tile of the same group, so the
-  // phase a group waits for can never be confused with the one two uses back.
-  static constexpr int stages(int ng, int nbuf) { return ng == 3 ? fit(3, nbuf) / 3 * 3 : fit(ng, nbuf); }
-  // Groups of four warps, one tile each: as many as tensor memory holds, at most 3, and 2 if
-  // three would leave fewer than three stages. Two query-operand buffers (the next unit's
-  // loads while the current one runs) when three stages remain beside them, else one.
-  static constexpr int NG_TM = 512 / TG >= 3 ? 3 : 512 / TG;
-  static_assert(NG_TM >= 2, "tensor memory for two groups");
-  static constexpr int NG = (NG_TM >= 3 && stages(3, 1) >= 3) ? 3 : 2;
-  static constexpr int NBUF = stages(NG, 2) >= 3 ? 2 : 1;
-  static constexpr int NST = stages(NG, NBUF);
-  static_assert(NST >= 2 && NST <= 6, "stages");
+  static constexpr int NBUF = 2;                       // query-operand buffers (next unit's loads)
   static constexpr int NCW = 4 * NG;                   // compute warps
-  static constexpr int THREADS = 32 * (NCW + 1);       // + the producer warp
+  static constexpr int THREADS = 32 * (NCW + 1 + NG);  // + the producer warp + one MMA warp per group
+  // Per compute warp: the probabilities of its 32 tokens as f16 high and low parts, [2][HG][32],
+  // read back in the B-fragment layout of the value MMAs.
+  static constexpr int PT = 2 * HG * 32 * 2;
+  static constexpr int RED_F = 5 * HG;                 // per warp: minima sums [HG][4], sums of p [HG]
+  static constexpr int NBAR = 2 * 6 + 3 + 3 + 2;       // full, empty [<= 6]; afull, mmad [<= 3]; fbfull [2]
   static constexpr int SM_B = 0;                                   // [NBUF] query operands
-  static constexpr int SM_V = NBUF * BBUF_AL;                      // [NG] value operands
-  static constexpr int SM_RED = SM_V + NG * GV;                    // [NG][4 warps][RED_F]
-  static constexpr int SM_RM = SM_RED + NG * 4 * RED_F * 4;        // [NG][4 warps][8] warp maxima
+  static constexpr int SM_PT = NBUF * BBUF_AL;                     // [NCW] probability parts
+  static constexpr int SM_RED = SM_PT + NCW * PT;                  // [NG][4 warps][128] value sums of a head
+  static constexpr int SM_REDF = SM_RED + NG * 4 * kD * 4;         // [NG][4 warps][RED_F]
+  static constexpr int SM_RM = SM_REDF + NG * 4 * RED_F * 4;       // [NG][4 warps][8] warp maxima
   static constexpr int SM_BAR = SM_RM + NG * 4 * 8 * 4;
   static constexpr int SM_MISC = SM_BAR + 8 * NBAR;                // TMEM address, abort flag, grp_unit[NG]
   static constexpr int SM_RING = (SM_MISC + 8 + 4 * NG + 127) / 128 * 128;
-  static_assert(SM_RING == front(NG, NBUF), "layout");
+  static constexpr int FIT = (227 * 1024 - 1024 - SM_RING) / STAGE > 6 ? 6 : (227 * 1024 - 1024 - SM_RING) / STAGE;
+  // Group g consumes tiles g, g + NG, ...; tile i sits in stage (i / 2) mod NST. With 2 NST a
+  // multiple of NG, the previous use of a group's stage held a tile of the same group, so the
+  // phase a group waits for can never be confused with the one two uses back.
+  static constexpr int NST = NG == 3 ? FIT / 3 * 3 : FIT;
+  static_assert(NST >= 2 && NST <= 6, "stages");
   static constexpr size_t SMEM = (size_t)SM_RING + (size_t)NST * STAGE + 1024;
   static_assert(SMEM <= 227 * 1024, "shared memory");
-  static_assert(STAGE % 16 == 0 && BBUF % 16 == 0 && SM_V % 1024 == 0 && GV % 16 == 0, "alignment");
+  static_assert(STAGE % 16 == 0 && BBUF % 16 == 0 && SM_PT % 16 == 0, "alignment");
 };
 
 struct TcArgs {
@@ -290,47 +271,6 @@ __device__ __forceinline__ uint32_t parity_word(uint32_t x0, uint32_t x1, uint32
   const uint32_t X1 = x1 ^ __funnelshift_r(x1, x2, 1) ^ __funnelshift_r(x1, x2, 2);
   const uint32_t X2 = x2 ^ (x2 >> 1) ^ (x2 >> 2);
   return (X0 & 0x49249249u) | (X1 & 0x92492492u) | (X2 & 0x24924924u);
-}
-
-// 16-byte shared-memory store.
-__device__ __forceinline__ void st_shared_v4(void* p, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_addr(p)), "r"(x), "r"(y), "r"(z), "r"(w)
-               : "memory");
-}
-
-// Instruction descriptor, kind::f16: f16 x f16 -> f32, both operands MN-major.
-__host__ __device__ constexpr uint32_t idesc_f16_mn(int M, int N) {
-  return (1u << 4)                       // D format f32
-         | (1u << 15) | (1u << 16)       // A and B MN-major
-         | ((uint32_t)(N >> 3) << 17)    // N / 8
-         | ((uint32_t)(M >> 4) << 24);   // M / 16
-}
-
-// Shared-memory descriptor of an MN-major operand without swizzle: core matrices of 8 rows x
-// 8 tokens (128 B: 16 B per token), 128 B apart along the tokens (leading byte offset) and
-// 2048 B apart along the rows (stride byte offset), sm_100 version bit, layout 0.
-__device__ __forceinline__ uint64_t desc_mn(uint32_t addr) {
-  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)(128u >> 4) << 16) | ((uint64_t)(2048u >> 4) << 32) |
-         ((uint64_t)1u << 46);
-}
-
-// Row m of the value MMA (tensor-memory lane m of the value sums) holds value coordinate
-// value_coord(m), its code times 2^-value_unscale-exponent (a code in bits b .. of an f16 is
-// the subnormal code * 2^(b - 24)). 2-bit codes: word w of a record (coordinates 16 w ..)
-// gives row chunks 2 w (bytes 0 and 2: codes 0, 1 at bits 6, 8 of the word shifted left by
-// 6, codes 2, 3 of the word shifted left by 2) and 2 w + 1 (bytes 1 and 3, shifted right
-// by 2 and 6). 4-bit codes: word w (coordinates 8 w ..) gives row chunk w, every code at bit
-// 6 (low and high nibbles of bytes 0, 2, then of bytes 1, 3). Either way rows 32 g .. 32 g +
-// 31 are value group g.
-template <int VB>
-__device__ __forceinline__ int value_coord(int m) {
-  if constexpr (VB == 2) return 16 * (m >> 4) + 4 * ((m >> 3) & 1) + ((m & 7) >> 1) + 8 * (m & 1);
-  else return 8 * (m >> 3) + ((m & 7) >> 1) + 4 * (m & 1);
-}
-template <int VB>
-__device__ __forceinline__ float value_unscale(int m) {
-  if constexpr (VB == 2) return __int_as_float((127 + 18 - 2 * (((m & 7) >> 1) & 1)) << 23);
-  else return __int_as_float((127 + 18) << 23);
 }
 
 // Walks a CTA's tiles in order without dividing: the unit, the tile within it, the unit's
@@ -550,6 +490,19 @@ __global__ void __launch_bounds__(kPrepTcThreads) prep_tc_kernel(const __grid_co
 
 // ------------------------------------------------------------------ decode kernel
 
+// D (fp32) += A (f16) x B (f16), m16n8k16, A row-major, B column-major (warp-level MMA).
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint4& a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t word_of(const uint4& w, int i) {
+  return i == 0 ? w.x : i == 1 ? w.y : i == 2 ? w.z : w.w;
+}
+
 template <int LMB, bool QJL, int VB, int NB>
 __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
     decode_tc_kernel(const __grid_constant__ TcArgs a) {
@@ -562,8 +515,8 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::SM_BAR);
   uint64_t* full = bars;           // [NST] stage landed
   uint64_t* empty = bars + 6;      // [NST] both tiles of the stage read (2 x 4 warps)
-  uint64_t* mmad = bars + 12;      // [NG] the group's score MMAs done (commit)
-  uint64_t* vdone = bars + 15;     // [NG] the group's value MMAs done (commit)
+  uint64_t* afull = bars + 12;     // [NG] the group's key elements of its next tile written (4 warps)
+  uint64_t* mmad = bars + 15;      // [NG] the group's score MMAs done (commit)
   uint64_t* fbfull = bars + 18;    // [NBUF] query operand landed
   uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + L::SM_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::SM_MISC + 4);
@@ -589,8 +542,8 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
       s1::mbar_init(&empty[s], 8);  // two tiles x four warps
     }
     for (int g = 0; g < NG; ++g) {
+      s1::mbar_init(&afull[g], 4);  // four warps
       s1::mbar_init(&mmad[g], 1);
-      s1::mbar_init(&vdone[g], 1);
       grp_unit[g] = -1;
     }
     for (int b = 0; b < NBUF; ++b) s1::mbar_init(&fbfull[b], 1);
@@ -739,64 +692,89 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
       for (int jj = (b_issued > NBUF ? b_issued - NBUF : 0); jj < b_issued; ++jj)
         s1::mbar_wait(&fbfull[jj % NBUF], (uint32_t)(jj / NBUF) & 1u);
     }
+  } else if (warp > L::NCW) {
+    // ============================================================ MMA warps
+    // Warp NCW + 1 + g issues the score MMAs of group g's tiles, in order: once the group's
+    // four warps have written a tile's key elements (afull), D = A x B over the tile's element
+    // words, committed to mmad. The query operand of each unit is waited for in unit order
+    // (every unit's phase, also of units the group has no tile of, so that no phase of a
+    // buffer is skipped).
+    const int gi = warp - L::NCW - 1;
+    const uint32_t tgrp = tmem + gi * L::TG;
+    int cur = -1, kt = 0, issued = 0;
+    for (int k = 0; k < gi; ++k) walk.next();
+    for (int i = gi; i < ntl; i += NG, ++kt) {
+      const int j = walk.u - u_first;
+      for (int k = 0; k < NG; ++k) walk.next();
+      if (lane == 0 && !failed) {
+        for (int jj = cur + 1; jj <= j && !failed; ++jj)
+          if (!wait_phase(&fbfull[jj % NBUF], (uint32_t)(jj / NBUF) & 1u, abort_flag)) failed = true;
+        cur = j;
+        if (!failed && !wait_phase(&afull[gi], (uint32_t)kt & 1u, abort_flag)) failed = true;
+        if (!failed) {
+          s1::fence_after_sync();
+          constexpr uint32_t idesc = idesc_u8s8_s32(kTileTc, L::N);
+          const uint32_t bbase = smem_addr(sm + L::SM_B + (j % NBUF) * L::BBUF_AL);
+          const uint32_t d_tm = tgrp + L::TA;
+#pragma unroll
+          for (int ks = 0; ks < L::EW; ++ks)
+            umma_i8_ts(d_tm, tgrp + 8 * ks, s1::sw128_desc(bbase, 16 * ks, L::N), idesc, ks > 0 ? 1u : 0u);
+          s1::umma_commit(&mmad[gi]);
+          ++issued;
+        }
+      }
+    }
+    if (lane == 0) {
+      if (failed) raise_abort(abort_flag);
+      // the last commit lands before the tensor memory goes away
+      if (issued > 0) s1::mbar_wait(&mmad[gi], (uint32_t)(issued - 1) & 1u);
+    }
+    __syncwarp();
   } else {
     // ============================================================ compute warps
     // Group gi (warps 4 gi .. 4 gi + 3) takes tiles gi, gi + NG, ...; warp q of the group owns
-    // tokens 32 q .. 32 q + 31 of each tile (tensor-memory lanes 32 q ..), and for the value
-    // sums the 32 value coordinates of value group q (rows 32 q .. of the value MMA).
+    // tokens 32 q .. 32 q + 31 of each tile (tensor-memory lanes 32 q ..), one token per thread
+    // for the key elements, the logits and the online softmax. Tile k + 1's key elements are
+    // written while the MMA warp still works on tile k: the loop waits for tile k's digit sums,
+    // reads them, writes tile k + 1's elements (the MMA warp then issues its MMAs), and only
+    // then runs tile k's softmax and value sums, so the score MMAs overlap that work.
+    // Value sums run on warp-level MMAs (mma.sync m16n8k16, f16 operands from registers,
+    // fp32 sums in registers): rows = 16 value coordinates, K = 16 tokens, columns = 4 query
+    // heads x (high, low part of p * scale). Lane (r, c) holds rows r and r + 8 of each of the
+    // eight row blocks, for head 4 nb + c.
     const int gi = warp >> 2, q = warp & 3;
     const int R = 32 * q + lane;
+    const int r = lane >> 2, c = lane & 3;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     const uint32_t tgrp = tmem + gi * L::TG;
     const uint32_t tA = tgrp + lane_base, tD = tgrp + L::TA + lane_base;
-    // this warp's value-sum columns: group q's (part, h), or (h) without VSPLIT
-    const uint32_t tV = tgrp + L::TA + L::N + lane_base + q * (L::NVC / 4);
     const int bar_id = 1 + gi;
     const bool leader = q == 0 && lane == 0;
-    unsigned char* av = sm + L::SM_V + gi * L::GV;   // codes [16 row chunks][128 tokens]
-    unsigned char* bv = av + L::AV;                   // weights [2 NV / 8 row chunks][128 tokens]
-    float* red = reinterpret_cast<float*>(sm + L::SM_RED) + gi * 4 * L::RED_F;  // [4][RED_F]
-    float* rm = reinterpret_cast<float*>(sm + L::SM_RM) + gi * 32;              // [4][8]
-    // this thread's 16-byte slot of a row chunk: chunk c of token R at c * 2048 + the slot
-    const uint32_t slot_off = (uint32_t)((R >> 3) * 128 + (R & 7) * 16);
+    float* red = reinterpret_cast<float*>(sm + L::SM_RED) + gi * 4 * kD;             // [4][128]
+    float* redf = reinterpret_cast<float*>(sm + L::SM_REDF) + gi * 4 * L::RED_F;      // [4][RED_F]
+    float* rm = reinterpret_cast<float*>(sm + L::SM_RM) + gi * 32;                     // [4][8]
+    __half* pt = reinterpret_cast<__half*>(sm + L::SM_PT + warp * L::PT);             // [2][HG][32]
 
     // Per thread: the group's reference maxima, this token's share of the sums of p and of
-    // p * min, and (as value row R) the unit's value sums of row R, to which the tensor-memory
-    // sums of each tile are added in fp32 (sums kept in tensor memory over many tiles drift
-    // low: each MMA truncates its result).
-    float Mref[HG], lsum[HG], mn[HG][4], acc[HG];
-    bool vpend = false;  // tensor memory holds value sums of a tile not yet added to acc
+    // p * min; per lane the value sums (fragment layout).
+    float Mref[HG], lsum[HG], mn[HG][4];
+    float dv[4][2][NB][4];  // [value group][half of the group][n-block][fragment]
     auto reset = [&]() {
 #pragma unroll
       for (int h = 0; h < HG; ++h) {
         Mref[h] = -INFINITY;
         lsum[h] = 0.f;
-        acc[h] = 0.f;
 #pragma unroll
         for (int g = 0; g < 4; ++g) mn[h][g] = 0.f;
       }
-      vpend = false;
-    };
-    // add the last tile's value sums of row R (issue; tmem_ld_wait before use)
-    uint32_t dvv[L::NVC / 4];
-    auto load_vsums = [&]() {
-      if constexpr (L::NVC / 4 == 8) {
-        asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                     : "=r"(dvv[0]), "=r"(dvv[1]), "=r"(dvv[2]), "=r"(dvv[3]), "=r"(dvv[4]), "=r"(dvv[5]),
-                       "=r"(dvv[6]), "=r"(dvv[7])
-                     : "r"(tV));
-      } else if constexpr (L::NVC / 4 == 4) {
-        asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(dvv[0]), "=r"(dvv[1]), "=r"(dvv[2]), "=r"(dvv[3])
-                     : "r"(tV));
-      } else {
-        tmem_ld16(tV, dvv);
-      }
-    };
-    auto add_vsums = [&]() {
 #pragma unroll
-      for (int h = 0; h < HG; ++h)
-        acc[h] += L::VSPLIT ? __uint_as_float(dvv[h]) + __uint_as_float(dvv[HG + h]) : __uint_as_float(dvv[h]);
+      for (int g = 0; g < 4; ++g)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dv[g][hf][nb][e] = 0.f;
     };
     auto part_ptr = [&](int j) -> float* {
       const int u = u_first + j;
@@ -811,218 +789,219 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
         pp[lane * RS + 1] = 0.f;
       }
     };
-    int kv = 0;  // value-MMA commits of this group so far
     // End of local unit j: the group's partial (m, l, acc) of the unit. The reference maxima
-    // are the group's; the sums of p and of p * min are added over the group's 128 lanes in a
-    // fixed order; row R of the value sums is value coordinate coord(R).
+    // are the group's; the sums of p, of p * min and the value sums are added over the
+    // group's four warps in a fixed order (warp 0 first).
     auto finish = [&](int j) {
       float* pp = part_ptr(j);
-      if (vpend) {
-        if (!failed && !wait_phase(&vdone[gi], (uint32_t)(kv - 1) & 1u, abort_flag)) failed = true;
-        s1::fence_after_sync();
-        load_vsums();
-        s1::tmem_ld_wait();
-        add_vsums();
-        vpend = false;
-      }
 #pragma unroll
       for (int h = 0; h < HG; ++h) {
         const float l = warp_sum(lsum[h]);
-        if (lane == 0) red[q * L::RED_F + 4 * HG + h] = l;
+        if (lane == 0) redf[q * L::RED_F + 4 * HG + h] = l;
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
           const float v = warp_sum(mn[h][g]);
-          if (lane == 0) red[q * L::RED_F + 4 * h + g] = v;
+          if (lane == 0) redf[q * L::RED_F + 4 * h + g] = v;
         }
       }
       named_sync(bar_id, 128);
-      const int coord = value_coord<VB>(R);
-      const float unscale = value_unscale<VB>(R);
       for (int h = 0; h < G; ++h) {
-        const float msum = ((red[4 * h + q] + red[L::RED_F + 4 * h + q]) + red[2 * L::RED_F + 4 * h + q]) +
-                           red[3 * L::RED_F + 4 * h + q];
-        pp[h * RS + 4 + coord] = failed ? 0.f : fmaf(acc[h], unscale, msum);
+        const int nb = h >> 2;
+        if (c == (h & 3)) {  // the 8 lanes holding head h: 16 coordinates each
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+              for (int nbb = 0; nbb < NB; ++nbb) {
+                if (nbb != nb) continue;
+                const float* d = dv[g][hf][nbb];
+                int j0;
+                float v0, v1;
+                // element = code * 2^(bit - 24): bit 6 (row r) and bit 8 (row r + 8) at 2 bits,
+                // bit 6 for both at 4 bits
+                if (VB == 2) {
+                  j0 = 4 * (8 * g + r) + 2 * hf;
+                  v0 = (d[0] + d[1]) * 262144.f;
+                  v1 = (d[2] + d[3]) * 65536.f;
+                } else {
+                  j0 = 2 * (16 * g + 8 * hf + r);
+                  v0 = (d[0] + d[1]) * 262144.f;
+                  v1 = (d[2] + d[3]) * 262144.f;
+                }
+                red[q * kD + j0] = v0;
+                red[q * kD + j0 + 1] = v1;
+              }
+        }
+        named_sync(bar_id, 128);
+        {
+          const int gq = R >> 5;  // value group of coordinate R
+          const float msum = ((redf[4 * h + gq] + redf[L::RED_F + 4 * h + gq]) + redf[2 * L::RED_F + 4 * h + gq]) +
+                             redf[3 * L::RED_F + 4 * h + gq];
+          const float acc = ((red[R] + red[kD + R]) + red[2 * kD + R]) + red[3 * kD + R];
+          pp[h * RS + 4 + R] = failed ? 0.f : acc + msum;
+        }
+        named_sync(bar_id, 128);
       }
       if (q == 0 && lane < G) {
         const int h = lane;
-        const float Ls = ((red[4 * HG + h] + red[L::RED_F + 4 * HG + h]) + red[2 * L::RED_F + 4 * HG + h]) +
-                         red[3 * L::RED_F + 4 * HG + h];
+        const float Ls = ((redf[4 * HG + h] + redf[L::RED_F + 4 * HG + h]) + redf[2 * L::RED_F + 4 * HG + h]) +
+                         redf[3 * L::RED_F + 4 * HG + h];
         pp[h * RS + 0] = failed ? -INFINITY : Mref[h];
         pp[h * RS + 1] = failed ? 0.f : Ls;
       }
+      named_sync(bar_id, 128);  // redf is reused by the next unit
+    };
+
+    // Key bits -> unsigned 8-bit elements in tensor memory (row R of the A operand) of the
+    // tile in slot `slot` of stage `st`.
+    auto expand_keys = [&](const unsigned char* st, int slot) {
+      uint32_t w[L::EW];
+      const uint4* kc = reinterpret_cast<const uint4*>(st + L::OFF_KC + (slot * kTileTc + R) * L::KCB);
+#pragma unroll
+      for (int cc = 0; cc < LMB; ++cc) {
+        const uint4 v = kc[cc];
+        w[4 * cc] = v.x;
+        w[4 * cc + 1] = v.y;
+        w[4 * cc + 2] = v.z;
+        w[4 * cc + 3] = v.w;
+      }
+      if constexpr (QJL) {
+        const uint4 v = *reinterpret_cast<const uint4*>(st + L::OFF_KS + (slot * kTileTc + R) * L::SB);
+        w[L::KSC] = v.x;
+        w[L::KSC + 1] = v.y;
+        w[L::KSC + 2] = v.z;
+        w[L::KSC + 3] = v.w;
+      }
+      if constexpr (LMB == 3) {
+#pragma unroll
+        for (int gq = 0; gq < 4; ++gq) w[L::CW + gq] = parity_word(w[3 * gq], w[3 * gq + 1], w[3 * gq + 2]);
+      }
+      static_assert(L::EW % 4 == 0, "element words in groups of four");
+#pragma unroll
+      for (int e4 = 0; e4 < L::EW / 4; ++e4) {
+        uint32_t m[32];  // four element words x eight masks: 32 tensor-memory columns
+#pragma unroll
+        for (int ee = 0; ee < 4; ++ee) {
+          const uint32_t x = w[4 * e4 + ee], x4 = x >> 4;
+          m[8 * ee + 0] = bitmask_el<0>(x, x4);
+          m[8 * ee + 1] = bitmask_el<1>(x, x4);
+          m[8 * ee + 2] = bitmask_el<2>(x, x4);
+          m[8 * ee + 3] = bitmask_el<3>(x, x4);
+          m[8 * ee + 4] = bitmask_el<4>(x, x4);
+          m[8 * ee + 5] = bitmask_el<5>(x, x4);
+          m[8 * ee + 6] = bitmask_el<6>(x, x4);
+          m[8 * ee + 7] = bitmask_el<7>(x, x4);
+        }
+        tmem_st32(tA + 32 * e4, m);
+      }
+      s1::tmem_st_wait();
+    };
+    // Writes the key elements of the group's tile i (if it exists) and signals the MMA warp;
+    // every warp arrives, also without work, so that the phases stay in step.
+    auto stage_keys = [&](int i) {
+      if (i >= ntl) return;
+      const int s = (i >> 1) % NST, slot = i & 1;
+      if (!failed && !wait_phase(&full[s], (uint32_t)((i >> 1) / NST) & 1u, abort_flag)) failed = true;
+      if (!failed) expand_keys(ring + s * L::STAGE, slot);
       s1::fence_before_sync();
-      named_sync(bar_id, 128);  // red is reused by the next unit
+      __syncwarp();
+      if (lane == 0) s1::mbar_arrive(&afull[gi]);
+    };
+
+    // Moves the group from local unit `from` (finished) to local unit `to` (n_units: none):
+    // units in between get empty partials; the leader steps through their operand phases in
+    // order, releasing each before waiting for the next, so that a buffer's phases are never
+    // skipped and no parity wait can match the phase of two loads back; then the group waits
+    // for the operand of unit `to`. Every warp of the group is past unit `from` here, so its
+    // operand buffer may be reloaded.
+    int cur = -1, qrow0 = 0;
+    auto enter_unit = [&](int from, int to) {
+      for (int jj = from + 1; jj < to; ++jj) mark_empty(jj);
+      if (leader) {
+        asm volatile("fence.acq_rel.cta;" ::: "memory");
+        for (int jj = from + 1; jj < to && !failed; ++jj) {
+          grp_unit[gi] = jj;
+          if (!wait_phase(&fbfull[jj % NBUF], (uint32_t)(jj / NBUF) & 1u, abort_flag)) failed = true;
+        }
+        grp_unit[gi] = to;
+        if (failed) raise_abort(abort_flag);
+      }
+      named_sync(bar_id, 128);
+      cur = to;
+      reset();
+      if (to < n_units) {
+        const int u = u_first + to;
+        const int bq = u / a.hkv, kvh = u - bq * a.hkv;
+        qrow0 = bq * a.hq + kvh * G;
+        if (!failed && !wait_phase(&fbfull[to % NBUF], (uint32_t)(to / NBUF) & 1u, abort_flag)) failed = true;
+      }
     };
 
     for (int k = 0; k < gi; ++k) walk.next();
-    reset();
-    int cur = -1, qrow0 = 0, kt = 0;  // local unit, its first query row, tiles of this group so far
+    if (gi < ntl) {
+      stage_keys(gi);
+      enter_unit(-1, walk.u - u_first);
+    }
+    int kt = 0;  // tiles of this group so far
     for (int i = gi; i < ntl; i += NG, ++kt) {
       const int s = (i >> 1) % NST, slot = i & 1;
-      const int u = walk.u, nt = walk.nt();
+      const int nt = walk.nt();
       const int64_t tok0 = walk.tok0();
       for (int k = 0; k < NG; ++k) walk.next();
-      const int j = u - u_first;
-      if (j != cur) {
-        if (cur >= 0) finish(cur);
-        for (int jj = cur + 1; jj < j; ++jj) mark_empty(jj);
-        // Every warp of the group is past its previous unit, so that unit's query operand may be
-        // reloaded. The leader steps through the operand phases of the units this group has no
-        // tile of, in order, releasing each before waiting for the next: a buffer's phases are
-        // then never skipped, and no parity wait can match the phase of two loads back.
-        if (leader) {
-          asm volatile("fence.acq_rel.cta;" ::: "memory");
-          for (int jj = cur + 1; jj < j && !failed; ++jj) {
-            grp_unit[gi] = jj;
-            if (!wait_phase(&fbfull[jj % NBUF], (uint32_t)(jj / NBUF) & 1u, abort_flag)) failed = true;
-          }
-          grp_unit[gi] = j;
-          if (failed) raise_abort(abort_flag);
-        }
-        named_sync(bar_id, 128);
-        cur = j;
-        reset();
-        const int bq = u / a.hkv, kvh = u - bq * a.hkv;
-        qrow0 = bq * a.hq + kvh * G;
-        if (!failed && !wait_phase(&fbfull[j % NBUF], (uint32_t)(j / NBUF) & 1u, abort_flag)) failed = true;
-      }
-      if (!failed && !wait_phase(&full[s], (uint32_t)((i >> 1) / NST) & 1u, abort_flag)) failed = true;
-      // the value operands are free once the group's previous value MMAs are done
-      if (kv > 0 && !failed && !wait_phase(&vdone[gi], (uint32_t)(kv - 1) & 1u, abort_flag)) failed = true;
-      s1::fence_after_sync();
+      const int j = cur;
       const unsigned char* st = ring + s * L::STAGE;
-      const bool valid = R < nt && !failed;
-      // ---- phase 1: this token's records out of the stage
-      uint32_t ngw, vp[4];
-      {
-        ngw = *reinterpret_cast<const uint32_t*>(st + L::OFF_KN + (slot * kTileTc + R) * 4);
-        const uint4 v4 = *reinterpret_cast<const uint4*>(st + L::OFF_VP + (slot * kTileTc + R) * L::PB);
-        vp[0] = v4.x;
-        vp[1] = v4.y;
-        vp[2] = v4.z;
-        vp[3] = v4.w;
-        // key bits -> unsigned 8-bit elements in tensor memory (row R of the A operand)
-        uint32_t w[L::EW];
-        const uint4* kc = reinterpret_cast<const uint4*>(st + L::OFF_KC + (slot * kTileTc + R) * L::KCB);
-#pragma unroll
-        for (int cc = 0; cc < LMB; ++cc) {
-          const uint4 v = kc[cc];
-          w[4 * cc] = v.x;
-          w[4 * cc + 1] = v.y;
-          w[4 * cc + 2] = v.z;
-          w[4 * cc + 3] = v.w;
-        }
-        if constexpr (QJL) {
-          const uint4 v = *reinterpret_cast<const uint4*>(st + L::OFF_KS + (slot * kTileTc + R) * L::SB);
-          w[L::KSC] = v.x;
-          w[L::KSC + 1] = v.y;
-          w[L::KSC + 2] = v.z;
-          w[L::KSC + 3] = v.w;
-        }
-        if constexpr (LMB == 3) {
-#pragma unroll
-          for (int gq = 0; gq < 4; ++gq) w[L::CW + gq] = parity_word(w[3 * gq], w[3 * gq + 1], w[3 * gq + 2]);
-        }
-        static_assert(L::EW % 4 == 0, "element words in groups of four");
-#pragma unroll
-        for (int e4 = 0; e4 < L::EW / 4; ++e4) {
-          uint32_t m[32];  // four element words x eight masks: 32 tensor-memory columns
-#pragma unroll
-          for (int ee = 0; ee < 4; ++ee) {
-            const uint32_t x = w[4 * e4 + ee], x4 = x >> 4;
-            m[8 * ee + 0] = bitmask_el<0>(x, x4);
-            m[8 * ee + 1] = bitmask_el<1>(x, x4);
-            m[8 * ee + 2] = bitmask_el<2>(x, x4);
-            m[8 * ee + 3] = bitmask_el<3>(x, x4);
-            m[8 * ee + 4] = bitmask_el<4>(x, x4);
-            m[8 * ee + 5] = bitmask_el<5>(x, x4);
-            m[8 * ee + 6] = bitmask_el<6>(x, x4);
-            m[8 * ee + 7] = bitmask_el<7>(x, x4);
-          }
-          tmem_st32(tA + 32 * e4, m);
-        }
-        // value codes -> f16 elements (row chunks of the value MMA's A operand)
-        const uint4* vc = reinterpret_cast<const uint4*>(st + L::OFF_VC + (slot * kTileTc + R) * L::VCB);
-#pragma unroll
-        for (int c4 = 0; c4 < VB; ++c4) {
-          const uint4 v = vc[c4];
-          const uint32_t x[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int wi = 0; wi < 4; ++wi) {
-            // Each code lands in bits 6..9 of its f16 (the largest subnormals: the tensor cores
-            // resolve products with small subnormal elements less finely, which showed as a
-            // 1e-4 error in strongly peaked attention with the codes in bits 0..7).
-            const uint32_t y = x[wi], l6 = y << 6, l2 = y << 2, r2 = y >> 2, r6 = y >> 6;
-            if constexpr (VB == 2) {
-              // word 4 c4 + wi: coordinates 16 (4 c4 + wi) + 0..15 -> chunks 2 (4 c4 + wi) + 0, 1;
-              // bytes 0 and 2 from the left shifts, bytes 1 and 3 from the right shifts
-              const int c = 2 * (4 * c4 + wi);
-              st_shared_v4(av + c * 2048 + slot_off, l6 & 0x00C000C0u, l6 & 0x03000300u, l2 & 0x00C000C0u,
-                           l2 & 0x03000300u);
-              st_shared_v4(av + (c + 1) * 2048 + slot_off, r2 & 0x00C000C0u, r2 & 0x03000300u, r6 & 0x00C000C0u,
-                           r6 & 0x03000300u);
-            } else {
-              // word 4 c4 + wi: coordinates 8 (4 c4 + wi) + 0..7 -> chunk 4 c4 + wi
-              const int c = 4 * c4 + wi;
-              st_shared_v4(av + c * 2048 + slot_off, l6 & 0x03C003C0u, l2 & 0x03C003C0u, r2 & 0x03C003C0u,
-                           r6 & 0x03C003C0u);
-            }
-          }
-        }
-        s1::tmem_st_wait();
-      }
-      __syncwarp();
-      if (lane == 0) s1::mbar_arrive(&empty[s]);  // the stage is no longer read by this warp
-      s1::fence_before_sync();
-      named_sync(bar_id, 128);  // all four quarters of the tile's key elements are written
-      if (leader) {
-        s1::fence_after_sync();
-        if (!failed) {
-          constexpr uint32_t idesc = idesc_u8s8_s32(kTileTc, L::N);
-          const uint32_t bbase = smem_addr(sm + L::SM_B + (j % NBUF) * L::BBUF_AL);
-          const uint32_t d_tm = tgrp + L::TA;
-#pragma unroll
-          for (int ks = 0; ks < L::EW; ++ks)
-            umma_i8_ts(d_tm, tgrp + 8 * ks, s1::sw128_desc(bbase, 16 * ks, L::N), idesc, ks > 0 ? 1u : 0u);
-          s1::umma_commit(&mmad[gi]);
-        }
-      }
+      // ---- tile i's digit sums (its MMAs done: the A operand is free again), logits
       if (!failed && !wait_phase(&mmad[gi], (uint32_t)kt & 1u, abort_flag)) failed = true;
       s1::fence_after_sync();
-      uint32_t dsum[L::N];
-#pragma unroll
-      for (int cc = 0; cc < L::N; cc += 16) tmem_ld16(tD + cc, dsum + cc);
-      if (vpend) load_vsums();  // the previous tile's value sums (its MMAs are done)
-      s1::tmem_ld_wait();
-      if (vpend) add_vsums();
-      vpend = false;
-      // ---- logits
-      const float2 ng = __half22float2(h2of(ngw));  // (n, gamma)
-      const float4* kc4 = reinterpret_cast<const float4*>(sm + L::SM_B + (j % NBUF) * L::BBUF_AL + L::BOP);
+      const bool valid = R < nt && !failed;
       float lg[HG];
+      {
+        // digit sums recombined: (s0 + 2^8 s1) + 2^16 (s2 + 2^8 s3), each part an exact int;
+        // the code columns first, then the sign columns (fewer live registers)
+        float code[HG], sg[HG];
+        {
+          uint32_t ds[L::NC];
 #pragma unroll
-      for (int h = 0; h < HG; ++h) {
-        const float4 k = kc4[h];
-        // digit sums recombined: (s0 + 2^8 s1) + 2^16 (s2 + 2^8 s3), each part an exact int
-        const int c0 = kDigits * h;
-        const float code = (float)((int)dsum[c0] + ((int)dsum[c0 + 1] << 8)) +
-                           65536.f * (float)((int)dsum[c0 + 2] + ((int)dsum[c0 + 3] << 8));
-        float sg = 0.f;
-        if constexpr (QJL) {
-          const int c1 = L::NC + kDigits * h;
-          sg = (float)((int)dsum[c1] + ((int)dsum[c1 + 1] << 8)) +
-               65536.f * (float)((int)dsum[c1 + 2] + ((int)dsum[c1 + 3] << 8));
+          for (int cc = 0; cc < L::NC; cc += 16) tmem_ld16(tD + cc, ds + cc);
+          s1::tmem_ld_wait();
+#pragma unroll
+          for (int h = 0; h < HG; ++h)
+            code[h] = (float)((int)ds[4 * h] + ((int)ds[4 * h + 1] << 8)) +
+                      65536.f * (float)((int)ds[4 * h + 2] + ((int)ds[4 * h + 3] << 8));
         }
-        const float l = ng.x * fmaf(ng.y, fmaf(k.z, sg, -k.w), fmaf(k.y, code, k.x));
-        lg[h] = (valid && h < G) ? l : -INFINITY;
+#pragma unroll
+        for (int h = 0; h < HG; ++h) sg[h] = 0.f;
+        if constexpr (QJL) {
+          uint32_t ds[L::NC];
+#pragma unroll
+          for (int cc = 0; cc < L::NC; cc += 16) tmem_ld16(tD + L::NC + cc, ds + cc);
+          s1::tmem_ld_wait();
+#pragma unroll
+          for (int h = 0; h < HG; ++h)
+            sg[h] = (float)((int)ds[4 * h] + ((int)ds[4 * h + 1] << 8)) +
+                    65536.f * (float)((int)ds[4 * h + 2] + ((int)ds[4 * h + 3] << 8));
+        }
+        const uint32_t ngw = *reinterpret_cast<const uint32_t*>(st + L::OFF_KN + (slot * kTileTc + R) * 4);
+        const float2 ng = __half22float2(h2of(ngw));  // (n, gamma)
+        const float4* kc4 = reinterpret_cast<const float4*>(sm + L::SM_B + (j % NBUF) * L::BBUF_AL + L::BOP);
+#pragma unroll
+        for (int h = 0; h < HG; ++h) {
+          const float4 k = kc4[h];
+          const float l = ng.x * fmaf(ng.y, fmaf(k.z, sg[h], -k.w), fmaf(k.y, code[h], k.x));
+          lg[h] = (valid && h < G) ? l : -INFINITY;
+        }
       }
+      s1::fence_before_sync();
+      // ---- the next tile's key elements: its MMAs overlap the rest of this tile
+      stage_keys(i + NG);
       if (a.scores && valid) {
 #pragma unroll
         for (int h = 0; h < HG; ++h)
           if (h < G) a.scores[(size_t)(qrow0 + h) * a.max_len + tok0 + R] = lg[h] * kLn2;
       }
       // ---- online softmax with the group's reference maxima, moved only when a logit exceeds
-      // them by more than the slack; the value sums so far are rescaled then
+      // them by more than the slack; the sums so far are rescaled then
       bool need = false;
 #pragma unroll
       for (int h = 0; h < HG; ++h) need |= lg[h] > Mref[h] + kSlackTc;
@@ -1043,103 +1022,140 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
             Mref[h] = Mn;
           }
           lsum[h] *= corr[h];
-          acc[h] *= corr[h];
 #pragma unroll
           for (int g = 0; g < 4; ++g) mn[h][g] *= corr[h];
         }
-      }
-      // p per head; the minima sums in fp32; the value weights p * scale as f16 hi + lo
-      float p[HG];
 #pragma unroll
-      for (int h = 0; h < HG; ++h) {
-        p[h] = lg[h] == -INFINITY ? 0.f : ex2f(lg[h] - Mref[h]);
-        lsum[h] += p[h];
-      }
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const float mg = valid ? __high2float(h2of(vp[g])) : 0.f;
-#pragma unroll
-        for (int h = 0; h < HG; ++h) mn[h][g] = fmaf(p[h], mg, mn[h][g]);
-      }
-      {
-        uint32_t ph2[HG / 2], pl2[HG / 2];
-#pragma unroll
-        for (int hp = 0; hp < HG / 2; ++hp) {
-          const __half2 hi = __floats2half2_rn(p[2 * hp], p[2 * hp + 1]);
-          const float2 hf = __half22float2(hi);
-          const __half2 lo = __floats2half2_rn(p[2 * hp] - hf.x, p[2 * hp + 1] - hf.y);
-          ph2[hp] = hbits(hi);
-          pl2[hp] = hbits(lo);
-        }
-        // weight (g, h), high and low parts, 2 per word
-        uint32_t whi[L::NV / 2], wlo[L::NV / 2];
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const uint32_t sw = valid ? vp[g] : 0u;
-          const __half2 s2 = h2of(__byte_perm(sw, sw, 0x1010));  // (scale, scale)
-#pragma unroll
-          for (int hp = 0; hp < HG / 2; ++hp) {
-            const __half2 ph = h2of(ph2[hp]), pl = h2of(pl2[hp]);
-            const __half2 hi = __hmul2(ph, s2);
-            const __half2 err = __hfma2(ph, s2, __hneg2(hi));
-            const __half2 lo = __hfma2(pl, s2, err);
-            whi[g * (HG / 2) + hp] = hbits(hi);
-            wlo[g * (HG / 2) + hp] = hbits(lo);
-          }
-        }
-        if constexpr (L::VSPLIT) {
-          // columns (g, part, h), 2 per word; row chunk c = words 4 c .. 4 c + 3
-          uint32_t wv[L::NV];
+        for (int nb = 0; nb < NB; ++nb) {
+          const float cf = corr[4 * nb + c];  // this lane's value sums are of head 4 nb + c
 #pragma unroll
           for (int g = 0; g < 4; ++g)
 #pragma unroll
-            for (int hp = 0; hp < HG / 2; ++hp) {
-              wv[g * HG + hp] = whi[g * (HG / 2) + hp];
-              wv[g * HG + HG / 2 + hp] = wlo[g * (HG / 2) + hp];
+            for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) dv[g][hf][nb][e] *= cf;
+        }
+      }
+      // ---- p per head (f16 high and low parts for the value MMAs); the minima sums in fp32
+      uint4 vp4;
+      {
+        vp4 = *reinterpret_cast<const uint4*>(st + L::OFF_VP + (slot * kTileTc + R) * L::PB);
+        float p[HG];
+#pragma unroll
+        for (int h = 0; h < HG; ++h) {
+          p[h] = lg[h] == -INFINITY ? 0.f : ex2f(lg[h] - Mref[h]);
+          lsum[h] += p[h];
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const float mg = valid ? __high2float(h2of(word_of(vp4, g))) : 0.f;
+#pragma unroll
+          for (int h = 0; h < HG; ++h) mn[h][g] = fmaf(p[h], mg, mn[h][g]);
+        }
+#pragma unroll
+        for (int h = 0; h < HG; ++h) {
+          const __half hi = __float2half_rn(p[h]);
+          const __half lo = __float2half_rn(p[h] - __half2float(hi));
+          pt[h * 32 + lane] = hi;
+          pt[(HG + h) * 32 + lane] = lo;
+        }
+      }
+      __syncwarp();
+      // ---- value sums of the warp's tokens: two K blocks of 16 tokens
+      {
+        const unsigned char* vcb = st + L::OFF_VC + (slot * kTileTc + 32 * q) * L::VCB;
+        const unsigned char* vpb = st + L::OFF_VP + (slot * kTileTc + 32 * q) * L::PB;
+        const int part = r & 1, hsel = r >> 1;
+        const uint32_t sel = (uint32_t)(r & 3) | ((uint32_t)(4 + (r & 3)) << 8);
+        const int nvw = nt - 32 * q;  // valid tokens of this warp (may be <= 0 or >= 32)
+        const bool wfail = __any_sync(kFull, failed);
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb) {
+          if (wfail || nvw <= 16 * kb) break;  // warp-uniform
+          // K order of the block: rows 2c, 2c + 1 (register 0) and 2c + 8, 2c + 9 (register 1)
+          // are tokens 16 kb + 2c, + 1, + 8, + 9 of the warp
+          const int tA0 = 16 * kb + 2 * c, tA1 = tA0 + 1, tB0 = tA0 + 8, tB1 = tA0 + 9;
+          uint32_t phA[NB], plA[NB], phB[NB], plB[NB];
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) {
+            const int h = 4 * nb + hsel;
+            phA[nb] = *reinterpret_cast<const uint32_t*>(pt + h * 32 + tA0);
+            plA[nb] = *reinterpret_cast<const uint32_t*>(pt + (HG + h) * 32 + tA0);
+            phB[nb] = *reinterpret_cast<const uint32_t*>(pt + h * 32 + tB0);
+            plB[nb] = *reinterpret_cast<const uint32_t*>(pt + (HG + h) * 32 + tB0);
+          }
+          uint4 pA0 = *reinterpret_cast<const uint4*>(vpb + tA0 * L::PB);
+          uint4 pA1 = *reinterpret_cast<const uint4*>(vpb + tA1 * L::PB);
+          uint4 pB0 = *reinterpret_cast<const uint4*>(vpb + tB0 * L::PB);
+          uint4 pB1 = *reinterpret_cast<const uint4*>(vpb + tB1 * L::PB);
+          if (nvw < 16 * kb + 16) {  // tokens past the end: scale 0 (their bytes are stale)
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+            if (tA0 >= nvw) pA0 = z;
+            if (tA1 >= nvw) pA1 = z;
+            if (tB0 >= nvw) pB0 = z;
+            if (tB1 >= nvw) pB1 = z;
+          }
+          const uint32_t* vA0 = reinterpret_cast<const uint32_t*>(vcb + tA0 * L::VCB);
+          const uint32_t* vA1 = reinterpret_cast<const uint32_t*>(vcb + tA1 * L::VCB);
+          const uint32_t* vB0 = reinterpret_cast<const uint32_t*>(vcb + tB0 * L::VCB);
+          const uint32_t* vB1 = reinterpret_cast<const uint32_t*>(vcb + tB1 * L::VCB);
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            // B element (token, head, part) = p * scale(token, g) in f16 hi + lo:
+            // hi = p_hi * s (rounded), err = fma(p_hi, s, -hi) (exact), lo = fma(p_lo, s, err)
+            const __half2 sA = h2of(__byte_perm(word_of(pA0, g), word_of(pA1, g), 0x5410));
+            const __half2 sB = h2of(__byte_perm(word_of(pB0, g), word_of(pB1, g), 0x5410));
+            uint32_t bA[NB], bB[NB];
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+              const __half2 hA = __hmul2(h2of(phA[nb]), sA), hB = __hmul2(h2of(phB[nb]), sB);
+              const __half2 eA = __hfma2(h2of(phA[nb]), sA, __hneg2(hA));
+              const __half2 eB = __hfma2(h2of(phB[nb]), sB, __hneg2(hB));
+              bA[nb] = part ? hbits(__hfma2(h2of(plA[nb]), sA, eA)) : hbits(hA);
+              bB[nb] = part ? hbits(__hfma2(h2of(plB[nb]), sB, eB)) : hbits(hB);
             }
+            // Row r of block (g, hf) is one byte of the group's codes; the codes of the two
+            // tokens of a K pair go to the low byte of each f16 half.
 #pragma unroll
-          for (int c = 0; c < L::NV / 4; ++c)
-            st_shared_v4(bv + c * 2048 + slot_off, wv[4 * c], wv[4 * c + 1], wv[4 * c + 2], wv[4 * c + 3]);
-        } else {
-          // columns (g, h) of the high parts, then of the low parts
+            for (int hf = 0; hf < 2; ++hf) {
+              uint32_t xA, xB;
+              uint4 av;
+              // Every code ends in mantissa bits 6..9 of its f16, the largest subnormals: the
+              // tensor cores resolve products with small subnormal elements less finely
+              // (strongly peaked attention showed errors near 1e-4 with codes in bits 0..3).
+              if (VB == 2) {
+                // byte 8g + r: rows r -> coordinate 4(8g + r) + 2hf (bits 4hf.. of the byte,
+                // to bits 6, 7), rows r + 8 -> + 1 (to bits 8, 9)
+                const int wv = 2 * g + (r >> 2);
+                xA = __byte_perm(vA0[wv], vA1[wv], sel) << (6 - 4 * hf);
+                xB = __byte_perm(vB0[wv], vB1[wv], sel) << (6 - 4 * hf);
+                av = make_uint4(xA & 0x00C000C0u, xA & 0x03000300u, xB & 0x00C000C0u, xB & 0x03000300u);
+              } else {
+                // byte 16g + 8hf + r: rows r -> coordinate 2(16g + 8hf + r) (low nibble), rows
+                // r + 8 -> + 1 (high nibble), both to bits 6..9
+                const int wv = 4 * g + 2 * hf + (r >> 2);
+                xA = __byte_perm(vA0[wv], vA1[wv], sel);
+                xB = __byte_perm(vB0[wv], vB1[wv], sel);
+                av = make_uint4((xA << 6) & 0x03C003C0u, (xA << 2) & 0x03C003C0u, (xB << 6) & 0x03C003C0u,
+                                (xB << 2) & 0x03C003C0u);
+              }
 #pragma unroll
-          for (int c = 0; c < L::NV / 8; ++c) {
-            st_shared_v4(bv + c * 2048 + slot_off, whi[4 * c], whi[4 * c + 1], whi[4 * c + 2], whi[4 * c + 3]);
-            st_shared_v4(bv + L::BVP + c * 2048 + slot_off, wlo[4 * c], wlo[4 * c + 1], wlo[4 * c + 2],
-                         wlo[4 * c + 3]);
+              for (int nb = 0; nb < NB; ++nb) mma16816(dv[g][hf][nb], av, bA[nb], bB[nb]);
+            }
           }
         }
       }
-      s1::fence_async_smem();  // the value operands, written by this thread, are read by the MMA
-      s1::fence_before_sync();
-      named_sync(bar_id, 128);
-      if (leader) {
-        s1::fence_after_sync();
-        if (!failed) {
-          const uint32_t abase = smem_addr(av), bbase = smem_addr(bv);
-          const uint32_t d_tm = tgrp + L::TA + L::N;
-          if constexpr (L::VSPLIT) {
-            constexpr uint32_t idesc = idesc_f16_mn(kTileTc, 2 * L::NV);
-#pragma unroll
-            for (int ks = 0; ks < kTileTc / 16; ++ks)
-              s1::umma_f16(d_tm, desc_mn(abase + 256 * ks), desc_mn(bbase + 256 * ks), idesc, ks > 0 ? 1u : 0u);
-          } else {
-            constexpr uint32_t idesc = idesc_f16_mn(kTileTc, L::NV);
-#pragma unroll
-            for (int ks = 0; ks < kTileTc / 16; ++ks) {
-              const uint64_t ad = desc_mn(abase + 256 * ks);
-              s1::umma_f16(d_tm, ad, desc_mn(bbase + 256 * ks), idesc, ks > 0 ? 1u : 0u);
-              s1::umma_f16(d_tm, ad, desc_mn(bbase + L::BVP + 256 * ks), idesc, 1u);
-            }
-          }
-        }
-        s1::umma_commit(&vdone[gi]);
+      __syncwarp();
+      if (lane == 0) s1::mbar_arrive(&empty[s]);  // the stage is no longer read by this warp
+      // ---- unit boundary: the group's next tile (walk) belongs to another unit, or there is none
+      const int jn = i + NG < ntl ? walk.u - u_first : n_units;
+      if (jn != cur) {
+        finish(cur);
+        enter_unit(cur, jn);
       }
-      vpend = true;
-      ++kv;
     }
-    if (cur >= 0) finish(cur);
-    for (int jj = cur + 1; jj < n_units; ++jj) mark_empty(jj);
+    if (gi >= ntl)
+      for (int jj = 0; jj < n_units; ++jj) mark_empty(jj);
     if (leader) grp_unit[gi] = 0x7fffffff;  // done: the producer may reload any buffer
     if (failed && lane == 0) raise_abort(abort_flag);
   }
