@@ -8,23 +8,20 @@
 // the per-token work is spread: with G query heads sharing a KV head, the three
 // contractions (key bits x query, signs x S q, value codes x probabilities) are
 // small dense products over a tile of tokens, so they run on the tensor cores
-// (mma.sync m16n8k16, f16 operands, fp32 accumulation) instead of G scalar loops.
+// (warp-level mma.sync) instead of G scalar loops.
 //
-// Operand layout: the 16 rows of every MMA are tokens (scores) or value
-// coordinates (values); the 8 columns of an n-block are 4 query heads x (hi, lo),
-// the two f16 halves of a query or probability operand (about 22 bits together).
-// G <= 4 needs one n-block, G <= 8 two.
-//
-// Operand construction (no unpacking loops):
+// Scores (mma.sync m16n8k32, u8 x s8 -> s32): rows = 16 tokens, columns = 2 query heads x 4
+// signed 8-bit digits of each key bit's weight (31 bits together, as fine as the fp32 weights;
+// the int32 sums are exact and recombined in fp32), so 4 heads take two n-blocks.
 //  * A 2-bit code with a symmetric codebook is affine in its two bits:
 //    c[b0 + 2 b1] = c0 + (c1 - c0) b0 + (c2 - c0) b1. So <qr, c[idx]> =
 //    c0 sum(qr) + sum over stream bits of (beta_plane * qr_j) * bit. Every packed
 //    bit, keys and signs alike, becomes one MMA operand element.
-//  * Masking one bit per 16-bit half of a word yields an f16 that is 0 or a power
-//    of two (2^-15 .. 2^-11 for bit positions 9..12); the query side is pre-divided
-//    by that power. Lane (r, c) rotates each key word so that its bits 4c..4c+3
-//    (and 16 higher) sit at positions 9..12, then one AND per operand register
-//    yields two exact elements.
+//  * Mask q of a packed word keeps bit q mod 4 of each of its four bytes (of the word shifted
+//    right by 4 for q >= 4): four u8 elements worth 2^(q mod 4) or 0 in one AND; the weights
+//    are divided by that power of two.
+// Values (mma.sync m16n8k16, f16 operands, fp32 accumulation): rows = 16 value coordinates,
+// K = 16 tokens, columns = 4 query heads x (hi, lo), the two f16 halves of p * scale.
 //  * A value code placed in the low mantissa bits of an f16 is a subnormal equal
 //    to code * 2^(pos - 24), so a byte permute plus a mask yields two exact
 //    operands; the power of two is undone once at the end.
@@ -67,17 +64,19 @@ constexpr float kSlack = 2.f;
 constexpr uint32_t kWaitLimit = 1u << 24;                 // polls of one mbarrier phase
 constexpr unsigned long long kWaitNs = 2000000000ull;    // and at most 2 s of wall time
 
-// 32-bit words of key bits per token (code stream, then signs) and the MMA k-steps
-// over them (each word feeds two k-steps of 16 bits).
+// 32-bit words of key bits per token (code stream, then signs). The score MMAs
+// (m16n8k32, u8 x s8) take one k-step of 32 elements per word and lane column: lane column
+// c of k-step s holds masks 2 (s mod 4) and 2 (s mod 4) + 1 of word c + 4 (s / 4).
 __host__ __device__ constexpr int key_words(int lmb) { return 4 * lmb + kM / 32; }
-__host__ __device__ constexpr int key_steps(int lmb) { return 2 * key_words(lmb); }
+__host__ __device__ constexpr int key_steps(int lmb) { return 2 * key_words(lmb); }  // k-steps x 2 n-blocks
 // n-blocks of 8 operand columns (4 heads x hi/lo) for G query heads.
 __host__ __device__ constexpr int n_blocks(int G) { return G <= 4 ? 1 : 2; }
 // 16-token row blocks per warp and tile (fewer when two n-blocks need the registers).
 __host__ __device__ constexpr int m_blocks(int nb) { return nb == 1 ? 2 : 1; }
 __host__ __device__ constexpr int tile_tokens(int nb) { return 16 * kWarpsMma * m_blocks(nb); }
-// Per (sequence, KV head): query operand words [k-step][n-block][32 lanes][2], then
-// [8 heads][4] logit constants (k1..k4 of the decode kernel).
+// Per (sequence, KV head): query operand words [k-step][digit n-block][32 lanes][2] (two
+// digit n-blocks per block of 4 heads), then [8 heads][4] logit constants (k1..k4 of the
+// decode kernel).
 __host__ __device__ constexpr int frag_words(int lmb, int nb) { return key_steps(lmb) * nb * 64 + 32; }
 
 struct PrepArgs {
@@ -171,6 +170,15 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint4& a, uint32_t
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
+}
+
+// D (s32) += A (u8) x B (s8), m16n8k32, A row-major, B column-major.
+__device__ __forceinline__ void mma_i8(int (&d)[4], const uint4& a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
       : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
 }
 
@@ -324,8 +332,8 @@ __global__ void __launch_bounds__(kPrepThreads) prep_mma_kernel(const __grid_con
       // decode kernel's raw tensor-core sums over the normalised operands.
       constexpr float kSignW = kQjl / (float)kM;
       head_s[h * 4 + 0] = a.sl2 * a.c0 * qsum;
-      head_s[h * 4 + 1] = a.sl2 * qs;
-      head_s[h * 4 + 2] = a.sl2 * kSignW * 2.f * ss;
+      head_s[h * 4 + 1] = a.sl2 * qs * (1.f / 1073741824.f);
+      head_s[h * 4 + 2] = a.sl2 * kSignW * 2.f * ss * (1.f / 1073741824.f);
       head_s[h * 4 + 3] = a.sl2 * kSignW * ssum;
       inv_s[h * 2 + 0] = 1.f / qs;
       inv_s[h * 2 + 1] = 1.f / ss;
@@ -334,26 +342,27 @@ __global__ void __launch_bounds__(kPrepThreads) prep_mma_kernel(const __grid_con
   __syncthreads();
   const int nb = a.nb;
   uint32_t* frag = a.frag + (size_t)unit * frag_words(LMB, nb);
-  // Word (k-step, n-block, lane (r, c), register) holds the two f16 B elements of
-  // the m16n8k16 fragment: column r = head 4 n-block + r / 2, part r % 2 (hi / lo);
-  // rows 2c, 2c + 1 (register 0) or 2c + 8, 2c + 9 (register 1). Register e' of
-  // k-step 2 w + h stands for bit 4c + e (e = 2h + e') of key word w and, in its
-  // upper half, bit 4c + e + 16; after the decode lane's rotation that bit is the
-  // lone f16 bit at position 9 + e, worth 2^-15, 2^-14, 2^-13 or 2^-11.
-  const int nwords = key_steps(LMB) * nb * 64;
+  // Word (k-step s, digit n-block nbi, lane (r, c), register reg) holds four signed 8-bit B
+  // elements of the m16n8k32 fragment: column r = head 4 (nbi / 2) + r / 2, digit 2 (nbi mod
+  // 2) + r mod 2; rows 4c + i (register 0) or 4c + 16 + i (register 1). Row 4c + i of
+  // register reg stands for bit 8i + q of key word c + 4 (s / 4), q = 2 (s mod 4) + reg,
+  // which the decode lane's mask q turns into an element worth 2^(q mod 4). The weight of
+  // that bit, normalised to [-1, 1] and divided by 2^(q mod 4), is Q = round(w 2^30) as four
+  // balanced 8-bit digits (Q = d0 + 2^8 d1 + 2^16 d2 + 2^24 d3); column digit d carries d_d.
+  const int nbi_n = 2 * nb;
+  const int nwords = key_words(LMB) * nbi_n * 64;
   for (int w = tid; w < nwords; w += kPrepThreads) {
     const int reg = w & 1, ln = (w >> 1) & 31, blk = w >> 6;
-    const int nbi = blk % nb, kstep = blk / nb;
+    const int nbi = blk % nbi_n, kstep = blk / nbi_n;
     const int rr = ln >> 2, cc = ln & 3;
-    const int head = 4 * nbi + (rr >> 1);
-    const bool lo_part = (rr & 1) != 0;
-    const int wi = kstep >> 1, e = 2 * (kstep & 1) + reg;
-    const float inv = e == 0 ? 32768.f : e == 1 ? 16384.f : e == 2 ? 8192.f : 2048.f;
-    float v2[2] = {0.f, 0.f};
+    const int head = 4 * (nbi >> 1) + (rr >> 1);
+    const int digit = 2 * (nbi & 1) + (rr & 1);
+    const int wi = cc + 4 * (kstep >> 2), q = 2 * (kstep & 3) + reg;
+    uint32_t word = 0u;
     if (head < G) {
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int o = 4 * cc + e + 16 * half;  // bit of the 32-bit key word
+      for (int i = 0; i < 4; ++i) {
+        const int o = 8 * i + q;  // bit of the 32-bit key word
         float x;
         if (wi < 4 * LMB) {
           const int sbit = 32 * wi + o;  // bit of the code stream: code sbit / LMB, plane sbit % LMB
@@ -362,12 +371,18 @@ __global__ void __launch_bounds__(kPrepThreads) prep_mma_kernel(const __grid_con
         } else {
           x = sq_s[head * kM + 32 * (wi - 4 * LMB) + o] * inv_s[head * 2 + 1];
         }
-        x *= inv;
-        const float hi = __half2float(__float2half_rn(x));
-        v2[half] = lo_part ? (x - hi) : hi;
+        const int Q = __float2int_rn(x * (1073741824.f / (float)(1 << (q & 3))));
+        const int d0 = ((Q + 128) & 255) - 128;
+        const int Q1 = (Q - d0) >> 8;
+        const int d1 = ((Q1 + 128) & 255) - 128;
+        const int Q2 = (Q1 - d1) >> 8;
+        const int d2 = ((Q2 + 128) & 255) - 128;
+        const int d3 = (Q2 - d2) >> 8;
+        const int dd = digit == 0 ? d0 : digit == 1 ? d1 : digit == 2 ? d2 : d3;
+        word |= ((uint32_t)dd & 0xffu) << (8 * i);
       }
     }
-    frag[w] = pack_h2(v2[0], v2[1]);
+    frag[w] = word;
   }
   if (tid < 32) reinterpret_cast<float*>(frag)[nwords + tid] = head_s[tid];
 }
@@ -504,8 +519,6 @@ __global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid
   // The combine kernel may launch now; it waits for this grid to finish.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  // Key bits 4c..4c+3 of each half of a word go to f16 positions 9..12.
-  const uint32_t rot = (uint32_t)(9 - 4 * c) & 31u;
   // Value-side B column of this lane: head 4 nb + hsel, part (hi / lo). Its tokens,
   // in K order, are (c, c + 8) and (c + 4, c + 12) of a 16-token block, whose
   // probabilities the lanes srcA and srcB hold after the score step.
@@ -675,53 +688,50 @@ __global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid
       const uint4* vp = reinterpret_cast<const uint4*>(st + L::OFF_VP);
       const uint32_t* vpw = reinterpret_cast<const uint32_t*>(st + L::OFF_VP);
 
-      // ---- scores: D[token rows][head columns] over all key bits ------------------
-      // Rows r and r + 8 of block mb are tokens wbase + 16 mb + r (+ 8).
-      float dl[MB][NB][4], ds[MB][NB][4];
+      // ---- scores: D[token rows][(head, digit) columns] over all key bits ---------
+      // Rows r and r + 8 of block mb are tokens wbase + 16 mb + r (+ 8). Lane column c takes
+      // words c, c + 4, ... of each token: mask q of a word keeps bit q mod 4 of each byte
+      // (of the word shifted right by 4 for q >= 4), four u8 elements in one AND.
+      int dl[MB][2 * NB][4], ds[MB][2 * NB][4];
 #pragma unroll
       for (int mb = 0; mb < MB; ++mb)
 #pragma unroll
-        for (int nb = 0; nb < NB; ++nb)
+        for (int nb = 0; nb < 2 * NB; ++nb)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dl[mb][nb][e] = ds[mb][nb][e] = 0.f;
+          for (int e = 0; e < 4; ++e) dl[mb][nb][e] = ds[mb][nb][e] = 0;
+      const uint32_t* kcw = reinterpret_cast<const uint32_t*>(st + L::OFF_KC);
+      const uint32_t* ksw = reinterpret_cast<const uint32_t*>(st + L::OFF_KS);
 #pragma unroll
-      for (int q = 0; q <= LMB; ++q) {  // 16-byte chunk q: code words 4q..4q+3, or the signs
-        uint4 kw[2 * MB];
+      for (int wg = 0; wg <= LMB; ++wg) {  // word group: code words 4 wg + c, or the signs
+        uint32_t w0[MB], w1[MB];
 #pragma unroll
-        for (int t = 0; t < 2 * MB; ++t) {
-          const int tok = wbase + 8 * t + r;
-          kw[t] = q < LMB ? kc4[tok * LMB + q] : ks4[tok];
+        for (int mb = 0; mb < MB; ++mb) {
+          const int tok = wbase + 16 * mb + r;
+          w0[mb] = wg < LMB ? kcw[tok * (4 * LMB) + 4 * wg + c] : ksw[tok * 4 + c];
+          w1[mb] = wg < LMB ? kcw[(tok + 8) * (4 * LMB) + 4 * wg + c] : ksw[(tok + 8) * 4 + c];
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          uint32_t v[2 * MB];
+        for (int s4 = 0; s4 < 4; ++s4) {
+          const int kstep = 4 * wg + s4;
+          uint2 bf[2 * NB];
 #pragma unroll
-          for (int t = 0; t < 2 * MB; ++t) {
-            const uint32_t w = word_of(kw[t], u);
-            v[t] = __funnelshift_l(w, w, rot);
-          }
+          for (int nb = 0; nb < 2 * NB; ++nb) bf[nb] = bq[(kstep * 2 * NB + nb) * 32 + lane];
 #pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int kstep = 2 * (4 * q + u) + h2;
-            const uint32_t mlo = 0x02000200u << (2 * h2);      // bit 9 + 2 h2 of each half
-            const uint32_t mhi = 0x02000200u << (2 * h2 + 1);  // bit 10 + 2 h2
-            uint2 bf[NB];
+          for (int mb = 0; mb < MB; ++mb) {
+            // masks 2 s4 and 2 s4 + 1: bits 2 s4, 2 s4 + 1 of each byte (of the word >> 4 past 3)
+            const uint32_t x0 = s4 < 2 ? w0[mb] : w0[mb] >> 4, x1 = s4 < 2 ? w1[mb] : w1[mb] >> 4;
+            const uint32_t m0 = 0x01010101u << (2 * (s4 & 1)), m1 = 0x02020202u << (2 * (s4 & 1));
+            uint4 af;
+            af.x = x0 & m0;
+            af.y = x1 & m0;
+            af.z = x0 & m1;
+            af.w = x1 & m1;
 #pragma unroll
-            for (int nb = 0; nb < NB; ++nb) bf[nb] = bq[(kstep * NB + nb) * 32 + lane];
-#pragma unroll
-            for (int mb = 0; mb < MB; ++mb) {
-              uint4 af;
-              af.x = v[2 * mb] & mlo;
-              af.y = v[2 * mb + 1] & mlo;
-              af.z = v[2 * mb] & mhi;
-              af.w = v[2 * mb + 1] & mhi;
-#pragma unroll
-              for (int nb = 0; nb < NB; ++nb) {
-                if (q < LMB)
-                  mma16816(dl[mb][nb], af, bf[nb].x, bf[nb].y);
-                else
-                  mma16816(ds[mb][nb], af, bf[nb].x, bf[nb].y);
-              }
+            for (int nb = 0; nb < 2 * NB; ++nb) {
+              if (wg < LMB)
+                mma_i8(dl[mb][nb], af, bf[nb].x, bf[nb].y);
+              else
+                mma_i8(ds[mb][nb], af, bf[nb].x, bf[nb].y);
             }
           }
         }
@@ -738,8 +748,15 @@ __global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid
         float lg[NB][2];
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) {
-          const float lm0 = dl[mb][nb][0] + dl[mb][nb][1], lm1 = dl[mb][nb][2] + dl[mb][nb][3];
-          const float sg0 = ds[mb][nb][0] + ds[mb][nb][1], sg1 = ds[mb][nb][2] + ds[mb][nb][3];
+          // lane (r, c) holds digits 0, 1 (n-block 2 nb) and 2, 3 (2 nb + 1) of head c + 4 nb
+          const int* L0 = dl[mb][2 * nb];
+          const int* L1 = dl[mb][2 * nb + 1];
+          const int* S0 = ds[mb][2 * nb];
+          const int* S1 = ds[mb][2 * nb + 1];
+          const float lm0 = fmaf(65536.f, (float)(L1[0] + (L1[1] << 8)), (float)(L0[0] + (L0[1] << 8)));
+          const float lm1 = fmaf(65536.f, (float)(L1[2] + (L1[3] << 8)), (float)(L0[2] + (L0[3] << 8)));
+          const float sg0 = fmaf(65536.f, (float)(S1[0] + (S1[1] << 8)), (float)(S0[0] + (S0[1] << 8)));
+          const float sg1 = fmaf(65536.f, (float)(S1[2] + (S1[3] << 8)), (float)(S0[2] + (S0[3] << 8)));
           // logit constants of head c + 4 nb (after the operand words of the buffer)
           const float4 kk = reinterpret_cast<const float4*>(bq + L::KS * NB * 32)[c + 4 * nb];
           lg[nb][0] = ng0.x * fmaf(ng0.y, fmaf(kk.z, sg0, -kk.w), fmaf(kk.y, lm0, kk.x));
