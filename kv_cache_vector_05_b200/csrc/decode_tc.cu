@@ -35,7 +35,8 @@
 // 2^(position - 24): a byte permute pairs the same code byte of two tokens and one AND makes
 // two elements; the power of two depends only on the row and is undone at the end. p * scale
 // is an exact TwoProduct in half2 (high part rounded, low part = the rounding error plus
-// p_low * scale). The group minima, sum_t p_t min_t, are fp32 sums per thread. (Value
+// p_low * scale). The group minima, sum_t p_t min_t, go through one more MMA (rows = value
+// groups, columns = p's high and low parts). (Value
 // operands staged in shared memory for tcgen05 cost 512 bytes of shared-memory traffic per
 // token; in registers they cost none.)
 // Online softmax in base 2 with one reference maximum per query head for a group of warps,
@@ -755,18 +756,22 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
     float* rm = reinterpret_cast<float*>(sm + L::SM_RM) + gi * 32;                     // [4][8]
     __half* pt = reinterpret_cast<__half*>(sm + L::SM_PT + warp * L::PT);             // [2][HG][32]
 
-    // Per thread: the group's reference maxima, this token's share of the sums of p and of
-    // p * min; per lane the value sums (fragment layout).
-    float Mref[HG], lsum[HG], mn[HG][4];
+    // Per thread: the group's reference maxima, this token's share of the sums of p; per lane
+    // the value sums and the sums of p * min (fragment layout: rows g < 4 of the minima MMA are
+    // value group g).
+    float Mref[HG], lsum[HG];
     float dv[4][2][NB][4];  // [value group][half of the group][n-block][fragment]
+    float dmin[NB][4];
     auto reset = [&]() {
 #pragma unroll
       for (int h = 0; h < HG; ++h) {
         Mref[h] = -INFINITY;
         lsum[h] = 0.f;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) mn[h][g] = 0.f;
       }
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dmin[nb][e] = 0.f;
 #pragma unroll
       for (int g = 0; g < 4; ++g)
 #pragma unroll
@@ -798,12 +803,11 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
       for (int h = 0; h < HG; ++h) {
         const float l = warp_sum(lsum[h]);
         if (lane == 0) redf[q * L::RED_F + 4 * HG + h] = l;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const float v = warp_sum(mn[h][g]);
-          if (lane == 0) redf[q * L::RED_F + 4 * h + g] = v;
-        }
       }
+      // lane (g, c), g < 4: sum_t p * min(t, g) of head 4 nb + c in dmin[nb][0] + dmin[nb][1]
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb)
+        if (r < 4) redf[q * L::RED_F + 4 * (4 * nb + c) + r] = dmin[nb][0] + dmin[nb][1];
       named_sync(bar_id, 128);
       for (int h = 0; h < G; ++h) {
         const int nb = h >> 2;
@@ -1022,12 +1026,12 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
             Mref[h] = Mn;
           }
           lsum[h] *= corr[h];
-#pragma unroll
-          for (int g = 0; g < 4; ++g) mn[h][g] *= corr[h];
         }
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) {
           const float cf = corr[4 * nb + c];  // this lane's value sums are of head 4 nb + c
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dmin[nb][e] *= cf;
 #pragma unroll
           for (int g = 0; g < 4; ++g)
 #pragma unroll
@@ -1036,21 +1040,13 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
               for (int e = 0; e < 4; ++e) dv[g][hf][nb][e] *= cf;
         }
       }
-      // ---- p per head (f16 high and low parts for the value MMAs); the minima sums in fp32
-      uint4 vp4;
+      // ---- p per head, as f16 high and low parts for the value MMAs
       {
-        vp4 = *reinterpret_cast<const uint4*>(st + L::OFF_VP + (slot * kTileTc + R) * L::PB);
         float p[HG];
 #pragma unroll
         for (int h = 0; h < HG; ++h) {
           p[h] = lg[h] == -INFINITY ? 0.f : ex2f(lg[h] - Mref[h]);
           lsum[h] += p[h];
-        }
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const float mg = valid ? __high2float(h2of(word_of(vp4, g))) : 0.f;
-#pragma unroll
-          for (int h = 0; h < HG; ++h) mn[h][g] = fmaf(p[h], mg, mn[h][g]);
         }
 #pragma unroll
         for (int h = 0; h < HG; ++h) {
@@ -1094,6 +1090,18 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
             if (tA1 >= nvw) pA1 = z;
             if (tB0 >= nvw) pB0 = z;
             if (tB1 >= nvw) pB1 = z;
+          }
+          {
+            // the group minima through one more MMA: rows g < 4 = min(token, g) of the K pairs,
+            // columns = p (high, low) of the heads
+            uint4 am = make_uint4(0u, 0u, 0u, 0u);
+            if (r < 4) {
+              am.x = __byte_perm(word_of(pA0, r), word_of(pA1, r), 0x7632);
+              am.z = __byte_perm(word_of(pB0, r), word_of(pB1, r), 0x7632);
+            }
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+              mma16816(dmin[nb], am, part ? plA[nb] : phA[nb], part ? plB[nb] : phB[nb]);
           }
           const uint32_t* vA0 = reinterpret_cast<const uint32_t*>(vcb + tA0 * L::VCB);
           const uint32_t* vA1 = reinterpret_cast<const uint32_t*>(vcb + tA1 * L::VCB);
