@@ -183,10 +183,10 @@ size_t tq_decode_workspace_bytes(const tq_ctx* ctx, int batch, int hq, int hkv, 
  *   out       device fp32 [batch][hq][d]
  *   workspace device scratch of at least tq_decode_workspace_bytes(...) bytes
  * At d = 128 with 1- to 3-bit Lloyd-Max codes of a codebook symmetric about zero,
- * 2- or 4-bit values and at most 8 query heads per KV head, the tensor-core decode
- * runs; it carries p * scale (p < 4) as f16 operands, so value-group scales must stay
- * below 16376 (values spanning less than 49000 at 2 bits). Other shapes run the
- * CUDA-core decode.
+ * 2- or 4-bit values and at most 8 query heads per KV head, a tensor-core decode runs
+ * (tq_set_decode_kernel); it carries p * scale (p < 4) as f16 operands, so value-group
+ * scales must stay below 16376 (values spanning less than 49000 at 2 bits). Other
+ * shapes run the CUDA-core decode.
  * Returns TQ_EINVAL if the workspace is too small or any pointer is misaligned. */
 tq_status tq_decode_attention(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int batch, int hq,
                               int hkv, const int32_t* seq_lens, int64_t max_len,
@@ -302,10 +302,10 @@ tq_status tq_set_profile_events(tq_ctx* ctx, void* start, void* stop);
 /* Which decode attention kernel family a context uses. Every family computes the
  * same results within the decode tolerance; they differ in speed and coverage.
  *   TQ_DECODE_AUTO      the fastest family that supports the shape (default)
- *   TQ_DECODE_TCGEN05   key scores and value sums on the 5th-generation tensor cores
- *                       (tcgen05, accumulators in tensor memory): d = 128, m = 128 or 0,
- *                       1- to 3-bit codes of a symmetric codebook, 2- or 4-bit values,
- *                       at most 8 query heads per KV head
+ *   TQ_DECODE_TCGEN05   key scores on the 5th-generation tensor cores (tcgen05, digit
+ *                       sums in tensor memory), value sums on warp-level MMAs: d = 128,
+ *                       m = 128 or 0, 1- to 3-bit codes of a symmetric codebook, 2- or
+ *                       4-bit values, at most 8 query heads per KV head
  *   TQ_DECODE_MMA       warp-level tensor-core MMAs (mma.sync) over the packed bits:
  *                       d = m = 128, 1- or 2-bit codes of a symmetric codebook, 2- or
  *                       4-bit values, at most 8 query heads per KV head
