@@ -75,6 +75,15 @@ def test_validation_without_gpu():
     assert lib.tq_lloyd_max_codebook(128, 2, None, None) == _lib.TQ_EINVAL
 
 
+def test_decode_kernel_selection_validates_without_gpu():
+    """Selecting a decode kernel family needs a context; the query of a NULL context or of
+    head counts that do not divide reports no family."""
+    lib = _lib.lib
+    assert lib.tq_set_decode_kernel(None, _lib.TQ_DECODE_MMA) == _lib.TQ_EINVAL
+    assert lib.tq_decode_kernel_for(None, 32, 8) == -1
+    assert (_lib.TQ_DECODE_AUTO, _lib.TQ_DECODE_TCGEN05, _lib.TQ_DECODE_MMA, _lib.TQ_DECODE_CUDA_CORE) == (0, 1, 2, 3)
+
+
 def test_split_sequence_entry_points_validate_without_gpu():
     """The partial decode and the merge reject bad sizes and pointers before any launch;
     a merge of zero rows is a no-op."""
