@@ -373,9 +373,10 @@ cudaError_t dispatch_lmb(const DecodeArgs& a, int lmb, int vb, dim3 grid, size_t
 DecodePlan plan_decode(const tq_ctx* ctx, int batch, int hq, int hkv, int64_t max_len) {
   DecodePlan p{};
   const int d = ctx->shape.d, m = ctx->shape.m, G = hq / hkv;
-  // TQ_DECODE_AUTO: mma.sync where it applies (1- and 2-bit codes with the QJL stage, the
-  // faster of the two tensor-core kernels on those shapes), then tcgen05, then the generic
-  // kernels. A family selected explicitly runs or the call is refused.
+  // TQ_DECODE_AUTO: mma.sync where it applies (1- to 3-bit codes with the QJL stage, the
+  // faster of the two tensor-core kernels on those shapes), then tcgen05 (keys without the
+  // QJL stage), then the generic kernels. A family selected explicitly runs or the call is
+  // refused.
   const bool tc_ok = tc_decode_supported(ctx, G), mma_ok = mma_decode_supported(ctx, G);
   p.supported = true;
   switch (ctx->decode_kernel) {

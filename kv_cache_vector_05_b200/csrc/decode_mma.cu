@@ -1,5 +1,5 @@
 // Tensor-core decode attention over the packed cache (d = m = 128, up to 8 query
-// heads per KV head, 1- or 2-bit Lloyd-Max keys, 2- or 4-bit values).
+// heads per KV head, 1- to 3-bit Lloyd-Max keys of a symmetric codebook, 2- or 4-bit values).
 //
 // Same mathematics as decode_kernel (the skill card "turboquant-pytorch", "Что
 // делает": scores straight from the compressed keys; the discosf news item:
@@ -13,10 +13,11 @@
 // Scores (mma.sync m16n8k32, u8 x s8 -> s32): rows = 16 tokens, columns = 2 query heads x 4
 // signed 8-bit digits of each key bit's weight (31 bits together, as fine as the fp32 weights;
 // the int32 sums are exact and recombined in fp32), so 4 heads take two n-blocks.
-//  * A 2-bit code with a symmetric codebook is affine in its two bits:
-//    c[b0 + 2 b1] = c0 + (c1 - c0) b0 + (c2 - c0) b1. So <qr, c[idx]> =
-//    c0 sum(qr) + sum over stream bits of (beta_plane * qr_j) * bit. Every packed
-//    bit, keys and signs alike, becomes one MMA operand element.
+//  * A symmetric codebook is affine in the code's bits: c[b0 + 2 b1] = c0 + (c1 - c0) b0 +
+//    (c2 - c0) b1 at 2 bits; at 3 bits the odd part also holds the product of the three signs,
+//    affine in the parity b0 ^ b1 ^ b2 (one parity word per 32 codes, built by each lane from
+//    three stream words). So <qr, c[idx]> = kappa sum(qr) + sum over bits of (beta_plane *
+//    qr_j) * bit: every packed bit, codes, parities and signs alike, is one operand element.
 //  * Mask q of a packed word keeps bit q mod 4 of each of its four bytes (of the word shifted
 //    right by 4 for q >= 4): four u8 elements worth 2^(q mod 4) or 0 in one AND; the weights
 //    are divided by that power of two.
@@ -67,7 +68,9 @@ constexpr unsigned long long kWaitNs = 2000000000ull;    // and at most 2 s of w
 // 32-bit words of key bits per token (code stream, then signs). The score MMAs
 // (m16n8k32, u8 x s8) take one k-step of 32 elements per word and lane column: lane column
 // c of k-step s holds masks 2 (s mod 4) and 2 (s mod 4) + 1 of word c + 4 (s / 4).
-__host__ __device__ constexpr int key_words(int lmb) { return 4 * lmb + kM / 32; }
+__host__ __device__ constexpr int code_words(int lmb) { return 4 * lmb; }
+__host__ __device__ constexpr int par_words(int lmb) { return lmb == 3 ? 4 : 0; }  // parities of 3-bit codes
+__host__ __device__ constexpr int key_words(int lmb) { return code_words(lmb) + par_words(lmb) + kM / 32; }
 __host__ __device__ constexpr int key_steps(int lmb) { return 2 * key_words(lmb); }  // k-steps x 2 n-blocks
 // n-blocks of 8 operand columns (4 heads x hi/lo) for G query heads.
 __host__ __device__ constexpr int n_blocks(int G) { return G <= 4 ? 1 : 2; }
@@ -87,8 +90,8 @@ struct PrepArgs {
   const float* St;   // [d][m]
   const float* PiT;  // [d][d] (Haar)
   Codebook cb;
-  float beta0, beta1;
-  float c0;          // lowest centroid
+  float kappa;       // c[idx] = kappa + sum_p beta[p] bit_p (bit 3: the parity of 3-bit codes)
+  float beta[4];
   float sl2;         // softmax scale * log2(e)
   int nb;            // n-blocks of the query operand
   uint32_t* frag;    // [units][frag_words]
@@ -325,13 +328,13 @@ __global__ void __launch_bounds__(kPrepThreads) prep_mma_kernel(const __grid_con
     qmax = warp_max(qmax);
     smax = warp_max(smax);
     if (lane == 0) {
-      const float bmax = fmaxf(fabsf(a.beta0), LMB > 1 ? fabsf(a.beta1) : 0.f);
+      const float bmax = fmaxf(fmaxf(fabsf(a.beta[0]), fabsf(a.beta[1])), fmaxf(fabsf(a.beta[2]), fabsf(a.beta[3])));
       const float qs = qmax * bmax > 0.f ? qmax * bmax : 1.f;  // LM operand scale
       const float ss = smax > 0.f ? smax : 1.f;                // sign operand scale
       // logit (base 2) = n * (k1 + k2 * lm + gamma * (k3 * sg - k4)), lm and sg being the
       // decode kernel's raw tensor-core sums over the normalised operands.
       constexpr float kSignW = kQjl / (float)kM;
-      head_s[h * 4 + 0] = a.sl2 * a.c0 * qsum;
+      head_s[h * 4 + 0] = a.sl2 * a.kappa * qsum;
       head_s[h * 4 + 1] = a.sl2 * qs * (1.f / 1073741824.f);
       head_s[h * 4 + 2] = a.sl2 * kSignW * 2.f * ss * (1.f / 1073741824.f);
       head_s[h * 4 + 3] = a.sl2 * kSignW * ssum;
@@ -364,12 +367,16 @@ __global__ void __launch_bounds__(kPrepThreads) prep_mma_kernel(const __grid_con
       for (int i = 0; i < 4; ++i) {
         const int o = 8 * i + q;  // bit of the 32-bit key word
         float x;
-        if (wi < 4 * LMB) {
+        if (wi < code_words(LMB)) {
           const int sbit = 32 * wi + o;  // bit of the code stream: code sbit / LMB, plane sbit % LMB
           const int j = sbit / LMB, plane = sbit % LMB;
-          x = qr_s[head * kD + j] * ((plane ? a.beta1 : a.beta0) * inv_s[head * 2 + 0]);
+          x = qr_s[head * kD + j] * (a.beta[plane] * inv_s[head * 2 + 0]);
+        } else if (wi < code_words(LMB) + par_words(LMB)) {
+          // parity word pw, bit o: the parity of code 32 pw + (32 (o mod 3) + o) / 3
+          const int j = 32 * (wi - code_words(LMB)) + (32 * (o % 3) + o) / 3;
+          x = qr_s[head * kD + j] * (a.beta[3] * inv_s[head * 2 + 0]);
         } else {
-          x = sq_s[head * kM + 32 * (wi - 4 * LMB) + o] * inv_s[head * 2 + 1];
+          x = sq_s[head * kM + 32 * (wi - code_words(LMB) - par_words(LMB)) + o] * inv_s[head * 2 + 1];
         }
         const int Q = __float2int_rn(x * (1073741824.f / (float)(1 << (q & 3))));
         const int d0 = ((Q + 128) & 255) - 128;
@@ -701,14 +708,25 @@ __global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid
           for (int e = 0; e < 4; ++e) dl[mb][nb][e] = ds[mb][nb][e] = 0;
       const uint32_t* kcw = reinterpret_cast<const uint32_t*>(st + L::OFF_KC);
       const uint32_t* ksw = reinterpret_cast<const uint32_t*>(st + L::OFF_KS);
+      constexpr int NWG = key_words(LMB) / 4;  // word groups: code words, parity words, signs
 #pragma unroll
-      for (int wg = 0; wg <= LMB; ++wg) {  // word group: code words 4 wg + c, or the signs
+      for (int wg = 0; wg < NWG; ++wg) {  // lane column c takes word 4 wg + c of each token
         uint32_t w0[MB], w1[MB];
 #pragma unroll
         for (int mb = 0; mb < MB; ++mb) {
           const int tok = wbase + 16 * mb + r;
-          w0[mb] = wg < LMB ? kcw[tok * (4 * LMB) + 4 * wg + c] : ksw[tok * 4 + c];
-          w1[mb] = wg < LMB ? kcw[(tok + 8) * (4 * LMB) + 4 * wg + c] : ksw[(tok + 8) * 4 + c];
+          if (wg < LMB) {
+            w0[mb] = kcw[tok * (4 * LMB) + 4 * wg + c];
+            w1[mb] = kcw[(tok + 8) * (4 * LMB) + 4 * wg + c];
+          } else if (wg == NWG - 1) {
+            w0[mb] = ksw[tok * 4 + c];
+            w1[mb] = ksw[(tok + 8) * 4 + c];
+          } else {  // parity word c: from the three code words 3c .. 3c + 2 of the token
+            const uint32_t* p0 = kcw + tok * (4 * LMB) + 3 * c;
+            const uint32_t* p1 = kcw + (tok + 8) * (4 * LMB) + 3 * c;
+            w0[mb] = parity_word(p0[0], p0[1], p0[2]);
+            w1[mb] = parity_word(p1[0], p1[1], p1[2]);
+          }
         }
 #pragma unroll
         for (int s4 = 0; s4 < 4; ++s4) {
@@ -728,7 +746,7 @@ __global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid
             af.w = x1 & m1;
 #pragma unroll
             for (int nb = 0; nb < 2 * NB; ++nb) {
-              if (wg < LMB)
+              if (wg < NWG - 1)
                 mma_i8(dl[mb][nb], af, bf[nb].x, bf[nb].y);
               else
                 mma_i8(ds[mb][nb], af, bf[nb].x, bf[nb].y);
@@ -1043,14 +1061,11 @@ cudaError_t launch_mma_nb(const MmaArgs& a, int nb, dim3 grid, cudaStream_t s) {
 bool mma_decode_supported(const tq_ctx* ctx, int G) {
   const Shape& sh = ctx->shape;
   if (sh.d != kD || sh.m != kM || G < 1 || G > 8) return false;
-  if (sh.lm_bits < 1 || sh.lm_bits > 2) return false;
-  if (sh.lm_bits == 2) {
-    // the codebook must be affine in its two bits (true for a symmetric codebook)
-    const float* cc = ctx->cb.c;
-    const float scale = fmaxf(fabsf(cc[0]), fabsf(cc[3]));
-    if (fabsf((cc[3] - cc[0]) - ((cc[1] - cc[0]) + (cc[2] - cc[0]))) > 1e-6f * scale) return false;
-  }
-  return sh.v_bits == 2 || sh.v_bits == 4;
+  if (sh.lm_bits < 1 || sh.lm_bits > 3) return false;
+  if (!(sh.v_bits == 2 || sh.v_bits == 4)) return false;
+  // the codebook must be affine in its bits (and the parity at 3 bits): true for a symmetric one
+  float kappa, beta[4];
+  return codebook_bits(ctx->cb, sh.lm_bits, kappa, beta);
 }
 
 int mma_ctas_per_sm(int lm_bits, int v_bits, int G) {
@@ -1059,8 +1074,12 @@ int mma_ctas_per_sm(int lm_bits, int v_bits, int G) {
     if (v_bits == 2) return nb == 1 ? ctas_per_sm_t<1, 2, 1>() : ctas_per_sm_t<1, 2, 2>();
     return nb == 1 ? ctas_per_sm_t<1, 4, 1>() : ctas_per_sm_t<1, 4, 2>();
   }
-  if (v_bits == 2) return nb == 1 ? ctas_per_sm_t<2, 2, 1>() : ctas_per_sm_t<2, 2, 2>();
-  return nb == 1 ? ctas_per_sm_t<2, 4, 1>() : ctas_per_sm_t<2, 4, 2>();
+  if (lm_bits == 2) {
+    if (v_bits == 2) return nb == 1 ? ctas_per_sm_t<2, 2, 1>() : ctas_per_sm_t<2, 2, 2>();
+    return nb == 1 ? ctas_per_sm_t<2, 4, 1>() : ctas_per_sm_t<2, 4, 2>();
+  }
+  if (v_bits == 2) return nb == 1 ? ctas_per_sm_t<3, 2, 1>() : ctas_per_sm_t<3, 2, 2>();
+  return nb == 1 ? ctas_per_sm_t<3, 4, 1>() : ctas_per_sm_t<3, 4, 2>();
 }
 
 size_t mma_frag_bytes(int lm_bits, int G) { return (size_t)frag_words(lm_bits, n_blocks(G)) * 4; }
@@ -1077,7 +1096,6 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
   uint32_t* frag = reinterpret_cast<uint32_t*>(ws + plan.off_frag);
   float* part = reinterpret_cast<float*>(ws + plan.off_part);
   const int G = hq / hkv, lmb = ctx->shape.lm_bits, vb = ctx->shape.v_bits, nb = n_blocks(G);
-  const float* cc = ctx->cb.c;
   if (plan.n_ctas < 1 || plan.tiles_per_unit < 1) return cudaErrorInvalidValue;
 
   PrepArgs pa;
@@ -1091,9 +1109,7 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
   pa.St = ctx->St;
   pa.PiT = ctx->PiT;
   pa.cb = ctx->cb;
-  pa.beta0 = cc[1] - cc[0];
-  pa.beta1 = lmb > 1 ? cc[2] - cc[0] : 0.f;
-  pa.c0 = cc[0];
+  if (!codebook_bits(ctx->cb, lmb, pa.kappa, pa.beta)) return cudaErrorInvalidValue;
   pa.sl2 = scale * 1.4426950408889634f;
   pa.nb = nb;
   pa.frag = frag;
@@ -1103,13 +1119,17 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
     cudaError_t ce = cudaFuncSetAttribute(prep_mma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep_smem);
     if (ce == cudaSuccess)
       ce = cudaFuncSetAttribute(prep_mma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep_smem);
+    if (ce == cudaSuccess)
+      ce = cudaFuncSetAttribute(prep_mma_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep_smem);
     if (ce != cudaSuccess) return ce;
     prep_configured = true;
   }
   if (lmb == 1)
     prep_mma_kernel<1><<<batch * hkv, kPrepThreads, prep_smem, stream>>>(pa);
-  else
+  else if (lmb == 2)
     prep_mma_kernel<2><<<batch * hkv, kPrepThreads, prep_smem, stream>>>(pa);
+  else
+    prep_mma_kernel<3><<<batch * hkv, kPrepThreads, prep_smem, stream>>>(pa);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
@@ -1138,8 +1158,10 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
   if (ctx->prof_start) cudaEventRecord(ctx->prof_start, stream);
   if (lmb == 1)
     e = vb == 2 ? launch_mma_nb<1, 2>(a, nb, grid, stream) : launch_mma_nb<1, 4>(a, nb, grid, stream);
-  else
+  else if (lmb == 2)
     e = vb == 2 ? launch_mma_nb<2, 2>(a, nb, grid, stream) : launch_mma_nb<2, 4>(a, nb, grid, stream);
+  else
+    e = vb == 2 ? launch_mma_nb<3, 2>(a, nb, grid, stream) : launch_mma_nb<3, 4>(a, nb, grid, stream);
   if (ctx->prof_stop) cudaEventRecord(ctx->prof_stop, stream);
   if (e != cudaSuccess) return e;
 

@@ -265,14 +265,6 @@ __device__ __forceinline__ uint32_t bitmask_el(uint32_t w, uint32_t w4) {
   return (Q < 4 ? w : w4) & (0x01010101u << (Q & 3));
 }
 
-// Parity word of the 32 three-bit codes held in three consecutive stream words: bit p is the
-// parity of code (32 (p mod 3) + p) / 3.
-__device__ __forceinline__ uint32_t parity_word(uint32_t x0, uint32_t x1, uint32_t x2) {
-  const uint32_t X0 = x0 ^ __funnelshift_r(x0, x1, 1) ^ __funnelshift_r(x0, x1, 2);
-  const uint32_t X1 = x1 ^ __funnelshift_r(x1, x2, 1) ^ __funnelshift_r(x1, x2, 2);
-  const uint32_t X2 = x2 ^ (x2 >> 1) ^ (x2 >> 2);
-  return (X0 & 0x49249249u) | (X1 & 0x92492492u) | (X2 & 0x24924924u);
-}
 
 // Walks a CTA's tiles in order without dividing: the unit, the tile within it, the unit's
 // valid length.
@@ -1237,6 +1229,8 @@ size_t tc_bbuf_t(int nb, int vb) {
   return nb == 1 ? TcLayout<LMB, QJL, 4, 1>::BBUF : TcLayout<LMB, QJL, 4, 2>::BBUF;
 }
 
+}  // namespace
+
 // Bit expansion of a symmetric codebook: c[idx] = kappa + sum_p beta_p bit_p (bit 3 = the
 // parity of the three code bits at 3 bits). False if the codebook is not of that form.
 bool codebook_bits(const Codebook& cb, int lmb, float& kappa, float beta[4]) {
@@ -1272,7 +1266,6 @@ bool codebook_bits(const Codebook& cb, int lmb, float& kappa, float beta[4]) {
   return true;
 }
 
-}  // namespace
 
 bool tc_decode_supported(const tq_ctx* ctx, int G) {
   const Shape& sh = ctx->shape;

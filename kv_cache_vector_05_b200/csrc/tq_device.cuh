@@ -149,4 +149,13 @@ __device__ __forceinline__ uint32_t stream_code(const uint32_t (&w)[NW], int j) 
   return v & ((1u << B) - 1u);
 }
 
+// Parity word of the 32 three-bit codes held in three consecutive stream words: bit p is the
+// parity of code (32 (p mod 3) + p) / 3.
+__device__ __forceinline__ uint32_t parity_word(uint32_t x0, uint32_t x1, uint32_t x2) {
+  const uint32_t X0 = x0 ^ __funnelshift_r(x0, x1, 1) ^ __funnelshift_r(x0, x1, 2);
+  const uint32_t X1 = x1 ^ __funnelshift_r(x1, x2, 1) ^ __funnelshift_r(x1, x2, 2);
+  const uint32_t X2 = x2 ^ (x2 >> 1) ^ (x2 >> 2);
+  return (X0 & 0x49249249u) | (X1 & 0x92492492u) | (X2 & 0x24924924u);
+}
+
 }  // namespace tq

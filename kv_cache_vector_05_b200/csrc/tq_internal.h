@@ -100,6 +100,9 @@ cudaError_t launch_decode(const tq_ctx* ctx, const DecodePlan& plan, const void*
                           cudaStream_t stream);
 
 bool mma_decode_supported(const tq_ctx* ctx, int G);
+// Bit expansion of a symmetric 1- to 3-bit codebook (decode_tc.cu): c[idx] = kappa + sum_p
+// beta_p bit_p, with bit 3 the parity of the three code bits at 3 bits; false otherwise.
+bool codebook_bits(const Codebook& cb, int lmb, float& kappa, float beta[4]);
 bool tc_decode_supported(const tq_ctx* ctx, int G);
 size_t tc_operand_bytes(const tq_ctx* ctx, int G);  // query operand bytes per (sequence, KV head)
 int tc_groups(const tq_ctx* ctx, int G);            // warp groups (partials per CTA and unit)

@@ -325,23 +325,24 @@ def test_decode_each_kernel_family(kernel, lm_bits, v_bits, G):
 
 
 def test_decode_kernel_selection():
-    """TQ_DECODE_AUTO takes the mma.sync kernel for 1- and 2-bit codes with the QJL stage,
-    the tcgen05 kernel for 3-bit codes or keys without QJL, and the generic kernels for
-    every other shape; an explicitly selected family that does not take the shape refuses
-    the call."""
+    """TQ_DECODE_AUTO takes the mma.sync kernel for 1- to 3-bit codes with the QJL stage,
+    the tcgen05 kernel for keys without QJL, and the generic kernels for every other shape;
+    an explicitly selected family that does not take the shape refuses the call."""
     ctx = make_ctx(T, 128, 2, 2)
     assert T.tq_decode_kernel_for(ctx, 32, 8) == T.TQ_DECODE_MMA
     assert T.tq_decode_kernel_for(ctx, 64, 2) == T.TQ_DECODE_CUDA_CORE        # G = 32
     ctx3 = make_ctx(T, 128, 3, 4)
+    assert T.tq_decode_kernel_for(ctx3, 24, 4) == T.TQ_DECODE_MMA
+    T.tq_set_decode_kernel(ctx3, T.TQ_DECODE_TCGEN05)
     assert T.tq_decode_kernel_for(ctx3, 24, 4) == T.TQ_DECODE_TCGEN05
     T.tq_set_decode_kernel(ctx3, T.TQ_DECODE_MMA)
-    assert T.tq_decode_kernel_for(ctx3, 24, 4) == -1
+    assert T.tq_decode_kernel_for(ctx3, 72, 4) == -1                          # G = 18
     packed = _upload(W.random_packed_cache(4 * 256, 128, 3, 128, 4))
-    q = torch.randn((1, 24, 128), device=DEV)
+    q = torch.randn((1, 72, 128), device=DEV)
     with pytest.raises(T.TQError):
-        T.tq_decode_attention(ctx3, q, packed, 1, 24, 4, 256)
+        T.tq_decode_attention(ctx3, q, packed, 1, 72, 4, 256)
     T.tq_set_decode_kernel(ctx3, T.TQ_DECODE_AUTO)
-    out, _ = T.tq_decode_attention(ctx3, q, packed, 1, 24, 4, 256)
+    out, _ = T.tq_decode_attention(ctx3, q, packed, 1, 72, 4, 256)
     torch.cuda.synchronize()
     assert torch.isfinite(out).all()
     dr = W.method_draws(128, 128, 1234)
