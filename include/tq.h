@@ -307,7 +307,7 @@ tq_status tq_set_profile_events(tq_ctx* ctx, void* start, void* stop);
  *                       m = 128 or 0, 1- to 3-bit codes of a symmetric codebook, 2- or
  *                       4-bit values, at most 8 query heads per KV head
  *   TQ_DECODE_MMA       warp-level tensor-core MMAs (mma.sync) over the packed bits:
- *                       d = m = 128, 1- or 2-bit codes of a symmetric codebook, 2- or
+ *                       d = m = 128, 1- to 3-bit codes of a symmetric codebook, 2- or
  *                       4-bit values, at most 8 query heads per KV head
  *   TQ_DECODE_CUDA_CORE the generic kernels: every shape the library accepts */
 typedef enum {
