@@ -1242,11 +1242,14 @@ cudaError_t launch_rot(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s)
 // exact power of two) so that the residual comes out as the x16 operand directly.
 constexpr int kPipeThreads = 640;  // warps 0-7 keys, 8-15 values, 16 producer (17-19 idle)
 
+// NT: bf16 terms of the rotation, 1 for H diag(sigma) (exact), 3 for the Haar matrix (about
+// 24 bits; keys only: its tiles take the space of the value rows).
+template <int NT>
 struct PipeSmem {
   static constexpr uint32_t KT = 0;                         // [2] key operand tiles (TMA, 128B swizzle)
-  static constexpr uint32_t HB = 2 * kTcTileBytes;          // H diag(sigma), bf16 operand tile
-  static constexpr uint32_t S = 3 * kTcTileBytes;           // QJL matrix, f16 hi and lo operand tiles
-  static constexpr uint32_t VR = 5 * kTcTileBytes;          // [2 passes][2 halves] value rows (2 panels each)
+  static constexpr uint32_t HB = 2 * kTcTileBytes;          // the rotation, NT bf16 operand tiles
+  static constexpr uint32_t S = (2 + NT) * kTcTileBytes;    // QJL matrix, f16 hi and lo operand tiles
+  static constexpr uint32_t VR = (4 + NT) * kTcTileBytes;   // [2 passes][2 halves] value rows (NT = 1)
   static constexpr uint32_t XR = 7 * kTcTileBytes;          // [2 passes][128] second-half sums of r^2
   static constexpr uint32_t BAR = XR + 2 * 128 * 4;         // eleven mbarriers
   static constexpr uint32_t TMEM = BAR + 88;                // TMEM base address
@@ -1287,9 +1290,9 @@ __device__ __forceinline__ float bucket_sym(float y, const float* tm, const floa
   return __uint_as_float(__float_as_uint(mag) | (yb & 0x80000000u));
 }
 
-template <int LMB, int VB>
+template <int LMB, int VB, int NT>
 __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __grid_constant__ CompressArgs a) {
-  using PS = PipeSmem;
+  using PS = PipeSmem<NT>;
   namespace s1 = tq::sm100;
   constexpr int L = 1 << LMB, HL = L / 2;
   extern __shared__ unsigned char smem_pipe[];
@@ -1324,7 +1327,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
     for (int w = tid; w < (int)(kTcTileBytes / 16); w += kPipeThreads) {
       sdst[w] = ssrc[w];
       sdst[w + kTcTileBytes / 16] = ssrc[w + kTcTileBytes / 16];
-      hdst[w] = hsrc[w];
+#pragma unroll
+      for (int t = 0; t < NT; ++t) hdst[w + t * (kTcTileBytes / 16)] = hsrc[w + t * (kTcTileBytes / 16)];
     }
   }
   s1::fence_async_smem();
@@ -1390,7 +1394,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
           }
           hs[c2] = (s01.x + s01.y) + (s23.x + s23.y);
         }
-        const float tot = hs[0] + hs[1];  // ||Y||^2 = d ||k||^2
+        const float tot = hs[0] + hs[1];  // ||Y||^2: d ||k||^2 with H diag(sigma), ||k||^2 with Haar
         const bool nz = tot > 0.f;
         const float sc16 = nz ? 16.f * (1.0f / sqrtf(tot)) : 0.f;
         const float2 sc2 = make_float2(sc16, sc16);
@@ -1452,7 +1456,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
         if (failed) break;
         if (ch == 0 && o >= 0) {
           const float gamma = sqrtf(rsum + xr[b * 128 + R]) * (1.f / 16.f);
-          const uint32_t nb = __half_as_ushort(__float2half_rn(sqrtf(tot * (1.0f / 128.f))));
+          // ||Y|| = sqrt(d) ||k|| with H diag(sigma); ||k|| with the orthonormal Haar matrix
+          const uint32_t nb = __half_as_ushort(__float2half_rn(NT == 1 ? sqrtf(tot * (1.0f / 128.f)) : sqrtf(tot)));
           const uint32_t gb = __half_as_ushort(__float2half_rn(gamma));
           reinterpret_cast<uint32_t*>(a.k_norms)[o] = nz ? (nb | (gb << 16)) : 0u;
         }
@@ -1471,7 +1476,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
     }
   } else if (warp < 16) {
     // ================================================================ values
-    if (a.v) {
+    if (NT == 1 && a.v) {
     const int vt = tid - 256, q = vt & 3, vrow = vt >> 2;  // 4 threads per value, 64 per half
     const bool leader = vt == 0;
     uint32_t vpar = 0u, vpend = 0u;  // bit f for value half buffer f: next parity, copy outstanding
@@ -1640,12 +1645,15 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
       kpend &= ~(1u << b);
       return true;
     };
-    auto rotation = [&](int b) {  // Y[b] = KT[b] (H diag sigma)^T
+    auto rotation = [&](int b) {  // Y[b] = KT[b] R^T, R = H diag(sigma) or the Haar matrix's NT terms
       constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
-        s1::umma_f16(tmem + kTmY + 128 * b, s1::sw128_desc(sbase + PS::KT + b * kTcTileBytes, 16 * ks, 128),
-                     s1::sw128_desc(sbase + PS::HB, 16 * ks, 128), idesc, ks > 0 ? 1u : 0u);
+      for (int t = 0; t < NT; ++t)
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          s1::umma_f16(tmem + kTmY + 128 * b, s1::sw128_desc(sbase + PS::KT + b * kTcTileBytes, 16 * ks, 128),
+                       s1::sw128_desc(sbase + PS::HB + t * kTcTileBytes, 16 * ks, 128), idesc,
+                       (t > 0 || ks > 0) ? 1u : 0u);
       s1::umma_commit(rotd + b);
     };
     auto projection = [&]() {  // S r = (A_hi + A_lo) S_hi^T + A_hi S_lo^T, A in tensor memory
@@ -1762,12 +1770,12 @@ bool codebook_symmetric(const Codebook& cb, int lm_bits) {
   return true;
 }
 
-template <int LMB, int VB>
+template <int LMB, int VB, int NT>
 cudaError_t launch_pipe_t(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) {
   static bool configured = false;
-  const size_t smem = PipeSmem::BYTES + 1024;
+  const size_t smem = PipeSmem<NT>::BYTES + 1024;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(compress_pipe_kernel<LMB, VB>,
+    cudaError_t e = cudaFuncSetAttribute(compress_pipe_kernel<LMB, VB, NT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured = true;
@@ -1775,7 +1783,7 @@ cudaError_t launch_pipe_t(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t
   int64_t blocks = (a.n_vec + 127) / 128;
   if (blocks > ctx->num_sms) blocks = ctx->num_sms;
   if (ctx->prof_start) cudaEventRecord(ctx->prof_start, s);
-  compress_pipe_kernel<LMB, VB><<<(unsigned)blocks, kPipeThreads, smem, s>>>(a);
+  compress_pipe_kernel<LMB, VB, NT><<<(unsigned)blocks, kPipeThreads, smem, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (ctx->prof_stop) cudaEventRecord(ctx->prof_stop, s);
   return e;
@@ -1783,9 +1791,17 @@ cudaError_t launch_pipe_t(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t
 
 cudaError_t launch_pipe(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) {
   const int lmb = ctx->shape.lm_bits, vb = ctx->shape.v_bits;
-  if (lmb == 1) return vb == 2 ? launch_pipe_t<1, 2>(ctx, a, s) : launch_pipe_t<1, 4>(ctx, a, s);
-  if (lmb == 2) return vb == 2 ? launch_pipe_t<2, 2>(ctx, a, s) : launch_pipe_t<2, 4>(ctx, a, s);
-  return vb == 2 ? launch_pipe_t<3, 2>(ctx, a, s) : launch_pipe_t<3, 4>(ctx, a, s);
+  if (lmb == 1) return vb == 2 ? launch_pipe_t<1, 2, 1>(ctx, a, s) : launch_pipe_t<1, 4, 1>(ctx, a, s);
+  if (lmb == 2) return vb == 2 ? launch_pipe_t<2, 2, 1>(ctx, a, s) : launch_pipe_t<2, 4, 1>(ctx, a, s);
+  return vb == 2 ? launch_pipe_t<3, 2, 1>(ctx, a, s) : launch_pipe_t<3, 4, 1>(ctx, a, s);
+}
+
+// Keys only with the Haar rotation (its three operand tiles in place of the value rows).
+cudaError_t launch_pipe_haar(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) {
+  const int lmb = ctx->shape.lm_bits;
+  if (lmb == 1) return launch_pipe_t<1, 2, 3>(ctx, a, s);
+  if (lmb == 2) return launch_pipe_t<2, 2, 3>(ctx, a, s);
+  return launch_pipe_t<3, 2, 3>(ctx, a, s);
 }
 
 // ---------------------------------------------------------------------------------
@@ -2369,6 +2385,24 @@ cudaError_t launch_compress(const tq_ctx* ctx, const void* k, const void* v, int
     }
     if (ctx->shape.rot == TQ_ROT_HAAR && dtype == TQ_BF16 && ctx->Pi_sw128) {
       a.H_sw128 = ctx->Pi_sw128;
+      if (!v || encode_rows_map(&a.vmap, v, n_vec, 64)) {
+        // Values (value coding does not depend on the rotation) on the value warps of the
+        // pipelined kernel in a launch of their own, so that they come out the same with or
+        // without keys in the call; keys on the pipelined kernel with the three Haar tiles,
+        // or one pass at a time for a codebook that is not symmetric.
+        if (k) {
+          CompressArgs ka = a;
+          ka.v = nullptr;
+          const cudaError_t e =
+              codebook_symmetric(ctx->cb, ctx->shape.lm_bits) && encode_rows_map(&ka.kmap, k, n_vec, 128)
+                  ? launch_pipe_haar(ctx, ka, stream)
+                  : launch_rot<true>(ctx, ka, stream);
+          if (e != cudaSuccess || !v) return e;
+        }
+        CompressArgs va = a;
+        va.k = nullptr;
+        return launch_pipe(ctx, va, stream);
+      }
       return launch_rot<true>(ctx, a, stream);
     }
     if (ctx->shape.rot == TQ_ROT_HADAMARD)

@@ -90,18 +90,20 @@ def test_compress_parity_full_sweep_size_sampled(rotation):
     assert_value_parity(vs)
 
 
+@pytest.mark.parametrize("rotation", ["hadamard", "haar"])
 @pytest.mark.parametrize("lm_bits", [1, 2, 3])
-def test_compress_parity_several_passes_per_cta(lm_bits):
-    """bf16 keys, Hadamard, d = 128: enough vectors for two to three passes of 128 on every
-    CTA and a ragged last pass, so the double-buffered key tiles, tensor-memory halves and
-    value halves all turn over; every vector is compared. Then keys alone and values alone."""
+def test_compress_parity_several_passes_per_cta(lm_bits, rotation):
+    """bf16 keys, d = 128 (Hadamard: H diag(sigma) as one bf16 operand tile; Haar: three
+    tiles): enough vectors for two to three passes of 128 on every CTA and a ragged last
+    pass, so the double-buffered key tiles, tensor-memory halves and value halves all turn
+    over; every vector is compared. Then keys alone and values alone."""
     d, v_bits = 128, (4 if lm_bits == 2 else 2)
     n = 148 * 128 * 2 + 7 * 128 + 77
     rng = np.random.default_rng([7, lm_bits])
     K = rng.standard_normal((n, d)).astype(np.float32) * rng.lognormal(0, 1, d).astype(np.float32)
     V = rng.standard_normal((n, d)).astype(np.float32) * 3.0 + 1.0
     K[[0, 128 * 148, n - 1]] = 0.0
-    ctx, g, ok, ov = _compress_both(K, V, d, lm_bits, v_bits, "hadamard", "bf16")
+    ctx, g, ok, ov = _compress_both(K, V, d, lm_bits, v_bits, rotation, "bf16")
     assert_key_parity(compare_keys(g, ok, d, lm_bits, d))
     assert_value_parity(compare_values(g, ov, d, v_bits))
     kt = torch.from_numpy(K).to(DEV).to(torch.bfloat16)
@@ -136,24 +138,28 @@ def test_compress_dense_tensor_core_several_passes(d, rotation, lm_bits):
     assert_value_parity(compare_values(g, ov, d, v_bits))
 
 
-def test_compress_parity_asymmetric_codebook():
+@pytest.mark.parametrize("rotation", ["hadamard", "haar"])
+def test_compress_parity_asymmetric_codebook(rotation):
     """A codebook that is not symmetric about zero (one outer centroid and boundary moved)
-    takes the general bucketize; bf16 keys, Hadamard, d = 128, several passes per CTA."""
+    takes the general bucketize (one pass at a time); bf16 keys, d = 128, several passes per
+    CTA."""
     d, lm_bits, v_bits = 128, 2, 2
     dr = W.method_draws(d, d, 1234)
     c32, t32 = T.tq_lloyd_max_codebook(d, lm_bits)
     c32, t32 = c32.copy(), t32.copy()
     c32[0] = np.float32(c32[0] * 1.25)
     t32[0] = np.float32(0.5 * (float(c32[0]) + float(c32[1])))
-    ctx = T.tq_codebook_load(d, lm_bits, v_bits, c32, t32, dr["qjl_S"], rotation="hadamard",
-                             hadamard_signs=dr["hadamard_signs"])
+    haar = T.tq_haar_from_gaussian(dr["haar_gaussian"]) if rotation == "haar" else None
+    ctx = T.tq_codebook_load(d, lm_bits, v_bits, c32, t32, dr["qjl_S"], rotation=rotation,
+                             hadamard_signs=dr["hadamard_signs"], haar=haar)
     n = 148 * 128 * 2 + 333
     rng = np.random.default_rng(99)
     K = rng.standard_normal((n, d)).astype(np.float32)
     kt = torch.from_numpy(K).to(DEV).to(torch.bfloat16)
     g = to_np(T.tq_compress_kv(ctx, kt, None))
     T.tq_check_device(ctx)
-    Pi = O.hadamard_rotation(dr["hadamard_signs"])
+    Pi = (O.hadamard_rotation(dr["hadamard_signs"]) if rotation == "hadamard"
+          else O.haar_rotation(dr["haar_gaussian"]))
     ok = O.compress_keys(kt.float().cpu().numpy().astype(np.float64), Pi, c32.astype(np.float64),
                          t32.astype(np.float64), dr["qjl_S"], with_diagnostics=True)
     assert_key_parity(compare_keys(g, ok, d, lm_bits, d))
