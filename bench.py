@@ -60,6 +60,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-paged", action="store_true", help="skip the paged-cache timings")
+    ap.add_argument("--no-varlen", action="store_true",
+                    help="skip the decode timing of the same cache with sequences of varied lengths")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the kernel timings of the other workloads (the `configs` object)")
     ap.add_argument("--config-steps", type=int, default=10)
@@ -545,6 +547,33 @@ def run_ours(args, w: W.Workload):
                                "compress_slots_vectors_per_s": job_throughput(2 * n_vec, world, pc)})
         del paged, rows, table, bt
 
+    # --- the same cache, each sequence holding a seeded uniform number of tokens in
+    # [tokens / 2, tokens] (seq_lens): decode kernel time and GB/s of the tokens present.
+    varlen_line = None
+    if not args.no_varlen:
+        lens = np.random.default_rng(21 + rank).integers(w.tokens // 2, w.tokens + 1, w.batch)
+        lens_t = torch.from_numpy(lens.astype(np.int32)).to(dev)
+        vdec = []
+        for it in range(args.warmup + args.steps):
+            e = [E(enable_timing=True) for _ in range(2)]
+            for ev in e:
+                ev.record()
+            flush_l2()
+            T.tq_set_profile_events(ctx, e[0], e[1])
+            T.tq_decode_attention(ctx, Q, packed, w.batch, w.hq, w.hkv, w.tokens, seq_lens=lens_t, out=out,
+                                  workspace=ws)
+            T.tq_set_profile_events(ctx, None, None)
+            if it >= args.warmup:
+                vdec.append(e)
+        torch.cuda.synchronize()
+        T.tq_check_device(ctx)
+        vd = slowest(statistics.fmean(e[0].elapsed_time(e[1]) for e in vdec) / 1e3)
+        present = int(lens.sum()) * w.hkv * (w.k_record_bytes() + w.v_record_bytes())
+        varlen_line = {"lengths": "uniform in [tokens / 2, tokens] per sequence (seeded)",
+                       "tokens_present_fraction": float(lens.sum()) / (w.batch * w.tokens),
+                       "decode_main_kernel_ms": vd * 1e3,
+                       "decode_gbs": job_throughput(present, world, vd) / 1e9}
+
     # --- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
@@ -678,6 +707,7 @@ def run_ours(args, w: W.Workload):
             "decode_ms": {"call": dec_total * 1e3 / args.steps, "main_kernel": dec_k_mean * 1e3,
                           "main_kernel_timing": "separate loop of `steps` steps with events around the kernel"},
             "paged": paged_line,
+            "varlen": varlen_line,
             "roofline": roof,
             "roofline_decode": roof_dec,
             "decode_kernel": KERNEL_NAMES[fam],

@@ -1290,6 +1290,16 @@ __device__ __forceinline__ float bucket_sym(float y, const float* tm, const floa
   return __uint_as_float(__float_as_uint(mag) | (yb & 0x80000000u));
 }
 
+// span / L rounded to nearest in fp64 without a division (Markstein's correction step:
+// q0 = span * RN(1/L) is within an ulp of the quotient, the remainder span - L q0 is exact
+// with an FMA, and q0 + remainder * RN(1/L) rounds to the quotient).
+template <int L>
+__device__ __forceinline__ double div_levels(double span) {
+  constexpr double inv = 1.0 / L;
+  const double q0 = span * inv;
+  return fma(fma(-(double)L, q0, span), inv, q0);
+}
+
 template <int LMB, int VB, int NT>
 __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __grid_constant__ CompressArgs a) {
   using PS = PipeSmem<NT>;
@@ -1611,7 +1621,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
           uint32_t* vo = reinterpret_cast<uint32_t*>(a.v_codes + o * (VB * 16) + q * (VB * 4));
 #pragma unroll
           for (int k = 0; k < VB; ++k) vo[k] = vw[k];
-          const uint32_t sb = __half_as_ushort(__double2half(span / levels));
+          const uint32_t sb = __half_as_ushort(__double2half(div_levels<levels>(span)));
           const uint32_t mb = __half_as_ushort(__float2half_rn(lo));
           reinterpret_cast<uint32_t*>(a.v_params)[o * 4 + q] = sb | (mb << 16);
         }

@@ -413,10 +413,12 @@ DecodePlan plan_decode(const tq_ctx* ctx, int batch, int hq, int hkv, int64_t ma
     return p;
   }
   if (p.mma) {
-    // Every unit (sequence x KV head) is cut into tiles; the units' tiles, laid end
-    // to end, are split evenly over one wave of resident CTAs (one per SM). A CTA's
-    // range may cross unit boundaries; each unit is merged from the partials of the
-    // CTAs that share it.
+    // Every unit (sequence x KV head) is cut into tiles; the tiles that hold tokens, of all
+    // units laid end to end, are split evenly over one wave of resident CTAs (one per SM),
+    // by the kernel itself from the lengths on the device. A CTA's range may cross unit
+    // boundaries; each unit is merged from the partials of the CTAs that share it, CTA k's
+    // partial of unit u in slot u + k (at most units + CTAs slots). The grid is sized for
+    // every sequence at max_len.
     const int64_t tile = mma_tile_tokens(G);
     const int64_t Tu = max_len > 0 ? (max_len + tile - 1) / tile : 1;
     const int64_t Tt = units * Tu;
@@ -425,17 +427,11 @@ DecodePlan plan_decode(const tq_ctx* ctx, int batch, int hq, int hkv, int64_t ma
     p.n_ctas = (int)P;
     p.tiles_per_unit = Tu;
     p.total_tiles = Tt;
-    int64_t s_max = 1;
-    for (int64_t u = 0; u < units; ++u) {
-      const int64_t first = ((u * Tu + 1) * P - 1) / Tt, last = ((u + 1) * Tu * P - 1) / Tt;
-      if (last - first + 1 > s_max) s_max = last - first + 1;
-    }
-    p.s_max = (int)s_max;
+    p.s_max = 0;
     p.n_chunks = 0;
     p.chunk_len = 0;
     p.ws_q_bytes = 0;
-    p.ws_part_bytes =
-        align256((size_t)units * s_max * G * (d + kPartPad) * sizeof(float));
+    p.ws_part_bytes = align256((size_t)(units + P) * G * (d + kPartPad) * sizeof(float));
     p.off_frag = 0;
     p.off_part = align256((size_t)units * mma_frag_bytes(ctx->shape.lm_bits, G));
     p.off_cnt = p.off_part + p.ws_part_bytes;  // no counters on this path

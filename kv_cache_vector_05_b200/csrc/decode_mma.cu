@@ -32,9 +32,11 @@
 //    (sign flip + Walsh-Hadamard butterflies, or the dense Haar matrix), forms
 //    S qr, and writes that KV head's query operand fragments once.
 //  * decode_mma_kernel, one 16-warp CTA per SM, launched with programmatic
-//    dependent launch: the tiles of all (sequence, KV head) units, laid end to end,
-//    are split evenly over the CTAs, so a CTA's range may start and end inside a
-//    unit and may span several. It starts streaming its cache tiles (cp.async.bulk
+//    dependent launch: the tiles that hold tokens, of all (sequence, KV head) units
+//    laid end to end, are split evenly over the CTAs (each CTA finds its range from
+//    the sequence lengths on the device), so a CTA's range may start and end inside a
+//    unit and may span several, and a batch of varied lengths costs the tokens it
+//    holds. It starts streaming its cache tiles (cp.async.bulk
 //    into a ring of stages, mbarrier completion) while the prep kernel finishes,
 //    then waits for the fragments of its first units (two operand buffers, refilled
 //    by bulk copy at each unit boundary). Each warp owns 16 or 32 consecutive tokens
@@ -107,13 +109,10 @@ struct MmaArgs {
   const int32_t* seq_lens;
   int64_t max_len;
   Paging pg;               // contiguous or paged cache addressing
-  int hq, hkv, G;
-  int64_t tiles_per_unit;  // tiles of each (sequence, KV head), from max_len
-  int64_t total_tiles;     // units x tiles_per_unit; CTA k takes [k T / P, (k + 1) T / P)
-  int s_max;               // partial slots per unit (most CTAs sharing one unit)
+  int batch, hq, hkv, G;
   float* scores;
   float* out;
-  float* ws_part;          // [units][s_max][G][kPartPadMma + d]
+  float* ws_part;          // [units + CTAs][G][kPartPadMma + d]: CTA k's partial of unit u in slot u + k
   int use_tma;             // 1 when every record array offset is 16-byte aligned
   unsigned int* err;       // device error word of the context
 };
@@ -422,7 +421,8 @@ struct Layout {
   static constexpr int OFF_FRAG = RING;                        // two query-operand buffers
   static constexpr int OFF_BAR = OFF_FRAG + 2 * FRAG_BYTES;    // STAGES + 2 mbarriers
   static constexpr int OFF_CNT = OFF_BAR + 8 * (STAGES + 2);   // arrive / issue counters
-  static constexpr int OFF_RED = OFF_CNT + 4 * (2 * STAGES + 4);  // unit-boundary reduction
+  static constexpr int OFF_PROD = OFF_CNT + 4 * (2 * STAGES + 4);  // the producer thread's unit walk
+  static constexpr int OFF_RED = OFF_PROD + 48;                      // unit-boundary reduction
   static constexpr size_t SMEM = (size_t)OFF_RED + RED_BYTES;
   static_assert(STAGE % 16 == 0 && FRAG_BYTES % 16 == 0, "16-byte aligned stages and fragments");
   static_assert(SMEM <= 227 * 1024, "fits one CTA per SM");
@@ -435,7 +435,9 @@ __device__ __forceinline__ uint32_t word_of(const uint4& w, int i) {
 // CTA owning global tile g when CTA k takes tiles [k T / P, (k + 1) T / P).
 __device__ __forceinline__ int64_t tile_owner(int64_t g, int64_t P, int64_t T) { return ((g + 1) * P - 1) / T; }
 
-template <int LMB, int VB, int NB>
+// VARLEN: lengths given (seq_lens); otherwise every sequence holds max_len tokens, and the
+// split below reduces to plain arithmetic on the tile index.
+template <int LMB, int VB, int NB, bool VARLEN>
 __global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid_constant__ MmaArgs a) {
   using L = Layout<LMB, VB, NB>;
   constexpr int MB = L::MB, TILE = L::TILE, NST = L::STAGES;
@@ -450,78 +452,211 @@ __global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid
   int* issued_s = arrive_s + NST;   // [NST] bulk-copy batches issued into the stage
   int* fissued_s = issued_s + NST;  // [2] copies issued into the operand buffer
   float* red_s = reinterpret_cast<float*>(smem + L::OFF_RED);  // [warps][d] one head's rescaled sums
+  // Thread 0's walk over the units whose query operands it fetches: the last unit issued,
+  // its tile 0 in the global order and its tiles, the CTA's range end, the units issued.
+  struct ProducerWalk {
+    int64_t fpre, fn, g1, pre0;
+    int fu, fj;
+    int cur_u;  // the unit whose partials the warps are accumulating
+  };
+  ProducerWalk* pw = reinterpret_cast<ProducerWalk*>(smem + L::OFF_PROD);
   float* rm_s = red_s + kWarpsMma * kD;                          // [warps][8] warp maxima
   float* rwl_s = rm_s + kWarpsMma * 8;                           // [warps][8] warp sums of p
   float* rM_s = rwl_s + kWarpsMma * 8;                           // [8] CTA maxima
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int r = lane >> 2, c = lane & 3;
-  const int G = a.G;
-  // Balanced split of the flattened (unit, tile) space: this CTA's tiles [g0, g1) may
-  // span several units (a unit = one sequence x KV head).
+  const int G = a.G, hkv = a.hkv;
+  const int units = a.batch * hkv;
   const int64_t P = gridDim.x, kcta = blockIdx.x;
-  const int64_t Tu = a.tiles_per_unit, Tt = a.total_tiles;
-  const int64_t g0 = kcta * Tt / P, g1 = (kcta + 1) * Tt / P;
-  const int ntl = (int)(g1 - g0);
-  const int u_first = ntl > 0 ? (int)(g0 / Tu) : 0;  // == u0 below
-  const int n_units = ntl > 0 ? (int)((g1 - 1) / Tu) - u_first + 1 : 0;
 
   if (tid == 0) {
     for (int s = 0; s < NST + 2; ++s) mbar_init(&bars[s], 1);
     for (int s = 0; s < 2 * NST + 4; ++s) arrive_s[s] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  __syncthreads();
 
-  auto unit_len = [&](int u) -> int64_t {
-    int64_t len = a.max_len;
-    if (a.seq_lens) len = min((int64_t)max(a.seq_lens[u / a.hkv], 0), a.max_len);
-    return len;
+  const int64_t Tu = (a.max_len + TILE - 1) / TILE;  // tiles of a sequence at max_len
+  auto seq_len = [&](int b) -> int64_t {
+    if constexpr (VARLEN) return min((int64_t)max(a.seq_lens[b], 0), a.max_len);
+    return a.max_len;
   };
-  const int u0 = (int)(g0 / Tu);
-  const int64_t tl0 = g0 - (int64_t)u0 * Tu;  // tile index of g0 within its unit
-  // One thread: start tile i. Every tile completes one phase of its stage's barrier:
-  // a full tile (with 16-byte aligned records) through its bulk copies, any other
-  // tile through a plain arrival (its warps then copy it themselves).
-  auto issue = [&](int i) {
-    int u = u0;
-    int64_t tl = tl0 + i;
-    if (tl >= Tu) {
-      u += (int)(tl / Tu);
-      tl -= (tl / Tu) * Tu;
+  auto unit_len = [&](int u) -> int64_t { return seq_len(u / hkv); };
+  auto unit_tiles = [&](int u) -> int {
+    if constexpr (VARLEN) return (int)((unit_len(u) + TILE - 1) / TILE);
+    return (int)Tu;
+  };
+  auto next_unit = [&](int u) -> int {  // the next unit after u that holds a token (or units)
+    if constexpr (!VARLEN) return u + 1;
+    do {
+      ++u;
+    } while (u < units && unit_tiles(u) == 0);
+    return u;
+  };
+  // Split by the tokens present: the tiles that hold at least one token, of every unit (a
+  // unit = one sequence x KV head) laid end to end, are split evenly over the CTAs, so a
+  // batch of short and long sequences costs what its tokens cost. CTA k takes the tiles
+  // [k Tv / P, (k + 1) Tv / P); its range may start and end inside a unit and span several.
+  // Every CTA finds Tv and its first (unit, tile) from the lengths: a block-wide scan of
+  // the per-sequence tile counts (the reduction area is free until the first unit ends).
+  int64_t* scan_s = reinterpret_cast<int64_t*>(red_s);
+  if constexpr (!VARLEN) {
+    if (tid == 0) {
+      const int64_t Tv = (int64_t)units * Tu, g0 = kcta * Tv / P, g1 = (kcta + 1) * Tv / P;
+      scan_s[2 * kWarpsMma] = Tv;
+      scan_s[2 * kWarpsMma + 4] = g1;
+      if (g0 < g1) {
+        scan_s[2 * kWarpsMma + 1] = g0 / Tu;
+        scan_s[2 * kWarpsMma + 2] = g0 % Tu;
+        scan_s[2 * kWarpsMma + 3] = g0 - g0 % Tu;
+        scan_s[2 * kWarpsMma + 5] = a.max_len;
+      }
     }
-    const int64_t tok0 = tl * TILE;
+    __syncthreads();
+  } else {
+    const int per = (a.batch + kThreadsMma - 1) / kThreadsMma;
+    const int b_lo = min(a.batch, tid * per), b_hi = min(a.batch, b_lo + per);
+    int64_t mine = 0, len_lo = 0;  // len_lo: the length of sequence b_lo (kept: no L1 for reloads)
+    for (int b = b_lo; b < b_hi; ++b) {
+      const int64_t len = seq_len(b);
+      if (b == b_lo) len_lo = len;
+      mine += (len + TILE - 1) / TILE;
+    }
+    mine *= hkv;
+    int64_t incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t t = __shfl_up_sync(kFull, incl, o);
+      if (lane >= o) incl += t;
+    }
+    if (lane == 31) scan_s[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const int64_t w = lane < kWarpsMma ? scan_s[lane] : 0;
+      int64_t wi = w;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int64_t t = __shfl_up_sync(kFull, wi, o);
+        if (lane >= o) wi += t;
+      }
+      if (lane < kWarpsMma) scan_s[kWarpsMma + lane] = wi - w;
+      if (lane == 31) scan_s[2 * kWarpsMma] = wi;
+    }
+    __syncthreads();
+    const int64_t Tv = scan_s[2 * kWarpsMma];
+    const int64_t g0 = kcta * Tv / P, g1 = (kcta + 1) * Tv / P;
+    const int64_t before = scan_s[kWarpsMma + warp] + incl - mine;  // tiles before sequence b_lo
+    if (g0 < g1 && before <= g0 && g0 < before + mine) {
+      int64_t pre = before, len = len_lo;
+      int b = b_lo;
+      for (;;) {
+        const int64_t t = hkv * ((len + TILE - 1) / TILE);
+        if (g0 < pre + t) break;
+        pre += t;
+        len = seq_len(++b);
+      }
+      const int64_t nb_t = (len + TILE - 1) / TILE, off = g0 - pre;
+      scan_s[2 * kWarpsMma + 1] = (int64_t)b * hkv + off / nb_t;         // first unit
+      scan_s[2 * kWarpsMma + 2] = off % nb_t;                            // its first tile here
+      scan_s[2 * kWarpsMma + 3] = pre + (off / nb_t) * nb_t;             // its tile 0, globally
+      scan_s[2 * kWarpsMma + 5] = len;                                   // its length
+    }
+    scan_s[2 * kWarpsMma + 4] = g1;
+    __syncthreads();
+  }
+  const int64_t Tv_all = scan_s[2 * kWarpsMma], g1 = scan_s[2 * kWarpsMma + 4];
+  const int64_t g0 = kcta * Tv_all / P;
+  const int ntl = (int)(g1 - g0);
+  const int u0 = ntl > 0 ? (int)scan_s[2 * kWarpsMma + 1] : 0;
+  const int tl0 = ntl > 0 ? (int)scan_s[2 * kWarpsMma + 2] : 0;
+  const int64_t len0 = ntl > 0 ? scan_s[2 * kWarpsMma + 5] : 0;  // tokens of unit u0
+  if (tid == 0) {
+    pw->pre0 = ntl > 0 ? scan_s[2 * kWarpsMma + 3] : 0;
+    pw->g1 = g1;
+    pw->fj = 0;
+  }
+  __syncthreads();  // the reduction area is free again
+  // One thread: start tile i. Every tile completes one phase of its stage's barrier:
+  // a tile with 16-byte aligned records through its bulk copies, any other tile (and one
+  // wholly past its sequence's end) through a plain arrival (its warps then copy it
+  // themselves). The last tile of a sequence copies its valid records rounded up to a
+  // multiple of 4 (16-byte sizes): with max_len a multiple of 4, and pages a multiple of
+  // the tile, those records still lie in the unit's rows or page; the rows past the
+  // sequence's end are masked by the warps.
+  // The tile after (u, tl) in this CTA's order (len: the tokens of unit u).
+  auto advance = [&](int& u, int& tl, int64_t& len) {
+    if constexpr (!VARLEN) {
+      if (++tl == (int)Tu) {
+        ++u;
+        tl = 0;
+      }
+      return;
+    }
+    if (++tl == (int)((len + TILE - 1) / TILE)) {
+      u = next_unit(u);
+      tl = 0;
+      len = u < units ? unit_len(u) : 0;
+    }
+  };
+  // Tile i of this CTA is tile tl of unit u: the first NST are issued by thread 0 at the
+  // start, each later one by the warp that frees its stage, NST tiles after the one it
+  // has just finished (every thread walks the same tiles).
+  auto issue = [&](int i, int u, int tl, int64_t len) {
+    const int64_t tok0 = (int64_t)tl * TILE;
     uint64_t* bar = &bars[i % NST];
-    if (!a.use_tma || unit_len(u) - tok0 < TILE) {
+    const int64_t nv = min((int64_t)TILE, len - tok0);
+    if (!a.use_tma || nv <= 0) {
       mbar_arrive(bar);
       return;
     }
+    const uint32_t n = (uint32_t)((nv + 3) & ~(int64_t)3);  // <= TILE
     unsigned char* st = stage_base + (i % NST) * L::STAGE;
     const int64_t v = record_row(a.pg, a.max_len, u, tok0, a.err);
     issued_s[i % NST] += 1;
-    mbar_expect_tx(bar, (uint32_t)L::STAGE);
-    bulk_g2s(st + L::OFF_KC, a.k_codes + v * L::KCB, TILE * L::KCB, bar);
-    bulk_g2s(st + L::OFF_KS, a.k_signs + v * L::SB, TILE * L::SB, bar);
-    bulk_g2s(st + L::OFF_KN, reinterpret_cast<const uint8_t*>(a.k_norms) + v * 4, TILE * 4, bar);
-    bulk_g2s(st + L::OFF_VC, a.v_codes + v * L::VCB, TILE * L::VCB, bar);
-    bulk_g2s(st + L::OFF_VP, reinterpret_cast<const uint8_t*>(a.v_params) + v * L::PB, TILE * L::PB, bar);
+    mbar_expect_tx(bar, n * (uint32_t)L::REC);
+    bulk_g2s(st + L::OFF_KC, a.k_codes + v * L::KCB, n * L::KCB, bar);
+    bulk_g2s(st + L::OFF_KS, a.k_signs + v * L::SB, n * L::SB, bar);
+    bulk_g2s(st + L::OFF_KN, reinterpret_cast<const uint8_t*>(a.k_norms) + v * 4, n * 4, bar);
+    bulk_g2s(st + L::OFF_VC, a.v_codes + v * L::VCB, n * L::VCB, bar);
+    bulk_g2s(st + L::OFF_VP, reinterpret_cast<const uint8_t*>(a.v_params) + v * L::PB, n * L::PB, bar);
   };
-  auto issue_frag = [&](int j) {  // one thread: query operands of local unit j into buffer j % 2
-    uint64_t* bar = &fbars[j & 1];
-    fissued_s[j & 1] += 1;
+  // One thread: the query operands of this CTA's next unit (local index fj) into buffer
+  // fj % 2, if that unit starts before the CTA's range ends. fu: the last unit issued, fpre
+  // its tile 0 in the global order, fn its tiles.
+  auto issue_frag = [&]() {
+    const int fj = pw->fj;
+    int u = u0;
+    int64_t pre = pw->pre0;
+    if (fj > 0) {
+      u = next_unit(pw->fu);
+      pre = pw->fpre + pw->fn;
+      if (u >= units || pre >= pw->g1) return;
+    }
+    pw->fu = u;
+    pw->fpre = pre;
+    pw->fn = unit_tiles(u);
+    uint64_t* bar = &fbars[fj & 1];
+    fissued_s[fj & 1] += 1;
     mbar_expect_tx(bar, (uint32_t)L::FRAG_BYTES);
-    bulk_g2s(frag_base + (j & 1) * L::FRAG_BYTES, a.frag + (size_t)(u_first + j) * frag_words(LMB, NB),
-             L::FRAG_BYTES, bar);
+    bulk_g2s(frag_base + (fj & 1) * L::FRAG_BYTES, a.frag + (size_t)u * frag_words(LMB, NB), L::FRAG_BYTES,
+             bar);
+    pw->fj = fj + 1;
   };
   // The packed cache does not depend on the prep kernel: start streaming it now.
   if (tid == 0) {
-    for (int i = 0; i < NST && i < ntl; ++i) issue(i);
+    int pu = u0, ptl = tl0;
+    int64_t plen = len0;
+    for (int i = 0; i < NST && i < ntl; ++i) {
+      issue(i, pu, ptl, plen);
+      advance(pu, ptl, plen);
+    }
   }
   // Wait for the prep kernel (programmatic dependent launch), then fetch the query
   // operands of this CTA's first two units.
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  if (tid == 0) {
-    for (int j = 0; j < 2 && j < n_units; ++j) issue_frag(j);
+  if (tid == 0 && ntl > 0) {
+    issue_frag();
+    issue_frag();
   }
   // The combine kernel may launch now; it waits for this grid to finish.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -545,12 +680,10 @@ __global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid
   // at a time, each warp rescales its sums to the CTA maximum and stores them in
   // red_s[warp][coordinate], then one thread per coordinate adds the 16 rows in order.
   // combine_mma_kernel merges the partials of the CTAs that shared the unit. Then buffer
-  // j % 2 is refilled with the operands of unit j + 2.
+  // j % 2 is refilled with the operands of local unit j + 2.
   auto finish_unit = [&](int j) {
-    const int u = u_first + j;
-    const int seg = (int)(kcta - tile_owner((int64_t)u * Tu, P, Tt));
-    float* part = a.ws_part + ((size_t)u * a.s_max + seg) * G * RS;
     __syncthreads();  // every warp has left the previous boundary's reduction
+    float* part = a.ws_part + ((size_t)pw->cur_u + (size_t)kcta) * G * RS;
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
       float l = l_run[nb];
@@ -622,25 +755,34 @@ __global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid
         __syncthreads();
       }
     }
-    if (tid == 0 && j + 2 < n_units) {
+    if (tid == 0 && pw->fj == j + 2) {
       // every warp is past unit j: its operand buffer may be refilled
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      issue_frag(j + 2);
+      issue_frag();
     }
   };
 
-  int u = u0;
-  int64_t tl = tl0 - 1, ulen = 0;
+  // ulen: the tokens of unit u when lengths are given (read once per unit: the lengths are
+  // not in L1, which the shared memory takes); max_len otherwise.
+  int u = u0, tl = tl0;
+  int64_t ulen = len0;
+  auto cur_len = [&]() -> int64_t {
+    if constexpr (VARLEN) return ulen;
+    return a.max_len;
+  };
   for (int i = 0; i < ntl; ++i) {
-    if (++tl == Tu && i > 0) {
+    bool enter = i == 0;
+    if (i > 0 && ++tl == (VARLEN ? (int)((cur_len() + TILE - 1) / TILE) : (int)Tu)) {  // u < units
+      u = next_unit(u);
       tl = 0;
-      ++u;
+      if constexpr (VARLEN) ulen = unit_len(u);
+      enter = true;
     }
-    const int j = u - u_first;
-    if (j != cur) {
-      ulen = unit_len(u);
+    const int j = enter ? cur + 1 : cur;
+    if (enter) {
       if (cur >= 0) finish_unit(cur);
       cur = j;
+      if (tid == 0) pw->cur_u = u;  // read in finish_unit, after its first barrier
       // Wait for the unit's query operands; after a timeout the warp keeps the loop's
       // structure (arrivals, barriers) but does no more work.
       if (!failed && !mbar_wait(&fbars[j & 1], (uint32_t)((j >> 1) & 1))) failed = true;
@@ -661,15 +803,15 @@ __global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid
       qrow0 = b * a.hq + kvh * G;
     }
     const uint2* bq = reinterpret_cast<const uint2*>(frag_base + (j & 1) * L::FRAG_BYTES);
-    const int64_t tok0 = tl * TILE;
-    const int nt = (int)max((int64_t)0, min((int64_t)TILE, ulen - tok0));
+    const int64_t tok0 = (int64_t)tl * TILE;
+    const int nt = (int)max((int64_t)0, min((int64_t)TILE, cur_len() - tok0));
 
     unsigned char* st = stage_base + (i % NST) * L::STAGE;
     // Warps run ahead of one another; each waits only for the tile it needs.
     if (!failed && !mbar_wait(&bars[i % NST], (uint32_t)((i / NST) & 1))) failed = true;
-    if ((nt < TILE || !a.use_tma) && nt > 0) {
-      // Ragged or unaligned tile: plain 4-byte copies (all record sizes are multiples
-      // of 4), after every warp has left the tile that used this stage before.
+    if (!a.use_tma && nt > 0) {
+      // Unaligned records: plain 4-byte copies (all record sizes are multiples of 4),
+      // after every warp has left the tile that used this stage before.
       __syncthreads();
       const int64_t v = record_row(a.pg, a.max_len, u, tok0, a.err);
       auto copy = [&](int off, const void* src, int bytes_per_tok) {
@@ -919,7 +1061,10 @@ __global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid
         arrive_s[i % NST] = 0;
         if (i + NST < ntl) {
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          issue(i + NST);
+          int nu = u, ntl_ = tl;
+          int64_t nlen = cur_len();
+          for (int k = 0; k < NST; ++k) advance(nu, ntl_, nlen);
+          issue(i + NST, nu, ntl_, nlen);
         }
       }
     }
@@ -948,9 +1093,14 @@ struct CombineArgs {
   const float* ws_part;
   float* out;
   float* lse;  // null, or the log of each row's softmax denominator
-  int hq, hkv, G, s_max;
+  int batch, hq, hkv, G, s_max;
   int ppc;     // partials per CTA and unit (consecutive slots)
   int64_t tiles_per_unit, total_tiles, n_ctas;
+  // Split by the tokens present (decode_mma_kernel): tile_tokens > 0, the lengths as there,
+  // and CTA k's partial of unit u in slot u + k.
+  int tile_tokens;
+  const int32_t* seq_lens;
+  int64_t max_len;
 };
 
 // One CTA per (unit, query head), one thread per coordinate: log-sum-exp merge of the
@@ -960,17 +1110,67 @@ __global__ void __launch_bounds__(kD) combine_mma_kernel(const __grid_constant__
   constexpr int RS = kPartPadMma + kD;
   __shared__ float w_s[kD];
   __shared__ float red_s[2][kD / 32];
+  __shared__ long long cnt_s[2][kD / 32];
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int u = blockIdx.x / a.G, h = blockIdx.x - u * a.G;
-  const int64_t Tu = a.tiles_per_unit;
-  const int64_t first = tile_owner((int64_t)u * Tu, a.n_ctas, a.total_tiles);
-  const int n_part = a.ppc * (int)(tile_owner((int64_t)(u + 1) * Tu - 1, a.n_ctas, a.total_tiles) - first + 1);
   const size_t pstride = (size_t)a.G * RS;  // partial p of head h at base + p * pstride
-  const float* base = a.ws_part + (size_t)u * a.s_max * a.ppc * pstride + (size_t)h * RS;
+  int n_part;
+  const float* base;
+  // Partial p comes from CTA first + p; with fewer tiles than CTAs some CTAs between the
+  // unit's first and last own no tile (and wrote nothing): they are skipped.
+  int64_t k_first = 0, Tv = 0, pre = 0, nu = 0;
+  auto live = [&](int p) -> bool {
+    if (a.tile_tokens == 0) return true;
+    const int64_t k = k_first + p;
+    return max(k * Tv / a.n_ctas, pre) < min((k + 1) * Tv / a.n_ctas, pre + nu);
+  };
+  if (a.tile_tokens > 0) {
+    // The decode kernel's split: the tiles holding tokens, all units end to end, Tv in all.
+    const int64_t T = a.tile_tokens;
+    auto tiles = [&](int b) -> int64_t {
+      const int64_t len = a.seq_lens ? min((int64_t)max(a.seq_lens[b], 0), a.max_len) : a.max_len;
+      return (len + T - 1) / T;
+    };
+    const int b = u / a.hkv, kvh = u - b * a.hkv;
+    long long all = 0, before = 0;
+    for (int s = tid; s < a.batch; s += kD) {
+      const long long t = tiles(s);
+      all += t;
+      if (s < b) before += t;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      all += __shfl_xor_sync(kFull, all, o);
+      before += __shfl_xor_sync(kFull, before, o);
+    }
+    if (lane == 0) {
+      cnt_s[0][warp] = all;
+      cnt_s[1][warp] = before;
+    }
+    __syncthreads();
+    Tv = a.hkv * ((cnt_s[0][0] + cnt_s[0][1]) + (cnt_s[0][2] + cnt_s[0][3]));
+    nu = tiles(b);
+    pre = a.hkv * ((cnt_s[1][0] + cnt_s[1][1]) + (cnt_s[1][2] + cnt_s[1][3])) + kvh * nu;
+    if (nu == 0) {  // no token: no partial
+      const int row = b * a.hq + kvh * a.G + h;
+      a.out[(size_t)row * kD + tid] = 0.f;
+      if (a.lse && tid == 0) a.lse[row] = -INFINITY;
+      return;
+    }
+    k_first = tile_owner(pre, a.n_ctas, Tv);
+    n_part = (int)(tile_owner(pre + nu - 1, a.n_ctas, Tv) - k_first + 1);
+    base = a.ws_part + ((size_t)u + (size_t)k_first) * pstride + (size_t)h * RS;
+  } else {
+    const int64_t Tu = a.tiles_per_unit;
+    const int64_t first = tile_owner((int64_t)u * Tu, a.n_ctas, a.total_tiles);
+    n_part = a.ppc * (int)(tile_owner((int64_t)(u + 1) * Tu - 1, a.n_ctas, a.total_tiles) - first + 1);
+    base = a.ws_part + (size_t)u * a.s_max * a.ppc * pstride + (size_t)h * RS;
+  }
 
   float M = -INFINITY;
-  for (int p = tid; p < n_part; p += kD) M = fmaxf(M, base[p * pstride]);
+  for (int p = tid; p < n_part; p += kD)
+    if (live(p)) M = fmaxf(M, base[p * pstride]);
   M = warp_max(M);
   if (lane == 0) red_s[0][warp] = M;
   __syncthreads();
@@ -979,7 +1179,7 @@ __global__ void __launch_bounds__(kD) combine_mma_kernel(const __grid_constant__
   for (int p0 = 0; p0 < n_part; p0 += kD) {
     const int p = p0 + tid;
     float w = 0.f;
-    if (p < n_part) {
+    if (p < n_part && live(p)) {
       const float mp = base[p * pstride];
       w = mp == -INFINITY ? 0.f : exp2f(mp - M);
       if (w != 0.f) den = fmaf(w, base[p * pstride + 1], den);
@@ -1008,10 +1208,10 @@ __global__ void __launch_bounds__(kD) combine_mma_kernel(const __grid_constant__
   if (a.lse && tid == 0) a.lse[row] = den > 0.f ? (M + log2f(den)) * 0.6931471805599453f : -INFINITY;
 }
 
-template <int LMB, int VB, int NB>
+template <int LMB, int VB, int NB, bool VARLEN>
 cudaError_t configure_mma_t() {
   using L = Layout<LMB, VB, NB>;
-  static cudaError_t status = cudaFuncSetAttribute(decode_mma_kernel<LMB, VB, NB>,
+  static cudaError_t status = cudaFuncSetAttribute(decode_mma_kernel<LMB, VB, NB, VARLEN>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::SMEM);
   return status;
 }
@@ -1021,8 +1221,8 @@ int ctas_per_sm_t() {
   using L = Layout<LMB, VB, NB>;
   static int n = [] {
     int blocks = 0;
-    if (configure_mma_t<LMB, VB, NB>() != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, decode_mma_kernel<LMB, VB, NB>, kThreadsMma,
+    if (configure_mma_t<LMB, VB, NB, false>() != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, decode_mma_kernel<LMB, VB, NB, false>, kThreadsMma,
                                                       L::SMEM) != cudaSuccess ||
         blocks < 1) {
       cudaGetLastError();
@@ -1033,10 +1233,10 @@ int ctas_per_sm_t() {
   return n;
 }
 
-template <int LMB, int VB, int NB>
+template <int LMB, int VB, int NB, bool VARLEN>
 cudaError_t launch_mma_t(const MmaArgs& a, dim3 grid, cudaStream_t s) {
   using L = Layout<LMB, VB, NB>;
-  cudaError_t e = configure_mma_t<LMB, VB, NB>();
+  cudaError_t e = configure_mma_t<LMB, VB, NB, VARLEN>();
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
@@ -1048,12 +1248,14 @@ cudaError_t launch_mma_t(const MmaArgs& a, dim3 grid, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_mma_kernel<LMB, VB, NB>, a);
+  return cudaLaunchKernelEx(&cfg, decode_mma_kernel<LMB, VB, NB, VARLEN>, a);
 }
 
 template <int LMB, int VB>
 cudaError_t launch_mma_nb(const MmaArgs& a, int nb, dim3 grid, cudaStream_t s) {
-  return nb == 1 ? launch_mma_t<LMB, VB, 1>(a, grid, s) : launch_mma_t<LMB, VB, 2>(a, grid, s);
+  if (a.seq_lens)
+    return nb == 1 ? launch_mma_t<LMB, VB, 1, true>(a, grid, s) : launch_mma_t<LMB, VB, 2, true>(a, grid, s);
+  return nb == 1 ? launch_mma_t<LMB, VB, 1, false>(a, grid, s) : launch_mma_t<LMB, VB, 2, false>(a, grid, s);
 }
 
 }  // namespace
@@ -1143,12 +1345,10 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
   a.seq_lens = seq_lens;
   a.max_len = max_len;
   a.pg = pg;
+  a.batch = batch;
   a.hq = hq;
   a.hkv = hkv;
   a.G = G;
-  a.tiles_per_unit = plan.tiles_per_unit;
-  a.total_tiles = plan.total_tiles;
-  a.s_max = plan.s_max;
   a.scores = scores;
   a.out = out;
   a.ws_part = part;
@@ -1166,13 +1366,18 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
   if (e != cudaSuccess) return e;
 
   return launch_combine_partials(part, out, lse, batch, hq, hkv, G, plan.s_max, 1, plan.tiles_per_unit,
-                                 plan.total_tiles, plan.n_ctas, stream);
+                                 plan.total_tiles, plan.n_ctas, stream, mma_tile_tokens(G), seq_lens, max_len);
 }
 
 cudaError_t launch_combine_partials(const float* part, float* out, float* lse, int batch, int hq, int hkv, int G,
                                     int s_max, int ppc, int64_t tiles_per_unit, int64_t total_tiles, int n_ctas,
-                                    cudaStream_t stream) {
+                                    cudaStream_t stream, int tile_tokens, const int32_t* seq_lens,
+                                    int64_t max_len) {
   CombineArgs ca;
+  ca.batch = batch;
+  ca.tile_tokens = tile_tokens;
+  ca.seq_lens = seq_lens;
+  ca.max_len = max_len;
   ca.ppc = ppc;
   ca.ws_part = part;
   ca.out = out;

@@ -330,6 +330,16 @@ def test_decode_each_kernel_family(kernel, lm_bits, v_bits, G):
     _decode_check(128, lm_bits, v_bits, batch=2, hkv=2, G=G, max_len=1500, lens=[1500, 701], kernel=kernel)
 
 
+@pytest.mark.parametrize("lm_bits,v_bits,G", [(2, 2, 4), (2, 4, 8), (3, 4, 6)])
+def test_decode_variable_lengths_split_by_tokens(lm_bits, v_bits, G):
+    """A batch of empty, one-token, partial and full sequences on the mma.sync decode, which
+    splits the tiles that hold tokens (not every sequence's max_len) over its CTAs: fewer
+    tiles than CTAs, CTAs whose range crosses several units, lengths that are not a multiple
+    of 4 (the last tile's bulk copy rounds up), every row against the oracle."""
+    _decode_check(128, lm_bits, v_bits, batch=7, hkv=2, G=G, max_len=2048,
+                  lens=[0, 2048, 1, 0, 1501, 513, 7], kernel="mma")
+
+
 def test_decode_kernel_selection():
     """TQ_DECODE_AUTO takes the mma.sync kernel for 1- to 3-bit codes with the QJL stage,
     the tcgen05 kernel for keys without QJL, and the generic kernels for every other shape;
