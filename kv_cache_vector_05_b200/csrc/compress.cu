@@ -1846,18 +1846,26 @@ struct DenseSmem {
   static constexpr uint32_t BYTES = TMEM + 8;
   static_assert(BYTES + 1024 <= 227 * 1024, "compress_dense_kernel shared memory");
 };
-// Tensor memory: Y (then S r) at columns [0, D), the residual operand's hi at 256 and lo at
-// 256 + D/2 (one f16 pair per column).
-constexpr uint32_t kDnA = 256;
+// Tensor memory: Y (then S r) at columns [0, D), the residual operand's hi at A and lo at
+// A + D/2 (one f16 pair per column). At d = 64 a CTA takes 256 columns (A = 128), so two CTAs
+// share an SM and one's MMAs and bulk copies run under the other's key work; at d = 256 one
+// CTA takes all 512 (A = 256).
+template <int D>
+struct DenseTmem {
+  static constexpr uint32_t A = D == 64 ? 128 : 256;
+  static constexpr uint32_t COLS = D == 64 ? 256 : 512;
+  static constexpr int CTAS_PER_SM = D == 64 ? 2 : 1;
+};
 
 __device__ __forceinline__ void dense_key_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(256) : "memory");
 }
 
 template <int D, int LMB, int NT>
-__global__ void __launch_bounds__(kDenseThreads, 1) compress_dense_kernel(const __grid_constant__ CompressArgs a,
-                                                                         const uint16_t* __restrict__ ops) {
+__global__ void __launch_bounds__(kDenseThreads, DenseTmem<D>::CTAS_PER_SM)
+    compress_dense_kernel(const __grid_constant__ CompressArgs a, const uint16_t* __restrict__ ops) {
   using DS = DenseSmem<D, NT>;
+  constexpr uint32_t kDnA = DenseTmem<D>::A;
   namespace s1 = tq::sm100;
   constexpr int NW = DS::NW, NCH = DS::NCH;
   constexpr int HALF = D / 2;  // columns per thread
@@ -1879,7 +1887,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) compress_dense_kernel(const 
   const int64_t ntile = (a.n_vec + 127) / 128, g = gridDim.x;
 
   if (warp == 0) {
-    s1::tmem_alloc(tmem_s, 512);
+    s1::tmem_alloc(tmem_s, DenseTmem<D>::COLS);
     s1::tmem_relinquish();
   }
   if (tid == 0) {
@@ -2170,17 +2178,19 @@ __global__ void __launch_bounds__(kDenseThreads, 1) compress_dense_kernel(const 
   __syncthreads();
   if (warp == 0) {
     s1::fence_after_sync();
-    s1::tmem_dealloc(tmem, 512);
+    s1::tmem_dealloc(tmem, DenseTmem<D>::COLS);
   }
 }
-
 
 template <int D, int LMB, int NT>
 cudaError_t launch_dense_t(const tq_ctx* ctx, const CompressArgs& a, const uint16_t* ops, cudaStream_t s) {
   using DS = DenseSmem<D, NT>;
   static bool configured = false;
-  // at least 120 KB, so that no two CTAs share an SM (each holds all 512 tensor-memory columns)
-  const size_t smem = DS::BYTES + 1024 > 120 * 1024 ? DS::BYTES + 1024 : 120 * 1024;
+  // Shared memory padded so that an SM holds no more CTAs than tensor memory takes: at least
+  // 120 KB at d = 256 (one CTA, all 512 columns), 80 KB at d = 64 (two CTAs of 256 columns).
+  constexpr size_t kFloor = DenseTmem<D>::CTAS_PER_SM == 2 ? 80 * 1024 : 120 * 1024;
+  static_assert(DenseTmem<D>::CTAS_PER_SM == 1 || DS::BYTES + 1024 <= kFloor, "two CTAs per SM at d = 64");
+  const size_t smem = DS::BYTES + 1024 > kFloor ? DS::BYTES + 1024 : kFloor;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(compress_dense_kernel<D, LMB, NT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -2188,7 +2198,7 @@ cudaError_t launch_dense_t(const tq_ctx* ctx, const CompressArgs& a, const uint1
     configured = true;
   }
   int64_t blocks = (a.n_vec + 127) / 128;
-  if (blocks > ctx->num_sms) blocks = ctx->num_sms;
+  if (blocks > (int64_t)DenseTmem<D>::CTAS_PER_SM * ctx->num_sms) blocks = (int64_t)DenseTmem<D>::CTAS_PER_SM * ctx->num_sms;
   if (ctx->prof_start) cudaEventRecord(ctx->prof_start, s);
   compress_dense_kernel<D, LMB, NT><<<(unsigned)blocks, kDenseThreads, smem, s>>>(a, ops);
   cudaError_t e = cudaGetLastError();
