@@ -434,8 +434,10 @@ DecodePlan plan_decode(const tq_ctx* ctx, int batch, int hq, int hkv, int64_t ma
     p.ws_part_bytes = align256((size_t)(units + P) * G * (d + kPartPad) * sizeof(float));
     p.off_frag = 0;
     p.off_part = align256((size_t)units * mma_frag_bytes(ctx->shape.lm_bits, G));
-    p.off_cnt = p.off_part + p.ws_part_bytes;  // no counters on this path
-    p.total_bytes = p.off_cnt;
+    // then, for calls with lengths, each sequence's first tile in the split order and the
+    // total ([batch + 1] int64, written by the decode grid for the combine kernel)
+    p.off_cnt = p.off_part + p.ws_part_bytes;
+    p.total_bytes = p.off_cnt + align256((size_t)(batch + 1) * sizeof(int64_t));
     return p;
   }
   const int64_t tiles = max_len > 0 ? (max_len + kTile - 1) / kTile : 1;

@@ -113,6 +113,7 @@ struct MmaArgs {
   float* scores;
   float* out;
   float* ws_part;          // [units + CTAs][G][kPartPadMma + d]: CTA k's partial of unit u in slot u + k
+  int64_t* seq_first;      // with lengths: [batch + 1] first tile of each sequence, then Tv (CTA 0 writes)
   int use_tma;             // 1 when every record array offset is 16-byte aligned
   unsigned int* err;       // device error word of the context
 };
@@ -546,6 +547,14 @@ __global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid
     const int64_t Tv = scan_s[2 * kWarpsMma];
     const int64_t g0 = kcta * Tv / P, g1 = (kcta + 1) * Tv / P;
     const int64_t before = scan_s[kWarpsMma + warp] + incl - mine;  // tiles before sequence b_lo
+    if (kcta == 0) {  // for the combine kernel: each sequence's first tile, and Tv
+      int64_t acc = before;
+      for (int b = b_lo; b < b_hi; ++b) {
+        a.seq_first[b] = acc;
+        acc += hkv * ((seq_len(b) + TILE - 1) / TILE);
+      }
+      if (tid == 0) a.seq_first[a.batch] = Tv;
+    }
     if (g0 < g1 && before <= g0 && g0 < before + mine) {
       int64_t pre = before, len = len_lo;
       int b = b_lo;
@@ -1096,10 +1105,12 @@ struct CombineArgs {
   int batch, hq, hkv, G, s_max;
   int ppc;     // partials per CTA and unit (consecutive slots)
   int64_t tiles_per_unit, total_tiles, n_ctas;
-  // Split by the tokens present (decode_mma_kernel): tile_tokens > 0, the lengths as there,
-  // and CTA k's partial of unit u in slot u + k.
+  // Split by the tokens present (decode_mma_kernel): tile_tokens > 0, the lengths as there
+  // (and with them each sequence's first tile and Tv, as the decode grid wrote them), and CTA
+  // k's partial of unit u in slot u + k.
   int tile_tokens;
   const int32_t* seq_lens;
+  const int64_t* seq_first;
   int64_t max_len;
 };
 
@@ -1110,7 +1121,6 @@ __global__ void __launch_bounds__(kD) combine_mma_kernel(const __grid_constant__
   constexpr int RS = kPartPadMma + kD;
   __shared__ float w_s[kD];
   __shared__ float red_s[2][kD / 32];
-  __shared__ long long cnt_s[2][kD / 32];
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int u = blockIdx.x / a.G, h = blockIdx.x - u * a.G;
@@ -1133,25 +1143,14 @@ __global__ void __launch_bounds__(kD) combine_mma_kernel(const __grid_constant__
       return (len + T - 1) / T;
     };
     const int b = u / a.hkv, kvh = u - b * a.hkv;
-    long long all = 0, before = 0;
-    for (int s = tid; s < a.batch; s += kD) {
-      const long long t = tiles(s);
-      all += t;
-      if (s < b) before += t;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      all += __shfl_xor_sync(kFull, all, o);
-      before += __shfl_xor_sync(kFull, before, o);
-    }
-    if (lane == 0) {
-      cnt_s[0][warp] = all;
-      cnt_s[1][warp] = before;
-    }
-    __syncthreads();
-    Tv = a.hkv * ((cnt_s[0][0] + cnt_s[0][1]) + (cnt_s[0][2] + cnt_s[0][3]));
     nu = tiles(b);
-    pre = a.hkv * ((cnt_s[1][0] + cnt_s[1][1]) + (cnt_s[1][2] + cnt_s[1][3])) + kvh * nu;
+    if (a.seq_lens) {
+      Tv = a.seq_first[a.batch];
+      pre = a.seq_first[b] + kvh * nu;
+    } else {
+      Tv = (int64_t)a.batch * a.hkv * nu;
+      pre = (int64_t)u * nu;
+    }
     if (nu == 0) {  // no token: no partial
       const int row = b * a.hq + kvh * a.G + h;
       a.out[(size_t)row * kD + tid] = 0.f;
@@ -1297,6 +1296,7 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
   char* ws = static_cast<char*>(workspace);
   uint32_t* frag = reinterpret_cast<uint32_t*>(ws + plan.off_frag);
   float* part = reinterpret_cast<float*>(ws + plan.off_part);
+  int64_t* seq_first = reinterpret_cast<int64_t*>(ws + plan.off_cnt);
   const int G = hq / hkv, lmb = ctx->shape.lm_bits, vb = ctx->shape.v_bits, nb = n_blocks(G);
   if (plan.n_ctas < 1 || plan.tiles_per_unit < 1) return cudaErrorInvalidValue;
 
@@ -1352,6 +1352,7 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
   a.scores = scores;
   a.out = out;
   a.ws_part = part;
+  a.seq_first = seq_first;
   a.use_tma = (max_len % 4 == 0) ? 1 : 0;
   a.err = ctx->d_err;
   const dim3 grid((unsigned)plan.n_ctas);
@@ -1366,17 +1367,19 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
   if (e != cudaSuccess) return e;
 
   return launch_combine_partials(part, out, lse, batch, hq, hkv, G, plan.s_max, 1, plan.tiles_per_unit,
-                                 plan.total_tiles, plan.n_ctas, stream, mma_tile_tokens(G), seq_lens, max_len);
+                                 plan.total_tiles, plan.n_ctas, stream, mma_tile_tokens(G), seq_lens, seq_first,
+                                 max_len);
 }
 
 cudaError_t launch_combine_partials(const float* part, float* out, float* lse, int batch, int hq, int hkv, int G,
                                     int s_max, int ppc, int64_t tiles_per_unit, int64_t total_tiles, int n_ctas,
                                     cudaStream_t stream, int tile_tokens, const int32_t* seq_lens,
-                                    int64_t max_len) {
+                                    const int64_t* seq_first, int64_t max_len) {
   CombineArgs ca;
   ca.batch = batch;
   ca.tile_tokens = tile_tokens;
   ca.seq_lens = seq_lens;
+  ca.seq_first = seq_first;
   ca.max_len = max_len;
   ca.ppc = ppc;
   ca.ws_part = part;

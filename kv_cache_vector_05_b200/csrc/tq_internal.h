@@ -117,13 +117,14 @@ cudaError_t launch_decode_tc(const tq_ctx* ctx, const DecodePlan& plan, const vo
 // into out (and lse), launched as a programmatic dependent of the decode grid (decode_mma.cu).
 // With tile_tokens = 0 the layout is [units][s_max][ppc][G][4 + 128] (ppc partials per CTA,
 // tiles split by max_len); with tile_tokens > 0 it is decode_mma_kernel's split by the tokens
-// present (tiles of tile_tokens, lengths from seq_lens and max_len): CTA k's partial of unit u
-// in slot u + k of [units + n_ctas][G][4 + 128]. A partial with m = -inf carries no token and
+// present (tiles of tile_tokens, lengths from seq_lens and max_len; with lengths, seq_first
+// holds each sequence's first tile in that order and the total, as the decode grid wrote
+// them): CTA k's partial of unit u in slot u + k of [units + n_ctas][G][4 + 128]. A partial with m = -inf carries no token and
 // its sums are not read.
 cudaError_t launch_combine_partials(const float* part, float* out, float* lse, int batch, int hq, int hkv, int G,
                                     int s_max, int ppc, int64_t tiles_per_unit, int64_t total_tiles, int n_ctas,
                                     cudaStream_t stream, int tile_tokens = 0, const int32_t* seq_lens = nullptr,
-                                    int64_t max_len = 0);
+                                    const int64_t* seq_first = nullptr, int64_t max_len = 0);
 
 size_t mma_frag_bytes(int lm_bits, int G);  // query operand bytes per (sequence, KV head)
 int mma_tile_tokens(int G);                  // tokens per tile of the tensor-core decode

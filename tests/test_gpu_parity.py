@@ -340,6 +340,21 @@ def test_decode_variable_lengths_split_by_tokens(lm_bits, v_bits, G):
                   lens=[0, 2048, 1, 0, 1501, 513, 7], kernel="mma")
 
 
+def test_decode_many_sequences_split_scan():
+    """1500 sequences of 0 to 300 tokens on the mma.sync decode: each of its 512 threads scans
+    three sequences' lengths to find the CTA's first tile, and the combine kernel reads each
+    sequence's first tile as the decode grid wrote it; rows on either side of the 512- and
+    1024-sequence chunk edges and a seeded sample against the oracle."""
+    batch = 1500
+    lens = np.random.default_rng(31).integers(0, 301, batch)
+    lens[[0, 511, 1024]] = 0
+    lens[[1, 512, 1499]] = 300
+    pick = sorted(set([0, 1, 2, 510, 511, 512, 513, 1023, 1024, 1025, 1499]
+                      + list(np.random.default_rng(32).integers(0, batch, 12))))
+    _decode_check(128, 2, 2, batch=batch, hkv=1, G=4, max_len=300, lens=[int(x) for x in lens],
+                  kernel="mma", units=pick)
+
+
 def test_decode_kernel_selection():
     """TQ_DECODE_AUTO takes the mma.sync kernel for 1- to 3-bit codes with the QJL stage,
     the tcgen05 kernel for keys without QJL, and the generic kernels for every other shape;
