@@ -219,7 +219,8 @@ __device__ __forceinline__ void stage_matrix(float* dst, const float* src, int t
   for (int u = 0; u < kPer; ++u) d4[tid + u * kPrepThreads] = v[u];
 }
 
-template <int LMB>
+// HS: query-head slots worked on (4 for one n-block of heads, 8 for two).
+template <int LMB, int HS>
 __global__ void __launch_bounds__(kPrepThreads) prep_mma_kernel(const __grid_constant__ PrepArgs a) {
   // Let the dependent decode grid start streaming its cache tiles right away.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -235,9 +236,9 @@ __global__ void __launch_bounds__(kPrepThreads) prep_mma_kernel(const __grid_con
   const int qrow0 = b * a.hq + kvh * G;
 
   {
-    float v[8 * kD / kPrepThreads];
+    float v[HS * kD / kPrepThreads];
 #pragma unroll
-    for (int u = 0; u < 8 * kD / kPrepThreads; ++u) {
+    for (int u = 0; u < HS * kD / kPrepThreads; ++u) {
       const int idx = tid + u * kPrepThreads, h = idx / kD, j = idx % kD;
       const size_t off = (size_t)(qrow0 + h) * kD + j;
       v[u] = 0.f;
@@ -246,7 +247,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_mma_kernel(const __grid_con
                                    : __bfloat162float(static_cast<const __nv_bfloat16*>(a.q)[off]);
     }
 #pragma unroll
-    for (int u = 0; u < 8 * kD / kPrepThreads; ++u) {
+    for (int u = 0; u < HS * kD / kPrepThreads; ++u) {
       const int idx = tid + u * kPrepThreads, j = idx % kD;
       float x = v[u];
       if (a.rot == TQ_ROT_HADAMARD) x = flip_sign(x, (a.cb.sign_bits[j / 32] >> (j % 32)) & 1u);
@@ -256,7 +257,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_mma_kernel(const __grid_con
   __syncthreads();
   if (a.rot == TQ_ROT_HADAMARD) {
     for (int hs = 1; hs < kD; hs <<= 1) {
-      for (int p = tid; p < 8 * (kD / 2); p += kPrepThreads) {
+      for (int p = tid; p < HS * (kD / 2); p += kPrepThreads) {
         const int h = p / (kD / 2), i = p % (kD / 2);
         const int i0 = h * kD + (i / hs) * 2 * hs + (i % hs);
         const float u = x_s[i0], w = x_s[i0 + hs];
@@ -265,57 +266,59 @@ __global__ void __launch_bounds__(kPrepThreads) prep_mma_kernel(const __grid_con
       }
       __syncthreads();
     }
-    for (int idx = tid; idx < 8 * kD; idx += kPrepThreads) qr_s[idx] = x_s[idx] * a.inv_sqrt_d;
+    for (int idx = tid; idx < HS * kD; idx += kPrepThreads) qr_s[idx] = x_s[idx] * a.inv_sqrt_d;
   } else {
     stage_matrix(st_s, a.PiT, tid);
     __syncthreads();
     const int i = tid % kD, half = tid / kD;
-    float acc[8];
+    float acc[HS];
 #pragma unroll
-    for (int h = 0; h < 8; ++h) acc[h] = 0.f;
+    for (int h = 0; h < HS; ++h) acc[h] = 0.f;
 #pragma unroll 8
     for (int j = half * (kD / 2); j < (half + 1) * (kD / 2); ++j) {
       const float pv = st_s[j * kD + i];
 #pragma unroll
-      for (int h = 0; h < 8; ++h) acc[h] = fmaf(pv, x_s[h * kD + j], acc[h]);
+      for (int h = 0; h < HS; ++h) acc[h] = fmaf(pv, x_s[h * kD + j], acc[h]);
     }
     if (half == 1)
 #pragma unroll
-      for (int h = 0; h < 8; ++h) sq_s[h * kD + i] = acc[h];  // scratch
+      for (int h = 0; h < HS; ++h) sq_s[h * kD + i] = acc[h];  // scratch
     __syncthreads();
     if (half == 0)
 #pragma unroll
-      for (int h = 0; h < 8; ++h) qr_s[h * kD + i] = acc[h] + sq_s[h * kD + i];
+      for (int h = 0; h < HS; ++h) qr_s[h * kD + i] = acc[h] + sq_s[h * kD + i];
     __syncthreads();  // st_s is reused for S^T below
   }
   __syncthreads();
   {
-    // sq = S qr for the 8 head slots at once. S^T is staged in shared memory with
+    // sq = S qr for the HS head slots at once. S^T is staged in shared memory with
     // independent 16-byte loads (its 64 KB would otherwise be read at L2 latency,
     // one dependent load per step); thread (i, half) then runs over half of j.
     stage_matrix(st_s, a.St, tid);
     __syncthreads();
     const int i = tid % kM, half = tid / kM;
-    float acc[8];
+    float acc[HS];
 #pragma unroll
-    for (int h = 0; h < 8; ++h) acc[h] = 0.f;
+    for (int h = 0; h < HS; ++h) acc[h] = 0.f;
 #pragma unroll 8
     for (int j = half * (kD / 2); j < (half + 1) * (kD / 2); ++j) {
       const float sv = st_s[j * kM + i];
 #pragma unroll
-      for (int h = 0; h < 8; ++h) acc[h] = fmaf(sv, qr_s[h * kD + j], acc[h]);
+      for (int h = 0; h < HS; ++h) acc[h] = fmaf(sv, qr_s[h * kD + j], acc[h]);
     }
     if (half == 1)
 #pragma unroll
-      for (int h = 0; h < 8; ++h) x_s[h * kM + i] = acc[h];
+      for (int h = 0; h < HS; ++h) x_s[h * kM + i] = acc[h];
     __syncthreads();
     if (half == 0)
 #pragma unroll
-      for (int h = 0; h < 8; ++h) sq_s[h * kM + i] = acc[h] + x_s[h * kM + i];
+      for (int h = 0; h < HS; ++h) sq_s[h * kM + i] = acc[h] + x_s[h * kM + i];
   }
   __syncthreads();
-  {
-    const int h = warp;  // 8 warps, one per head slot
+  if (warp >= HS) {  // slots past HS: constants of an empty head (never read)
+    if (lane < 4) head_s[warp * 4 + lane] = 0.f;
+  } else {
+    const int h = warp;  // one warp per head slot
     float qsum = 0.f, ssum = 0.f, qmax = 0.f, smax = 0.f;
     for (int j = lane; j < kD; j += 32) {
       qsum += qr_s[h * kD + j];
@@ -1318,20 +1321,25 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
   const size_t prep_smem = sizeof(float) * kD * kM;
   static bool prep_configured = false;
   if (!prep_configured) {
-    cudaError_t ce = cudaFuncSetAttribute(prep_mma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep_smem);
-    if (ce == cudaSuccess)
-      ce = cudaFuncSetAttribute(prep_mma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep_smem);
-    if (ce == cudaSuccess)
-      ce = cudaFuncSetAttribute(prep_mma_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep_smem);
-    if (ce != cudaSuccess) return ce;
+    const void* kernels[6] = {(const void*)prep_mma_kernel<1, 4>, (const void*)prep_mma_kernel<2, 4>,
+                              (const void*)prep_mma_kernel<3, 4>, (const void*)prep_mma_kernel<1, 8>,
+                              (const void*)prep_mma_kernel<2, 8>, (const void*)prep_mma_kernel<3, 8>};
+    for (const void* k : kernels) {
+      const cudaError_t ce = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep_smem);
+      if (ce != cudaSuccess) return ce;
+    }
     prep_configured = true;
   }
-  if (lmb == 1)
-    prep_mma_kernel<1><<<batch * hkv, kPrepThreads, prep_smem, stream>>>(pa);
-  else if (lmb == 2)
-    prep_mma_kernel<2><<<batch * hkv, kPrepThreads, prep_smem, stream>>>(pa);
-  else
-    prep_mma_kernel<3><<<batch * hkv, kPrepThreads, prep_smem, stream>>>(pa);
+  const unsigned prep_grid = (unsigned)(batch * hkv);
+  if (nb == 1) {
+    if (lmb == 1) prep_mma_kernel<1, 4><<<prep_grid, kPrepThreads, prep_smem, stream>>>(pa);
+    else if (lmb == 2) prep_mma_kernel<2, 4><<<prep_grid, kPrepThreads, prep_smem, stream>>>(pa);
+    else prep_mma_kernel<3, 4><<<prep_grid, kPrepThreads, prep_smem, stream>>>(pa);
+  } else {
+    if (lmb == 1) prep_mma_kernel<1, 8><<<prep_grid, kPrepThreads, prep_smem, stream>>>(pa);
+    else if (lmb == 2) prep_mma_kernel<2, 8><<<prep_grid, kPrepThreads, prep_smem, stream>>>(pa);
+    else prep_mma_kernel<3, 8><<<prep_grid, kPrepThreads, prep_smem, stream>>>(pa);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
