@@ -1300,7 +1300,9 @@ __device__ __forceinline__ double div_levels(double span) {
   return fma(fma(-(double)L, q0, span), inv, q0);
 }
 
-template <int LMB, int VB, int NT>
+// QJL: the QJL stage is on (m = 128); without it (m = 0) the S tiles, the residual operand,
+// the projection and the sign readout are left out, and gamma = ||r|| is stored as before.
+template <int LMB, int VB, int NT, bool QJL>
 __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __grid_constant__ CompressArgs a) {
   using PS = PipeSmem<NT>;
   namespace s1 = tq::sm100;
@@ -1335,8 +1337,10 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
     uint4* hdst = reinterpret_cast<uint4*>(sm + PS::HB);
     uint4* sdst = reinterpret_cast<uint4*>(sm + PS::S);
     for (int w = tid; w < (int)(kTcTileBytes / 16); w += kPipeThreads) {
-      sdst[w] = ssrc[w];
-      sdst[w + kTcTileBytes / 16] = ssrc[w + kTcTileBytes / 16];
+      if constexpr (QJL) {
+        sdst[w] = ssrc[w];
+        sdst[w + kTcTileBytes / 16] = ssrc[w + kTcTileBytes / 16];
+      }
 #pragma unroll
       for (int t = 0; t < NT; ++t) hdst[w + t * (kTcTileBytes / 16)] = hsrc[w + t * (kTcTileBytes / 16)];
     }
@@ -1409,7 +1413,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
         const float sc16 = nz ? 16.f * (1.0f / sqrtf(tot)) : 0.f;
         const float2 sc2 = make_float2(sc16, sc16);
         // the previous projection has finished: its S r is readable and the operand free
-        if (it > 0) {
+        if (QJL && it > 0) {
           if (!failed && !s1::mbar_wait(projd, (uint32_t)(it - 1) & 1u)) failed = true;
           s1::fence_after_sync();
           read_signs(prev_o, prev_nz);
@@ -1446,8 +1450,10 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
             }
             // row R's coordinates 64ch + 32h + 16o8 .. + 15: 8 columns of hi and of lo
             const uint32_t col = 32 * ch + 16 * h + 8 * o8;
-            s1::tmem_st8(tmem + kTmA + lane_base + col, hw);
-            s1::tmem_st8(tmem + kTmA + 64 + lane_base + col, lw);
+            if constexpr (QJL) {
+              s1::tmem_st8(tmem + kTmA + lane_base + col, hw);
+              s1::tmem_st8(tmem + kTmA + 64 + lane_base + col, lw);
+            }
           }
           if (o >= 0) {
             uint32_t* co = reinterpret_cast<uint32_t*>(a.k_codes + o * (LMB * 16) + ch * (LMB * 8) + h * (LMB * 4));
@@ -1475,7 +1481,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
         prev_nz = nz;
       }
       // the last pass's signs
-      if (!failed && it > 0) {
+      if (QJL && !failed && it > 0) {
         if (!s1::mbar_wait(projd, (uint32_t)(it - 1) & 1u)) {
           failed = true;
         } else {
@@ -1712,7 +1718,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
         break;
       }
       s1::fence_after_sync();
-      projection();
+      if constexpr (QJL) projection();
       // Y[b] is free again: rotate pass j+2 once its keys have landed
       if (j + 2 < n_my) {
         if (!wait_keys(b)) {
@@ -1780,12 +1786,12 @@ bool codebook_symmetric(const Codebook& cb, int lm_bits) {
   return true;
 }
 
-template <int LMB, int VB, int NT>
+template <int LMB, int VB, int NT, bool QJL = true>
 cudaError_t launch_pipe_t(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) {
   static bool configured = false;
   const size_t smem = PipeSmem<NT>::BYTES + 1024;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(compress_pipe_kernel<LMB, VB, NT>,
+    cudaError_t e = cudaFuncSetAttribute(compress_pipe_kernel<LMB, VB, NT, QJL>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured = true;
@@ -1793,7 +1799,7 @@ cudaError_t launch_pipe_t(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t
   int64_t blocks = (a.n_vec + 127) / 128;
   if (blocks > ctx->num_sms) blocks = ctx->num_sms;
   if (ctx->prof_start) cudaEventRecord(ctx->prof_start, s);
-  compress_pipe_kernel<LMB, VB, NT><<<(unsigned)blocks, kPipeThreads, smem, s>>>(a);
+  compress_pipe_kernel<LMB, VB, NT, QJL><<<(unsigned)blocks, kPipeThreads, smem, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (ctx->prof_stop) cudaEventRecord(ctx->prof_stop, s);
   return e;
@@ -1804,6 +1810,19 @@ cudaError_t launch_pipe(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s
   if (lmb == 1) return vb == 2 ? launch_pipe_t<1, 2, 1>(ctx, a, s) : launch_pipe_t<1, 4, 1>(ctx, a, s);
   if (lmb == 2) return vb == 2 ? launch_pipe_t<2, 2, 1>(ctx, a, s) : launch_pipe_t<2, 4, 1>(ctx, a, s);
   return vb == 2 ? launch_pipe_t<3, 2, 1>(ctx, a, s) : launch_pipe_t<3, 4, 1>(ctx, a, s);
+}
+
+// Keys without the QJL stage (m = 0; either rotation), or values alone, on the same kernel.
+cudaError_t launch_pipe_nq(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) {
+  const int lmb = ctx->shape.lm_bits, vb = ctx->shape.v_bits;
+  if (a.k && ctx->shape.rot == TQ_ROT_HAAR) {  // keys only: the Haar tiles take the value rows
+    if (lmb == 1) return launch_pipe_t<1, 2, 3, false>(ctx, a, s);
+    if (lmb == 2) return launch_pipe_t<2, 2, 3, false>(ctx, a, s);
+    return launch_pipe_t<3, 2, 3, false>(ctx, a, s);
+  }
+  if (lmb == 1) return vb == 4 ? launch_pipe_t<1, 4, 1, false>(ctx, a, s) : launch_pipe_t<1, 2, 1, false>(ctx, a, s);
+  if (lmb == 2) return vb == 4 ? launch_pipe_t<2, 4, 1, false>(ctx, a, s) : launch_pipe_t<2, 2, 1, false>(ctx, a, s);
+  return vb == 4 ? launch_pipe_t<3, 4, 1, false>(ctx, a, s) : launch_pipe_t<3, 2, 1, false>(ctx, a, s);
 }
 
 // Keys only with the Haar rotation (its three operand tiles in place of the value rows).
@@ -2428,6 +2447,26 @@ cudaError_t launch_compress(const tq_ctx* ctx, const void* k, const void* v, int
     if (ctx->shape.rot == TQ_ROT_HADAMARD)
       return dtype == TQ_F32 ? launch_q4<float>(ctx, a, stream) : launch_q4<__nv_bfloat16>(ctx, a, stream);
     return dtype == TQ_F32 ? launch_tc<float>(ctx, a, stream) : launch_tc<__nv_bfloat16>(ctx, a, stream);
+  }
+  if (ctx->shape.d == 128 && ctx->shape.m == 0 && dtype == TQ_BF16 &&
+      codebook_symmetric(ctx->cb, ctx->shape.lm_bits)) {
+    // Keys without the QJL stage on the pipelined kernel (rotation on the tensor cores, no
+    // projection); values there too at 2 or 4 bits, else on the warp-per-vector kernel.
+    a.H_sw128 = ctx->shape.rot == TQ_ROT_HAAR ? ctx->Pi_sw128 : ctx->H_sw128;
+    const bool keys_ok = !k || (a.H_sw128 && encode_rows_map(&a.kmap, k, n_vec, 128));
+    if (keys_ok) {
+      if (k) {
+        CompressArgs ka = a;
+        ka.v = nullptr;
+        const cudaError_t e = launch_pipe_nq(ctx, ka, stream);
+        if (e != cudaSuccess || !v) return e;
+      }
+      CompressArgs va = a;
+      va.k = nullptr;
+      if (ctx->shape.v_bits != 3 && a.H_sw128 && encode_rows_map(&va.vmap, v, n_vec, 64))
+        return launch_pipe_nq(ctx, va, stream);
+      return generic(va);
+    }
   }
   return generic(a);
 }

@@ -168,7 +168,10 @@ tq_status tq_codebook_load(const tq_params* p, void* stream, tq_ctx** out) {
     if (e == cudaSuccess && !s_op.empty()) e = cudaMalloc((void**)&c->S_sw128, s_op.size() * sizeof(uint16_t));
   }
   std::vector<uint16_t> h_op;
-  if (d == 128 && m == 128 && !s_op.empty() && p->rot == TQ_ROT_HADAMARD) {
+  // the rotation operand of the pipelined compression kernel: with the QJL stage when S fits
+  // its operand tiles, and for keys without it (m = 0)
+  const bool pipe_rot = d == 128 && ((m == 128 && !s_op.empty()) || m == 0);
+  if (pipe_rot && p->rot == TQ_ROT_HADAMARD) {
     h_op.assign((size_t)d * d, 0);
     tq::pack_hadamard_operand(c->cb.sign_bits, h_op.data());
     if (e == cudaSuccess) e = cudaMalloc((void**)&c->H_sw128, h_op.size() * sizeof(uint16_t));
@@ -180,7 +183,7 @@ tq_status tq_codebook_load(const tq_params* p, void* stream, tq_ctx** out) {
       e = cudaMalloc((void**)&c->dense_ops, dense_op.size() * sizeof(uint16_t));
   }
   std::vector<uint16_t> pi_op;
-  if (d == 128 && m == 128 && !s_op.empty() && p->rot == TQ_ROT_HAAR) {
+  if (pipe_rot && p->rot == TQ_ROT_HAAR) {
     pi_op.assign((size_t)3 * d * d, 0);
     tq::pack_haar_operand(p->haar, pi_op.data());
     if (e == cudaSuccess) e = cudaMalloc((void**)&c->Pi_sw128, pi_op.size() * sizeof(uint16_t));

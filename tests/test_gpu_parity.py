@@ -584,6 +584,43 @@ def test_keys_without_qjl_stage(d, lm_bits, v_bits, rotation, dtype):
     assert_close(kx.cpu().numpy(), O.decompress_keys(pk, Pi, c, S0, d), rtol=1e-4, atol=1e-5, what="keys")
 
 
+@pytest.mark.parametrize("lm_bits,v_bits,rotation", [
+    (1, 2, "hadamard"), (2, 4, "hadamard"), (3, 3, "hadamard"), (2, 2, "haar"), (3, 4, "haar")])
+def test_keys_without_qjl_pipelined_compression(lm_bits, v_bits, rotation):
+    """qjl_m = 0, bf16, d = 128: keys on the pipelined tensor-core kernel without its
+    projection (values on its value warps at 2 and 4 bits, on the warp-per-vector kernel at
+    3); two to three passes per CTA and a ragged last pass, zero keys, every vector against
+    the oracle; keys alone and values alone give the same records."""
+    d = 128
+    dr = W.method_draws(d, d, 1234)
+    c32, t32 = T.tq_lloyd_max_codebook(d, lm_bits)
+    haar = T.tq_haar_from_gaussian(dr["haar_gaussian"]) if rotation == "haar" else None
+    S0 = np.zeros((0, d))
+    ctx = T.tq_codebook_load(d, lm_bits, v_bits, c32, t32, S0, rotation=rotation,
+                             hadamard_signs=dr["hadamard_signs"], haar=haar)
+    n = 148 * 128 * 2 + 5 * 128 + 77
+    rng = np.random.default_rng([41, lm_bits, v_bits])
+    K = rng.standard_normal((n, d)) * rng.lognormal(0, 1, d)
+    V = rng.standard_normal((n, d)) * 2.0 - 0.5
+    K[[0, 128 * 148, n - 1]] = 0.0
+    kt = torch.from_numpy(K.astype(np.float32)).to(DEV).to(torch.bfloat16)
+    vt = torch.from_numpy(V.astype(np.float32)).to(DEV).to(torch.bfloat16)
+    g = to_np(T.tq_compress_kv(ctx, kt, vt))
+    T.tq_check_device(ctx)
+    Pi, c, t, _ = oracle_setup(d, lm_bits, d, rotation)
+    ok = O.compress_keys(kt.float().cpu().numpy().astype(np.float64), Pi, c, t, S0, with_diagnostics=True)
+    ov = O.quantize_values(vt.float().cpu().numpy().astype(np.float64), v_bits, with_diagnostics=True)
+    assert_key_parity(compare_keys(g, ok, d, lm_bits, 0))
+    assert_value_parity(compare_values(g, ov, d, v_bits))
+    gk = to_np(T.tq_compress_kv(ctx, kt, None))
+    gv = to_np(T.tq_compress_kv(ctx, None, vt))
+    T.tq_check_device(ctx)
+    for name in ("k_codes", "k_norms"):
+        assert np.array_equal(gk[name], g[name]), name
+    for name in ("v_codes", "v_params"):
+        assert np.array_equal(gv[name], g[name]), name
+
+
 # ------------------------------------------------------------------ 3-bit values (K = V = 3)
 
 @pytest.mark.parametrize("d,lm_bits,rotation,dtype", [
