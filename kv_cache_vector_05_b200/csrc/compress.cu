@@ -1336,7 +1336,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
     const uint4* ssrc = reinterpret_cast<const uint4*>(a.S_sw128);
     uint4* hdst = reinterpret_cast<uint4*>(sm + PS::HB);
     uint4* sdst = reinterpret_cast<uint4*>(sm + PS::S);
-    for (int w = tid; w < (int)(kTcTileBytes / 16); w += kPipeThreads) {
+    for (int w = tid; a.k && w < (int)(kTcTileBytes / 16); w += kPipeThreads) {  // values alone: none
       if constexpr (QJL) {
         sdst[w] = ssrc[w];
         sdst[w + kTcTileBytes / 16] = ssrc[w + kTcTileBytes / 16];
@@ -1597,12 +1597,18 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
               if (fabsf(e.x) > 0.5f - 5e-6f) near |= 1u << (2 * k);
               if (fabsf(e.y) > 0.5f - 5e-6f) near |= 2u << (2 * k);
             }
-            // tr's bits are those of the magic constant plus the code
-            add_field<VB, VB>(vw, VB * 2 * k, __float_as_uint(tr.x));
-            add_field<VB, VB>(vw2, VB * (2 * k + 1), __float_as_uint(tr.y));
+            if constexpr (VB == 3) {
+              // 3-bit fields straddle words: the code alone, masked out of tr's low bits
+              add_field<VB, VB>(vw, VB * 2 * k, __float_as_uint(tr.x) & 7u);
+              add_field<VB, VB>(vw2, VB * (2 * k + 1), __float_as_uint(tr.y) & 7u);
+            } else {
+              // tr's bits are those of the magic constant plus the code
+              add_field<VB, VB>(vw, VB * 2 * k, __float_as_uint(tr.x));
+              add_field<VB, VB>(vw2, VB * (2 * k + 1), __float_as_uint(tr.y));
+            }
           }
 #pragma unroll
-          for (int k = 0; k < VB; ++k) vw[k] = vw[k] + vw2[k] - magic_sum;
+          for (int k = 0; k < VB; ++k) vw[k] = vw[k] + vw2[k] - (VB == 3 ? 0u : magic_sum);
           if (kRedoNearHalf && near) {
             // Some coordinate lies within 5e-6 of a half step (with bf16 inputs a ratio of
             // small integers lands exactly on one in about one group of twenty): redo only
@@ -1621,6 +1627,11 @@ __global__ void __launch_bounds__(kPipeThreads, 1) compress_pipe_kernel(const __
                 const uint32_t sel = (wi == k) ? 0xffffffffu : 0u;
                 const uint32_t old = (vw[k] >> sh) & (uint32_t)levels;
                 vw[k] ^= ((old ^ qv) << sh) & sel;
+                if (VB == 3 && sh > 29) {  // the field's high bits, at the bottom of the next word
+                  const uint32_t selh = (wi + 1 == k) ? 0xffffffffu : 0u;
+                  const uint32_t mh = (1u << (sh - 29)) - 1u;
+                  vw[k] ^= ((vw[k] & mh) ^ (qv >> (32 - sh))) & selh;
+                }
               }
             }
           }
@@ -1805,11 +1816,17 @@ cudaError_t launch_pipe_t(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t
   return e;
 }
 
+template <int VB>
+cudaError_t launch_pipe_vb(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) {
+  const int lmb = ctx->shape.lm_bits;
+  if (lmb == 1) return launch_pipe_t<1, VB, 1>(ctx, a, s);
+  if (lmb == 2) return launch_pipe_t<2, VB, 1>(ctx, a, s);
+  return launch_pipe_t<3, VB, 1>(ctx, a, s);
+}
+
 cudaError_t launch_pipe(const tq_ctx* ctx, const CompressArgs& a, cudaStream_t s) {
-  const int lmb = ctx->shape.lm_bits, vb = ctx->shape.v_bits;
-  if (lmb == 1) return vb == 2 ? launch_pipe_t<1, 2, 1>(ctx, a, s) : launch_pipe_t<1, 4, 1>(ctx, a, s);
-  if (lmb == 2) return vb == 2 ? launch_pipe_t<2, 2, 1>(ctx, a, s) : launch_pipe_t<2, 4, 1>(ctx, a, s);
-  return vb == 2 ? launch_pipe_t<3, 2, 1>(ctx, a, s) : launch_pipe_t<3, 4, 1>(ctx, a, s);
+  const int vb = ctx->shape.v_bits;
+  return vb == 2 ? launch_pipe_vb<2>(ctx, a, s) : vb == 3 ? launch_pipe_vb<3>(ctx, a, s) : launch_pipe_vb<4>(ctx, a, s);
 }
 
 // Keys without the QJL stage (m = 0; either rotation), or values alone, on the same kernel.
@@ -1820,9 +1837,12 @@ cudaError_t launch_pipe_nq(const tq_ctx* ctx, const CompressArgs& a, cudaStream_
     if (lmb == 2) return launch_pipe_t<2, 2, 3, false>(ctx, a, s);
     return launch_pipe_t<3, 2, 3, false>(ctx, a, s);
   }
-  if (lmb == 1) return vb == 4 ? launch_pipe_t<1, 4, 1, false>(ctx, a, s) : launch_pipe_t<1, 2, 1, false>(ctx, a, s);
-  if (lmb == 2) return vb == 4 ? launch_pipe_t<2, 4, 1, false>(ctx, a, s) : launch_pipe_t<2, 2, 1, false>(ctx, a, s);
-  return vb == 4 ? launch_pipe_t<3, 4, 1, false>(ctx, a, s) : launch_pipe_t<3, 2, 1, false>(ctx, a, s);
+  if (!a.k)  // values alone: the key settings do not matter
+    return vb == 2 ? launch_pipe_t<1, 2, 1, false>(ctx, a, s)
+           : vb == 3 ? launch_pipe_t<1, 3, 1, false>(ctx, a, s) : launch_pipe_t<1, 4, 1, false>(ctx, a, s);
+  if (lmb == 1) return launch_pipe_t<1, 2, 1, false>(ctx, a, s);
+  if (lmb == 2) return launch_pipe_t<2, 2, 1, false>(ctx, a, s);
+  return launch_pipe_t<3, 2, 1, false>(ctx, a, s);
 }
 
 // Keys only with the Haar rotation (its three operand tiles in place of the value rows).
@@ -2406,9 +2426,35 @@ cudaError_t launch_compress(const tq_ctx* ctx, const void* k, const void* v, int
     va.k = nullptr;
     return generic(va);
   }
+  // d = 128, bf16, a symmetric codebook, with the QJL stage (S on its operand tiles) or
+  // without it: the pipelined tensor-core kernel. Values (value coding does not depend on the
+  // keys' settings) run on its value warps, 2 to 4 bits, in the same launch as the keys with the
+  // QJL stage and the Hadamard rotation, in a launch of their own otherwise; the records are the
+  // same either way.
+  const bool pipe_shape = ctx->shape.d == 128 && dtype == TQ_BF16 && codebook_symmetric(ctx->cb, ctx->shape.lm_bits) &&
+                          ((ctx->shape.m == 128 && ctx->S_sw128) || ctx->shape.m == 0);
+  const uint16_t* rot_tiles = ctx->shape.rot == TQ_ROT_HAAR ? ctx->Pi_sw128 : ctx->H_sw128;
+  if (pipe_shape && rot_tiles && (!k || encode_rows_map(&a.kmap, k, n_vec, 128))) {
+    a.H_sw128 = rot_tiles;
+    const bool vmap_ok = v && encode_rows_map(&a.vmap, v, n_vec, 64);
+    auto values_alone = [&]() -> cudaError_t {
+      CompressArgs va = a;
+      va.k = nullptr;
+      return vmap_ok ? launch_pipe_nq(ctx, va, stream) : generic(va);
+    };
+    if (!k) return values_alone();
+    if (ctx->shape.m == 128 && ctx->shape.rot == TQ_ROT_HADAMARD && (!v || vmap_ok))
+      return launch_pipe(ctx, a, stream);  // keys and values in one launch
+    CompressArgs ka = a;
+    ka.v = nullptr;
+    const cudaError_t e = ctx->shape.m == 0 ? launch_pipe_nq(ctx, ka, stream)
+                          : ctx->shape.rot == TQ_ROT_HAAR ? launch_pipe_haar(ctx, ka, stream)
+                                                          : launch_pipe(ctx, ka, stream);
+    if (e != cudaSuccess || !v) return e;
+    return values_alone();
+  }
   if (ctx->shape.v_bits == 3 && k && v && ctx->S_sw128) {
-    // 3-bit value codes straddle words: the tensor-core kernels take the keys alone and
-    // the warp-per-vector kernel the values
+    // 3-bit values on the warp-per-vector kernel, the keys alone on the tensor-core kernels
     CompressArgs vv = a;
     vv.k = nullptr;
     const cudaError_t e = launch_compress(ctx, k, nullptr, dtype, n_vec, slot, n_rows, k_codes, k_signs, k_norms,
@@ -2416,57 +2462,15 @@ cudaError_t launch_compress(const tq_ctx* ctx, const void* k, const void* v, int
     return e != cudaSuccess ? e : generic(vv);
   }
   if (ctx->S_sw128 && ctx->shape.d == 128 && ctx->shape.m == 128 && !(ctx->shape.v_bits == 3 && v)) {
-    if (ctx->shape.rot == TQ_ROT_HADAMARD && dtype == TQ_BF16 && ctx->H_sw128) {
-      if (codebook_symmetric(ctx->cb, ctx->shape.lm_bits) && (!k || encode_rows_map(&a.kmap, k, n_vec, 128)) &&
-          (!v || encode_rows_map(&a.vmap, v, n_vec, 64)))
-        return launch_pipe(ctx, a, stream);
-      return launch_rot<false>(ctx, a, stream);
-    }
+    // fp32 keys, a codebook that is not symmetric, or rows no tensor map takes
+    if (ctx->shape.rot == TQ_ROT_HADAMARD && dtype == TQ_BF16 && ctx->H_sw128) return launch_rot<false>(ctx, a, stream);
     if (ctx->shape.rot == TQ_ROT_HAAR && dtype == TQ_BF16 && ctx->Pi_sw128) {
       a.H_sw128 = ctx->Pi_sw128;
-      if (!v || encode_rows_map(&a.vmap, v, n_vec, 64)) {
-        // Values (value coding does not depend on the rotation) on the value warps of the
-        // pipelined kernel in a launch of their own, so that they come out the same with or
-        // without keys in the call; keys on the pipelined kernel with the three Haar tiles,
-        // or one pass at a time for a codebook that is not symmetric.
-        if (k) {
-          CompressArgs ka = a;
-          ka.v = nullptr;
-          const cudaError_t e =
-              codebook_symmetric(ctx->cb, ctx->shape.lm_bits) && encode_rows_map(&ka.kmap, k, n_vec, 128)
-                  ? launch_pipe_haar(ctx, ka, stream)
-                  : launch_rot<true>(ctx, ka, stream);
-          if (e != cudaSuccess || !v) return e;
-        }
-        CompressArgs va = a;
-        va.k = nullptr;
-        return launch_pipe(ctx, va, stream);
-      }
       return launch_rot<true>(ctx, a, stream);
     }
     if (ctx->shape.rot == TQ_ROT_HADAMARD)
       return dtype == TQ_F32 ? launch_q4<float>(ctx, a, stream) : launch_q4<__nv_bfloat16>(ctx, a, stream);
     return dtype == TQ_F32 ? launch_tc<float>(ctx, a, stream) : launch_tc<__nv_bfloat16>(ctx, a, stream);
-  }
-  if (ctx->shape.d == 128 && ctx->shape.m == 0 && dtype == TQ_BF16 &&
-      codebook_symmetric(ctx->cb, ctx->shape.lm_bits)) {
-    // Keys without the QJL stage on the pipelined kernel (rotation on the tensor cores, no
-    // projection); values there too at 2 or 4 bits, else on the warp-per-vector kernel.
-    a.H_sw128 = ctx->shape.rot == TQ_ROT_HAAR ? ctx->Pi_sw128 : ctx->H_sw128;
-    const bool keys_ok = !k || (a.H_sw128 && encode_rows_map(&a.kmap, k, n_vec, 128));
-    if (keys_ok) {
-      if (k) {
-        CompressArgs ka = a;
-        ka.v = nullptr;
-        const cudaError_t e = launch_pipe_nq(ctx, ka, stream);
-        if (e != cudaSuccess || !v) return e;
-      }
-      CompressArgs va = a;
-      va.k = nullptr;
-      if (ctx->shape.v_bits != 3 && a.H_sw128 && encode_rows_map(&va.vmap, v, n_vec, 64))
-        return launch_pipe_nq(ctx, va, stream);
-      return generic(va);
-    }
   }
   return generic(a);
 }

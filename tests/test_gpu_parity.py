@@ -117,6 +117,33 @@ def test_compress_parity_several_passes_per_cta(lm_bits, rotation):
         assert np.array_equal(gv[name], g[name]), name
 
 
+@pytest.mark.parametrize("lm_bits,rotation", [(2, "hadamard"), (3, "haar"), (1, "hadamard")])
+def test_compress_three_bit_values_pipelined_several_passes(lm_bits, rotation):
+    """3-bit value codes (fields straddling 32-bit words, the near-tie redo across a word
+    boundary) on the pipelined kernel's value warps, bf16, d = 128, with the QJL stage: two to
+    three passes per CTA, every vector against the oracle, values alone and keys alone
+    giving the same records as the call with both."""
+    d, v_bits = 128, 3
+    n = 148 * 128 * 2 + 3 * 128 + 45
+    rng = np.random.default_rng([43, lm_bits])
+    K = rng.standard_normal((n, d)).astype(np.float32) * rng.lognormal(0, 1, d).astype(np.float32)
+    V = rng.standard_normal((n, d)).astype(np.float32)
+    V[7, :32] = 0.25                                      # a constant value group
+    V[9, 32:64] = np.arange(32, dtype=np.float32) / 7.0  # codes on exact half steps
+    ctx, g, ok, ov = _compress_both(K, V, d, lm_bits, v_bits, rotation, "bf16")
+    assert_key_parity(compare_keys(g, ok, d, lm_bits, d))
+    assert_value_parity(compare_values(g, ov, d, v_bits))
+    kt = torch.from_numpy(K).to(DEV).to(torch.bfloat16)
+    vt = torch.from_numpy(V).to(DEV).to(torch.bfloat16)
+    gk = to_np(T.tq_compress_kv(ctx, kt, None))
+    gv = to_np(T.tq_compress_kv(ctx, None, vt))
+    T.tq_check_device(ctx)
+    for name in ("k_codes", "k_signs", "k_norms"):
+        assert np.array_equal(gk[name], g[name]), name
+    for name in ("v_codes", "v_params"):
+        assert np.array_equal(gv[name], g[name]), name
+
+
 @pytest.mark.parametrize("d", [64, 256])
 @pytest.mark.parametrize("rotation", ["hadamard", "haar"])
 @pytest.mark.parametrize("lm_bits", [1, 3])
