@@ -186,7 +186,10 @@ size_t tq_decode_workspace_bytes(const tq_ctx* ctx, int batch, int hq, int hkv, 
  * 2- or 4-bit values and at most 8 query heads per KV head, a tensor-core decode runs
  * (tq_set_decode_kernel); it carries p * scale (p < 4) as f16 operands, so value-group
  * scales must stay below 16376 (values spanning less than 49000 at 2 bits). Other
- * shapes run the CUDA-core decode.
+ * shapes run the CUDA-core decode. With seq_lens, the mma.sync decode (the default for
+ * codes with the QJL stage) spreads only the tokens present over the SMs, reading the
+ * lengths on the device, so a batch of varied lengths costs the tokens it holds; the
+ * workspace is sized for max_len either way.
  * Returns TQ_EINVAL if the workspace is too small or any pointer is misaligned. */
 tq_status tq_decode_attention(const tq_ctx* ctx, const void* q, tq_dtype q_dtype, int batch, int hq,
                               int hkv, const int32_t* seq_lens, int64_t max_len,

@@ -185,11 +185,6 @@ __device__ __forceinline__ void mma_i8(int (&d)[4], const uint4& a, uint32_t b0,
       : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint32_t pack_h2(float lo_half, float hi_half) {
-  const __half2 h = __floats2half2_rn(lo_half, hi_half);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-
 __device__ __forceinline__ float2 unpack_h2(uint32_t w) {
   return __half22float2(*reinterpret_cast<const __half2*>(&w));
 }
@@ -491,11 +486,14 @@ __global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid
     return (int)Tu;
   };
   auto next_unit = [&](int u) -> int {  // the next unit after u that holds a token (or units)
-    if constexpr (!VARLEN) return u + 1;
-    do {
-      ++u;
-    } while (u < units && unit_tiles(u) == 0);
-    return u;
+    if constexpr (VARLEN) {
+      do {
+        ++u;
+      } while (u < units && unit_tiles(u) == 0);
+      return u;
+    } else {
+      return u + 1;
+    }
   };
   // Split by the tokens present: the tiles that hold at least one token, of every unit (a
   // unit = one sequence x KV head) laid end to end, are split evenly over the CTAs, so a

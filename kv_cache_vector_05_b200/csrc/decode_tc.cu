@@ -295,7 +295,6 @@ struct TileWalk {
   __device__ __forceinline__ int nt() const {
     return (int)max((int64_t)0, min((int64_t)kTileTc, len - tl * kTileTc));
   }
-  __device__ __forceinline__ bool last_tile() const { return tl == Tu - 1; }
 };
 
 // CTA owning global tile g when CTA k takes tiles [k T / P, (k + 1) T / P).
