@@ -1,5 +1,5 @@
 // Tensor-core decode attention over the packed cache (d = m = 128, up to 8 query
-// heads per KV head, 1- to 3-bit Lloyd-Max keys of a symmetric codebook, 2- or 4-bit values).
+// heads per KV head, 1- to 3-bit Lloyd-Max keys of a symmetric codebook, 2- to 4-bit values).
 //
 // Same mathematics as decode_kernel (the skill card "turboquant-pytorch", "Что
 // делает": scores straight from the compressed keys; the discosf news item:
@@ -23,9 +23,11 @@
 //    are divided by that power of two.
 // Values (mma.sync m16n8k16, f16 operands, fp32 accumulation): rows = 16 value coordinates,
 // K = 16 tokens, columns = 4 query heads x (hi, lo), the two f16 halves of p * scale.
-//  * A value code placed in the low mantissa bits of an f16 is a subnormal equal
-//    to code * 2^(pos - 24), so a byte permute plus a mask yields two exact
-//    operands; the power of two is undone once at the end.
+//  * A value code placed in the mantissa bits of an f16 is a subnormal equal to
+//    code * 2^(pos - 24), so a byte permute, a shift and a mask yield two exact
+//    operands; the power of two is undone once at the end. The codes sit at bit 3 or
+//    higher: products of codes at the lowest positions with the small low parts of
+//    p * scale lost about 1e-4 of the output on the tensor cores.
 //
 // Kernels:
 //  * prep_mma_kernel, one CTA per (sequence, KV head): rotates the G queries
@@ -743,12 +745,16 @@ __global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid
               int j0;
               float v0, v1;
               if (VB == 2) {
-                j0 = 4 * (8 * g + r) + 2 * hf;  // code at mantissa bits 4hf (row r), 4hf + 2 (row r + 8)
-                v0 = (d[0] + d[1]) * ldexpf(1.f, 24 - 4 * hf) + mt[g];
-                v1 = (d[2] + d[3]) * ldexpf(1.f, 22 - 4 * hf) + mt[g];
+                j0 = 4 * (8 * g + r) + 2 * hf;  // code at mantissa bits 4 (row r), 6 (row r + 8)
+                v0 = (d[0] + d[1]) * 1048576.f + mt[g];
+                v1 = (d[2] + d[3]) * 262144.f + mt[g];
+              } else if (VB == 3) {
+                j0 = 32 * g + 4 * r + 2 * hf;  // code at mantissa bit 3 (hf = 0) or 6 (hf = 1)
+                v0 = (d[0] + d[1]) * (hf == 0 ? 2097152.f : 262144.f) + mt[g];
+                v1 = (d[2] + d[3]) * (hf == 0 ? 2097152.f : 262144.f) + mt[g];
               } else {
-                j0 = 2 * (16 * g + 8 * hf + r);  // low nibble (row r), high nibble (row r + 8)
-                v0 = (d[0] + d[1]) * 16777216.f + mt[g];
+                j0 = 2 * (16 * g + 8 * hf + r);  // low nibble (row r), high nibble (row r + 8), both at bit 4
+                v0 = (d[0] + d[1]) * 1048576.f + mt[g];
                 v1 = (d[2] + d[3]) * 1048576.f + mt[g];
               }
               red[j0] = wsc != 0.f ? wsc * v0 : 0.f;
@@ -1039,22 +1045,44 @@ __global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid
             uint32_t xA, xB;
             uint4 av;
             if (VB == 2) {
-              // byte 8g + r: rows r -> coordinate 4(8g + r) + 2hf, rows r + 8 -> + 1
+              // byte 8g + r: rows r -> coordinate 4(8g + r) + 2hf, rows r + 8 -> + 1; codes at
+              // mantissa bits 4 (rows r) and 6 (rows r + 8), those of hf = 0 shifted up by 4
               constexpr int WPT = L::VCB / 4;
               const int wv = 2 * g + (r >> 2);
               if (hf == 0) {
                 xA = __byte_perm(vc[tA0 * WPT + wv], vc[tA1 * WPT + wv], sel);
                 xB = __byte_perm(vc[tB0 * WPT + wv], vc[tB1 * WPT + wv], sel);
               }
-              const uint32_t m0 = 0x00030003u << (4 * hf), m1 = 0x00030003u << (4 * hf + 2);
-              av = make_uint4(xA & m0, xA & m1, xB & m0, xB & m1);
+              const uint32_t yA = hf == 0 ? xA << 4 : xA, yB = hf == 0 ? xB << 4 : xB;
+              av = make_uint4(yA & 0x00300030u, yA & 0x00C000C0u, yB & 0x00300030u, yB & 0x00C000C0u);
+            } else if (VB == 3) {
+              // Lane row r takes coordinates 32g + 4r .. + 3: the 12 bits at bit 12r of the
+              // group's 96 (one funnel shift per token), two tokens' windows in the f16 halves.
+              // Rows r -> coordinate 32g + 4r + 2hf, rows r + 8 -> + 1: codes at mantissa bits
+              // 3 (hf = 0; the code at bits 0-2 shifted up) or 6 (hf = 1; the code at 9-11
+              // shifted down). The lowest subnormal positions are left out: codes there lost
+              // about 1e-4 of the output on the tensor cores.
+              constexpr int WPT = L::VCB / 4;
+              if (hf == 0) {
+                const int bo = 12 * r, wi = 3 * g + (bo >> 5), wj = 3 * g + min((bo >> 5) + 1, 2), sh = bo & 31;
+                auto win = [&](int t) { return __funnelshift_r(vc[t * WPT + wi], vc[t * WPT + wj], sh); };
+                xA = __byte_perm(win(tA0), win(tA1), 0x5410);
+                xB = __byte_perm(win(tB0), win(tB1), 0x5410);
+                av = make_uint4((xA << 3) & 0x00380038u, xA & 0x00380038u, (xB << 3) & 0x00380038u,
+                                xB & 0x00380038u);
+              } else {
+                av = make_uint4(xA & 0x01C001C0u, (xA >> 3) & 0x01C001C0u, xB & 0x01C001C0u,
+                                (xB >> 3) & 0x01C001C0u);
+              }
             } else {
               // byte 16g + 8hf + r: rows r -> coordinate 2(16g + 8hf + r), rows r + 8 -> + 1
               constexpr int WPT = L::VCB / 4;
               const int wv = 4 * g + 2 * hf + (r >> 2);
               xA = __byte_perm(vc[tA0 * WPT + wv], vc[tA1 * WPT + wv], sel);
               xB = __byte_perm(vc[tB0 * WPT + wv], vc[tB1 * WPT + wv], sel);
-              av = make_uint4(xA & 0x000F000Fu, xA & 0x00F000F0u, xB & 0x000F000Fu, xB & 0x00F000F0u);
+              // both nibbles at mantissa bits 4-7 (the low one shifted up)
+              av = make_uint4((xA << 4) & 0x00F000F0u, xA & 0x00F000F0u, (xB << 4) & 0x00F000F0u,
+                              xB & 0x00F000F0u);
             }
 #pragma unroll
             for (int nb = 0; nb < NB; ++nb) mma16816(dv[g][hf][nb], av, bA[nb], bB[nb]);
@@ -1264,24 +1292,23 @@ bool mma_decode_supported(const tq_ctx* ctx, int G) {
   const Shape& sh = ctx->shape;
   if (sh.d != kD || sh.m != kM || G < 1 || G > 8) return false;
   if (sh.lm_bits < 1 || sh.lm_bits > 3) return false;
-  if (!(sh.v_bits == 2 || sh.v_bits == 4)) return false;
+  if (sh.v_bits < 2 || sh.v_bits > 4) return false;
   // the codebook must be affine in its bits (and the parity at 3 bits): true for a symmetric one
   float kappa, beta[4];
   return codebook_bits(ctx->cb, sh.lm_bits, kappa, beta);
 }
 
+template <int LMB>
+int ctas_per_sm_l(int v_bits, int nb) {
+  if (v_bits == 2) return nb == 1 ? ctas_per_sm_t<LMB, 2, 1>() : ctas_per_sm_t<LMB, 2, 2>();
+  if (v_bits == 3) return nb == 1 ? ctas_per_sm_t<LMB, 3, 1>() : ctas_per_sm_t<LMB, 3, 2>();
+  return nb == 1 ? ctas_per_sm_t<LMB, 4, 1>() : ctas_per_sm_t<LMB, 4, 2>();
+}
+
 int mma_ctas_per_sm(int lm_bits, int v_bits, int G) {
   const int nb = n_blocks(G);
-  if (lm_bits == 1) {
-    if (v_bits == 2) return nb == 1 ? ctas_per_sm_t<1, 2, 1>() : ctas_per_sm_t<1, 2, 2>();
-    return nb == 1 ? ctas_per_sm_t<1, 4, 1>() : ctas_per_sm_t<1, 4, 2>();
-  }
-  if (lm_bits == 2) {
-    if (v_bits == 2) return nb == 1 ? ctas_per_sm_t<2, 2, 1>() : ctas_per_sm_t<2, 2, 2>();
-    return nb == 1 ? ctas_per_sm_t<2, 4, 1>() : ctas_per_sm_t<2, 4, 2>();
-  }
-  if (v_bits == 2) return nb == 1 ? ctas_per_sm_t<3, 2, 1>() : ctas_per_sm_t<3, 2, 2>();
-  return nb == 1 ? ctas_per_sm_t<3, 4, 1>() : ctas_per_sm_t<3, 4, 2>();
+  return lm_bits == 1 ? ctas_per_sm_l<1>(v_bits, nb) : lm_bits == 2 ? ctas_per_sm_l<2>(v_bits, nb)
+                                                                  : ctas_per_sm_l<3>(v_bits, nb);
 }
 
 size_t mma_frag_bytes(int lm_bits, int G) { return (size_t)frag_words(lm_bits, n_blocks(G)) * 4; }
@@ -1364,11 +1391,14 @@ cudaError_t launch_decode_mma(const tq_ctx* ctx, const DecodePlan& plan, const v
   const dim3 grid((unsigned)plan.n_ctas);
   if (ctx->prof_start) cudaEventRecord(ctx->prof_start, stream);
   if (lmb == 1)
-    e = vb == 2 ? launch_mma_nb<1, 2>(a, nb, grid, stream) : launch_mma_nb<1, 4>(a, nb, grid, stream);
+    e = vb == 2 ? launch_mma_nb<1, 2>(a, nb, grid, stream)
+        : vb == 3 ? launch_mma_nb<1, 3>(a, nb, grid, stream) : launch_mma_nb<1, 4>(a, nb, grid, stream);
   else if (lmb == 2)
-    e = vb == 2 ? launch_mma_nb<2, 2>(a, nb, grid, stream) : launch_mma_nb<2, 4>(a, nb, grid, stream);
+    e = vb == 2 ? launch_mma_nb<2, 2>(a, nb, grid, stream)
+        : vb == 3 ? launch_mma_nb<2, 3>(a, nb, grid, stream) : launch_mma_nb<2, 4>(a, nb, grid, stream);
   else
-    e = vb == 2 ? launch_mma_nb<3, 2>(a, nb, grid, stream) : launch_mma_nb<3, 4>(a, nb, grid, stream);
+    e = vb == 2 ? launch_mma_nb<3, 2>(a, nb, grid, stream)
+        : vb == 3 ? launch_mma_nb<3, 3>(a, nb, grid, stream) : launch_mma_nb<3, 4>(a, nb, grid, stream);
   if (ctx->prof_stop) cudaEventRecord(ctx->prof_stop, stream);
   if (e != cudaSuccess) return e;
 

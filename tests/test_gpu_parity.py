@@ -350,14 +350,15 @@ def test_decode_parity_random_cache(d, lm_bits, v_bits, G):
 
 
 @pytest.mark.parametrize("kernel", ["tcgen05", "mma", "cuda_core"])
-@pytest.mark.parametrize("lm_bits,v_bits,G", [(2, 2, 4), (2, 4, 8), (1, 2, 3), (3, 4, 6), (2, 2, 1)])
+@pytest.mark.parametrize("lm_bits,v_bits,G", [(2, 2, 4), (2, 4, 8), (1, 2, 3), (3, 4, 6), (2, 2, 1), (2, 3, 4),
+                                              (3, 3, 8)])
 def test_decode_each_kernel_family(kernel, lm_bits, v_bits, G):
     """Every decode kernel family, selected explicitly, on the shapes it takes: the same
     packed cache decodes to the oracle's scores and outputs whichever kernel runs."""
     _decode_check(128, lm_bits, v_bits, batch=2, hkv=2, G=G, max_len=1500, lens=[1500, 701], kernel=kernel)
 
 
-@pytest.mark.parametrize("lm_bits,v_bits,G", [(2, 2, 4), (2, 4, 8), (3, 4, 6)])
+@pytest.mark.parametrize("lm_bits,v_bits,G", [(2, 2, 4), (2, 4, 8), (3, 4, 6), (2, 3, 4)])
 def test_decode_variable_lengths_split_by_tokens(lm_bits, v_bits, G):
     """A batch of empty, one-token, partial and full sequences on the mma.sync decode, which
     splits the tiles that hold tokens (not every sequence's max_len) over its CTAs: fewer
@@ -383,7 +384,8 @@ def test_decode_many_sequences_split_scan():
 
 
 def test_decode_kernel_selection():
-    """TQ_DECODE_AUTO takes the mma.sync kernel for 1- to 3-bit codes with the QJL stage,
+    """TQ_DECODE_AUTO takes the mma.sync kernel for 1- to 3-bit codes with the QJL stage
+    (2- to 4-bit values),
     the tcgen05 kernel for keys without QJL, and the generic kernels for every other shape;
     an explicitly selected family that does not take the shape refuses the call."""
     ctx = make_ctx(T, 128, 2, 2)
@@ -409,6 +411,8 @@ def test_decode_kernel_selection():
     assert T.tq_decode_kernel_for(ctx0, 32, 8) == T.TQ_DECODE_TCGEN05
     ctx64 = make_ctx(T, 64, 2, 2)
     assert T.tq_decode_kernel_for(ctx64, 32, 8) == T.TQ_DECODE_CUDA_CORE
+    ctx33 = make_ctx(T, 128, 2, 3)                                            # K = V = 3
+    assert T.tq_decode_kernel_for(ctx33, 32, 8) == T.TQ_DECODE_MMA
 
 
 @pytest.mark.parametrize("G", [4, 8])
@@ -646,6 +650,29 @@ def test_keys_without_qjl_pipelined_compression(lm_bits, v_bits, rotation):
         assert np.array_equal(gk[name], g[name]), name
     for name in ("v_codes", "v_params"):
         assert np.array_equal(gv[name], g[name]), name
+
+
+@pytest.mark.parametrize("v_bits", [2, 3, 4])
+def test_decode_value_codes_keep_the_low_parts(v_bits):
+    """Values N(0.5, 2^2) per coordinate (groups with large minima and spans), Haar keys, fp32
+    queries, decoded on the mma.sync kernel: the value codes enter the MMAs as f16 subnormals
+    at mantissa bit 3 or higher; at the lowest positions their products with the low parts of
+    p * scale lost up to 3e-4 of the output (outside the elementwise bound for small outputs)."""
+    d, lm_bits, n, G = 128, 2, 2500, 4
+    rng = np.random.default_rng([d, 3])
+    K = rng.standard_normal((n, d)) * rng.lognormal(0, 1, d)
+    V = rng.standard_normal((n, d)) * 2.0 + 0.5
+    ctx, g, ok, ov = _compress_both(K, V, d, lm_bits, v_bits, "haar", "f32")
+    T.tq_set_decode_kernel(ctx, T.TQ_DECODE_MMA)
+    gp = _upload({k: g[k] for k in ("k_codes", "k_signs", "k_norms", "v_codes", "v_params")})
+    q = W.queries((1, G, d), dtype="f32")
+    out, _ = T.tq_decode_attention(ctx, torch.from_numpy(q).to(DEV), gp, 1, G, 1, n)
+    T.tq_check_device(ctx)
+    Pi, c, t, S = oracle_setup(d, lm_bits, d, "haar")
+    pk = {"codes": g["k_codes"], "signs": g["k_signs"], "norms": g["k_norms"]}
+    pv = {"codes": g["v_codes"], "params": g["v_params"]}
+    _, oo = O.decode_attention(q[0].astype(np.float64), pk, pv, Pi, c, S, d, v_bits)
+    assert_close(out[0].cpu().numpy(), oo, what="out")
 
 
 # ------------------------------------------------------------------ 3-bit values (K = V = 3)
