@@ -183,8 +183,7 @@ size_t tq_decode_workspace_bytes(const tq_ctx* ctx, int batch, int hq, int hkv, 
  *   out       device fp32 [batch][hq][d]
  *   workspace device scratch of at least tq_decode_workspace_bytes(...) bytes
  * At d = 128 with 1- to 3-bit Lloyd-Max codes of a codebook symmetric about zero,
- * 2- to 4-bit values (keys without the QJL stage: 2 or 4) and at most 8 query heads per
- * KV head, a tensor-core decode runs
+ * 2- to 4-bit values and at most 8 query heads per KV head, a tensor-core decode runs
  * (tq_set_decode_kernel); it carries p * scale (p < 4) as f16 operands, so value-group
  * scales must stay below 16376 (values spanning less than 49000 at 2 bits). Other
  * shapes run the CUDA-core decode. With seq_lens, the mma.sync decode (the default for

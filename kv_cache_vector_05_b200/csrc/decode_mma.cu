@@ -25,9 +25,9 @@
 // K = 16 tokens, columns = 4 query heads x (hi, lo), the two f16 halves of p * scale.
 //  * A value code placed in the mantissa bits of an f16 is a subnormal equal to
 //    code * 2^(pos - 24), so a byte permute, a shift and a mask yield two exact
-//    operands; the power of two is undone once at the end. The codes sit at bit 3 or
-//    higher: products of codes at the lowest positions with the small low parts of
-//    p * scale lost about 1e-4 of the output on the tensor cores.
+//    operands; the power of two is undone once at the end. The codes sit at bit 4 or
+//    higher (6 and up at 2 and 3 bits): products of codes at the lowest positions with
+//    the small low parts of p * scale lost about 1e-4 of the output on the tensor cores.
 //
 // Kernels:
 //  * prep_mma_kernel, one CTA per (sequence, KV head): rotates the G queries
@@ -745,13 +745,13 @@ __global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid
               int j0;
               float v0, v1;
               if (VB == 2) {
-                j0 = 4 * (8 * g + r) + 2 * hf;  // code at mantissa bits 4 (row r), 6 (row r + 8)
-                v0 = (d[0] + d[1]) * 1048576.f + mt[g];
-                v1 = (d[2] + d[3]) * 262144.f + mt[g];
+                j0 = 4 * (8 * g + r) + 2 * hf;  // code at mantissa bits 6 (row r), 8 (row r + 8)
+                v0 = (d[0] + d[1]) * 262144.f + mt[g];
+                v1 = (d[2] + d[3]) * 65536.f + mt[g];
               } else if (VB == 3) {
-                j0 = 32 * g + 4 * r + 2 * hf;  // code at mantissa bit 3 (hf = 0) or 6 (hf = 1)
-                v0 = (d[0] + d[1]) * (hf == 0 ? 2097152.f : 262144.f) + mt[g];
-                v1 = (d[2] + d[3]) * (hf == 0 ? 2097152.f : 262144.f) + mt[g];
+                j0 = 32 * g + 4 * r + 2 * hf;  // codes at mantissa bit 6
+                v0 = (d[0] + d[1]) * 262144.f + mt[g];
+                v1 = (d[2] + d[3]) * 262144.f + mt[g];
               } else {
                 j0 = 2 * (16 * g + 8 * hf + r);  // low nibble (row r), high nibble (row r + 8), both at bit 4
                 v0 = (d[0] + d[1]) * 1048576.f + mt[g];
@@ -1045,31 +1045,29 @@ __global__ void __launch_bounds__(kThreadsMma, 1) decode_mma_kernel(const __grid
             uint32_t xA, xB;
             uint4 av;
             if (VB == 2) {
-              // byte 8g + r: rows r -> coordinate 4(8g + r) + 2hf, rows r + 8 -> + 1; codes at
-              // mantissa bits 4 (rows r) and 6 (rows r + 8), those of hf = 0 shifted up by 4
+              // byte 8g + r: rows r -> coordinate 4(8g + r) + 2hf, rows r + 8 -> + 1; codes moved
+              // to mantissa bits 6 (rows r) and 8 (rows r + 8)
               constexpr int WPT = L::VCB / 4;
               const int wv = 2 * g + (r >> 2);
               if (hf == 0) {
                 xA = __byte_perm(vc[tA0 * WPT + wv], vc[tA1 * WPT + wv], sel);
                 xB = __byte_perm(vc[tB0 * WPT + wv], vc[tB1 * WPT + wv], sel);
               }
-              const uint32_t yA = hf == 0 ? xA << 4 : xA, yB = hf == 0 ? xB << 4 : xB;
-              av = make_uint4(yA & 0x00300030u, yA & 0x00C000C0u, yB & 0x00300030u, yB & 0x00C000C0u);
+              const uint32_t yA = xA << (6 - 4 * hf), yB = xB << (6 - 4 * hf);
+              av = make_uint4(yA & 0x00C000C0u, yA & 0x03000300u, yB & 0x00C000C0u, yB & 0x03000300u);
             } else if (VB == 3) {
               // Lane row r takes coordinates 32g + 4r .. + 3: the 12 bits at bit 12r of the
               // group's 96 (one funnel shift per token), two tokens' windows in the f16 halves.
-              // Rows r -> coordinate 32g + 4r + 2hf, rows r + 8 -> + 1: codes at mantissa bits
-              // 3 (hf = 0; the code at bits 0-2 shifted up) or 6 (hf = 1; the code at 9-11
-              // shifted down). The lowest subnormal positions are left out: codes there lost
-              // about 1e-4 of the output on the tensor cores.
+              // Rows r -> coordinate 32g + 4r + 2hf, rows r + 8 -> + 1: every code moved to
+              // mantissa bits 6..8.
               constexpr int WPT = L::VCB / 4;
               if (hf == 0) {
                 const int bo = 12 * r, wi = 3 * g + (bo >> 5), wj = 3 * g + min((bo >> 5) + 1, 2), sh = bo & 31;
                 auto win = [&](int t) { return __funnelshift_r(vc[t * WPT + wi], vc[t * WPT + wj], sh); };
                 xA = __byte_perm(win(tA0), win(tA1), 0x5410);
                 xB = __byte_perm(win(tB0), win(tB1), 0x5410);
-                av = make_uint4((xA << 3) & 0x00380038u, xA & 0x00380038u, (xB << 3) & 0x00380038u,
-                                xB & 0x00380038u);
+                av = make_uint4((xA << 6) & 0x01C001C0u, (xA << 3) & 0x01C001C0u, (xB << 6) & 0x01C001C0u,
+                                (xB << 3) & 0x01C001C0u);
               } else {
                 av = make_uint4(xA & 0x01C001C0u, (xA >> 3) & 0x01C001C0u, xB & 0x01C001C0u,
                                 (xB >> 3) & 0x01C001C0u);

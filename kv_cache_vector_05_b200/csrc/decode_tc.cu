@@ -819,6 +819,10 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
                   j0 = 4 * (8 * g + r) + 2 * hf;
                   v0 = (d[0] + d[1]) * 262144.f;
                   v1 = (d[2] + d[3]) * 65536.f;
+                } else if (VB == 3) {  // coordinates 32g + 4r + 2hf (+ 1), codes at bit 6
+                  j0 = 32 * g + 4 * r + 2 * hf;
+                  v0 = (d[0] + d[1]) * 262144.f;
+                  v1 = (d[2] + d[3]) * 262144.f;
                 } else {
                   j0 = 2 * (16 * g + 8 * hf + r);
                   v0 = (d[0] + d[1]) * 262144.f;
@@ -1129,6 +1133,20 @@ __global__ void __launch_bounds__(TcLayout<LMB, QJL, VB, NB>::THREADS, 1)
                 xA = __byte_perm(vA0[wv], vA1[wv], sel) << (6 - 4 * hf);
                 xB = __byte_perm(vB0[wv], vB1[wv], sel) << (6 - 4 * hf);
                 av = make_uint4(xA & 0x00C000C0u, xA & 0x03000300u, xB & 0x00C000C0u, xB & 0x03000300u);
+              } else if (VB == 3) {
+                // 3-bit fields straddle bytes: row r takes coordinates 32g + 4r .. + 3, the 12 bits
+                // at bit 12r of the group's 96 (one funnel shift per token); rows r -> coordinate
+                // 32g + 4r + 2hf, rows r + 8 -> + 1, every code moved to bits 6..8
+                if (hf == 0) {
+                  const int bo = 12 * r, wi = 3 * g + (bo >> 5), wj = 3 * g + min((bo >> 5) + 1, 2), sh = bo & 31;
+                  xA = __byte_perm(__funnelshift_r(vA0[wi], vA0[wj], sh), __funnelshift_r(vA1[wi], vA1[wj], sh), 0x5410);
+                  xB = __byte_perm(__funnelshift_r(vB0[wi], vB0[wj], sh), __funnelshift_r(vB1[wi], vB1[wj], sh), 0x5410);
+                  av = make_uint4((xA << 6) & 0x01C001C0u, (xA << 3) & 0x01C001C0u, (xB << 6) & 0x01C001C0u,
+                                  (xB << 3) & 0x01C001C0u);
+                } else {
+                  av = make_uint4(xA & 0x01C001C0u, (xA >> 3) & 0x01C001C0u, xB & 0x01C001C0u,
+                                  (xB >> 3) & 0x01C001C0u);
+                }
               } else {
                 // byte 16g + 8hf + r: rows r -> coordinate 2(16g + 8hf + r) (low nibble), rows
                 // r + 8 -> + 1 (high nibble), both to bits 6..9
@@ -1212,19 +1230,22 @@ cudaError_t launch_tc_nb(const tq_ctx* ctx, const PrepTcArgs& pa, int units, con
 template <int LMB, bool QJL>
 cudaError_t launch_tc_vb(const tq_ctx* ctx, const PrepTcArgs& pa, int units, const TcArgs& a, int n_ctas, int nb,
                          int vb, cudaStream_t s) {
-  return vb == 2 ? launch_tc_nb<LMB, QJL, 2>(ctx, pa, units, a, n_ctas, nb, s)
-                 : launch_tc_nb<LMB, QJL, 4>(ctx, pa, units, a, n_ctas, nb, s);
+  return vb == 2   ? launch_tc_nb<LMB, QJL, 2>(ctx, pa, units, a, n_ctas, nb, s)
+         : vb == 3 ? launch_tc_nb<LMB, QJL, 3>(ctx, pa, units, a, n_ctas, nb, s)
+                   : launch_tc_nb<LMB, QJL, 4>(ctx, pa, units, a, n_ctas, nb, s);
 }
 
 template <int LMB, bool QJL>
 int tc_groups_t(int nb, int vb) {
   if (vb == 2) return nb == 1 ? TcLayout<LMB, QJL, 2, 1>::NG : TcLayout<LMB, QJL, 2, 2>::NG;
+  if (vb == 3) return nb == 1 ? TcLayout<LMB, QJL, 3, 1>::NG : TcLayout<LMB, QJL, 3, 2>::NG;
   return nb == 1 ? TcLayout<LMB, QJL, 4, 1>::NG : TcLayout<LMB, QJL, 4, 2>::NG;
 }
 
 template <int LMB, bool QJL>
 size_t tc_bbuf_t(int nb, int vb) {
   if (vb == 2) return nb == 1 ? TcLayout<LMB, QJL, 2, 1>::BBUF : TcLayout<LMB, QJL, 2, 2>::BBUF;
+  if (vb == 3) return nb == 1 ? TcLayout<LMB, QJL, 3, 1>::BBUF : TcLayout<LMB, QJL, 3, 2>::BBUF;
   return nb == 1 ? TcLayout<LMB, QJL, 4, 1>::BBUF : TcLayout<LMB, QJL, 4, 2>::BBUF;
 }
 
@@ -1270,7 +1291,7 @@ bool tc_decode_supported(const tq_ctx* ctx, int G) {
   const Shape& sh = ctx->shape;
   if (sh.d != kD || !(sh.m == kM || sh.m == 0) || G < 1 || G > 8) return false;
   if (sh.lm_bits < 1 || sh.lm_bits > 3) return false;
-  if (!(sh.v_bits == 2 || sh.v_bits == 4)) return false;
+  if (sh.v_bits < 2 || sh.v_bits > 4) return false;
   float kappa, beta[4];
   return codebook_bits(ctx->cb, sh.lm_bits, kappa, beta);
 }

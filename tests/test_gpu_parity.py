@@ -571,7 +571,8 @@ def test_sweep_mse_and_inner_product_distortion_vs_oracle(d, b, rotation):
 # ------------------------------------------------------------------ keys without the QJL stage
 
 @pytest.mark.parametrize("d,lm_bits,v_bits,rotation,dtype", [
-    (128, 2, 2, "hadamard", "bf16"), (128, 1, 4, "haar", "f32"), (64, 3, 4, "hadamard", "bf16")])
+    (128, 2, 2, "hadamard", "bf16"), (128, 1, 4, "haar", "f32"), (64, 3, 4, "hadamard", "bf16"),
+    (128, 3, 3, "hadamard", "bf16")])
 def test_keys_without_qjl_stage(d, lm_bits, v_bits, rotation, dtype):
     """qjl_m = 0 (Lloyd-Max codes only; no sign bytes): compression, decode attention and
     decompression through the C ABI against the oracle given an empty S."""
